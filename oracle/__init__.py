@@ -1,0 +1,154 @@
+"""fp64 CPU oracle for the paged-KV-cache decode path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The product library
+(``paged_kv_cache_415_b200``) never imports it and shares no code with it.
+
+``pa_oracle.c`` holds the definitions (reshape_and_cache, copy_blocks, paged
+decode in fp64); this module compiles it with gcc (``-O2``, OpenMP, no
+fast-math) into ``liboracle.so`` beside it and wraps it with ctypes.
+``brute.py`` holds pure-Python/numpy restatements used to pin it.
+
+Arrays are numpy: fp16/bf16 tensors are passed as their raw ``uint16`` bit
+patterns together with a dtype name ("f16" or "bf16").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "pa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_DTYPES = {"f16": 0, "bf16": 1}
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle source into a shared library (gcc -O2 -fopenmp)."""
+    if (not force and os.path.exists(out)
+            and os.path.getmtime(out) >= os.path.getmtime(src)):
+        return out
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                           "-Wall", "-Wextra", "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def load(path: str | None = None):
+    """ctypes handle of the oracle library (the default build, or ``path``:
+    the tests load deliberately broken variants to check that the pins
+    catch them)."""
+    global _lib
+    if path is None and _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build() if path is None else path)
+    p = ctypes.c_void_p
+    i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+    lib.oracle_decode_bits.argtypes = [p, p, i64, i32]
+    lib.oracle_decode_bits.restype = None
+    lib.oracle_reshape_and_cache.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64]
+    lib.oracle_reshape_and_cache.restype = i32
+    lib.oracle_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i64]
+    lib.oracle_copy_blocks.restype = i32
+    lib.oracle_paged_decode.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64,
+                                        f64, i32, i32, i32]
+    lib.oracle_paged_decode.restype = i32
+    lib.oracle_paged_decode_rows.argtypes = [p, p, i32, p, p, p, p, p, i32, i32, i32, i32,
+                                             i32, i64, f64, i32, i32]
+    lib.oracle_paged_decode_rows.restype = i32
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = i32
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray) -> ctypes.c_void_p:
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _u16(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    assert a.dtype == np.uint16, f"expected 16-bit patterns, got {a.dtype}"
+    return a
+
+
+def max_threads(lib=None) -> int:
+    return int((lib or load()).oracle_max_threads())
+
+
+def decode_bits(bits: np.ndarray, dtype: str, lib=None) -> np.ndarray:
+    """Exact fp16/bf16 bit pattern -> float64."""
+    bits = _u16(bits)
+    out = np.empty(bits.shape, dtype=np.float64)
+    (lib or load()).oracle_decode_bits(_ptr(bits), _ptr(out), bits.size, _DTYPES[dtype])
+    return out
+
+
+def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, block_size, lib=None) -> int:
+    """In place on k_cache / v_cache ([num_blocks][block_size][Hkv][D] uint16).
+
+    key/value: [T][Hkv][D]; slot_mapping int64 [T].  Returns status bits."""
+    key, value = _u16(key), _u16(value)
+    assert k_cache.dtype == np.uint16 and v_cache.dtype == np.uint16
+    slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    num_blocks, bs, hkv, d = k_cache.shape
+    assert bs == block_size
+    return int((lib or load()).oracle_reshape_and_cache(
+        _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+        key.shape[0], hkv, d, block_size, num_blocks))
+
+
+def copy_blocks(k_cache, v_cache, block_mapping, lib=None) -> int:
+    """In place: for each (src, dst) row of block_mapping, copy block src to dst."""
+    block_mapping = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+    num_blocks, bs, hkv, d = k_cache.shape
+    return int((lib or load()).oracle_copy_blocks(
+        _ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), block_mapping.shape[0],
+        hkv, d, bs, num_blocks))
+
+
+def paged_decode(query, k_cache, v_cache, block_tables, context_lens, scale, dtype,
+                 blocked=False, num_threads=0, lib=None):
+    """fp64 paged decode attention.  Returns (out [S][Hq][D] float64, status)."""
+    query = _u16(query)
+    k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+    block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    s, hq, d = query.shape
+    num_blocks, bs, hkv, d2 = k_cache.shape
+    assert d2 == d
+    out = np.empty((s, hq, d), dtype=np.float64)
+    st = (lib or load()).oracle_paged_decode(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), s, hq, hkv, d, bs, block_tables.shape[1], num_blocks,
+        float(scale), _DTYPES[dtype], 1 if blocked else 0, num_threads)
+    return out, int(st)
+
+
+def paged_decode_rows(rows, query, k_cache, v_cache, block_tables, context_lens, scale, dtype,
+                      num_threads=0, lib=None):
+    """fp64 paged decode for selected (sequence, query head) rows only.
+
+    rows: int [n][2].  Returns (out [n][D] float64, status)."""
+    rows = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 2)
+    query = _u16(query)
+    k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+    block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    s, hq, d = query.shape
+    num_blocks, bs, hkv, _ = k_cache.shape
+    out = np.empty((rows.shape[0], d), dtype=np.float64)
+    st = (lib or load()).oracle_paged_decode_rows(
+        _ptr(out), _ptr(rows), rows.shape[0], _ptr(query), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), hq, hkv, d, bs, block_tables.shape[1],
+        num_blocks, float(scale), _DTYPES[dtype], num_threads)
+    return out, int(st)

@@ -1,0 +1,323 @@
+/*
+ * pa_oracle.c -- plain fp64 CPU oracle for the paged-KV-cache decode path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path
+ * (the CUDA library under paged_kv_cache_415_b200/) shares no code with it
+ * and never calls it.
+ *
+ * It is deliberately slow and obvious: every output is the textbook
+ * definition written out in double precision, with no blocking, fusion or
+ * reordering beyond what the definition states.
+ *
+ * Pages cited (title, then section):
+ *   [VM-paging] "vLLM用虚拟内存分页思想管理KV Cache"
+ *   [Practice]  "PagedAttention：大模型KV Cache分页管理优化实践"
+ *   [Manager]   "深入解析 vLLM 的 KV Cache 管理器：从内存碎片到 PagedAttention 的完整技术剖析"
+ *
+ * Cache layout (one layer, K and V in separate pools):
+ *   k_cache, v_cache : [num_blocks][block_size][num_kv_heads][head_dim]
+ * A physical block holds block_size tokens x kv heads x head_dim for K (and
+ * the same for V) [Practice §3.1 物理块分配器设计].  Token t of a sequence
+ * lives in logical block t / block_size at offset t % block_size, and the
+ * sequence's block table maps the logical block to a physical block id
+ * [Practice §3.2 块表与地址转换].
+ *
+ * Element storage is the raw 16-bit pattern (IEEE binary16 or bfloat16);
+ * the oracle decodes the bits itself, exactly, into double.
+ *
+ * Status bits returned by the functions (same meaning as the library's):
+ *   1 = a block-table entry outside [0, num_blocks)   (that block is skipped)
+ *   2 = a slot at or beyond num_blocks * block_size   (that token is skipped)
+ *   4 = a context length that is negative or longer than the block table
+ *       (the output row is written as zeros)
+ *   8 = copy_blocks: a destination written twice, or also used as a source
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { OR_DTYPE_F16 = 0, OR_DTYPE_BF16 = 1 };
+
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction
+ * bits.  Subnormals are fraction x 2^-24.  Every binary16 value is exact in
+ * double. */
+static double f16_bits_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 10) & 0x1f;
+    int frac = h & 0x3ff;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -24);
+    else if (expo == 31)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp((double)(frac + 1024), expo - 25);
+    return sign ? -v : v;
+}
+
+/* bfloat16: the upper half of an IEEE binary32, 8 exponent bits (bias 127),
+ * 7 fraction bits.  Subnormals are fraction x 2^-133. */
+static double bf16_bits_to_f64(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 7) & 0xff;
+    int frac = h & 0x7f;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -133);
+    else if (expo == 255)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp((double)(frac + 128), expo - 134);
+    return sign ? -v : v;
+}
+
+static double decode(uint16_t bits, int dtype)
+{
+    return dtype == OR_DTYPE_BF16 ? bf16_bits_to_f64(bits) : f16_bits_to_f64(bits);
+}
+
+/* Exposed so the tests can pin the bit decoding against numpy's float16 and
+ * against hand-computed bfloat16 values. */
+void oracle_decode_bits(const uint16_t* bits, double* out, int64_t n, int32_t dtype)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = decode(bits[i], dtype);
+}
+
+/* ------------------------------------------------------------------------
+ * reshape_and_cache: write each new token's K and V rows into the slot the
+ * allocator gave it ([Practice §3.3 按需分配策略], step 4 "write the new
+ * token's KV vectors"; [Manager, 第一部分 KV Cache 的核心价值]: the new K/V is
+ * appended before attention).  slot = physical_block * block_size + offset.
+ * A negative slot is a padding token and writes nothing.  It is a raw bit
+ * copy: no value changes.
+ * ---------------------------------------------------------------------- */
+int32_t oracle_reshape_and_cache(const uint16_t* key, const uint16_t* value,
+                                 uint16_t* k_cache, uint16_t* v_cache,
+                                 const int64_t* slot_mapping, int32_t num_tokens,
+                                 int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int64_t num_blocks)
+{
+    int32_t status = 0;
+    const int64_t row = (int64_t)num_kv_heads * head_dim; /* elements per token */
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * (int64_t)block_size) { status |= 2; continue; }
+        int64_t block = slot / block_size;
+        int64_t offset = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            for (int32_t d = 0; d < head_dim; ++d) {
+                int64_t src = (int64_t)t * row + (int64_t)h * head_dim + d;
+                int64_t dst = ((block * block_size + offset) * num_kv_heads + h) * head_dim + d;
+                k_cache[dst] = key[src];
+                v_cache[dst] = value[src];
+            }
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------
+ * copy_blocks: the data half of copy-on-write.  When a sequence must modify
+ * a block whose reference count is above one, the manager allocates a new
+ * block, copies the original's data into it, remaps privately and drops the
+ * old reference ([VM-paging, 写时复制与块共享机制]; [Practice §4.1 共享内存管理]
+ * steps 1-4).  This is step 2, for every (src, dst) pair, in order, for K
+ * and V.  src == dst is a no-op.  A destination that appears twice, or that
+ * is also a source in the same call, raises status bit 8 (the pairs are
+ * still applied in order here).
+ * ---------------------------------------------------------------------- */
+int32_t oracle_copy_blocks(uint16_t* k_cache, uint16_t* v_cache,
+                           const int64_t* block_mapping, int32_t num_pairs,
+                           int32_t num_kv_heads, int32_t head_dim,
+                           int32_t block_size, int64_t num_blocks)
+{
+    int32_t status = 0;
+    const int64_t block_elems = (int64_t)block_size * num_kv_heads * head_dim;
+    for (int32_t i = 0; i < num_pairs; ++i) {
+        int64_t dst = block_mapping[2 * i + 1];
+        for (int32_t j = 0; j < num_pairs; ++j) {
+            if (j == i) continue;
+            if (block_mapping[2 * j + 1] == dst && j < i) status |= 8;
+            if (block_mapping[2 * j] == dst && block_mapping[2 * j] != block_mapping[2 * j + 1])
+                status |= 8;
+        }
+    }
+    for (int32_t i = 0; i < num_pairs; ++i) {
+        int64_t src = block_mapping[2 * i];
+        int64_t dst = block_mapping[2 * i + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) { status |= 1; continue; }
+        if (src == dst) continue;
+        for (int64_t e = 0; e < block_elems; ++e) {
+            k_cache[dst * block_elems + e] = k_cache[src * block_elems + e];
+            v_cache[dst * block_elems + e] = v_cache[src * block_elems + e];
+        }
+    }
+    return status;
+}
+
+/* Address translation: token t of sequence s -> element offset of row
+ * (t, kv head g) in the pool, or -1 when the table entry is out of range
+ * ([Practice §3.2]: logical block j -> table[j] -> physical id -> base +
+ * offset). */
+static int64_t token_row(const int32_t* table, int32_t t, int32_t g,
+                         int32_t num_kv_heads, int32_t head_dim,
+                         int32_t block_size, int64_t num_blocks)
+{
+    int64_t phys = table[t / block_size];
+    if (phys < 0 || phys >= num_blocks) return -1;
+    return ((phys * block_size + t % block_size) * num_kv_heads + g) * (int64_t)head_dim;
+}
+
+/* ------------------------------------------------------------------------
+ * Paged decode attention for one (sequence, query head), direct form.
+ *
+ * [VM-paging, PagedAttention的注意力计算流程]: for request i and head l, take
+ * the physical blocks from the block table; pass 1 scores the query against
+ * every Key in those blocks; softmax gives the weights; pass 2 sums the
+ * Values with those weights.  [Manager, 第二部分 PagedAttention 的核心思想]
+ * step 4: the kernel reassembles K/V through the block table at run time.
+ *
+ * Query head h reads kv head h / (num_q_heads / num_kv_heads) (consecutive
+ * grouping; with equal head counts this is plain multi-head attention).
+ *
+ *   x_t = scale * sum_d q[d] * K_t[d]          t < context_len
+ *   w_t = exp(x_t - max x) / sum_u exp(x_u - max x)
+ *   out = sum_t w_t * V_t
+ * ---------------------------------------------------------------------- */
+static int32_t decode_row(double* out, const uint16_t* query, const uint16_t* k_cache,
+                          const uint16_t* v_cache, const int32_t* block_tables,
+                          const int32_t* context_lens, int32_t s, int32_t h,
+                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t block_size, int32_t max_blocks_per_seq,
+                          int64_t num_blocks, double scale, int32_t dtype,
+                          int32_t blocked)
+{
+    int32_t status = 0;
+    const int32_t group = num_q_heads / num_kv_heads;
+    const int32_t g = h / group;
+    const int32_t ctx = context_lens[s];
+    const int32_t* table = block_tables + (int64_t)s * max_blocks_per_seq;
+    for (int32_t d = 0; d < head_dim; ++d) out[d] = 0.0;
+    if (ctx < 0 || ctx > (int64_t)max_blocks_per_seq * block_size) return 4;
+    if (ctx == 0) return 0;
+
+    double* q = (double*)malloc(sizeof(double) * head_dim);
+    double* x = (double*)malloc(sizeof(double) * ctx);
+    unsigned char* valid = (unsigned char*)malloc(ctx);
+    const uint16_t* qbits = query + ((int64_t)s * num_q_heads + h) * head_dim;
+    for (int32_t d = 0; d < head_dim; ++d) q[d] = decode(qbits[d], dtype);
+
+    /* pass 1: scores */
+    int32_t any = 0;
+    for (int32_t t = 0; t < ctx; ++t) {
+        int64_t r = token_row(table, t, g, num_kv_heads, head_dim, block_size, num_blocks);
+        valid[t] = r >= 0;
+        if (r < 0) { status |= 1; x[t] = 0.0; continue; }
+        double acc = 0.0;
+        for (int32_t d = 0; d < head_dim; ++d) acc += q[d] * decode(k_cache[r + d], dtype);
+        x[t] = scale * acc;
+        any = 1;
+    }
+
+    if (any) {
+        double m = -INFINITY, l = 0.0;
+        if (!blocked) {
+            /* softmax, direct */
+            for (int32_t t = 0; t < ctx; ++t) if (valid[t] && x[t] > m) m = x[t];
+        } else {
+            /* the five steps of [Practice §5.1 分块Softmax算法]:
+             * (1) local max m_j of every block j, (2) global max over the
+             * m_j, (3) the exps exp(s - m_global), (4) their global sum,
+             * (5) w = exp(s - m_global) / l_global.  Steps 3-5 are shared
+             * with the direct form below; steps 1-2 differ. */
+            int32_t nb = (ctx + block_size - 1) / block_size;
+            for (int32_t j = 0; j < nb; ++j) {
+                double mj = -INFINITY;
+                for (int32_t t = j * block_size; t < ctx && t < (j + 1) * block_size; ++t)
+                    if (valid[t] && x[t] > mj) mj = x[t];
+                if (mj > m) m = mj;
+            }
+        }
+        for (int32_t t = 0; t < ctx; ++t) if (valid[t]) l += exp(x[t] - m);
+        /* pass 2: weighted sum of Values */
+        for (int32_t t = 0; t < ctx; ++t) {
+            if (!valid[t]) continue;
+            double w = exp(x[t] - m) / l;
+            int64_t r = token_row(table, t, g, num_kv_heads, head_dim, block_size, num_blocks);
+            for (int32_t d = 0; d < head_dim; ++d) out[d] += w * decode(v_cache[r + d], dtype);
+        }
+    }
+    free(q); free(x); free(valid);
+    return status;
+}
+
+static void set_threads(int32_t num_threads)
+{
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#else
+    (void)num_threads;
+#endif
+}
+
+/* Full output: out is double [num_seqs][num_q_heads][head_dim]. */
+int32_t oracle_paged_decode(double* out, const uint16_t* query, const uint16_t* k_cache,
+                            const uint16_t* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, int32_t num_seqs,
+                            int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t block_size, int32_t max_blocks_per_seq,
+                            int64_t num_blocks, double scale, int32_t dtype,
+                            int32_t blocked, int32_t num_threads)
+{
+    int32_t status = 0;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads;
+    set_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : status)
+    for (int64_t r = 0; r < rows; ++r) {
+        int32_t s = (int32_t)(r / num_q_heads), h = (int32_t)(r % num_q_heads);
+        status |= decode_row(out + r * head_dim, query, k_cache, v_cache, block_tables,
+                             context_lens, s, h, num_q_heads, num_kv_heads, head_dim,
+                             block_size, max_blocks_per_seq, num_blocks, scale, dtype, blocked);
+    }
+    return status;
+}
+
+/* Selected rows only: rows is int32 [n_rows][2] of (sequence, query head);
+ * out is double [n_rows][head_dim].  Used to check full-size launches on a
+ * sample of outputs. */
+int32_t oracle_paged_decode_rows(double* out, const int32_t* rows, int32_t n_rows,
+                                 const uint16_t* query, const uint16_t* k_cache,
+                                 const uint16_t* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int32_t num_q_heads,
+                                 int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                 int32_t max_blocks_per_seq, int64_t num_blocks, double scale,
+                                 int32_t dtype, int32_t num_threads)
+{
+    int32_t status = 0;
+    set_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : status)
+    for (int32_t i = 0; i < n_rows; ++i) {
+        status |= decode_row(out + (int64_t)i * head_dim, query, k_cache, v_cache, block_tables,
+                             context_lens, rows[2 * i], rows[2 * i + 1], num_q_heads,
+                             num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                             scale, dtype, 0);
+    }
+    return status;
+}
+
+int32_t oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

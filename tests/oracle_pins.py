@@ -1,0 +1,308 @@
+"""Pins of the fp64 oracle: checks against things other than the oracle
+itself (numpy / scipy library routines, brute-force loops, closed forms,
+invariances the mathematics fixes).  Each pin takes an oracle library handle
+so the same battery can run against deliberately broken builds of the
+oracle (tests/test_oracle_mutants.py) and must catch every one of them.
+
+Pages cited (title, then section):
+  [VM-paging] "vLLM用虚拟内存分页思想管理KV Cache"
+  [Practice]  "PagedAttention：大模型KV Cache分页管理优化实践"
+  [Manager]   "深入解析 vLLM 的 KV Cache 管理器：从内存碎片到 PagedAttention 的完整技术剖析"
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import oracle
+from oracle import brute
+from workloads import generators as gen
+
+F16_ONE = 0x3C00
+
+
+# ---------------------------------------------------------------- helpers
+def pool_after_step(wl):
+    """numpy-only: the pools after the step's copies and appends."""
+    kc, vc = wl.k_cache.copy(), wl.v_cache.copy()
+    for src, dst in wl.block_mapping:
+        if src != dst:
+            kc[dst] = kc[src]
+            vc[dst] = vc[src]
+    b = wl.block_size
+    sl = wl.slot_mapping
+    keep = sl >= 0
+    kc[sl[keep] // b, sl[keep] % b] = wl.new_key[keep]
+    vc[sl[keep] // b, sl[keep] % b] = wl.new_value[keep]
+    return kc, vc
+
+
+def small_llama(seed_shift=0, seqs=4, max_ctx=300, keep_logical=True):
+    return gen.make_decode("llama7b-small", seed=gen.SEED_BASE + 2 + seed_shift, dtype="f16",
+                           context_lens=np.random.Generator(np.random.PCG64(7 + seed_shift))
+                           .integers(1, max_ctx, size=seqs, endpoint=True),
+                           num_q_heads=8, num_kv_heads=8, head_dim=128, block_size=16,
+                           num_blocks=160, scale=1 / math.sqrt(128), keep_logical=keep_logical)
+
+
+def small_gqa(block_size=16, dtype="bf16", seqs=5, head_dim=128, keep_logical=True):
+    ctx = np.random.Generator(np.random.PCG64(11)).integers(1, 260, size=seqs, endpoint=True)
+    nb = int(sum(-(-int(c) // block_size) for c in ctx)) + 16
+    return gen.make_decode("gqa-small", seed=gen.SEED_BASE + 3, dtype=dtype, context_lens=ctx,
+                           num_q_heads=8, num_kv_heads=2, head_dim=head_dim,
+                           block_size=block_size, num_blocks=nb, scale=1 / math.sqrt(head_dim),
+                           keep_logical=keep_logical)
+
+
+def small_beams():
+    return gen.beam_search(prompts=2, beams=4, prompt_len=40, max_new=24, num_heads=4,
+                           num_blocks=64, keep_logical=True)
+
+
+def run_decode(lib, wl, kc=None, vc=None, tables=None, query=None, ctx=None, blocked=False):
+    if kc is None:
+        kc, vc = pool_after_step(wl)
+    return oracle.paged_decode(wl.query if query is None else query, kc, vc,
+                               wl.block_tables if tables is None else tables,
+                               wl.context_lens if ctx is None else ctx, wl.scale, wl.dtype,
+                               blocked=blocked, lib=lib)
+
+
+def close(a, b, tol=1e-12):
+    assert np.all(np.isfinite(a)), "non-finite oracle output"
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol * (1 + np.max(np.abs(b))), f"max abs diff {err:g}"
+
+
+# ------------------------------------------------------------------- pins
+def pin_decode_bits_f16(lib):
+    """Every binary16 pattern decodes to numpy's float16 value."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.decode_bits(bits, "f16", lib=lib)
+    assert np.array_equal(got, bits.view(np.float16).astype(np.float64), equal_nan=True)
+
+
+def pin_decode_bits_bf16(lib):
+    """Every bfloat16 pattern decodes to the binary32 with the same upper half."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle.decode_bits(bits, "bf16", lib=lib)
+    with np.errstate(invalid="ignore"):
+        ref = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(got, ref, equal_nan=True)
+
+
+def pin_reshape_layout(lib):
+    """One token lands at element ((block*B + offset)*Hkv + h)*D + d of the
+    [num_blocks][B][Hkv][D] pool, K from key and V from value; nothing else
+    changes; negative slots write nothing; slots past the pool raise bit 2."""
+    nb, b, h, d = 5, 4, 3, 8
+    kc = np.full((nb, b, h, d), 0xAAAA, np.uint16)
+    vc = np.full((nb, b, h, d), 0x5555, np.uint16)
+    key = (np.arange(h * d, dtype=np.uint16) + 1).reshape(1, h, d)
+    value = key + 1000
+    st = oracle.reshape_and_cache(key, value, kc, vc, np.array([2 * b + 3]), b, lib=lib)
+    assert st == 0
+    fk, fv = kc.reshape(-1), vc.reshape(-1)
+    for hh in range(h):
+        for dd in range(d):
+            off = ((2 * b + 3) * h + hh) * d + dd
+            assert fk[off] == key[0, hh, dd] and fv[off] == value[0, hh, dd]
+    assert int((fk != 0xAAAA).sum()) == h * d and int((fv != 0x5555).sum()) == h * d
+    before_k, before_v = kc.copy(), vc.copy()
+    assert oracle.reshape_and_cache(key, value, kc, vc, np.array([-1]), b, lib=lib) == 0
+    assert oracle.reshape_and_cache(key, value, kc, vc, np.array([nb * b]), b, lib=lib) == 2
+    assert np.array_equal(kc, before_k) and np.array_equal(vc, before_v)
+
+
+def pin_reshape_matches_scatter(lib):
+    """The oracle's cache write of the step's tokens equals numpy fancy-index
+    assignment of the same rows into the same slots."""
+    for wl in (gen.tiny(), small_beams()):
+        kc, vc = wl.k_cache.copy(), wl.v_cache.copy()
+        for src, dst in wl.block_mapping:
+            kc[dst], vc[dst] = kc[src], vc[src]
+        st = oracle.reshape_and_cache(wl.new_key, wl.new_value, kc, vc, wl.slot_mapping,
+                                      wl.block_size, lib=lib)
+        ek, ev = pool_after_step(wl)
+        assert st == 0 and np.array_equal(kc, ek) and np.array_equal(vc, ev)
+
+
+def pin_copy_blocks(lib):
+    """Pairs copy whole K and V blocks in order; src == dst is a no-op; a
+    destination used twice, or also used as a source, raises bit 8."""
+    rng = np.random.Generator(np.random.PCG64(5))
+    kc = rng.integers(0, 65535, size=(6, 4, 2, 8), dtype=np.uint16)
+    vc = rng.integers(0, 65535, size=(6, 4, 2, 8), dtype=np.uint16)
+    ek, ev = kc.copy(), vc.copy()
+    ek[4], ev[4] = kc[1], vc[1]
+    ek[3], ev[3] = kc[0], vc[0]
+    st = oracle.copy_blocks(kc, vc, np.array([[1, 4], [2, 2], [0, 3]]), lib=lib)
+    assert st == 0 and np.array_equal(kc, ek) and np.array_equal(vc, ev)
+    assert oracle.copy_blocks(kc.copy(), vc.copy(), np.array([[1, 4], [2, 4]]), lib=lib) & 8
+    assert oracle.copy_blocks(kc.copy(), vc.copy(), np.array([[1, 4], [4, 2]]), lib=lib) & 8
+
+
+def pin_brute_force_tiny(lib):
+    """The tiny workload against element-by-element Python loops."""
+    wl = gen.tiny()
+    kc, vc = pool_after_step(wl)
+    out, st = run_decode(lib, wl, kc, vc)
+    ref = brute.brute_paged_decode(wl.query, kc, vc, wl.block_tables, wl.context_lens,
+                                   wl.scale, wl.dtype)
+    assert st == 0
+    close(out, ref)
+
+
+def pin_contiguous(lib):
+    """Paged attention equals textbook softmax(scale q K^T) V (numpy einsum +
+    scipy softmax) on the un-paged per-sequence K/V: paging changes only
+    where the bytes are ([Manager, 第二部分 PagedAttention 的核心思想])."""
+    for wl in (gen.tiny(), small_llama(), small_gqa(), small_gqa(block_size=8, dtype="f16"),
+               small_gqa(block_size=32, head_dim=64), small_beams()):
+        out, st = run_decode(lib, wl)
+        ref = brute.contiguous_attention(wl.query, wl.keys, wl.values, wl.context_lens,
+                                         wl.scale, wl.dtype)
+        assert st == 0
+        close(out, ref)
+
+
+def pin_permutation_invariance(lib):
+    """Relabelling physical blocks (moving every block to pi(b) and mapping
+    the tables through pi) leaves the output bit-identical."""
+    wl = small_gqa()
+    kc, vc = pool_after_step(wl)
+    pi = np.random.Generator(np.random.PCG64(3)).permutation(wl.num_blocks)
+    kc2, vc2 = np.empty_like(kc), np.empty_like(vc)
+    kc2[pi], vc2[pi] = kc, vc
+    t2 = np.where(wl.block_tables >= 0, pi[np.maximum(wl.block_tables, 0)], -1).astype(np.int32)
+    a, _ = run_decode(lib, wl, kc, vc)
+    b, _ = run_decode(lib, wl, kc2, vc2, tables=t2)
+    assert np.array_equal(a, b)
+
+
+def pin_gqa_equals_repeated_mha(lib):
+    """Query head h reads kv head h // (Hq/Hkv): GQA equals MHA over K/V with
+    every kv head repeated Hq/Hkv times consecutively."""
+    wl = small_gqa()
+    kc, vc = pool_after_step(wl)
+    g = wl.num_q_heads // wl.num_kv_heads
+    a, _ = run_decode(lib, wl, kc, vc)
+    b, _ = run_decode(lib, wl, np.ascontiguousarray(np.repeat(kc, g, axis=2)),
+                      np.ascontiguousarray(np.repeat(vc, g, axis=2)))
+    assert np.array_equal(a, b)
+
+
+def pin_single_token(lib):
+    """A one-token context returns that token's V row exactly."""
+    wl = small_llama()
+    kc, vc = pool_after_step(wl)
+    ctx = np.ones(wl.num_seqs, dtype=np.int32)
+    out, _ = run_decode(lib, wl, kc, vc, ctx=ctx)
+    b = wl.block_size
+    for s in range(wl.num_seqs):
+        blk = wl.block_tables[s, 0]
+        v0 = vc[blk, 0].view(np.float16).astype(np.float64)           # [Hkv][D]
+        g = wl.num_q_heads // wl.num_kv_heads
+        assert np.array_equal(out[s], np.repeat(v0, g, axis=0)), b
+
+
+def pin_equal_keys_mean(lib):
+    """When every key is the same, the weights are uniform and the output is
+    the mean of the V rows."""
+    wl = small_llama(seqs=3)
+    kc, vc = pool_after_step(wl)
+    kc[:] = kc[wl.block_tables[0, 0], 0]
+    out, _ = run_decode(lib, wl, kc, vc)
+    for s in range(wl.num_seqs):
+        v = brute._f64(wl.values[s], wl.dtype)                         # [ctx][Hkv][D]
+        close(out[s], v.mean(0))
+
+
+def pin_closed_form_weights(lib):
+    """q = e_0, K_t = a_t e_0, V_t = e_t, scale 1: the output row is the
+    softmax of (a_t), i.e. exp(a_t) / sum exp(a_u), in closed form."""
+    a = [0.0, 1.0, 2.0, -1.5, 0.5, 3.0, 2.0, -4.0, 0.0, 1.0, 1.25, -0.75, 2.5, 0.0, 0.0, 1.0,
+         0.5, -2.0, 3.5]                                              # 19 tokens: ragged tail
+    n, d, b = len(a), 32, 16
+    kc = np.zeros((4, b, 1, d), np.uint16)
+    vc = np.zeros((4, b, 1, d), np.uint16)
+    table = np.array([[2, 0, -1]], np.int32)
+    for t in range(n):
+        blk, off = table[0, t // b], t % b
+        kc[blk, off, 0, 0] = np.float16(a[t]).view(np.uint16)
+        vc[blk, off, 0, t] = F16_ONE
+    q = np.zeros((1, 1, d), np.uint16)
+    q[0, 0, 0] = F16_ONE
+    out, st = oracle.paged_decode(q, kc, vc, table, np.array([n], np.int32), 1.0, "f16", lib=lib)
+    z = sum(math.exp(x) for x in a)
+    ref = np.zeros(d)
+    ref[:n] = [math.exp(x) / z for x in a]
+    assert st == 0
+    close(out[0, 0], ref, tol=1e-14)
+
+
+def pin_blocked_equals_direct(lib):
+    """The five blocked-softmax steps of [Practice §5.1 分块Softmax算法] give
+    the direct softmax result."""
+    for wl in (small_gqa(block_size=8), small_gqa(block_size=32), small_llama()):
+        a, _ = run_decode(lib, wl)
+        b, _ = run_decode(lib, wl, blocked=True)
+        close(b, a)
+
+
+def pin_large_magnitude(lib):
+    """Scores of several thousand (q scaled by 1000) stay finite thanks to the
+    max subtraction, and each output is a convex combination of V rows."""
+    wl = small_llama(seqs=3)
+    q = (wl.query.view(np.float16).astype(np.float32) * 1000).astype(np.float16).view(np.uint16)
+    kc, vc = pool_after_step(wl)
+    out, _ = run_decode(lib, wl, kc, vc, query=q)
+    assert np.all(np.isfinite(out))
+    for s in range(wl.num_seqs):
+        v = brute._f64(wl.values[s], wl.dtype)
+        assert np.all(out[s] >= v.min(0) - 1e-9) and np.all(out[s] <= v.max(0) + 1e-9)
+
+
+def pin_edge_contexts(lib):
+    """Empty context -> zero row, status 0; negative or longer-than-table
+    context -> zero row, bit 4; a table entry outside the pool -> bit 1 and
+    that block's tokens are left out of the softmax."""
+    wl = small_llama(seqs=4)
+    kc, vc = pool_after_step(wl)
+    ctx = wl.context_lens.copy()
+    ctx[0] = 0
+    out, st = run_decode(lib, wl, kc, vc, ctx=ctx)
+    assert st == 0 and not out[0].any()
+    ctx[0] = -3
+    out, st = run_decode(lib, wl, kc, vc, ctx=ctx)
+    assert st == 4 and not out[0].any()
+    ctx[0] = wl.max_blocks_per_seq * wl.block_size + 1
+    out, st = run_decode(lib, wl, kc, vc, ctx=ctx)
+    assert st == 4 and not out[0].any()
+    # drop block 0 of the longest sequence
+    s = int(np.argmax(wl.context_lens))
+    tables = wl.block_tables.copy()
+    tables[s, 0] = wl.num_blocks + 7
+    out, st = run_decode(lib, wl, kc, vc, tables=tables)
+    assert st == 1
+    b = wl.block_size
+    keys = [k[b:] if i == s else k for i, k in enumerate(wl.keys)]
+    vals = [v[b:] if i == s else v for i, v in enumerate(wl.values)]
+    lens = np.array([len(k) for k in keys], np.int32)
+    ref = brute.contiguous_attention(wl.query, keys, vals, lens, wl.scale, wl.dtype)
+    close(out, ref)
+
+
+def pin_rows_match_full(lib):
+    """The sampled-row entry point returns exactly the full run's rows."""
+    wl = small_gqa()
+    kc, vc = pool_after_step(wl)
+    full, _ = run_decode(lib, wl, kc, vc)
+    rows = np.array([[0, 0], [2, 5], [4, 7], [1, 3]], np.int32)
+    got, _ = oracle.paged_decode_rows(rows, wl.query, kc, vc, wl.block_tables,
+                                      wl.context_lens, wl.scale, wl.dtype, lib=lib)
+    assert np.array_equal(got, full[rows[:, 0], rows[:, 1]])
+
+
+PINS = {name: fn for name, fn in globals().items() if name.startswith("pin_")}

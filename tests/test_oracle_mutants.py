@@ -1,0 +1,59 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case copies the oracle's C source, plants one mistake by text
+substitution (a dropped term, a wrong sign or index, a transposed layout, a
+swapped operand), builds it into a temporary library and runs the whole pin
+battery against it: at least one pin must fail.  Nothing here touches a GPU.
+"""
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import oracle_pins
+
+MUTANTS = {
+    "gqa_head_mapping": ("const int32_t g = h / group;", "const int32_t g = h % num_kv_heads;"),
+    "dropped_scale": ("x[t] = scale * acc;", "x[t] = acc;"),
+    "reversed_offset": ("(phys * block_size + t % block_size)",
+                        "(phys * block_size + (block_size - 1 - t % block_size))"),
+    "head_major_layout": ("((phys * block_size + t % block_size) * num_kv_heads + g)",
+                          "((phys * num_kv_heads + g) * block_size + t % block_size)"),
+    "no_max_subtraction": ("double w = exp(x[t] - m) / l;", "double w = exp(x[t]) / l * exp(-m);"),
+    "no_normalisation": ("double w = exp(x[t] - m) / l;", "double w = exp(x[t] - m);"),
+    "sign_error": ("l += exp(x[t] - m);", "l += exp(m - x[t]);"),
+    "f16_exponent_bias": ("expo - 25", "expo - 24"),
+    "bf16_subnormal_scale": ("ldexp((double)frac, -133)", "ldexp((double)frac, -134)"),
+    "cache_write_swapped": ("k_cache[dst] = key[src];", "k_cache[dst] = value[src];"),
+    "copy_only_k": ("v_cache[dst * block_elems + e] = v_cache[src * block_elems + e];", ""),
+    "context_off_by_one": ("const int32_t ctx = context_lens[s];",
+                           "const int32_t ctx = context_lens[s] - 1;"),
+    "cache_write_slot_block": ("int64_t offset = slot % block_size;",
+                               "int64_t offset = (slot + 1) % block_size;"),
+    "table_row_stride": ("block_tables + (int64_t)s * max_blocks_per_seq",
+                         "block_tables + (int64_t)s * (max_blocks_per_seq - 1)"),
+}
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle._SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, source, tmp_path):
+    old, new = MUTANTS[name]
+    assert source.count(old) >= 1, f"mutation site for {name} not found"
+    src = tmp_path / "mutant.c"
+    src.write_text(source.replace(old, new))
+    lib_path = oracle.build(force=True, src=str(src), out=str(tmp_path / "libmutant.so"))
+    lib = oracle.load(lib_path)
+    caught = []
+    with np.errstate(all="ignore"):
+        for pin_name, pin in oracle_pins.PINS.items():
+            try:
+                pin(lib)
+            except Exception:            # noqa: BLE001 - any failure counts as caught
+                caught.append(pin_name)
+    assert caught, f"no pin caught mutant {name}"
