@@ -1,0 +1,456 @@
+"""Benchmark of one decode step (one layer) over a paged KV cache on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is the whole hot path over one batch of synthetic input:
+copy_blocks (when the workload has copy-on-write pairs), reshape_and_cache
+of the step's new tokens, paged_decode (plus its split-context reduction).
+The default workload is the LLaMA-7B-shaped decode: 64 sequences, 32/32
+heads, head_dim 128, block_size 16, fp16, contexts uniform in [128, 2048],
+16384-block pool, one new token per sequence.
+
+Metric: algorithmic HBM bytes of the step / device time (GB/s), with the
+time per step.  The K/V a step reads (about 1.1 GB) is far larger than the
+126 MB L2, so no flush is needed between steps.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (the
+only other code path here that runs it), on a bounded sample of the same
+workload.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the
+workload on its own GPU; nothing is exchanged (the path has no collective).
+The time is the max over ranks and the value sums all ranks' bytes.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged-decode attention HBM GB/s (% of B200 peak) and µs per layer-step"
+UNIT = "GB/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_GLOB_DIR = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = ["paged_kv_cache_415_b200/csrc/paged_decode.cu",
+                  "paged_kv_cache_415_b200/csrc/pa_common.cuh"]
+NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                0x100: "display_clock_setting"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="llama7b",
+                    choices=["tiny", "llama7b", "mistral7b", "beam_search", "long_context"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="shrink the batch (and the pool) for profiling; 0 = the full workload")
+    return ap.parse_args()
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config: str):
+    """DRAM bytes per launch of the decode kernel from a committed ncu
+    summary, if it was taken on the current kernel source."""
+    want = kernel_source_hash()
+    if not os.path.isdir(PROFILE_GLOB_DIR):
+        return None
+    for name in sorted(os.listdir(PROFILE_GLOB_DIR)):
+        if not name.endswith((".md", ".txt")):
+            continue
+        with open(os.path.join(PROFILE_GLOB_DIR, name)) as f:
+            for line in f:
+                m = re.search(r"bench-traffic:\s*workload=(\S+)\s+bytes_per_launch=(\d+)\s+"
+                              r"source_sha256=(\w+)", line)
+                if m and m.group(1) == config and m.group(3) == want:
+                    return int(m.group(2))
+    return None
+
+
+class ClockSampler:
+    """Polls NVML (SM clock, clock-event reasons) in a thread while the
+    timed region runs."""
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            handle = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                handle = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:   # noqa: BLE001
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.h, self.nv = handle, pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:       # noqa: BLE001
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_reasons(self.h))
+            except Exception:   # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable"}
+        names = [n for bit, n in NVML_REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples), "source": "nvml"}
+
+
+def make_workload(config: str, seqs: int = 0):
+    """The named workload; with seqs > 0 a smaller batch of the same shape
+    and a pool sized to it (profiling captures stay a few GB)."""
+    from workloads import generators as gen
+    if seqs <= 0:
+        return gen.CONFIGS[config]()
+    if config == "llama7b":
+        return gen.llama7b(seqs=seqs, num_blocks=seqs * 130 + 64)
+    if config == "mistral7b":
+        return gen.mistral7b(seqs=seqs, num_blocks=seqs * 520 + 64)
+    if config == "long_context":
+        return gen.long_context(seqs=seqs, num_blocks=seqs * 2048 + 64)
+    if config == "beam_search":
+        return gen.beam_search(prompts=max(1, seqs // 4))
+    return gen.CONFIGS[config]()
+
+
+def workload_config(wl, partition_size, l2_note):
+    return {"workload": f"{wl.name}: {wl.num_seqs} seqs, {wl.num_q_heads}/{wl.num_kv_heads} heads, "
+                        f"head_dim {wl.head_dim}, block {wl.block_size}, {wl.dtype}, "
+                        f"contexts {int(wl.context_lens.min())}..{int(wl.context_lens.max())} "
+                        f"(sum {int(wl.context_lens.sum())}), pool {wl.num_blocks} blocks, "
+                        f"{wl.num_new_tokens} new tokens, {int(wl.block_mapping.shape[0])} block copies",
+            "num_seqs": wl.num_seqs, "num_q_heads": wl.num_q_heads,
+            "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim,
+            "block_size": wl.block_size, "partition_size": partition_size,
+            "layers": 1, "l2": l2_note}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+
+class OracleStep:
+    """The oracle's whole step (block copies, cache write, fp64 decode of the
+    first ``max_seqs`` sequences) on host copies of the workload."""
+
+    def __init__(self, wl, max_seqs=None):
+        import oracle
+        from workloads import byte_model as bm
+        self.oracle, self.wl = oracle, wl
+        n = wl.num_seqs if max_seqs is None else max(1, min(max_seqs, wl.num_seqs))
+        self.n = n
+        self.ctx = np.ascontiguousarray(wl.context_lens[:n])
+        self.tables = np.ascontiguousarray(wl.block_tables[:n])
+        self.q = np.ascontiguousarray(wl.query[:n])
+        self.kc, self.vc = wl.k_cache.copy(), wl.v_cache.copy()
+        att = bm.decode_bytes(self.ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                              wl.block_size, 2)
+        full = bm.step_bytes(wl)
+        self.bytes = att["total"] + full["append"] + full["copy"]
+        self.threads = oracle.max_threads()
+
+    def run(self) -> float:
+        o, wl = self.oracle, self.wl
+        t0 = time.perf_counter()
+        if wl.block_mapping.shape[0]:
+            o.copy_blocks(self.kc, self.vc, wl.block_mapping)
+        if wl.num_new_tokens:
+            o.reshape_and_cache(wl.new_key, wl.new_value, self.kc, self.vc, wl.slot_mapping,
+                                wl.block_size)
+        o.paged_decode(self.q, self.kc, self.vc, self.tables, self.ctx, wl.scale, wl.dtype)
+        return time.perf_counter() - t0
+
+    def describe(self) -> str:
+        wl = self.wl
+        return (f"{wl.name}: one full step (block copies, all {wl.num_new_tokens} new tokens, "
+                f"fp64 decode of {self.n} of {wl.num_seqs} sequences)")
+
+
+def oracle_sample_time(wl, seconds: float):
+    """Repeat the oracle's full step until ``seconds`` have passed (at least
+    once).  Returns (GB/s, seconds per step, sample description, threads)."""
+    st = OracleStep(wl)
+    reps, total = 0, 0.0
+    while reps == 0 or total < seconds:
+        total += st.run()
+        reps += 1
+    per = total / reps
+    return st.bytes / per / 1e9, per, f"{st.describe()}, repeated {reps}x in {total:.1f}s", st.threads
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = make_workload(args.config, args.seqs)
+    # size the per-step sample so warm-up + timed steps end within ~2 minutes
+    probe = OracleStep(wl, max_seqs=max(1, wl.num_seqs // 8))
+    per_seq = probe.run() / probe.n
+    del probe
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    st = OracleStep(wl, max_seqs=int(max(1, min(wl.num_seqs, budget / max(per_seq, 1e-9)))))
+    for _ in range(args.warmup):
+        st.run()
+    times = [st.run() for _ in range(args.steps)]
+    per_step = statistics.mean(times)
+    value = st.bytes / per_step / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(per_step * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, None, "host memory"),
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": st.threads,
+                             "kind": "oracle", "sample": st.describe() + " per step"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+
+    from paged_kv_cache_415_b200 import binding as B
+    from workloads import byte_model as bm
+
+    wl = make_workload(args.config, args.seqs)
+    dev = torch.device("cuda", local)
+    tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
+
+    def up(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(tdt)
+
+    k_cache, v_cache = up(wl.k_cache), up(wl.v_cache)
+    query = up(wl.query)
+    new_key, new_value = up(wl.new_key), up(wl.new_value)
+    slot_mapping = torch.from_numpy(wl.slot_mapping).to(dev)
+    block_tables = torch.from_numpy(wl.block_tables).to(dev)
+    context_lens = torch.from_numpy(wl.context_lens).to(dev)
+    block_mapping = torch.from_numpy(np.ascontiguousarray(wl.block_mapping)).to(dev)
+    out = torch.empty_like(query)
+    d_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    mcl = wl.max_context_len
+    part = B.pa_paged_decode_partition_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                            wl.head_dim, wl.block_size, mcl, wl.partition_size)
+    ws_bytes = B.pa_paged_decode_workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                                wl.head_dim, wl.block_size, mcl, part)
+    workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    max_parts = -(-mcl // part) if mcl > 0 else 1
+    n_pairs = int(wl.block_mapping.shape[0])
+    stream = torch.cuda.current_stream(dev)
+
+    def cache_ops():
+        if n_pairs:
+            B.pa_copy_blocks(k_cache, v_cache, block_mapping, d_status, stream)
+        if wl.num_new_tokens:
+            B.pa_reshape_and_cache(new_key, new_value, k_cache, v_cache, slot_mapping, d_status,
+                                   stream)
+
+    def decode():
+        B.pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl, wl.scale,
+                          part, workspace, d_status, stream)
+
+    launches_per_step = (1 if n_pairs else 0) + (1 if wl.num_new_tokens else 0) + 1 + \
+        (1 if max_parts > 1 else 0)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # warm-up
+    for _ in range(args.warmup):
+        cache_ops()
+        decode()
+    barrier()
+    if int(d_status.item()) != 0 or not torch.isfinite(out.float()).all():
+        raise SystemExit(f"rank {rank}: bad step (status {int(d_status.item())})")
+
+    # timed region: K steps; events bracket the decode kernels of every step
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier()
+    with sampler:
+        start.record(stream)
+        for i in range(args.steps):
+            cache_ops()
+            ev[i][0].record(stream)
+            decode()
+            ev[i][1].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    decode_ms = [a.elapsed_time(b) for a, b in ev]
+
+    # end to end through the public API: pinned host inputs -> device -> step -> host output
+    from paged_kv_cache_415_b200.step import DecodeStep
+    stepper = DecodeStep(k_cache, v_cache, wl.num_seqs, wl.num_q_heads, mcl, part)
+    host = {"query": torch.from_numpy(wl.query.view(np.int16)).view(tdt).pin_memory(),
+            "block_tables": torch.from_numpy(wl.block_tables).pin_memory(),
+            "context_lens": torch.from_numpy(wl.context_lens).pin_memory(),
+            "out": torch.empty(out.shape, dtype=tdt).pin_memory()}
+    devb = {"query": torch.empty_like(query), "block_tables": torch.empty_like(block_tables),
+            "context_lens": torch.empty_like(context_lens), "out": torch.empty_like(out)}
+    if wl.num_new_tokens:
+        host["new_key"] = torch.from_numpy(wl.new_key.view(np.int16)).view(tdt).pin_memory()
+        host["new_value"] = torch.from_numpy(wl.new_value.view(np.int16)).view(tdt).pin_memory()
+        host["slot_mapping"] = torch.from_numpy(wl.slot_mapping).pin_memory()
+        for k in ("new_key", "new_value", "slot_mapping"):
+            devb[k] = torch.empty_like(host[k], device=dev)
+    if n_pairs:
+        host["block_mapping"] = torch.from_numpy(np.ascontiguousarray(wl.block_mapping)).pin_memory()
+        devb["block_mapping"] = torch.empty_like(host["block_mapping"], device=dev)
+    h2d = sum(t.numel() * t.element_size() for k, t in host.items() if k != "out")
+    d2h = host["out"].numel() * host["out"].element_size()
+    for _ in range(max(3, args.warmup)):
+        stepper.run_from_host(host, devb, wl.scale, stream)
+    barrier()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        stepper.run_from_host(host, devb, wl.scale, stream)
+    e_stop.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_stop)
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, e2e_ms, statistics.mean(decode_ms)], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms, decode_avg = [float(x) for x in t.tolist()]
+    else:
+        decode_avg = statistics.mean(decode_ms)
+
+    step = bm.step_bytes(wl)
+    per_step_ms = elapsed_ms / args.steps
+    value = world * step["total"] * args.steps / (elapsed_ms * 1e-3) / 1e9
+    e2e_value = world * step["total"] * args.steps / (e2e_ms * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+    achieved = step["attention"] / (decode_avg * 1e-3) / 1e9
+    traffic = profiled_traffic(args.config)
+    clocks = sampler.summary()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        g, _, desc, threads = oracle_sample_time(wl, args.cpu_seconds)
+        cpu = {"value": round(g, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": desc}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    l2 = (f"no flush: {step['kv'] / 1e9:.2f} GB of K/V per step > 126 MB L2"
+          if step["kv"] > 4 * 126e6 else "working set smaller than L2 (values include L2 hits)")
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "data": "synthetic", "config": workload_config(wl, part, l2),
+        "us_per_layer_step": round(per_step_ms * 1e3, 2),
+        "kv_tokens_per_s": round(world * int(wl.context_lens.sum()) * args.steps / (elapsed_ms * 1e-3)),
+        "pct_of_hbm_peak": round(100 * value / world / peak, 2),
+        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + paged_decode_reduce_kernel",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic, "algorithmic_bytes_per_launch": step["attention"],
+                     "avg_launch_us": round(decode_avg * 1e3, 2)},
+        "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+        "bytes_per_step": step,
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,241 @@
+/*
+ * pa.h -- C ABI of the paged-KV-cache decode library (libpa.so, sm_100a).
+ *
+ * Three operations make one decode step of one attention layer:
+ *
+ *   pa_copy_blocks        copy-on-write block copies decided by the host
+ *   pa_reshape_and_cache  write this step's new K/V rows into their slots
+ *   pa_paged_decode       single-query attention over each sequence's
+ *                         context, reached through its block table
+ *
+ * Pages cited (title, then section):
+ *   [VM-paging] "vLLM用虚拟内存分页思想管理KV Cache"
+ *   [Practice]  "PagedAttention：大模型KV Cache分页管理优化实践"
+ *   [Manager]   "深入解析 vLLM 的 KV Cache 管理器：从内存碎片到 PagedAttention 的完整技术剖析"
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.  Every pointer argument is caller-owned DEVICE memory unless its
+ *   comment says otherwise.  The library allocates nothing, keeps no state
+ *   between calls, never synchronises the device and only enqueues work on
+ *   `stream` (a cudaStream_t; NULL is the legacy default stream).  Calls
+ *   return as soon as the work is enqueued.
+ *
+ * Element types.  query, key, value, k_cache, v_cache and out share one
+ *   element type: IEEE binary16 (PA_DTYPE_F16) or bfloat16 (PA_DTYPE_BF16).
+ *   Attention accumulates in fp32 and rounds the output to nearest even.
+ *
+ * KV-cache layout (one layer; K and V in two pools of the same shape):
+ *   k_cache, v_cache : [num_blocks][block_size][num_kv_heads][head_dim],
+ *   row-major and contiguous.  A physical block holds block_size tokens of
+ *   every kv head ([Practice §3.1 物理块分配器设计]).  The slot of a token is
+ *   physical_block * block_size + offset_in_block, so the pools are also
+ *   [num_blocks * block_size][num_kv_heads][head_dim] indexed by slot.
+ *   Pool base addresses must be 16-byte aligned (256-byte alignment, which
+ *   every CUDA allocation has, is what the pages recommend:
+ *   [Practice §4.2 访存优化技术]).
+ *
+ * Synchronous errors (return value; nothing is enqueued when it is not
+ *   PA_OK):
+ *   PA_ERR_INVALID_ARG  null pointer, negative or zero size where a positive
+ *                       one is needed, num_q_heads not a multiple of
+ *                       num_kv_heads, partition_size not a multiple of
+ *                       block_size, workspace too small, a pointer that is
+ *                       not 16-byte aligned;
+ *   PA_ERR_UNSUPPORTED  head_dim not 64 or 128, block_size not 8, 16 or 32,
+ *                       num_q_heads / num_kv_heads not 1, 2, 4 or 8, an
+ *                       unknown dtype;
+ *   PA_ERR_CUDA         the launch failed (cudaGetLastError after launch).
+ *
+ * Asynchronous data errors (device status word).  `d_status` is an optional
+ *   (may be NULL) device int32 that the kernels OR bits into; the caller
+ *   clears it.  The offending token or block is skipped and the kernels
+ *   finish normally (they never trap and every wait they make is bounded):
+ *   PA_STATUS_BAD_BLOCK    a block id outside [0, num_blocks) -- in a block
+ *                          table (that block's tokens are left out of the
+ *                          softmax) or in a copy pair (the pair is skipped);
+ *   PA_STATUS_BAD_SLOT     a slot at or beyond num_blocks * block_size (the
+ *                          token is not written; negative slots are padding
+ *                          and are skipped silently);
+ *   PA_STATUS_BAD_CONTEXT  a context length that is negative, larger than
+ *                          max_context_len or larger than
+ *                          max_blocks_per_seq * block_size (the output row is
+ *                          written as zeros);
+ *   PA_STATUS_COPY_CONFLICT a copy destination that appears twice or is also
+ *                          a source in the same call (those blocks' contents
+ *                          are unspecified);
+ *   PA_STATUS_TIMEOUT      a bounded wait for an asynchronous copy gave up
+ *                          (should never happen; the output is unspecified).
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,
+    PA_ERR_UNSUPPORTED = 2,
+    PA_ERR_CUDA = 3
+} pa_status;
+
+typedef enum pa_dtype {
+    PA_DTYPE_F16 = 0,
+    PA_DTYPE_BF16 = 1
+} pa_dtype;
+
+#define PA_STATUS_BAD_BLOCK 1
+#define PA_STATUS_BAD_SLOT 2
+#define PA_STATUS_BAD_CONTEXT 4
+#define PA_STATUS_COPY_CONFLICT 8
+#define PA_STATUS_TIMEOUT 16
+
+/*
+ * pa_reshape_and_cache -- write each new token's K and V rows into its slot.
+ *
+ * Defined by: [Practice §3.3 按需分配策略] step 4 (after the allocator has
+ * found or created room in the sequence's last block, write the new token's
+ * K/V vectors) and [Manager, 第一部分 KV Cache 的核心价值] (each decode step
+ * stores the new token's K and V, then attends over the whole cache).
+ *
+ *   for t < num_tokens with slot = slot_mapping[t] >= 0:
+ *     k_cache[slot][h][d] = key[t][h][d],  v_cache[slot][h][d] = value[t][h][d]
+ *
+ * A bit-exact copy.  Every other cache element is left untouched.
+ *
+ * key, value     [num_tokens][num_kv_heads][head_dim], contiguous, 16-byte aligned.
+ * k_cache, v_cache  the pools (layout above); written in place.
+ * slot_mapping   int64 [num_tokens]; negative = padding token, skipped.
+ * num_tokens     >= 0 (0 enqueues nothing).
+ * num_blocks     pool size in blocks (bounds check of the slots).
+ * d_status       optional; PA_STATUS_BAD_SLOT.
+ */
+PA_API pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                               void* v_cache, const int64_t* slot_mapping,
+                               int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t block_size, int64_t num_blocks, pa_dtype dtype,
+                               int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks -- the data copy of copy-on-write.
+ *
+ * Defined by: [VM-paging, 写时复制与块共享机制] and [Practice §4.1 共享内存管理]
+ * steps 1-4: a sequence that must modify a block shared with others (count
+ * above 1) gets a new block holding a copy of the original's data, remaps
+ * its table entry and drops one reference on the original.  The host decides
+ * which blocks to copy and keeps the reference counts; this call performs
+ * step 2 (copy the original data) for every pair at once.
+ *
+ *   for i < num_pairs: block block_mapping[i][1] of k_cache and v_cache
+ *                      becomes a bit-exact copy of block block_mapping[i][0]
+ *
+ * block_mapping  int64 [num_pairs][2] of (src, dst) physical block ids.
+ *                src == dst is a no-op.  Destinations must be distinct and
+ *                must not be sources of other pairs (else
+ *                PA_STATUS_COPY_CONFLICT).
+ * num_pairs      >= 0 (0 enqueues nothing).
+ * d_status       optional; PA_STATUS_BAD_BLOCK, PA_STATUS_COPY_CONFLICT.
+ */
+PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                         int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t block_size, int64_t num_blocks, pa_dtype dtype,
+                         int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_paged_decode_partition_size -- the context partition length (tokens)
+ * pa_paged_decode uses: `partition_size` itself when it is positive, else
+ * the library's choice for this shape.  Host-only; returns 0 for arguments
+ * pa_paged_decode would reject.
+ */
+PA_API int32_t pa_paged_decode_partition_size(int32_t num_seqs, int32_t num_q_heads,
+                                       int32_t num_kv_heads, int32_t head_dim,
+                                       int32_t block_size, int32_t max_context_len,
+                                       int32_t partition_size);
+
+/*
+ * pa_paged_decode_workspace_size -- bytes of scratch pa_paged_decode needs
+ * for these arguments (0 when every context fits in one partition).  The
+ * workspace holds, per (sequence, query head, partition), the partition's
+ * running max, exp-sum and normalised partial output in fp32.  Host-only.
+ */
+PA_API size_t pa_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                      int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, int32_t max_context_len,
+                                      int32_t partition_size);
+
+/*
+ * pa_paged_decode -- single-query (decode) attention over a paged KV cache.
+ *
+ * Defined by: [VM-paging, PagedAttention的注意力计算流程] (for each request and
+ * head: look up the physical blocks in the block table, score the query
+ * against the Keys of every block, normalise with softmax, sum the Values
+ * with those weights, all in one kernel launch); [Manager, 第二部分
+ * PagedAttention 的核心思想] step 4 (the kernel reassembles K/V through the
+ * block table at run time); [Practice §3.2 块表与地址转换] (logical block j ->
+ * table[j] -> physical id -> base + offset); the softmax is taken blockwise
+ * as [Practice §5.1 分块Softmax算法] lays out (per-block max, global max,
+ * rescaled exp-sum, normalise), here in its single-pass running form, and
+ * across context partitions by a second, reduction kernel.
+ *
+ * For sequence s, query head h, kv head g = h / (num_q_heads / num_kv_heads),
+ * token t < context_lens[s] stored at
+ *   k_cache[block_tables[s][t / block_size]][t % block_size][g][:]:
+ *   x_t = scale * sum_d query[s][h][d] * K_t[d]
+ *   out[s][h][:] = sum_t softmax(x)_t * V_t[:]
+ * An empty context (context_lens[s] == 0) gives a zero row.
+ *
+ * out            [num_seqs][num_q_heads][head_dim], 16-byte aligned; written.
+ * query          [num_seqs][num_q_heads][head_dim], 16-byte aligned.
+ * block_tables   int32 [num_seqs][max_blocks_per_seq]; entries past a
+ *                sequence's last block are never read.
+ * context_lens   int32 [num_seqs]; includes the token appended this step.
+ * max_context_len  host value: an upper bound of context_lens (it sizes the
+ *                grid; the library never reads device data back).
+ * scale          multiplier of q.k before the softmax (e.g. 1/sqrt(head_dim)).
+ * partition_size 0 = library's choice; else a multiple of block_size.
+ *                Contexts longer than one partition are split; the partial
+ *                results go to `workspace` and a reduction kernel merges them.
+ * workspace      device scratch of at least
+ *                pa_paged_decode_workspace_size(...) bytes, 16-byte aligned
+ *                (may be NULL when that size is 0).  Its contents on entry do
+ *                not matter; calls that share it must not overlap.
+ * d_status       optional; PA_STATUS_BAD_BLOCK, PA_STATUS_BAD_CONTEXT,
+ *                PA_STATUS_TIMEOUT.
+ *
+ * Deterministic: the same inputs give bit-identical outputs, whatever the
+ * physical placement of the blocks.
+ */
+PA_API pa_status pa_paged_decode(void* out, const void* query, const void* k_cache,
+                          const void* v_cache, const int32_t* block_tables,
+                          const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads,
+                          int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                          int32_t max_blocks_per_seq, int64_t num_blocks,
+                          int32_t max_context_len, float scale, int32_t partition_size,
+                          void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                          int32_t* d_status, pa_stream_t stream);
+
+/* Human-readable name of a pa_status (static string, never NULL). */
+PA_API const char* pa_status_string(pa_status status);
+
+/* Library version, e.g. "0.1.0" (static string). */
+PA_API const char* pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,150 @@
+"""Thin ctypes binding of libpa.so: argument marshalling only.
+
+Every function has the name of the C entry point it calls and takes torch
+CUDA tensors (for device memory) plus the few host scalars the C call needs.
+All arithmetic runs in the library's CUDA kernels; nothing here computes a
+result, and there is no fallback: if libpa.so is missing or cannot be
+loaded, importing this module raises.
+
+Errors: a non-PA_OK return raises ``PAError`` carrying the status name.
+Asynchronous data errors land in the optional ``d_status`` device int32
+tensor (bits PA_STATUS_*).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+
+PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
+PA_DTYPE_F16, PA_DTYPE_BF16 = 0, 1
+PA_STATUS_BAD_BLOCK = 1
+PA_STATUS_BAD_SLOT = 2
+PA_STATUS_BAD_CONTEXT = 4
+PA_STATUS_COPY_CONFLICT = 8
+PA_STATUS_TIMEOUT = 16
+
+_DTYPES = {torch.float16: PA_DTYPE_F16, torch.bfloat16: PA_DTYPE_BF16}
+
+# Every entry point declared in include/pa.h.
+EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_size",
+           "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_status_string",
+           "pa_version")
+
+
+class PAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {pa_status_string(code)}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run `python -m paged_kv_cache_415_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                            ctypes.c_size_t)
+    lib.pa_reshape_and_cache.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i32, p, p]
+    lib.pa_reshape_and_cache.restype = i32
+    lib.pa_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i64, i32, p, p]
+    lib.pa_copy_blocks.restype = i32
+    lib.pa_paged_decode_partition_size.argtypes = [i32] * 7
+    lib.pa_paged_decode_partition_size.restype = i32
+    lib.pa_paged_decode_workspace_size.argtypes = [i32] * 7
+    lib.pa_paged_decode_workspace_size.restype = sz
+    lib.pa_paged_decode.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64, i32, f32,
+                                    i32, p, sz, i32, p, p]
+    lib.pa_paged_decode.restype = i32
+    lib.pa_status_string.argtypes = [i32]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = ctypes.c_char_p
+    return lib
+
+
+LIB = _load()
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    try:
+        return _DTYPES[t.dtype]
+    except KeyError:
+        return 99          # rejected by the library as PA_ERR_UNSUPPORTED
+
+
+def _check(fn: str, code: int) -> None:
+    if code != PA_OK:
+        raise PAError(fn, code)
+
+
+def pa_status_string(code: int) -> str:
+    return LIB.pa_status_string(int(code)).decode()
+
+
+def pa_version() -> str:
+    return LIB.pa_version().decode()
+
+
+def pa_reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, d_status=None,
+                         stream=None) -> None:
+    """key/value [T][Hkv][D]; k_cache/v_cache [num_blocks][B][Hkv][D];
+    slot_mapping int64 [T]."""
+    num_blocks, block_size, hkv, d = k_cache.shape
+    _check("pa_reshape_and_cache", LIB.pa_reshape_and_cache(
+        _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+        int(slot_mapping.shape[0]), hkv, d, block_size, num_blocks, _dtype(k_cache),
+        _ptr(d_status), _stream(stream)))
+
+
+def pa_copy_blocks(k_cache, v_cache, block_mapping, d_status=None, stream=None) -> None:
+    """block_mapping int64 [P][2] of (src, dst) block ids, on the device."""
+    num_blocks, block_size, hkv, d = k_cache.shape
+    _check("pa_copy_blocks", LIB.pa_copy_blocks(
+        _ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), int(block_mapping.shape[0]), hkv, d,
+        block_size, num_blocks, _dtype(k_cache), _ptr(d_status), _stream(stream)))
+
+
+def pa_paged_decode_partition_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                   max_context_len, partition_size=0) -> int:
+    return int(LIB.pa_paged_decode_partition_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                  block_size, max_context_len, partition_size))
+
+
+def pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                   max_context_len, partition_size=0) -> int:
+    return int(LIB.pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                  block_size, max_context_len, partition_size))
+
+
+def pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, max_context_len,
+                    scale, partition_size=0, workspace=None, d_status=None, stream=None) -> None:
+    """out/query [S][Hq][D]; k_cache/v_cache [num_blocks][B][Hkv][D];
+    block_tables int32 [S][max_blocks_per_seq]; context_lens int32 [S];
+    workspace: a uint8 device tensor of at least
+    pa_paged_decode_workspace_size(...) bytes (or None when that is 0)."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_paged_decode", LIB.pa_paged_decode(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), num_seqs, hq, hkv, d, block_size, int(block_tables.shape[1]),
+        num_blocks, int(max_context_len), float(scale), int(partition_size), _ptr(workspace),
+        ws_bytes, _dtype(query), _ptr(d_status), _stream(stream)))

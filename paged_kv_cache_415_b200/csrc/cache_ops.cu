@@ -1,0 +1,158 @@
+// cache_ops.cu -- the two kernels that feed the paged KV cache:
+//   reshape_and_cache : scatter this step's new K/V rows into their slots
+//   copy_blocks       : copy-on-write block copies
+//
+// Both are bit copies moved in 16-byte vectors; neither looks at values,
+// so one instance serves fp16 and bf16.
+//
+// Pages cited (title, then section):
+//   [VM-paging] "vLLM用虚拟内存分页思想管理KV Cache"
+//   [Practice]  "PagedAttention：大模型KV Cache分页管理优化实践"
+//   [Manager]   "深入解析 vLLM 的 KV Cache 管理器：从内存碎片到 PagedAttention 的完整技术剖析"
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+#include "pa_common.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+constexpr int kCopyThreads = 256;
+constexpr int kCopyVecsPerThread = 4;
+
+// One CTA per new token.  The pools are [num_slots][Hkv][D], so a token's
+// K row (all kv heads) is one contiguous run of row_vecs 16-byte vectors at
+// slot * row_vecs ([Practice §3.3 按需分配策略], step 4: write the new
+// token's KV vectors into the slot the allocator gave it).
+__global__ void __launch_bounds__(128) reshape_and_cache_kernel(
+    const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ k_cache,
+    uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int32_t row_vecs,
+    int64_t num_slots, int32_t* d_status)
+{
+    const int64_t t = blockIdx.x;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;                       // padding token
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_SLOT);
+        return;
+    }
+    const uint4* ks = key + t * row_vecs;
+    const uint4* vs = value + t * row_vecs;
+    uint4* kd = k_cache + slot * row_vecs;
+    uint4* vd = v_cache + slot * row_vecs;
+    for (int32_t i = threadIdx.x; i < row_vecs; i += blockDim.x) {
+        const uint4 a = ld_nc_v4(ks + i);
+        const uint4 b = ld_nc_v4(vs + i);
+        kd[i] = a;
+        vd[i] = b;
+    }
+}
+
+// Grid (pair, K-or-V, chunk of the block).  Whole-block bit copy src -> dst
+// ([VM-paging, 写时复制与块共享机制]; [Practice §4.1 共享内存管理] step 2).
+// The first CTA of each pair also checks the pair against all the others:
+// a destination that appears twice, or that another pair reads, makes the
+// result order-dependent, which is flagged.
+__global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
+    uint4* __restrict__ k_cache, uint4* __restrict__ v_cache,
+    const int64_t* __restrict__ block_mapping, int32_t num_pairs, int64_t block_vecs,
+    int64_t num_blocks, int32_t* d_status)
+{
+    const int32_t pair = blockIdx.x;
+    const int64_t src = block_mapping[2 * pair];
+    const int64_t dst = block_mapping[2 * pair + 1];
+    const bool first_cta = blockIdx.y == 0 && blockIdx.z == 0;
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+        if (first_cta && threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_BLOCK);
+        return;
+    }
+    if (first_cta && d_status != nullptr) {
+        bool conflict = false;
+        for (int32_t j = threadIdx.x; j < num_pairs; j += blockDim.x) {
+            if (j == pair) continue;
+            const int64_t sj = block_mapping[2 * j], dj = block_mapping[2 * j + 1];
+            if (dj == dst && j < pair) conflict = true;
+            if (sj == dst && sj != dj) conflict = true;
+        }
+        if (__syncthreads_or(conflict) && threadIdx.x == 0) status_or(d_status, PA_STATUS_COPY_CONFLICT);
+    }
+    if (src == dst) return;
+    uint4* base = blockIdx.y == 0 ? k_cache : v_cache;
+    const uint4* s = base + src * block_vecs;
+    uint4* d = base + dst * block_vecs;
+    const int64_t begin = static_cast<int64_t>(blockIdx.z) * kCopyThreads * kCopyVecsPerThread;
+    const int64_t end = min(block_vecs, begin + static_cast<int64_t>(kCopyThreads) * kCopyVecsPerThread);
+    uint4 buf[kCopyVecsPerThread];
+#pragma unroll
+    for (int k = 0; k < kCopyVecsPerThread; ++k) {
+        const int64_t i = begin + threadIdx.x + static_cast<int64_t>(k) * kCopyThreads;
+        if (i < end) buf[k] = s[i];
+    }
+#pragma unroll
+    for (int k = 0; k < kCopyVecsPerThread; ++k) {
+        const int64_t i = begin + threadIdx.x + static_cast<int64_t>(k) * kCopyThreads;
+        if (i < end) d[i] = buf[k];
+    }
+}
+
+static pa_status check_pool_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int64_t num_blocks, int32_t dtype)
+{
+    if (num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !supported_dtype(dtype))
+        return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+}  // namespace pa
+
+extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, void* k_cache,
+                                          void* v_cache, const int64_t* slot_mapping,
+                                          int32_t num_tokens, int32_t num_kv_heads,
+                                          int32_t head_dim, int32_t block_size,
+                                          int64_t num_blocks, pa_dtype dtype, int32_t* d_status,
+                                          pa_stream_t stream)
+{
+    using namespace pa;
+    if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+    pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned8(slot_mapping) || (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    const int32_t row_vecs = num_kv_heads * head_dim * 2 / 16;
+    reshape_and_cache_kernel<<<num_tokens, 128, 0, stream>>>(
+        static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, row_vecs,
+        num_blocks * block_size, d_status);
+    return launch_status();
+}
+
+extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                                    int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t block_size, int64_t num_blocks, pa_dtype dtype,
+                                    int32_t* d_status, pa_stream_t stream)
+{
+    using namespace pa;
+    if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+    pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (!k_cache || !v_cache || !block_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned8(block_mapping) ||
+        (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    const int64_t block_vecs = static_cast<int64_t>(block_size) * num_kv_heads * head_dim * 2 / 16;
+    const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kCopyVecsPerThread;
+    const int64_t chunks = (block_vecs + per_cta - 1) / per_cta;
+    if (chunks > 65535) return PA_ERR_UNSUPPORTED;
+    dim3 grid(num_pairs, 2, static_cast<unsigned>(chunks));
+    copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping, num_pairs,
+        block_vecs, num_blocks, d_status);
+    return launch_status();
+}

@@ -1,0 +1,189 @@
+// pa_common.cuh -- device helpers shared by the library's kernels (sm_100a).
+//
+// Inline PTX wrappers for the asynchronous bulk copy engine (cp.async.bulk,
+// global -> shared, completion counted on an mbarrier), mbarrier waits that
+// give up after a bounded time, and fp16 / bf16 <-> fp32 conversions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// A wait for an asynchronous copy gives up after this long (the copy of a
+// few KB normally lands within microseconds).
+constexpr uint64_t kWaitTimeoutNs = 1000ull * 1000ull * 1000ull;   // 1 s
+constexpr uint32_t kWaitMaxPolls = 1u << 30;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+// Makes barrier initialisation visible to the asynchronous proxy.
+__device__ __forceinline__ void fence_barrier_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Orders this thread's earlier shared-memory accesses before later
+// asynchronous-proxy (bulk copy) accesses to shared memory.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// One arrival that also announces `bytes` of copies still to land.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Waits for the barrier phase with the given parity.  Returns false if it
+// has not completed after kWaitTimeoutNs (or kWaitMaxPolls polls).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 0; i < kWaitMaxPolls; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 63u && global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+    return false;
+}
+
+// Asynchronous bulk copy global -> shared of `bytes` (multiple of 16, both
+// addresses 16-byte aligned); its completion is counted on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst_smem, const void* src_gmem, uint32_t bytes,
+                                              uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Same, with an L2 eviction-priority policy (a createpolicy value).
+__device__ __forceinline__ void bulk_copy_g2s_hint(void* dst_smem, const void* src_gmem,
+                                                   uint32_t bytes, uint64_t* bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
+        "%2, [%3], %4;" ::"r"(smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// ---------------------------------------------------------------------------
+// Element types.  Both are 16-bit; a 16-byte vector holds 8 elements.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Elem;
+
+template <>
+struct Elem<__half> {
+    // Two packed binary16 values -> two floats (exact).
+    static __device__ __forceinline__ float2 to_float2(uint32_t w)
+    {
+        __half2 h = *reinterpret_cast<const __half2*>(&w);
+        return __half22float2(h);
+    }
+    // Two floats -> packed binary16, each rounded to nearest even.
+    static __device__ __forceinline__ uint32_t from_float2(float a, float b)
+    {
+        __half2 h = __floats2half2_rn(a, b);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+};
+
+template <>
+struct Elem<__nv_bfloat16> {
+    // bfloat16 is the upper half of a binary32, so widening is a shift.
+    static __device__ __forceinline__ float2 to_float2(uint32_t w)
+    {
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+    static __device__ __forceinline__ uint32_t from_float2(float a, float b)
+    {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        return *reinterpret_cast<const uint32_t*>(&h);
+    }
+};
+
+// 8 packed elements -> 8 floats.
+template <typename T>
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8])
+{
+    float2 a = Elem<T>::to_float2(v.x), b = Elem<T>::to_float2(v.y);
+    float2 c = Elem<T>::to_float2(v.z), d = Elem<T>::to_float2(v.w);
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+    f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+
+template <typename T>
+__device__ __forceinline__ uint4 pack8(const float (&f)[8])
+{
+    uint4 v;
+    v.x = Elem<T>::from_float2(f[0], f[1]);
+    v.y = Elem<T>::from_float2(f[2], f[3]);
+    v.z = Elem<T>::from_float2(f[4], f[5]);
+    v.w = Elem<T>::from_float2(f[6], f[7]);
+    return v;
+}
+
+__device__ __forceinline__ void status_or(int32_t* d_status, int32_t bits)
+{
+    if (d_status != nullptr) atomicOr(d_status, bits);
+}
+
+}  // namespace pa

@@ -1,0 +1,25 @@
+// pa_host.h -- host-side argument checks shared by the C-ABI entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pa.h"
+
+namespace pa {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+inline bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+inline bool supported_head_dim(int32_t d) { return d == 64 || d == 128; }
+inline bool supported_block_size(int32_t b) { return b == 8 || b == 16 || b == 32; }
+inline bool supported_dtype(int32_t t) { return t == PA_DTYPE_F16 || t == PA_DTYPE_BF16; }
+
+// Launch-error check after a kernel launch.
+inline pa_status launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace pa

@@ -1,0 +1,729 @@
+// paged_decode.cu -- single-query attention over a paged KV cache (sm_100a).
+//
+// Kernel 1, paged_decode_kernel: one CTA per (kv head, context partition,
+// sequence).  The CTA carries the G = Hq / Hkv query heads of its kv head,
+// so every K/V byte is read from HBM once for all of them.  Each of its four
+// warps runs its own pipeline over every fourth physical block of the
+// partition:
+//   * the warp's block-table entries are prefetched into one register per
+//     lane (32 blocks per load) and broadcast with a shuffle
+//     ("PagedAttention：大模型KV Cache分页管理优化实践" §3.2: flattened table,
+//     warp-level prefetch);
+//   * each block's K and V rows of this kv head (block_size rows of
+//     head_dim elements each, one contiguous 128/256-byte row per token) are
+//     fetched by the bulk-copy engine (cp.async.bulk) straight into a shared
+//     memory ring of NSTAGE stages, completion counted on one mbarrier per
+//     stage, so NSTAGE - 1 blocks are in flight while one is computed
+//     (§4.2 prefetch, §5.2 overlap of copy and compute);
+//   * scores q.k in fp32: 8 (or 16) lanes share a token row, each holding
+//     16 (or 8) elements of q for every head of the group in registers; the
+//     partial dot products are reduced across those lanes with a transposing
+//     butterfly of warp shuffles;
+//   * the softmax is the blocked form of §5.1 (分块Softmax算法) run online:
+//     per block the local max, the running (global) max, the exp-sum
+//     rescaled to it, then the weighted V rows accumulate into fp32 outputs
+//     rescaled the same way; scores are kept in log2 units (q is
+//     pre-multiplied by scale * log2(e)) so exponentials are exp2.
+// At the end the four warps' (max, sum, output) are merged through shared
+// memory in a fixed order.  A sequence whose context fits one partition gets
+// its output row written directly; otherwise the partition's max, sum and
+// normalised output go to the workspace.
+//
+// Kernel 2, paged_decode_reduce_kernel: one warp per (sequence, query head)
+// with more than one partition merges the partitions with the same rule:
+//   M = max_p m_p,  w_p = l_p * 2^(m_p - M),  out = sum_p w_p Ohat_p / sum_p w_p.
+//
+// The whole computation has a fixed summation order, so results are
+// deterministic and do not depend on where the blocks sit in the pool.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "pa.h"
+#include "pa_common.cuh"
+#include "pa_host.h"
+
+namespace pa {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kDefaultPartition = 512;
+constexpr int kReduceRowsPerCta = 4;
+
+template <int D, int BS, int G>
+struct DecodeShape {
+    static constexpr int LPT = (G == 8 && D == 128) ? 16 : 8;   // lanes per token row
+    static constexpr int RPW = 32 / LPT;                        // token rows per warp pass
+    static constexpr int EPT = D / LPT;                         // elements per lane
+    static constexpr int NCHUNK = EPT / 8;                      // 16-byte chunks per lane
+    // Tokens scored per softmax step: the whole block, or a slice of it so
+    // that a lane never holds more than 16 partial scores.
+    static constexpr int CT_MAX = 16 * RPW / G > RPW ? 16 * RPW / G : RPW;
+    static constexpr int CT = BS < CT_MAX ? BS : CT_MAX;
+    static constexpr int TILES = BS / CT;
+    static constexpr int ITERS = CT / RPW;                      // passes per tile
+    static constexpr int ROW_BYTES = D * 2;
+    static constexpr int TILE_BYTES = BS * ROW_BYTES;           // K (or V) of one block, one head
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int NSTAGE = STAGE_BYTES <= 4096 ? 4 : (STAGE_BYTES <= 8192 ? 3 : 2);
+    static constexpr int NVAL = ITERS * G;                      // partial scores per lane
+    static constexpr int NHELD = NVAL >= LPT ? NVAL / LPT : 1;  // scores per lane after reduce
+    static constexpr int SM_TPL = (CT * G + 31) / 32;           // softmax items per lane
+    static constexpr int WARP_STAGE_BYTES = NSTAGE * STAGE_BYTES;
+    static constexpr int OFF_SCORES = kWarps * WARP_STAGE_BYTES;
+    static constexpr int SCORE_FLOATS = CT * G;
+    static constexpr int OFF_CORR = OFF_SCORES + kWarps * SCORE_FLOATS * 4;
+    static constexpr int CORR_FLOATS = (G + 3) / 4 * 4;
+    static constexpr int OFF_BARS = OFF_CORR + kWarps * CORR_FLOATS * 4;
+    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8;
+    static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
+    static_assert(EPI_BYTES <= OFF_SCORES, "epilogue must fit in the stage buffers");
+    static_assert(EPT % 8 == 0, "lanes hold whole 16-byte chunks");
+    static_assert(CT % RPW == 0 && BS % CT == 0, "tiles split evenly over the warp");
+    static_assert(32 % G == 0, "group size divides the warp");
+    static_assert(NVAL <= 16, "partial scores per lane");
+};
+
+// Sums NVAL per-lane partial values over groups of LPT lanes.  Each halving
+// step sends the half of the values this lane does not keep and adds the
+// partner's copy of the half it keeps, so the shuffle count falls from
+// NVAL*log2(LPT) to about NVAL.  Returns the index of the first value the
+// lane now holds in full; it holds NHELD consecutive values.
+template <int NVAL, int LPT>
+__device__ __forceinline__ int transpose_reduce(float (&v)[NVAL], int c)
+{
+    int base = 0;
+    int n = NVAL;
+#pragma unroll
+    for (int m = LPT / 2; m >= 1; m >>= 1) {
+        if (n > 1) {
+            const bool upper = (c & m) != 0;
+            const int half = n / 2;
+#pragma unroll
+            for (int j = 0; j < NVAL / 2; ++j) {
+                if (j < half) {
+                    const float lo = v[j], hi = v[j + half];
+                    const float send = upper ? lo : hi;
+                    const float keep = upper ? hi : lo;
+                    v[j] = keep + __shfl_xor_sync(kFullMask, send, m);
+                }
+            }
+            if (upper) base += half;
+            n = half;
+        } else {
+            v[0] += __shfl_xor_sync(kFullMask, v[0], m);
+        }
+    }
+    return base;
+}
+
+template <typename T, int D, int G>
+__device__ __forceinline__ void write_zero_rows(T* out, int s, int kvh, int num_q_heads)
+{
+    T* row = out + (static_cast<int64_t>(s) * num_q_heads + kvh * G) * D;
+    for (int i = threadIdx.x; i < G * D / 8; i += blockDim.x)
+        reinterpret_cast<uint4*>(row)[i] = make_uint4(0, 0, 0, 0);
+}
+
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
+    T* __restrict__ out, const T* __restrict__ query, const T* __restrict__ k_cache,
+    const T* __restrict__ v_cache, const int32_t* __restrict__ block_tables,
+    const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale_log2,
+    int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
+    float2* __restrict__ ws_ml, int32_t* d_status)
+{
+    using S = DecodeShape<D, BS, G>;
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int kvh = blockIdx.x;
+    const int part = blockIdx.y;
+    const int s = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int c = lane % S::LPT;        // position within the token row
+    const int r = lane / S::LPT;        // token row within a pass
+
+    const int32_t ctx = context_lens[s];
+    if (ctx < 0 || ctx > max_context_len ||
+        static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * BS) {
+        if (part == 0) {
+            write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
+            if (threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_CONTEXT);
+        }
+        return;
+    }
+    if (ctx == 0) {
+        if (part == 0) write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
+        return;
+    }
+    const int tok_begin = part * partition_size;
+    if (tok_begin >= ctx) return;
+    const int tok_end = min(ctx, tok_begin + partition_size);
+    const int nparts = (ctx + partition_size - 1) / partition_size;
+    const int blk_begin = tok_begin / BS;
+    const int nblk = (tok_end - tok_begin + BS - 1) / BS;
+    const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;   // this warp's blocks
+
+    unsigned char* wstage = smem + warp * S::WARP_STAGE_BYTES;
+    float* wscore = reinterpret_cast<float*>(smem + S::OFF_SCORES) + warp * S::SCORE_FLOATS;
+    float* wcorr = reinterpret_cast<float*>(smem + S::OFF_CORR) + warp * S::CORR_FLOATS;
+    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
+
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < S::NSTAGE; ++st) mbar_init(&wbar[st], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+
+    // q of every head in the group, this lane's elements, pre-scaled so the
+    // scores come out in log2 units.
+    float q[G][S::EPT];
+    {
+        const T* qrow = query + (static_cast<int64_t>(s) * num_q_heads + kvh * G) * D;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
+                const uint4 w = *reinterpret_cast<const uint4*>(qrow + g * D + k2 * 8 * S::LPT + 8 * c);
+                float f[8];
+                unpack8<T>(w, f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) q[g][k2 * 8 + e] = f[e] * scale_log2;
+            }
+        }
+    }
+
+    const int32_t* table = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq + blk_begin;
+    // The warp's k-th block is block warp + kWarps * k of the partition.
+    auto load_table = [&](int chunk) -> int {
+        const int kk = chunk * 32 + lane;
+        return kk < nk ? table[warp + kWarps * kk] : -1;
+    };
+    int prod_chunk = 0, cons_chunk = 0;
+    int prod_tbl = load_table(0);
+    int cons_tbl = prod_tbl;
+
+    auto block_tokens = [&](int k) -> int {   // valid tokens of the warp's k-th block
+        const int t0 = tok_begin + (warp + kWarps * k) * BS;
+        return min(BS, tok_end - t0);
+    };
+
+    // Producer: start the copies of block k into its stage.
+    auto issue = [&](int k) {
+        const int chunk = k >> 5;
+        if (chunk != prod_chunk) {
+            prod_tbl = load_table(chunk);
+            prod_chunk = chunk;
+        }
+        const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
+        const int st = k % S::NSTAGE;
+        int nv = block_tokens(k);
+        const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
+        if (!ok) nv = 0;
+        fence_proxy_async_smem();
+        if (lane == 0) {
+            if (!ok) status_or(d_status, PA_STATUS_BAD_BLOCK);
+            mbar_arrive_expect_tx(&wbar[st], static_cast<uint32_t>(2 * nv * S::ROW_BYTES));
+        }
+        __syncwarp();
+        unsigned char* dst = wstage + st * S::STAGE_BYTES;
+        const int64_t row0 = (static_cast<int64_t>(phys) * BS * num_kv_heads + kvh) * D;
+        for (int i = lane; i < 2 * nv; i += 32) {
+            const bool is_v = i >= nv;
+            const int t = is_v ? i - nv : i;
+            const T* src = (is_v ? v_cache : k_cache) + row0 + static_cast<int64_t>(t) * num_kv_heads * D;
+            bulk_copy_g2s(dst + (is_v ? S::TILE_BYTES : 0) + t * S::ROW_BYTES, src, S::ROW_BYTES,
+                          &wbar[st]);
+        }
+    };
+
+    float m_run = -INFINITY;     // running max of head (lane % G), log2 units
+    float l_run = 0.f;           // this lane's share of the running exp-sum
+    float o[G][S::EPT];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < S::EPT; ++e) o[g][e] = 0.f;
+
+    const int prologue = min(nk, S::NSTAGE);
+    for (int k = 0; k < prologue; ++k) issue(k);
+    int issued = prologue;
+    bool aborted = false;
+    int first_pending = 0;
+
+    for (int k = 0; k < nk; ++k) {
+        const int st = k % S::NSTAGE;
+        if (!mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1)) {
+            aborted = true;
+            first_pending = k;
+            break;
+        }
+        const int chunk = k >> 5;
+        if (chunk != cons_chunk) {
+            cons_tbl = load_table(chunk);
+            cons_chunk = chunk;
+        }
+        const int phys = __shfl_sync(kFullMask, cons_tbl, k & 31);
+        const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
+        const int nv = ok ? block_tokens(k) : 0;
+        const unsigned char* stage = wstage + st * S::STAGE_BYTES;
+#pragma unroll 1
+        for (int tile = 0; tile < S::TILES; ++tile) {
+            const unsigned char* ktile = stage + tile * S::CT * S::ROW_BYTES;
+            const unsigned char* vtile = ktile + S::TILE_BYTES;
+            const int tv = nv - tile * S::CT;     // valid tokens in this tile (may be <= 0)
+
+            // ---- scores: this lane's partial dot products ----
+            float acc[S::NVAL];
+#pragma unroll
+            for (int i = 0; i < S::NVAL; ++i) acc[i] = 0.f;
+#pragma unroll
+            for (int i = 0; i < S::ITERS; ++i) {
+                const int t = i * S::RPW + r;
+#pragma unroll
+                for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(
+                        ktile + t * S::ROW_BYTES + (k2 * 8 * S::LPT + 8 * c) * 2);
+                    float f[8];
+                    unpack8<T>(w, f);
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            acc[i * G + g] = fmaf(q[g][k2 * 8 + e], f[e], acc[i * G + g]);
+                }
+            }
+            const int base = transpose_reduce<S::NVAL, S::LPT>(acc, c);
+#pragma unroll
+            for (int j = 0; j < S::NHELD; ++j) {
+                const int n = base + j;
+                const int t = (n / G) * S::RPW + r;
+                wscore[t * G + (n % G)] = t < tv ? acc[j] : -INFINITY;
+            }
+            __syncwarp();
+
+            // ---- blocked softmax, online: tile max, running max, rescale ----
+            {
+                const int g = lane % G;
+                float sv[S::SM_TPL];
+                float mloc = -INFINITY;
+#pragma unroll
+                for (int kk = 0; kk < S::SM_TPL; ++kk) {
+                    const int t = lane / G + (32 / G) * kk;
+                    sv[kk] = t < S::CT ? wscore[t * G + g] : -INFINITY;
+                    mloc = fmaxf(mloc, sv[kk]);
+                }
+#pragma unroll
+                for (int m = G; m < 32; m <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFullMask, mloc, m));
+                const float m_new = fmaxf(m_run, mloc);
+                const float m_sub = m_new == -INFINITY ? 0.f : m_new;
+                const float corr = exp2f(m_run - m_sub);
+                l_run *= corr;
+#pragma unroll
+                for (int kk = 0; kk < S::SM_TPL; ++kk) {
+                    const int t = lane / G + (32 / G) * kk;
+                    if (t < S::CT) {
+                        const float p = exp2f(sv[kk] - m_sub);
+                        l_run += p;
+                        wscore[t * G + g] = p;
+                    }
+                }
+                m_run = m_new;
+                if (lane < G) wcorr[lane] = corr;
+            }
+            __syncwarp();
+
+            // ---- values: rescale, then accumulate p * V ----
+            {
+                float corr[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) corr[g] = wcorr[g];
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < S::EPT; ++e) o[g][e] *= corr[g];
+#pragma unroll
+                for (int i = 0; i < S::ITERS; ++i) {
+                    const int t = i * S::RPW + r;
+                    if (t < tv) {
+                        float p[G];
+#pragma unroll
+                        for (int g = 0; g < G; ++g) p[g] = wscore[t * G + g];
+#pragma unroll
+                        for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
+                            const uint4 w = *reinterpret_cast<const uint4*>(
+                                vtile + t * S::ROW_BYTES + (k2 * 8 * S::LPT + 8 * c) * 2);
+                            float f[8];
+                            unpack8<T>(w, f);
+#pragma unroll
+                            for (int g = 0; g < G; ++g)
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    o[g][k2 * 8 + e] = fmaf(p[g], f[e], o[g][k2 * 8 + e]);
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        __syncwarp();
+        if (issued < nk) issue(issued++);
+    }
+
+    if (aborted) {
+        if (lane == 0) status_or(d_status, PA_STATUS_TIMEOUT);
+        // Let the copies already started land (each wait bounded) before the
+        // shared memory is reused.
+        for (int k = first_pending; k < issued; ++k) {
+            const int st = k % S::NSTAGE;
+            mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1);
+        }
+    }
+
+    // ---- merge inside the warp ----
+#pragma unroll
+    for (int m = G; m < 32; m <<= 1) l_run += __shfl_xor_sync(kFullMask, l_run, m);
+#pragma unroll
+    for (int m = S::LPT; m < 32; m <<= 1)
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < S::EPT; ++e) o[g][e] += __shfl_xor_sync(kFullMask, o[g][e], m);
+
+    __syncthreads();   // every warp is done with its stage buffers
+    float* epi_o = reinterpret_cast<float*>(smem);                 // [warp][g][D]
+    float* epi_m = epi_o + kWarps * G * D;                         // [warp][g]
+    float* epi_l = epi_m + kWarps * G;
+    if (r == 0) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int k2 = 0; k2 < S::NCHUNK; ++k2)
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    epi_o[(warp * G + g) * D + k2 * 8 * S::LPT + 8 * c + e] = o[g][k2 * 8 + e];
+    }
+    if (lane < G) {
+        epi_m[warp * G + lane] = m_run;
+        epi_l[warp * G + lane] = l_run;
+    }
+    __syncthreads();
+
+    // ---- merge the warps, fixed order ----
+    for (int idx = threadIdx.x; idx < G * D / 8; idx += kThreads) {
+        const int g = idx / (D / 8);
+        const int d0 = (idx % (D / 8)) * 8;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, epi_m[w * G + g]);
+        const float msub = M == -INFINITY ? 0.f : M;
+        float L = 0.f;
+        float O[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) O[e] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float f = exp2f(epi_m[w * G + g] - msub);
+            L = fmaf(f, epi_l[w * G + g], L);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) O[e] = fmaf(f, epi_o[(w * G + g) * D + d0 + e], O[e]);
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) O[e] *= inv;
+        const int h = kvh * G + g;
+        const int64_t row = static_cast<int64_t>(s) * num_q_heads + h;
+        if (nparts == 1) {
+            *reinterpret_cast<uint4*>(out + row * D + d0) = pack8<T>(O);
+        } else {
+            const int64_t prow = row * max_parts + part;
+            float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + d0);
+            dst[0] = make_float4(O[0], O[1], O[2], O[3]);
+            dst[1] = make_float4(O[4], O[5], O[6], O[7]);
+            if (d0 == 0) ws_ml[prow] = make_float2(M, L);
+        }
+    }
+}
+
+// One warp per (sequence, query head) whose context spans several
+// partitions: merge the partitions' (max, exp-sum, normalised output).
+template <typename T, int D>
+__global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_reduce_kernel(
+    T* __restrict__ out, const float* __restrict__ ws_o, const float2* __restrict__ ws_ml,
+    const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t num_q_heads,
+    int32_t max_context_len, int32_t max_blocks_per_seq, int32_t block_size,
+    int32_t partition_size, int32_t max_parts)
+{
+    constexpr int EPL = D / 32;     // elements per lane
+    const int lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kReduceRowsPerCta + (threadIdx.x >> 5);
+    if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;
+    const int s = static_cast<int>(row / num_q_heads);
+    const int32_t ctx = context_lens[s];
+    if (ctx <= 0 || ctx > max_context_len ||
+        static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+        return;                                     // written by the first kernel
+    const int np = (ctx + partition_size - 1) / partition_size;
+    if (np <= 1) return;
+    const float2* ml = ws_ml + row * max_parts;
+    float M = -INFINITY;
+    for (int p = lane; p < np; p += 32) M = fmaxf(M, ml[p].x);
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, m));
+    const float msub = M == -INFINITY ? 0.f : M;
+    float acc[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+    float W = 0.f;
+    const float* orow = ws_o + row * max_parts * D + lane * EPL;
+    for (int p = 0; p < np; ++p) {
+        const float2 v = ml[p];
+        const float w = v.y * exp2f(v.x - msub);
+        W += w;
+        if (EPL == 4) {
+            const float4 x = *reinterpret_cast<const float4*>(orow + static_cast<int64_t>(p) * D);
+            acc[0] = fmaf(w, x.x, acc[0]);
+            acc[1] = fmaf(w, x.y, acc[1]);
+            acc[2] = fmaf(w, x.z, acc[2]);
+            acc[3] = fmaf(w, x.w, acc[3]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, orow[static_cast<int64_t>(p) * D + e], acc[e]);
+        }
+    }
+    const float inv = W > 0.f ? 1.f / W : 0.f;
+    T* dst = out + row * D + lane * EPL;
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) {
+        const uint32_t packed = Elem<T>::from_float2(acc[e] * inv, acc[e + 1] * inv);
+        *reinterpret_cast<uint32_t*>(dst + e) = packed;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+
+struct DecodeArgs {
+    void* out;
+    const void* query;
+    const void* k_cache;
+    const void* v_cache;
+    const int32_t* block_tables;
+    const int32_t* context_lens;
+    int32_t num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq;
+    int64_t num_blocks;
+    int32_t max_context_len;
+    float scale_log2;
+    int32_t partition_size, max_parts;
+    float* ws_o;
+    float2* ws_ml;
+    int32_t* d_status;
+    cudaStream_t stream;
+};
+
+template <typename Kernel>
+static bool ensure_smem_attr(Kernel kernel, int bytes, std::atomic<uint64_t>& done_mask)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+    if (bit && (done_mask.load(std::memory_order_relaxed) & bit)) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    done_mask.fetch_or(bit, std::memory_order_relaxed);
+    return true;
+}
+
+template <typename T, int D, int BS, int G>
+static pa_status launch_decode(const DecodeArgs& a)
+{
+    using S = DecodeShape<D, BS, G>;
+    static std::atomic<uint64_t> attr_done{0};
+    auto kernel = paged_decode_kernel<T, D, BS, G>;
+    if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
+    dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
+    kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
+        static_cast<T*>(a.out), static_cast<const T*>(a.query), static_cast<const T*>(a.k_cache),
+        static_cast<const T*>(a.v_cache), a.block_tables, a.context_lens, a.num_q_heads,
+        a.num_kv_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2,
+        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+    pa_status st = launch_status();
+    if (st != PA_OK || a.max_parts <= 1) return st;
+    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
+    const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
+    paged_decode_reduce_kernel<T, D><<<ctas, kReduceRowsPerCta * 32, 0, a.stream>>>(
+        static_cast<T*>(a.out), a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
+        a.max_context_len, a.max_blocks_per_seq, a.block_size, a.partition_size, a.max_parts);
+    return launch_status();
+}
+
+template <typename T, int D, int BS>
+static pa_status dispatch_group(const DecodeArgs& a)
+{
+    switch (a.num_q_heads / a.num_kv_heads) {
+    case 1: return launch_decode<T, D, BS, 1>(a);
+    case 2: return launch_decode<T, D, BS, 2>(a);
+    case 4: return launch_decode<T, D, BS, 4>(a);
+    case 8: return launch_decode<T, D, BS, 8>(a);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T, int D>
+static pa_status dispatch_block(const DecodeArgs& a)
+{
+    switch (a.block_size) {
+    case 8: return dispatch_group<T, D, 8>(a);
+    case 16: return dispatch_group<T, D, 16>(a);
+    case 32: return dispatch_group<T, D, 32>(a);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+static pa_status dispatch_dim(const DecodeArgs& a)
+{
+    switch (a.head_dim) {
+    case 64: return dispatch_block<T, 64>(a);
+    case 128: return dispatch_block<T, 128>(a);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+static bool supported_group(int32_t hq, int32_t hkv)
+{
+    if (hkv <= 0 || hq <= 0 || hq % hkv != 0) return false;
+    const int32_t g = hq / hkv;
+    return g == 1 || g == 2 || g == 4 || g == 8;
+}
+
+// Partition length: the caller's, else kDefaultPartition tokens (a whole
+// number of blocks), or the whole context when it is shorter.
+static int32_t choose_partition(int32_t block_size, int32_t max_context_len, int32_t requested)
+{
+    if (requested > 0) return requested;
+    int32_t p = kDefaultPartition / block_size * block_size;
+    if (max_context_len <= p) {
+        const int32_t whole = (max_context_len + block_size - 1) / block_size * block_size;
+        return whole > 0 ? whole : block_size;
+    }
+    return p;
+}
+
+static size_t workspace_bytes_for(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                  int32_t max_parts)
+{
+    if (max_parts <= 1) return 0;
+    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * max_parts;
+    return rows * head_dim * sizeof(float) + rows * sizeof(float2);
+}
+
+static int32_t parts_for(int32_t max_context_len, int32_t partition)
+{
+    return max_context_len <= 0 ? 1 : (max_context_len + partition - 1) / partition;
+}
+
+static pa_status check_decode_shape(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                    int32_t head_dim, int32_t block_size, int32_t max_context_len,
+                                    int32_t partition_size)
+{
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || max_context_len < 0 || partition_size < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size) ||
+        !supported_group(num_q_heads, num_kv_heads))
+        return PA_ERR_UNSUPPORTED;
+    if (partition_size % block_size != 0) return PA_ERR_INVALID_ARG;
+    return PA_OK;
+}
+
+}  // namespace pa
+
+extern "C" int32_t pa_paged_decode_partition_size(int32_t num_seqs, int32_t num_q_heads,
+                                                  int32_t num_kv_heads, int32_t head_dim,
+                                                  int32_t block_size, int32_t max_context_len,
+                                                  int32_t partition_size)
+{
+    using namespace pa;
+    if (check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                           max_context_len, partition_size) != PA_OK)
+        return 0;
+    return choose_partition(block_size, max_context_len, partition_size);
+}
+
+extern "C" size_t pa_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                                 int32_t num_kv_heads, int32_t head_dim,
+                                                 int32_t block_size, int32_t max_context_len,
+                                                 int32_t partition_size)
+{
+    using namespace pa;
+    if (check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                           max_context_len, partition_size) != PA_OK)
+        return 0;
+    const int32_t p = choose_partition(block_size, max_context_len, partition_size);
+    return workspace_bytes_for(num_seqs, num_q_heads, head_dim, parts_for(max_context_len, p));
+}
+
+extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int32_t max_blocks_per_seq,
+                                     int64_t num_blocks, int32_t max_context_len, float scale,
+                                     int32_t partition_size, void* workspace,
+                                     size_t workspace_bytes, pa_dtype dtype, int32_t* d_status,
+                                     pa_stream_t stream)
+{
+    using namespace pa;
+    pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, partition_size);
+    if (st != PA_OK) return st;
+    if (!supported_dtype(dtype)) return PA_ERR_UNSUPPORTED;
+    if (max_blocks_per_seq <= 0 || num_blocks <= 0 || !isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (!out || !query || !k_cache || !v_cache || !block_tables || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned4(block_tables) || !aligned4(context_lens) || (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    const int32_t partition = choose_partition(block_size, max_context_len, partition_size);
+    const int32_t max_parts = parts_for(max_context_len, partition);
+    const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, max_parts);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return PA_ERR_INVALID_ARG;
+    if (max_parts > 65535 || num_seqs > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+
+    DecodeArgs a;
+    a.out = out;
+    a.query = query;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.head_dim = head_dim;
+    a.block_size = block_size;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.max_context_len = max_context_len;
+    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    a.partition_size = partition;
+    a.max_parts = max_parts;
+    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * max_parts;
+    a.ws_o = need ? static_cast<float*>(workspace) : nullptr;
+    a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
+                                               rows * head_dim * sizeof(float))
+                   : nullptr;
+    a.d_status = d_status;
+    a.stream = stream;
+    return dtype == PA_DTYPE_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
+}

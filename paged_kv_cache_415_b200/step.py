@@ -1,0 +1,72 @@
+"""One decode step of one attention layer over a paged KV cache.
+
+    copy_blocks(block_mapping)         copy-on-write copies, if any
+    reshape_and_cache(new K/V, slots)  append this step's tokens
+    paged_decode(query, ...)           attend over each context, the new
+                                       tokens included
+
+``DecodeStep`` owns the scratch the step needs (the split-context workspace
+and a device status word), allocated once with torch, and issues the three
+C-ABI calls on one stream.  ``run_from_host`` is the same step fed from
+pinned host buffers: it copies the step's inputs to the device, runs the
+step and copies the output back, all on the same stream.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import binding as B
+
+
+class DecodeStep:
+    def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor, num_seqs: int,
+                 num_q_heads: int, max_context_len: int, partition_size: int = 0):
+        self.k_cache, self.v_cache = k_cache, v_cache
+        num_blocks, self.block_size, self.num_kv_heads, self.head_dim = k_cache.shape
+        self.num_blocks = num_blocks
+        self.num_seqs, self.num_q_heads = num_seqs, num_q_heads
+        self.max_context_len = max_context_len
+        self.partition_size = B.pa_paged_decode_partition_size(
+            num_seqs, num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
+            max_context_len, partition_size)
+        if self.partition_size <= 0:
+            raise B.PAError("pa_paged_decode_partition_size", B.PA_ERR_INVALID_ARG)
+        ws = B.pa_paged_decode_workspace_size(num_seqs, num_q_heads, self.num_kv_heads,
+                                              self.head_dim, self.block_size, max_context_len,
+                                              self.partition_size)
+        dev = k_cache.device
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev) if ws else None
+        self.d_status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def __call__(self, query, block_tables, context_lens, scale, out=None, new_key=None,
+                 new_value=None, slot_mapping=None, block_mapping=None, stream=None,
+                 max_context_len=None):
+        if block_mapping is not None and block_mapping.shape[0] > 0:
+            B.pa_copy_blocks(self.k_cache, self.v_cache, block_mapping, self.d_status, stream)
+        if slot_mapping is not None and slot_mapping.shape[0] > 0:
+            B.pa_reshape_and_cache(new_key, new_value, self.k_cache, self.v_cache, slot_mapping,
+                                   self.d_status, stream)
+        if out is None:
+            out = torch.empty_like(query)
+        B.pa_paged_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens,
+                          self.max_context_len if max_context_len is None else max_context_len,
+                          scale, self.partition_size, self.workspace, self.d_status, stream)
+        return out
+
+    def run_from_host(self, host: dict, dev: dict, scale, stream=None):
+        """host / dev: dicts of same-shaped tensors (pinned host / device) for
+        'query', 'block_tables', 'context_lens', 'new_key', 'new_value',
+        'slot_mapping', 'block_mapping' (the last four optional) and 'out'.
+        Copies host -> device, runs the step, copies out -> host, all on
+        ``stream`` (default: the current stream)."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            for name, h in host.items():
+                if name != "out":
+                    dev[name].copy_(h, non_blocking=True)
+            self(dev["query"], dev["block_tables"], dev["context_lens"], scale, out=dev["out"],
+                 new_key=dev.get("new_key"), new_value=dev.get("new_value"),
+                 slot_mapping=dev.get("slot_mapping"), block_mapping=dev.get("block_mapping"),
+                 stream=s)
+            host["out"].copy_(dev["out"], non_blocking=True)
+        return host["out"]

@@ -1,0 +1,133 @@
+"""The C-ABI library: it loads, exports every entry point include/pa.h
+declares, and its host-side argument checks reject bad calls before any
+device work (CPU only: no call here reaches a kernel launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pa.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return re.findall(r"^PA_API\s+[\w\s\*]+?\b(pa_\w+)\s*\(", text, flags=re.M)
+
+
+@pytest.fixture(scope="module")
+def pa():
+    from paged_kv_cache_415_b200 import build
+    build.build()
+    from paged_kv_cache_415_b200 import binding
+    return binding
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode",
+              "pa_paged_decode_workspace_size", "pa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(pa):
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), f"libpa.so does not export {name}"
+    assert set(_declared()) == set(pa.EXPORTS)
+
+
+def test_status_strings(pa):
+    assert pa.pa_status_string(0) == "PA_OK"
+    assert pa.pa_status_string(1) == "PA_ERR_INVALID_ARG"
+    assert pa.pa_status_string(2) == "PA_ERR_UNSUPPORTED"
+    assert pa.pa_status_string(3) == "PA_ERR_CUDA"
+    assert pa.pa_status_string(77) == "PA_ERR_UNKNOWN"
+    assert re.match(r"\d+\.\d+\.\d+", pa.pa_version())
+
+
+def test_partition_and_workspace_sizes(pa):
+    ps, ws = pa.pa_paged_decode_partition_size, pa.pa_paged_decode_workspace_size
+    # short contexts: one partition covering the whole (block-rounded) context, no workspace
+    assert ps(4, 2, 2, 64, 16, 40, 0) == 48 and ws(4, 2, 2, 64, 16, 40, 0) == 0
+    # long contexts: 512-token partitions, (D + 2) floats per (seq, q head, partition)
+    assert ps(16, 32, 8, 128, 16, 32768, 0) == 512
+    assert ws(16, 32, 8, 128, 16, 32768, 0) == 16 * 32 * 64 * (128 + 2) * 4
+    assert ws(16, 32, 8, 128, 16, 32768, 1024) == 16 * 32 * 32 * (128 + 2) * 4
+    # the caller's partition wins; it must be a multiple of block_size
+    assert ps(1, 1, 1, 128, 16, 100, 32) == 32
+    assert ps(1, 1, 1, 128, 16, 100, 24) == 0
+    # unsupported shapes
+    assert ps(1, 3, 1, 128, 16, 100, 0) == 0          # group of 3
+    assert ps(1, 2, 2, 96, 16, 100, 0) == 0           # head_dim 96
+    assert ps(1, 2, 2, 128, 12, 100, 0) == 0          # block 12
+
+
+FAKE = 1 << 20                       # 16-byte aligned, never dereferenced
+
+
+def _decode(pa, **kw):
+    args = dict(out=FAKE, query=FAKE, k_cache=FAKE, v_cache=FAKE, block_tables=FAKE,
+                context_lens=FAKE, num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                block_size=16, max_blocks_per_seq=8, num_blocks=64, max_context_len=100,
+                scale=0.1, partition_size=0, workspace=None, workspace_bytes=0, dtype=0,
+                d_status=None, stream=None)
+    args.update(kw)
+    return pa.LIB.pa_paged_decode(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(out=None), 1), (dict(query=None), 1), (dict(k_cache=None), 1),
+    (dict(block_tables=None), 1), (dict(context_lens=None), 1),
+    (dict(out=FAKE + 8), 1), (dict(k_cache=FAKE + 4), 1), (dict(block_tables=FAKE + 2), 1),
+    (dict(num_q_heads=6, num_kv_heads=4), 1), (dict(num_q_heads=0), 1),
+    (dict(num_seqs=-1), 1), (dict(max_context_len=-5), 1), (dict(partition_size=24), 1),
+    (dict(partition_size=-16), 1), (dict(max_blocks_per_seq=0), 1), (dict(num_blocks=0), 1),
+    (dict(scale=float("nan")), 1),
+    (dict(max_context_len=4096, workspace=None), 1),
+    (dict(max_context_len=4096, workspace=FAKE, workspace_bytes=16), 1),
+    (dict(head_dim=96), 2), (dict(block_size=12), 2), (dict(num_q_heads=6, num_kv_heads=2), 2),
+    (dict(num_q_heads=32, num_kv_heads=2), 2), (dict(dtype=5), 2),
+])
+def test_decode_rejects_bad_arguments(pa, kw, code):
+    assert _decode(pa, **kw) == code
+
+
+def test_decode_with_no_sequences_is_a_no_op(pa):
+    assert _decode(pa, num_seqs=0) == 0
+
+
+def _cache(pa, **kw):
+    args = dict(key=FAKE, value=FAKE, k_cache=FAKE, v_cache=FAKE, slot_mapping=FAKE, num_tokens=4,
+                num_kv_heads=2, head_dim=64, block_size=16, num_blocks=64, dtype=0, d_status=None,
+                stream=None)
+    args.update(kw)
+    return pa.LIB.pa_reshape_and_cache(*args.values())
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(key=None), 1), (dict(v_cache=None), 1), (dict(slot_mapping=None), 1),
+    (dict(key=FAKE + 8), 1), (dict(slot_mapping=FAKE + 4), 1), (dict(num_tokens=-1), 1),
+    (dict(num_kv_heads=0), 1), (dict(num_blocks=0), 1), (dict(d_status=FAKE + 1), 1),
+    (dict(head_dim=80), 2), (dict(block_size=64), 2), (dict(dtype=9), 2),
+])
+def test_reshape_and_cache_rejects_bad_arguments(pa, kw, code):
+    assert _cache(pa, **kw) == code
+
+
+def test_empty_calls_are_no_ops(pa):
+    assert _cache(pa, num_tokens=0) == 0
+    assert pa.LIB.pa_copy_blocks(FAKE, FAKE, FAKE, 0, 2, 64, 16, 64, 0, None, None) == 0
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, FAKE, FAKE, 2, 2, 64, 16, 64, 0, None, None), 1),
+    ((FAKE, FAKE, None, 2, 2, 64, 16, 64, 0, None, None), 1),
+    ((FAKE, FAKE, FAKE + 4, 2, 2, 64, 16, 64, 0, None, None), 1),
+    ((FAKE, FAKE, FAKE, -1, 2, 64, 16, 64, 0, None, None), 1),
+    ((FAKE, FAKE, FAKE, 2, 2, 48, 16, 64, 0, None, None), 2),
+    ((FAKE, FAKE, FAKE, 2, 2, 64, 16, 64, 3, None, None), 2),
+])
+def test_copy_blocks_rejects_bad_arguments(pa, args, code):
+    assert pa.LIB.pa_copy_blocks(*args) == code

@@ -195,7 +195,8 @@ def tiny(keep_logical=True) -> DecodeWorkload:
     return wl
 
 
-def llama7b(seqs=64, max_ctx=2048, min_ctx=128, keep_logical=False) -> DecodeWorkload:
+def llama7b(seqs=64, max_ctx=2048, min_ctx=128, num_blocks=16384,
+            keep_logical=False) -> DecodeWorkload:
     """LLaMA-7B-shaped MHA decode: 32/32 heads, head_dim 128, block 16, fp16,
     contexts uniform in [128, 2048], 16384-block pool, scale 1/sqrt(128),
     one new token per sequence."""
@@ -203,7 +204,7 @@ def llama7b(seqs=64, max_ctx=2048, min_ctx=128, keep_logical=False) -> DecodeWor
     ctx = rng.integers(min_ctx, max_ctx, size=seqs, endpoint=True)
     return make_decode("llama7b", seed=SEED_BASE + 2, dtype="f16", context_lens=ctx,
                        num_q_heads=32, num_kv_heads=32, head_dim=128, block_size=16,
-                       num_blocks=16384, scale=1.0 / math.sqrt(128.0),
+                       num_blocks=num_blocks, scale=1.0 / math.sqrt(128.0),
                        keep_logical=keep_logical)
 
 
