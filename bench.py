@@ -156,6 +156,23 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples), "source": "nvml"}
 
 
+def max_over_ranks(values, device=None):
+    """Elementwise max of per-rank floats over the process group (identity
+    without one).  Every rank must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_gbs(bytes_per_step: int, steps: int, world: int, max_elapsed_ms: float) -> float:
+    """Every rank runs its own replica: total bytes over the slowest rank's time."""
+    return world * bytes_per_step * steps / (max_elapsed_ms * 1e-3) / 1e9
+
+
 def make_workload(config: str, seqs: int = 0):
     """The named workload; with seqs > 0 a smaller batch of the same shape
     and a pool sized to it (profiling captures stay a few GB)."""
@@ -393,17 +410,13 @@ def run_ours(args):
     barrier()
     e2e_ms = e_start.elapsed_time(e_stop)
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms, e2e_ms, statistics.mean(decode_ms)], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, e2e_ms, decode_avg = [float(x) for x in t.tolist()]
-    else:
-        decode_avg = statistics.mean(decode_ms)
+    elapsed_ms, e2e_ms, decode_avg = max_over_ranks(
+        [elapsed_ms, e2e_ms, statistics.mean(decode_ms)], dev)
 
     step = bm.step_bytes(wl)
     per_step_ms = elapsed_ms / args.steps
-    value = world * step["total"] * args.steps / (elapsed_ms * 1e-3) / 1e9
-    e2e_value = world * step["total"] * args.steps / (e2e_ms * 1e-3) / 1e9
+    value = whole_job_gbs(step["total"], args.steps, world, elapsed_ms)
+    e2e_value = whole_job_gbs(step["total"], args.steps, world, e2e_ms)
     peak, peak_kind = hbm_peak()
     achieved = step["attention"] / (decode_avg * 1e-3) / 1e9
     traffic = profiled_traffic(args.config)
