@@ -228,6 +228,48 @@ PA_API pa_status pa_paged_decode(void* out, const void* query, const void* k_cac
                           void* workspace, size_t workspace_bytes, pa_dtype dtype,
                           int32_t* d_status, pa_stream_t stream);
 
+/*
+ * pa_paged_decode_no_alloc -- pa_paged_decode without a caller-supplied
+ * workspace.
+ *
+ * The pages have no counterpart to this entry point.  It exists for callers
+ * that cannot allocate device memory themselves: a plugin or custom operator
+ * inside a host framework that owns every device allocation and hands the
+ * plugin only its inputs and outputs, or code on a latency-critical path
+ * that must not call cudaMalloc (which can synchronise the whole device) in
+ * the middle of a step.
+ *
+ * Arguments and results are those of pa_paged_decode, minus `workspace` and
+ * `workspace_bytes`.  The split-context scratch is instead a file-scope
+ * device array of PA_NO_ALLOC_WORKSPACE_BYTES inside libpa.so; every GPU that
+ * loads the library holds that memory until the process exits.  The call
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *
+ *  - A shape whose pa_paged_decode_workspace_size(...) is larger than
+ *    PA_NO_ALLOC_WORKSPACE_BYTES is rejected with PA_ERR_INVALID_ARG before
+ *    anything is enqueued; use pa_paged_decode with your own workspace (or a
+ *    longer partition_size) for it.
+ *  - The first call on a device that needs the scratch looks up the array's
+ *    device address (cudaGetSymbolAddress, with that device current) and
+ *    keeps it; make that first call before any stream capture.
+ *  - Every call shares the one array, which keeps the previous call's
+ *    contents.  Nothing in it needs clearing (every value the reduction reads
+ *    is written earlier in the same call), but calls that overlap on the GPU
+ *    -- on different streams, or issued from different host threads -- race
+ *    on it: order them.
+ */
+#define PA_NO_ALLOC_WORKSPACE_BYTES ((size_t)32 << 20)
+
+PA_API pa_status pa_paged_decode_no_alloc(void* out, const void* query, const void* k_cache,
+                                          const void* v_cache, const int32_t* block_tables,
+                                          const int32_t* context_lens, int32_t num_seqs,
+                                          int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim, int32_t block_size,
+                                          int32_t max_blocks_per_seq, int64_t num_blocks,
+                                          int32_t max_context_len, float scale,
+                                          int32_t partition_size, pa_dtype dtype,
+                                          int32_t* d_status, pa_stream_t stream);
+
 /* Human-readable name of a pa_status (static string, never NULL). */
 PA_API const char* pa_status_string(pa_status status);
 

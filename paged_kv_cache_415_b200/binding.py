@@ -32,8 +32,10 @@ _DTYPES = {torch.float16: PA_DTYPE_F16, torch.bfloat16: PA_DTYPE_BF16}
 
 # Every entry point declared in include/pa.h.
 EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_size",
-           "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_status_string",
-           "pa_version")
+           "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_paged_decode_no_alloc",
+           "pa_status_string", "pa_version")
+# Size of the library-owned scratch of pa_paged_decode_no_alloc.
+PA_NO_ALLOC_WORKSPACE_BYTES = 32 << 20
 
 
 class PAError(RuntimeError):
@@ -59,6 +61,9 @@ def _load() -> ctypes.CDLL:
     lib.pa_paged_decode.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64, i32, f32,
                                     i32, p, sz, i32, p, p]
     lib.pa_paged_decode.restype = i32
+    lib.pa_paged_decode_no_alloc.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64,
+                                             i32, f32, i32, i32, p, p]
+    lib.pa_paged_decode_no_alloc.restype = i32
     lib.pa_status_string.argtypes = [i32]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
@@ -148,3 +153,20 @@ def pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, ma
         _ptr(context_lens), num_seqs, hq, hkv, d, block_size, int(block_tables.shape[1]),
         num_blocks, int(max_context_len), float(scale), int(partition_size), _ptr(workspace),
         ws_bytes, _dtype(query), _ptr(d_status), _stream(stream)))
+
+
+def pa_paged_decode_no_alloc(out, query, k_cache, v_cache, block_tables, context_lens,
+                             max_context_len, scale, partition_size=0, d_status=None,
+                             stream=None) -> None:
+    """pa_paged_decode for callers that cannot allocate device memory: the
+    split-context scratch is the library's own fixed array of
+    PA_NO_ALLOC_WORKSPACE_BYTES per GPU.  Shapes needing more raise PAError
+    (PA_ERR_INVALID_ARG) before any work is enqueued.  Calls share that
+    array, so calls that overlap on the GPU must not be issued."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    _check("pa_paged_decode_no_alloc", LIB.pa_paged_decode_no_alloc(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), num_seqs, hq, hkv, d, block_size, int(block_tables.shape[1]),
+        num_blocks, int(max_context_len), float(scale), int(partition_size), _dtype(query),
+        _ptr(d_status), _stream(stream)))

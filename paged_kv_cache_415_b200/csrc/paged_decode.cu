@@ -40,6 +40,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "pa.h"
 #include "pa_common.cuh"
@@ -726,4 +727,65 @@ extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k
     a.d_status = d_status;
     a.stream = stream;
     return dtype == PA_DTYPE_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
+}
+
+// ---------------------------------------------------------------------------
+// pa_paged_decode_no_alloc: the same decode with its split-context scratch in
+// a file-scope device array instead of caller memory.
+// ---------------------------------------------------------------------------
+namespace pa {
+
+static __device__ __align__(256) unsigned char g_no_alloc_workspace[PA_NO_ALLOC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_no_alloc_mutex;
+static void* g_no_alloc_ptr[kMaxDevices];   // device address of the array, per device
+
+// Device address of the array on the current device; looked up once per
+// device (host code may not use the symbol itself as a device pointer).
+static pa_status no_alloc_workspace(void** ptr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_no_alloc_mutex);
+    if (g_no_alloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_no_alloc_workspace) != cudaSuccess || p == nullptr)
+            return PA_ERR_CUDA;
+        g_no_alloc_ptr[dev] = p;
+    }
+    *ptr = g_no_alloc_ptr[dev];
+    return PA_OK;
+}
+
+}  // namespace pa
+
+extern "C" pa_status pa_paged_decode_no_alloc(void* out, const void* query, const void* k_cache,
+                                              const void* v_cache, const int32_t* block_tables,
+                                              const int32_t* context_lens, int32_t num_seqs,
+                                              int32_t num_q_heads, int32_t num_kv_heads,
+                                              int32_t head_dim, int32_t block_size,
+                                              int32_t max_blocks_per_seq, int64_t num_blocks,
+                                              int32_t max_context_len, float scale,
+                                              int32_t partition_size, pa_dtype dtype,
+                                              int32_t* d_status, pa_stream_t stream)
+{
+    using namespace pa;
+    pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, partition_size);
+    if (st != PA_OK) return st;
+    const size_t need = pa_paged_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads,
+                                                       head_dim, block_size, max_context_len,
+                                                       partition_size);
+    if (need > PA_NO_ALLOC_WORKSPACE_BYTES) return PA_ERR_INVALID_ARG;
+    void* ws = nullptr;
+    if (need > 0) {
+        st = no_alloc_workspace(&ws);
+        if (st != PA_OK) return st;
+    }
+    return pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, ws,
+                           need > 0 ? PA_NO_ALLOC_WORKSPACE_BYTES : 0, dtype, d_status, stream);
 }
