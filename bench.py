@@ -61,6 +61,8 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--partition", type=int, default=-1,
+                    help="context partition in tokens (-1 = the workload's, 0 = library's choice)")
     ap.add_argument("--seqs", type=int, default=0,
                     help="shrink the batch (and the pool) for profiling; 0 = the full workload")
     return ap.parse_args()
@@ -128,13 +130,14 @@ class ClockSampler:
         nv = self.nv
         get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
             nv.nvmlDeviceGetCurrentClocksThrottleReasons
-        while not self._stop.is_set():
+        while True:
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
                 self.reasons |= int(get_reasons(self.h))
             except Exception:   # noqa: BLE001
                 pass
-            time.sleep(0.002)
+            if self._stop.wait(0.001):
+                break
 
     def __enter__(self):
         if self.ok:
@@ -323,8 +326,9 @@ def run_ours(args):
     out = torch.empty_like(query)
     d_status = torch.zeros(1, dtype=torch.int32, device=dev)
     mcl = wl.max_context_len
+    want = wl.partition_size if args.partition < 0 else args.partition
     part = B.pa_paged_decode_partition_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
-                                            wl.head_dim, wl.block_size, mcl, wl.partition_size)
+                                            wl.head_dim, wl.block_size, mcl, want)
     ws_bytes = B.pa_paged_decode_workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
                                                 wl.head_dim, wl.block_size, mcl, part)
     workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)

@@ -35,7 +35,9 @@
 //
 // The whole computation has a fixed summation order, so results are
 // deterministic and do not depend on where the blocks sit in the pool.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 #include <stdint.h>
 
@@ -50,12 +52,11 @@ namespace pa {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
-constexpr int kDefaultPartition = 512;
 constexpr int kReduceRowsPerCta = 4;
 
 template <int D, int BS, int G>
 struct DecodeShape {
-    static constexpr int LPT = (G == 8 && D == 128) ? 16 : 8;   // lanes per token row
+    static constexpr int LPT = (G >= 4 && D == 128) ? 16 : 8;   // lanes per token row
     static constexpr int RPW = 32 / LPT;                        // token rows per warp pass
     static constexpr int EPT = D / LPT;                         // elements per lane
     static constexpr int NCHUNK = EPT / 8;                      // 16-byte chunks per lane
@@ -68,7 +69,7 @@ struct DecodeShape {
     static constexpr int ROW_BYTES = D * 2;
     static constexpr int TILE_BYTES = BS * ROW_BYTES;           // K (or V) of one block, one head
     static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int NSTAGE = STAGE_BYTES <= 4096 ? 4 : (STAGE_BYTES <= 8192 ? 3 : 2);
+    static constexpr int NSTAGE = STAGE_BYTES <= 4096 ? 3 : 2;
     static constexpr int NVAL = ITERS * G;                      // partial scores per lane
     static constexpr int NHELD = NVAL >= LPT ? NVAL / LPT : 1;  // scores per lane after reduce
     static constexpr int SM_TPL = (CT * G + 31) / 32;           // softmax items per lane
@@ -80,6 +81,9 @@ struct DecodeShape {
     static constexpr int OFF_BARS = OFF_CORR + kWarps * CORR_FLOATS * 4;
     static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8;
     static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
+    // CTAs per SM the register budget is sized for: larger groups keep more
+    // live state per lane (q and the output accumulators of every head).
+    static constexpr int MIN_CTAS = G >= 8 ? 2 : 3;
     static_assert(EPI_BYTES <= OFF_SCORES, "epilogue must fit in the stage buffers");
     static_assert(EPT % 8 == 0, "lanes hold whole 16-byte chunks");
     static_assert(CT % RPW == 0 && BS % CT == 0, "tiles split evenly over the warp");
@@ -128,16 +132,66 @@ __device__ __forceinline__ void write_zero_rows(T* out, int s, int kvh, int num_
         reinterpret_cast<uint4*>(row)[i] = make_uint4(0, 0, 0, 0);
 }
 
+// The CTA's last step: merge the four warps' (max, exp-sum, output) for the
+// G heads of its kv head in a fixed order, then either write the output row
+// (context in one partition) or the partition's max, sum and normalised
+// output to the workspace.  epi_o is [warp][g][D], epi_m / epi_l [warp][g],
+// in shared memory, complete (the caller synchronised the CTA).
+template <typename T, int D, int G>
+__device__ __forceinline__ void merge_warps_and_store(
+    const float* epi_o, const float* epi_m, const float* epi_l, T* __restrict__ out,
+    float* __restrict__ ws_o, float2* __restrict__ ws_ml, int s, int kvh, int part, int nparts,
+    int num_q_heads, int max_parts)
+{
+    for (int idx = threadIdx.x; idx < G * D / 8; idx += kThreads) {
+        const int g = idx / (D / 8);
+        const int d0 = (idx % (D / 8)) * 8;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, epi_m[w * G + g]);
+        const float msub = M == -INFINITY ? 0.f : M;
+        float L = 0.f;
+        float O[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) O[e] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const float f = exp2f(epi_m[w * G + g] - msub);
+            L = fmaf(f, epi_l[w * G + g], L);
+            const float4* src = reinterpret_cast<const float4*>(epi_o + (w * G + g) * D + d0);
+            const float4 a = src[0], b = src[1];
+            O[0] = fmaf(f, a.x, O[0]); O[1] = fmaf(f, a.y, O[1]);
+            O[2] = fmaf(f, a.z, O[2]); O[3] = fmaf(f, a.w, O[3]);
+            O[4] = fmaf(f, b.x, O[4]); O[5] = fmaf(f, b.y, O[5]);
+            O[6] = fmaf(f, b.z, O[6]); O[7] = fmaf(f, b.w, O[7]);
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) O[e] *= inv;
+        const int h = kvh * G + g;
+        const int64_t row = static_cast<int64_t>(s) * num_q_heads + h;
+        if (nparts == 1) {
+            *reinterpret_cast<uint4*>(out + row * D + d0) = pack8<T>(O);
+        } else {
+            const int64_t prow = row * max_parts + part;
+            float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + d0);
+            dst[0] = make_float4(O[0], O[1], O[2], O[3]);
+            dst[1] = make_float4(O[4], O[5], O[6], O[7]);
+            if (d0 == 0) ws_ml[prow] = make_float2(M, L);
+        }
+    }
+}
+
 template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
-    T* __restrict__ out, const T* __restrict__ query, const T* __restrict__ k_cache,
-    const T* __restrict__ v_cache, const int32_t* __restrict__ block_tables,
-    const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t num_kv_heads,
-    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale_log2,
-    int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
-    float2* __restrict__ ws_ml, int32_t* d_status)
+__global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) paged_decode_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
+    const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
+    int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
+    int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status)
 {
     using S = DecodeShape<D, BS, G>;
+    constexpr int EP = S::EPT / 2;      // element pairs per lane
     extern __shared__ __align__(128) unsigned char smem[];
 
     const int kvh = blockIdx.x;
@@ -181,26 +235,9 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
     }
     __syncwarp();
 
-    // q of every head in the group, this lane's elements, pre-scaled so the
-    // scores come out in log2 units.
-    float q[G][S::EPT];
-    {
-        const T* qrow = query + (static_cast<int64_t>(s) * num_q_heads + kvh * G) * D;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
-                const uint4 w = *reinterpret_cast<const uint4*>(qrow + g * D + k2 * 8 * S::LPT + 8 * c);
-                float f[8];
-                unpack8<T>(w, f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) q[g][k2 * 8 + e] = f[e] * scale_log2;
-            }
-        }
-    }
-
     const int32_t* table = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq + blk_begin;
-    // The warp's k-th block is block warp + kWarps * k of the partition.
+    // The warp's k-th block is block warp + kWarps * k of the partition; one
+    // table entry per lane, 32 blocks per load.
     auto load_table = [&](int chunk) -> int {
         const int kk = chunk * 32 + lane;
         return kk < nk ? table[warp + kWarps * kk] : -1;
@@ -214,7 +251,8 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
         return min(BS, tok_end - t0);
     };
 
-    // Producer: start the copies of block k into its stage.
+    // Producer: one lane starts the two tensor copies (the K and V tiles of
+    // this kv head: BS rows of D elements) of block k into its stage.
     auto issue = [&](int k) {
         const int chunk = k >> 5;
         if (chunk != prod_chunk) {
@@ -222,38 +260,53 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
             prod_chunk = chunk;
         }
         const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
-        const int st = k % S::NSTAGE;
-        int nv = block_tokens(k);
-        const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
-        if (!ok) nv = 0;
-        fence_proxy_async_smem();
         if (lane == 0) {
-            if (!ok) status_or(d_status, PA_STATUS_BAD_BLOCK);
-            mbar_arrive_expect_tx(&wbar[st], static_cast<uint32_t>(2 * nv * S::ROW_BYTES));
-        }
-        __syncwarp();
-        unsigned char* dst = wstage + st * S::STAGE_BYTES;
-        const int64_t row0 = (static_cast<int64_t>(phys) * BS * num_kv_heads + kvh) * D;
-        for (int i = lane; i < 2 * nv; i += 32) {
-            const bool is_v = i >= nv;
-            const int t = is_v ? i - nv : i;
-            const T* src = (is_v ? v_cache : k_cache) + row0 + static_cast<int64_t>(t) * num_kv_heads * D;
-            bulk_copy_g2s(dst + (is_v ? S::TILE_BYTES : 0) + t * S::ROW_BYTES, src, S::ROW_BYTES,
-                          &wbar[st]);
+            const int st = k % S::NSTAGE;
+            const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
+            fence_proxy_async_smem();
+            if (ok) {
+                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE_BYTES);
+                unsigned char* dst = wstage + st * S::STAGE_BYTES;
+                tma_load_4d(dst, &tm_k, 0, kvh, 0, phys, &wbar[st]);
+                tma_load_4d(dst + S::TILE_BYTES, &tm_v, 0, kvh, 0, phys, &wbar[st]);
+            } else {
+                status_or(d_status, PA_STATUS_BAD_BLOCK);
+                mbar_arrive_expect_tx(&wbar[st], 0u);
+            }
         }
     };
-
-    float m_run = -INFINITY;     // running max of head (lane % G), log2 units
-    float l_run = 0.f;           // this lane's share of the running exp-sum
-    float o[G][S::EPT];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < S::EPT; ++e) o[g][e] = 0.f;
 
     const int prologue = min(nk, S::NSTAGE);
     for (int k = 0; k < prologue; ++k) issue(k);
     int issued = prologue;
+
+    // q of every head in the group, this lane's elements, kept as the raw
+    // 16-bit input pairs (the products with K are exact in fp32; the scale
+    // is applied to the reduced scores).
+    uint32_t qw[G][EP];
+    {
+        const T* qrow = query + (static_cast<int64_t>(s) * num_q_heads + kvh * G) * D;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
+                const uint4 w = *reinterpret_cast<const uint4*>(qrow + g * D + k2 * 8 * S::LPT + 8 * c);
+                qw[g][k2 * 4 + 0] = w.x;
+                qw[g][k2 * 4 + 1] = w.y;
+                qw[g][k2 * 4 + 2] = w.z;
+                qw[g][k2 * 4 + 3] = w.w;
+            }
+        }
+    }
+
+    float m_run = -INFINITY;     // running max of head (lane % G), log2 units
+    float l_run = 0.f;           // this lane's share of the running exp-sum
+    float2 o2[G][EP];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < EP; ++e) o2[g][e] = make_float2(0.f, 0.f);
+
     bool aborted = false;
     int first_pending = 0;
 
@@ -279,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
             const unsigned char* vtile = ktile + S::TILE_BYTES;
             const int tv = nv - tile * S::CT;     // valid tokens in this tile (may be <= 0)
 
-            // ---- scores: this lane's partial dot products ----
+            // ---- scores: this lane's partial dot products (fp32 accumulation) ----
             float acc[S::NVAL];
 #pragma unroll
             for (int i = 0; i < S::NVAL; ++i) acc[i] = 0.f;
@@ -290,13 +343,12 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
                 for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
                     const uint4 w = *reinterpret_cast<const uint4*>(
                         ktile + t * S::ROW_BYTES + (k2 * 8 * S::LPT + 8 * c) * 2);
-                    float f[8];
-                    unpack8<T>(w, f);
+                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                    for (int g = 0; g < G; ++g)
+                    for (int j = 0; j < 4; ++j)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            acc[i * G + g] = fmaf(q[g][k2 * 8 + e], f[e], acc[i * G + g]);
+                        for (int g = 0; g < G; ++g)
+                            acc[i * G + g] = fma_pair<T>(qw[g][k2 * 4 + j], words[j], acc[i * G + g]);
                 }
             }
             const int base = transpose_reduce<S::NVAL, S::LPT>(acc, c);
@@ -304,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
             for (int j = 0; j < S::NHELD; ++j) {
                 const int n = base + j;
                 const int t = (n / G) * S::RPW + r;
-                wscore[t * G + (n % G)] = t < tv ? acc[j] : -INFINITY;
+                wscore[t * G + (n % G)] = t < tv ? acc[j] * scale_log2 : -INFINITY;
             }
             __syncwarp();
 
@@ -339,40 +391,43 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
             }
             __syncwarp();
 
-            // ---- values: rescale, then accumulate p * V ----
+            // ---- values: rescale, then accumulate p * V (packed fp32 FMA) ----
             {
-                float corr[G];
 #pragma unroll
-                for (int g = 0; g < G; ++g) corr[g] = wcorr[g];
+                for (int g = 0; g < G; ++g) {
+                    const float cg = wcorr[g];
+                    const float2 c2 = make_float2(cg, cg);
 #pragma unroll
-                for (int g = 0; g < G; ++g)
-#pragma unroll
-                    for (int e = 0; e < S::EPT; ++e) o[g][e] *= corr[g];
+                    for (int e = 0; e < EP; ++e) o2[g][e] = __fmul2_rn(o2[g][e], c2);
+                }
 #pragma unroll
                 for (int i = 0; i < S::ITERS; ++i) {
                     const int t = i * S::RPW + r;
                     if (t < tv) {
-                        float p[G];
+                        float2 p2[G];
 #pragma unroll
-                        for (int g = 0; g < G; ++g) p[g] = wscore[t * G + g];
+                        for (int g = 0; g < G; ++g) {
+                            const float pg = wscore[t * G + g];
+                            p2[g] = make_float2(pg, pg);
+                        }
 #pragma unroll
                         for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
                             const uint4 w = *reinterpret_cast<const uint4*>(
                                 vtile + t * S::ROW_BYTES + (k2 * 8 * S::LPT + 8 * c) * 2);
-                            float f[8];
-                            unpack8<T>(w, f);
+                            const uint32_t words[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                            for (int g = 0; g < G; ++g)
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 vf = Elem<T>::to_float2(words[j]);
 #pragma unroll
-                                for (int e = 0; e < 8; ++e)
-                                    o[g][k2 * 8 + e] = fmaf(p[g], f[e], o[g][k2 * 8 + e]);
+                                for (int g = 0; g < G; ++g)
+                                    o2[g][k2 * 4 + j] = __ffma2_rn(p2[g], vf, o2[g][k2 * 4 + j]);
+                            }
                         }
                     }
                 }
             }
             __syncwarp();
         }
-        __syncwarp();
         if (issued < nk) issue(issued++);
     }
 
@@ -394,7 +449,10 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int e = 0; e < S::EPT; ++e) o[g][e] += __shfl_xor_sync(kFullMask, o[g][e], m);
+            for (int e = 0; e < EP; ++e) {
+                o2[g][e].x += __shfl_xor_sync(kFullMask, o2[g][e].x, m);
+                o2[g][e].y += __shfl_xor_sync(kFullMask, o2[g][e].y, m);
+            }
 
     __syncthreads();   // every warp is done with its stage buffers
     float* epi_o = reinterpret_cast<float*>(smem);                 // [warp][g][D]
@@ -404,10 +462,13 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
 #pragma unroll
         for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int k2 = 0; k2 < S::NCHUNK; ++k2)
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    epi_o[(warp * G + g) * D + k2 * 8 * S::LPT + 8 * c + e] = o[g][k2 * 8 + e];
+            for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
+                float4* dst = reinterpret_cast<float4*>(epi_o + (warp * G + g) * D + k2 * 8 * S::LPT + 8 * c);
+                dst[0] = make_float4(o2[g][k2 * 4 + 0].x, o2[g][k2 * 4 + 0].y,
+                                     o2[g][k2 * 4 + 1].x, o2[g][k2 * 4 + 1].y);
+                dst[1] = make_float4(o2[g][k2 * 4 + 2].x, o2[g][k2 * 4 + 2].y,
+                                     o2[g][k2 * 4 + 3].x, o2[g][k2 * 4 + 3].y);
+            }
     }
     if (lane < G) {
         epi_m[warp * G + lane] = m_run;
@@ -415,41 +476,15 @@ __global__ void __launch_bounds__(kThreads, 2) paged_decode_kernel(
     }
     __syncthreads();
 
-    // ---- merge the warps, fixed order ----
-    for (int idx = threadIdx.x; idx < G * D / 8; idx += kThreads) {
-        const int g = idx / (D / 8);
-        const int d0 = (idx % (D / 8)) * 8;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, epi_m[w * G + g]);
-        const float msub = M == -INFINITY ? 0.f : M;
-        float L = 0.f;
-        float O[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) O[e] = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float f = exp2f(epi_m[w * G + g] - msub);
-            L = fmaf(f, epi_l[w * G + g], L);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) O[e] = fmaf(f, epi_o[(w * G + g) * D + d0 + e], O[e]);
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) O[e] *= inv;
-        const int h = kvh * G + g;
-        const int64_t row = static_cast<int64_t>(s) * num_q_heads + h;
-        if (nparts == 1) {
-            *reinterpret_cast<uint4*>(out + row * D + d0) = pack8<T>(O);
-        } else {
-            const int64_t prow = row * max_parts + part;
-            float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + d0);
-            dst[0] = make_float4(O[0], O[1], O[2], O[3]);
-            dst[1] = make_float4(O[4], O[5], O[6], O[7]);
-            if (d0 == 0) ws_ml[prow] = make_float2(M, L);
-        }
-    }
+    merge_warps_and_store<T, D, G>(epi_o, epi_m, epi_l, out, ws_o, ws_ml, s, kvh, part, nparts,
+                                   num_q_heads, max_parts);
 }
+
+}  // namespace pa
+
+#include "paged_decode_mma.cuh"
+
+namespace pa {
 
 // One warp per (sequence, query head) whose context spans several
 // partitions: merge the partitions' (max, exp-sum, normalised output).
@@ -541,19 +576,103 @@ static bool ensure_smem_attr(Kernel kernel, int bytes, std::atomic<uint64_t>& do
     return true;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+// (no link-time dependency on libcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A pool [num_blocks][B][Hkv][D] of 16-bit elements as a 4-D tensor
+// (innermost first: D, Hkv, B, num_blocks) whose box is one block of one kv
+// head: D x 1 x B x 1, landing in shared memory as B dense rows of D.
+static bool encode_pool_map(CUtensorMap* map, const void* pool, int32_t head_dim,
+                            int32_t num_kv_heads, int32_t block_size, int64_t num_blocks)
+{
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim),
+                                static_cast<cuuint64_t>(num_kv_heads),
+                                static_cast<cuuint64_t>(block_size),
+                                static_cast<cuuint64_t>(num_blocks)};
+    const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * 2;
+    const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(head_dim), 1u,
+                               static_cast<cuuint32_t>(block_size), 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, const_cast<void*>(pool), dims,
+                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return res == CUDA_SUCCESS;
+}
+
+// The same pool as a 5-D tensor (innermost first: 64 dims, B tokens, D/64
+// halves, Hkv, num_blocks) whose box is one block of one kv head, stored in
+// shared memory as [D/64][B][64] rows of 128 bytes with the 128-byte swizzle
+// (16-byte chunk c of row r kept at chunk c ^ (r % 8)).
+static bool encode_pool_map_swizzled(CUtensorMap* map, const void* pool, int32_t head_dim,
+                                     int32_t num_kv_heads, int32_t block_size, int64_t num_blocks)
+{
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * 2;
+    const cuuint64_t dims[5] = {64u, static_cast<cuuint64_t>(block_size),
+                                static_cast<cuuint64_t>(head_dim / 64),
+                                static_cast<cuuint64_t>(num_kv_heads),
+                                static_cast<cuuint64_t>(num_blocks)};
+    const cuuint64_t strides[4] = {row * num_kv_heads, 128u, row, row * num_kv_heads * block_size};
+    const cuuint32_t box[5] = {64u, static_cast<cuuint32_t>(block_size),
+                               static_cast<cuuint32_t>(head_dim / 64), 1u, 1u};
+    const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 5, const_cast<void*>(pool), dims,
+                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return res == CUDA_SUCCESS;
+}
+
 template <typename T, int D, int BS, int G>
 static pa_status launch_decode(const DecodeArgs& a)
 {
-    using S = DecodeShape<D, BS, G>;
-    static std::atomic<uint64_t> attr_done{0};
-    auto kernel = paged_decode_kernel<T, D, BS, G>;
-    if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
+    // Grouped heads (G >= 4) in 16-token slices: tensor-core contractions.
+    constexpr bool kMma = G >= 4 && BS % 16 == 0;
     dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
-    kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
-        static_cast<T*>(a.out), static_cast<const T*>(a.query), static_cast<const T*>(a.k_cache),
-        static_cast<const T*>(a.v_cache), a.block_tables, a.context_lens, a.num_q_heads,
-        a.num_kv_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2,
-        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+    CUtensorMap tm_k, tm_v;
+    if constexpr (kMma) {
+        using S = MmaShape<D, BS, G>;
+        static std::atomic<uint64_t> attr_done{0};
+        auto kernel = paged_decode_mma_kernel<T, D, BS, G>;
+        if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
+        if (!encode_pool_map_swizzled(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
+            !encode_pool_map_swizzled(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
+            return PA_ERR_CUDA;
+        kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
+            tm_k, tm_v, static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables,
+            a.context_lens, a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len,
+            a.scale_log2, a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+    } else {
+        using S = DecodeShape<D, BS, G>;
+        static std::atomic<uint64_t> attr_done{0};
+        auto kernel = paged_decode_kernel<T, D, BS, G>;
+        if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
+        if (!encode_pool_map(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
+            !encode_pool_map(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
+            return PA_ERR_CUDA;
+        kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
+            tm_k, tm_v, static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables,
+            a.context_lens, a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len,
+            a.scale_log2, a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+    }
     pa_status st = launch_status();
     if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
@@ -604,17 +723,31 @@ static bool supported_group(int32_t hq, int32_t hkv)
     return g == 1 || g == 2 || g == 4 || g == 8;
 }
 
-// Partition length: the caller's, else kDefaultPartition tokens (a whole
-// number of blocks), or the whole context when it is shorter.
-static int32_t choose_partition(int32_t block_size, int32_t max_context_len, int32_t requested)
+// Partition length: the caller's; else the whole (block-rounded) context
+// when it is at most kMaxSinglePartition tokens and there are enough
+// (sequence, kv head) pairs to fill the GPU on their own; else about an
+// eighth of the longest context (so the longest sequences split into at
+// least 8 CTAs), as a power of two between kMinPartition and
+// kMaxPartition tokens (short enough to balance ragged contexts, long
+// enough to amortise each CTA's start-up).
+constexpr int kMinPartition = 512;
+constexpr int kMaxPartition = 2048;
+constexpr int kMaxSinglePartition = 2048;
+constexpr int64_t kFillUnits = 888;    // 148 SMs x 3 CTAs x 2 waves
+
+static int32_t choose_partition(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
+                                int32_t max_context_len, int32_t requested)
 {
     if (requested > 0) return requested;
-    int32_t p = kDefaultPartition / block_size * block_size;
-    if (max_context_len <= p) {
-        const int32_t whole = (max_context_len + block_size - 1) / block_size * block_size;
-        return whole > 0 ? whole : block_size;
-    }
-    return p;
+    const int32_t whole = max_context_len > 0
+                              ? (max_context_len + block_size - 1) / block_size * block_size
+                              : block_size;
+    const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
+    if (max_context_len <= kMaxSinglePartition && units >= kFillUnits) return whole;
+    int32_t p = kMinPartition;
+    while (p < kMaxPartition && p * 8 < max_context_len) p *= 2;
+    p = p / block_size * block_size;
+    return whole < p ? whole : p;
 }
 
 static size_t workspace_bytes_for(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
@@ -656,7 +789,7 @@ extern "C" int32_t pa_paged_decode_partition_size(int32_t num_seqs, int32_t num_
     if (check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                            max_context_len, partition_size) != PA_OK)
         return 0;
-    return choose_partition(block_size, max_context_len, partition_size);
+    return choose_partition(num_seqs, num_kv_heads, block_size, max_context_len, partition_size);
 }
 
 extern "C" size_t pa_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
@@ -668,7 +801,8 @@ extern "C" size_t pa_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q
     if (check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                            max_context_len, partition_size) != PA_OK)
         return 0;
-    const int32_t p = choose_partition(block_size, max_context_len, partition_size);
+    const int32_t p = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                       partition_size);
     return workspace_bytes_for(num_seqs, num_q_heads, head_dim, parts_for(max_context_len, p));
 }
 
@@ -693,7 +827,8 @@ extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k
     if (!aligned16(out) || !aligned16(query) || !aligned16(k_cache) || !aligned16(v_cache) ||
         !aligned4(block_tables) || !aligned4(context_lens) || (d_status && !aligned4(d_status)))
         return PA_ERR_INVALID_ARG;
-    const int32_t partition = choose_partition(block_size, max_context_len, partition_size);
+    const int32_t partition = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                               partition_size);
     const int32_t max_parts = parts_for(max_context_len, partition);
     const size_t need = workspace_bytes_for(num_seqs, num_q_heads, head_dim, max_parts);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))

@@ -51,9 +51,14 @@ def test_partition_and_workspace_sizes(pa):
     ps, ws = pa.pa_paged_decode_partition_size, pa.pa_paged_decode_workspace_size
     # short contexts: one partition covering the whole (block-rounded) context, no workspace
     assert ps(4, 2, 2, 64, 16, 40, 0) == 48 and ws(4, 2, 2, 64, 16, 40, 0) == 0
-    # long contexts: 512-token partitions, (D + 2) floats per (seq, q head, partition)
-    assert ps(16, 32, 8, 128, 16, 32768, 0) == 512
-    assert ws(16, 32, 8, 128, 16, 32768, 0) == 16 * 32 * 64 * (128 + 2) * 4
+    # many (seq, kv head) pairs and contexts up to 2048: one partition per context
+    assert ps(64, 32, 32, 128, 16, 1982, 0) == 1984 and ws(64, 32, 32, 128, 16, 1982, 0) == 0
+    # longer contexts: about 1/8 of the longest, a power of two in [512, 2048]
+    assert ps(256, 32, 8, 128, 16, 8192, 0) == 1024
+    assert ps(16, 32, 8, 128, 16, 32768, 0) == 2048
+    assert ps(16, 32, 8, 128, 16, 3000, 0) == 512
+    # workspace: (D + 2) floats per (seq, q head, partition)
+    assert ws(16, 32, 8, 128, 16, 32768, 0) == 16 * 32 * 16 * (128 + 2) * 4
     assert ws(16, 32, 8, 128, 16, 32768, 1024) == 16 * 32 * 32 * (128 + 2) * 4
     # the caller's partition wins; it must be a multiple of block_size
     assert ps(1, 1, 1, 128, 16, 100, 32) == 32
