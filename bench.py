@@ -63,6 +63,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--partition", type=int, default=-1,
                     help="context partition in tokens (-1 = the workload's, 0 = library's choice)")
+    ap.add_argument("--shared-prefix", action="store_true",
+                    help="beam_search: decode with pa_paged_decode_shared_prefix (shared "
+                         "prompt blocks read once per group)")
     ap.add_argument("--seqs", type=int, default=0,
                     help="shrink the batch (and the pool) for profiling; 0 = the full workload")
     return ap.parse_args()
@@ -343,12 +346,27 @@ def run_ours(args):
             B.pa_reshape_and_cache(new_key, new_value, k_cache, v_cache, slot_mapping, d_status,
                                    stream)
 
+    shared = args.shared_prefix and "prefix_lens" in wl.extra
+    if shared:
+        group_size = int(wl.extra["group_size"])
+        prefix_lens = torch.from_numpy(wl.extra["prefix_lens"]).to(dev)
+        mpl = int(wl.extra["prefix_lens"].max())
+        sws = B.pa_paged_decode_shared_prefix_workspace_size(
+            wl.num_seqs, group_size, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
+            mcl, mpl, part)
+        workspace = torch.empty(max(sws, 16), dtype=torch.uint8, device=dev)
+
     def decode():
-        B.pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl, wl.scale,
-                          part, workspace, d_status, stream)
+        if shared:
+            B.pa_paged_decode_shared_prefix(out, query, k_cache, v_cache, block_tables,
+                                            context_lens, prefix_lens, group_size, mcl, mpl,
+                                            wl.scale, workspace, part, d_status, stream)
+        else:
+            B.pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl,
+                              wl.scale, part, workspace, d_status, stream)
 
     launches_per_step = (1 if n_pairs else 0) + (1 if wl.num_new_tokens else 0) + 1 + \
-        (1 if max_parts > 1 else 0)
+        (1 if (max_parts > 1 or shared) else 0)
 
     def barrier():
         if world > 1:
@@ -436,6 +454,14 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank != 0:
         return 0
+    group = wl.num_q_heads // wl.num_kv_heads
+    if shared:
+        kernel_name = "paged_decode_shared_kernel + paged_decode_shared_reduce_kernel"
+    else:
+        kernel_name = ("paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
+                       else "paged_decode_kernel")
+        if max_parts > 1:
+            kernel_name += " + paged_decode_reduce_kernel"
     l2 = (f"no flush: {step['kv'] / 1e9:.2f} GB of K/V per step > 126 MB L2"
           if step["kv"] > 4 * 126e6 else "working set smaller than L2 (values include L2 hits)")
     line = {
@@ -446,7 +472,7 @@ def run_ours(args):
         "us_per_layer_step": round(per_step_ms * 1e3, 2),
         "kv_tokens_per_s": round(world * int(wl.context_lens.sum()) * args.steps / (elapsed_ms * 1e-3)),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-        "roofline": {"bound": "hbm", "kernel": "paged_decode_kernel + paged_decode_reduce_kernel",
+        "roofline": {"bound": "hbm", "kernel": kernel_name,
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic, "algorithmic_bytes_per_launch": step["attention"],
@@ -457,7 +483,12 @@ def run_ours(args):
         "clocks": clocks,
         "cpu_baseline": cpu,
         "bytes_per_step": step,
+        "decode_entry": "pa_paged_decode_shared_prefix" if shared else "pa_paged_decode",
     }
+    if "prefix_lens" in wl.extra:
+        uniq = bm.unique_kv_bytes(wl)
+        line["unique_kv_bytes"] = uniq
+        line["unique_kv_gbs_decode"] = round(uniq / (decode_avg * 1e-3) / 1e9, 1)
     print(json.dumps(line))
     return 0
 

@@ -229,6 +229,49 @@ PA_API pa_status pa_paged_decode(void* out, const void* query, const void* k_cac
                           int32_t* d_status, pa_stream_t stream);
 
 /*
+ * pa_paged_decode_shared_prefix -- pa_paged_decode for batches whose
+ * sequences come in groups that share a stored prefix (the beams of one
+ * prompt, parallel samples of one request).
+ *
+ * Defined by: [Practice §5.2 非连续KV访问优化] step 1 (process together the
+ * queries that touch the same physical block) over the block sharing of
+ * [VM-paging, 写时复制与块共享机制] and [Practice §4.1]: the members of a group
+ * point at the same physical blocks for their first prefix_lens[g] tokens,
+ * and those blocks are read from HBM once for all members.  The output is
+ * that of pa_paged_decode on the same arguments (within rounding).
+ *
+ * Groups are group_size consecutive sequences: group g is sequences
+ * [g * group_size, (g + 1) * group_size); num_seqs % group_size == 0.
+ * prefix_lens    int32 [num_seqs / group_size], device: tokens group g shares,
+ *                a multiple of block_size, at most every member's context
+ *                length and at most max_prefix_len; 0 = nothing shared.  The
+ *                members' block-table entries for those blocks must be equal.
+ * max_prefix_len host: upper bound of prefix_lens (sizes the grid).
+ * group_size * (num_q_heads / num_kv_heads) must be at most 8 and
+ * block_size 16 or 32 (else PA_ERR_UNSUPPORTED).
+ * workspace      at least pa_paged_decode_shared_prefix_workspace_size(...)
+ *                bytes, 16-byte aligned (always needed).
+ * d_status       as pa_paged_decode; a group whose prefix is not a whole
+ *                number of blocks or is longer than a member's context (or
+ *                max_prefix_len) sets PA_STATUS_BAD_CONTEXT and gets zero
+ *                rows; members whose prefix block-table entries differ set
+ *                PA_STATUS_BAD_BLOCK (their result is then unspecified).
+ */
+PA_API size_t pa_paged_decode_shared_prefix_workspace_size(
+    int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_context_len, int32_t max_prefix_len,
+    int32_t partition_size);
+
+PA_API pa_status pa_paged_decode_shared_prefix(
+    void* out, const void* query, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* prefix_lens,
+    int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, int32_t max_prefix_len, float scale, int32_t partition_size,
+    void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* d_status,
+    pa_stream_t stream);
+
+/*
  * pa_paged_decode_no_alloc -- pa_paged_decode without a caller-supplied
  * workspace.
  *

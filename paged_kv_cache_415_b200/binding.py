@@ -33,6 +33,7 @@ _DTYPES = {torch.float16: PA_DTYPE_F16, torch.bfloat16: PA_DTYPE_BF16}
 # Every entry point declared in include/pa.h.
 EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_size",
            "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_paged_decode_no_alloc",
+           "pa_paged_decode_shared_prefix_workspace_size", "pa_paged_decode_shared_prefix",
            "pa_status_string", "pa_version")
 # Size of the library-owned scratch of pa_paged_decode_no_alloc.
 PA_NO_ALLOC_WORKSPACE_BYTES = 32 << 20
@@ -64,6 +65,12 @@ def _load() -> ctypes.CDLL:
     lib.pa_paged_decode_no_alloc.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64,
                                              i32, f32, i32, i32, p, p]
     lib.pa_paged_decode_no_alloc.restype = i32
+    lib.pa_paged_decode_shared_prefix_workspace_size.argtypes = [i32] * 9
+    lib.pa_paged_decode_shared_prefix_workspace_size.restype = sz
+    lib.pa_paged_decode_shared_prefix.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32,
+                                                  i32, i32, i64, i32, i32, f32, i32, p, sz, i32,
+                                                  p, p]
+    lib.pa_paged_decode_shared_prefix.restype = i32
     lib.pa_status_string.argtypes = [i32]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
@@ -169,4 +176,29 @@ def pa_paged_decode_no_alloc(out, query, k_cache, v_cache, block_tables, context
         _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         _ptr(context_lens), num_seqs, hq, hkv, d, block_size, int(block_tables.shape[1]),
         num_blocks, int(max_context_len), float(scale), int(partition_size), _dtype(query),
+        _ptr(d_status), _stream(stream)))
+
+
+def pa_paged_decode_shared_prefix_workspace_size(num_seqs, group_size, num_q_heads, num_kv_heads,
+                                                 head_dim, block_size, max_context_len,
+                                                 max_prefix_len, partition_size=0) -> int:
+    return int(LIB.pa_paged_decode_shared_prefix_workspace_size(
+        num_seqs, group_size, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+        max_prefix_len, partition_size))
+
+
+def pa_paged_decode_shared_prefix(out, query, k_cache, v_cache, block_tables, context_lens,
+                                  prefix_lens, group_size, max_context_len, max_prefix_len, scale,
+                                  workspace, partition_size=0, d_status=None, stream=None) -> None:
+    """pa_paged_decode for groups of group_size consecutive sequences that
+    share their first prefix_lens[g] tokens (int32 device tensor, one entry
+    per group, whole blocks)."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check("pa_paged_decode_shared_prefix", LIB.pa_paged_decode_shared_prefix(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), _ptr(prefix_lens), num_seqs, int(group_size), hq, hkv, d, block_size,
+        int(block_tables.shape[1]), num_blocks, int(max_context_len), int(max_prefix_len),
+        float(scale), int(partition_size), _ptr(workspace), ws_bytes, _dtype(query),
         _ptr(d_status), _stream(stream)))

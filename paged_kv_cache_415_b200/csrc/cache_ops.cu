@@ -21,11 +21,15 @@ namespace pa {
 constexpr int kCopyThreads = 256;
 constexpr int kCopyVecsPerThread = 4;
 
-// One CTA per new token.  The pools are [num_slots][Hkv][D], so a token's
-// K row (all kv heads) is one contiguous run of row_vecs 16-byte vectors at
-// slot * row_vecs ([Practice §3.3 按需分配策略], step 4: write the new
-// token's KV vectors into the slot the allocator gave it).
-__global__ void __launch_bounds__(128) reshape_and_cache_kernel(
+// Grid (token, chunk of the row).  The pools are [num_slots][Hkv][D], so a
+// token's K row (all kv heads) is one contiguous run of row_vecs 16-byte
+// vectors at slot * row_vecs ([Practice §3.3 按需分配策略], step 4: write the
+// new token's KV vectors into the slot the allocator gave it).  Each thread
+// moves up to kCacheVecsPerThread vectors of K and of V, all loads first.
+constexpr int kCacheThreads = 128;
+constexpr int kCacheVecsPerThread = 2;
+
+__global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ k_cache,
     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int32_t row_vecs,
     int64_t num_slots, int32_t* d_status)
@@ -34,18 +38,30 @@ __global__ void __launch_bounds__(128) reshape_and_cache_kernel(
     const int64_t slot = slot_mapping[t];
     if (slot < 0) return;                       // padding token
     if (slot >= num_slots) {
-        if (threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_SLOT);
+        if (threadIdx.x == 0 && blockIdx.y == 0) status_or(d_status, PA_STATUS_BAD_SLOT);
         return;
     }
     const uint4* ks = key + t * row_vecs;
     const uint4* vs = value + t * row_vecs;
     uint4* kd = k_cache + slot * row_vecs;
     uint4* vd = v_cache + slot * row_vecs;
-    for (int32_t i = threadIdx.x; i < row_vecs; i += blockDim.x) {
-        const uint4 a = ld_nc_v4(ks + i);
-        const uint4 b = ld_nc_v4(vs + i);
-        kd[i] = a;
-        vd[i] = b;
+    const int32_t base = blockIdx.y * kCacheThreads * kCacheVecsPerThread + threadIdx.x;
+    uint4 a[kCacheVecsPerThread], b[kCacheVecsPerThread];
+#pragma unroll
+    for (int j = 0; j < kCacheVecsPerThread; ++j) {
+        const int32_t i = base + j * kCacheThreads;
+        if (i < row_vecs) {
+            a[j] = ld_nc_v4(ks + i);
+            b[j] = ld_nc_v4(vs + i);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kCacheVecsPerThread; ++j) {
+        const int32_t i = base + j * kCacheThreads;
+        if (i < row_vecs) {
+            kd[i] = a[j];
+            vd[i] = b[j];
+        }
     }
 }
 
@@ -125,7 +141,11 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, vo
         return PA_ERR_INVALID_ARG;
     if (num_tokens == 0) return PA_OK;
     const int32_t row_vecs = num_kv_heads * head_dim * 2 / 16;
-    reshape_and_cache_kernel<<<num_tokens, 128, 0, stream>>>(
+    const int32_t per_cta = kCacheThreads * kCacheVecsPerThread;
+    const int32_t chunks = (row_vecs + per_cta - 1) / per_cta;
+    if (chunks > 65535) return PA_ERR_UNSUPPORTED;
+    dim3 grid(num_tokens, chunks);
+    reshape_and_cache_kernel<<<grid, kCacheThreads, 0, stream>>>(
         static_cast<const uint4*>(key), static_cast<const uint4*>(value),
         static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, row_vecs,
         num_blocks * block_size, d_status);

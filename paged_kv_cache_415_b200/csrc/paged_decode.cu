@@ -483,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
 }  // namespace pa
 
 #include "paged_decode_mma.cuh"
+#include "paged_decode_shared.cuh"
 
 namespace pa {
 
@@ -716,6 +717,55 @@ static pa_status dispatch_dim(const DecodeArgs& a)
     }
 }
 
+struct SharedArgs {
+    DecodeArgs d;
+    const int32_t* prefix_lens;
+    int32_t group_size, max_prefix_len, prefix_slots, slots;
+};
+
+template <typename T, int D, int BS>
+static pa_status launch_shared(const SharedArgs& sa)
+{
+    using S = SharedShape<D, BS>;
+    const DecodeArgs& a = sa.d;
+    static std::atomic<uint64_t> attr_done{0};
+    auto kernel = paged_decode_shared_kernel<T, D, BS>;
+    if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
+    CUtensorMap tm_k, tm_v;
+    if (!encode_pool_map_swizzled(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
+        !encode_pool_map_swizzled(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
+        return PA_ERR_CUDA;
+    const int32_t num_groups = a.num_seqs / sa.group_size;
+    const int32_t parts = sa.slots - sa.prefix_slots > sa.prefix_slots ? sa.slots - sa.prefix_slots
+                                                                       : sa.prefix_slots;
+    dim3 grid(a.num_kv_heads, parts > 0 ? parts : 1, num_groups + a.num_seqs);
+    kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
+        tm_k, tm_v, static_cast<const T*>(a.query), a.block_tables, a.context_lens,
+        sa.prefix_lens, num_groups, sa.group_size, a.num_q_heads / a.num_kv_heads, a.num_q_heads,
+        a.max_blocks_per_seq, a.num_blocks, a.max_context_len, sa.max_prefix_len, a.scale_log2,
+        a.partition_size, sa.prefix_slots, sa.slots, a.ws_o, a.ws_ml, a.d_status);
+    pa_status st = launch_status();
+    if (st != PA_OK) return st;
+    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
+    const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
+    paged_decode_shared_reduce_kernel<T, D><<<ctas, kReduceRowsPerCta * 32, 0, a.stream>>>(
+        static_cast<T*>(a.out), a.ws_o, a.ws_ml, a.context_lens, sa.prefix_lens, a.num_seqs,
+        sa.group_size, a.num_q_heads, a.max_context_len, a.max_blocks_per_seq, a.block_size,
+        sa.max_prefix_len, a.partition_size, sa.prefix_slots, sa.slots, a.d_status);
+    return launch_status();
+}
+
+template <typename T>
+static pa_status dispatch_shared(const SharedArgs& sa)
+{
+    const int32_t d = sa.d.head_dim, b = sa.d.block_size;
+    if (d == 64 && b == 16) return launch_shared<T, 64, 16>(sa);
+    if (d == 64 && b == 32) return launch_shared<T, 64, 32>(sa);
+    if (d == 128 && b == 16) return launch_shared<T, 128, 16>(sa);
+    if (d == 128 && b == 32) return launch_shared<T, 128, 32>(sa);
+    return PA_ERR_UNSUPPORTED;
+}
+
 static bool supported_group(int32_t hq, int32_t hkv)
 {
     if (hkv <= 0 || hq <= 0 || hq % hkv != 0) return false;
@@ -862,6 +912,119 @@ extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k
     a.d_status = d_status;
     a.stream = stream;
     return dtype == PA_DTYPE_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
+}
+
+// ---------------------------------------------------------------------------
+// Shared-prefix decode
+// ---------------------------------------------------------------------------
+namespace pa {
+
+static pa_status check_shared_shape(int32_t num_seqs, int32_t group_size, int32_t num_q_heads,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                    int32_t max_context_len, int32_t max_prefix_len,
+                                    int32_t partition_size)
+{
+    pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                      max_context_len, partition_size);
+    if (st != PA_OK) return st;
+    if (group_size <= 0 || num_seqs % group_size != 0 || max_prefix_len < 0 ||
+        max_prefix_len > max_context_len)
+        return PA_ERR_INVALID_ARG;
+    if (block_size % 16 != 0 || group_size * (num_q_heads / num_kv_heads) > kSharedRows)
+        return PA_ERR_UNSUPPORTED;
+    return PA_OK;
+}
+
+static void shared_slots(int32_t max_context_len, int32_t max_prefix_len, int32_t partition,
+                         int32_t* prefix_slots, int32_t* slots)
+{
+    *prefix_slots = (max_prefix_len + partition - 1) / partition;
+    const int32_t suffix = max_context_len > 0 ? (max_context_len + partition - 1) / partition : 1;
+    *slots = *prefix_slots + suffix;
+}
+
+}  // namespace pa
+
+extern "C" size_t pa_paged_decode_shared_prefix_workspace_size(
+    int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_context_len, int32_t max_prefix_len,
+    int32_t partition_size)
+{
+    using namespace pa;
+    if (check_shared_shape(num_seqs, group_size, num_q_heads, num_kv_heads, head_dim, block_size,
+                           max_context_len, max_prefix_len, partition_size) != PA_OK)
+        return 0;
+    const int32_t p = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                       partition_size);
+    int32_t prefix_slots, slots;
+    shared_slots(max_context_len, max_prefix_len, p, &prefix_slots, &slots);
+    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * slots;
+    return rows * head_dim * sizeof(float) + rows * sizeof(float2);
+}
+
+extern "C" pa_status pa_paged_decode_shared_prefix(
+    void* out, const void* query, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* prefix_lens,
+    int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, int32_t max_prefix_len, float scale, int32_t partition_size,
+    void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream)
+{
+    using namespace pa;
+    pa_status st = check_shared_shape(num_seqs, group_size, num_q_heads, num_kv_heads, head_dim,
+                                      block_size, max_context_len, max_prefix_len, partition_size);
+    if (st != PA_OK) return st;
+    if (!supported_dtype(dtype)) return PA_ERR_UNSUPPORTED;
+    if (max_blocks_per_seq <= 0 || num_blocks <= 0 || !isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (!out || !query || !k_cache || !v_cache || !block_tables || !context_lens || !prefix_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(query) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned4(block_tables) || !aligned4(context_lens) || !aligned4(prefix_lens) ||
+        (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    const int32_t partition = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
+                                               partition_size);
+    int32_t prefix_slots, slots;
+    shared_slots(max_context_len, max_prefix_len, partition, &prefix_slots, &slots);
+    const size_t need = pa_paged_decode_shared_prefix_workspace_size(
+        num_seqs, group_size, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
+        max_prefix_len, partition_size);
+    if (num_seqs == 0) return PA_OK;
+    if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+        return PA_ERR_INVALID_ARG;
+    const int64_t items = static_cast<int64_t>(num_seqs / group_size) + num_seqs;
+    if (items > 65535 || slots > 65535) return PA_ERR_UNSUPPORTED;
+
+    SharedArgs sa;
+    DecodeArgs& a = sa.d;
+    a.out = out;
+    a.query = query;
+    a.k_cache = k_cache;
+    a.v_cache = v_cache;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.head_dim = head_dim;
+    a.block_size = block_size;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.max_context_len = max_context_len;
+    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    a.partition_size = partition;
+    a.max_parts = slots;
+    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * slots;
+    a.ws_o = static_cast<float*>(workspace);
+    a.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + rows * head_dim * sizeof(float));
+    a.d_status = d_status;
+    a.stream = stream;
+    sa.prefix_lens = prefix_lens;
+    sa.group_size = group_size;
+    sa.max_prefix_len = max_prefix_len;
+    sa.prefix_slots = prefix_slots;
+    sa.slots = slots;
+    return dtype == PA_DTYPE_F16 ? dispatch_shared<__half>(sa) : dispatch_shared<__nv_bfloat16>(sa);
 }
 
 // ---------------------------------------------------------------------------

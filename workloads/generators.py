@@ -291,6 +291,10 @@ def beam_search(prompts=32, beams=4, prompt_len=1000, max_new=256, num_heads=40,
         wl.keys, wl.values = keys_l, vals_l
     wl.extra["manager"] = mgr
     wl.extra["n_new"] = n_new
+    # the beams of a prompt share its full blocks (the partial last block is
+    # copied on write by every beam but the last writer)
+    wl.extra["group_size"] = beams
+    wl.extra["prefix_lens"] = np.full(prompts, (prompt_len // b) * b, dtype=np.int32)
     return wl
 
 
