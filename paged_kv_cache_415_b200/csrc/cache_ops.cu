@@ -34,6 +34,8 @@ __global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_kernel(
     uint4* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int32_t row_vecs,
     int64_t num_slots, int32_t* d_status)
 {
+    grid_dependency_wait();
+    allow_dependents();
     const int64_t t = blockIdx.x;
     const int64_t slot = slot_mapping[t];
     if (slot < 0) return;                       // padding token
@@ -75,6 +77,8 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
     const int64_t* __restrict__ block_mapping, int32_t num_pairs, int64_t block_vecs,
     int64_t num_blocks, int32_t* d_status)
 {
+    grid_dependency_wait();
+    allow_dependents();
     const int32_t pair = blockIdx.x;
     const int64_t src = block_mapping[2 * pair];
     const int64_t dst = block_mapping[2 * pair + 1];
@@ -145,11 +149,10 @@ extern "C" pa_status pa_reshape_and_cache(const void* key, const void* value, vo
     const int32_t chunks = (row_vecs + per_cta - 1) / per_cta;
     if (chunks > 65535) return PA_ERR_UNSUPPORTED;
     dim3 grid(num_tokens, chunks);
-    reshape_and_cache_kernel<<<grid, kCacheThreads, 0, stream>>>(
-        static_cast<const uint4*>(key), static_cast<const uint4*>(value),
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), slot_mapping, row_vecs,
-        num_blocks * block_size, d_status);
-    return launch_status();
+    return launch_overlapped(reshape_and_cache_kernel, grid, dim3(kCacheThreads), 0, stream,
+                             static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+                             static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                             slot_mapping, row_vecs, num_blocks * block_size, d_status);
 }
 
 extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
@@ -171,8 +174,7 @@ extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t*
     const int64_t chunks = (block_vecs + per_cta - 1) / per_cta;
     if (chunks > 65535) return PA_ERR_UNSUPPORTED;
     dim3 grid(num_pairs, 2, static_cast<unsigned>(chunks));
-    copy_blocks_kernel<<<grid, kCopyThreads, 0, stream>>>(
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), block_mapping, num_pairs,
-        block_vecs, num_blocks, d_status);
-    return launch_status();
+    return launch_overlapped(copy_blocks_kernel, grid, dim3(kCopyThreads), 0, stream,
+                             static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                             block_mapping, num_pairs, block_vecs, num_blocks, d_status);
 }

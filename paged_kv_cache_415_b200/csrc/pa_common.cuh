@@ -20,6 +20,22 @@ constexpr unsigned kFullMask = 0xffffffffu;
 constexpr uint64_t kWaitTimeoutNs = 1000ull * 1000ull * 1000ull;   // 1 s
 constexpr uint32_t kWaitMaxPolls = 1u << 30;
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start while the previous kernel in the
+// stream is still running; it must call grid_dependency_wait() before it
+// touches any global memory that earlier work produces or reads.  A kernel
+// that calls allow_dependents() lets the next one start launching early.
+// Both are no-ops when the launch carries no such dependency.
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void allow_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "pa.h"
 
 namespace pa {
@@ -20,6 +22,29 @@ inline bool supported_dtype(int32_t t) { return t == PA_DTYPE_F16 || t == PA_DTY
 inline pa_status launch_status()
 {
     return cudaGetLastError() == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialisation: the kernel may begin while
+// the previous kernel in the stream finishes; every kernel of this library
+// waits (griddepcontrol.wait) before touching global memory, so only the
+// launch and ramp-up overlap.
+template <typename... KArgs, typename... Args>
+inline pa_status launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                   cudaStream_t stream, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+               ? launch_status()
+               : PA_ERR_CUDA;
 }
 
 }  // namespace pa

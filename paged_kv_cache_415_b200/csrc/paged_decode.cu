@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
     int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
     int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status)
 {
+    grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = DecodeShape<D, BS, G>;
     constexpr int EP = S::EPT / 2;      // element pairs per lane
     extern __shared__ __align__(128) unsigned char smem[];
@@ -496,6 +497,7 @@ __global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_reduce_ke
     int32_t max_context_len, int32_t max_blocks_per_seq, int32_t block_size,
     int32_t partition_size, int32_t max_parts)
 {
+    grid_dependency_wait();
     constexpr int EPL = D / 32;     // elements per lane
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kReduceRowsPerCta + (threadIdx.x >> 5);
@@ -657,10 +659,12 @@ static pa_status launch_decode(const DecodeArgs& a)
         if (!encode_pool_map_swizzled(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
             !encode_pool_map_swizzled(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
             return PA_ERR_CUDA;
-        kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
-            tm_k, tm_v, static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables,
-            a.context_lens, a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len,
-            a.scale_log2, a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+        const pa_status ls = launch_overlapped(
+            kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v,
+            static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables, a.context_lens,
+            a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2,
+            a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+        if (ls != PA_OK) return ls;
     } else {
         using S = DecodeShape<D, BS, G>;
         static std::atomic<uint64_t> attr_done{0};
@@ -669,19 +673,21 @@ static pa_status launch_decode(const DecodeArgs& a)
         if (!encode_pool_map(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
             !encode_pool_map(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
             return PA_ERR_CUDA;
-        kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
-            tm_k, tm_v, static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables,
-            a.context_lens, a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len,
-            a.scale_log2, a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+        const pa_status ls = launch_overlapped(
+            kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v,
+            static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables, a.context_lens,
+            a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2,
+            a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+        if (ls != PA_OK) return ls;
     }
-    pa_status st = launch_status();
-    if (st != PA_OK || a.max_parts <= 1) return st;
+    if (a.max_parts <= 1) return PA_OK;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
-    paged_decode_reduce_kernel<T, D><<<ctas, kReduceRowsPerCta * 32, 0, a.stream>>>(
-        static_cast<T*>(a.out), a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
-        a.max_context_len, a.max_blocks_per_seq, a.block_size, a.partition_size, a.max_parts);
-    return launch_status();
+    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(ctas),
+                             dim3(kReduceRowsPerCta * 32), 0, a.stream, static_cast<T*>(a.out),
+                             a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
+                             a.max_context_len, a.max_blocks_per_seq, a.block_size,
+                             a.partition_size, a.max_parts);
 }
 
 template <typename T, int D, int BS>
@@ -739,20 +745,21 @@ static pa_status launch_shared(const SharedArgs& sa)
     const int32_t parts = sa.slots - sa.prefix_slots > sa.prefix_slots ? sa.slots - sa.prefix_slots
                                                                        : sa.prefix_slots;
     dim3 grid(a.num_kv_heads, parts > 0 ? parts : 1, num_groups + a.num_seqs);
-    kernel<<<grid, kThreads, S::SMEM_BYTES, a.stream>>>(
-        tm_k, tm_v, static_cast<const T*>(a.query), a.block_tables, a.context_lens,
-        sa.prefix_lens, num_groups, sa.group_size, a.num_q_heads / a.num_kv_heads, a.num_q_heads,
-        a.max_blocks_per_seq, a.num_blocks, a.max_context_len, sa.max_prefix_len, a.scale_log2,
-        a.partition_size, sa.prefix_slots, sa.slots, a.ws_o, a.ws_ml, a.d_status);
-    pa_status st = launch_status();
+    pa_status st = launch_overlapped(
+        kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v,
+        static_cast<const T*>(a.query), a.block_tables, a.context_lens, sa.prefix_lens, num_groups,
+        sa.group_size, a.num_q_heads / a.num_kv_heads, a.num_q_heads, a.max_blocks_per_seq,
+        a.num_blocks, a.max_context_len, sa.max_prefix_len, a.scale_log2, a.partition_size,
+        sa.prefix_slots, sa.slots, a.ws_o, a.ws_ml, a.d_status);
     if (st != PA_OK) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
-    paged_decode_shared_reduce_kernel<T, D><<<ctas, kReduceRowsPerCta * 32, 0, a.stream>>>(
-        static_cast<T*>(a.out), a.ws_o, a.ws_ml, a.context_lens, sa.prefix_lens, a.num_seqs,
-        sa.group_size, a.num_q_heads, a.max_context_len, a.max_blocks_per_seq, a.block_size,
-        sa.max_prefix_len, a.partition_size, sa.prefix_slots, sa.slots, a.d_status);
-    return launch_status();
+    return launch_overlapped(paged_decode_shared_reduce_kernel<T, D>, dim3(ctas),
+                             dim3(kReduceRowsPerCta * 32), 0, a.stream, static_cast<T*>(a.out),
+                             a.ws_o, a.ws_ml, a.context_lens, sa.prefix_lens, a.num_seqs,
+                             sa.group_size, a.num_q_heads, a.max_context_len, a.max_blocks_per_seq,
+                             a.block_size, sa.max_prefix_len, a.partition_size, sa.prefix_slots,
+                             sa.slots, a.d_status);
 }
 
 template <typename T>

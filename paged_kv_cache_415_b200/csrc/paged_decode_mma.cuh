@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
     int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
     int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status)
 {
+    grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = MmaShape<D, BS, G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // the 128-byte swizzle repeats every 1024 bytes: align the tiles to it

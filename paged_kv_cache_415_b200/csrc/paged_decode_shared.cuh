@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
     int32_t max_prefix_len, float scale_log2, int32_t partition_size, int32_t prefix_slots,
     int32_t slots, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status)
 {
+    grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = SharedShape<D, BS>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -346,6 +347,7 @@ __global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_shared_re
     int32_t max_blocks_per_seq, int32_t block_size, int32_t max_prefix_len,
     int32_t partition_size, int32_t prefix_slots, int32_t slots, int32_t* d_status)
 {
+    grid_dependency_wait();
     constexpr int EPL = D / 32;
     const int lane = threadIdx.x & 31;
     const int64_t row = static_cast<int64_t>(blockIdx.x) * kReduceRowsPerCta + (threadIdx.x >> 5);
