@@ -63,6 +63,9 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--partition", type=int, default=-1,
                     help="context partition in tokens (-1 = the workload's, 0 = library's choice)")
+    ap.add_argument("--separate", action="store_true",
+                    help="run the cache write and the decode as separate calls even when every "
+                         "sequence appends one token (default: pa_paged_decode_append)")
     ap.add_argument("--shared-prefix", action="store_true",
                     help="beam_search: decode with pa_paged_decode_shared_prefix (shared "
                          "prompt blocks read once per group)")
@@ -339,10 +342,13 @@ def run_ours(args):
     n_pairs = int(wl.block_mapping.shape[0])
     stream = torch.cuda.current_stream(dev)
 
+    fused = (not args.separate and not args.shared_prefix
+             and wl.extra.get("one_token_per_seq", False) and wl.num_new_tokens == wl.num_seqs)
+
     def cache_ops():
         if n_pairs:
             B.pa_copy_blocks(k_cache, v_cache, block_mapping, d_status, stream)
-        if wl.num_new_tokens:
+        if wl.num_new_tokens and not fused:
             B.pa_reshape_and_cache(new_key, new_value, k_cache, v_cache, slot_mapping, d_status,
                                    stream)
 
@@ -357,7 +363,11 @@ def run_ours(args):
         workspace = torch.empty(max(sws, 16), dtype=torch.uint8, device=dev)
 
     def decode():
-        if shared:
+        if fused:
+            B.pa_paged_decode_append(out, query, new_key, new_value, k_cache, v_cache,
+                                     block_tables, context_lens, mcl, wl.scale, part, workspace,
+                                     d_status, stream)
+        elif shared:
             B.pa_paged_decode_shared_prefix(out, query, k_cache, v_cache, block_tables,
                                             context_lens, prefix_lens, group_size, mcl, mpl,
                                             wl.scale, workspace, part, d_status, stream)
@@ -365,8 +375,8 @@ def run_ours(args):
             B.pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl,
                               wl.scale, part, workspace, d_status, stream)
 
-    launches_per_step = (1 if n_pairs else 0) + (1 if wl.num_new_tokens else 0) + 1 + \
-        (1 if (max_parts > 1 or shared) else 0)
+    launches_per_step = (1 if n_pairs else 0) + (1 if (wl.num_new_tokens and not fused) else 0) + \
+        1 + (1 if (max_parts > 1 or shared) else 0)
 
     def barrier():
         if world > 1:
@@ -412,8 +422,11 @@ def run_ours(args):
     if wl.num_new_tokens:
         host["new_key"] = torch.from_numpy(wl.new_key.view(np.int16)).view(tdt).pin_memory()
         host["new_value"] = torch.from_numpy(wl.new_value.view(np.int16)).view(tdt).pin_memory()
-        host["slot_mapping"] = torch.from_numpy(wl.slot_mapping).pin_memory()
-        for k in ("new_key", "new_value", "slot_mapping"):
+        names = ("new_key", "new_value")
+        if not fused:
+            host["slot_mapping"] = torch.from_numpy(wl.slot_mapping).pin_memory()
+            names += ("slot_mapping",)
+        for k in names:
             devb[k] = torch.empty_like(host[k], device=dev)
     if n_pairs:
         host["block_mapping"] = torch.from_numpy(np.ascontiguousarray(wl.block_mapping)).pin_memory()
@@ -421,12 +434,12 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for k, t in host.items() if k != "out")
     d2h = host["out"].numel() * host["out"].element_size()
     for _ in range(max(3, args.warmup)):
-        stepper.run_from_host(host, devb, wl.scale, stream)
+        stepper.run_from_host(host, devb, wl.scale, stream, fused_append=fused)
     barrier()
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(stream)
     for _ in range(args.steps):
-        stepper.run_from_host(host, devb, wl.scale, stream)
+        stepper.run_from_host(host, devb, wl.scale, stream, fused_append=fused)
     e_stop.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
@@ -440,7 +453,9 @@ def run_ours(args):
     value = whole_job_gbs(step["total"], args.steps, world, elapsed_ms)
     e2e_value = whole_job_gbs(step["total"], args.steps, world, e2e_ms)
     peak, peak_kind = hbm_peak()
-    achieved = step["attention"] / (decode_avg * 1e-3) / 1e9
+    # the decode launch also carries the step's cache write when it is fused
+    decode_bytes = step["attention"] + (step["append"] if fused else 0)
+    achieved = decode_bytes / (decode_avg * 1e-3) / 1e9
     traffic = profiled_traffic(args.config)
     clocks = sampler.summary()
 
@@ -475,7 +490,7 @@ def run_ours(args):
         "roofline": {"bound": "hbm", "kernel": kernel_name,
                      "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "algorithmic_bytes_per_launch": step["attention"],
+                     "traffic": traffic, "algorithmic_bytes_per_launch": decode_bytes,
                      "avg_launch_us": round(decode_avg * 1e3, 2)},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5)},
@@ -483,7 +498,9 @@ def run_ours(args):
         "clocks": clocks,
         "cpu_baseline": cpu,
         "bytes_per_step": step,
-        "decode_entry": "pa_paged_decode_shared_prefix" if shared else "pa_paged_decode",
+        "decode_entry": ("pa_paged_decode_shared_prefix" if shared else
+                         "pa_paged_decode_append (cache write fused)" if fused else
+                         "pa_reshape_and_cache + pa_paged_decode"),
     }
     if "prefix_lens" in wl.extra:
         uniq = bm.unique_kv_bytes(wl)

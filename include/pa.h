@@ -229,6 +229,38 @@ PA_API pa_status pa_paged_decode(void* out, const void* query, const void* k_cac
                           int32_t* d_status, pa_stream_t stream);
 
 /*
+ * pa_paged_decode_append -- one decode step in one launch: each sequence's
+ * new token is written into the cache and attended to, as
+ * pa_reshape_and_cache followed by pa_paged_decode would do.
+ *
+ * Defined by: [Manager, 第一部分 KV Cache 的核心价值] (store the new token's K and
+ * V, then attend over the whole cache) with the write of [Practice §3.3] step
+ * 4 and the attention of pa_paged_decode.  For the usual decode batch in
+ * which sequence s appends exactly one token, at position context_lens[s] - 1,
+ * whose slot is given by its own block table:
+ *   slot = block_tables[s][(ctx - 1) / block_size] * block_size + (ctx - 1) % block_size.
+ * The CTA that owns a sequence's last context partition writes that token's
+ * K/V row for its kv head before loading any tile, so no separate cache-write
+ * kernel (and no launch dependency) is needed.
+ *
+ * key, value     [num_seqs][num_kv_heads][head_dim], 16-byte aligned: the new
+ *                token of every sequence.  k_cache / v_cache are written.
+ * Other arguments, results and errors as pa_paged_decode; a table entry
+ * outside the pool for the new token sets PA_STATUS_BAD_SLOT and the token
+ * is not written.  Sequences with context length 0 append nothing.
+ */
+PA_API pa_status pa_paged_decode_append(void* out, const void* query, const void* key,
+                                        const void* value, void* k_cache, void* v_cache,
+                                        const int32_t* block_tables, const int32_t* context_lens,
+                                        int32_t num_seqs, int32_t num_q_heads,
+                                        int32_t num_kv_heads, int32_t head_dim,
+                                        int32_t block_size, int32_t max_blocks_per_seq,
+                                        int64_t num_blocks, int32_t max_context_len, float scale,
+                                        int32_t partition_size, void* workspace,
+                                        size_t workspace_bytes, pa_dtype dtype,
+                                        int32_t* d_status, pa_stream_t stream);
+
+/*
  * pa_paged_decode_shared_prefix -- pa_paged_decode for batches whose
  * sequences come in groups that share a stored prefix (the beams of one
  * prompt, parallel samples of one request).

@@ -34,6 +34,7 @@ _DTYPES = {torch.float16: PA_DTYPE_F16, torch.bfloat16: PA_DTYPE_BF16}
 EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_size",
            "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_paged_decode_no_alloc",
            "pa_paged_decode_shared_prefix_workspace_size", "pa_paged_decode_shared_prefix",
+           "pa_paged_decode_append",
            "pa_status_string", "pa_version")
 # Size of the library-owned scratch of pa_paged_decode_no_alloc.
 PA_NO_ALLOC_WORKSPACE_BYTES = 32 << 20
@@ -71,6 +72,9 @@ def _load() -> ctypes.CDLL:
                                                   i32, i32, i64, i32, i32, f32, i32, p, sz, i32,
                                                   p, p]
     lib.pa_paged_decode_shared_prefix.restype = i32
+    lib.pa_paged_decode_append.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, i32, i32, i32,
+                                           i64, i32, f32, i32, p, sz, i32, p, p]
+    lib.pa_paged_decode_append.restype = i32
     lib.pa_status_string.argtypes = [i32]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
@@ -202,3 +206,20 @@ def pa_paged_decode_shared_prefix(out, query, k_cache, v_cache, block_tables, co
         int(block_tables.shape[1]), num_blocks, int(max_context_len), int(max_prefix_len),
         float(scale), int(partition_size), _ptr(workspace), ws_bytes, _dtype(query),
         _ptr(d_status), _stream(stream)))
+
+
+def pa_paged_decode_append(out, query, key, value, k_cache, v_cache, block_tables, context_lens,
+                           max_context_len, scale, partition_size=0, workspace=None,
+                           d_status=None, stream=None) -> None:
+    """One decode step in one launch: key/value [S][Hkv][D] hold each
+    sequence's new token (position context_lens[s] - 1, slot from its block
+    table); it is written into k_cache/v_cache and attended to."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_paged_decode_append", LIB.pa_paged_decode_append(
+        _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), num_seqs, hq, hkv, d, block_size,
+        int(block_tables.shape[1]), num_blocks, int(max_context_len), float(scale),
+        int(partition_size), _ptr(workspace), ws_bytes, _dtype(query), _ptr(d_status),
+        _stream(stream)))

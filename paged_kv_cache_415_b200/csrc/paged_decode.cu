@@ -132,6 +132,32 @@ __device__ __forceinline__ void write_zero_rows(T* out, int s, int kvh, int num_
         reinterpret_cast<uint4*>(row)[i] = make_uint4(0, 0, 0, 0);
 }
 
+// Fused append: the warp that loads the block holding a sequence's new token
+// (position ctx - 1) first writes that token's K and V row for its kv head
+// into the pools at the given physical block, then makes the writes visible
+// to the tensor-copy engine before the block's tiles are requested.  No
+// other warp or CTA reads that (token, kv head) row.  Warp-uniform; the
+// caller issues the block's copies right after.
+template <typename T, int D, int BS>
+__device__ __forceinline__ void append_row_warp(
+    const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
+    T* __restrict__ v_cache, int s, int kvh, int num_kv_heads, int32_t pos, int32_t phys,
+    int lane)
+{
+    const int64_t slot = static_cast<int64_t>(phys) * BS + pos % BS;
+    const int64_t src = (static_cast<int64_t>(s) * num_kv_heads + kvh) * D;
+    const int64_t dst = (slot * num_kv_heads + kvh) * D;
+    if (lane < D / 8) {
+        const uint4 kv = ld_nc_v4(new_key + src + lane * 8);
+        const uint4 vv = ld_nc_v4(new_value + src + lane * 8);
+        *reinterpret_cast<uint4*>(k_cache + dst + lane * 8) = kv;
+        *reinterpret_cast<uint4*>(v_cache + dst + lane * 8) = vv;
+        fence_proxy_async_global();
+    }
+    __syncwarp();
+    fence_proxy_async_global();
+}
+
 // The CTA's last step: merge the four warps' (max, exp-sum, output) for the
 // G heads of its kv head in a fixed order, then either write the output row
 // (context in one partition) or the partition's max, sum and normalised
@@ -188,7 +214,9 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
     T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
     const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
     int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
-    int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status)
+    int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status,
+    const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
+    T* __restrict__ v_cache, int32_t num_kv_heads)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = DecodeShape<D, BS, G>;
@@ -223,6 +251,8 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
     const int blk_begin = tok_begin / BS;
     const int nblk = (tok_end - tok_begin + BS - 1) / BS;
     const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;   // this warp's blocks
+    // the block (of this partition) holding the new token, when appending
+    const int append_blk = (new_key != nullptr && part == nparts - 1) ? (ctx - 1) / BS - blk_begin : -1;
 
     unsigned char* wstage = smem + warp * S::WARP_STAGE_BYTES;
     float* wscore = reinterpret_cast<float*>(smem + S::OFF_SCORES) + warp * S::SCORE_FLOATS;
@@ -261,6 +291,13 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
             prod_chunk = chunk;
         }
         const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
+        if (warp + kWarps * k == append_blk) {
+            if (phys >= 0 && static_cast<int64_t>(phys) < num_blocks)
+                append_row_warp<T, D, BS>(new_key, new_value, k_cache, v_cache, s, kvh,
+                                          num_kv_heads, ctx - 1, phys, lane);
+            else if (lane == 0)
+                status_or(d_status, PA_STATUS_BAD_SLOT);
+        }
         if (lane == 0) {
             const int st = k % S::NSTAGE;
             const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
@@ -564,6 +601,8 @@ struct DecodeArgs {
     float2* ws_ml;
     int32_t* d_status;
     cudaStream_t stream;
+    const void* new_key = nullptr;     // fused append (one token per sequence), or null
+    const void* new_value = nullptr;
 };
 
 template <typename Kernel>
@@ -663,7 +702,10 @@ static pa_status launch_decode(const DecodeArgs& a)
             kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v,
             static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables, a.context_lens,
             a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2,
-            a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+            a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status,
+            static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
+            static_cast<T*>(const_cast<void*>(a.k_cache)), static_cast<T*>(const_cast<void*>(a.v_cache)),
+            a.num_kv_heads);
         if (ls != PA_OK) return ls;
     } else {
         using S = DecodeShape<D, BS, G>;
@@ -677,7 +719,10 @@ static pa_status launch_decode(const DecodeArgs& a)
             kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v,
             static_cast<T*>(a.out), static_cast<const T*>(a.query), a.block_tables, a.context_lens,
             a.num_q_heads, a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2,
-            a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+            a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status,
+            static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
+            static_cast<T*>(const_cast<void*>(a.k_cache)), static_cast<T*>(const_cast<void*>(a.v_cache)),
+            a.num_kv_heads);
         if (ls != PA_OK) return ls;
     }
     if (a.max_parts <= 1) return PA_OK;
@@ -863,17 +908,17 @@ extern "C" size_t pa_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q
     return workspace_bytes_for(num_seqs, num_q_heads, head_dim, parts_for(max_context_len, p));
 }
 
-extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k_cache,
-                                     const void* v_cache, const int32_t* block_tables,
-                                     const int32_t* context_lens, int32_t num_seqs,
-                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                                     int32_t block_size, int32_t max_blocks_per_seq,
-                                     int64_t num_blocks, int32_t max_context_len, float scale,
-                                     int32_t partition_size, void* workspace,
-                                     size_t workspace_bytes, pa_dtype dtype, int32_t* d_status,
-                                     pa_stream_t stream)
+namespace pa {
+
+static pa_status decode_impl(void* out, const void* query, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                             int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq,
+                             int64_t num_blocks, int32_t max_context_len, float scale,
+                             int32_t partition_size, void* workspace, size_t workspace_bytes,
+                             pa_dtype dtype, int32_t* d_status, pa_stream_t stream,
+                             const void* new_key, const void* new_value)
 {
-    using namespace pa;
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       max_context_len, partition_size);
     if (st != PA_OK) return st;
@@ -883,6 +928,9 @@ extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k
         return PA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(query) || !aligned16(k_cache) || !aligned16(v_cache) ||
         !aligned4(block_tables) || !aligned4(context_lens) || (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    if (new_key != nullptr &&
+        (new_value == nullptr || !aligned16(new_key) || !aligned16(new_value)))
         return PA_ERR_INVALID_ARG;
     const int32_t partition = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
                                                partition_size);
@@ -918,7 +966,46 @@ extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k
                    : nullptr;
     a.d_status = d_status;
     a.stream = stream;
+    a.new_key = new_key;
+    a.new_value = new_value;
     return dtype == PA_DTYPE_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
+}
+
+}  // namespace pa
+
+extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int32_t max_blocks_per_seq,
+                                     int64_t num_blocks, int32_t max_context_len, float scale,
+                                     int32_t partition_size, void* workspace,
+                                     size_t workspace_bytes, pa_dtype dtype, int32_t* d_status,
+                                     pa_stream_t stream)
+{
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, nullptr, nullptr);
+}
+
+extern "C" pa_status pa_paged_decode_append(void* out, const void* query, const void* key,
+                                            const void* value, void* k_cache, void* v_cache,
+                                            const int32_t* block_tables,
+                                            const int32_t* context_lens, int32_t num_seqs,
+                                            int32_t num_q_heads, int32_t num_kv_heads,
+                                            int32_t head_dim, int32_t block_size,
+                                            int32_t max_blocks_per_seq, int64_t num_blocks,
+                                            int32_t max_context_len, float scale,
+                                            int32_t partition_size, void* workspace,
+                                            size_t workspace_bytes, pa_dtype dtype,
+                                            int32_t* d_status, pa_stream_t stream)
+{
+    if (key == nullptr || value == nullptr) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, key, value);
 }
 
 // ---------------------------------------------------------------------------

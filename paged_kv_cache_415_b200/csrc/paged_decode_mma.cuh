@@ -67,7 +67,9 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
     T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
     const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
     int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
-    int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status)
+    int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status,
+    const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
+    T* __restrict__ v_cache, int32_t num_kv_heads)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = MmaShape<D, BS, G>;
@@ -103,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
     const int blk_begin = tok_begin / BS;
     const int nblk = (tok_end - tok_begin + BS - 1) / BS;
     const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
+    const int append_blk = (new_key != nullptr && part == nparts - 1) ? (ctx - 1) / BS - blk_begin : -1;
 
     unsigned char* wstage = smem + warp * S::WARP_STAGE_BYTES;
     uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
@@ -135,6 +138,13 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
             prod_chunk = chunk;
         }
         const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
+        if (warp + kWarps * k == append_blk) {
+            if (phys >= 0 && static_cast<int64_t>(phys) < num_blocks)
+                append_row_warp<T, D, BS>(new_key, new_value, k_cache, v_cache, s, kvh,
+                                          num_kv_heads, ctx - 1, phys, lane);
+            else if (lane == 0)
+                status_or(d_status, PA_STATUS_BAD_SLOT);
+        }
         if (lane == 0) {
             const int st = k % S::NSTAGE;
             const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;

@@ -40,20 +40,29 @@ class DecodeStep:
 
     def __call__(self, query, block_tables, context_lens, scale, out=None, new_key=None,
                  new_value=None, slot_mapping=None, block_mapping=None, stream=None,
-                 max_context_len=None):
+                 max_context_len=None, fused_append=False):
+        """fused_append: every sequence appends exactly one token (new_key /
+        new_value hold one row per sequence, at position context_lens - 1);
+        the cache write then runs inside the decode launch
+        (pa_paged_decode_append) and slot_mapping is not used."""
         if block_mapping is not None and block_mapping.shape[0] > 0:
             B.pa_copy_blocks(self.k_cache, self.v_cache, block_mapping, self.d_status, stream)
+        if out is None:
+            out = torch.empty_like(query)
+        mcl = self.max_context_len if max_context_len is None else max_context_len
+        if fused_append:
+            B.pa_paged_decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache,
+                                     block_tables, context_lens, mcl, scale, self.partition_size,
+                                     self.workspace, self.d_status, stream)
+            return out
         if slot_mapping is not None and slot_mapping.shape[0] > 0:
             B.pa_reshape_and_cache(new_key, new_value, self.k_cache, self.v_cache, slot_mapping,
                                    self.d_status, stream)
-        if out is None:
-            out = torch.empty_like(query)
-        B.pa_paged_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens,
-                          self.max_context_len if max_context_len is None else max_context_len,
+        B.pa_paged_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, mcl,
                           scale, self.partition_size, self.workspace, self.d_status, stream)
         return out
 
-    def run_from_host(self, host: dict, dev: dict, scale, stream=None):
+    def run_from_host(self, host: dict, dev: dict, scale, stream=None, fused_append=False):
         """host / dev: dicts of same-shaped tensors (pinned host / device) for
         'query', 'block_tables', 'context_lens', 'new_key', 'new_value',
         'slot_mapping', 'block_mapping' (the last four optional) and 'out'.
@@ -67,6 +76,6 @@ class DecodeStep:
             self(dev["query"], dev["block_tables"], dev["context_lens"], scale, out=dev["out"],
                  new_key=dev.get("new_key"), new_value=dev.get("new_value"),
                  slot_mapping=dev.get("slot_mapping"), block_mapping=dev.get("block_mapping"),
-                 stream=s)
+                 stream=s, fused_append=fused_append)
             host["out"].copy_(dev["out"], non_blocking=True)
         return host["out"]

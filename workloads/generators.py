@@ -157,6 +157,8 @@ def make_decode(name, *, seed, dtype, context_lens, num_q_heads, num_kv_heads, h
         wl.keys = [keys[starts[s]:starts[s] + ctx[s]] for s in range(s_n)]
         wl.values = [vals[starts[s]:starts[s] + ctx[s]] for s in range(s_n)]
     wl.extra["manager"] = mgr
+    # every sequence appends exactly one token, at position ctx - 1
+    wl.extra["one_token_per_seq"] = bool(np.all(ctx > 0))
     return wl
 
 
