@@ -136,7 +136,7 @@ class BlockManager:
         return slots, cow
 
     def free_sequence(self, seq: int) -> None:
-        for blk in self.tables.pop(seq):
+        for blk in reversed(self.tables.pop(seq)):         # last block first
             self.ref[blk] -= 1
             assert self.ref[blk] >= 0
             if self.ref[blk] == 0:
