@@ -61,6 +61,16 @@ def load(path: str | None = None):
     lib.oracle_paged_decode_rows.argtypes = [p, p, i32, p, p, p, p, p, i32, i32, i32, i32,
                                              i32, i64, f64, i32, i32]
     lib.oracle_paged_decode_rows.restype = i32
+    lib.oracle_decode_e4m3.argtypes = [p, p, i64]
+    lib.oracle_decode_e4m3.restype = None
+    lib.oracle_encode_e4m3.argtypes = [p, p, i64]
+    lib.oracle_encode_e4m3.restype = None
+    lib.oracle_reshape_and_cache_fp8.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i32,
+                                                 ctypes.c_float, ctypes.c_float]
+    lib.oracle_reshape_and_cache_fp8.restype = i32
+    lib.oracle_paged_decode_fp8.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64,
+                                            f64, i32, f64, f64, i32]
+    lib.oracle_paged_decode_fp8.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     if path is None:
@@ -151,4 +161,52 @@ def paged_decode_rows(rows, query, k_cache, v_cache, block_tables, context_lens,
         _ptr(out), _ptr(rows), rows.shape[0], _ptr(query), _ptr(k_cache), _ptr(v_cache),
         _ptr(block_tables), _ptr(context_lens), hq, hkv, d, bs, block_tables.shape[1],
         num_blocks, float(scale), _DTYPES[dtype], num_threads)
+    return out, int(st)
+
+
+# ---- FP8 (e4m3) caches: uint8 codes, per-tensor scales ------------------------
+
+def decode_e4m3(codes: np.ndarray, lib=None) -> np.ndarray:
+    """e4m3 code -> float64 (exact; 0x7F / 0xFF -> NaN)."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape, dtype=np.float64)
+    (lib or load()).oracle_decode_e4m3(_ptr(codes), _ptr(out), codes.size)
+    return out
+
+
+def encode_e4m3(x: np.ndarray, lib=None) -> np.ndarray:
+    """float32 -> e4m3 code, round to nearest even, saturating at +-448."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    (lib or load()).oracle_encode_e4m3(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, block_size, dtype,
+                          k_scale, v_scale, lib=None) -> int:
+    """Quantising cache write into uint8 pools [num_blocks][B][Hkv][D]."""
+    key, value = _u16(key), _u16(value)
+    assert k_cache.dtype == np.uint8 and v_cache.dtype == np.uint8
+    slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    num_blocks, bs, hkv, d = k_cache.shape
+    return int((lib or load()).oracle_reshape_and_cache_fp8(
+        _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+        key.shape[0], hkv, d, block_size, num_blocks, _DTYPES[dtype], float(k_scale),
+        float(v_scale)))
+
+
+def paged_decode_fp8(query, k_cache, v_cache, block_tables, context_lens, scale, dtype, k_scale,
+                     v_scale, num_threads=0, lib=None):
+    """fp64 paged decode over e4m3 pools (dequantised with the scales)."""
+    query = _u16(query)
+    block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    s, hq, d = query.shape
+    num_blocks, bs, hkv, _ = k_cache.shape
+    out = np.empty((s, hq, d), dtype=np.float64)
+    st = (lib or load()).oracle_paged_decode_fp8(
+        _ptr(out), _ptr(query), _ptr(np.ascontiguousarray(k_cache, dtype=np.uint8)),
+        _ptr(np.ascontiguousarray(v_cache, dtype=np.uint8)), _ptr(block_tables),
+        _ptr(context_lens), s, hq, hkv, d, bs, block_tables.shape[1], num_blocks, float(scale),
+        _DTYPES[dtype], float(k_scale), float(v_scale), num_threads)
     return out, int(st)

@@ -91,6 +91,91 @@ void oracle_decode_bits(const uint16_t* bits, double* out, int64_t n, int32_t dt
 }
 
 /* ------------------------------------------------------------------------
+ * FP8 E4M3 (OCP "e4m3fn"): 1 sign bit, 4 exponent bits (bias 7), 3 fraction
+ * bits, no infinities; 0x7F / 0xFF are NaN; the largest finite value is
+ * 448 = 1.75 x 2^8; subnormals are fraction x 2^-9.  Cached K/V stored in
+ * 8 bits with a per-tensor scale ("PagedAttention：大模型KV Cache分页管理优化实践"
+ * §7: FP8/INT8 storage of history blocks; "vLLM用虚拟内存分页思想管理KV Cache",
+ * 工程实践与局限: low-precision storage of block KV values).
+ * ---------------------------------------------------------------------- */
+static double e4m3_to_f64(uint8_t b)
+{
+    int sign = (b >> 7) & 1;
+    int expo = (b >> 3) & 0xf;
+    int frac = b & 7;
+    double v;
+    if (expo == 15 && frac == 7)
+        v = NAN;
+    else if (expo == 0)
+        v = ldexp((double)frac, -9);
+    else
+        v = ldexp((double)(frac + 8), expo - 10);
+    return sign ? -v : v;
+}
+
+void oracle_decode_e4m3(const uint8_t* codes, double* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_to_f64(codes[i]);
+}
+
+/* fp32 -> e4m3, round to nearest (ties to even), values beyond the largest
+ * finite magnitude saturate to +-448, NaN -> 0x7F.  Done by exact search
+ * over the 126 finite non-negative codes in double: the candidates below and
+ * above |x| and the tie rule decide. */
+static uint8_t f32_to_e4m3(float x)
+{
+    if (x != x) return 0x7f;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7e);
+    /* largest code with value <= a */
+    int lo = 0;
+    for (int c = 0; c <= 0x7e; ++c)
+        if (e4m3_to_f64((uint8_t)c) <= a) lo = c;
+    int hi = lo < 0x7e ? lo + 1 : lo;
+    double vlo = e4m3_to_f64((uint8_t)lo), vhi = e4m3_to_f64((uint8_t)hi);
+    int pick;
+    if (a - vlo < vhi - a) pick = lo;
+    else if (a - vlo > vhi - a) pick = hi;
+    else pick = (lo & 1) ? hi : lo;        /* tie: even fraction (even code) */
+    return (uint8_t)(sign | pick);
+}
+
+void oracle_encode_e4m3(const float* x, uint8_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = f32_to_e4m3(x[i]);
+}
+
+/* Quantising cache write: code = e4m3(fp32(x) * fp32(1 / scale)), the
+ * product rounded once in fp32, then rounded to e4m3 as above. */
+int32_t oracle_reshape_and_cache_fp8(const uint16_t* key, const uint16_t* value, uint8_t* k_cache,
+                                     uint8_t* v_cache, const int64_t* slot_mapping,
+                                     int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int64_t num_blocks, int32_t dtype,
+                                     float k_scale, float v_scale)
+{
+    int32_t status = 0;
+    const float k_inv = 1.0f / k_scale, v_inv = 1.0f / v_scale;
+    const int64_t row = (int64_t)num_kv_heads * head_dim;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * (int64_t)block_size) { status |= 2; continue; }
+        for (int64_t e = 0; e < row; ++e) {
+            const float kx = (float)(dtype == OR_DTYPE_BF16 ? bf16_bits_to_f64(key[t * row + e])
+                                                            : f16_bits_to_f64(key[t * row + e]));
+            const float vx = (float)(dtype == OR_DTYPE_BF16 ? bf16_bits_to_f64(value[t * row + e])
+                                                            : f16_bits_to_f64(value[t * row + e]));
+            const float kq = kx * k_inv;
+            const float vq = vx * v_inv;
+            k_cache[slot * row + e] = f32_to_e4m3(kq);
+            v_cache[slot * row + e] = f32_to_e4m3(vq);
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------
  * reshape_and_cache: write each new token's K and V rows into the slot the
  * allocator gave it ([Practice §3.3 按需分配策略], step 4 "write the new
  * token's KV vectors"; [Manager, 第一部分 KV Cache 的核心价值]: the new K/V is
@@ -259,6 +344,56 @@ static int32_t decode_row(double* out, const uint16_t* query, const uint16_t* k_
     return status;
 }
 
+/* Paged decode over e4m3 pools: every cached element is dequantised,
+ * K = decode(code) * k_scale, V = decode(code) * v_scale, in double, and the
+ * attention is the direct form of decode_row.  Query and output as in
+ * oracle_paged_decode (query bits of `dtype`). */
+static int32_t decode_row_fp8(double* out, const uint16_t* query, const uint8_t* k_cache,
+                              const uint8_t* v_cache, const int32_t* block_tables,
+                              const int32_t* context_lens, int32_t s, int32_t h,
+                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+                              double scale, int32_t dtype, double k_scale, double v_scale)
+{
+    int32_t status = 0;
+    const int32_t group = num_q_heads / num_kv_heads;
+    const int32_t g = h / group;
+    const int32_t ctx = context_lens[s];
+    const int32_t* table = block_tables + (int64_t)s * max_blocks_per_seq;
+    for (int32_t d = 0; d < head_dim; ++d) out[d] = 0.0;
+    if (ctx < 0 || ctx > (int64_t)max_blocks_per_seq * block_size) return 4;
+    if (ctx == 0) return 0;
+    double* q = (double*)malloc(sizeof(double) * head_dim);
+    double* x = (double*)malloc(sizeof(double) * ctx);
+    unsigned char* valid = (unsigned char*)malloc(ctx);
+    const uint16_t* qbits = query + ((int64_t)s * num_q_heads + h) * head_dim;
+    for (int32_t d = 0; d < head_dim; ++d) q[d] = decode(qbits[d], dtype);
+    int32_t any = 0;
+    for (int32_t t = 0; t < ctx; ++t) {
+        int64_t r = token_row(table, t, g, num_kv_heads, head_dim, block_size, num_blocks);
+        valid[t] = r >= 0;
+        if (r < 0) { status |= 1; x[t] = 0.0; continue; }
+        double acc = 0.0;
+        for (int32_t d = 0; d < head_dim; ++d) acc += q[d] * (e4m3_to_f64(k_cache[r + d]) * k_scale);
+        x[t] = scale * acc;
+        any = 1;
+    }
+    if (any) {
+        double m = -INFINITY, l = 0.0;
+        for (int32_t t = 0; t < ctx; ++t) if (valid[t] && x[t] > m) m = x[t];
+        for (int32_t t = 0; t < ctx; ++t) if (valid[t]) l += exp(x[t] - m);
+        for (int32_t t = 0; t < ctx; ++t) {
+            if (!valid[t]) continue;
+            double w = exp(x[t] - m) / l;
+            int64_t r = token_row(table, t, g, num_kv_heads, head_dim, block_size, num_blocks);
+            for (int32_t d = 0; d < head_dim; ++d)
+                out[d] += w * (e4m3_to_f64(v_cache[r + d]) * v_scale);
+        }
+    }
+    free(q); free(x); free(valid);
+    return status;
+}
+
 static void set_threads(int32_t num_threads)
 {
 #ifdef _OPENMP
@@ -320,4 +455,26 @@ int32_t oracle_max_threads(void)
 #else
     return 1;
 #endif
+}
+
+int32_t oracle_paged_decode_fp8(double* out, const uint16_t* query, const uint8_t* k_cache,
+                                const uint8_t* v_cache, const int32_t* block_tables,
+                                const int32_t* context_lens, int32_t num_seqs,
+                                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t block_size, int32_t max_blocks_per_seq,
+                                int64_t num_blocks, double scale, int32_t dtype, double k_scale,
+                                double v_scale, int32_t num_threads)
+{
+    int32_t status = 0;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads;
+    set_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : status)
+    for (int64_t r = 0; r < rows; ++r) {
+        int32_t s = (int32_t)(r / num_q_heads), h = (int32_t)(r % num_q_heads);
+        status |= decode_row_fp8(out + r * head_dim, query, k_cache, v_cache, block_tables,
+                                 context_lens, s, h, num_q_heads, num_kv_heads, head_dim,
+                                 block_size, max_blocks_per_seq, num_blocks, scale, dtype,
+                                 k_scale, v_scale);
+    }
+    return status;
 }

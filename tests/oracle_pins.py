@@ -305,4 +305,80 @@ def pin_rows_match_full(lib):
     assert np.array_equal(got, full[rows[:, 0], rows[:, 1]])
 
 
+# ---- FP8 (e4m3) caches ------------------------------------------------------
+
+def _torch_e4m3():
+    import torch
+    return torch
+
+
+def pin_e4m3_decode_all_codes(lib):
+    """Every e4m3 code decodes to torch.float8_e4m3fn's value."""
+    torch = _torch_e4m3()
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(oracle.decode_e4m3(codes, lib=lib), ref, equal_nan=True)
+
+
+def pin_e4m3_encode_rounding(lib):
+    """fp32 -> e4m3 rounds to nearest, ties to even (torch.float8_e4m3fn for
+    in-range values, including every exact midpoint); saturates at +-448;
+    keeps the sign of zero; NaN -> 0x7F."""
+    torch = _torch_e4m3()
+    codes = np.arange(0, 0x7f, dtype=np.uint8)                 # finite non-negative codes
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mids = (vals[:-1] + vals[1:]) / 2
+    rng = np.random.Generator(np.random.PCG64(8))
+    x = np.concatenate([vals, mids, rng.uniform(-447, 447, 4000), rng.normal(0, 0.01, 2000)])
+    x = np.concatenate([x, -x]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.encode_e4m3(x, lib=lib), ref)
+    sat = np.array([448.0, 449.0, 1e6, -500.0, np.inf, -np.inf, np.nan, -0.0, 0.0], np.float32)
+    assert oracle.encode_e4m3(sat, lib=lib).tolist() == [0x7e, 0x7e, 0x7e, 0xfe, 0x7e, 0xfe,
+                                                         0x7f, 0x80, 0x00]
+
+
+def pin_fp8_cache_write(lib):
+    """The quantising write stores e4m3(fp32(x) * fp32(1/scale)) at the slot's
+    offset; other bytes unchanged."""
+    rng = np.random.Generator(np.random.PCG64(9))
+    nb, b, h, d = 6, 4, 2, 8
+    kc = np.full((nb, b, h, d), 0x7f, np.uint8)
+    vc = np.full((nb, b, h, d), 0x7f, np.uint8)
+    key = gen.normal_bits(rng, (3, h, d), "f16")
+    val = gen.normal_bits(rng, (3, h, d), "f16")
+    slots = np.array([5, -1, 17])
+    st = oracle.reshape_and_cache_fp8(key, val, kc, vc, slots, b, "f16", 0.05, 0.03, lib=lib)
+    assert st == 0
+    inv_k, inv_v = np.float32(1) / np.float32(0.05), np.float32(1) / np.float32(0.03)
+    for t, sl in ((0, 5), (2, 17)):
+        kx = key[t].view(np.float16).astype(np.float32) * inv_k
+        vx = val[t].view(np.float16).astype(np.float32) * inv_v
+        assert np.array_equal(kc[sl // b, sl % b], oracle.encode_e4m3(kx, lib=lib))
+        assert np.array_equal(vc[sl // b, sl % b], oracle.encode_e4m3(vx, lib=lib))
+    touched = np.zeros((nb, b), bool)
+    touched[1, 1] = touched[4, 1] = True
+    assert np.all(kc[~touched] == 0x7f) and np.all(vc[~touched] == 0x7f)
+
+
+def pin_fp8_decode_equals_dequantised_fp16(lib):
+    """With power-of-two scales the dequantised cache is exact in fp16, so the
+    fp8 decode must equal the (pinned) fp16 decode of the dequantised pools."""
+    rng = np.random.Generator(np.random.PCG64(10))
+    wl = small_gqa(dtype="f16")
+    codes_k = rng.integers(0, 256, size=wl.k_cache.shape).astype(np.uint8)
+    codes_v = rng.integers(0, 256, size=wl.v_cache.shape).astype(np.uint8)
+    for c in (codes_k, codes_v):
+        c[(c & 0x7f) == 0x7f] = 0x3c                            # no NaN codes
+    ks, vs = 0.25, 0.5
+    deq_k = (oracle.decode_e4m3(codes_k, lib=lib) * ks).astype(np.float16).view(np.uint16)
+    deq_v = (oracle.decode_e4m3(codes_v, lib=lib) * vs).astype(np.float16).view(np.uint16)
+    a, sa = oracle.paged_decode_fp8(wl.query, codes_k, codes_v, wl.block_tables, wl.context_lens,
+                                    wl.scale, "f16", ks, vs, lib=lib)
+    b, sb = oracle.paged_decode(wl.query, deq_k, deq_v, wl.block_tables, wl.context_lens,
+                                wl.scale, "f16", lib=lib)
+    assert sa == sb == 0
+    assert np.array_equal(a, b)
+
+
 PINS = {name: fn for name, fn in globals().items() if name.startswith("pin_")}

@@ -32,6 +32,14 @@ MUTANTS = {
                                "int64_t offset = (slot + 1) % block_size;"),
     "table_row_stride": ("block_tables + (int64_t)s * max_blocks_per_seq",
                          "block_tables + (int64_t)s * (max_blocks_per_seq - 1)"),
+    "e4m3_exponent_bias": ("ldexp((double)(frac + 8), expo - 10)",
+                           "ldexp((double)(frac + 8), expo - 9)"),
+    "e4m3_ties_away": ("else pick = (lo & 1) ? hi : lo;", "else pick = hi;"),
+    "e4m3_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7e);",
+                           "if (a >= 448.0) return (uint8_t)(sign | 0x7f);"),
+    "fp8_scale_dropped": ("(e4m3_to_f64(k_cache[r + d]) * k_scale)",
+                          "(e4m3_to_f64(k_cache[r + d]))"),
+    "fp8_write_divides_twice": ("const float kq = kx * k_inv;", "const float kq = kx * k_inv * k_inv;"),
 }
 
 
