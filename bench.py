@@ -44,6 +44,8 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_GLOB_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["paged_kv_cache_415_b200/csrc/paged_decode.cu",
+                  "paged_kv_cache_415_b200/csrc/paged_decode_mma.cuh",
+                  "paged_kv_cache_415_b200/csrc/paged_decode_fp8.cuh",
                   "paged_kv_cache_415_b200/csrc/pa_common.cuh"]
 NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -69,6 +71,9 @@ def parse_args():
     ap.add_argument("--shared-prefix", action="store_true",
                     help="beam_search: decode with pa_paged_decode_shared_prefix (shared "
                          "prompt blocks read once per group)")
+    ap.add_argument("--kv-dtype", default="auto", choices=["auto", "fp8"],
+                    help="fp8: the same workload with e4m3 K/V pools (per-pool scales), "
+                         "quantising cache write + e4m3 decode")
     ap.add_argument("--seqs", type=int, default=0,
                     help="shrink the batch (and the pool) for profiling; 0 = the full workload")
     return ap.parse_args()
@@ -182,9 +187,18 @@ def whole_job_gbs(bytes_per_step: int, steps: int, world: int, max_elapsed_ms: f
     return world * bytes_per_step * steps / (max_elapsed_ms * 1e-3) / 1e9
 
 
-def make_workload(config: str, seqs: int = 0):
+def make_workload(config: str, seqs: int = 0, kv_dtype: str = "auto"):
     """The named workload; with seqs > 0 a smaller batch of the same shape
-    and a pool sized to it (profiling captures stay a few GB)."""
+    and a pool sized to it (profiling captures stay a few GB); kv_dtype fp8
+    redraws its pools as e4m3 codes."""
+    from workloads import generators as gen
+    wl = _make_workload(config, seqs)
+    if kv_dtype == "fp8":
+        wl = gen.with_fp8_pools(wl, seed=gen.SEED_BASE + 50)
+    return wl
+
+
+def _make_workload(config: str, seqs: int = 0):
     from workloads import generators as gen
     if seqs <= 0:
         return gen.CONFIGS[config]()
@@ -200,8 +214,9 @@ def make_workload(config: str, seqs: int = 0):
 
 
 def workload_config(wl, partition_size, l2_note):
+    kv = ", e4m3 K/V pools" if wl.extra.get("kv_dtype") == "fp8" else ""
     return {"workload": f"{wl.name}: {wl.num_seqs} seqs, {wl.num_q_heads}/{wl.num_kv_heads} heads, "
-                        f"head_dim {wl.head_dim}, block {wl.block_size}, {wl.dtype}, "
+                        f"head_dim {wl.head_dim}, block {wl.block_size}, {wl.dtype}{kv}, "
                         f"contexts {int(wl.context_lens.min())}..{int(wl.context_lens.max())} "
                         f"(sum {int(wl.context_lens.sum())}), pool {wl.num_blocks} blocks, "
                         f"{wl.num_new_tokens} new tokens, {int(wl.block_mapping.shape[0])} block copies",
@@ -230,7 +245,8 @@ class OracleStep:
         self.q = np.ascontiguousarray(wl.query[:n])
         self.kc, self.vc = wl.k_cache.copy(), wl.v_cache.copy()
         att = bm.decode_bytes(self.ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
-                              wl.block_size, 2)
+                              wl.block_size, 2, bm.kv_elem_bytes(wl))
+        self.fp8 = wl.extra.get("kv_dtype") == "fp8"
         full = bm.step_bytes(wl)
         self.bytes = att["total"] + full["append"] + full["copy"]
         self.threads = oracle.max_threads()
@@ -240,6 +256,14 @@ class OracleStep:
         t0 = time.perf_counter()
         if wl.block_mapping.shape[0]:
             o.copy_blocks(self.kc, self.vc, wl.block_mapping)
+        if self.fp8:
+            ks, vs = wl.extra["k_scale"], wl.extra["v_scale"]
+            if wl.num_new_tokens:
+                o.reshape_and_cache_fp8(wl.new_key, wl.new_value, self.kc, self.vc,
+                                        wl.slot_mapping, wl.block_size, wl.dtype, ks, vs)
+            o.paged_decode_fp8(self.q, self.kc, self.vc, self.tables, self.ctx, wl.scale,
+                               wl.dtype, ks, vs)
+            return time.perf_counter() - t0
         if wl.num_new_tokens:
             o.reshape_and_cache(wl.new_key, wl.new_value, self.kc, self.vc, wl.slot_mapping,
                                 wl.block_size)
@@ -268,7 +292,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    wl = make_workload(args.config, args.seqs)
+    wl = make_workload(args.config, args.seqs, args.kv_dtype)
     # size the per-step sample so warm-up + timed steps end within ~2 minutes
     probe = OracleStep(wl, max_seqs=max(1, wl.num_seqs // 8))
     per_seq = probe.run() / probe.n
@@ -315,14 +339,20 @@ def run_ours(args):
     from paged_kv_cache_415_b200 import binding as B
     from workloads import byte_model as bm
 
-    wl = make_workload(args.config, args.seqs)
+    wl = make_workload(args.config, args.seqs, args.kv_dtype)
     dev = torch.device("cuda", local)
     tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
+    fp8 = wl.extra.get("kv_dtype") == "fp8"
+    k_scale, v_scale = wl.extra.get("k_scale", 1.0), wl.extra.get("v_scale", 1.0)
 
     def up(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(tdt)
 
-    k_cache, v_cache = up(wl.k_cache), up(wl.v_cache)
+    if fp8:
+        k_cache = torch.from_numpy(wl.k_cache).to(dev)
+        v_cache = torch.from_numpy(wl.v_cache).to(dev)
+    else:
+        k_cache, v_cache = up(wl.k_cache), up(wl.v_cache)
     query = up(wl.query)
     new_key, new_value = up(wl.new_key), up(wl.new_value)
     slot_mapping = torch.from_numpy(wl.slot_mapping).to(dev)
@@ -342,17 +372,20 @@ def run_ours(args):
     n_pairs = int(wl.block_mapping.shape[0])
     stream = torch.cuda.current_stream(dev)
 
-    fused = (not args.separate and not args.shared_prefix
+    fused = (not args.separate and not args.shared_prefix and not fp8
              and wl.extra.get("one_token_per_seq", False) and wl.num_new_tokens == wl.num_seqs)
 
     def cache_ops():
         if n_pairs:
             B.pa_copy_blocks(k_cache, v_cache, block_mapping, d_status, stream)
-        if wl.num_new_tokens and not fused:
+        if wl.num_new_tokens and fp8:
+            B.pa_reshape_and_cache_fp8(new_key, new_value, k_cache, v_cache, slot_mapping,
+                                       k_scale, v_scale, d_status, stream)
+        elif wl.num_new_tokens and not fused:
             B.pa_reshape_and_cache(new_key, new_value, k_cache, v_cache, slot_mapping, d_status,
                                    stream)
 
-    shared = args.shared_prefix and "prefix_lens" in wl.extra
+    shared = args.shared_prefix and "prefix_lens" in wl.extra and not fp8
     if shared:
         group_size = int(wl.extra["group_size"])
         prefix_lens = torch.from_numpy(wl.extra["prefix_lens"]).to(dev)
@@ -363,7 +396,10 @@ def run_ours(args):
         workspace = torch.empty(max(sws, 16), dtype=torch.uint8, device=dev)
 
     def decode():
-        if fused:
+        if fp8:
+            B.pa_paged_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, mcl,
+                                  wl.scale, k_scale, v_scale, part, workspace, d_status, stream)
+        elif fused:
             B.pa_paged_decode_append(out, query, new_key, new_value, k_cache, v_cache,
                                      block_tables, context_lens, mcl, wl.scale, part, workspace,
                                      d_status, stream)
@@ -412,7 +448,8 @@ def run_ours(args):
 
     # end to end through the public API: pinned host inputs -> device -> step -> host output
     from paged_kv_cache_415_b200.step import DecodeStep
-    stepper = DecodeStep(k_cache, v_cache, wl.num_seqs, wl.num_q_heads, mcl, part)
+    stepper = DecodeStep(k_cache, v_cache, wl.num_seqs, wl.num_q_heads, mcl, part, k_scale,
+                         v_scale)
     host = {"query": torch.from_numpy(wl.query.view(np.int16)).view(tdt).pin_memory(),
             "block_tables": torch.from_numpy(wl.block_tables).pin_memory(),
             "context_lens": torch.from_numpy(wl.context_lens).pin_memory(),
@@ -456,7 +493,7 @@ def run_ours(args):
     # the decode launch also carries the step's cache write when it is fused
     decode_bytes = step["attention"] + (step["append"] if fused else 0)
     achieved = decode_bytes / (decode_avg * 1e-3) / 1e9
-    traffic = profiled_traffic(args.config)
+    traffic = profiled_traffic(args.config + ("-fp8" if fp8 else ""))
     clocks = sampler.summary()
 
     cpu = None
@@ -473,7 +510,8 @@ def run_ours(args):
     if shared:
         kernel_name = "paged_decode_shared_kernel + paged_decode_shared_reduce_kernel"
     else:
-        kernel_name = ("paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
+        kernel_name = ("paged_decode_fp8_kernel" if fp8 else
+                       "paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
                        else "paged_decode_kernel")
         if max_parts > 1:
             kernel_name += " + paged_decode_reduce_kernel"
@@ -482,7 +520,8 @@ def run_ours(args):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 (e4m3 K/V)" if fp8 else wl.dtype,
         "data": "synthetic", "config": workload_config(wl, part, l2),
         "us_per_layer_step": round(per_step_ms * 1e3, 2),
         "kv_tokens_per_s": round(world * int(wl.context_lens.sum()) * args.steps / (elapsed_ms * 1e-3)),
@@ -498,7 +537,8 @@ def run_ours(args):
         "clocks": clocks,
         "cpu_baseline": cpu,
         "bytes_per_step": step,
-        "decode_entry": ("pa_paged_decode_shared_prefix" if shared else
+        "decode_entry": ("pa_reshape_and_cache_fp8 + pa_paged_decode_fp8" if fp8 else
+                         "pa_paged_decode_shared_prefix" if shared else
                          "pa_paged_decode_append (cache write fused)" if fused else
                          "pa_reshape_and_cache + pa_paged_decode"),
     }

@@ -95,7 +95,8 @@ typedef enum pa_status {
 
 typedef enum pa_dtype {
     PA_DTYPE_F16 = 0,
-    PA_DTYPE_BF16 = 1
+    PA_DTYPE_BF16 = 1,
+    PA_DTYPE_FP8_E4M3 = 2   /* cache pools only: pa_copy_blocks and the *_fp8 calls */
 } pa_dtype;
 
 #define PA_STATUS_BAD_BLOCK 1
@@ -259,6 +260,49 @@ PA_API pa_status pa_paged_decode_append(void* out, const void* query, const void
                                         int32_t partition_size, void* workspace,
                                         size_t workspace_bytes, pa_dtype dtype,
                                         int32_t* d_status, pa_stream_t stream);
+
+/*
+ * FP8 KV cache -- pools of e4m3 codes (1 byte per element, OCP e4m3fn: no
+ * infinities, largest finite 448) with one scale per pool: the cached value
+ * of code c is decode(c) * k_scale (or v_scale).  Halves the bytes a decode
+ * step moves.  Defined by: [Practice §7 演进方向与优化空间] (FP8/INT8 storage of
+ * history blocks) and [VM-paging, PagedAttention的工程实践与局限] (low-precision
+ * storage of the KV values in blocks); the scale-per-tensor form is this
+ * library's reading.  Layout and slots as the 16-bit pools.  pa_copy_blocks
+ * copies such pools with dtype PA_DTYPE_FP8_E4M3.
+ *
+ * pa_reshape_and_cache_fp8 -- the cache write, quantising:
+ *   code = e4m3(fp32(x) * fp32(1 / scale)), round to nearest even,
+ *   saturating at +-448 (NaN stays NaN).
+ * key, value     [num_tokens][num_kv_heads][head_dim] of `dtype` (F16/BF16).
+ * k_scale, v_scale  positive finite (else PA_ERR_INVALID_ARG).
+ * Other arguments and errors as pa_reshape_and_cache.
+ */
+PA_API pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                          void* v_cache, const int64_t* slot_mapping,
+                                          int32_t num_tokens, int32_t num_kv_heads,
+                                          int32_t head_dim, int32_t block_size,
+                                          int64_t num_blocks, pa_dtype dtype, float k_scale,
+                                          float v_scale, int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_paged_decode_fp8 -- pa_paged_decode over FP8 pools.  query and out are
+ * of `dtype` (F16/BF16); K and V are dequantised exactly (e4m3 values are
+ * fp16 values) and the contractions run on fp16 tensor cores with fp32
+ * accumulation, so a bf16 query is rounded to fp16 first (exact in its
+ * normal range).  block_size 16 or 32 (else PA_ERR_UNSUPPORTED).  The
+ * workspace is sized by pa_paged_decode_workspace_size.  Other arguments,
+ * results and errors as pa_paged_decode.
+ */
+PA_API pa_status pa_paged_decode_fp8(void* out, const void* query, const void* k_cache,
+                                     const void* v_cache, const int32_t* block_tables,
+                                     const int32_t* context_lens, int32_t num_seqs,
+                                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int32_t max_blocks_per_seq,
+                                     int64_t num_blocks, int32_t max_context_len, float scale,
+                                     float k_scale, float v_scale, int32_t partition_size,
+                                     void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                                     int32_t* d_status, pa_stream_t stream);
 
 /*
  * pa_paged_decode_shared_prefix -- pa_paged_decode for batches whose

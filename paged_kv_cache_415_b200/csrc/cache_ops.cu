@@ -9,7 +9,9 @@
 //   [VM-paging] "vLLM用虚拟内存分页思想管理KV Cache"
 //   [Practice]  "PagedAttention：大模型KV Cache分页管理优化实践"
 //   [Manager]   "深入解析 vLLM 的 KV Cache 管理器：从内存碎片到 PagedAttention 的完整技术剖析"
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include "pa.h"
@@ -67,6 +69,56 @@ __global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_kernel(
     }
 }
 
+// Quantising variant for e4m3 pools: each vector of 8 input elements
+// becomes 8 codes, e4m3(fp32(x) * inv_scale) rounded to nearest even and
+// saturated at +-448.
+template <typename T>
+__global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_fp8_kernel(
+    const uint4* __restrict__ key, const uint4* __restrict__ value, uint2* __restrict__ k_cache,
+    uint2* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int32_t row_vecs,
+    int64_t num_slots, float k_inv, float v_inv, int32_t* d_status)
+{
+    grid_dependency_wait();
+    allow_dependents();
+    const int64_t t = blockIdx.x;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) status_or(d_status, PA_STATUS_BAD_SLOT);
+        return;
+    }
+    auto quant8 = [](const uint4& w, float inv) -> uint2 {
+        float f[8];
+        unpack8<T>(w, f);
+        uint32_t r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
+                make_float2(f[2 * j] * inv, f[2 * j + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+            r[j] = static_cast<uint32_t>(c);
+        }
+        return make_uint2(r[0] | (r[1] << 16), r[2] | (r[3] << 16));
+    };
+    const int32_t base = blockIdx.y * kCacheThreads * kCacheVecsPerThread + threadIdx.x;
+    uint4 a[kCacheVecsPerThread], b[kCacheVecsPerThread];
+#pragma unroll
+    for (int j = 0; j < kCacheVecsPerThread; ++j) {
+        const int32_t i = base + j * kCacheThreads;
+        if (i < row_vecs) {
+            a[j] = ld_nc_v4(key + t * row_vecs + i);
+            b[j] = ld_nc_v4(value + t * row_vecs + i);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kCacheVecsPerThread; ++j) {
+        const int32_t i = base + j * kCacheThreads;
+        if (i < row_vecs) {
+            k_cache[slot * row_vecs + i] = quant8(a[j], k_inv);
+            v_cache[slot * row_vecs + i] = quant8(b[j], v_inv);
+        }
+    }
+}
+
 // Grid (pair, K-or-V, chunk of the block).  Whole-block bit copy src -> dst
 // ([VM-paging, 写时复制与块共享机制]; [Practice §4.1 共享内存管理] step 2).
 // The first CTA of each pair also checks the pair against all the others:
@@ -117,11 +169,12 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
 }
 
 static pa_status check_pool_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                                  int64_t num_blocks, int32_t dtype)
+                                  int64_t num_blocks, int32_t dtype, bool allow_fp8 = false)
 {
     if (num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
         return PA_ERR_INVALID_ARG;
-    if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !supported_dtype(dtype))
+    const bool dtype_ok = supported_dtype(dtype) || (allow_fp8 && dtype == PA_DTYPE_FP8_E4M3);
+    if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !dtype_ok)
         return PA_ERR_UNSUPPORTED;
     return PA_OK;
 }
@@ -162,14 +215,16 @@ extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t*
 {
     using namespace pa;
     if (num_pairs < 0) return PA_ERR_INVALID_ARG;
-    pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype, true);
     if (st != PA_OK) return st;
     if (!k_cache || !v_cache || !block_mapping) return PA_ERR_INVALID_ARG;
     if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned8(block_mapping) ||
         (d_status && !aligned4(d_status)))
         return PA_ERR_INVALID_ARG;
     if (num_pairs == 0) return PA_OK;
-    const int64_t block_vecs = static_cast<int64_t>(block_size) * num_kv_heads * head_dim * 2 / 16;
+    const int elem_bytes = dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2;
+    const int64_t block_vecs =
+        static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes / 16;
     const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kCopyVecsPerThread;
     const int64_t chunks = (block_vecs + per_cta - 1) / per_cta;
     if (chunks > 65535) return PA_ERR_UNSUPPORTED;
@@ -177,4 +232,42 @@ extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t*
     return launch_overlapped(copy_blocks_kernel, grid, dim3(kCopyThreads), 0, stream,
                              static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
                              block_mapping, num_pairs, block_vecs, num_blocks, d_status);
+}
+
+extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                              void* v_cache, const int64_t* slot_mapping,
+                                              int32_t num_tokens, int32_t num_kv_heads,
+                                              int32_t head_dim, int32_t block_size,
+                                              int64_t num_blocks, pa_dtype dtype, float k_scale,
+                                              float v_scale, int32_t* d_status,
+                                              pa_stream_t stream)
+{
+    using namespace pa;
+    if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+    pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale))
+        return PA_ERR_INVALID_ARG;
+    if (!key || !value || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned8(slot_mapping) || (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    const int32_t row_vecs = num_kv_heads * head_dim / 8;
+    const int32_t per_cta = kCacheThreads * kCacheVecsPerThread;
+    const int32_t chunks = (row_vecs + per_cta - 1) / per_cta;
+    if (chunks > 65535) return PA_ERR_UNSUPPORTED;
+    dim3 grid(num_tokens, chunks);
+    const float k_inv = 1.0f / k_scale, v_inv = 1.0f / v_scale;
+    if (dtype == PA_DTYPE_F16)
+        return launch_overlapped(reshape_and_cache_fp8_kernel<__half>, grid, dim3(kCacheThreads), 0,
+                                 stream, static_cast<const uint4*>(key),
+                                 static_cast<const uint4*>(value), static_cast<uint2*>(k_cache),
+                                 static_cast<uint2*>(v_cache), slot_mapping, row_vecs,
+                                 num_blocks * block_size, k_inv, v_inv, d_status);
+    return launch_overlapped(reshape_and_cache_fp8_kernel<__nv_bfloat16>, grid,
+                             dim3(kCacheThreads), 0, stream, static_cast<const uint4*>(key),
+                             static_cast<const uint4*>(value), static_cast<uint2*>(k_cache),
+                             static_cast<uint2*>(v_cache), slot_mapping, row_vecs,
+                             num_blocks * block_size, k_inv, v_inv, d_status);
 }

@@ -36,6 +36,7 @@
 // The whole computation has a fixed summation order, so results are
 // deterministic and do not depend on where the blocks sit in the pool.
 #include <cuda.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -522,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
 
 #include "paged_decode_mma.cuh"
 #include "paged_decode_shared.cuh"
+#include "paged_decode_fp8.cuh"
 
 namespace pa {
 
@@ -681,6 +683,79 @@ static bool encode_pool_map_swizzled(CUtensorMap* map, const void* pool, int32_t
                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return res == CUDA_SUCCESS;
+}
+
+// An e4m3 pool [num_blocks][B][Hkv][D] of bytes as a 4-D tensor whose box is
+// one block of one kv head (B rows of D bytes, dense in shared memory).
+static bool encode_pool_map_fp8(CUtensorMap* map, const void* pool, int32_t head_dim,
+                                int32_t num_kv_heads, int32_t block_size, int64_t num_blocks)
+{
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim),
+                                static_cast<cuuint64_t>(num_kv_heads),
+                                static_cast<cuuint64_t>(block_size),
+                                static_cast<cuuint64_t>(num_blocks)};
+    const cuuint64_t row = static_cast<cuuint64_t>(head_dim);
+    const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(head_dim), 1u,
+                               static_cast<cuuint32_t>(block_size), 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(pool), dims,
+                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return res == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int BS, int G>
+static pa_status launch_decode_fp8(const DecodeArgs& a, float v_scale)
+{
+    using S = Fp8Shape<D, BS, G>;
+    static std::atomic<uint64_t> attr_done{0};
+    auto kernel = paged_decode_fp8_kernel<T, D, BS, G>;
+    if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
+    CUtensorMap tm_k, tm_v;
+    if (!encode_pool_map_fp8(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
+        !encode_pool_map_fp8(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
+        return PA_ERR_CUDA;
+    dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
+    pa_status st = launch_overlapped(
+        kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v, static_cast<T*>(a.out),
+        static_cast<const T*>(a.query), a.block_tables, a.context_lens, a.num_q_heads,
+        a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2, v_scale,
+        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+    if (st != PA_OK || a.max_parts <= 1) return st;
+    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
+    const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
+    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(ctas),
+                             dim3(kReduceRowsPerCta * 32), 0, a.stream, static_cast<T*>(a.out),
+                             a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
+                             a.max_context_len, a.max_blocks_per_seq, a.block_size,
+                             a.partition_size, a.max_parts);
+}
+
+template <typename T, int D, int BS>
+static pa_status dispatch_fp8_group(const DecodeArgs& a, float v_scale)
+{
+    switch (a.num_q_heads / a.num_kv_heads) {
+    case 1: return launch_decode_fp8<T, D, BS, 1>(a, v_scale);
+    case 2: return launch_decode_fp8<T, D, BS, 2>(a, v_scale);
+    case 4: return launch_decode_fp8<T, D, BS, 4>(a, v_scale);
+    case 8: return launch_decode_fp8<T, D, BS, 8>(a, v_scale);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
+template <typename T>
+static pa_status dispatch_fp8(const DecodeArgs& a, float v_scale)
+{
+    const int32_t d = a.head_dim, b = a.block_size;
+    if (d == 64 && b == 16) return dispatch_fp8_group<T, 64, 16>(a, v_scale);
+    if (d == 64 && b == 32) return dispatch_fp8_group<T, 64, 32>(a, v_scale);
+    if (d == 128 && b == 16) return dispatch_fp8_group<T, 128, 16>(a, v_scale);
+    if (d == 128 && b == 32) return dispatch_fp8_group<T, 128, 32>(a, v_scale);
+    return PA_ERR_UNSUPPORTED;
 }
 
 template <typename T, int D, int BS, int G>
@@ -917,7 +992,8 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
                              int64_t num_blocks, int32_t max_context_len, float scale,
                              int32_t partition_size, void* workspace, size_t workspace_bytes,
                              pa_dtype dtype, int32_t* d_status, pa_stream_t stream,
-                             const void* new_key, const void* new_value)
+                             const void* new_key, const void* new_value, bool fp8 = false,
+                             float k_scale = 1.f, float v_scale = 1.f)
 {
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       max_context_len, partition_size);
@@ -932,6 +1008,11 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     if (new_key != nullptr &&
         (new_value == nullptr || !aligned16(new_key) || !aligned16(new_value)))
         return PA_ERR_INVALID_ARG;
+    if (fp8) {
+        if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale))
+            return PA_ERR_INVALID_ARG;
+        if (block_size % 16 != 0) return PA_ERR_UNSUPPORTED;
+    }
     const int32_t partition = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
                                                partition_size);
     const int32_t max_parts = parts_for(max_context_len, partition);
@@ -956,7 +1037,8 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.num_blocks = num_blocks;
     a.max_context_len = max_context_len;
-    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * (fp8 ? k_scale : 1.0) *
+                                      1.4426950408889634);
     a.partition_size = partition;
     a.max_parts = max_parts;
     const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * max_parts;
@@ -968,6 +1050,9 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.stream = stream;
     a.new_key = new_key;
     a.new_value = new_value;
+    if (fp8)
+        return dtype == PA_DTYPE_F16 ? dispatch_fp8<__half>(a, v_scale)
+                                     : dispatch_fp8<__nv_bfloat16>(a, v_scale);
     return dtype == PA_DTYPE_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
 }
 
@@ -987,6 +1072,24 @@ extern "C" pa_status pa_paged_decode(void* out, const void* query, const void* k
                            num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                            num_blocks, max_context_len, scale, partition_size, workspace,
                            workspace_bytes, dtype, d_status, stream, nullptr, nullptr);
+}
+
+extern "C" pa_status pa_paged_decode_fp8(void* out, const void* query, const void* k_cache,
+                                         const void* v_cache, const int32_t* block_tables,
+                                         const int32_t* context_lens, int32_t num_seqs,
+                                         int32_t num_q_heads, int32_t num_kv_heads,
+                                         int32_t head_dim, int32_t block_size,
+                                         int32_t max_blocks_per_seq, int64_t num_blocks,
+                                         int32_t max_context_len, float scale, float k_scale,
+                                         float v_scale, int32_t partition_size, void* workspace,
+                                         size_t workspace_bytes, pa_dtype dtype,
+                                         int32_t* d_status, pa_stream_t stream)
+{
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, nullptr, nullptr, true,
+                           k_scale, v_scale);
 }
 
 extern "C" pa_status pa_paged_decode_append(void* out, const void* query, const void* key,

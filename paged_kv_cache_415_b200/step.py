@@ -7,7 +7,8 @@
 
 ``DecodeStep`` owns the scratch the step needs (the split-context workspace
 and a device status word), allocated once with torch, and issues the three
-C-ABI calls on one stream.  ``run_from_host`` is the same step fed from
+C-ABI calls on one stream.  Pools of dtype uint8 hold e4m3 codes: the step
+then uses the quantising write and the e4m3 decode with the pools' scales.  ``run_from_host`` is the same step fed from
 pinned host buffers: it copies the step's inputs to the device, runs the
 step and copies the output back, all on the same stream.
 """
@@ -20,8 +21,11 @@ from . import binding as B
 
 class DecodeStep:
     def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor, num_seqs: int,
-                 num_q_heads: int, max_context_len: int, partition_size: int = 0):
+                 num_q_heads: int, max_context_len: int, partition_size: int = 0,
+                 k_scale: float = 1.0, v_scale: float = 1.0):
         self.k_cache, self.v_cache = k_cache, v_cache
+        self.fp8 = k_cache.dtype == torch.uint8
+        self.k_scale, self.v_scale = float(k_scale), float(v_scale)
         num_blocks, self.block_size, self.num_kv_heads, self.head_dim = k_cache.shape
         self.num_blocks = num_blocks
         self.num_seqs, self.num_q_heads = num_seqs, num_q_heads
@@ -50,6 +54,17 @@ class DecodeStep:
         if out is None:
             out = torch.empty_like(query)
         mcl = self.max_context_len if max_context_len is None else max_context_len
+        if self.fp8:
+            if fused_append:
+                raise B.PAError("pa_paged_decode_append", B.PA_ERR_UNSUPPORTED)
+            if slot_mapping is not None and slot_mapping.shape[0] > 0:
+                B.pa_reshape_and_cache_fp8(new_key, new_value, self.k_cache, self.v_cache,
+                                           slot_mapping, self.k_scale, self.v_scale,
+                                           self.d_status, stream)
+            B.pa_paged_decode_fp8(out, query, self.k_cache, self.v_cache, block_tables,
+                                  context_lens, mcl, scale, self.k_scale, self.v_scale,
+                                  self.partition_size, self.workspace, self.d_status, stream)
+            return out
         if fused_append:
             B.pa_paged_decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache,
                                      block_tables, context_lens, mcl, scale, self.partition_size,

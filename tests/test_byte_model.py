@@ -75,3 +75,32 @@ def test_unique_bytes_of_shared_prefixes():
     n_new = int(wl.extra["n_new"].sum())
     copies = wl.block_mapping.shape[0]
     assert uniq == (2 * 40 + n_new + copies * (40 % 16)) * row
+
+
+def test_fp8_step_bytes_by_hand():
+    """e4m3 pools: one byte per cached element; the appended rows are read in
+    the 16-bit type and written as codes."""
+    wl = gen.make_decode("b", seed=1, dtype="f16", context_lens=[17, 16], num_q_heads=4,
+                         num_kv_heads=2, head_dim=8, block_size=16, num_blocks=8, scale=0.5)
+    w8 = gen.with_fp8_pools(wl, seed=2)
+    a, b = bm.step_bytes(wl), bm.step_bytes(w8)
+    assert b["kv"] * 2 == a["kv"] == (17 + 16) * 2 * 8 * 2 * 2
+    assert b["append"] == 2 * 2 * 16 * 2 + 2 * 2 * 16 + 8 * 2
+    assert a["attention"] - b["attention"] == a["kv"] - b["kv"]
+
+
+def test_fp8_pools_mark_every_unheld_slot():
+    """with_fp8_pools: history slots hold finite codes, every other slot
+    (free blocks, block tails, this step's new slots) the NaN code."""
+    wl = gen.make_decode("b", seed=3, dtype="bf16", context_lens=[1, 33, 20], num_q_heads=2,
+                         num_kv_heads=2, head_dim=16, block_size=16, num_blocks=12, scale=0.25)
+    w8 = gen.with_fp8_pools(wl, seed=4)
+    for pool in (w8.k_cache, w8.v_cache):
+        assert pool.dtype == np.uint8
+        held = np.zeros(pool.shape[:2], bool)
+        for s, c in enumerate(w8.context_lens):
+            for pos in range(int(c) - 1):
+                held[w8.block_tables[s, pos // 16], pos % 16] = True
+        assert np.all((pool[held] & 0x7F) != 0x7F)
+        assert np.all(pool[~held] == 0x7F)
+        assert ((pool[held] >> 3) & 0xF).max() <= 14

@@ -1,0 +1,258 @@
+"""FP8 (e4m3) K/V pools on the GPU against the oracle.
+
+The quantising cache write is compared bit for bit with the oracle over the
+whole pool (every untouched byte included).  Decode over e4m3 pools is
+compared with the fp64 oracle of the dequantised pools at the tolerance of
+the 16-bit path, |gpu - oracle| <= 2e-3 + 1e-2 |oracle|: the codes widen to
+fp16 exactly, so the only extra rounding is the query's to fp16 (exact for
+fp16 queries; for bf16 ones it only touches values below 2^-14) next to the
+probabilities' rounding that the 16-bit tensor-core path has already."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import oracle_pins
+from tests.gpu_utils import assert_close, to_dev, to_f64
+from workloads import generators as gen
+
+pytestmark = pytest.mark.gpu
+
+
+def _u8(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+
+class Fp8Device:
+    """A with_fp8_pools workload on the device; step = write, then decode."""
+
+    def __init__(self, wl):
+        self.wl = wl
+        self.query = to_dev(wl.query, wl.dtype)
+        self.k_cache, self.v_cache = _u8(wl.k_cache), _u8(wl.v_cache)
+        self.block_tables = torch.from_numpy(wl.block_tables).cuda()
+        self.context_lens = torch.from_numpy(wl.context_lens).cuda()
+        self.new_key = to_dev(wl.new_key, wl.dtype)
+        self.new_value = to_dev(wl.new_value, wl.dtype)
+        self.slot_mapping = torch.from_numpy(wl.slot_mapping).cuda()
+        self.d_status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.ks, self.vs = wl.extra["k_scale"], wl.extra["v_scale"]
+
+    def write(self):
+        from paged_kv_cache_415_b200 import binding as B
+        B.pa_reshape_and_cache_fp8(self.new_key, self.new_value, self.k_cache, self.v_cache,
+                                   self.slot_mapping, self.ks, self.vs, self.d_status)
+
+    def decode(self, partition_size=None, block_tables=None, context_lens=None,
+               max_context_len=None):
+        from paged_kv_cache_415_b200 import binding as B
+        wl = self.wl
+        p = wl.partition_size if partition_size is None else partition_size
+        bt = self.block_tables if block_tables is None else block_tables
+        cl = self.context_lens if context_lens is None else context_lens
+        mcl = wl.max_context_len if max_context_len is None else max_context_len
+        ws_bytes = B.pa_paged_decode_workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                                    wl.head_dim, wl.block_size, mcl, p)
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+        out = torch.full_like(self.query, float("nan"))
+        B.pa_paged_decode_fp8(out, self.query, self.k_cache, self.v_cache, bt, cl, mcl, wl.scale,
+                              self.ks, self.vs, p, ws, self.d_status)
+        return out
+
+    def status(self) -> int:
+        return int(self.d_status.item())
+
+
+def _oracle_pools(wl):
+    kc, vc = wl.k_cache.copy(), wl.v_cache.copy()
+    st = oracle.reshape_and_cache_fp8(wl.new_key, wl.new_value, kc, vc, wl.slot_mapping,
+                                      wl.block_size, wl.dtype, wl.extra["k_scale"],
+                                      wl.extra["v_scale"])
+    return kc, vc, st
+
+
+def _parity(wl, partition_size=None, what=""):
+    dev = Fp8Device(wl)
+    dev.write()
+    out = dev.decode(partition_size)
+    torch.cuda.synchronize()
+    kc, vc, st = _oracle_pools(wl)
+    assert st == 0
+    assert np.array_equal(dev.k_cache.cpu().numpy(), kc), f"{what}: K pool"
+    assert np.array_equal(dev.v_cache.cpu().numpy(), vc), f"{what}: V pool"
+    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, wl.context_lens,
+                                      wl.scale, wl.dtype, wl.extra["k_scale"], wl.extra["v_scale"])
+    assert st == 0
+    assert_close(to_f64(out), ref, what or wl.name)
+    assert dev.status() == 0
+    return dev, out
+
+
+# ---- the quantising cache write -------------------------------------------------
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("scales", [(1 / 64, 1 / 64), (0.0371, 0.2113)], ids=["pow2", "odd"])
+def test_cache_write_bit_exact(dtype, scales):
+    """Random codes in the pools (a stray write anywhere shows), a mix of
+    ordinary, saturating and special values (inf, NaN, -0) in the rows,
+    padding slots (-1) and one slot past the pool (status 2)."""
+    from paged_kv_cache_415_b200 import binding as B
+    rng = np.random.Generator(np.random.PCG64(31 if dtype == "f16" else 32))
+    nb, b, h, d = 24, 16, 4, 128
+    kc = rng.integers(0, 256, size=(nb, b, h, d), dtype=np.uint8)
+    vc = rng.integers(0, 256, size=(nb, b, h, d), dtype=np.uint8)
+    t = 40
+    x = rng.standard_normal((2, t, h, d)).astype(np.float32)
+    x[:, ::3] *= 40.0                                       # saturates for small scales
+    x[0, 1, 0, :4] = [np.inf, -np.inf, np.nan, -0.0]
+    key = gen.f32_to_bits(x[0], dtype)
+    val = gen.f32_to_bits(x[1], dtype)
+    slots = rng.permutation(nb * b)[:t].astype(np.int64)
+    slots[5] = -1
+    slots[9] = nb * b + 3
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dk, dv = _u8(kc), _u8(vc)
+    B.pa_reshape_and_cache_fp8(to_dev(key, dtype), to_dev(val, dtype), dk, dv,
+                               torch.from_numpy(slots).cuda(), scales[0], scales[1], status)
+    torch.cuda.synchronize()
+    ek, ev = kc.copy(), vc.copy()
+    st = oracle.reshape_and_cache_fp8(key, val, ek, ev, slots, b, dtype, scales[0], scales[1])
+    assert np.array_equal(dk.cpu().numpy(), ek)
+    assert np.array_equal(dv.cpu().numpy(), ev)
+    assert int(status.item()) == st == 2
+
+
+def test_cache_write_rejects_bad_scales():
+    from paged_kv_cache_415_b200 import binding as B
+    kc = torch.zeros((4, 16, 2, 64), dtype=torch.uint8, device="cuda")
+    key = torch.zeros((1, 2, 64), dtype=torch.float16, device="cuda")
+    slots = torch.zeros(1, dtype=torch.int64, device="cuda")
+    for ks in (0.0, -1.0, float("inf"), float("nan")):
+        with pytest.raises(B.PAError):
+            B.pa_reshape_and_cache_fp8(key, key, kc, kc.clone(), slots, ks, 1.0)
+    assert not kc.any()
+
+
+def test_copy_blocks_on_fp8_pools():
+    """pa_copy_blocks with the one-byte element type moves whole blocks of
+    codes (checked against the oracle's copy on the same bytes)."""
+    from paged_kv_cache_415_b200 import binding as B
+    rng = np.random.Generator(np.random.PCG64(33))
+    kc = rng.integers(0, 256, size=(12, 16, 2, 64), dtype=np.uint8)
+    vc = rng.integers(0, 256, size=(12, 16, 2, 64), dtype=np.uint8)
+    m = np.array([[1, 4], [7, 2], [3, 11]], dtype=np.int64)
+    dk, dv = _u8(kc), _u8(vc)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    B.pa_copy_blocks(dk, dv, torch.from_numpy(m).cuda(), status)
+    torch.cuda.synchronize()
+    # the oracle copies 16-bit elements: the same bytes seen as pairs
+    ek, ev = kc.copy().view(np.uint16), vc.copy().view(np.uint16)
+    assert oracle.copy_blocks(ek, ev, m) == 0
+    assert np.array_equal(dk.cpu().numpy(), ek.view(np.uint8))
+    assert np.array_equal(dv.cpu().numpy(), ev.view(np.uint8))
+    assert int(status.item()) == 0
+
+
+# ---- decode over e4m3 pools -------------------------------------------------------
+
+def _instance(head_dim, block_size, group, dtype, partition_blocks=4):
+    rng = np.random.Generator(np.random.PCG64(head_dim * 1000 + block_size * 10 + group + 5))
+    ctx = rng.integers(1, 300, size=3, endpoint=True)
+    ctx[0] = 1
+    nb = int(sum(-(-int(c) // block_size) for c in ctx)) + 8
+    wl = gen.make_decode("fp8-instance", seed=78, dtype=dtype, context_lens=ctx,
+                         num_q_heads=2 * group, num_kv_heads=2, head_dim=head_dim,
+                         block_size=block_size, num_blocks=nb, scale=1 / math.sqrt(head_dim),
+                         partition_size=partition_blocks * block_size)
+    return gen.with_fp8_pools(wl, seed=head_dim + block_size + group)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+@pytest.mark.parametrize("block_size", [16, 32])
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_every_fp8_instance(head_dim, block_size, group, dtype):
+    """Each (head_dim, block_size, group, query dtype) instance on ragged
+    contexts spanning several blocks, warps and partitions of 4 blocks."""
+    _parity(_instance(head_dim, block_size, group, dtype),
+            what=f"fp8 D{head_dim} B{block_size} G{group} {dtype}")
+
+
+@pytest.mark.parametrize("partition", [16, 512, 0])
+def test_fp8_partition_sweep(partition):
+    wl = gen.with_fp8_pools(oracle_pins.small_gqa(seqs=6), seed=40)
+    _parity(wl, partition_size=partition, what=f"fp8 gqa P{partition}")
+
+
+def test_fp8_odd_scales_and_single_token():
+    """Scales that are not powers of two; a one-token context returns
+    v_scale * v0 (to output rounding)."""
+    wl = oracle_pins.small_llama(seqs=5)
+    ctx = wl.context_lens.copy()
+    ctx[0] = 1
+    wl = gen.make_decode("fp8-odd", seed=79, dtype="bf16", context_lens=ctx, num_q_heads=8,
+                         num_kv_heads=8, head_dim=128, block_size=16, num_blocks=160,
+                         scale=1 / math.sqrt(128))
+    wl = gen.with_fp8_pools(wl, seed=41, k_scale=0.0371, v_scale=0.2113)
+    _parity(wl, partition_size=64, what="fp8 odd scales")
+
+
+def test_fp8_unsupported_and_invalid():
+    """Block size 8 has no one-byte tile path (UNSUPPORTED); non-positive or
+    non-finite scales are INVALID_ARG; nothing is written."""
+    from paged_kv_cache_415_b200 import binding as B
+    wl8 = gen.make_decode("fp8-b8", seed=80, dtype="f16", context_lens=[20, 5], num_q_heads=2,
+                          num_kv_heads=2, head_dim=64, block_size=8, num_blocks=8, scale=0.125)
+    wl8 = gen.with_fp8_pools(wl8, seed=42)
+    dev = Fp8Device(wl8)
+    with pytest.raises(B.PAError, match="UNSUPPORTED|unsupported"):
+        dev.decode()
+    dev = Fp8Device(_instance(64, 16, 1, "f16"))
+    for ks in (0.0, float("nan")):
+        dev.ks = ks
+        with pytest.raises(B.PAError):
+            dev.decode()
+
+
+def test_fp8_empty_context_and_bad_block():
+    """ctx 0 -> zero row; an out-of-pool block id is skipped and flagged
+    (status 1) exactly as the oracle does."""
+    wl = gen.with_fp8_pools(oracle_pins.small_llama(seqs=4), seed=43)
+    kc, vc, _ = _oracle_pools(wl)
+    wl.k_cache, wl.v_cache = kc, vc
+    dev = Fp8Device(wl)
+    ctx = wl.context_lens.copy()
+    ctx[0] = 0
+    out = dev.decode(context_lens=torch.from_numpy(ctx).cuda(), partition_size=64)
+    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, ctx, wl.scale, wl.dtype,
+                                      dev.ks, dev.vs)
+    assert_close(to_f64(out), ref)
+    assert dev.status() == st == 0
+    tables = wl.block_tables.copy()
+    s = int(np.argmax(wl.context_lens))
+    tables[s, 0] = wl.num_blocks + 7
+    out = dev.decode(block_tables=torch.from_numpy(tables).cuda(), partition_size=64)
+    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, tables, wl.context_lens, wl.scale,
+                                      wl.dtype, dev.ks, dev.vs)
+    assert st == 1 and dev.status() == 1
+    assert_close(to_f64(out), ref)
+
+
+def test_fp8_deterministic():
+    wl = _instance(128, 16, 4, "bf16")
+    dev = Fp8Device(wl)
+    dev.write()
+    a = dev.decode()
+    b = dev.decode()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["llama7b", "mistral7b"])
+def test_fp8_full_size(name):
+    """The full-size workload with e4m3 pools, in the launch configuration
+    the benchmark times: write + decode against the whole oracle."""
+    wl = gen.with_fp8_pools(gen.CONFIGS[name](), seed=44)
+    _parity(wl, what=name + "-fp8")

@@ -43,11 +43,13 @@ def paged_waste_slots(context_len: int, block_size: int) -> int:
 
 
 def decode_bytes(ctx: np.ndarray, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                 block_size: int, elem_bytes: int) -> dict:
-    """Algorithmic bytes of the attention part of one decode step."""
+                 block_size: int, elem_bytes: int, kv_elem_bytes: int | None = None) -> dict:
+    """Algorithmic bytes of the attention part of one decode step
+    (kv_elem_bytes: bytes of a cached K/V element when it differs from the
+    query's, e.g. 1 for e4m3 pools)."""
     ctx = np.asarray(ctx, dtype=np.int64)
     s = ctx.shape[0]
-    row = num_kv_heads * head_dim * elem_bytes
+    row = num_kv_heads * head_dim * (elem_bytes if kv_elem_bytes is None else kv_elem_bytes)
     kv = int(ctx.sum()) * row * 2
     q = s * num_q_heads * head_dim * elem_bytes
     out = q
@@ -58,15 +60,23 @@ def decode_bytes(ctx: np.ndarray, num_q_heads: int, num_kv_heads: int, head_dim:
             "total": kv + q + out + table + lens}
 
 
+def kv_elem_bytes(wl) -> int:
+    """Bytes of one cached K/V element: 1 for e4m3 pools, else the element
+    type's."""
+    return 1 if wl.extra.get("kv_dtype") == "fp8" else ELEM_BYTES[wl.dtype]
+
+
 def step_bytes(wl) -> dict:
     """Algorithmic bytes of a whole decode step of a workload (attention,
     appended tokens, copy-on-write copies)."""
     e = ELEM_BYTES[wl.dtype]
+    ekv = kv_elem_bytes(wl)
     att = decode_bytes(wl.context_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
-                       wl.block_size, e)
-    row = wl.num_kv_heads * wl.head_dim * e
+                       wl.block_size, e, ekv)
+    row_in = wl.num_kv_heads * wl.head_dim * e
+    row = wl.num_kv_heads * wl.head_dim * ekv
     t = wl.num_new_tokens
-    append = 2 * (2 * t * row) + 8 * t          # K,V read + written, slot ids
+    append = 2 * t * row_in + 2 * t * row + 8 * t   # K,V read + written, slot ids
     blk = wl.block_size * row
     p = int(wl.block_mapping.shape[0])
     copies = 2 * (2 * p * blk) + 16 * p          # K,V blocks read + written, pairs
@@ -77,8 +87,7 @@ def step_bytes(wl) -> dict:
 def unique_kv_bytes(wl) -> int:
     """K/V bytes of the distinct physical blocks the step reads (shared
     blocks counted once), for workloads with block sharing."""
-    e = ELEM_BYTES[wl.dtype]
-    row = wl.num_kv_heads * wl.head_dim * e
+    row = wl.num_kv_heads * wl.head_dim * kv_elem_bytes(wl)
     seen = {}
     for s in range(wl.num_seqs):
         c = int(wl.context_lens[s])

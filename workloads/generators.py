@@ -163,6 +163,58 @@ def make_decode(name, *, seed, dtype, context_lens, num_q_heads, num_kv_heads, h
 
 
 # ---------------------------------------------------------------------------
+# FP8 (e4m3) pools: the same workload with its cached K/V held as one-byte
+# codes.  The codes are drawn directly (sign, exponent field, mantissa field
+# uniform), so nothing here quantises; the step's new tokens stay in the
+# 16-bit element type and are quantised by the cache write under test.
+# ---------------------------------------------------------------------------
+
+E4M3_NAN = 0x7F
+
+
+def e4m3_codes(rng: np.random.Generator, shape, max_exponent_field: int = 14) -> np.ndarray:
+    """Random e4m3 codes: sign and mantissa uniform, exponent field uniform in
+    [0, max_exponent_field] (14 keeps clear of the NaN code 0x7F / 0xFF)."""
+    sign = rng.integers(0, 2, size=shape, dtype=np.uint8) << 7
+    exp = rng.integers(0, max_exponent_field + 1, size=shape, dtype=np.uint8) << 3
+    mant = rng.integers(0, 8, size=shape, dtype=np.uint8)
+    return (sign | exp | mant).astype(np.uint8)
+
+
+def with_fp8_pools(wl: DecodeWorkload, seed: int, k_scale: float = 1.0 / 64.0,
+                   v_scale: float = 1.0 / 64.0) -> DecodeWorkload:
+    """A copy of a make_decode workload whose pools are e4m3 codes: every
+    slot that holds a history token gets random codes, every other slot the
+    NaN code (so reading a slot the kernel must not read poisons the
+    output).  Scales are per pool; with 1/64 the largest code (240) stands
+    for 3.75.  extra: kv_dtype = "fp8", k_scale, v_scale."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    b = wl.block_size
+    shape = (wl.num_blocks, b, wl.num_kv_heads, wl.head_dim)
+    k_cache = np.full(shape, E4M3_NAN, dtype=np.uint8)
+    v_cache = np.full(shape, E4M3_NAN, dtype=np.uint8)
+    new = set(int(x) for x in wl.slot_mapping if x >= 0)
+    slots = []
+    for s in range(wl.num_seqs):
+        c = int(wl.context_lens[s])
+        pos = np.arange(c, dtype=np.int64)
+        table = wl.block_tables[s].astype(np.int64)
+        slots.extend(int(x) for x in table[pos // b] * b + pos % b if int(x) not in new)
+    slots = np.asarray(sorted(set(slots)), dtype=np.int64)
+    row = (wl.num_kv_heads, wl.head_dim)
+    if slots.size:
+        _scatter(k_cache, slots, e4m3_codes(rng, (slots.size,) + row), b)
+        _scatter(v_cache, slots, e4m3_codes(rng, (slots.size,) + row), b)
+    out = DecodeWorkload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
+    out.name = wl.name + "-fp8"
+    out.k_cache, out.v_cache = k_cache, v_cache
+    out.keys = out.values = None
+    out.extra = dict(wl.extra, kv_dtype="fp8", k_scale=float(np.float32(k_scale)),
+                     v_scale=float(np.float32(v_scale)))
+    return out
+
+
+# ---------------------------------------------------------------------------
 # The five workloads.  ``seqs`` shrinks the batch (and ``max_ctx`` the
 # contexts) for oracle-sized parity cases; the head layout is unchanged.
 # ---------------------------------------------------------------------------
