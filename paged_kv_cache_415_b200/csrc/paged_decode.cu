@@ -133,6 +133,36 @@ __device__ __forceinline__ void write_zero_rows(T* out, int s, int kvh, int num_
         reinterpret_cast<uint4*>(row)[i] = make_uint4(0, 0, 0, 0);
 }
 
+// Longest-first dispatch.  The CTAs of a grid start in blockIdx order, so
+// when CTA z serves the sequence with the z-th longest context (ties by
+// index), the long contexts start first and the last wave holds the short
+// ones: the tail where few CTAs are left shrinks.  Every thread of the CTA
+// calls this before anything else uses `scratch` (num_seqs + 1 ints of
+// shared memory, reused afterwards); needs num_seqs <= blockDim.x.  The
+// mapping is a permutation, so each sequence is served exactly once; the
+// work of a (sequence, head, partition) does not depend on which CTA runs
+// it, so results are unchanged.
+__device__ __forceinline__ int lpt_sequence(const int32_t* __restrict__ context_lens,
+                                            int32_t num_seqs, int rank, int32_t* scratch)
+{
+    const int t = threadIdx.x;
+    const int32_t c = t < num_seqs ? context_lens[t] : 0;
+    if (t < num_seqs) scratch[t] = c;
+    __syncthreads();
+    if (t < num_seqs) {
+        int r = 0;
+        for (int j = 0; j < num_seqs; ++j) {
+            const int32_t cj = scratch[j];
+            r += (cj > c || (cj == c && j < t)) ? 1 : 0;
+        }
+        if (r == rank) scratch[num_seqs] = t;
+    }
+    __syncthreads();
+    const int pick = scratch[num_seqs];
+    __syncthreads();   // scratch is free again
+    return pick;
+}
+
 // Fused append: the warp that loads the block holding a sequence's new token
 // (position ctx - 1) first writes that token's K and V row for its kv head
 // into the pools at the given physical block, then makes the writes visible
@@ -217,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
     int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
     int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status,
     const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
-    T* __restrict__ v_cache, int32_t num_kv_heads)
+    T* __restrict__ v_cache, int32_t num_kv_heads, int32_t lpt_seqs)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = DecodeShape<D, BS, G>;
@@ -226,7 +256,9 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
 
     const int kvh = blockIdx.x;
     const int part = blockIdx.y;
-    const int s = blockIdx.z;
+    const int s = lpt_seqs > 0 ? lpt_sequence(context_lens, lpt_seqs, blockIdx.z,
+                                              reinterpret_cast<int32_t*>(smem))
+                               : static_cast<int>(blockIdx.z);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int c = lane % S::LPT;        // position within the token row
@@ -605,7 +637,27 @@ struct DecodeArgs {
     cudaStream_t stream;
     const void* new_key = nullptr;     // fused append (one token per sequence), or null
     const void* new_value = nullptr;
+    int32_t lpt_seqs = 0;              // > 0: longest-first dispatch over this many sequences
 };
+
+constexpr int kMaxDevices = 64;
+
+// Streaming multiprocessors of the current device (queried once per device).
+static int sm_count()
+{
+    static std::atomic<int> cached[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < kMaxDevices) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < kMaxDevices) cached[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
 
 template <typename Kernel>
 static bool ensure_smem_attr(Kernel kernel, int bytes, std::atomic<uint64_t>& done_mask)
@@ -686,10 +738,13 @@ static bool encode_pool_map_swizzled(CUtensorMap* map, const void* pool, int32_t
 }
 
 // An e4m3 pool [num_blocks][B][Hkv][D] of bytes as a 4-D tensor whose box is
-// one block of one kv head (B rows of D bytes, dense in shared memory).
+// one block of one kv head: B rows of D bytes, with the 128-byte swizzle
+// when a row is 128 bytes (else dense).
 static bool encode_pool_map_fp8(CUtensorMap* map, const void* pool, int32_t head_dim,
                                 int32_t num_kv_heads, int32_t block_size, int64_t num_blocks)
 {
+    const CUtensorMapSwizzle swz =
+        head_dim == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
     auto enc = tensor_map_encoder();
     if (enc == nullptr) return false;
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(head_dim),
@@ -702,8 +757,8 @@ static bool encode_pool_map_fp8(CUtensorMap* map, const void* pool, int32_t head
                                static_cast<cuuint32_t>(block_size), 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(pool), dims,
-                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return res == CUDA_SUCCESS;
 }
@@ -724,7 +779,7 @@ static pa_status launch_decode_fp8(const DecodeArgs& a, float v_scale)
         kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v, static_cast<T*>(a.out),
         static_cast<const T*>(a.query), a.block_tables, a.context_lens, a.num_q_heads,
         a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2, v_scale,
-        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status, a.lpt_seqs);
     if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
@@ -780,7 +835,7 @@ static pa_status launch_decode(const DecodeArgs& a)
             a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status,
             static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
             static_cast<T*>(const_cast<void*>(a.k_cache)), static_cast<T*>(const_cast<void*>(a.v_cache)),
-            a.num_kv_heads);
+            a.num_kv_heads, a.lpt_seqs);
         if (ls != PA_OK) return ls;
     } else {
         using S = DecodeShape<D, BS, G>;
@@ -797,7 +852,7 @@ static pa_status launch_decode(const DecodeArgs& a)
             a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status,
             static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
             static_cast<T*>(const_cast<void*>(a.k_cache)), static_cast<T*>(const_cast<void*>(a.v_cache)),
-            a.num_kv_heads);
+            a.num_kv_heads, a.lpt_seqs);
         if (ls != PA_OK) return ls;
     }
     if (a.max_parts <= 1) return PA_OK;
@@ -1050,6 +1105,10 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.stream = stream;
     a.new_key = new_key;
     a.new_value = new_value;
+    // longest-first dispatch pays off once the grid spans more than about
+    // two CTAs per SM (a tail exists) and the batch fits one CTA's threads
+    const int64_t ctas = static_cast<int64_t>(num_kv_heads) * max_parts * num_seqs;
+    if (num_seqs <= kThreads && ctas > 2 * static_cast<int64_t>(sm_count())) a.lpt_seqs = num_seqs;
     if (fp8)
         return dtype == PA_DTYPE_F16 ? dispatch_fp8<__half>(a, v_scale)
                                      : dispatch_fp8<__nv_bfloat16>(a, v_scale);
@@ -1232,7 +1291,6 @@ namespace pa {
 
 static __device__ __align__(256) unsigned char g_no_alloc_workspace[PA_NO_ALLOC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
 static std::mutex g_no_alloc_mutex;
 static void* g_no_alloc_ptr[kMaxDevices];   // device address of the array, per device
 

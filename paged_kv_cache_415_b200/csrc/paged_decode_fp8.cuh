@@ -5,64 +5,116 @@
 // 管理KV Cache" (工程实践与局限) name low-precision storage of the cached blocks;
 // at one byte per element every decode step moves half the bytes.
 //
-// Same work split, TMA pipeline, softmax and merge as paged_decode_mma_kernel.
-// Per block, the warp's K and V tiles arrive as bytes (B rows x D codes);
-// the warp widens them exactly to fp16 (every e4m3 value is an fp16 value)
-// into the 128-byte-swizzled 16-bit layout the tensor-core contraction reads
-// with ldmatrix, clearing V rows past the context on the way.  Both
-// contractions run as fp16 mma.sync with fp32 accumulation, whatever the
-// query type (a bf16 query is rounded to fp16 once per CTA).  The scales are
-// folded in: k_scale into the score scale, v_scale into the output.
+// Same work split, TMA pipeline, online softmax and merge as the 16-bit
+// kernels; the tiles arrive as bytes (B rows x D codes, 128-byte swizzle for
+// D = 128) and never go back to shared memory in a wider type.  Both
+// contractions run on the tensor cores (mma.sync m16n8k16, fp16 in, fp32
+// accumulate) with the cache tile as the A operand and the heads of the
+// group as the 8 columns of N, so a lone query head wastes 7/8 of an MMA
+// rather than 15/16:
+//
+//   S^T [16 tokens x 8 heads]  = K [16 x D] . Q^T [D x 8]
+//   O^T [D x 8 heads]         += V^T [D x 16 tokens] . P^T [16 x 8]
+//
+// Each lane reads its A fragments straight from the byte tile, pairs codes
+// with byte permutes where two tokens share a register (V^T), and widens
+// them exactly with cvt.rn.f16x2.e4m3x2 (every e4m3 value is an fp16 value).
+// The contraction index may be permuted freely as long as both operands
+// follow it, so every lane reads whole 16-byte runs of one token row.  P
+// moves from the accumulator layout (tokens x heads) to the B layout (heads
+// x tokens) through a 384-byte shared tile with stmatrix.trans / ldmatrix.
+// Scales: k_scale folds into the score scale, v_scale into the output.  The
+// query is rounded once to fp16 (exact for fp16 queries).
 
 namespace pa {
 
 template <int D, int BS, int G>
 struct Fp8Shape {
-    static constexpr int NH = D / 64;
-    static constexpr int KSTEPS = D / 16;
-    static constexpr int NTILES = D / 8;
-    static constexpr int SLICES = BS / 16;
-    static constexpr int TILE8 = BS * D;                 // bytes of one K (or V) tile, one head
-    static constexpr int TILE16 = BS * D * 2;            // the same tile widened to fp16
-    static constexpr int STAGE8 = 2 * TILE8;
-    static constexpr int NSTAGE = 2;
-    static constexpr int WARP_BYTES = NSTAGE * STAGE8 + 2 * TILE16;   // byte ring + fp16 K, V
-    static constexpr int OFF_BARS = kWarps * WARP_BYTES;
-    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8 + 1024;
+    static constexpr int SLICES = BS / 16;           // 16-token MMA slices per block
+    static constexpr int KW = D / 16;                // k-steps of S^T; 4-code words per K row per lane
+    static constexpr int KV16 = KW / 4;              // 16-byte K loads per row per lane
+    static constexpr int DPT = D / 8;                // output dims per lane (V^T rows)
+    static constexpr int VQ = DPT / 4;               // 4-code words per V row per lane
+    static constexpr int MT = D / 16;                // m-tiles of V^T
+    static constexpr bool SWIZZLE = (D == 128);      // 128-byte rows, 128B TMA swizzle
+    static constexpr int TILE = BS * D;              // bytes of one K (or V) tile of one head
+    static constexpr int STAGE = 2 * TILE;
+#ifndef PA_FP8_NSTAGE
+#define PA_FP8_NSTAGE 3
+#endif
+    static constexpr int NSTAGE = STAGE <= 4096 ? PA_FP8_NSTAGE : 2;
+    static constexpr int PT_STRIDE = 48;             // bytes per head row of the P^T tile
+    static constexpr int PT_BYTES = 8 * PT_STRIDE;
+    static constexpr int WARP_BYTES = NSTAGE * STAGE;
+    static constexpr int OFF_PT = kWarps * WARP_BYTES;
+    static constexpr int OFF_BARS = OFF_PT + kWarps * PT_BYTES;
+    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8 + 1024;   // + alignment slack
     static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
-    static_assert(BS % 16 == 0 && D % 64 == 0, "whole 16-token slices, 128-byte rows");
-    static_assert(G >= 1 && G <= 8, "heads fit rows 0..7 of the A operand");
+    static_assert(BS % 16 == 0 && (D == 64 || D == 128), "whole 16-token slices");
+    static_assert(G >= 1 && G <= 8, "heads are the 8 columns of N");
+    static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
     static_assert(EPI_BYTES <= OFF_BARS, "epilogue fits in the warp buffers");
-    static_assert((NSTAGE * STAGE8) % 1024 == 0 && TILE16 % 1024 == 0,
-                  "fp16 tiles keep the 1024-byte swizzle alignment");
 };
 
-// 16 e4m3 codes -> 16 fp16 values, exact.
-__device__ __forceinline__ void widen16(const uint4& w, uint4& lo, uint4& hi)
+// Byte offset of (row, byte) in a tile; byte is a multiple of 8 within the
+// row.  D = 128: 128-byte rows with the TMA 128B swizzle (16-byte chunk c
+// of row r sits at chunk c ^ (r & 7)); D = 64: dense 64-byte rows.
+template <int D>
+__device__ __forceinline__ uint32_t fp8_tile_off(int row, int byte)
 {
-    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-    uint32_t r[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(
-            static_cast<__nv_fp8x2_storage_t>(in[i] & 0xffffu), __NV_E4M3);
-        const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(
-            static_cast<__nv_fp8x2_storage_t>(in[i] >> 16), __NV_E4M3);
-        r[2 * i] = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
-        r[2 * i + 1] = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
-    }
-    lo = make_uint4(r[0], r[1], r[2], r[3]);
-    hi = make_uint4(r[4], r[5], r[6], r[7]);
+    if constexpr (D == 128)
+        return static_cast<uint32_t>(row * 128 + ((((byte >> 4) ^ (row & 7)) << 4) | (byte & 15)));
+    else
+        return static_cast<uint32_t>(row * D + byte);
+}
+
+// Two e4m3 codes per 16-bit half of w -> two packed fp16 pairs, exact:
+// lo = (code0, code1), hi = (code2, code3), low byte in the low half.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi)
+{
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+
+__device__ __forceinline__ void stmatrix_x2_trans(uint32_t smem_addr, uint32_t r0, uint32_t r1)
+{
+    asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1, %2};"
+                 :
+                 : "r"(smem_addr), "r"(r0), "r"(r1)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, uint32_t smem_addr)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(smem_addr)
+                 : "memory");
+}
+
+template <int D>
+__device__ __forceinline__ void load_words(const unsigned char* tile, int row, int byte,
+                                           uint32_t (&w)[4])
+{
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + fp8_tile_off<D>(row, byte));
+    w[0] = v.x;
+    w[1] = v.y;
+    w[2] = v.z;
+    w[3] = v.w;
 }
 
 template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(
+__global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
     const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
     int64_t num_blocks, int32_t max_context_len, float scale_log2, float v_scale,
     int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
-    float2* __restrict__ ws_ml, int32_t* d_status)
+    float2* __restrict__ ws_ml, int32_t* d_status, int32_t lpt_seqs)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = Fp8Shape<D, BS, G>;
@@ -71,7 +123,9 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(
 
     const int kvh = blockIdx.x;
     const int part = blockIdx.y;
-    const int s = blockIdx.z;
+    const int s = lpt_seqs > 0 ? lpt_sequence(context_lens, lpt_seqs, blockIdx.z,
+                                              reinterpret_cast<int32_t*>(smem))
+                               : static_cast<int>(blockIdx.z);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int grp = lane >> 2;
@@ -99,8 +153,6 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(
     const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
 
     unsigned char* wbase = smem + warp * S::WARP_BYTES;
-    unsigned char* k16 = wbase + S::NSTAGE * S::STAGE8;
-    unsigned char* v16 = k16 + S::TILE16;
     uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
     if (lane == 0) {
 #pragma unroll
@@ -133,10 +185,10 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(
             const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
             fence_proxy_async_smem();
             if (ok) {
-                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE8);
-                unsigned char* dst = wbase + st * S::STAGE8;
+                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE);
+                unsigned char* dst = wbase + st * S::STAGE;
                 tma_load_4d(dst, &tm_k, 0, kvh, 0, phys, &wbar[st]);
-                tma_load_4d(dst + S::TILE8, &tm_v, 0, kvh, 0, phys, &wbar[st]);
+                tma_load_4d(dst + S::TILE, &tm_v, 0, kvh, 0, phys, &wbar[st]);
             } else {
                 status_or(d_status, PA_STATUS_BAD_BLOCK);
                 mbar_arrive_expect_tx(&wbar[st], 0u);
@@ -147,36 +199,39 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(
     for (int k = 0; k < prologue; ++k) issue(k);
     int issued = prologue;
 
-    // q as fp16 A fragments (rows = heads; rows >= G zero)
-    uint32_t qa[S::KSTEPS][2];
+    // Q^T as B fragments, fp16: k-step j holds head grp's dims
+    // (D/4)*tig + 4j .. +3, the same dims the lane's K words carry.
+    uint32_t qb[S::KW][2];
     {
-        const T* qrow = query + (static_cast<int64_t>(s) * num_q_heads + kvh * G + grp) * D;
+        const T* qrow = query + (static_cast<int64_t>(s) * num_q_heads + kvh * G + grp) * D +
+                        (D / 4) * tig;
 #pragma unroll
-        for (int ks = 0; ks < S::KSTEPS; ++ks) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t packed = 0u;
-                if (grp < G) {
-                    const float2 f = Elem<T>::to_float2(
-                        *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + half * 8 + 2 * tig));
-                    packed = Elem<__half>::from_float2(f.x, f.y);
-                }
-                qa[ks][half] = packed;
+        for (int j = 0; j < S::KW; ++j) {
+            uint32_t b0 = 0u, b1 = 0u;
+            if (grp < G) {
+                const uint2 w = *reinterpret_cast<const uint2*>(qrow + 4 * j);
+                const float2 f0 = Elem<T>::to_float2(w.x);
+                const float2 f1 = Elem<T>::to_float2(w.y);
+                b0 = Elem<__half>::from_float2(f0.x, f0.y);
+                b1 = Elem<__half>::from_float2(f1.x, f1.y);
             }
+            qb[j][0] = b0;
+            qb[j][1] = b1;
         }
     }
 
-    const int mi = lane >> 3;
-    const int ri = lane & 7;
-    const uint32_t k16_base = smem_u32(k16);
-    const uint32_t v16_base = smem_u32(v16);
-    float m_run = -INFINITY;
-    float l_run = 0.f;
-    float o[S::NTILES][4];
+    // P^T staging rows: lanes 0-7 address head rows of tokens 0-7, lanes
+    // 8-15 the same rows' tokens 8-15 (lanes 16-31 repeat them).
+    const uint32_t pt_addr = smem_u32(smem + S::OFF_PT + warp * S::PT_BYTES) +
+                             (lane & 7) * S::PT_STRIDE + ((lane >> 3) & 1) * 16;
+
+    float o[S::MT][4];
 #pragma unroll
-    for (int nt = 0; nt < S::NTILES; ++nt)
+    for (int mt = 0; mt < S::MT; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
+    float m_run0 = -INFINITY, m_run1 = -INFINITY;   // heads 2*tig, 2*tig + 1 (log2 units)
+    float l_run0 = 0.f, l_run1 = 0.f;               // this lane's share of the exp-sums
 
     bool aborted = false;
     int first_pending = 0;
@@ -196,85 +251,134 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(
         const int phys = __shfl_sync(kFullMask, cons_tbl, k & 31);
         const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
         const int nv = ok ? block_tokens(k) : 0;
-        const unsigned char* k8 = wbase + st * S::STAGE8;
-        const unsigned char* v8 = k8 + S::TILE8;
-
-        // widen both tiles to fp16 in the swizzled layout; V rows past the
-        // context are cleared (p = 0 does not cancel a NaN in the sum)
-        for (int i = lane; i < S::TILE8 / 16; i += 32) {
-            const int t = i / (D / 16);
-            const int d0 = (i % (D / 16)) * 16;
-            uint4 lo, hi;
-            widen16(*reinterpret_cast<const uint4*>(k8 + i * 16), lo, hi);
-            *reinterpret_cast<uint4*>(k16 + swz_offset<BS>(t, d0)) = lo;
-            *reinterpret_cast<uint4*>(k16 + swz_offset<BS>(t, d0 + 8)) = hi;
-            if (t < nv) {
-                widen16(*reinterpret_cast<const uint4*>(v8 + i * 16), lo, hi);
-            } else {
-                lo = make_uint4(0, 0, 0, 0);
-                hi = lo;
-            }
-            *reinterpret_cast<uint4*>(v16 + swz_offset<BS>(t, d0)) = lo;
-            *reinterpret_cast<uint4*>(v16 + swz_offset<BS>(t, d0 + 8)) = hi;
-        }
-        __syncwarp();
-        // the byte stage is free again: request the next block now
-        if (issued < nk) issue(issued++);
+        const unsigned char* kt = wbase + st * S::STAGE;
+        const unsigned char* vt = kt + S::TILE;
 
 #pragma unroll 1
         for (int sl = 0; sl < S::SLICES; ++sl) {
             const int t0 = sl * 16;
-            const int tv = nv - t0;
-            float sc[2][4];
+            const int tv = nv - t0;             // valid tokens of this slice
+            if (tv <= 0) break;
+
+            // ---- S^T = K . Q^T: rows grp and grp + 8 of the slice ----
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
+            for (int h = 0; h < S::KV16; ++h) {
+                uint32_t w0[4], w1[4];
+                load_words<D>(kt, t0 + grp, (D / 4) * tig + 16 * h, w0);
+                load_words<D>(kt, t0 + grp + 8, (D / 4) * tig + 16 * h, w1);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-                const int t = t0 + nt * 8 + ri;
-#pragma unroll
-                for (int kp = 0; kp < S::KSTEPS / 2; ++kp) {
-                    uint32_t b[4];
-                    ldmatrix_x4(b, k16_base + swz_offset<BS>(t, kp * 32 + mi * 8));
-                    mma_16816<__half>(sc[nt], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b[0], b[1]);
-                    mma_16816<__half>(sc[nt], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b[2], b[3]);
+                for (int i = 0; i < 4; ++i) {
+                    const int j = 4 * h + i;
+                    uint32_t a0, a2, a1, a3;
+                    e4m3x4_to_f16x4(w0[i], a0, a2);
+                    e4m3x4_to_f16x4(w1[i], a1, a3);
+                    if (j & 1)
+                        mma_16816<__half>(sb, a0, a1, a2, a3, qb[j][0], qb[j][1]);
+                    else
+                        mma_16816<__half>(sa, a0, a1, a2, a3, qb[j][0], qb[j][1]);
                 }
             }
-            float x[4];
-            x[0] = 2 * tig < tv ? sc[0][0] * scale_log2 : -INFINITY;
-            x[1] = 2 * tig + 1 < tv ? sc[0][1] * scale_log2 : -INFINITY;
-            x[2] = 8 + 2 * tig < tv ? sc[1][0] * scale_log2 : -INFINITY;
-            x[3] = 8 + 2 * tig + 1 < tv ? sc[1][1] * scale_log2 : -INFINITY;
-            float mloc = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-            mloc = fmaxf(mloc, __shfl_xor_sync(kFullMask, mloc, 1));
-            mloc = fmaxf(mloc, __shfl_xor_sync(kFullMask, mloc, 2));
-            const float m_new = fmaxf(m_run, mloc);
-            const float m_sub = m_new == -INFINITY ? 0.f : m_new;
-            const float corr = exp2f(m_run - m_sub);
-            m_run = m_new;
-            float p[4];
+            // this lane: tokens grp (x0, x1) and grp + 8 (x2, x3); heads 2tig, 2tig + 1
+            const float x0 = grp < tv ? (sa[0] + sb[0]) * scale_log2 : -INFINITY;
+            const float x1 = grp < tv ? (sa[1] + sb[1]) * scale_log2 : -INFINITY;
+            const float x2 = grp + 8 < tv ? (sa[2] + sb[2]) * scale_log2 : -INFINITY;
+            const float x3 = grp + 8 < tv ? (sa[3] + sb[3]) * scale_log2 : -INFINITY;
+
+            // ---- online softmax per head over the slice's 16 tokens ----
+            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) p[e] = grp < G ? exp2f(x[e] - m_sub) : 0.f;
-            const uint32_t pa0 = Elem<__half>::from_float2(p[0], p[1]);
-            const uint32_t pa2 = Elem<__half>::from_float2(p[2], p[3]);
-            const float2 r0 = Elem<__half>::to_float2(pa0), r2 = Elem<__half>::to_float2(pa2);
-            l_run = l_run * corr + ((r0.x + r0.y) + (r2.x + r2.y));
-#pragma unroll
-            for (int nt = 0; nt < S::NTILES; ++nt) {
-                o[nt][0] *= corr;
-                o[nt][1] *= corr;
+            for (int m = 4; m < 32; m <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, m));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, m));
             }
-            {
-                const int t = t0 + (mi & 1) * 8 + ri;
+            const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
+            const float ms0 = mn0 == -INFINITY ? 0.f : mn0;
+            const float ms1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float c0 = exp2f(m_run0 - ms0), c1 = exp2f(m_run1 - ms1);
+            m_run0 = mn0;
+            m_run1 = mn1;
+            // P rounds to fp16 for the tensor cores; the sums use the rounded values
+            const uint32_t pk0 = Elem<__half>::from_float2(exp2f(x0 - ms0), exp2f(x1 - ms1));
+            const uint32_t pk1 = Elem<__half>::from_float2(exp2f(x2 - ms0), exp2f(x3 - ms1));
+            const float2 r0 = Elem<__half>::to_float2(pk0), r1 = Elem<__half>::to_float2(pk1);
+            l_run0 = l_run0 * c0 + (r0.x + r1.x);
+            l_run1 = l_run1 * c1 + (r0.y + r1.y);
+            const float2 cc = make_float2(c0, c1);
 #pragma unroll
-                for (int np = 0; np < S::NTILES / 2; ++np) {
-                    uint32_t b[4];
-                    ldmatrix_x4_trans(b, v16_base + swz_offset<BS>(t, np * 16 + (mi >> 1) * 8));
-                    mma_16816<__half>(o[2 * np], pa0, 0u, pa2, 0u, b[0], b[1]);
-                    mma_16816<__half>(o[2 * np + 1], pa0, 0u, pa2, 0u, b[2], b[3]);
+            for (int mt = 0; mt < S::MT; ++mt) {
+                float2 u = __fmul2_rn(make_float2(o[mt][0], o[mt][1]), cc);
+                float2 v = __fmul2_rn(make_float2(o[mt][2], o[mt][3]), cc);
+                o[mt][0] = u.x;
+                o[mt][1] = u.y;
+                o[mt][2] = v.x;
+                o[mt][3] = v.y;
+            }
+
+            // ---- P (tokens x heads) -> P^T B fragments (heads x tokens) ----
+            uint32_t pb0, pb1;
+            __syncwarp();
+            stmatrix_x2_trans(pt_addr, pk0, pk1);
+            __syncwarp();
+            ldmatrix_x2(pb0, pb1, pt_addr);
+
+            // ---- O^T += V^T . P^T: tokens 2tig, 2tig+1, 2tig+8, 2tig+9 ----
+            const int ta = t0 + 2 * tig;
+            uint32_t va[S::VQ], vb[S::VQ], vc[S::VQ], vd[S::VQ];
+            if constexpr (S::VQ == 4) {
+                uint32_t w[4];
+                load_words<D>(vt, ta, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) va[q] = w[q];
+                load_words<D>(vt, ta + 1, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vb[q] = w[q];
+                load_words<D>(vt, ta + 8, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vc[q] = w[q];
+                load_words<D>(vt, ta + 9, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vd[q] = w[q];
+            } else {
+                const uint2 a = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta, S::DPT * grp));
+                const uint2 b = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta + 1, S::DPT * grp));
+                const uint2 c = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta + 8, S::DPT * grp));
+                const uint2 d = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta + 9, S::DPT * grp));
+                va[0] = a.x; va[1] = a.y;
+                vb[0] = b.x; vb[1] = b.y;
+                vc[0] = c.x; vc[1] = c.y;
+                vd[0] = d.x; vd[1] = d.y;
+            }
+            if (tv < 16) {   // rows past the context may hold any code (NaN included)
+                const int ra = 2 * tig;
+#pragma unroll
+                for (int q = 0; q < S::VQ; ++q) {
+                    va[q] = ra < tv ? va[q] : 0u;
+                    vb[q] = ra + 1 < tv ? vb[q] : 0u;
+                    vc[q] = ra + 8 < tv ? vc[q] : 0u;
+                    vd[q] = ra + 9 < tv ? vd[q] : 0u;
                 }
+            }
+#pragma unroll
+            for (int q = 0; q < S::VQ; ++q) {
+                // token pairs per dim: [b1 a1 b0 a0] and [b3 a3 b2 a2]
+                const uint32_t lo_ab = __byte_perm(va[q], vb[q], 0x5140);
+                const uint32_t hi_ab = __byte_perm(va[q], vb[q], 0x7362);
+                const uint32_t lo_cd = __byte_perm(vc[q], vd[q], 0x5140);
+                const uint32_t hi_cd = __byte_perm(vc[q], vd[q], 0x7362);
+                uint32_t a0, a1, a2, a3;
+                // m-tile 2q: rows grp / grp + 8 are dims DPT*grp + 4q + 0 / + 1
+                e4m3x4_to_f16x4(lo_ab, a0, a1);
+                e4m3x4_to_f16x4(lo_cd, a2, a3);
+                mma_16816<__half>(o[2 * q], a0, a1, a2, a3, pb0, pb1);
+                // m-tile 2q + 1: dims + 2 / + 3
+                e4m3x4_to_f16x4(hi_ab, a0, a1);
+                e4m3x4_to_f16x4(hi_cd, a2, a3);
+                mma_16816<__half>(o[2 * q + 1], a0, a1, a2, a3, pb0, pb1);
             }
         }
-        __syncwarp();   // the fp16 tiles are rewritten by the next block
+        __syncwarp();   // every lane is done with this stage
+        if (issued < nk) issue(issued++);
     }
 
     if (aborted) {
@@ -285,21 +389,37 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(
         }
     }
 
-    l_run += __shfl_xor_sync(kFullMask, l_run, 1);
-    l_run += __shfl_xor_sync(kFullMask, l_run, 2);
+#pragma unroll
+    for (int m = 4; m < 32; m <<= 1) {
+        l_run0 += __shfl_xor_sync(kFullMask, l_run0, m);
+        l_run1 += __shfl_xor_sync(kFullMask, l_run1, m);
+    }
 
-    __syncthreads();
-    float* epi_o = reinterpret_cast<float*>(smem);
+    __syncthreads();   // every warp is done with its stage buffers
+    float* epi_o = reinterpret_cast<float*>(smem);   // [warp][g][D]
     float* epi_m = epi_o + kWarps * G * D;
     float* epi_l = epi_m + kWarps * G;
-    if (grp < G) {
+    const int h0 = 2 * tig, h1 = 2 * tig + 1;
 #pragma unroll
-        for (int nt = 0; nt < S::NTILES; ++nt)
-            *reinterpret_cast<float2*>(epi_o + (warp * G + grp) * D + nt * 8 + 2 * tig) =
-                make_float2(o[nt][0] * v_scale, o[nt][1] * v_scale);
-        if (tig == 0) {
-            epi_m[warp * G + grp] = m_run;
-            epi_l[warp * G + grp] = l_run;
+    for (int q = 0; q < S::VQ; ++q) {
+        const int d = S::DPT * grp + 4 * q;
+        if (h0 < G)
+            *reinterpret_cast<float4*>(epi_o + (warp * G + h0) * D + d) =
+                make_float4(o[2 * q][0] * v_scale, o[2 * q][2] * v_scale,
+                            o[2 * q + 1][0] * v_scale, o[2 * q + 1][2] * v_scale);
+        if (h1 < G)
+            *reinterpret_cast<float4*>(epi_o + (warp * G + h1) * D + d) =
+                make_float4(o[2 * q][1] * v_scale, o[2 * q][3] * v_scale,
+                            o[2 * q + 1][1] * v_scale, o[2 * q + 1][3] * v_scale);
+    }
+    if (grp == 0) {
+        if (h0 < G) {
+            epi_m[warp * G + h0] = m_run0;
+            epi_l[warp * G + h0] = l_run0;
+        }
+        if (h1 < G) {
+            epi_m[warp * G + h1] = m_run1;
+            epi_l[warp * G + h1] = l_run1;
         }
     }
     __syncthreads();

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
     int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
     int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status,
     const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
-    T* __restrict__ v_cache, int32_t num_kv_heads)
+    T* __restrict__ v_cache, int32_t num_kv_heads, int32_t lpt_seqs)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = MmaShape<D, BS, G>;
@@ -79,7 +79,9 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
 
     const int kvh = blockIdx.x;
     const int part = blockIdx.y;
-    const int s = blockIdx.z;
+    const int s = lpt_seqs > 0 ? lpt_sequence(context_lens, lpt_seqs, blockIdx.z,
+                                              reinterpret_cast<int32_t*>(smem))
+                               : static_cast<int>(blockIdx.z);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int grp = lane >> 2;          // row group of the mma fragments (head)
