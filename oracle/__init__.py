@@ -55,6 +55,8 @@ def load(path: str | None = None):
     lib.oracle_reshape_and_cache.restype = i32
     lib.oracle_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i64]
     lib.oracle_copy_blocks.restype = i32
+    lib.oracle_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64, i32]
+    lib.oracle_swap_blocks.restype = i32
     lib.oracle_paged_decode.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64,
                                         f64, i32, i32, i32]
     lib.oracle_paged_decode.restype = i32
@@ -124,6 +126,20 @@ def copy_blocks(k_cache, v_cache, block_mapping, lib=None) -> int:
     return int((lib or load()).oracle_copy_blocks(
         _ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), block_mapping.shape[0],
         hkv, d, bs, num_blocks))
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, lib=None) -> int:
+    """In place on dst: for each (src, dst) row of block_mapping, block src of
+    the source pools becomes block dst of the destination pools (raw bytes;
+    pools of any one element type, [num_blocks][B][Hkv][D])."""
+    block_mapping = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+    assert src_k.dtype == dst_k.dtype and src_k.shape[1:] == dst_k.shape[1:]
+    for a in (src_k, src_v, dst_k, dst_v):
+        assert a.flags["C_CONTIGUOUS"]
+    src_nb, bs, hkv, d = src_k.shape
+    return int((lib or load()).oracle_swap_blocks(
+        _ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v), _ptr(block_mapping),
+        block_mapping.shape[0], hkv, d, bs, src_nb, dst_k.shape[0], src_k.dtype.itemsize))
 
 
 def paged_decode(query, k_cache, v_cache, block_tables, context_lens, scale, dtype,

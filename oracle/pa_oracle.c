@@ -248,6 +248,40 @@ int32_t oracle_copy_blocks(uint16_t* k_cache, uint16_t* v_cache,
     return status;
 }
 
+/* ------------------------------------------------------------------------
+ * swap_blocks: eviction of a waiting request's blocks to CPU memory and
+ * their return when it is rescheduled ([VM-paging, 显存管理与调度策略设计],
+ * the eviction paragraph).  For every (src, dst) pair, in order, block src of
+ * the source pools becomes block dst of the destination pools, K and V, as
+ * raw bytes (elem_bytes per element).  An id outside its own pool raises bit
+ * 1 and the pair is skipped; a destination that appears twice raises bit 8
+ * (the pairs are still applied in order here).
+ * ---------------------------------------------------------------------- */
+int32_t oracle_swap_blocks(const uint8_t* src_k, const uint8_t* src_v, uint8_t* dst_k,
+                           uint8_t* dst_v, const int64_t* block_mapping, int32_t num_pairs,
+                           int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                           int64_t src_num_blocks, int64_t dst_num_blocks, int32_t elem_bytes)
+{
+    int32_t status = 0;
+    const int64_t block_bytes = (int64_t)block_size * num_kv_heads * head_dim * elem_bytes;
+    for (int32_t i = 0; i < num_pairs; ++i)
+        for (int32_t j = 0; j < i; ++j)
+            if (block_mapping[2 * j + 1] == block_mapping[2 * i + 1]) status |= 8;
+    for (int32_t i = 0; i < num_pairs; ++i) {
+        int64_t src = block_mapping[2 * i];
+        int64_t dst = block_mapping[2 * i + 1];
+        if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) {
+            status |= 1;
+            continue;
+        }
+        for (int64_t b = 0; b < block_bytes; ++b) {
+            dst_k[dst * block_bytes + b] = src_k[src * block_bytes + b];
+            dst_v[dst * block_bytes + b] = src_v[src * block_bytes + b];
+        }
+    }
+    return status;
+}
+
 /* Address translation: token t of sequence s -> element offset of row
  * (t, kv head g) in the pool, or -1 when the table entry is out of range
  * ([Practice §3.2]: logical block j -> table[j] -> physical id -> base +

@@ -381,4 +381,71 @@ def pin_fp8_decode_equals_dequantised_fp16(lib):
     assert np.array_equal(a, b)
 
 
+# ---- swap_blocks (eviction to host memory and back) ---------------------------
+
+def pin_swap_round_trip(lib):
+    """Swapping blocks out to a second pool and back through the inverse
+    mapping restores the first pool exactly; destination blocks outside the
+    mapping keep their bytes."""
+    rng = np.random.Generator(np.random.PCG64(12))
+    dev_k = rng.integers(0, 65536, size=(9, 4, 2, 8), dtype=np.uint16)
+    dev_v = rng.integers(0, 65536, size=(9, 4, 2, 8), dtype=np.uint16)
+    host_k = rng.integers(0, 65536, size=(5, 4, 2, 8), dtype=np.uint16)
+    host_v = rng.integers(0, 65536, size=(5, 4, 2, 8), dtype=np.uint16)
+    out = np.array([[7, 0], [2, 3], [5, 1]])
+    hk0, hv0 = host_k.copy(), host_v.copy()
+    assert oracle.swap_blocks(dev_k, dev_v, host_k, host_v, out, lib=lib) == 0
+    for blk in (2, 4):
+        assert np.array_equal(host_k[blk], hk0[blk]) and np.array_equal(host_v[blk], hv0[blk])
+    back_k = np.zeros_like(dev_k)
+    back_v = np.zeros_like(dev_v)
+    assert oracle.swap_blocks(host_k, host_v, back_k, back_v, out[:, ::-1], lib=lib) == 0
+    for src, _ in out:
+        assert np.array_equal(back_k[src], dev_k[src]) and np.array_equal(back_v[src], dev_v[src])
+
+
+def pin_swap_equals_copy_on_joined_pool(lib):
+    """A swap between two pools is copy_blocks on the pool made of both, with
+    destination ids shifted past the source pool (copy_blocks is pinned by
+    its own definition above); statuses agree, including a bad id and a
+    repeated destination."""
+    rng = np.random.Generator(np.random.PCG64(13))
+    a_k = rng.integers(0, 65536, size=(6, 4, 2, 8), dtype=np.uint16)
+    a_v = rng.integers(0, 65536, size=(6, 4, 2, 8), dtype=np.uint16)
+    b_k = rng.integers(0, 65536, size=(4, 4, 2, 8), dtype=np.uint16)
+    b_v = rng.integers(0, 65536, size=(4, 4, 2, 8), dtype=np.uint16)
+    for pairs, want in (([[0, 3], [5, 0], [2, 1]], 0), ([[1, 2], [4, 2]], 8), ([[-1, 0], [3, 1]], 1)):
+        m = np.array(pairs, dtype=np.int64)
+        jk, jv = np.concatenate([a_k, b_k]), np.concatenate([a_v, b_v])
+        mj = m.copy()
+        mj[:, 1] += a_k.shape[0]
+        st_copy = oracle.copy_blocks(jk, jv, mj, lib=lib)
+        dk, dv = b_k.copy(), b_v.copy()
+        st_swap = oracle.swap_blocks(a_k, a_v, dk, dv, m, lib=lib)
+        assert st_swap == st_copy == want
+        assert np.array_equal(dk, jk[a_k.shape[0]:]) and np.array_equal(dv, jv[a_k.shape[0]:])
+
+
+def pin_swap_bytes_of_fp8_pools(lib):
+    """One-byte pools swap as bytes: the same data seen as 16-bit pairs
+    swaps identically."""
+    rng = np.random.Generator(np.random.PCG64(14))
+    src_k = rng.integers(0, 256, size=(5, 4, 2, 16), dtype=np.uint8)
+    src_v = rng.integers(0, 256, size=(5, 4, 2, 16), dtype=np.uint8)
+    dst_k = rng.integers(0, 256, size=(3, 4, 2, 16), dtype=np.uint8)
+    dst_v = rng.integers(0, 256, size=(3, 4, 2, 16), dtype=np.uint8)
+    m = np.array([[4, 0], [1, 2]])
+    w_k, w_v = dst_k.copy().view(np.uint16), dst_v.copy().view(np.uint16)
+    assert oracle.swap_blocks(src_k, src_v, dst_k, dst_v, m, lib=lib) == 0
+    assert oracle.swap_blocks(src_k.view(np.uint16), src_v.view(np.uint16), w_k, w_v, m,
+                              lib=lib) == 0
+    assert np.array_equal(dst_k, w_k.view(np.uint8)) and np.array_equal(dst_v, w_v.view(np.uint8))
+    assert np.array_equal(dst_k[0], src_k[4]) and np.array_equal(dst_v[2], src_v[1])
+    # an id past either pool is flagged and its pair skipped
+    before = dst_k.copy()
+    assert oracle.swap_blocks(src_k, src_v, dst_k, dst_v, np.array([[0, 3]]), lib=lib) == 1
+    assert oracle.swap_blocks(src_k, src_v, dst_k, dst_v, np.array([[5, 0]]), lib=lib) == 1
+    assert np.array_equal(dst_k, before)
+
+
 PINS = {name: fn for name, fn in globals().items() if name.startswith("pin_")}

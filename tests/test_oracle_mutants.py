@@ -40,6 +40,11 @@ MUTANTS = {
     "fp8_scale_dropped": ("(e4m3_to_f64(k_cache[r + d]) * k_scale)",
                           "(e4m3_to_f64(k_cache[r + d]))"),
     "fp8_write_divides_twice": ("const float kq = kx * k_inv;", "const float kq = kx * k_inv * k_inv;"),
+    "swap_only_k": ("dst_v[dst * block_bytes + b] = src_v[src * block_bytes + b];", ""),
+    "swap_dst_index_of_src": ("dst_k[dst * block_bytes + b] = src_k[src * block_bytes + b];",
+                              "dst_k[src % dst_num_blocks * block_bytes + b] = src_k[src * block_bytes + b];"),
+    "swap_bad_id_not_flagged": ("            status |= 1;\n            continue;", "            continue;"),
+    "swap_no_conflict_check": ("if (block_mapping[2 * j + 1] == block_mapping[2 * i + 1]) status |= 8;", ""),
 }
 
 
