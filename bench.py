@@ -74,6 +74,9 @@ def parse_args():
     ap.add_argument("--kv-dtype", default="auto", choices=["auto", "fp8"],
                     help="fp8: the same workload with e4m3 K/V pools (per-pool scales), "
                          "quantising cache write + e4m3 decode")
+    ap.add_argument("--swap", choices=["out", "in"], default=None,
+                    help="measure pa_swap_blocks instead of the decode step: 512 LLaMA-7B-shaped "
+                         "blocks (K and V, 256 KB a pair) device -> pinned host (out) or back (in)")
     ap.add_argument("--seqs", type=int, default=0,
                     help="shrink the batch (and the pool) for profiling; 0 = the full workload")
     return ap.parse_args()
@@ -550,10 +553,127 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# Swap of blocks over the host link (pa_swap_blocks)
+# ---------------------------------------------------------------------------
+
+SWAP_SHAPE = (16, 32, 128)          # LLaMA-7B block: 16 tokens x 32 heads x 128, fp16
+SWAP_DEVICE_BLOCKS, SWAP_HOST_BLOCKS, SWAP_PAIRS = 4096, 1024, 512
+
+
+def run_swap(args):
+    """One step = one pa_swap_blocks call moving SWAP_PAIRS scattered blocks
+    (K and V) between a device pool and a pinned host pool.  The roofline
+    peak is the copy engine's own rate for the same byte count as one
+    contiguous pinned copy in the same direction, measured here."""
+    import torch
+    from paged_kv_cache_415_b200 import binding as B
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    rng = np.random.Generator(np.random.PCG64(4150 + 60))
+    dk = torch.randint(-32768, 32767, (SWAP_DEVICE_BLOCKS,) + SWAP_SHAPE, dtype=torch.int16,
+                       device=dev).view(torch.float16)
+    dv = torch.randint(-32768, 32767, (SWAP_DEVICE_BLOCKS,) + SWAP_SHAPE, dtype=torch.int16,
+                       device=dev).view(torch.float16)
+    hk = torch.zeros((SWAP_HOST_BLOCKS,) + SWAP_SHAPE, dtype=torch.float16).pin_memory()
+    hv = torch.zeros((SWAP_HOST_BLOCKS,) + SWAP_SHAPE, dtype=torch.float16).pin_memory()
+    pairs = np.stack([rng.permutation(SWAP_DEVICE_BLOCKS)[:SWAP_PAIRS],
+                      rng.permutation(SWAP_HOST_BLOCKS)[:SWAP_PAIRS]], 1).astype(np.int64)
+    if args.swap == "in":
+        pairs = pairs[:, ::-1].copy()
+        src, dst = (hk, hv), (dk, dv)
+    else:
+        src, dst = (dk, dv), (hk, hv)
+    mapping = torch.from_numpy(pairs).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    block_bytes = int(np.prod(SWAP_SHAPE)) * 2
+    moved = SWAP_PAIRS * block_bytes * 2
+
+    def step():
+        B.pa_swap_blocks(src[0], src[1], dst[0], dst[1], mapping, status, stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise SystemExit(f"swap status {int(status.item())}")
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        start.record(stream)
+        for _ in range(args.steps):
+            step()
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    ms = start.elapsed_time(stop) / args.steps
+    # the copy engine on one contiguous buffer of the same size and direction
+    hbuf = torch.empty(moved // 2, dtype=torch.int16).pin_memory()
+    dbuf = torch.empty(moved // 2, dtype=torch.int16, device=dev)
+    a, b = (dbuf, hbuf) if args.swap == "in" else (hbuf, dbuf)
+    for _ in range(3):
+        a.copy_(b, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for _ in range(args.steps):
+        a.copy_(b, non_blocking=True)
+    stop.record(stream)
+    torch.cuda.synchronize(dev)
+    dma_ms = start.elapsed_time(stop) / args.steps
+    value = moved / (ms * 1e-3) / 1e9
+    peak = moved / (dma_ms * 1e-3) / 1e9
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        host_src = [np.zeros((SWAP_PAIRS,) + SWAP_SHAPE, np.uint16) for _ in range(2)]
+        host_dst = [np.zeros((SWAP_PAIRS,) + SWAP_SHAPE, np.uint16) for _ in range(2)]
+        local_map = np.stack([np.arange(SWAP_PAIRS), rng.permutation(SWAP_PAIRS)], 1)
+        t0 = time.perf_counter()
+        reps = 0
+        while reps == 0 or time.perf_counter() - t0 < min(args.cpu_seconds, 5.0):
+            oracle.swap_blocks(host_src[0], host_src[1], host_dst[0], host_dst[1], local_map)
+            reps += 1
+        per = (time.perf_counter() - t0) / reps
+        cpu = {"value": round(moved / per / 1e9, 3), "unit": "GB/s", "cores": 1,
+               "kind": "oracle",
+               "sample": f"oracle swap of the same {SWAP_PAIRS} block pairs between host arrays, "
+                         f"repeated {reps}x"}
+    if rank != 0:
+        return 0
+    line = {
+        "metric": f"swap_blocks GB/s over the host link ({args.swap})", "value": round(value, 2),
+        "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 (bit copy)", "data": "synthetic",
+        "config": {"workload": f"swap {args.swap}: {SWAP_PAIRS} scattered LLaMA-7B blocks "
+                               f"(16 x 32 x 128 fp16, K and V) between a {SWAP_DEVICE_BLOCKS}-block "
+                               f"device pool and a {SWAP_HOST_BLOCKS}-block pinned host pool",
+                   "bytes_per_step": moved, "l2": "host pool in pinned memory; no flush"},
+        "roofline": {"bound": "link", "kernel": "swap_blocks_kernel", "achieved": round(value, 1),
+                     "peak": round(peak, 1),
+                     "peak_kind": "measured here: copy engine, one contiguous pinned copy",
+                     "unit": "GB/s", "frac": round(value / peak, 4), "traffic": None},
+        "e2e": {"value": round(value, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": moved if args.swap == "in" else 0,
+                "d2h_bytes_per_step": moved if args.swap == "out" else 0},
+        "gpu_launches": args.steps, "clocks": sampler.summary(), "cpu_baseline": cpu,
+        "decode_entry": "pa_swap_blocks",
+    }
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.swap:
+        return run_swap(args)
     return run_ours(args)
 
 

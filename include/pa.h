@@ -96,7 +96,7 @@ typedef enum pa_status {
 typedef enum pa_dtype {
     PA_DTYPE_F16 = 0,
     PA_DTYPE_BF16 = 1,
-    PA_DTYPE_FP8_E4M3 = 2   /* cache pools only: pa_copy_blocks and the *_fp8 calls */
+    PA_DTYPE_FP8_E4M3 = 2   /* cache pools only: block copies/swaps and the *_fp8 calls */
 } pa_dtype;
 
 #define PA_STATUS_BAD_BLOCK 1
@@ -155,6 +155,48 @@ PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* blo
                          int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
                          int32_t block_size, int64_t num_blocks, pa_dtype dtype,
                          int32_t* d_status, pa_stream_t stream);
+
+/*
+ * pa_swap_blocks -- whole-block copies between two pools, one of which is
+ * normally in pinned host memory: swap out (device -> host) when a waiting
+ * request's blocks are evicted to make room, swap in (host -> device) when
+ * it is scheduled again.
+ *
+ * Defined by: [VM-paging, 显存管理与调度策略设计] (eviction: under sustained
+ * memory pressure the KV data of waiting requests moves to CPU memory and
+ * comes back to the GPU when they are rescheduled) and [Manager, 第四部分]
+ * (LRU block eviction and request preemption).  The host chooses the blocks
+ * and keeps the tables; this call moves the data for every pair at once, in
+ * one launch, with the GPU reading and writing the host pool directly.
+ *
+ *   for i < num_pairs: block block_mapping[i][1] of dst_k / dst_v becomes a
+ *                      bit-exact copy of block block_mapping[i][0] of
+ *                      src_k / src_v
+ *
+ * src_k, src_v   [src_num_blocks][block_size][num_kv_heads][head_dim]
+ * dst_k, dst_v   [dst_num_blocks][...] of the same element type.  Each is
+ *                device memory or pinned host memory that the device can
+ *                address (cudaHostAlloc / cudaHostRegister with mapping; on a
+ *                system with unified addressing the host pointer is the
+ *                device pointer).  16-byte aligned.
+ * block_mapping  int64 [num_pairs][2] of (src, dst) block ids, device or
+ *                device-addressable host memory.  Destinations must be
+ *                distinct (else PA_STATUS_COPY_CONFLICT); when the source
+ *                and destination pools are the same memory this is
+ *                pa_copy_blocks, with its conflict rule.
+ * dtype          PA_DTYPE_F16, _BF16 or _FP8_E4M3 (element size only).
+ * d_status       optional; PA_STATUS_BAD_BLOCK (an id outside its pool;
+ *                the pair is skipped), PA_STATUS_COPY_CONFLICT.
+ * Errors: PA_ERR_INVALID_ARG for null or misaligned pointers, a pointer the
+ * device cannot address (pageable host memory: checked with
+ * cudaPointerGetAttributes before anything is enqueued), a negative count
+ * or pool size; PA_ERR_UNSUPPORTED for shapes pa_copy_blocks refuses.
+ */
+PA_API pa_status pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                                const int64_t* block_mapping, int32_t num_pairs,
+                                int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                int64_t src_num_blocks, int64_t dst_num_blocks, pa_dtype dtype,
+                                int32_t* d_status, pa_stream_t stream);
 
 /*
  * pa_paged_decode_partition_size -- the context partition length (tokens)

@@ -36,6 +36,7 @@ EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_
            "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_paged_decode_no_alloc",
            "pa_paged_decode_shared_prefix_workspace_size", "pa_paged_decode_shared_prefix",
            "pa_paged_decode_append", "pa_reshape_and_cache_fp8", "pa_paged_decode_fp8",
+           "pa_swap_blocks",
            "pa_status_string", "pa_version")
 # Size of the library-owned scratch of pa_paged_decode_no_alloc.
 PA_NO_ALLOC_WORKSPACE_BYTES = 32 << 20
@@ -82,6 +83,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_paged_decode_fp8.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64, i32,
                                         f32, f32, f32, i32, p, sz, i32, p, p]
     lib.pa_paged_decode_fp8.restype = i32
+    lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64, i32, p, p]
+    lib.pa_swap_blocks.restype = i32
     lib.pa_status_string.argtypes = [i32]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
@@ -256,3 +259,25 @@ def pa_paged_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens
         num_blocks, int(max_context_len), float(scale), float(k_scale), float(v_scale),
         int(partition_size), _ptr(workspace), ws_bytes, _dtype(query), _ptr(d_status),
         _stream(stream)))
+
+
+def _addr(t) -> int:
+    """Device-usable address of a CUDA tensor or a pinned host tensor (on a
+    system with unified addressing the pinned host pointer is the device
+    pointer)."""
+    if t is None:
+        return None
+    if not t.is_cuda and not t.is_pinned():
+        raise ValueError("host pools must be pinned memory")
+    return t.data_ptr()
+
+
+def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, d_status=None, stream=None) -> None:
+    """Whole-block copies src -> dst between two pools (one of them usually
+    a pinned host tensor): block_mapping int64 [P][2] of (src, dst) ids."""
+    src_nb, block_size, hkv, d = src_k.shape
+    dst_nb = dst_k.shape[0]
+    _check("pa_swap_blocks", LIB.pa_swap_blocks(
+        _addr(src_k), _addr(src_v), _addr(dst_k), _addr(dst_v), _addr(block_mapping),
+        int(block_mapping.shape[0]), hkv, d, block_size, src_nb, dst_nb, _dtype(src_k),
+        _ptr(d_status), _stream(stream)))

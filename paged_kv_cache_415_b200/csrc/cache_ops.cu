@@ -168,6 +168,60 @@ __global__ void __launch_bounds__(kCopyThreads) copy_blocks_kernel(
     }
 }
 
+// Grid (pair, K-or-V, chunk of the block).  Whole-block bit copy from one
+// pool to another, either of which may be pinned host memory reached over
+// the host link ([VM-paging, 显存管理与调度策略设计], eviction to CPU memory and
+// back).  Every thread keeps kSwapVecsPerThread 16-byte loads in flight, so
+// the link's read latency is covered.  The first CTA of each pair checks
+// the pair against the others (repeated destinations; with one shared pool,
+// also destinations that other pairs read).
+constexpr int kSwapThreads = 256;
+constexpr int kSwapVecsPerThread = 8;
+
+__global__ void __launch_bounds__(kSwapThreads) swap_blocks_kernel(
+    const uint4* __restrict__ src_k, const uint4* __restrict__ src_v, uint4* __restrict__ dst_k,
+    uint4* __restrict__ dst_v, const int64_t* __restrict__ block_mapping, int32_t num_pairs,
+    int64_t block_vecs, int64_t src_num_blocks, int64_t dst_num_blocks, int32_t same_pool,
+    int32_t* d_status)
+{
+    grid_dependency_wait();
+    allow_dependents();
+    const int32_t pair = blockIdx.x;
+    const int64_t src = block_mapping[2 * pair];
+    const int64_t dst = block_mapping[2 * pair + 1];
+    const bool first_cta = blockIdx.y == 0 && blockIdx.z == 0;
+    if (src < 0 || src >= src_num_blocks || dst < 0 || dst >= dst_num_blocks) {
+        if (first_cta && threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_BLOCK);
+        return;
+    }
+    if (first_cta && d_status != nullptr) {
+        bool conflict = false;
+        for (int32_t j = threadIdx.x; j < num_pairs; j += blockDim.x) {
+            if (j == pair) continue;
+            const int64_t sj = block_mapping[2 * j], dj = block_mapping[2 * j + 1];
+            if (dj == dst && j < pair) conflict = true;
+            if (same_pool && sj == dst && sj != dj) conflict = true;
+        }
+        if (__syncthreads_or(conflict) && threadIdx.x == 0) status_or(d_status, PA_STATUS_COPY_CONFLICT);
+    }
+    if (same_pool && src == dst) return;
+    const uint4* s = (blockIdx.y == 0 ? src_k : src_v) + src * block_vecs;
+    uint4* d = (blockIdx.y == 0 ? dst_k : dst_v) + dst * block_vecs;
+    const int64_t begin = static_cast<int64_t>(blockIdx.z) * kSwapThreads * kSwapVecsPerThread;
+    const int64_t end = min(block_vecs, begin + static_cast<int64_t>(kSwapThreads) * kSwapVecsPerThread);
+    uint4 buf[kSwapVecsPerThread];
+#pragma unroll
+    for (int k = 0; k < kSwapVecsPerThread; ++k) {
+        const int64_t i = begin + threadIdx.x + static_cast<int64_t>(k) * kSwapThreads;
+        if (i < end) buf[k] = s[i];
+    }
+#pragma unroll
+    for (int k = 0; k < kSwapVecsPerThread; ++k) {
+        const int64_t i = begin + threadIdx.x + static_cast<int64_t>(k) * kSwapThreads;
+        if (i < end) d[i] = buf[k];
+    }
+}
+
 static pa_status check_pool_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                   int64_t num_blocks, int32_t dtype, bool allow_fp8 = false)
 {
@@ -270,4 +324,66 @@ extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value
                              static_cast<const uint4*>(value), static_cast<uint2*>(k_cache),
                              static_cast<uint2*>(v_cache), slot_mapping, row_vecs,
                              num_blocks * block_size, k_inv, v_inv, d_status);
+}
+
+namespace pa {
+// The address the device uses for p: device and managed memory as is,
+// pinned host memory through its mapping; anything else (pageable host
+// memory, an unknown pointer) is refused, so no kernel ever dereferences it.
+static bool device_address(const void* p, const void** out)
+{
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    switch (attr.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged:
+        *out = p;
+        return true;
+    case cudaMemoryTypeHost:
+        if (attr.devicePointer == nullptr) return false;
+        *out = attr.devicePointer;
+        return true;
+    default:
+        return false;
+    }
+}
+}  // namespace pa
+
+extern "C" pa_status pa_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                                    const int64_t* block_mapping, int32_t num_pairs,
+                                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                    int64_t src_num_blocks, int64_t dst_num_blocks, pa_dtype dtype,
+                                    int32_t* d_status, pa_stream_t stream)
+{
+    using namespace pa;
+    if (num_pairs < 0 || dst_num_blocks <= 0) return PA_ERR_INVALID_ARG;
+    pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, src_num_blocks, dtype, true);
+    if (st != PA_OK) return st;
+    if (!src_k || !src_v || !dst_k || !dst_v || !block_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v) ||
+        !aligned8(block_mapping) || (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    const void *sk, *sv, *dk, *dv, *map;
+    if (!device_address(src_k, &sk) || !device_address(src_v, &sv) ||
+        !device_address(dst_k, &dk) || !device_address(dst_v, &dv) ||
+        !device_address(block_mapping, &map))
+        return PA_ERR_INVALID_ARG;
+    const int elem_bytes = dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2;
+    const int64_t block_vecs =
+        static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes / 16;
+    const int64_t per_cta = static_cast<int64_t>(kSwapThreads) * kSwapVecsPerThread;
+    const int64_t chunks = (block_vecs + per_cta - 1) / per_cta;
+    if (chunks > 65535) return PA_ERR_UNSUPPORTED;
+    const int32_t same_pool = (src_k == dst_k && src_v == dst_v) ? 1 : 0;
+    dim3 grid(num_pairs, 2, static_cast<unsigned>(chunks));
+    return launch_overlapped(swap_blocks_kernel, grid, dim3(kSwapThreads), 0, stream,
+                             static_cast<const uint4*>(sk), static_cast<const uint4*>(sv),
+                             static_cast<uint4*>(const_cast<void*>(dk)),
+                             static_cast<uint4*>(const_cast<void*>(dv)),
+                             static_cast<const int64_t*>(map), num_pairs, block_vecs,
+                             src_num_blocks, dst_num_blocks, same_pool, d_status);
 }
