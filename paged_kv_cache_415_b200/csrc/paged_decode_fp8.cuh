@@ -80,6 +80,15 @@ __device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32
         : "r"(w));
 }
 
+// 2^x with the special-function unit's approximation (flushes subnormal
+// results to zero); the probabilities it produces are rounded to fp16 next.
+__device__ __forceinline__ float fp8_exp2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ void stmatrix_x2_trans(uint32_t smem_addr, uint32_t r0, uint32_t r1)
 {
     asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1, %2};"
@@ -295,24 +304,27 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
             const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
             const float ms0 = mn0 == -INFINITY ? 0.f : mn0;
             const float ms1 = mn1 == -INFINITY ? 0.f : mn1;
-            const float c0 = exp2f(m_run0 - ms0), c1 = exp2f(m_run1 - ms1);
+            const float c0 = fp8_exp2(m_run0 - ms0), c1 = fp8_exp2(m_run1 - ms1);
             m_run0 = mn0;
             m_run1 = mn1;
             // P rounds to fp16 for the tensor cores; the sums use the rounded values
-            const uint32_t pk0 = Elem<__half>::from_float2(exp2f(x0 - ms0), exp2f(x1 - ms1));
-            const uint32_t pk1 = Elem<__half>::from_float2(exp2f(x2 - ms0), exp2f(x3 - ms1));
+            const uint32_t pk0 = Elem<__half>::from_float2(fp8_exp2(x0 - ms0), fp8_exp2(x1 - ms1));
+            const uint32_t pk1 = Elem<__half>::from_float2(fp8_exp2(x2 - ms0), fp8_exp2(x3 - ms1));
             const float2 r0 = Elem<__half>::to_float2(pk0), r1 = Elem<__half>::to_float2(pk1);
             l_run0 = l_run0 * c0 + (r0.x + r1.x);
             l_run1 = l_run1 * c1 + (r0.y + r1.y);
             const float2 cc = make_float2(c0, c1);
+            // once the running maxima settle, most slices leave them unchanged
+            if (__any_sync(kFullMask, c0 != 1.f || c1 != 1.f)) {
 #pragma unroll
-            for (int mt = 0; mt < S::MT; ++mt) {
-                float2 u = __fmul2_rn(make_float2(o[mt][0], o[mt][1]), cc);
-                float2 v = __fmul2_rn(make_float2(o[mt][2], o[mt][3]), cc);
-                o[mt][0] = u.x;
-                o[mt][1] = u.y;
-                o[mt][2] = v.x;
-                o[mt][3] = v.y;
+                for (int mt = 0; mt < S::MT; ++mt) {
+                    float2 u = __fmul2_rn(make_float2(o[mt][0], o[mt][1]), cc);
+                    float2 v = __fmul2_rn(make_float2(o[mt][2], o[mt][3]), cc);
+                    o[mt][0] = u.x;
+                    o[mt][1] = u.y;
+                    o[mt][2] = v.x;
+                    o[mt][3] = v.y;
+                }
             }
 
             // ---- P (tokens x heads) -> P^T B fragments (heads x tokens) ----

@@ -7,7 +7,9 @@
 
 ``DecodeStep`` owns the scratch the step needs (the split-context workspace
 and a device status word), allocated once with torch, and issues the three
-C-ABI calls on one stream.  Pools of dtype uint8 hold e4m3 codes: the step
+C-ABI calls on one stream.  ``HostPipeline`` feeds a ``DecodeStep`` from
+pinned host buffers step after step with the host-device copies of one step
+overlapping the kernels of the previous one.  Pools of dtype uint8 hold e4m3 codes: the step
 then uses the quantising write and the e4m3 decode with the pools' scales.  ``run_from_host`` is the same step fed from
 pinned host buffers: it copies the step's inputs to the device, runs the
 step and copies the output back, all on the same stream.
@@ -94,3 +96,70 @@ class DecodeStep:
                  stream=s, fused_append=fused_append)
             host["out"].copy_(dev["out"], non_blocking=True)
         return host["out"]
+
+
+class HostPipeline:
+    """Runs a DecodeStep once per call of ``submit`` from pinned host inputs,
+    with the copies of consecutive steps overlapping the kernels.
+
+    Three streams: uploads (host -> device), the step's kernels, downloads
+    (device -> host).  Device inputs and outputs are double-buffered, so the
+    upload of step i+1 runs while step i computes, and the download of step
+    i's output runs while step i+1 computes.  Events order each buffer's
+    reuse: an upload into set b waits until the step that last read set b
+    has finished, a download waits for its step, and the step waits for its
+    upload.  Every step still copies all of its own inputs in and its output
+    out; only the waiting is overlapped.  Kernels of consecutive steps stay
+    in order on the compute stream (the cache writes of one step precede the
+    next step's reads).
+    """
+
+    def __init__(self, stepper: DecodeStep, dev_like: dict, device=None):
+        """dev_like: name -> device tensor giving the shape and dtype of each
+        input ('query', 'block_tables', 'context_lens' and the optional
+        'new_key', 'new_value', 'slot_mapping', 'block_mapping') and 'out'."""
+        self.stepper = stepper
+        dev = device if device is not None else stepper.k_cache.device
+        self.sets = [{k: torch.empty_like(t, device=dev) for k, t in dev_like.items()}
+                     for _ in range(2)]
+        self.up = torch.cuda.Stream(dev)
+        self.compute = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        self.uploaded = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.downloaded = [torch.cuda.Event() for _ in range(2)]
+        self.used = [False, False]
+        self.i = 0
+
+    def submit(self, host: dict, scale, host_out: torch.Tensor, fused_append=False):
+        """Enqueue one step: host holds pinned inputs by name, host_out the
+        pinned tensor that receives the output.  Returns without waiting;
+        host_out is valid after ``synchronize`` (or the download stream's
+        work up to this step) completes.  The host input tensors must not be
+        modified until the upload of this step has run."""
+        b = self.i % 2
+        dev = self.sets[b]
+        if self.used[b]:
+            self.up.wait_event(self.computed[b])        # the step that last read set b
+            self.compute.wait_event(self.downloaded[b])  # its output has left set b's 'out'
+        with torch.cuda.stream(self.up):
+            for name, h in host.items():
+                dev[name].copy_(h, non_blocking=True)
+            self.uploaded[b].record(self.up)
+        self.compute.wait_event(self.uploaded[b])
+        self.stepper(dev["query"], dev["block_tables"], dev["context_lens"], scale, out=dev["out"],
+                     new_key=dev.get("new_key"), new_value=dev.get("new_value"),
+                     slot_mapping=dev.get("slot_mapping"), block_mapping=dev.get("block_mapping"),
+                     stream=self.compute, fused_append=fused_append)
+        self.computed[b].record(self.compute)
+        self.down.wait_event(self.computed[b])
+        with torch.cuda.stream(self.down):
+            host_out.copy_(dev["out"], non_blocking=True)
+            self.downloaded[b].record(self.down)
+        self.used[b] = True
+        self.i += 1
+        return host_out
+
+    def synchronize(self):
+        for st in (self.up, self.compute, self.down):
+            st.synchronize()

@@ -1,0 +1,75 @@
+"""The step API from pinned host buffers: DecodeStep.run_from_host (one
+stream, blocking order) and HostPipeline (uploads, kernels and downloads on
+three streams, double-buffered).  Both must give, step by step, exactly the
+output of the device-resident step, and that output must match the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from tests import oracle_pins
+from tests.gpu_utils import DeviceWorkload, assert_close, oracle_step, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _host_inputs(wl, query_bits, fused):
+    host = {"query": torch.from_numpy(query_bits.view(np.int16)).view(torch.float16).pin_memory(),
+            "block_tables": torch.from_numpy(wl.block_tables).pin_memory(),
+            "context_lens": torch.from_numpy(wl.context_lens).pin_memory(),
+            "new_key": torch.from_numpy(wl.new_key.view(np.int16)).view(torch.float16).pin_memory(),
+            "new_value": torch.from_numpy(wl.new_value.view(np.int16)).view(torch.float16).pin_memory()}
+    if not fused:
+        host["slot_mapping"] = torch.from_numpy(wl.slot_mapping).pin_memory()
+    return host
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-append", "separate"])
+def test_pipelined_steps_match_device_steps(fused):
+    """Six steps, each with its own query, through HostPipeline: every
+    step's host output equals the device-resident step on the same query
+    (bit for bit), and the first one matches the oracle."""
+    from paged_kv_cache_415_b200.step import DecodeStep, HostPipeline
+    wl = oracle_pins.small_llama(seqs=6)
+    assert wl.extra["one_token_per_seq"]
+    rng = np.random.Generator(np.random.PCG64(31))
+    queries = [wl.query] + [rng.integers(0, 1 << 15, size=wl.query.shape, dtype=np.uint16) & 0xBBFF
+                            for _ in range(5)]             # finite fp16 patterns
+    dw = DeviceWorkload(wl)
+    stepper = DecodeStep(dw.k_cache, dw.v_cache, wl.num_seqs, wl.num_q_heads,
+                         wl.max_context_len, 64)
+    like = {"query": dw.query, "block_tables": dw.block_tables, "context_lens": dw.context_lens,
+            "new_key": dw.new_key, "new_value": dw.new_value, "out": dw.query}
+    if not fused:
+        like["slot_mapping"] = dw.slot_mapping
+    pipe = HostPipeline(stepper, like)
+    outs = [torch.empty(wl.query.shape, dtype=torch.float16).pin_memory() for _ in queries]
+    hosts = [_host_inputs(wl, q, fused) for q in queries]
+    for h, o in zip(hosts, outs):
+        pipe.submit(h, wl.scale, o, fused_append=fused)
+    pipe.synchronize()
+    assert int(stepper.d_status.item()) == 0
+    # reference: the same steps on device-resident inputs, one stream
+    for q, o in zip(queries, outs):
+        dq = torch.from_numpy(q.view(np.int16)).cuda().view(torch.float16)
+        ref = stepper(dq, dw.block_tables, dw.context_lens, wl.scale, new_key=dw.new_key,
+                      new_value=dw.new_value, slot_mapping=dw.slot_mapping,
+                      fused_append=fused)
+        torch.cuda.synchronize()
+        assert torch.equal(ref.cpu().view(torch.int16), o.view(torch.int16))
+    _, _, want, _ = oracle_step(wl)
+    assert_close(to_f64(outs[0]), want, "pipelined step 0")
+
+
+def test_run_from_host_blocking_order():
+    from paged_kv_cache_415_b200.step import DecodeStep
+    wl = oracle_pins.small_llama(seqs=4)
+    dw = DeviceWorkload(wl)
+    stepper = DecodeStep(dw.k_cache, dw.v_cache, wl.num_seqs, wl.num_q_heads,
+                         wl.max_context_len, 0)
+    host = _host_inputs(wl, wl.query, fused=False)
+    host["out"] = torch.empty(wl.query.shape, dtype=torch.float16).pin_memory()
+    dev = {k: torch.empty_like(v, device="cuda") for k, v in host.items()}
+    out = stepper.run_from_host(host, dev, wl.scale)
+    torch.cuda.synchronize()
+    _, _, want, _ = oracle_step(wl)
+    assert_close(to_f64(out), want, "run_from_host")
