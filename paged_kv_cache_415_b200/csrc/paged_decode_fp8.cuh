@@ -39,10 +39,7 @@ struct Fp8Shape {
     static constexpr bool SWIZZLE = (D == 128);      // 128-byte rows, 128B TMA swizzle
     static constexpr int TILE = BS * D;              // bytes of one K (or V) tile of one head
     static constexpr int STAGE = 2 * TILE;
-#ifndef PA_FP8_NSTAGE
-#define PA_FP8_NSTAGE 3
-#endif
-    static constexpr int NSTAGE = STAGE <= 4096 ? PA_FP8_NSTAGE : 2;
+    static constexpr int NSTAGE = STAGE <= 4096 ? 3 : 2;
     static constexpr int PT_STRIDE = 48;             // bytes per head row of the P^T tile
     static constexpr int PT_BYTES = 8 * PT_STRIDE;
     static constexpr int WARP_BYTES = NSTAGE * STAGE;
@@ -116,101 +113,33 @@ __device__ __forceinline__ void load_words(const unsigned char* tile, int row, i
     w[3] = v.w;
 }
 
+// One warp's share of a (sequence, kv head, partition) unit: Q^T fragments,
+// the O^T accumulators and the online-softmax state of heads 2*tig and
+// 2*tig + 1 (rows of N), and the code that consumes one block of K/V bytes.
 template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
-    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-    T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
-    const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
-    int64_t num_blocks, int32_t max_context_len, float scale_log2, float v_scale,
-    int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
-    float2* __restrict__ ws_ml, int32_t* d_status, int32_t lpt_seqs)
-{
-    grid_dependency_wait();   // before any global access (see pa_common.cuh)
+struct Fp8Warp {
     using S = Fp8Shape<D, BS, G>;
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    int grp, tig;
+    uint32_t pt_addr;               // this lane's row of the P^T staging tile
+    uint32_t qb[S::KW][2];
+    float o[S::MT][4];
+    float m_run0, m_run1;           // running maxima (log2 units)
+    float l_run0, l_run1;           // this lane's share of the exp-sums
 
-    const int kvh = blockIdx.x;
-    const int part = blockIdx.y;
-    const int s = lpt_seqs > 0 ? lpt_sequence(context_lens, lpt_seqs, blockIdx.z,
-                                              reinterpret_cast<int32_t*>(smem))
-                               : static_cast<int>(blockIdx.z);
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int grp = lane >> 2;
-    const int tig = lane & 3;
-
-    const int32_t ctx = context_lens[s];
-    if (ctx < 0 || ctx > max_context_len ||
-        static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * BS) {
-        if (part == 0) {
-            write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
-            if (threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_CONTEXT);
-        }
-        return;
-    }
-    if (ctx == 0) {
-        if (part == 0) write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
-        return;
-    }
-    const int tok_begin = part * partition_size;
-    if (tok_begin >= ctx) return;
-    const int tok_end = min(ctx, tok_begin + partition_size);
-    const int nparts = (ctx + partition_size - 1) / partition_size;
-    const int blk_begin = tok_begin / BS;
-    const int nblk = (tok_end - tok_begin + BS - 1) / BS;
-    const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
-
-    unsigned char* wbase = smem + warp * S::WARP_BYTES;
-    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
-    if (lane == 0) {
+    __device__ __forceinline__ void reset()
+    {
 #pragma unroll
-        for (int st = 0; st < S::NSTAGE; ++st) mbar_init(&wbar[st], 1);
-        fence_barrier_init();
+        for (int mt = 0; mt < S::MT; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
+        m_run0 = m_run1 = -INFINITY;
+        l_run0 = l_run1 = 0.f;
     }
-    __syncwarp();
-
-    const int32_t* table = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq + blk_begin;
-    auto load_table = [&](int chunk) -> int {
-        const int kk = chunk * 32 + lane;
-        return kk < nk ? table[warp + kWarps * kk] : -1;
-    };
-    int prod_chunk = 0, cons_chunk = 0;
-    int prod_tbl = load_table(0);
-    int cons_tbl = prod_tbl;
-    auto block_tokens = [&](int k) -> int {
-        const int t0 = tok_begin + (warp + kWarps * k) * BS;
-        return min(BS, tok_end - t0);
-    };
-    auto issue = [&](int k) {
-        const int chunk = k >> 5;
-        if (chunk != prod_chunk) {
-            prod_tbl = load_table(chunk);
-            prod_chunk = chunk;
-        }
-        const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
-        if (lane == 0) {
-            const int st = k % S::NSTAGE;
-            const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
-            fence_proxy_async_smem();
-            if (ok) {
-                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE);
-                unsigned char* dst = wbase + st * S::STAGE;
-                tma_load_4d(dst, &tm_k, 0, kvh, 0, phys, &wbar[st]);
-                tma_load_4d(dst + S::TILE, &tm_v, 0, kvh, 0, phys, &wbar[st]);
-            } else {
-                status_or(d_status, PA_STATUS_BAD_BLOCK);
-                mbar_arrive_expect_tx(&wbar[st], 0u);
-            }
-        }
-    };
-    const int prologue = min(nk, S::NSTAGE);
-    for (int k = 0; k < prologue; ++k) issue(k);
-    int issued = prologue;
 
     // Q^T as B fragments, fp16: k-step j holds head grp's dims
     // (D/4)*tig + 4j .. +3, the same dims the lane's K words carry.
-    uint32_t qb[S::KW][2];
+    __device__ __forceinline__ void load_q(const T* __restrict__ query, int s, int kvh,
+                                           int num_q_heads)
     {
         const T* qrow = query + (static_cast<int64_t>(s) * num_q_heads + kvh * G + grp) * D +
                         (D / 4) * tig;
@@ -229,40 +158,10 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
         }
     }
 
-    // P^T staging rows: lanes 0-7 address head rows of tokens 0-7, lanes
-    // 8-15 the same rows' tokens 8-15 (lanes 16-31 repeat them).
-    const uint32_t pt_addr = smem_u32(smem + S::OFF_PT + warp * S::PT_BYTES) +
-                             (lane & 7) * S::PT_STRIDE + ((lane >> 3) & 1) * 16;
-
-    float o[S::MT][4];
-#pragma unroll
-    for (int mt = 0; mt < S::MT; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
-    float m_run0 = -INFINITY, m_run1 = -INFINITY;   // heads 2*tig, 2*tig + 1 (log2 units)
-    float l_run0 = 0.f, l_run1 = 0.f;               // this lane's share of the exp-sums
-
-    bool aborted = false;
-    int first_pending = 0;
-
-    for (int k = 0; k < nk; ++k) {
-        const int st = k % S::NSTAGE;
-        if (!mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1)) {
-            aborted = true;
-            first_pending = k;
-            break;
-        }
-        const int chunk = k >> 5;
-        if (chunk != cons_chunk) {
-            cons_tbl = load_table(chunk);
-            cons_chunk = chunk;
-        }
-        const int phys = __shfl_sync(kFullMask, cons_tbl, k & 31);
-        const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
-        const int nv = ok ? block_tokens(k) : 0;
-        const unsigned char* kt = wbase + st * S::STAGE;
-        const unsigned char* vt = kt + S::TILE;
-
+    // One block: kt / vt are its K and V byte tiles, nv its valid tokens.
+    __device__ __forceinline__ void block(const unsigned char* kt, const unsigned char* vt, int nv,
+                                          float scale_log2)
+    {
 #pragma unroll 1
         for (int sl = 0; sl < S::SLICES; ++sl) {
             const int t0 = sl * 16;
@@ -389,6 +288,158 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
                 mma_16816<__half>(o[2 * q + 1], a0, a1, a2, a3, pb0, pb1);
             }
         }
+    }
+
+    // The warp's (max, exp-sum, output) of its heads into the epilogue area.
+    __device__ __forceinline__ void store(float* epi_o, float* epi_m, float* epi_l, int warp,
+                                          float v_scale)
+    {
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            l_run0 += __shfl_xor_sync(kFullMask, l_run0, m);
+            l_run1 += __shfl_xor_sync(kFullMask, l_run1, m);
+        }
+        const int h0 = 2 * tig, h1 = 2 * tig + 1;
+#pragma unroll
+        for (int q = 0; q < S::VQ; ++q) {
+            const int d = S::DPT * grp + 4 * q;
+            if (h0 < G)
+                *reinterpret_cast<float4*>(epi_o + (warp * G + h0) * D + d) =
+                    make_float4(o[2 * q][0] * v_scale, o[2 * q][2] * v_scale,
+                                o[2 * q + 1][0] * v_scale, o[2 * q + 1][2] * v_scale);
+            if (h1 < G)
+                *reinterpret_cast<float4*>(epi_o + (warp * G + h1) * D + d) =
+                    make_float4(o[2 * q][1] * v_scale, o[2 * q][3] * v_scale,
+                                o[2 * q + 1][1] * v_scale, o[2 * q + 1][3] * v_scale);
+        }
+        if (grp == 0) {
+            if (h0 < G) {
+                epi_m[warp * G + h0] = m_run0;
+                epi_l[warp * G + h0] = l_run0;
+            }
+            if (h1 < G) {
+                epi_m[warp * G + h1] = m_run1;
+                epi_l[warp * G + h1] = l_run1;
+            }
+        }
+    }
+};
+
+
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
+    const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
+    int64_t num_blocks, int32_t max_context_len, float scale_log2, float v_scale,
+    int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
+    float2* __restrict__ ws_ml, int32_t* d_status, int32_t lpt_seqs)
+{
+    grid_dependency_wait();   // before any global access (see pa_common.cuh)
+    using S = Fp8Shape<D, BS, G>;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+    const int kvh = blockIdx.x;
+    const int part = blockIdx.y;
+    const int s = lpt_seqs > 0 ? lpt_sequence(context_lens, lpt_seqs, blockIdx.z,
+                                              reinterpret_cast<int32_t*>(smem))
+                               : static_cast<int>(blockIdx.z);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int32_t ctx = context_lens[s];
+    if (ctx < 0 || ctx > max_context_len ||
+        static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * BS) {
+        if (part == 0) {
+            write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
+            if (threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_CONTEXT);
+        }
+        return;
+    }
+    if (ctx == 0) {
+        if (part == 0) write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
+        return;
+    }
+    const int tok_begin = part * partition_size;
+    if (tok_begin >= ctx) return;
+    const int tok_end = min(ctx, tok_begin + partition_size);
+    const int nparts = (ctx + partition_size - 1) / partition_size;
+    const int blk_begin = tok_begin / BS;
+    const int nblk = (tok_end - tok_begin + BS - 1) / BS;
+    const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
+
+    unsigned char* wbase = smem + warp * S::WARP_BYTES;
+    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
+    if (lane == 0) {
+#pragma unroll
+        for (int st = 0; st < S::NSTAGE; ++st) mbar_init(&wbar[st], 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+
+    const int32_t* table = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq + blk_begin;
+    auto load_table = [&](int chunk) -> int {
+        const int kk = chunk * 32 + lane;
+        return kk < nk ? table[warp + kWarps * kk] : -1;
+    };
+    int prod_chunk = 0, cons_chunk = 0;
+    int prod_tbl = load_table(0);
+    int cons_tbl = prod_tbl;
+    auto issue = [&](int k) {
+        const int chunk = k >> 5;
+        if (chunk != prod_chunk) {
+            prod_tbl = load_table(chunk);
+            prod_chunk = chunk;
+        }
+        const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
+        if (lane == 0) {
+            const int st = k % S::NSTAGE;
+            const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
+            fence_proxy_async_smem();
+            if (ok) {
+                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE);
+                unsigned char* dst = wbase + st * S::STAGE;
+                tma_load_4d(dst, &tm_k, 0, kvh, 0, phys, &wbar[st]);
+                tma_load_4d(dst + S::TILE, &tm_v, 0, kvh, 0, phys, &wbar[st]);
+            } else {
+                status_or(d_status, PA_STATUS_BAD_BLOCK);
+                mbar_arrive_expect_tx(&wbar[st], 0u);
+            }
+        }
+    };
+    const int prologue = min(nk, S::NSTAGE);
+    for (int k = 0; k < prologue; ++k) issue(k);
+    int issued = prologue;
+
+    Fp8Warp<T, D, BS, G> w;
+    w.grp = lane >> 2;
+    w.tig = lane & 3;
+    w.pt_addr = smem_u32(smem + S::OFF_PT + warp * S::PT_BYTES) + (lane & 7) * S::PT_STRIDE +
+                ((lane >> 3) & 1) * 16;
+    w.reset();
+    w.load_q(query, s, kvh, num_q_heads);
+
+    bool aborted = false;
+    int first_pending = 0;
+    for (int k = 0; k < nk; ++k) {
+        const int st = k % S::NSTAGE;
+        if (!mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1)) {
+            aborted = true;
+            first_pending = k;
+            break;
+        }
+        const int chunk = k >> 5;
+        if (chunk != cons_chunk) {
+            cons_tbl = load_table(chunk);
+            cons_chunk = chunk;
+        }
+        const int phys = __shfl_sync(kFullMask, cons_tbl, k & 31);
+        const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
+        const int t0 = tok_begin + (warp + kWarps * k) * BS;
+        const int nv = ok ? min(BS, tok_end - t0) : 0;
+        const unsigned char* kt = wbase + st * S::STAGE;
+        w.block(kt, kt + S::TILE, nv, scale_log2);
         __syncwarp();   // every lane is done with this stage
         if (issued < nk) issue(issued++);
     }
@@ -401,39 +452,11 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
         }
     }
 
-#pragma unroll
-    for (int m = 4; m < 32; m <<= 1) {
-        l_run0 += __shfl_xor_sync(kFullMask, l_run0, m);
-        l_run1 += __shfl_xor_sync(kFullMask, l_run1, m);
-    }
-
     __syncthreads();   // every warp is done with its stage buffers
     float* epi_o = reinterpret_cast<float*>(smem);   // [warp][g][D]
     float* epi_m = epi_o + kWarps * G * D;
     float* epi_l = epi_m + kWarps * G;
-    const int h0 = 2 * tig, h1 = 2 * tig + 1;
-#pragma unroll
-    for (int q = 0; q < S::VQ; ++q) {
-        const int d = S::DPT * grp + 4 * q;
-        if (h0 < G)
-            *reinterpret_cast<float4*>(epi_o + (warp * G + h0) * D + d) =
-                make_float4(o[2 * q][0] * v_scale, o[2 * q][2] * v_scale,
-                            o[2 * q + 1][0] * v_scale, o[2 * q + 1][2] * v_scale);
-        if (h1 < G)
-            *reinterpret_cast<float4*>(epi_o + (warp * G + h1) * D + d) =
-                make_float4(o[2 * q][1] * v_scale, o[2 * q][3] * v_scale,
-                            o[2 * q + 1][1] * v_scale, o[2 * q + 1][3] * v_scale);
-    }
-    if (grp == 0) {
-        if (h0 < G) {
-            epi_m[warp * G + h0] = m_run0;
-            epi_l[warp * G + h0] = l_run0;
-        }
-        if (h1 < G) {
-            epi_m[warp * G + h1] = m_run1;
-            epi_l[warp * G + h1] = l_run1;
-        }
-    }
+    w.store(epi_o, epi_m, epi_l, warp, v_scale);
     __syncthreads();
     merge_warps_and_store<T, D, G>(epi_o, epi_m, epi_l, out, ws_o, ws_ml, s, kvh, part, nparts,
                                    num_q_heads, max_parts);

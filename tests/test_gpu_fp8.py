@@ -240,6 +240,28 @@ def test_fp8_empty_context_and_bad_block():
     assert_close(to_f64(out), ref)
 
 
+def test_fp8_bad_context():
+    """A negative context gives a zero row and PA_STATUS_BAD_CONTEXT, the other
+    rows are unaffected, for a small batch and for one of 300 sequences."""
+    for seqs in (5, 300):
+        ctx = np.random.Generator(np.random.PCG64(seqs)).integers(1, 70, size=seqs, endpoint=True)
+        nb = int(sum(-(-int(c) // 16) for c in ctx)) + 8
+        wl = gen.make_decode("fp8-many", seed=81, dtype="bf16", context_lens=ctx, num_q_heads=4,
+                             num_kv_heads=2, head_dim=64, block_size=16, num_blocks=nb,
+                             scale=0.125, partition_size=32)
+        wl = gen.with_fp8_pools(wl, seed=45)
+        kc, vc, _ = _oracle_pools(wl)
+        wl.k_cache, wl.v_cache = kc, vc
+        dev = Fp8Device(wl)
+        bad = wl.context_lens.copy()
+        bad[1] = -3
+        out = dev.decode(context_lens=torch.from_numpy(bad).cuda())
+        ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, bad, wl.scale,
+                                          wl.dtype, dev.ks, dev.vs)
+        assert st == 4 and dev.status() == 4, (seqs, st, dev.status())
+        assert_close(to_f64(out), ref, f"{seqs} seqs")
+
+
 def test_fp8_deterministic():
     wl = _instance(128, 16, 4, "bf16")
     dev = Fp8Device(wl)
