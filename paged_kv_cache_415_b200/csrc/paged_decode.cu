@@ -134,21 +134,34 @@ __device__ __forceinline__ void write_zero_rows(T* out, int s, int kvh, int num_
 }
 
 // Longest-first dispatch.  The CTAs of a grid start in blockIdx order, so
-// when CTA z serves the sequence with the z-th longest context (ties by
-// index), the long contexts start first and the last wave holds the short
-// ones: the tail where few CTAs are left shrinks.  Every thread of the CTA
-// calls this before anything else uses `scratch` (num_seqs + 1 ints of
-// shared memory, reused afterwards); needs num_seqs <= blockDim.x.  The
-// mapping is a permutation, so each sequence is served exactly once; the
-// work of a (sequence, head, partition) does not depend on which CTA runs
-// it, so results are unchanged.
+// when CTA z serves the z-th sequence in order of decreasing context length
+// (ties by index), the long contexts start first and the last wave holds
+// the short ones: the tail where few CTAs are left shrinks.  A batch in
+// which adjacent sequences share their stored prefix (the same first
+// physical block, as the beams of one prompt) keeps the grid order instead:
+// there the CTAs of one group running together, reusing the shared blocks
+// in L2, is worth more than the order.  Every thread of the CTA calls this
+// before anything else uses `scratch` (num_seqs + 1 ints of shared memory,
+// reused afterwards); needs num_seqs <= blockDim.x.  The mapping is a
+// permutation, so each sequence is served exactly once; the work of a
+// (sequence, head, partition) does not depend on which CTA runs it, so
+// results are unchanged.
 __device__ __forceinline__ int lpt_sequence(const int32_t* __restrict__ context_lens,
-                                            int32_t num_seqs, int rank, int32_t* scratch)
+                                            const int32_t* __restrict__ block_tables,
+                                            int32_t max_blocks_per_seq, int32_t num_seqs,
+                                            int rank, int32_t* scratch)
 {
     const int t = threadIdx.x;
-    const int32_t c = t < num_seqs ? context_lens[t] : 0;
-    if (t < num_seqs) scratch[t] = c;
-    __syncthreads();
+    int32_t c = 0;
+    bool shares = false;
+    if (t < num_seqs) {
+        c = context_lens[t];
+        scratch[t] = c;
+        if (t > 0)
+            shares = block_tables[static_cast<int64_t>(t) * max_blocks_per_seq] ==
+                     block_tables[static_cast<int64_t>(t - 1) * max_blocks_per_seq];
+    }
+    if (__syncthreads_or(shares)) return rank;   // grid order; scratch is not read again
     if (t < num_seqs) {
         int r = 0;
         for (int j = 0; j < num_seqs; ++j) {
@@ -161,6 +174,21 @@ __device__ __forceinline__ int lpt_sequence(const int32_t* __restrict__ context_
     const int pick = scratch[num_seqs];
     __syncthreads();   // scratch is free again
     return pick;
+}
+
+// A warp's first chunk of table entries (blocks warp + kWarps * lane of the
+// partition), read before the context length is known: the index is checked
+// against the table row only, so the load is in bounds whatever the context,
+// and it overlaps the context-length load instead of following it.  Lanes
+// past the warp's block count discard their entry.
+__device__ __forceinline__ int prefetch_table_chunk(const int32_t* __restrict__ block_tables,
+                                                    int s, int max_blocks_per_seq, int blk_begin,
+                                                    int warp, int lane)
+{
+    const int idx = blk_begin + warp + kWarps * lane;
+    return idx < max_blocks_per_seq
+               ? block_tables[static_cast<int64_t>(s) * max_blocks_per_seq + idx]
+               : -1;
 }
 
 // Fused append: the warp that loads the block holding a sequence's new token
@@ -256,14 +284,17 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
 
     const int kvh = blockIdx.x;
     const int part = blockIdx.y;
-    const int s = lpt_seqs > 0 ? lpt_sequence(context_lens, lpt_seqs, blockIdx.z,
-                                              reinterpret_cast<int32_t*>(smem))
-                               : static_cast<int>(blockIdx.z);
+    const int s = lpt_seqs > 0
+                      ? lpt_sequence(context_lens, block_tables, max_blocks_per_seq, lpt_seqs,
+                                     blockIdx.z, reinterpret_cast<int32_t*>(smem))
+                      : static_cast<int>(blockIdx.z);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int c = lane % S::LPT;        // position within the token row
     const int r = lane / S::LPT;        // token row within a pass
 
+    const int pre_tbl = prefetch_table_chunk(block_tables, s, max_blocks_per_seq,
+                                             blockIdx.y * partition_size / BS, warp, lane);
     const int32_t ctx = context_lens[s];
     if (ctx < 0 || ctx > max_context_len ||
         static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * BS) {
@@ -307,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
         return kk < nk ? table[warp + kWarps * kk] : -1;
     };
     int prod_chunk = 0, cons_chunk = 0;
-    int prod_tbl = load_table(0);
+    int prod_tbl = lane < nk ? pre_tbl : -1;   // load_table(0), already in flight
     int cons_tbl = prod_tbl;
 
     auto block_tokens = [&](int k) -> int {   // valid tokens of the warp's k-th block
@@ -957,15 +988,18 @@ static bool supported_group(int32_t hq, int32_t hkv)
 
 // Partition length: the caller's; else the whole (block-rounded) context
 // when it is at most kMaxSinglePartition tokens and there are enough
-// (sequence, kv head) pairs to fill the GPU on their own; else about an
-// eighth of the longest context (so the longest sequences split into at
-// least 8 CTAs), as a power of two between kMinPartition and
+// (sequence, kv head) pairs to fill the GPU on their own; else about a
+// quarter of the longest context (so the longest sequences split into at
+// least 4 CTAs), as a power of two between kMinPartition and
 // kMaxPartition tokens (short enough to balance ragged contexts, long
-// enough to amortise each CTA's start-up).
+// enough to amortise each CTA's start-up), halved while the grid would
+// hold fewer than four CTAs per SM.  Fitted to partition sweeps of the
+// Mistral-7B-shaped and long-context workloads on B200.
 constexpr int kMinPartition = 512;
 constexpr int kMaxPartition = 2048;
 constexpr int kMaxSinglePartition = 2048;
 constexpr int64_t kFillUnits = 888;    // 148 SMs x 3 CTAs x 2 waves
+constexpr int64_t kFillSms = 148;
 
 static int32_t choose_partition(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
                                 int32_t max_context_len, int32_t requested)
@@ -977,7 +1011,10 @@ static int32_t choose_partition(int32_t num_seqs, int32_t num_kv_heads, int32_t 
     const int64_t units = static_cast<int64_t>(num_seqs) * num_kv_heads;
     if (max_context_len <= kMaxSinglePartition && units >= kFillUnits) return whole;
     int32_t p = kMinPartition;
-    while (p < kMaxPartition && p * 8 < max_context_len) p *= 2;
+    while (p < kMaxPartition && p * 4 < max_context_len) p *= 2;
+    // keep at least four CTAs per SM in the grid: halve while it is smaller
+    const int64_t floor_ctas = 4 * static_cast<int64_t>(kFillSms);
+    while (p > kMinPartition && units * ((max_context_len + p - 1) / p) < floor_ctas) p /= 2;
     p = p / block_size * block_size;
     return whole < p ? whole : p;
 }
@@ -1105,10 +1142,15 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.stream = stream;
     a.new_key = new_key;
     a.new_value = new_value;
-    // longest-first dispatch pays off once the grid spans more than about
-    // two CTAs per SM (a tail exists) and the batch fits one CTA's threads
+    // Longest-first dispatch pays off once the grid spans more than about two
+    // CTAs per SM (a tail exists) and the batch fits one CTA's threads.  Every
+    // CTA ranks the batch itself (about num_seqs steps per thread), which is
+    // small next to a whole context but not next to one partition of many:
+    // with split contexts it is kept to small batches.
     const int64_t ctas = static_cast<int64_t>(num_kv_heads) * max_parts * num_seqs;
-    if (num_seqs <= kThreads && ctas > 2 * static_cast<int64_t>(sm_count())) a.lpt_seqs = num_seqs;
+    if (num_seqs <= kThreads && ctas > 2 * static_cast<int64_t>(sm_count()) &&
+        (max_parts == 1 || num_seqs <= 32))
+        a.lpt_seqs = num_seqs;
     if (fp8)
         return dtype == PA_DTYPE_F16 ? dispatch_fp8<__half>(a, v_scale)
                                      : dispatch_fp8<__nv_bfloat16>(a, v_scale);

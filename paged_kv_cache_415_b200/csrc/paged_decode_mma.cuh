@@ -79,14 +79,17 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
 
     const int kvh = blockIdx.x;
     const int part = blockIdx.y;
-    const int s = lpt_seqs > 0 ? lpt_sequence(context_lens, lpt_seqs, blockIdx.z,
-                                              reinterpret_cast<int32_t*>(smem))
-                               : static_cast<int>(blockIdx.z);
+    const int s = lpt_seqs > 0
+                      ? lpt_sequence(context_lens, block_tables, max_blocks_per_seq, lpt_seqs,
+                                     blockIdx.z, reinterpret_cast<int32_t*>(smem))
+                      : static_cast<int>(blockIdx.z);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int grp = lane >> 2;          // row group of the mma fragments (head)
     const int tig = lane & 3;           // thread in group (column pair)
 
+    const int pre_tbl = prefetch_table_chunk(block_tables, s, max_blocks_per_seq,
+                                             blockIdx.y * partition_size / BS, warp, lane);
     const int32_t ctx = context_lens[s];
     if (ctx < 0 || ctx > max_context_len ||
         static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * BS) {
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
         return kk < nk ? table[warp + kWarps * kk] : -1;
     };
     int prod_chunk = 0, cons_chunk = 0;
-    int prod_tbl = load_table(0);
+    int prod_tbl = lane < nk ? pre_tbl : -1;   // load_table(0), already in flight
     int cons_tbl = prod_tbl;
 
     auto block_tokens = [&](int k) -> int {

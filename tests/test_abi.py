@@ -60,12 +60,15 @@ def test_partition_and_workspace_sizes(pa):
     assert ps(4, 2, 2, 64, 16, 40, 0) == 48 and ws(4, 2, 2, 64, 16, 40, 0) == 0
     # many (seq, kv head) pairs and contexts up to 2048: one partition per context
     assert ps(64, 32, 32, 128, 16, 1982, 0) == 1984 and ws(64, 32, 32, 128, 16, 1982, 0) == 0
-    # longer contexts: about 1/8 of the longest, a power of two in [512, 2048]
-    assert ps(256, 32, 8, 128, 16, 8192, 0) == 1024
+    # longer contexts: about 1/4 of the longest, a power of two in [512, 2048] ...
+    assert ps(256, 32, 8, 128, 16, 8192, 0) == 2048
+    assert ps(256, 32, 8, 128, 16, 3900, 0) == 1024
     assert ps(16, 32, 8, 128, 16, 32768, 0) == 2048
+    # ... halved while the grid would hold fewer than 4 x 148 CTAs
     assert ps(16, 32, 8, 128, 16, 3000, 0) == 512
+    assert ps(2, 32, 8, 128, 16, 32768, 0) == 512
     # workspace: (D + 2) floats per (seq, q head, partition)
-    assert ws(16, 32, 8, 128, 16, 32768, 0) == 16 * 32 * 16 * (128 + 2) * 4
+    assert ws(16, 32, 8, 128, 16, 32768, 0) == 16 * 32 * 16 * (128 + 2) * 4      # P = 2048
     assert ws(16, 32, 8, 128, 16, 32768, 1024) == 16 * 32 * 32 * (128 + 2) * 4
     # the caller's partition wins; it must be a multiple of block_size
     assert ps(1, 1, 1, 128, 16, 100, 32) == 32
