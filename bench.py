@@ -77,6 +77,10 @@ def parse_args():
     ap.add_argument("--swap", choices=["out", "in"], default=None,
                     help="measure pa_swap_blocks instead of the decode step: 512 LLaMA-7B-shaped "
                          "blocks (K and V, 256 KB a pair) device -> pinned host (out) or back (in)")
+    ap.add_argument("--eager", action="store_true",
+                    help="issue every launch from the host in the timed region (default: the "
+                         "step's cache operations and its decode are captured into two CUDA "
+                         "graphs once and replayed)")
     ap.add_argument("--seqs", type=int, default=0,
                     help="shrink the batch (and the pool) for profiling; 0 = the full workload")
     return ap.parse_args()
@@ -427,6 +431,25 @@ def run_ours(args):
         cache_ops()
         decode()
     barrier()
+    run_cache, run_decode = cache_ops, decode
+    if not args.eager:
+        # the step's launches captured once; replay issues them with no host work
+        g_cache, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        has_cache = bool(n_pairs or (wl.num_new_tokens and not fused))
+        saved = stream
+        with torch.cuda.graph(g_dec):
+            stream = torch.cuda.current_stream(dev)
+            decode()
+        if has_cache:
+            with torch.cuda.graph(g_cache):
+                stream = torch.cuda.current_stream(dev)
+                cache_ops()
+        stream = saved
+        run_cache = g_cache.replay if has_cache else (lambda: None)
+        run_decode = g_dec.replay
+        run_cache()
+        run_decode()
+        barrier()
     if int(d_status.item()) != 0 or not torch.isfinite(out.float()).all():
         raise SystemExit(f"rank {rank}: bad step (status {int(d_status.item())})")
 
@@ -439,9 +462,9 @@ def run_ours(args):
     with sampler:
         start.record(stream)
         for i in range(args.steps):
-            cache_ops()
+            run_cache()
             ev[i][0].record(stream)
-            decode()
+            run_decode()
             ev[i][1].record(stream)
         stop.record(stream)
         torch.cuda.synchronize(dev)
@@ -547,6 +570,7 @@ def run_ours(args):
         "clocks": clocks,
         "cpu_baseline": cpu,
         "bytes_per_step": step,
+        "launch": "eager" if args.eager else "CUDA-graph replay (cache ops graph, decode graph)",
         "decode_entry": ("pa_reshape_and_cache_fp8 + pa_paged_decode_fp8" if fp8 else
                          "pa_paged_decode_shared_prefix" if shared else
                          "pa_paged_decode_append (cache write fused)" if fused else

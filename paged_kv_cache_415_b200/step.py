@@ -79,6 +79,26 @@ class DecodeStep:
                           scale, self.partition_size, self.workspace, self.d_status, stream)
         return out
 
+    def graph(self, query, block_tables, context_lens, scale, out, new_key=None, new_value=None,
+              slot_mapping=None, block_mapping=None, fused_append=False):
+        """Capture one step on these device buffers into a CUDA graph and
+        return it (``torch.cuda.CUDAGraph``); ``replay()`` re-runs the step's
+        launches with no host work per launch.  The step runs once eagerly on
+        a side stream first, so every per-kernel setting is in place before
+        capture.  Refill the captured buffers in place between replays."""
+        args = dict(out=out, new_key=new_key, new_value=new_value, slot_mapping=slot_mapping,
+                    block_mapping=block_mapping, fused_append=fused_append)
+        side = torch.cuda.Stream(device=query.device)
+        side.wait_stream(torch.cuda.current_stream(query.device))
+        with torch.cuda.stream(side):
+            self(query, block_tables, context_lens, scale, stream=side, **args)
+        torch.cuda.current_stream(query.device).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self(query, block_tables, context_lens, scale,
+                 stream=torch.cuda.current_stream(query.device), **args)
+        return g
+
     def run_from_host(self, host: dict, dev: dict, scale, stream=None, fused_append=False):
         """host / dev: dicts of same-shaped tensors (pinned host / device) for
         'query', 'block_tables', 'context_lens', 'new_key', 'new_value',

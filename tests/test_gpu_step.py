@@ -8,6 +8,7 @@ import torch
 
 from tests import oracle_pins
 from tests.gpu_utils import DeviceWorkload, assert_close, oracle_step, to_f64
+from workloads import generators as gen
 
 pytestmark = pytest.mark.gpu
 
@@ -73,3 +74,34 @@ def test_run_from_host_blocking_order():
     torch.cuda.synchronize()
     _, _, want, _ = oracle_step(wl)
     assert_close(to_f64(out), want, "run_from_host")
+
+
+@pytest.mark.parametrize("make", [gen.tiny, lambda: oracle_pins.small_gqa(seqs=6)],
+                         ids=["tiny-copies", "gqa-split"])
+def test_graph_replay_matches_eager(make):
+    """A step captured into a CUDA graph (block copies, cache write, decode
+    and, for split contexts, the merge) replays to exactly the eager step's
+    output, also after the captured query buffer is refilled."""
+    from paged_kv_cache_415_b200.step import DecodeStep
+    wl = make()
+    dw = DeviceWorkload(wl)
+    part = 64 if wl.max_context_len > 64 else 0
+    stepper = DecodeStep(dw.k_cache, dw.v_cache, wl.num_seqs, wl.num_q_heads,
+                         wl.max_context_len, part)
+    kw = dict(new_key=dw.new_key, new_value=dw.new_value, slot_mapping=dw.slot_mapping,
+              block_mapping=dw.block_mapping if wl.block_mapping.shape[0] else None)
+    eager = stepper(dw.query, dw.block_tables, dw.context_lens, wl.scale, **kw).clone()
+    out = torch.empty_like(dw.query)
+    g = stepper.graph(dw.query, dw.block_tables, dw.context_lens, wl.scale, out, **kw)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+    _, _, want, _ = oracle_step(wl)
+    assert_close(to_f64(out), want, "graph replay")
+    q2 = torch.flip(dw.query, dims=[0]).contiguous()
+    ref2 = stepper(q2, dw.block_tables, dw.context_lens, wl.scale, **kw).clone()
+    dw.query.copy_(q2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
+    assert int(stepper.d_status.item()) == 0
