@@ -45,8 +45,10 @@ def test_append_mha(partition):
     _check(oracle_pins.small_llama(seqs=6), partition)
 
 
-@pytest.mark.parametrize("partition", [0, 48, 256])
+@pytest.mark.parametrize("partition", [0, 16, 48, 256])
 def test_append_gqa_tensor_core_path(partition):
+    """16-token partitions split every context into many; the appended row
+    is written by a warp of the last one."""
     _check(oracle_pins.small_gqa(), partition)
 
 

@@ -146,6 +146,28 @@ def test_empty_and_invalid_contexts():
     assert not to_f64(out)[s_long].any()
 
 
+@pytest.mark.parametrize("partition", [16, 0], ids=["many-partitions", "auto"])
+def test_gqa_empty_invalid_contexts_and_bad_block(partition):
+    """The tensor-core path, with contexts split into many 16-token
+    partitions and with the library's partition:
+    ctx 0 -> zero row; negative ctx -> zero row + bit 4; an out-of-pool block
+    id -> skipped + bit 1; every other row as the oracle."""
+    wl = oracle_pins.small_gqa(seqs=6)
+    kc, vc = oracle_pins.pool_after_step(wl)
+    wl.k_cache, wl.v_cache = kc, vc
+    dw = DeviceWorkload(wl)
+    ctx = wl.context_lens.copy()
+    ctx[0], ctx[2] = 0, -3
+    tables = wl.block_tables.copy()
+    s_long = int(np.argmax(ctx))
+    tables[s_long, 1] = wl.num_blocks + 5
+    out = dw.decode(context_lens=torch.from_numpy(ctx).cuda(),
+                    block_tables=torch.from_numpy(tables).cuda(), partition_size=partition)
+    ref, st = oracle.paged_decode(wl.query, kc, vc, tables, ctx, wl.scale, wl.dtype)
+    assert st == 5 and dw.status() == 5
+    assert_close(to_f64(out), ref)
+
+
 def test_bad_block_id_is_skipped_and_flagged():
     wl = oracle_pins.small_llama(seqs=4)
     kc, vc = oracle_pins.pool_after_step(wl)
