@@ -379,13 +379,13 @@ def run_ours(args):
     n_pairs = int(wl.block_mapping.shape[0])
     stream = torch.cuda.current_stream(dev)
 
-    fused = (not args.separate and not args.shared_prefix and not fp8
+    fused = (not args.separate and not args.shared_prefix
              and wl.extra.get("one_token_per_seq", False) and wl.num_new_tokens == wl.num_seqs)
 
     def cache_ops():
         if n_pairs:
             B.pa_copy_blocks(k_cache, v_cache, block_mapping, d_status, stream)
-        if wl.num_new_tokens and fp8:
+        if wl.num_new_tokens and fp8 and not fused:
             B.pa_reshape_and_cache_fp8(new_key, new_value, k_cache, v_cache, slot_mapping,
                                        k_scale, v_scale, d_status, stream)
         elif wl.num_new_tokens and not fused:
@@ -403,7 +403,11 @@ def run_ours(args):
         workspace = torch.empty(max(sws, 16), dtype=torch.uint8, device=dev)
 
     def decode():
-        if fp8:
+        if fp8 and fused:
+            B.pa_paged_decode_fp8_append(out, query, new_key, new_value, k_cache, v_cache,
+                                         block_tables, context_lens, mcl, wl.scale, k_scale,
+                                         v_scale, part, workspace, d_status, stream)
+        elif fp8:
             B.pa_paged_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, mcl,
                                   wl.scale, k_scale, v_scale, part, workspace, d_status, stream)
         elif fused:
@@ -571,7 +575,9 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "bytes_per_step": step,
         "launch": "eager" if args.eager else "CUDA-graph replay (cache ops graph, decode graph)",
-        "decode_entry": ("pa_reshape_and_cache_fp8 + pa_paged_decode_fp8" if fp8 else
+        "decode_entry": ("pa_paged_decode_fp8_append (quantising cache write fused)"
+                         if fp8 and fused else
+                         "pa_reshape_and_cache_fp8 + pa_paged_decode_fp8" if fp8 else
                          "pa_paged_decode_shared_prefix" if shared else
                          "pa_paged_decode_append (cache write fused)" if fused else
                          "pa_reshape_and_cache + pa_paged_decode"),

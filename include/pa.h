@@ -347,6 +347,25 @@ PA_API pa_status pa_paged_decode_fp8(void* out, const void* query, const void* k
                                      int32_t* d_status, pa_stream_t stream);
 
 /*
+ * pa_paged_decode_fp8_append -- pa_paged_decode_append over FP8 pools: each
+ * sequence's new token (key, value of `dtype`, [num_seqs][num_kv_heads]
+ * [head_dim], 16-byte aligned) is quantised exactly as
+ * pa_reshape_and_cache_fp8 does and written to its slot (the position
+ * context_lens[s] - 1 of its own block table) inside the decode launch,
+ * then attended to with the other tokens.  Arguments, results and errors as
+ * pa_paged_decode_fp8 and pa_paged_decode_append; a table entry outside the
+ * pool for the new token sets PA_STATUS_BAD_SLOT and the token is not
+ * written.
+ */
+PA_API pa_status pa_paged_decode_fp8_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale,
+    float k_scale, float v_scale, int32_t partition_size, void* workspace, size_t workspace_bytes,
+    pa_dtype dtype, int32_t* d_status, pa_stream_t stream);
+
+/*
  * pa_paged_decode_shared_prefix -- pa_paged_decode for batches whose
  * sequences come in groups that share a stored prefix (the beams of one
  * prompt, parallel samples of one request).

@@ -36,7 +36,7 @@ EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_
            "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_paged_decode_no_alloc",
            "pa_paged_decode_shared_prefix_workspace_size", "pa_paged_decode_shared_prefix",
            "pa_paged_decode_append", "pa_reshape_and_cache_fp8", "pa_paged_decode_fp8",
-           "pa_swap_blocks",
+           "pa_paged_decode_fp8_append", "pa_swap_blocks",
            "pa_status_string", "pa_version")
 # Size of the library-owned scratch of pa_paged_decode_no_alloc.
 PA_NO_ALLOC_WORKSPACE_BYTES = 32 << 20
@@ -83,6 +83,9 @@ def _load() -> ctypes.CDLL:
     lib.pa_paged_decode_fp8.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64, i32,
                                         f32, f32, f32, i32, p, sz, i32, p, p]
     lib.pa_paged_decode_fp8.restype = i32
+    lib.pa_paged_decode_fp8_append.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, i32, i32,
+                                               i32, i64, i32, f32, f32, f32, i32, p, sz, i32, p, p]
+    lib.pa_paged_decode_fp8_append.restype = i32
     lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64, i32, p, p]
     lib.pa_swap_blocks.restype = i32
     lib.pa_status_string.argtypes = [i32]
@@ -260,6 +263,22 @@ def pa_paged_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens
         int(partition_size), _ptr(workspace), ws_bytes, _dtype(query), _ptr(d_status),
         _stream(stream)))
 
+
+def pa_paged_decode_fp8_append(out, query, key, value, k_cache, v_cache, block_tables,
+                               context_lens, max_context_len, scale, k_scale, v_scale,
+                               partition_size=0, workspace=None, d_status=None,
+                               stream=None) -> None:
+    """pa_paged_decode_fp8 with each sequence's new token (key/value
+    [S][Hkv][D], fp16/bf16) quantised into its slot inside the launch."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_paged_decode_fp8_append", LIB.pa_paged_decode_fp8_append(
+        _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), num_seqs, hq, hkv, d, block_size,
+        int(block_tables.shape[1]), num_blocks, int(max_context_len), float(scale),
+        float(k_scale), float(v_scale), int(partition_size), _ptr(workspace), ws_bytes,
+        _dtype(query), _ptr(d_status), _stream(stream)))
 
 def _addr(t) -> int:
     """Device-usable address of a CUDA tensor or a pinned host tensor (on a

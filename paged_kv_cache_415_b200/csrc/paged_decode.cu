@@ -669,6 +669,7 @@ struct DecodeArgs {
     const void* new_key = nullptr;     // fused append (one token per sequence), or null
     const void* new_value = nullptr;
     int32_t lpt_seqs = 0;              // > 0: longest-first dispatch over this many sequences
+    float k_inv = 1.f, v_inv = 1.f;    // e4m3 pools: reciprocal scales of the fused write
 };
 
 constexpr int kMaxDevices = 64;
@@ -810,7 +811,10 @@ static pa_status launch_decode_fp8(const DecodeArgs& a, float v_scale)
         kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v, static_cast<T*>(a.out),
         static_cast<const T*>(a.query), a.block_tables, a.context_lens, a.num_q_heads,
         a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2, v_scale,
-        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status, a.lpt_seqs);
+        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status, a.lpt_seqs,
+        static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
+        static_cast<uint8_t*>(const_cast<void*>(a.k_cache)),
+        static_cast<uint8_t*>(const_cast<void*>(a.v_cache)), a.num_kv_heads, a.k_inv, a.v_inv);
     if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
@@ -1142,6 +1146,10 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.stream = stream;
     a.new_key = new_key;
     a.new_value = new_value;
+    if (fp8) {
+        a.k_inv = 1.0f / k_scale;      // the quantising write's fp32(1 / scale)
+        a.v_inv = 1.0f / v_scale;
+    }
     // Longest-first dispatch pays off once the grid spans more than about two
     // CTAs per SM (a tail exists) and the batch fits one CTA's threads.  Every
     // CTA ranks the batch itself (about num_seqs steps per thread), which is
@@ -1191,6 +1199,22 @@ extern "C" pa_status pa_paged_decode_fp8(void* out, const void* query, const voi
                            num_blocks, max_context_len, scale, partition_size, workspace,
                            workspace_bytes, dtype, d_status, stream, nullptr, nullptr, true,
                            k_scale, v_scale);
+}
+
+extern "C" pa_status pa_paged_decode_fp8_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale,
+    float k_scale, float v_scale, int32_t partition_size, void* workspace, size_t workspace_bytes,
+    pa_dtype dtype, int32_t* d_status, pa_stream_t stream)
+{
+    if (key == nullptr || value == nullptr) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, key, value, true, k_scale,
+                           v_scale);
 }
 
 extern "C" pa_status pa_paged_decode_append(void* out, const void* query, const void* key,

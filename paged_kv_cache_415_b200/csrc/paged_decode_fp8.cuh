@@ -102,6 +102,42 @@ __device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, uint32_t
                  : "memory");
 }
 
+// Fused cache write for e4m3 pools: the warp that loads the block holding a
+// sequence's new token first quantises that token's K and V row for its kv
+// head exactly as the cache-write kernel does (fp32(x) * fp32(1 / scale),
+// round to nearest even, saturating at +-448) and stores the codes, then
+// makes the writes visible to the tensor-copy engine before the block's
+// tiles are requested.  Warp-uniform.
+template <typename T, int D, int BS>
+__device__ __forceinline__ void append_row_warp_fp8(
+    const T* __restrict__ new_key, const T* __restrict__ new_value, uint8_t* __restrict__ k_cache,
+    uint8_t* __restrict__ v_cache, int s, int kvh, int num_kv_heads, int32_t pos, int32_t phys,
+    float k_inv, float v_inv, int lane)
+{
+    const int64_t slot = static_cast<int64_t>(phys) * BS + pos % BS;
+    const int64_t src = (static_cast<int64_t>(s) * num_kv_heads + kvh) * D;
+    const int64_t dst = (slot * num_kv_heads + kvh) * D;
+    auto quant8 = [](const uint4& w, float inv) -> uint2 {
+        float f[8];
+        unpack8<T>(w, f);
+        uint32_t r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            r[j] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
+                make_float2(f[2 * j] * inv, f[2 * j + 1] * inv), __NV_SATFINITE, __NV_E4M3));
+        return make_uint2(r[0] | (r[1] << 16), r[2] | (r[3] << 16));
+    };
+    if (lane < D / 8) {
+        const uint4 kv = ld_nc_v4(new_key + src + lane * 8);
+        const uint4 vv = ld_nc_v4(new_value + src + lane * 8);
+        *reinterpret_cast<uint2*>(k_cache + dst + lane * 8) = quant8(kv, k_inv);
+        *reinterpret_cast<uint2*>(v_cache + dst + lane * 8) = quant8(vv, v_inv);
+        fence_proxy_async_global();
+    }
+    __syncwarp();
+    fence_proxy_async_global();
+}
+
 template <int D>
 __device__ __forceinline__ void load_words(const unsigned char* tile, int row, int byte,
                                            uint32_t (&w)[4])
@@ -333,7 +369,9 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
     const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
     int64_t num_blocks, int32_t max_context_len, float scale_log2, float v_scale,
     int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
-    float2* __restrict__ ws_ml, int32_t* d_status, int32_t lpt_seqs)
+    float2* __restrict__ ws_ml, int32_t* d_status, int32_t lpt_seqs,
+    const T* __restrict__ new_key, const T* __restrict__ new_value, uint8_t* __restrict__ k_cache,
+    uint8_t* __restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = Fp8Shape<D, BS, G>;
@@ -371,6 +409,8 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
     const int blk_begin = tok_begin / BS;
     const int nblk = (tok_end - tok_begin + BS - 1) / BS;
     const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
+    // the block (of this partition) holding the new token, when appending
+    const int append_blk = (new_key != nullptr && part == nparts - 1) ? (ctx - 1) / BS - blk_begin : -1;
 
     unsigned char* wbase = smem + warp * S::WARP_BYTES;
     uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
@@ -396,6 +436,13 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
             prod_chunk = chunk;
         }
         const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
+        if (warp + kWarps * k == append_blk) {
+            if (phys >= 0 && static_cast<int64_t>(phys) < num_blocks)
+                append_row_warp_fp8<T, D, BS>(new_key, new_value, k_cache, v_cache, s, kvh,
+                                              num_kv_heads, ctx - 1, phys, k_inv, v_inv, lane);
+            else if (lane == 0)
+                status_or(d_status, PA_STATUS_BAD_SLOT);
+        }
         if (lane == 0) {
             const int st = k % S::NSTAGE;
             const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;

@@ -58,7 +58,11 @@ class DecodeStep:
         mcl = self.max_context_len if max_context_len is None else max_context_len
         if self.fp8:
             if fused_append:
-                raise B.PAError("pa_paged_decode_append", B.PA_ERR_UNSUPPORTED)
+                B.pa_paged_decode_fp8_append(out, query, new_key, new_value, self.k_cache,
+                                             self.v_cache, block_tables, context_lens, mcl, scale,
+                                             self.k_scale, self.v_scale, self.partition_size,
+                                             self.workspace, self.d_status, stream)
+                return out
             if slot_mapping is not None and slot_mapping.shape[0] > 0:
                 B.pa_reshape_and_cache_fp8(new_key, new_value, self.k_cache, self.v_cache,
                                            slot_mapping, self.k_scale, self.v_scale,

@@ -278,3 +278,61 @@ def test_fp8_full_size(name):
     the benchmark times: write + decode against the whole oracle."""
     wl = gen.with_fp8_pools(gen.CONFIGS[name](), seed=44)
     _parity(wl, what=name + "-fp8")
+
+
+# ---- the quantising write fused into the decode launch ----------------------------
+
+def _fused(wl, partition_size=None, tables=None):
+    from paged_kv_cache_415_b200 import binding as B
+    dev = Fp8Device(wl)
+    p = wl.partition_size if partition_size is None else partition_size
+    ws_bytes = B.pa_paged_decode_workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                                wl.head_dim, wl.block_size, wl.max_context_len, p)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
+    out = torch.full_like(dev.query, float("nan"))
+    bt = dev.block_tables if tables is None else torch.from_numpy(tables).cuda()
+    B.pa_paged_decode_fp8_append(out, dev.query, dev.new_key, dev.new_value, dev.k_cache,
+                                 dev.v_cache, bt, dev.context_lens, wl.max_context_len, wl.scale,
+                                 dev.ks, dev.vs, p, ws, dev.d_status)
+    torch.cuda.synchronize()
+    return dev, out
+
+
+@pytest.mark.parametrize("head_dim,block_size,group,dtype,partition",
+                         [(128, 16, 1, "f16", 0), (128, 16, 4, "bf16", 64), (64, 32, 2, "f16", 0),
+                          (128, 32, 8, "bf16", 96)])
+def test_fp8_fused_append(head_dim, block_size, group, dtype, partition):
+    """pa_paged_decode_fp8_append leaves the pools exactly as the quantising
+    cache write does and returns the decode of the written pools."""
+    wl = _instance(head_dim, block_size, group, dtype)
+    assert wl.extra["one_token_per_seq"]
+    dev, out = _fused(wl, partition)
+    kc, vc, st = _oracle_pools(wl)
+    assert st == 0
+    assert np.array_equal(dev.k_cache.cpu().numpy(), kc)
+    assert np.array_equal(dev.v_cache.cpu().numpy(), vc)
+    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, wl.context_lens,
+                                      wl.scale, wl.dtype, dev.ks, dev.vs)
+    assert st == 0 and dev.status() == 0
+    assert_close(to_f64(out), ref, "fp8 fused append")
+
+
+def test_fp8_fused_append_bad_slot_is_flagged():
+    """A new token whose block id lies outside the pool is not written
+    (PA_STATUS_BAD_SLOT, plus PA_STATUS_BAD_BLOCK for the skipped block)."""
+    wl = _instance(128, 16, 4, "bf16")
+    s = int(np.argmax(wl.context_lens))
+    c = int(wl.context_lens[s])
+    tables = wl.block_tables.copy()
+    tables[s, (c - 1) // 16] = wl.num_blocks + 3
+    dev, _ = _fused(wl, 0, tables)
+    assert dev.status() & 2 and dev.status() & 1
+    # every other new token is written as the quantising write would
+    keep = np.ones(wl.num_seqs, bool)
+    keep[s] = False
+    kc, vc = wl.k_cache.copy(), wl.v_cache.copy()
+    oracle.reshape_and_cache_fp8(wl.new_key[keep], wl.new_value[keep], kc, vc,
+                                 wl.slot_mapping[keep], wl.block_size, wl.dtype,
+                                 wl.extra["k_scale"], wl.extra["v_scale"])
+    assert np.array_equal(dev.k_cache.cpu().numpy(), kc)
+    assert np.array_equal(dev.v_cache.cpu().numpy(), vc)
