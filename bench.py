@@ -502,14 +502,17 @@ def run_ours(args):
     d2h = host["out"].numel() * host["out"].element_size()
     host_out = host.pop("out")
     pipe = HostPipeline(stepper, devb, dev)
+    packed, views = pipe.host_buffer()
+    for name, t in host.items():
+        views[name].copy_(t)
     for _ in range(max(3, args.warmup)):
-        pipe.submit(host, wl.scale, host_out, fused_append=fused)
+        pipe.submit(packed, wl.scale, host_out, fused_append=fused)
     pipe.synchronize()
     barrier()
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e_start.record(pipe.up)
     for _ in range(args.steps):
-        pipe.submit(host, wl.scale, host_out, fused_append=fused)
+        pipe.submit(packed, wl.scale, host_out, fused_append=fused)
     e_stop.record(pipe.down)
     pipe.synchronize()
     torch.cuda.synchronize(dev)
@@ -567,9 +570,10 @@ def run_ours(args):
                      "avg_launch_us": round(decode_avg * 1e3, 2)},
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5),
-                "api": "step.HostPipeline: per step, pinned inputs uploaded on one stream, the "
-                       "step's kernels on another, the output downloaded on a third; "
-                       "double-buffered so copies overlap the neighbouring steps' kernels"},
+                "api": "step.HostPipeline: per step, the packed pinned inputs uploaded in one "
+                       "copy on one stream, the step's kernels on another, the output "
+                       "downloaded on a third; double-buffered so copies overlap the "
+                       "neighbouring steps' kernels"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "cpu_baseline": cpu,

@@ -126,26 +126,44 @@ class HostPipeline:
     """Runs a DecodeStep once per call of ``submit`` from pinned host inputs,
     with the copies of consecutive steps overlapping the kernels.
 
+    A step's inputs travel packed: ``host_buffer()`` hands out a pinned byte
+    buffer with named views ('query', 'block_tables', ... at 256-byte aligned
+    offsets) that the caller fills, and each step uploads it with one copy.
     Three streams: uploads (host -> device), the step's kernels, downloads
     (device -> host).  Device inputs and outputs are double-buffered, so the
     upload of step i+1 runs while step i computes, and the download of step
     i's output runs while step i+1 computes.  Events order each buffer's
-    reuse: an upload into set b waits until the step that last read set b
-    has finished, a download waits for its step, and the step waits for its
-    upload.  Every step still copies all of its own inputs in and its output
-    out; only the waiting is overlapped.  Kernels of consecutive steps stay
-    in order on the compute stream (the cache writes of one step precede the
-    next step's reads).
+    reuse: an upload into set b waits until the step that last read set b has
+    finished, the step waits for its upload (and for the download of the
+    output it overwrites), a download waits for its step.  Every step still
+    copies all of its own inputs in and its output out; only the waiting is
+    overlapped.  Kernels of consecutive steps stay in order on the compute
+    stream (the cache writes of one step precede the next step's reads).
+    With ``use_graphs`` the step's kernels are captured into a CUDA graph per
+    buffer set on that set's first use and replayed afterwards.
     """
 
-    def __init__(self, stepper: DecodeStep, dev_like: dict, device=None):
+    def __init__(self, stepper: DecodeStep, dev_like: dict, device=None, use_graphs=False):
         """dev_like: name -> device tensor giving the shape and dtype of each
         input ('query', 'block_tables', 'context_lens' and the optional
         'new_key', 'new_value', 'slot_mapping', 'block_mapping') and 'out'."""
         self.stepper = stepper
         dev = device if device is not None else stepper.k_cache.device
-        self.sets = [{k: torch.empty_like(t, device=dev) for k, t in dev_like.items()}
-                     for _ in range(2)]
+        self.layout = {}
+        off = 0
+        for name, t in dev_like.items():
+            if name == "out":
+                continue
+            nbytes = t.numel() * t.element_size()
+            self.layout[name] = (off, tuple(t.shape), t.dtype, nbytes)
+            off = (off + nbytes + 255) // 256 * 256
+        self.packed_bytes = max(off, 256)
+        self.sets = []
+        for _ in range(2):
+            buf = torch.empty(self.packed_bytes, dtype=torch.uint8, device=dev)
+            views = self._views(buf)
+            views["out"] = torch.empty_like(dev_like["out"], device=dev)
+            self.sets.append((buf, views))
         self.up = torch.cuda.Stream(dev)
         self.compute = torch.cuda.Stream(dev)
         self.down = torch.cuda.Stream(dev)
@@ -154,27 +172,53 @@ class HostPipeline:
         self.downloaded = [torch.cuda.Event() for _ in range(2)]
         self.used = [False, False]
         self.i = 0
+        self.use_graphs = use_graphs
+        self.graphs = {}
 
-    def submit(self, host: dict, scale, host_out: torch.Tensor, fused_append=False):
-        """Enqueue one step: host holds pinned inputs by name, host_out the
-        pinned tensor that receives the output.  Returns without waiting;
-        host_out is valid after ``synchronize`` (or the download stream's
-        work up to this step) completes.  The host input tensors must not be
-        modified until the upload of this step has run."""
+    def _views(self, buf: torch.Tensor) -> dict:
+        return {name: buf[off:off + nbytes].view(dtype).view(shape)
+                for name, (off, shape, dtype, nbytes) in self.layout.items()}
+
+    def host_buffer(self):
+        """(pinned byte buffer, {name: view}) in the packed input layout."""
+        buf = torch.empty(self.packed_bytes, dtype=torch.uint8).pin_memory()
+        return buf, self._views(buf)
+
+    def submit(self, host_packed: torch.Tensor, scale, host_out: torch.Tensor,
+               fused_append=False):
+        """Enqueue one step: host_packed is a buffer from ``host_buffer()``
+        holding this step's inputs, host_out the pinned tensor that receives
+        the output.  Returns without waiting; host_out is valid once
+        ``synchronize`` returns.  host_packed must not be modified until the
+        upload of this step has run."""
         b = self.i % 2
-        dev = self.sets[b]
+        dev_buf, dev = self.sets[b]
         if self.used[b]:
             self.up.wait_event(self.computed[b])        # the step that last read set b
             self.compute.wait_event(self.downloaded[b])  # its output has left set b's 'out'
         with torch.cuda.stream(self.up):
-            for name, h in host.items():
-                dev[name].copy_(h, non_blocking=True)
+            dev_buf.copy_(host_packed, non_blocking=True)
             self.uploaded[b].record(self.up)
         self.compute.wait_event(self.uploaded[b])
-        self.stepper(dev["query"], dev["block_tables"], dev["context_lens"], scale, out=dev["out"],
-                     new_key=dev.get("new_key"), new_value=dev.get("new_value"),
-                     slot_mapping=dev.get("slot_mapping"), block_mapping=dev.get("block_mapping"),
-                     stream=self.compute, fused_append=fused_append)
+        key = (b, float(scale), bool(fused_append))
+        graph = self.graphs.get(key)
+        step_args = dict(new_key=dev.get("new_key"), new_value=dev.get("new_value"),
+                         slot_mapping=dev.get("slot_mapping"),
+                         block_mapping=dev.get("block_mapping"), fused_append=fused_append)
+        if graph is not None:
+            with torch.cuda.stream(self.compute):
+                graph.replay()
+        else:
+            self.stepper(dev["query"], dev["block_tables"], dev["context_lens"], scale,
+                         out=dev["out"], stream=self.compute, **step_args)
+            if self.use_graphs:
+                # capture once the set holds a real step's inputs (the capture
+                # re-runs the step eagerly first; a step is idempotent on the
+                # same inputs: the same tokens into the same slots)
+                self.compute.synchronize()
+                self.graphs[key] = self.stepper.graph(dev["query"], dev["block_tables"],
+                                                      dev["context_lens"], scale, dev["out"],
+                                                      **step_args)
         self.computed[b].record(self.compute)
         self.down.wait_event(self.computed[b])
         with torch.cuda.stream(self.down):

@@ -26,9 +26,10 @@ def _host_inputs(wl, query_bits, fused):
 
 @pytest.mark.parametrize("fused", [True, False], ids=["fused-append", "separate"])
 def test_pipelined_steps_match_device_steps(fused):
-    """Six steps, each with its own query, through HostPipeline: every
-    step's host output equals the device-resident step on the same query
-    (bit for bit), and the first one matches the oracle."""
+    """Six steps, each with its own query, through HostPipeline (eager, then
+    with graph replays): every step's host output equals the device-resident
+    step on the same query (bit for bit), and the first one matches the
+    oracle."""
     from paged_kv_cache_415_b200.step import DecodeStep, HostPipeline
     wl = oracle_pins.small_llama(seqs=6)
     assert wl.extra["one_token_per_seq"]
@@ -42,12 +43,22 @@ def test_pipelined_steps_match_device_steps(fused):
             "new_key": dw.new_key, "new_value": dw.new_value, "out": dw.query}
     if not fused:
         like["slot_mapping"] = dw.slot_mapping
-    pipe = HostPipeline(stepper, like)
     outs = [torch.empty(wl.query.shape, dtype=torch.float16).pin_memory() for _ in queries]
-    hosts = [_host_inputs(wl, q, fused) for q in queries]
-    for h, o in zip(hosts, outs):
-        pipe.submit(h, wl.scale, o, fused_append=fused)
-    pipe.synchronize()
+    for graphs in (False, True):
+        pipe = HostPipeline(stepper, like, use_graphs=graphs)
+        packed = []
+        for q in queries:
+            buf, views = pipe.host_buffer()
+            for name, t in _host_inputs(wl, q, fused).items():
+                views[name].copy_(t)
+            packed.append(buf)
+        for buf, o in zip(packed, outs):
+            pipe.submit(buf, wl.scale, o, fused_append=fused)
+        pipe.synchronize()
+        if not graphs:
+            first = [o.clone() for o in outs]
+    for a, o in zip(first, outs):           # graph replays == eager steps
+        assert torch.equal(a.view(torch.int16), o.view(torch.int16))
     assert int(stepper.d_status.item()) == 0
     # reference: the same steps on device-resident inputs, one stream
     for q, o in zip(queries, outs):
