@@ -399,7 +399,7 @@ def run_ours(args):
         mpl = int(wl.extra["prefix_lens"].max())
         sws = B.pa_paged_decode_shared_prefix_workspace_size(
             wl.num_seqs, group_size, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
-            mcl, mpl, part)
+            mcl, mpl, 0)
         workspace = torch.empty(max(sws, 16), dtype=torch.uint8, device=dev)
 
     def decode():
@@ -417,13 +417,14 @@ def run_ours(args):
         elif shared:
             B.pa_paged_decode_shared_prefix(out, query, k_cache, v_cache, block_tables,
                                             context_lens, prefix_lens, group_size, mcl, mpl,
-                                            wl.scale, workspace, part, d_status, stream)
+                                            wl.scale, workspace, 0, d_status, stream)
         else:
             B.pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl,
                               wl.scale, part, workspace, d_status, stream)
 
+    shared_parts_gt1 = shared and sws > 0            # a reduction runs after the shared kernel
     launches_per_step = (1 if n_pairs else 0) + (1 if (wl.num_new_tokens and not fused) else 0) + \
-        1 + (1 if (max_parts > 1 or shared) else 0)
+        1 + (1 if (max_parts > 1 and not shared) or shared_parts_gt1 else 0)
 
     def barrier():
         if world > 1:
@@ -545,7 +546,8 @@ def run_ours(args):
         return 0
     group = wl.num_q_heads // wl.num_kv_heads
     if shared:
-        kernel_name = "paged_decode_shared_kernel + paged_decode_shared_reduce_kernel"
+        kernel_name = "paged_decode_shared_kernel" + (
+            " + paged_decode_shared_reduce_kernel" if shared_parts_gt1 else "")
     else:
         kernel_name = ("paged_decode_fp8_kernel" if fp8 else
                        "paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0

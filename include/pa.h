@@ -386,8 +386,14 @@ PA_API pa_status pa_paged_decode_fp8_append(
  * max_prefix_len host: upper bound of prefix_lens (sizes the grid).
  * group_size * (num_q_heads / num_kv_heads) must be at most 8 and
  * block_size 16 or 32 (else PA_ERR_UNSUPPORTED).
+ * Work split: each group's blocks form one list (the prefix blocks, then
+ * every member's own blocks); one CTA covers a part of that list for one kv
+ * head.  partition_size (0 = library's choice) is the part length in
+ * tokens of that list; a group whose list fits one part is written
+ * directly, others leave partials merged by a reduction kernel.
  * workspace      at least pa_paged_decode_shared_prefix_workspace_size(...)
- *                bytes, 16-byte aligned (always needed).
+ *                bytes, 16-byte aligned (may be NULL when that size is 0:
+ *                every group's list fits one part).
  * d_status       as pa_paged_decode; a group whose prefix is not a whole
  *                number of blocks or is longer than a member's context (or
  *                max_prefix_len) sets PA_STATUS_BAD_CONTEXT and gets zero

@@ -936,7 +936,7 @@ static pa_status dispatch_dim(const DecodeArgs& a)
 struct SharedArgs {
     DecodeArgs d;
     const int32_t* prefix_lens;
-    int32_t group_size, max_prefix_len, prefix_slots, slots;
+    int32_t group_size, max_prefix_len, part_blocks;
 };
 
 template <typename T, int D, int BS>
@@ -952,24 +952,21 @@ static pa_status launch_shared(const SharedArgs& sa)
         !encode_pool_map_swizzled(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
         return PA_ERR_CUDA;
     const int32_t num_groups = a.num_seqs / sa.group_size;
-    const int32_t parts = sa.slots - sa.prefix_slots > sa.prefix_slots ? sa.slots - sa.prefix_slots
-                                                                       : sa.prefix_slots;
-    dim3 grid(a.num_kv_heads, parts > 0 ? parts : 1, num_groups + a.num_seqs);
+    dim3 grid(a.num_kv_heads, a.max_parts, num_groups);
     pa_status st = launch_overlapped(
-        kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v,
-        static_cast<const T*>(a.query), a.block_tables, a.context_lens, sa.prefix_lens, num_groups,
+        kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v, static_cast<T*>(a.out),
+        static_cast<const T*>(a.query), a.block_tables, a.context_lens, sa.prefix_lens,
         sa.group_size, a.num_q_heads / a.num_kv_heads, a.num_q_heads, a.max_blocks_per_seq,
-        a.num_blocks, a.max_context_len, sa.max_prefix_len, a.scale_log2, a.partition_size,
-        sa.prefix_slots, sa.slots, a.ws_o, a.ws_ml, a.d_status);
-    if (st != PA_OK) return st;
+        a.num_blocks, a.max_context_len, sa.max_prefix_len, a.scale_log2, sa.part_blocks,
+        a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+    if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
     return launch_overlapped(paged_decode_shared_reduce_kernel<T, D>, dim3(ctas),
                              dim3(kReduceRowsPerCta * 32), 0, a.stream, static_cast<T*>(a.out),
                              a.ws_o, a.ws_ml, a.context_lens, sa.prefix_lens, a.num_seqs,
                              sa.group_size, a.num_q_heads, a.max_context_len, a.max_blocks_per_seq,
-                             a.block_size, sa.max_prefix_len, a.partition_size, sa.prefix_slots,
-                             sa.slots, a.d_status);
+                             a.block_size, sa.max_prefix_len, sa.part_blocks, a.max_parts);
 }
 
 template <typename T>
@@ -1257,12 +1254,23 @@ static pa_status check_shared_shape(int32_t num_seqs, int32_t group_size, int32_
     return PA_OK;
 }
 
-static void shared_slots(int32_t max_context_len, int32_t max_prefix_len, int32_t partition,
-                         int32_t* prefix_slots, int32_t* slots)
+// The shared-prefix path splits each group's block list (prefix blocks, then
+// every member's own): its partition is chosen as for a context as long as
+// the longest list can be (group_size x the longest context), over the
+// groups.  Returns the parts of the longest list.
+static int32_t shared_parts(int32_t num_seqs, int32_t group_size, int32_t num_kv_heads,
+                            int32_t block_size, int32_t max_context_len, int32_t partition_size,
+                            int32_t* part_blocks)
 {
-    *prefix_slots = (max_prefix_len + partition - 1) / partition;
-    const int32_t suffix = max_context_len > 0 ? (max_context_len + partition - 1) / partition : 1;
-    *slots = *prefix_slots + suffix;
+    const int64_t list_tokens = static_cast<int64_t>(group_size) * max_context_len;
+    const int32_t span = list_tokens > (1 << 30) ? (1 << 30) : static_cast<int32_t>(list_tokens);
+    const int32_t partition = choose_partition(num_seqs / group_size, num_kv_heads, block_size,
+                                               span, partition_size);
+    *part_blocks = partition / block_size;
+    const int64_t max_blocks = static_cast<int64_t>(group_size) *
+                               ((max_context_len + block_size - 1) / block_size);
+    const int64_t parts = (max_blocks + *part_blocks - 1) / *part_blocks;
+    return static_cast<int32_t>(parts < 1 ? 1 : parts > (1 << 30) ? (1 << 30) : parts);
 }
 
 }  // namespace pa
@@ -1276,11 +1284,11 @@ extern "C" size_t pa_paged_decode_shared_prefix_workspace_size(
     if (check_shared_shape(num_seqs, group_size, num_q_heads, num_kv_heads, head_dim, block_size,
                            max_context_len, max_prefix_len, partition_size) != PA_OK)
         return 0;
-    const int32_t p = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
-                                       partition_size);
-    int32_t prefix_slots, slots;
-    shared_slots(max_context_len, max_prefix_len, p, &prefix_slots, &slots);
-    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * slots;
+    int32_t part_blocks;
+    const int32_t parts = shared_parts(num_seqs, group_size, num_kv_heads, block_size,
+                                       max_context_len, partition_size, &part_blocks);
+    if (parts <= 1) return 0;
+    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * parts;
     return rows * head_dim * sizeof(float) + rows * sizeof(float2);
 }
 
@@ -1304,18 +1312,16 @@ extern "C" pa_status pa_paged_decode_shared_prefix(
         !aligned4(block_tables) || !aligned4(context_lens) || !aligned4(prefix_lens) ||
         (d_status && !aligned4(d_status)))
         return PA_ERR_INVALID_ARG;
-    const int32_t partition = choose_partition(num_seqs, num_kv_heads, block_size, max_context_len,
-                                               partition_size);
-    int32_t prefix_slots, slots;
-    shared_slots(max_context_len, max_prefix_len, partition, &prefix_slots, &slots);
+    int32_t part_blocks;
+    const int32_t parts = shared_parts(num_seqs, group_size, num_kv_heads, block_size,
+                                       max_context_len, partition_size, &part_blocks);
     const size_t need = pa_paged_decode_shared_prefix_workspace_size(
         num_seqs, group_size, num_q_heads, num_kv_heads, head_dim, block_size, max_context_len,
         max_prefix_len, partition_size);
     if (num_seqs == 0) return PA_OK;
-    if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
         return PA_ERR_INVALID_ARG;
-    const int64_t items = static_cast<int64_t>(num_seqs / group_size) + num_seqs;
-    if (items > 65535 || slots > 65535) return PA_ERR_UNSUPPORTED;
+    if (num_seqs / group_size > 65535 || parts > 65535) return PA_ERR_UNSUPPORTED;
 
     SharedArgs sa;
     DecodeArgs& a = sa.d;
@@ -1334,18 +1340,19 @@ extern "C" pa_status pa_paged_decode_shared_prefix(
     a.num_blocks = num_blocks;
     a.max_context_len = max_context_len;
     a.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-    a.partition_size = partition;
-    a.max_parts = slots;
-    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * slots;
-    a.ws_o = static_cast<float*>(workspace);
-    a.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + rows * head_dim * sizeof(float));
+    a.partition_size = part_blocks * block_size;
+    a.max_parts = parts;
+    const size_t rows = static_cast<size_t>(num_seqs) * num_q_heads * parts;
+    a.ws_o = need > 0 ? static_cast<float*>(workspace) : nullptr;
+    a.ws_ml = need > 0 ? reinterpret_cast<float2*>(static_cast<char*>(workspace) +
+                                                   rows * head_dim * sizeof(float))
+                       : nullptr;
     a.d_status = d_status;
     a.stream = stream;
     sa.prefix_lens = prefix_lens;
     sa.group_size = group_size;
     sa.max_prefix_len = max_prefix_len;
-    sa.prefix_slots = prefix_slots;
-    sa.slots = slots;
+    sa.part_blocks = part_blocks;
     return dtype == PA_DTYPE_F16 ? dispatch_shared<__half>(sa) : dispatch_shared<__nv_bfloat16>(sa);
 }
 

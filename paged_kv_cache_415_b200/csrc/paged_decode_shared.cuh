@@ -10,14 +10,16 @@
 // group: the members' query heads become extra rows of the tensor-core
 // tile, exactly as the query heads of a GQA group do.
 //
-// One launch covers two kinds of work item (blockIdx.z):
-//   z <  num_groups : the shared prefix [0, L) of group z, every member's
-//                     query rows at once (rows = members x G <= 8), K/V
-//                     through the first member's block table;
-//   z >= num_groups : the private suffix [L, ctx) of one sequence.
-// Both are split into context partitions and leave (max, exp-sum,
-// normalised output) partials in the workspace; a reduction kernel merges
-// each row's prefix and suffix partials with the rule of §5.1.
+// A work item is (kv head, part, group z).  The group's blocks form one list:
+// the prefix blocks [0, L / B) through the first member's table (every
+// member's rows of the tile live: rows = members x G <= 8), then each
+// member's private blocks [L / B, ceil(ctx / B)) in member order (only that
+// member's G rows live; the others' scores are masked out).  The list is
+// cut into parts of part_blocks blocks; a part's blocks are dealt
+// round-robin to the four warps.  A group whose list fits one part writes
+// its output rows directly; otherwise each part leaves (max, exp-sum,
+// normalised output) partials that a reduction merges with the rule of
+// §5.1.  So a private suffix costs no CTA of its own and no merge.
 
 namespace pa {
 
@@ -56,15 +58,25 @@ __device__ __forceinline__ bool prefix_ok(const int32_t* context_lens, int32_t L
     return true;
 }
 
+// Group z's list of blocks: the shared prefix, then each member's own.
+__device__ __forceinline__ int group_blocks(const int32_t* __restrict__ context_lens, int seq0,
+                                            int group_size, int nb_pre, int block_size)
+{
+    int total = nb_pre;
+    for (int j = 0; j < group_size; ++j)
+        total += (context_lens[seq0 + j] + block_size - 1) / block_size - nb_pre;
+    return total;
+}
+
 template <typename T, int D, int BS>
 __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-    const T* __restrict__ query, const int32_t* __restrict__ block_tables,
+    T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
     const int32_t* __restrict__ context_lens, const int32_t* __restrict__ prefix_lens,
-    int32_t num_groups, int32_t group_size, int32_t G, int32_t num_q_heads,
-    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
-    int32_t max_prefix_len, float scale_log2, int32_t partition_size, int32_t prefix_slots,
-    int32_t slots, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status)
+    int32_t group_size, int32_t G, int32_t num_q_heads, int32_t max_blocks_per_seq,
+    int64_t num_blocks, int32_t max_context_len, int32_t max_prefix_len, float scale_log2,
+    int32_t part_blocks, int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml,
+    int32_t* d_status)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = SharedShape<D, BS>;
@@ -79,24 +91,36 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
     const int grp = lane >> 2;
     const int tig = lane & 3;
     const int32_t max_tokens = max_blocks_per_seq * BS;
+    const int seq0 = z * group_size;
+    const int rows = group_size * G;
 
-    // ---- the work item: rows, token range, block table, output slot ----
-    const bool is_prefix = z < num_groups;
-    const int group = is_prefix ? z : (z - num_groups) / group_size;
-    const int seq0 = is_prefix ? z * group_size : z - num_groups;   // first row's sequence
-    const int rows = is_prefix ? group_size * G : G;
-    const int32_t L = prefix_lens[group];
-    if (!prefix_ok(context_lens, L, group, group_size, BS, max_prefix_len, max_context_len,
-                   max_tokens))
-        return;                              // the reduction reports it and writes zero rows
-    const int32_t ctx_end = is_prefix ? L : context_lens[seq0];
-    const int32_t start = is_prefix ? 0 : L;
-    const int tok_begin = start + part * partition_size;
-    if (tok_begin >= ctx_end) return;
-    const int tok_end = min(ctx_end, tok_begin + partition_size);
-    const int slot = is_prefix ? part : prefix_slots + part;
-    const int blk_begin = tok_begin / BS;
-    const int nblk = (tok_end - tok_begin + BS - 1) / BS;
+    // output rows of the group for this kv head, all zero
+    auto zero_rows = [&]() {
+        for (int idx = threadIdx.x; idx < rows * (D / 8); idx += kThreads) {
+            const int r = idx / (D / 8);
+            const int64_t row = static_cast<int64_t>(seq0 + r / G) * num_q_heads + kvh * G + r % G;
+            reinterpret_cast<uint4*>(out + row * D)[idx % (D / 8)] = make_uint4(0, 0, 0, 0);
+        }
+    };
+    const int32_t L = prefix_lens[z];
+    if (!prefix_ok(context_lens, L, z, group_size, BS, max_prefix_len, max_context_len,
+                   max_tokens)) {
+        if (part == 0) {
+            zero_rows();
+            if (threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_CONTEXT);
+        }
+        return;
+    }
+    const int nb_pre = L / BS;
+    const int total = group_blocks(context_lens, seq0, group_size, nb_pre, BS);
+    if (total == 0) {                        // every member's context is empty
+        if (part == 0) zero_rows();
+        return;
+    }
+    const int nparts = (total + part_blocks - 1) / part_blocks;
+    const int v_begin = part * part_blocks;
+    if (v_begin >= total) return;
+    const int nblk = min(part_blocks, total - v_begin);
     const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
 
     unsigned char* wstage = smem + warp * S::WARP_STAGE_BYTES;
@@ -108,37 +132,54 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
     }
     __syncwarp();
 
-    const int32_t* table = block_tables + static_cast<int64_t>(seq0) * max_blocks_per_seq + blk_begin;
-    const int members = is_prefix ? group_size : 1;
-    // One table entry per lane, 32 blocks per load; for a prefix, every
-    // member's entry must name the same physical block.
-    auto load_table = [&](int chunk) -> int {
+    // Block v of the list: its physical id and (valid tokens | (member + 1)
+    // << 8), member -1 for a shared prefix block.  Every member's entry for
+    // a prefix block must name the same physical block.
+    auto resolve = [&](int v, int& phys, int& info) {
+        if (v < nb_pre) {
+            const int32_t e = block_tables[static_cast<int64_t>(seq0) * max_blocks_per_seq + v];
+            bool same = true;
+            for (int m = 1; m < group_size; ++m)
+                same &= block_tables[static_cast<int64_t>(seq0 + m) * max_blocks_per_seq + v] == e;
+            if (!same) status_or(d_status, PA_STATUS_BAD_BLOCK);
+            phys = e;
+            info = BS;
+            return;
+        }
+        int r = v - nb_pre;
+        for (int j = 0; j < group_size; ++j) {
+            const int32_t c = context_lens[seq0 + j];
+            const int n = (c + BS - 1) / BS - nb_pre;
+            if (r < n) {
+                const int b = nb_pre + r;
+                phys = block_tables[static_cast<int64_t>(seq0 + j) * max_blocks_per_seq + b];
+                info = min(BS, c - b * BS) | ((j + 1) << 8);
+                return;
+            }
+            r -= n;
+        }
+        phys = -1;
+        info = 0;
+    };
+    // one list entry per lane, 32 blocks of this warp per load
+    auto load_chunk = [&](int chunk, int& phys, int& info) {
         const int kk = chunk * 32 + lane;
-        if (kk >= nk) return -1;
-        const int j = warp + kWarps * kk;
-        const int32_t e = table[j];
-        bool same = true;
-        for (int m = 1; m < members; ++m)
-            same &= table[static_cast<int64_t>(m) * max_blocks_per_seq + j] == e;
-        if (!same) status_or(d_status, PA_STATUS_BAD_BLOCK);
-        return e;
+        phys = -1;
+        info = 0;
+        if (kk < nk) resolve(v_begin + warp + kWarps * kk, phys, info);
     };
     int prod_chunk = 0, cons_chunk = 0;
-    int prod_tbl = load_table(0);
-    int cons_tbl = prod_tbl;
-
-    auto block_tokens = [&](int k) -> int {
-        const int t0 = tok_begin + (warp + kWarps * k) * BS;
-        return min(BS, tok_end - t0);
-    };
+    int prod_phys, prod_info;
+    load_chunk(0, prod_phys, prod_info);
+    int cons_phys = prod_phys, cons_info = prod_info;
 
     auto issue = [&](int k) {
         const int chunk = k >> 5;
         if (chunk != prod_chunk) {
-            prod_tbl = load_table(chunk);
+            load_chunk(chunk, prod_phys, prod_info);
             prod_chunk = chunk;
         }
-        const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
+        const int phys = __shfl_sync(kFullMask, prod_phys, k & 31);
         if (lane == 0) {
             const int st = k % S::NSTAGE;
             const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
@@ -161,6 +202,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
 
     // Row grp of the A operand: member grp / G's query head kvh * G + grp % G.
     const bool row_live = grp < rows;
+    const int row_member = row_live ? grp / G : -2;
     uint32_t qa[S::KSTEPS][2];
     {
         const int member = row_live ? grp / G : 0;
@@ -195,12 +237,16 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
         }
         const int chunk = k >> 5;
         if (chunk != cons_chunk) {
-            cons_tbl = load_table(chunk);
+            load_chunk(chunk, cons_phys, cons_info);
             cons_chunk = chunk;
         }
-        const int phys = __shfl_sync(kFullMask, cons_tbl, k & 31);
+        const int phys = __shfl_sync(kFullMask, cons_phys, k & 31);
+        const int info = __shfl_sync(kFullMask, cons_info, k & 31);
         const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
-        const int nv = ok ? block_tokens(k) : 0;
+        const int nv = ok ? (info & 0xff) : 0;
+        const int owner = (info >> 8) - 1;            // -1: shared by every member
+        // this lane's row takes part in this block's scores
+        const bool row_on = row_live && (owner < 0 || owner == row_member);
         unsigned char* ktile = wstage + st * S::STAGE_BYTES;
         unsigned char* vtile = ktile + S::TILE_BYTES;
         const uint32_t ks_base = smem_u32(ktile);
@@ -222,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
 #pragma unroll 1
         for (int sl = 0; sl < S::SLICES; ++sl) {
             const int t0 = sl * 16;
-            const int tv = nv - t0;
+            const int tv = row_on ? nv - t0 : 0;     // tokens this row may see
             float sc[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
@@ -303,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
     }
     __syncthreads();
 
-    // merge the warps in a fixed order; every row leaves a partial
+    // merge the warps in a fixed order: the output row, or this part's partial
     for (int idx = threadIdx.x; idx < rows * (D / 8); idx += kThreads) {
         const int r = idx / (D / 8);
         const int d0 = (idx % (D / 8)) * 8;
@@ -327,25 +373,31 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
             O[6] = fmaf(f, b.z, O[6]); O[7] = fmaf(f, b.w, O[7]);
         }
         const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) O[e] *= inv;
         const int64_t row = static_cast<int64_t>(seq0 + r / G) * num_q_heads + kvh * G + r % G;
-        const int64_t prow = row * slots + slot;
-        float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + d0);
-        dst[0] = make_float4(O[0] * inv, O[1] * inv, O[2] * inv, O[3] * inv);
-        dst[1] = make_float4(O[4] * inv, O[5] * inv, O[6] * inv, O[7] * inv);
-        if (d0 == 0) ws_ml[prow] = make_float2(M, Lsum);
+        if (nparts == 1) {
+            *reinterpret_cast<uint4*>(out + row * D + d0) = pack8<T>(O);
+        } else {
+            const int64_t prow = row * max_parts + part;
+            float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + d0);
+            dst[0] = make_float4(O[0], O[1], O[2], O[3]);
+            dst[1] = make_float4(O[4], O[5], O[6], O[7]);
+            if (d0 == 0) ws_ml[prow] = make_float2(M, Lsum);
+        }
     }
 }
 
-// One warp per (sequence, query head): merge the prefix partials (slots
-// [0, ceil(L / P))) and the suffix partials (slots [prefix_slots,
-// prefix_slots + ceil((ctx - L) / P))) into the output row.
+// One warp per (sequence, query head) of a group whose block list spans
+// several parts: merge the parts' partials into the output row.  Groups that
+// fit one part (or were refused) were written by the decode kernel.
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_shared_reduce_kernel(
     T* __restrict__ out, const float* __restrict__ ws_o, const float2* __restrict__ ws_ml,
     const int32_t* __restrict__ context_lens, const int32_t* __restrict__ prefix_lens,
     int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t max_context_len,
-    int32_t max_blocks_per_seq, int32_t block_size, int32_t max_prefix_len,
-    int32_t partition_size, int32_t prefix_slots, int32_t slots, int32_t* d_status)
+    int32_t max_blocks_per_seq, int32_t block_size, int32_t max_prefix_len, int32_t part_blocks,
+    int32_t max_parts)
 {
     grid_dependency_wait();
     constexpr int EPL = D / 32;
@@ -354,23 +406,17 @@ __global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_shared_re
     if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;
     const int s = static_cast<int>(row / num_q_heads);
     const int z = s / group_size;
-    const int32_t ctx = context_lens[s];
     const int32_t L = prefix_lens[z];
-    T* dst = out + row * D + lane * EPL;
     if (!prefix_ok(context_lens, L, z, group_size, block_size, max_prefix_len, max_context_len,
-                   max_blocks_per_seq * block_size)) {
-        if (lane == 0) status_or(d_status, PA_STATUS_BAD_CONTEXT);
-#pragma unroll
-        for (int e = 0; e < EPL; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = 0u;
+                   max_blocks_per_seq * block_size))
         return;
-    }
-    const int n_pre = (L + partition_size - 1) / partition_size;
-    const int n_suf = (ctx - L + partition_size - 1) / partition_size;
-    const int n = n_pre + n_suf;
-    auto slot_of = [&](int i) { return i < n_pre ? i : prefix_slots + (i - n_pre); };
-    const float2* ml = ws_ml + row * slots;
+    const int total = group_blocks(context_lens, z * group_size, group_size, L / block_size,
+                                   block_size);
+    const int n = (total + part_blocks - 1) / part_blocks;
+    if (n <= 1) return;
+    const float2* ml = ws_ml + row * max_parts;
     float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[slot_of(i)].x);
+    for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[i].x);
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, m));
     const float msub = M == -INFINITY ? 0.f : M;
@@ -378,16 +424,16 @@ __global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_shared_re
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
     float W = 0.f;
-    const float* orow = ws_o + row * slots * D + lane * EPL;
+    const float* orow = ws_o + row * max_parts * D + lane * EPL;
     for (int i = 0; i < n; ++i) {
-        const int sl = slot_of(i);
-        const float2 v = ml[sl];
+        const float2 v = ml[i];
         const float w = v.y * exp2f(v.x - msub);
         W += w;
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, orow[static_cast<int64_t>(sl) * D + e], acc[e]);
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, orow[static_cast<int64_t>(i) * D + e], acc[e]);
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
+    T* dst = out + row * D + lane * EPL;
 #pragma unroll
     for (int e = 0; e < EPL; e += 2)
         *reinterpret_cast<uint32_t*>(dst + e) = Elem<T>::from_float2(acc[e] * inv, acc[e + 1] * inv);
