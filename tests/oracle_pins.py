@@ -381,6 +381,36 @@ def pin_fp8_decode_equals_dequantised_fp16(lib):
     assert np.array_equal(a, b)
 
 
+def pin_fp8_decode_matches_numpy_attention(lib):
+    """Scales that are not powers of two: the fp8 decode equals numpy
+    softmax attention over K/V gathered through the tables and dequantised
+    with torch's e4m3 decoding times the scales (<= 1e-12)."""
+    torch = _torch_e4m3()
+    from scipy.special import softmax
+    wl = small_gqa(dtype="bf16", seqs=4, head_dim=64)
+    rng = np.random.Generator(np.random.PCG64(15))
+    kc = rng.integers(0, 256, size=wl.k_cache.shape).astype(np.uint8)
+    vc = rng.integers(0, 256, size=wl.v_cache.shape).astype(np.uint8)
+    for c in (kc, vc):
+        c[(c & 0x7f) == 0x7f] = 0x11                             # no NaN codes
+    ks, vs = 0.0371, 0.2113
+    got, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, wl.context_lens,
+                                      wl.scale, wl.dtype, ks, vs, lib=lib)
+    assert st == 0
+    deq = lambda c: torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    q = (torch.from_numpy(wl.query.view(np.int16)).view(torch.bfloat16)
+         .to(torch.float64).numpy())
+    b, group = wl.block_size, wl.num_q_heads // wl.num_kv_heads
+    for s in range(wl.num_seqs):
+        c = int(wl.context_lens[s])
+        pos = np.arange(c)
+        phys = wl.block_tables[s][pos // b]
+        k = np.repeat(deq(kc[phys, pos % b]) * ks, group, axis=1)      # scales as given
+        v = np.repeat(deq(vc[phys, pos % b]) * vs, group, axis=1)
+        w = softmax(wl.scale * np.einsum("hd,thd->ht", q[s], k), axis=1)
+        close(got[s], np.einsum("ht,thd->hd", w, v), 1e-12)
+
+
 # ---- swap_blocks (eviction to host memory and back) ---------------------------
 
 def pin_swap_round_trip(lib):

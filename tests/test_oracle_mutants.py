@@ -44,6 +44,8 @@ MUTANTS = {
     "swap_dst_index_of_src": ("dst_k[dst * block_bytes + b] = src_k[src * block_bytes + b];",
                               "dst_k[src % dst_num_blocks * block_bytes + b] = src_k[src * block_bytes + b];"),
     "swap_bad_id_not_flagged": ("            status |= 1;\n            continue;", "            continue;"),
+    "fp8_v_scaled_by_k_scale": ("(e4m3_to_f64(v_cache[r + d]) * v_scale)",
+                                "(e4m3_to_f64(v_cache[r + d]) * k_scale)"),
     "swap_no_conflict_check": ("if (block_mapping[2 * j + 1] == block_mapping[2 * i + 1]) status |= 8;", ""),
 }
 
