@@ -209,10 +209,11 @@ def pa_paged_decode_shared_prefix(out, query, k_cache, v_cache, block_tables, co
                                   workspace, partition_size=0, d_status=None, stream=None) -> None:
     """pa_paged_decode for groups of group_size consecutive sequences that
     share their first prefix_lens[g] tokens (int32 device tensor, one entry
-    per group, whole blocks)."""
+    per group, whole blocks).  workspace may be None when
+    pa_paged_decode_shared_prefix_workspace_size(...) is 0."""
     num_seqs, hq, d = query.shape
     num_blocks, block_size, hkv, _ = k_cache.shape
-    ws_bytes = workspace.numel() * workspace.element_size()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("pa_paged_decode_shared_prefix", LIB.pa_paged_decode_shared_prefix(
         _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
         _ptr(context_lens), _ptr(prefix_lens), num_seqs, int(group_size), hq, hkv, d, block_size,
