@@ -1,0 +1,58 @@
+"""Host-side logic of bench.py (no GPU): workload construction for every
+mode, the JSON config block, the byte accounting of the CPU legs and the
+committed profile lines the roofline object reads."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bench
+from workloads import byte_model as bm
+
+
+@pytest.mark.parametrize("config", ["tiny", "llama7b", "mistral7b", "long_context", "beam_search"])
+def test_small_workloads_and_config_block(config):
+    wl = bench.make_workload(config, seqs=4 if config != "tiny" else 0)
+    cfg = bench.workload_config(wl, 64, "note")
+    assert cfg["num_seqs"] == wl.num_seqs and cfg["partition_size"] == 64
+    for key in ("workload", "num_q_heads", "num_kv_heads", "head_dim", "block_size", "layers", "l2"):
+        assert key in cfg
+    assert cfg["workload"].startswith(wl.name)
+
+
+def test_fp8_workload_mode():
+    wl = bench.make_workload("llama7b", seqs=3, kv_dtype="fp8")
+    assert wl.extra["kv_dtype"] == "fp8" and wl.k_cache.dtype == np.uint8
+    assert "e4m3" in bench.workload_config(wl, 0, "")["workload"]
+    full = bm.step_bytes(wl)
+    base = bm.step_bytes(bench.make_workload("llama7b", seqs=3))
+    assert full["kv"] * 2 == base["kv"]
+
+
+def test_oracle_step_counts_the_step_bytes():
+    """The CPU leg times the oracle on the same step the GPU runs and
+    counts the same algorithmic bytes (all sequences, 16-bit and e4m3)."""
+    for kv in ("auto", "fp8"):
+        wl = bench.make_workload("llama7b", seqs=2, kv_dtype=kv)
+        st = bench.OracleStep(wl)
+        assert st.bytes == bm.step_bytes(wl)["total"]
+        assert st.run() > 0.0
+
+
+def test_committed_traffic_lines_parse():
+    """Every bench-traffic line under profiles/ has a workload, a byte count
+    and a source hash, and names one of the bench's workloads."""
+    names = {"tiny", "llama7b", "mistral7b", "long_context", "beam_search"}
+    found = 0
+    for name in os.listdir(bench.PROFILE_GLOB_DIR):
+        with open(os.path.join(bench.PROFILE_GLOB_DIR, name)) as f:
+            for line in f:
+                if line.startswith("bench-traffic:"):
+                    m = re.match(r"bench-traffic:\s*workload=(\S+)\s+bytes_per_launch=(\d+)\s+"
+                                 r"source_sha256=(\w{16})\s*$", line)
+                    assert m, line
+                    assert m.group(1).replace("-fp8", "") in names
+                    assert int(m.group(2)) > 0
+                    found += 1
+    assert found >= 3
