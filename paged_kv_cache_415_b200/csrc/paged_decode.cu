@@ -1,37 +1,41 @@
 // paged_decode.cu -- single-query attention over a paged KV cache (sm_100a).
 //
-// Kernel 1, paged_decode_kernel: one CTA per (kv head, context partition,
-// sequence).  The CTA carries the G = Hq / Hkv query heads of its kv head,
-// so every K/V byte is read from HBM once for all of them.  Each of its four
-// warps runs its own pipeline over every fourth physical block of the
-// partition:
-//   * the warp's block-table entries are prefetched into one register per
-//     lane (32 blocks per load) and broadcast with a shuffle
-//     ("PagedAttention：大模型KV Cache分页管理优化实践" §3.2: flattened table,
-//     warp-level prefetch);
-//   * each block's K and V rows of this kv head (block_size rows of
-//     head_dim elements each, one contiguous 128/256-byte row per token) are
-//     fetched by the bulk-copy engine (cp.async.bulk) straight into a shared
-//     memory ring of NSTAGE stages, completion counted on one mbarrier per
-//     stage, so NSTAGE - 1 blocks are in flight while one is computed
+// Kernel 1, paged_decode_kernel (query groups G < 4): one CTA per (kv head,
+// context partition, sequence).  The CTA carries the G = Hq / Hkv query heads
+// of its kv head, so every K/V byte is read from HBM once for all of them.
+// Each of its four warps runs its own pipeline over every fourth physical
+// block of the partition:
+//   * the warp's block-table entries sit one per lane (32 blocks per load,
+//     the first chunk read together with the context length) and are
+//     broadcast with a shuffle ("PagedAttention：大模型KV Cache分页管理优化实践"
+//     §3.2: flattened table, warp-level prefetch);
+//   * one lane requests each block's K and V tile of this kv head (block_size
+//     rows of head_dim elements) with two TMA tensor copies into the warp's
+//     shared-memory ring of NSTAGE stages, completion counted on one mbarrier
+//     per stage, so the next blocks are in flight while one is computed
 //     (§4.2 prefetch, §5.2 overlap of copy and compute);
-//   * scores q.k in fp32: 8 (or 16) lanes share a token row, each holding
-//     16 (or 8) elements of q for every head of the group in registers; the
-//     partial dot products are reduced across those lanes with a transposing
-//     butterfly of warp shuffles;
+//   * scores q.k in fp32 (fma.rn.f32 on the 16-bit operands): 8 (or 16)
+//     lanes share a token row and the partial dot products are reduced with
+//     a transposing butterfly of warp shuffles; scale * log2(e) multiplies
+//     the reduced score, so the exponentials are exp2;
 //   * the softmax is the blocked form of §5.1 (分块Softmax算法) run online:
-//     per block the local max, the running (global) max, the exp-sum
-//     rescaled to it, then the weighted V rows accumulate into fp32 outputs
-//     rescaled the same way; scores are kept in log2 units (q is
-//     pre-multiplied by scale * log2(e)) so exponentials are exp2.
+//     per tile the local max, the running (global) max, the exp-sum rescaled
+//     to it, then the weighted V rows accumulate into fp32 outputs rescaled
+//     the same way.
 // At the end the four warps' (max, sum, output) are merged through shared
 // memory in a fixed order.  A sequence whose context fits one partition gets
 // its output row written directly; otherwise the partition's max, sum and
-// normalised output go to the workspace.
+// normalised output go to the workspace.  With a fused append, the warp that
+// loads the block holding a sequence's new token writes that token's K/V row
+// first.  Small batches are dispatched longest context first (lpt_sequence).
 //
 // Kernel 2, paged_decode_reduce_kernel: one warp per (sequence, query head)
 // with more than one partition merges the partitions with the same rule:
 //   M = max_p m_p,  w_p = l_p * 2^(m_p - M),  out = sum_p w_p Ohat_p / sum_p w_p.
+//
+// The grouped-head (paged_decode_mma.cuh), e4m3 (paged_decode_fp8.cuh) and
+// shared-prefix (paged_decode_shared.cuh) kernels are included below; this
+// file also holds the host entry points and their launch logic.
 //
 // The whole computation has a fixed summation order, so results are
 // deterministic and do not depend on where the blocks sit in the pool.

@@ -56,3 +56,12 @@ def test_committed_traffic_lines_parse():
                     assert int(m.group(2)) > 0
                     found += 1
     assert found >= 3
+
+
+def test_source_hash_ignores_comments_only():
+    """The profile hash covers code, not comments: stripping removes // and
+    /* */ comments and blank lines, keeps string and character literals."""
+    src = 'int a = 1; // note\n/* block\n comment */ const char* s = "a//b"; char q = \'/\';\n\n'
+    assert bench.strip_comments(src) == 'int a = 1;\n const char* s = "a//b"; char q = \'/\';'
+    assert bench.strip_comments(src) == bench.strip_comments(src.replace("note", "other"))
+    assert bench.strip_comments(src) != bench.strip_comments(src.replace("a = 1", "a = 2"))
