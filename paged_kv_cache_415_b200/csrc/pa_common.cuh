@@ -1,8 +1,10 @@
 // pa_common.cuh -- device helpers shared by the library's kernels (sm_100a).
 //
-// Inline PTX wrappers for the asynchronous bulk copy engine (cp.async.bulk,
-// global -> shared, completion counted on an mbarrier), mbarrier waits that
-// give up after a bounded time, and fp16 / bf16 <-> fp32 conversions.
+// Inline PTX wrappers for the tensor-copy engine (TMA: cp.async.bulk.tensor
+// tiles, and the untiled cp.async.bulk, global -> shared, completion counted
+// on an mbarrier), mbarrier waits that give up after a bounded time,
+// programmatic dependent launch, ldmatrix and warp-level mma.sync, and
+// fp16 / bf16 <-> fp32 conversions.
 #pragma once
 
 #include <cuda_bf16.h>
