@@ -4,8 +4,9 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  The product library
 (``paged_kv_cache_415_b200``) never imports it and shares no code with it.
 
-``pa_oracle.c`` holds the definitions (reshape_and_cache, copy_blocks, paged
-decode in fp64); this module compiles it with gcc (``-O2``, OpenMP, no
+``pa_oracle.c`` holds the definitions (reshape_and_cache, copy_blocks,
+swap_blocks, paged decode in fp64; the e4m3 and int8 pools' encode, write and
+decode); this module compiles it with gcc (``-O2``, OpenMP, no
 fast-math) into ``liboracle.so`` beside it and wraps it with ctypes.
 ``brute.py`` holds pure-Python/numpy restatements used to pin it.
 
@@ -73,6 +74,16 @@ def load(path: str | None = None):
     lib.oracle_paged_decode_fp8.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64,
                                             f64, i32, f64, f64, i32]
     lib.oracle_paged_decode_fp8.restype = i32
+    lib.oracle_decode_int8.argtypes = [p, p, i64]
+    lib.oracle_decode_int8.restype = None
+    lib.oracle_encode_int8.argtypes = [p, p, i64]
+    lib.oracle_encode_int8.restype = None
+    lib.oracle_reshape_and_cache_int8.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i32,
+                                                  ctypes.c_float, ctypes.c_float]
+    lib.oracle_reshape_and_cache_int8.restype = i32
+    lib.oracle_paged_decode_int8.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32,
+                                             i64, f64, i32, f64, f64, i32]
+    lib.oracle_paged_decode_int8.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     if path is None:
@@ -198,31 +209,85 @@ def encode_e4m3(x: np.ndarray, lib=None) -> np.ndarray:
     return out
 
 
-def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, block_size, dtype,
-                          k_scale, v_scale, lib=None) -> int:
-    """Quantising cache write into uint8 pools [num_blocks][B][Hkv][D]."""
+def _code_bytes(a: np.ndarray) -> np.ndarray:
+    """An 8-bit pool (uint8 or int8) as contiguous raw bytes."""
+    a = np.ascontiguousarray(a)
+    assert a.dtype in (np.uint8, np.int8), f"expected 8-bit codes, got {a.dtype}"
+    return a.view(np.uint8)
+
+
+def _reshape_and_cache_q8(fn, key, value, k_cache, v_cache, slot_mapping, block_size, dtype,
+                          k_scale, v_scale):
     key, value = _u16(key), _u16(value)
-    assert k_cache.dtype == np.uint8 and v_cache.dtype == np.uint8
+    assert k_cache.dtype in (np.uint8, np.int8) and v_cache.dtype == k_cache.dtype
+    assert k_cache.flags["C_CONTIGUOUS"] and v_cache.flags["C_CONTIGUOUS"]
     slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
     num_blocks, bs, hkv, d = k_cache.shape
-    return int((lib or load()).oracle_reshape_and_cache_fp8(
-        _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
-        key.shape[0], hkv, d, block_size, num_blocks, _DTYPES[dtype], float(k_scale),
-        float(v_scale)))
+    return int(fn(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+                  key.shape[0], hkv, d, block_size, num_blocks, _DTYPES[dtype], float(k_scale),
+                  float(v_scale)))
 
 
-def paged_decode_fp8(query, k_cache, v_cache, block_tables, context_lens, scale, dtype, k_scale,
-                     v_scale, num_threads=0, lib=None):
-    """fp64 paged decode over e4m3 pools (dequantised with the scales)."""
+def _paged_decode_q8(fn, query, k_cache, v_cache, block_tables, context_lens, scale, dtype,
+                     k_scale, v_scale, num_threads):
     query = _u16(query)
     block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
     context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
     s, hq, d = query.shape
     num_blocks, bs, hkv, _ = k_cache.shape
     out = np.empty((s, hq, d), dtype=np.float64)
-    st = (lib or load()).oracle_paged_decode_fp8(
-        _ptr(out), _ptr(query), _ptr(np.ascontiguousarray(k_cache, dtype=np.uint8)),
-        _ptr(np.ascontiguousarray(v_cache, dtype=np.uint8)), _ptr(block_tables),
-        _ptr(context_lens), s, hq, hkv, d, bs, block_tables.shape[1], num_blocks, float(scale),
-        _DTYPES[dtype], float(k_scale), float(v_scale), num_threads)
+    st = fn(_ptr(out), _ptr(query), _ptr(_code_bytes(k_cache)), _ptr(_code_bytes(v_cache)),
+            _ptr(block_tables), _ptr(context_lens), s, hq, hkv, d, bs, block_tables.shape[1],
+            num_blocks, float(scale), _DTYPES[dtype], float(k_scale), float(v_scale), num_threads)
     return out, int(st)
+
+
+def reshape_and_cache_fp8(key, value, k_cache, v_cache, slot_mapping, block_size, dtype,
+                          k_scale, v_scale, lib=None) -> int:
+    """Quantising cache write into uint8 e4m3 pools [num_blocks][B][Hkv][D]."""
+    return _reshape_and_cache_q8((lib or load()).oracle_reshape_and_cache_fp8, key, value,
+                                 k_cache, v_cache, slot_mapping, block_size, dtype, k_scale,
+                                 v_scale)
+
+
+def paged_decode_fp8(query, k_cache, v_cache, block_tables, context_lens, scale, dtype, k_scale,
+                     v_scale, num_threads=0, lib=None):
+    """fp64 paged decode over e4m3 pools (dequantised with the scales)."""
+    return _paged_decode_q8((lib or load()).oracle_paged_decode_fp8, query, k_cache, v_cache,
+                            block_tables, context_lens, scale, dtype, k_scale, v_scale,
+                            num_threads)
+
+
+# ---- INT8 caches: two's-complement codes, per-tensor scales -------------------
+
+def decode_int8(codes: np.ndarray, lib=None) -> np.ndarray:
+    """int8 code (given as raw bytes, uint8 or int8) -> float64."""
+    codes = _code_bytes(codes)
+    out = np.empty(codes.shape, dtype=np.float64)
+    (lib or load()).oracle_decode_int8(_ptr(codes), _ptr(out), codes.size)
+    return out
+
+
+def encode_int8(x: np.ndarray, lib=None) -> np.ndarray:
+    """float32 -> int8 code (returned as int8): nearest, ties to even,
+    saturating at -128 / 127, NaN -> 0."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, dtype=np.uint8)
+    (lib or load()).oracle_encode_int8(_ptr(x), _ptr(out), x.size)
+    return out.view(np.int8)
+
+
+def reshape_and_cache_int8(key, value, k_cache, v_cache, slot_mapping, block_size, dtype,
+                           k_scale, v_scale, lib=None) -> int:
+    """Quantising cache write into int8 pools [num_blocks][B][Hkv][D]."""
+    return _reshape_and_cache_q8((lib or load()).oracle_reshape_and_cache_int8, key, value,
+                                 k_cache, v_cache, slot_mapping, block_size, dtype, k_scale,
+                                 v_scale)
+
+
+def paged_decode_int8(query, k_cache, v_cache, block_tables, context_lens, scale, dtype, k_scale,
+                      v_scale, num_threads=0, lib=None):
+    """fp64 paged decode over int8 pools (code x scale)."""
+    return _paged_decode_q8((lib or load()).oracle_paged_decode_int8, query, k_cache, v_cache,
+                            block_tables, context_lens, scale, dtype, k_scale, v_scale,
+                            num_threads)

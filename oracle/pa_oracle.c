@@ -24,7 +24,9 @@
  * [Practice §3.2 块表与地址转换].
  *
  * Element storage is the raw 16-bit pattern (IEEE binary16 or bfloat16);
- * the oracle decodes the bits itself, exactly, into double.
+ * the oracle decodes the bits itself, exactly, into double.  Quantised
+ * pools hold one byte per element (an e4m3 or an int8 code) and one scale
+ * per pool; their functions carry the _fp8 / _int8 suffix.
  *
  * Status bits returned by the functions (same meaning as the library's):
  *   1 = a block-table entry outside [0, num_blocks)   (that block is skipped)
@@ -146,13 +148,49 @@ void oracle_encode_e4m3(const float* x, uint8_t* out, int64_t n)
     for (int64_t i = 0; i < n; ++i) out[i] = f32_to_e4m3(x[i]);
 }
 
-/* Quantising cache write: code = e4m3(fp32(x) * fp32(1 / scale)), the
- * product rounded once in fp32, then rounded to e4m3 as above. */
-int32_t oracle_reshape_and_cache_fp8(const uint16_t* key, const uint16_t* value, uint8_t* k_cache,
-                                     uint8_t* v_cache, const int64_t* slot_mapping,
-                                     int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
-                                     int32_t block_size, int64_t num_blocks, int32_t dtype,
-                                     float k_scale, float v_scale)
+/* ------------------------------------------------------------------------
+ * INT8: two's-complement codes; the stored value is code x scale, one scale
+ * per pool (the same passages name INT8 beside FP8).
+ * ---------------------------------------------------------------------- */
+static double int8_to_f64(uint8_t b)
+{
+    return (double)(int8_t)b;
+}
+
+void oracle_decode_int8(const uint8_t* codes, double* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = int8_to_f64(codes[i]);
+}
+
+/* fp32 -> int8: NaN -> 0; values at or beyond the ends of [-128, 127]
+ * saturate; in-range values round to the nearest integer, ties to the even
+ * one.  floor() and the fraction are exact in double. */
+static uint8_t f32_to_int8(float x)
+{
+    if (x != x) return 0;
+    if (x <= -128.0f) return (uint8_t)(int8_t)-128;
+    if (x >= 127.0f) return 127;
+    const double a = (double)x;
+    const double lo = floor(a), frac = a - lo;
+    double r;
+    if (frac < 0.5) r = lo;
+    else if (frac > 0.5) r = lo + 1.0;
+    else r = fmod(lo, 2.0) == 0.0 ? lo : lo + 1.0;
+    return (uint8_t)(int8_t)r;
+}
+
+void oracle_encode_int8(const float* x, uint8_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = f32_to_int8(x[i]);
+}
+
+/* Quantising cache write: code = encode(fp32(x) * fp32(1 / scale)), the
+ * product rounded once in fp32, then encoded as above (e4m3 or int8). */
+static int32_t reshape_and_cache_q8(const uint16_t* key, const uint16_t* value, uint8_t* k_cache,
+                                    uint8_t* v_cache, const int64_t* slot_mapping,
+                                    int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t block_size, int64_t num_blocks, int32_t dtype,
+                                    float k_scale, float v_scale, uint8_t (*encode)(float))
 {
     int32_t status = 0;
     const float k_inv = 1.0f / k_scale, v_inv = 1.0f / v_scale;
@@ -168,11 +206,34 @@ int32_t oracle_reshape_and_cache_fp8(const uint16_t* key, const uint16_t* value,
                                                             : f16_bits_to_f64(value[t * row + e]));
             const float kq = kx * k_inv;
             const float vq = vx * v_inv;
-            k_cache[slot * row + e] = f32_to_e4m3(kq);
-            v_cache[slot * row + e] = f32_to_e4m3(vq);
+            k_cache[slot * row + e] = encode(kq);
+            v_cache[slot * row + e] = encode(vq);
         }
     }
     return status;
+}
+
+int32_t oracle_reshape_and_cache_fp8(const uint16_t* key, const uint16_t* value, uint8_t* k_cache,
+                                     uint8_t* v_cache, const int64_t* slot_mapping,
+                                     int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t block_size, int64_t num_blocks, int32_t dtype,
+                                     float k_scale, float v_scale)
+{
+    return reshape_and_cache_q8(key, value, k_cache, v_cache, slot_mapping, num_tokens,
+                                num_kv_heads, head_dim, block_size, num_blocks, dtype, k_scale,
+                                v_scale, f32_to_e4m3);
+}
+
+int32_t oracle_reshape_and_cache_int8(const uint16_t* key, const uint16_t* value,
+                                      uint8_t* k_cache, uint8_t* v_cache,
+                                      const int64_t* slot_mapping, int32_t num_tokens,
+                                      int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                      int64_t num_blocks, int32_t dtype, float k_scale,
+                                      float v_scale)
+{
+    return reshape_and_cache_q8(key, value, k_cache, v_cache, slot_mapping, num_tokens,
+                                num_kv_heads, head_dim, block_size, num_blocks, dtype, k_scale,
+                                v_scale, f32_to_int8);
 }
 
 /* ------------------------------------------------------------------------
@@ -378,16 +439,17 @@ static int32_t decode_row(double* out, const uint16_t* query, const uint16_t* k_
     return status;
 }
 
-/* Paged decode over e4m3 pools: every cached element is dequantised,
- * K = decode(code) * k_scale, V = decode(code) * v_scale, in double, and the
- * attention is the direct form of decode_row.  Query and output as in
- * oracle_paged_decode (query bits of `dtype`). */
-static int32_t decode_row_fp8(double* out, const uint16_t* query, const uint8_t* k_cache,
-                              const uint8_t* v_cache, const int32_t* block_tables,
-                              const int32_t* context_lens, int32_t s, int32_t h,
-                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
-                              double scale, int32_t dtype, double k_scale, double v_scale)
+/* Paged decode over 8-bit pools (e4m3 or int8 codes): every cached element
+ * is dequantised, K = dec(code) * k_scale, V = dec(code) * v_scale, in
+ * double, and the attention is the direct form of decode_row.  Query and
+ * output as in oracle_paged_decode (query bits of `dtype`). */
+static int32_t decode_row_q8(double* out, const uint16_t* query, const uint8_t* k_cache,
+                             const uint8_t* v_cache, const int32_t* block_tables,
+                             const int32_t* context_lens, int32_t s, int32_t h,
+                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                             int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+                             double scale, int32_t dtype, double k_scale, double v_scale,
+                             double (*dec)(uint8_t))
 {
     int32_t status = 0;
     const int32_t group = num_q_heads / num_kv_heads;
@@ -408,7 +470,7 @@ static int32_t decode_row_fp8(double* out, const uint16_t* query, const uint8_t*
         valid[t] = r >= 0;
         if (r < 0) { status |= 1; x[t] = 0.0; continue; }
         double acc = 0.0;
-        for (int32_t d = 0; d < head_dim; ++d) acc += q[d] * (e4m3_to_f64(k_cache[r + d]) * k_scale);
+        for (int32_t d = 0; d < head_dim; ++d) acc += q[d] * (dec(k_cache[r + d]) * k_scale);
         x[t] = scale * acc;
         any = 1;
     }
@@ -421,7 +483,7 @@ static int32_t decode_row_fp8(double* out, const uint16_t* query, const uint8_t*
             double w = exp(x[t] - m) / l;
             int64_t r = token_row(table, t, g, num_kv_heads, head_dim, block_size, num_blocks);
             for (int32_t d = 0; d < head_dim; ++d)
-                out[d] += w * (e4m3_to_f64(v_cache[r + d]) * v_scale);
+                out[d] += w * (dec(v_cache[r + d]) * v_scale);
         }
     }
     free(q); free(x); free(valid);
@@ -491,6 +553,28 @@ int32_t oracle_max_threads(void)
 #endif
 }
 
+static int32_t paged_decode_q8(double* out, const uint16_t* query, const uint8_t* k_cache,
+                               const uint8_t* v_cache, const int32_t* block_tables,
+                               const int32_t* context_lens, int32_t num_seqs,
+                               int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t block_size, int32_t max_blocks_per_seq,
+                               int64_t num_blocks, double scale, int32_t dtype, double k_scale,
+                               double v_scale, int32_t num_threads, double (*dec)(uint8_t))
+{
+    int32_t status = 0;
+    const int64_t rows = (int64_t)num_seqs * num_q_heads;
+    set_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : status)
+    for (int64_t r = 0; r < rows; ++r) {
+        int32_t s = (int32_t)(r / num_q_heads), h = (int32_t)(r % num_q_heads);
+        status |= decode_row_q8(out + r * head_dim, query, k_cache, v_cache, block_tables,
+                                context_lens, s, h, num_q_heads, num_kv_heads, head_dim,
+                                block_size, max_blocks_per_seq, num_blocks, scale, dtype,
+                                k_scale, v_scale, dec);
+    }
+    return status;
+}
+
 int32_t oracle_paged_decode_fp8(double* out, const uint16_t* query, const uint8_t* k_cache,
                                 const uint8_t* v_cache, const int32_t* block_tables,
                                 const int32_t* context_lens, int32_t num_seqs,
@@ -499,16 +583,20 @@ int32_t oracle_paged_decode_fp8(double* out, const uint16_t* query, const uint8_
                                 int64_t num_blocks, double scale, int32_t dtype, double k_scale,
                                 double v_scale, int32_t num_threads)
 {
-    int32_t status = 0;
-    const int64_t rows = (int64_t)num_seqs * num_q_heads;
-    set_threads(num_threads);
-#pragma omp parallel for schedule(dynamic, 1) reduction(| : status)
-    for (int64_t r = 0; r < rows; ++r) {
-        int32_t s = (int32_t)(r / num_q_heads), h = (int32_t)(r % num_q_heads);
-        status |= decode_row_fp8(out + r * head_dim, query, k_cache, v_cache, block_tables,
-                                 context_lens, s, h, num_q_heads, num_kv_heads, head_dim,
-                                 block_size, max_blocks_per_seq, num_blocks, scale, dtype,
-                                 k_scale, v_scale);
-    }
-    return status;
+    return paged_decode_q8(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, scale, dtype, k_scale, v_scale, num_threads, e4m3_to_f64);
+}
+
+int32_t oracle_paged_decode_int8(double* out, const uint16_t* query, const uint8_t* k_cache,
+                                 const uint8_t* v_cache, const int32_t* block_tables,
+                                 const int32_t* context_lens, int32_t num_seqs,
+                                 int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                 int32_t block_size, int32_t max_blocks_per_seq,
+                                 int64_t num_blocks, double scale, int32_t dtype, double k_scale,
+                                 double v_scale, int32_t num_threads)
+{
+    return paged_decode_q8(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, scale, dtype, k_scale, v_scale, num_threads, int8_to_f64);
 }

@@ -411,6 +411,101 @@ def pin_fp8_decode_matches_numpy_attention(lib):
         close(got[s], np.einsum("ht,thd->hd", w, v), 1e-12)
 
 
+# ---- INT8 caches ---------------------------------------------------------------
+
+def pin_int8_decode_all_codes(lib):
+    """Every byte decodes to its two's-complement value (numpy's int8 view)."""
+    codes = np.arange(256, dtype=np.uint8)
+    assert np.array_equal(oracle.decode_int8(codes, lib=lib),
+                          codes.view(np.int8).astype(np.float64))
+
+
+def pin_int8_encode_rounding(lib):
+    """fp32 -> int8 agrees with torch.round (ties to even) clamped to
+    [-128, 127] on random values, every integer and every midpoint of the
+    range; beyond it saturates (inf too) and NaN gives 0."""
+    import torch
+    rng = np.random.Generator(np.random.PCG64(16))
+    ints = np.arange(-128, 128, dtype=np.float64)
+    x = np.concatenate([ints, ints[:-1] + 0.5, rng.uniform(-130, 130, 4000),
+                        rng.normal(0, 2, 2000)]).astype(np.float32)
+    ref = torch.clamp(torch.round(torch.from_numpy(x)), -128, 127).to(torch.int8).numpy()
+    assert np.array_equal(oracle.encode_int8(x, lib=lib), ref)
+    assert np.array_equal(oracle.encode_int8(ints.astype(np.float32), lib=lib),
+                          ints.astype(np.int8))
+    special = np.array([127.4, 127.5, 127.6, 128.0, 1e6, np.inf, -128.4, -128.5, -129.0, -np.inf,
+                        np.nan, 0.5, -0.5, 1.5, -2.5], np.float32)
+    assert oracle.encode_int8(special, lib=lib).tolist() == [127, 127, 127, 127, 127, 127, -128,
+                                                             -128, -128, -128, 0, 0, 0, 2, -2]
+
+
+def pin_int8_cache_write(lib):
+    """The quantising write stores int8(fp32(x) * fp32(1/scale)) at the slot's
+    offset; other bytes unchanged; a slot past the pool is flagged."""
+    rng = np.random.Generator(np.random.PCG64(17))
+    nb, b, h, d = 6, 4, 2, 8
+    kc = np.full((nb, b, h, d), 0x55, np.uint8).view(np.int8)
+    vc = np.full((nb, b, h, d), 0x55, np.uint8).view(np.int8)
+    key = gen.normal_bits(rng, (3, h, d), "bf16")
+    val = gen.normal_bits(rng, (3, h, d), "bf16")
+    slots = np.array([5, -1, 17])
+    st = oracle.reshape_and_cache_int8(key, val, kc, vc, slots, b, "bf16", 0.02, 0.03, lib=lib)
+    assert st == 0
+    inv_k, inv_v = np.float32(1) / np.float32(0.02), np.float32(1) / np.float32(0.03)
+    as_f32 = lambda bits: (bits.astype(np.uint32) << 16).view(np.float32)   # bf16 -> fp32, exact
+    for t, sl in ((0, 5), (2, 17)):
+        assert np.array_equal(kc[sl // b, sl % b], oracle.encode_int8(as_f32(key[t]) * inv_k, lib=lib))
+        assert np.array_equal(vc[sl // b, sl % b], oracle.encode_int8(as_f32(val[t]) * inv_v, lib=lib))
+    touched = np.zeros((nb, b), bool)
+    touched[1, 1] = touched[4, 1] = True
+    assert np.all(kc[~touched] == 0x55) and np.all(vc[~touched] == 0x55)
+    assert oracle.reshape_and_cache_int8(key, val, kc, vc, np.array([nb * b, 0, 1]), b, "bf16",
+                                         0.02, 0.03, lib=lib) == 2
+
+
+def pin_int8_decode_equals_dequantised_fp16(lib):
+    """With power-of-two scales every code x scale is exact in fp16, so the
+    int8 decode must equal the (pinned) fp16 decode of the dequantised pools."""
+    rng = np.random.Generator(np.random.PCG64(18))
+    wl = small_gqa(dtype="f16")
+    codes_k = rng.integers(-128, 128, size=wl.k_cache.shape).astype(np.int8)
+    codes_v = rng.integers(-128, 128, size=wl.v_cache.shape).astype(np.int8)
+    ks, vs = 2.0 ** -6, 2.0 ** -5
+    deq_k = (codes_k.astype(np.float64) * ks).astype(np.float16).view(np.uint16)
+    deq_v = (codes_v.astype(np.float64) * vs).astype(np.float16).view(np.uint16)
+    a, sa = oracle.paged_decode_int8(wl.query, codes_k, codes_v, wl.block_tables, wl.context_lens,
+                                     wl.scale, "f16", ks, vs, lib=lib)
+    b, sb = oracle.paged_decode(wl.query, deq_k, deq_v, wl.block_tables, wl.context_lens,
+                                wl.scale, "f16", lib=lib)
+    assert sa == sb == 0
+    assert np.array_equal(a, b)
+
+
+def pin_int8_decode_matches_numpy_attention(lib):
+    """Scales that are not powers of two: the int8 decode equals numpy
+    softmax attention over K/V gathered through the tables, dequantised as
+    code x scale (<= 1e-12)."""
+    from scipy.special import softmax
+    wl = small_gqa(dtype="f16", seqs=4, head_dim=64)
+    rng = np.random.Generator(np.random.PCG64(19))
+    kc = rng.integers(-128, 128, size=wl.k_cache.shape).astype(np.int8)
+    vc = rng.integers(-128, 128, size=wl.v_cache.shape).astype(np.int8)
+    ks, vs = 0.0173, 0.0291
+    got, st = oracle.paged_decode_int8(wl.query, kc, vc, wl.block_tables, wl.context_lens,
+                                       wl.scale, wl.dtype, ks, vs, lib=lib)
+    assert st == 0
+    q = wl.query.view(np.float16).astype(np.float64)
+    b, group = wl.block_size, wl.num_q_heads // wl.num_kv_heads
+    for s in range(wl.num_seqs):
+        c = int(wl.context_lens[s])
+        pos = np.arange(c)
+        phys = wl.block_tables[s][pos // b]
+        k = np.repeat(kc[phys, pos % b].astype(np.float64) * ks, group, axis=1)
+        v = np.repeat(vc[phys, pos % b].astype(np.float64) * vs, group, axis=1)
+        w = softmax(wl.scale * np.einsum("hd,thd->ht", q[s], k), axis=1)
+        close(got[s], np.einsum("ht,thd->hd", w, v), 1e-12)
+
+
 # ---- swap_blocks (eviction to host memory and back) ---------------------------
 
 def pin_swap_round_trip(lib):

@@ -37,15 +37,21 @@ MUTANTS = {
     "e4m3_ties_away": ("else pick = (lo & 1) ? hi : lo;", "else pick = hi;"),
     "e4m3_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7e);",
                            "if (a >= 448.0) return (uint8_t)(sign | 0x7f);"),
-    "fp8_scale_dropped": ("(e4m3_to_f64(k_cache[r + d]) * k_scale)",
-                          "(e4m3_to_f64(k_cache[r + d]))"),
+    "fp8_scale_dropped": ("(dec(k_cache[r + d]) * k_scale)", "(dec(k_cache[r + d]))"),
     "fp8_write_divides_twice": ("const float kq = kx * k_inv;", "const float kq = kx * k_inv * k_inv;"),
     "swap_only_k": ("dst_v[dst * block_bytes + b] = src_v[src * block_bytes + b];", ""),
     "swap_dst_index_of_src": ("dst_k[dst * block_bytes + b] = src_k[src * block_bytes + b];",
                               "dst_k[src % dst_num_blocks * block_bytes + b] = src_k[src * block_bytes + b];"),
     "swap_bad_id_not_flagged": ("            status |= 1;\n            continue;", "            continue;"),
-    "fp8_v_scaled_by_k_scale": ("(e4m3_to_f64(v_cache[r + d]) * v_scale)",
-                                "(e4m3_to_f64(v_cache[r + d]) * k_scale)"),
+    "fp8_v_scaled_by_k_scale": ("(dec(v_cache[r + d]) * v_scale)",
+                                "(dec(v_cache[r + d]) * k_scale)"),
+    "int8_unsigned_codes": ("return (double)(int8_t)b;", "return (double)b;"),
+    "int8_ties_away": ("else r = fmod(lo, 2.0) == 0.0 ? lo : lo + 1.0;", "else r = lo + 1.0;"),
+    "int8_wraps_past_127": ("if (x >= 127.0f) return 127;", "if (x >= 128.0f) return 127;"),
+    "int8_nan_saturates": ("if (x != x) return 0;", "if (x != x) return 127;"),
+    "int8_decodes_as_e4m3": ("num_blocks, scale, dtype, k_scale, v_scale, num_threads, int8_to_f64);",
+                             "num_blocks, scale, dtype, k_scale, v_scale, num_threads, e4m3_to_f64);"),
+    "int8_write_uses_e4m3": ("v_scale, f32_to_int8);", "v_scale, f32_to_e4m3);"),
     "swap_no_conflict_check": ("if (block_mapping[2 * j + 1] == block_mapping[2 * i + 1]) status |= 8;", ""),
 }
 
