@@ -45,7 +45,8 @@ FALLBACK_HBM_GBS = 6650.0
 PROFILE_GLOB_DIR = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = ["paged_kv_cache_415_b200/csrc/paged_decode.cu",
                   "paged_kv_cache_415_b200/csrc/paged_decode_mma.cuh",
-                  "paged_kv_cache_415_b200/csrc/paged_decode_fp8.cuh",
+                  "paged_kv_cache_415_b200/csrc/paged_decode_q8.cuh",
+                  "paged_kv_cache_415_b200/csrc/pa_codes.cuh",
                   "paged_kv_cache_415_b200/csrc/pa_common.cuh"]
 NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
@@ -71,9 +72,9 @@ def parse_args():
     ap.add_argument("--shared-prefix", action="store_true",
                     help="beam_search: decode with pa_paged_decode_shared_prefix (shared "
                          "prompt blocks read once per group)")
-    ap.add_argument("--kv-dtype", default="auto", choices=["auto", "fp8"],
-                    help="fp8: the same workload with e4m3 K/V pools (per-pool scales), "
-                         "quantising cache write + e4m3 decode")
+    ap.add_argument("--kv-dtype", default="auto", choices=["auto", "fp8", "int8"],
+                    help="fp8 / int8: the same workload with e4m3 / int8 K/V pools (per-pool "
+                         "scales), quantising cache write + decode over the codes")
     ap.add_argument("--swap", choices=["out", "in"], default=None,
                     help="measure pa_swap_blocks instead of the decode step: 512 LLaMA-7B-shaped "
                          "blocks (K and V, 256 KB a pair) device -> pinned host (out) or back (in)")
@@ -225,11 +226,11 @@ def whole_job_gbs(bytes_per_step: int, steps: int, world: int, max_elapsed_ms: f
 def make_workload(config: str, seqs: int = 0, kv_dtype: str = "auto"):
     """The named workload; with seqs > 0 a smaller batch of the same shape
     and a pool sized to it (profiling captures stay a few GB); kv_dtype fp8
-    redraws its pools as e4m3 codes."""
+    or int8 redraws its pools as e4m3 or int8 codes."""
     from workloads import generators as gen
     wl = _make_workload(config, seqs)
-    if kv_dtype == "fp8":
-        wl = gen.with_fp8_pools(wl, seed=gen.SEED_BASE + 50)
+    if kv_dtype in ("fp8", "int8"):
+        wl = gen.with_code_pools(wl, kv_dtype, seed=gen.SEED_BASE + 50)
     return wl
 
 
@@ -249,7 +250,7 @@ def _make_workload(config: str, seqs: int = 0):
 
 
 def workload_config(wl, partition_size, l2_note):
-    kv = ", e4m3 K/V pools" if wl.extra.get("kv_dtype") == "fp8" else ""
+    kv = {"fp8": ", e4m3 K/V pools", "int8": ", int8 K/V pools"}.get(wl.extra.get("kv_dtype"), "")
     return {"workload": f"{wl.name}: {wl.num_seqs} seqs, {wl.num_q_heads}/{wl.num_kv_heads} heads, "
                         f"head_dim {wl.head_dim}, block {wl.block_size}, {wl.dtype}{kv}, "
                         f"contexts {int(wl.context_lens.min())}..{int(wl.context_lens.max())} "
@@ -281,7 +282,7 @@ class OracleStep:
         self.kc, self.vc = wl.k_cache.copy(), wl.v_cache.copy()
         att = bm.decode_bytes(self.ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
                               wl.block_size, 2, bm.kv_elem_bytes(wl))
-        self.fp8 = wl.extra.get("kv_dtype") == "fp8"
+        self.codes = wl.extra.get("kv_dtype")          # None, "fp8" or "int8"
         full = bm.step_bytes(wl)
         self.bytes = att["total"] + full["append"] + full["copy"]
         self.threads = oracle.max_threads()
@@ -291,13 +292,14 @@ class OracleStep:
         t0 = time.perf_counter()
         if wl.block_mapping.shape[0]:
             o.copy_blocks(self.kc, self.vc, wl.block_mapping)
-        if self.fp8:
+        if self.codes is not None:
             ks, vs = wl.extra["k_scale"], wl.extra["v_scale"]
+            write = getattr(o, f"reshape_and_cache_{self.codes}")
+            decode = getattr(o, f"paged_decode_{self.codes}")
             if wl.num_new_tokens:
-                o.reshape_and_cache_fp8(wl.new_key, wl.new_value, self.kc, self.vc,
-                                        wl.slot_mapping, wl.block_size, wl.dtype, ks, vs)
-            o.paged_decode_fp8(self.q, self.kc, self.vc, self.tables, self.ctx, wl.scale,
-                               wl.dtype, ks, vs)
+                write(wl.new_key, wl.new_value, self.kc, self.vc, wl.slot_mapping, wl.block_size,
+                      wl.dtype, ks, vs)
+            decode(self.q, self.kc, self.vc, self.tables, self.ctx, wl.scale, wl.dtype, ks, vs)
             return time.perf_counter() - t0
         if wl.num_new_tokens:
             o.reshape_and_cache(wl.new_key, wl.new_value, self.kc, self.vc, wl.slot_mapping,
@@ -377,13 +379,18 @@ def run_ours(args):
     wl = make_workload(args.config, args.seqs, args.kv_dtype)
     dev = torch.device("cuda", local)
     tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
-    fp8 = wl.extra.get("kv_dtype") == "fp8"
+    codes = wl.extra.get("kv_dtype")                  # None, "fp8" or "int8"
+    quant = codes is not None
+    if quant:
+        q_write, q_decode, q_decode_append = (
+            getattr(B, f"pa_reshape_and_cache_{codes}"), getattr(B, f"pa_paged_decode_{codes}"),
+            getattr(B, f"pa_paged_decode_{codes}_append"))
     k_scale, v_scale = wl.extra.get("k_scale", 1.0), wl.extra.get("v_scale", 1.0)
 
     def up(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(tdt)
 
-    if fp8:
+    if quant:
         k_cache = torch.from_numpy(wl.k_cache).to(dev)
         v_cache = torch.from_numpy(wl.v_cache).to(dev)
     else:
@@ -413,14 +420,14 @@ def run_ours(args):
     def cache_ops():
         if n_pairs:
             B.pa_copy_blocks(k_cache, v_cache, block_mapping, d_status, stream)
-        if wl.num_new_tokens and fp8 and not fused:
-            B.pa_reshape_and_cache_fp8(new_key, new_value, k_cache, v_cache, slot_mapping,
-                                       k_scale, v_scale, d_status, stream)
+        if wl.num_new_tokens and quant and not fused:
+            q_write(new_key, new_value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                    d_status, stream)
         elif wl.num_new_tokens and not fused:
             B.pa_reshape_and_cache(new_key, new_value, k_cache, v_cache, slot_mapping, d_status,
                                    stream)
 
-    shared = args.shared_prefix and "prefix_lens" in wl.extra and not fp8
+    shared = args.shared_prefix and "prefix_lens" in wl.extra and not quant
     if shared:
         group_size = int(wl.extra["group_size"])
         prefix_lens = torch.from_numpy(wl.extra["prefix_lens"]).to(dev)
@@ -431,13 +438,13 @@ def run_ours(args):
         workspace = torch.empty(max(sws, 16), dtype=torch.uint8, device=dev)
 
     def decode():
-        if fp8 and fused:
-            B.pa_paged_decode_fp8_append(out, query, new_key, new_value, k_cache, v_cache,
-                                         block_tables, context_lens, mcl, wl.scale, k_scale,
-                                         v_scale, part, workspace, d_status, stream)
-        elif fp8:
-            B.pa_paged_decode_fp8(out, query, k_cache, v_cache, block_tables, context_lens, mcl,
-                                  wl.scale, k_scale, v_scale, part, workspace, d_status, stream)
+        if quant and fused:
+            q_decode_append(out, query, new_key, new_value, k_cache, v_cache, block_tables,
+                            context_lens, mcl, wl.scale, k_scale, v_scale, part, workspace,
+                            d_status, stream)
+        elif quant:
+            q_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl, wl.scale,
+                     k_scale, v_scale, part, workspace, d_status, stream)
         elif fused:
             B.pa_paged_decode_append(out, query, new_key, new_value, k_cache, v_cache,
                                      block_tables, context_lens, mcl, wl.scale, part, workspace,
@@ -559,7 +566,7 @@ def run_ours(args):
     # the decode launch also carries the step's cache write when it is fused
     decode_bytes = step["attention"] + (step["append"] if fused else 0)
     achieved = decode_bytes / (decode_avg * 1e-3) / 1e9
-    traffic = profiled_traffic(args.config + ("-fp8" if fp8 else ""))
+    traffic = profiled_traffic(args.config + (f"-{codes}" if quant else ""))
     clocks = sampler.summary()
 
     cpu = None
@@ -577,7 +584,7 @@ def run_ours(args):
         kernel_name = "paged_decode_shared_kernel" + (
             " + paged_decode_shared_reduce_kernel" if shared_parts_gt1 else "")
     else:
-        kernel_name = ("paged_decode_fp8_kernel" if fp8 else
+        kernel_name = (f"paged_decode_{codes}_kernel" if quant else
                        "paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
                        else "paged_decode_kernel")
         if max_parts > 1:
@@ -588,7 +595,8 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16 (e4m3 K/V)" if fp8 else wl.dtype,
+        "dtype": ({"fp8": "f16 (e4m3 K/V)", "int8": "f16 (int8 K/V)"}[codes] if quant
+                  else wl.dtype),
         "data": "synthetic", "config": workload_config(wl, part, l2),
         "us_per_layer_step": round(per_step_ms * 1e3, 2),
         "kv_tokens_per_s": round(world * int(wl.context_lens.sum()) * args.steps / (elapsed_ms * 1e-3)),
@@ -609,9 +617,9 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "bytes_per_step": step,
         "launch": "eager" if args.eager else "CUDA-graph replay (cache ops graph, decode graph)",
-        "decode_entry": ("pa_paged_decode_fp8_append (quantising cache write fused)"
-                         if fp8 and fused else
-                         "pa_reshape_and_cache_fp8 + pa_paged_decode_fp8" if fp8 else
+        "decode_entry": (f"pa_paged_decode_{codes}_append (quantising cache write fused)"
+                         if quant and fused else
+                         f"pa_reshape_and_cache_{codes} + pa_paged_decode_{codes}" if quant else
                          "pa_paged_decode_shared_prefix" if shared else
                          "pa_paged_decode_append (cache write fused)" if fused else
                          "pa_reshape_and_cache + pa_paged_decode"),

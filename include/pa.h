@@ -96,7 +96,8 @@ typedef enum pa_status {
 typedef enum pa_dtype {
     PA_DTYPE_F16 = 0,
     PA_DTYPE_BF16 = 1,
-    PA_DTYPE_FP8_E4M3 = 2   /* cache pools only: block copies/swaps and the *_fp8 calls */
+    PA_DTYPE_FP8_E4M3 = 2,  /* cache pools only: block copies/swaps and the *_fp8 calls */
+    PA_DTYPE_INT8 = 3       /* cache pools only: block copies/swaps and the *_int8 calls */
 } pa_dtype;
 
 #define PA_STATUS_BAD_BLOCK 1
@@ -184,7 +185,7 @@ PA_API pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t* blo
  *                distinct (else PA_STATUS_COPY_CONFLICT); when the source
  *                and destination pools are the same memory this is
  *                pa_copy_blocks, with its conflict rule.
- * dtype          PA_DTYPE_F16, _BF16 or _FP8_E4M3 (element size only).
+ * dtype          PA_DTYPE_F16, _BF16, _FP8_E4M3 or _INT8 (element size only).
  * d_status       optional; PA_STATUS_BAD_BLOCK (an id outside its pool;
  *                the pair is skipped), PA_STATUS_COPY_CONFLICT.
  * Errors: PA_ERR_INVALID_ARG for null or misaligned pointers, a pointer the
@@ -358,6 +359,50 @@ PA_API pa_status pa_paged_decode_fp8(void* out, const void* query, const void* k
  * written.
  */
 PA_API pa_status pa_paged_decode_fp8_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale,
+    float k_scale, float v_scale, int32_t partition_size, void* workspace, size_t workspace_bytes,
+    pa_dtype dtype, int32_t* d_status, pa_stream_t stream);
+
+/*
+ * INT8 KV cache -- pools of two's-complement int8 codes (1 byte per element)
+ * with one scale per pool: the cached value of code c is c * k_scale (or
+ * v_scale).  Defined by the same passages as the FP8 pools above, which
+ * name INT8 beside FP8; the scale-per-tensor form is this library's
+ * reading.  Layout and slots as the 16-bit pools.  pa_copy_blocks and
+ * pa_swap_blocks move such pools with dtype PA_DTYPE_INT8.
+ *
+ * pa_reshape_and_cache_int8 -- the cache write, quantising:
+ *   code = fp32(x) * fp32(1 / scale), rounded to the nearest integer (ties
+ *   to even) and saturated to [-128, 127]; NaN gives 0.
+ * Other arguments and errors as pa_reshape_and_cache_fp8.
+ *
+ * pa_paged_decode_int8, pa_paged_decode_int8_append -- as the FP8 calls
+ * above, over int8 pools (every code is an fp16 value, so K and V are again
+ * dequantised exactly); the fused write quantises as
+ * pa_reshape_and_cache_int8.  Arguments, results and errors as
+ * pa_paged_decode_fp8 and pa_paged_decode_fp8_append.
+ */
+PA_API pa_status pa_reshape_and_cache_int8(const void* key, const void* value, void* k_cache,
+                                           void* v_cache, const int64_t* slot_mapping,
+                                           int32_t num_tokens, int32_t num_kv_heads,
+                                           int32_t head_dim, int32_t block_size,
+                                           int64_t num_blocks, pa_dtype dtype, float k_scale,
+                                           float v_scale, int32_t* d_status, pa_stream_t stream);
+
+PA_API pa_status pa_paged_decode_int8(void* out, const void* query, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      const int32_t* context_lens, int32_t num_seqs,
+                                      int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, int32_t max_blocks_per_seq,
+                                      int64_t num_blocks, int32_t max_context_len, float scale,
+                                      float k_scale, float v_scale, int32_t partition_size,
+                                      void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                                      int32_t* d_status, pa_stream_t stream);
+
+PA_API pa_status pa_paged_decode_int8_append(
     void* out, const void* query, const void* key, const void* value, void* k_cache,
     void* v_cache, const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,

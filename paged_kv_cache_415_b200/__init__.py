@@ -17,7 +17,8 @@ _BINDING_NAMES = {
     "pa_copy_blocks", "pa_paged_decode", "pa_paged_decode_no_alloc",
     "pa_paged_decode_shared_prefix", "pa_paged_decode_shared_prefix_workspace_size",
     "pa_paged_decode_append", "pa_reshape_and_cache_fp8", "pa_paged_decode_fp8",
-    "pa_paged_decode_fp8_append", "pa_swap_blocks",
+    "pa_paged_decode_fp8_append", "pa_reshape_and_cache_int8", "pa_paged_decode_int8",
+    "pa_paged_decode_int8_append", "pa_swap_blocks",
     "pa_paged_decode_partition_size", "pa_paged_decode_workspace_size", "pa_reshape_and_cache",
     "pa_status_string", "pa_version",
 }

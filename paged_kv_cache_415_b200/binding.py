@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpa.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
-PA_DTYPE_F16, PA_DTYPE_BF16, PA_DTYPE_FP8_E4M3 = 0, 1, 2
+PA_DTYPE_F16, PA_DTYPE_BF16, PA_DTYPE_FP8_E4M3, PA_DTYPE_INT8 = 0, 1, 2, 3
 PA_STATUS_BAD_BLOCK = 1
 PA_STATUS_BAD_SLOT = 2
 PA_STATUS_BAD_CONTEXT = 4
@@ -29,14 +29,16 @@ PA_STATUS_COPY_CONFLICT = 8
 PA_STATUS_TIMEOUT = 16
 
 _DTYPES = {torch.float16: PA_DTYPE_F16, torch.bfloat16: PA_DTYPE_BF16,
-           torch.uint8: PA_DTYPE_FP8_E4M3, torch.float8_e4m3fn: PA_DTYPE_FP8_E4M3}
+           torch.uint8: PA_DTYPE_FP8_E4M3, torch.float8_e4m3fn: PA_DTYPE_FP8_E4M3,
+           torch.int8: PA_DTYPE_INT8}
 
 # Every entry point declared in include/pa.h.
 EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_size",
            "pa_paged_decode_workspace_size", "pa_paged_decode", "pa_paged_decode_no_alloc",
            "pa_paged_decode_shared_prefix_workspace_size", "pa_paged_decode_shared_prefix",
            "pa_paged_decode_append", "pa_reshape_and_cache_fp8", "pa_paged_decode_fp8",
-           "pa_paged_decode_fp8_append", "pa_swap_blocks",
+           "pa_paged_decode_fp8_append", "pa_reshape_and_cache_int8", "pa_paged_decode_int8",
+           "pa_paged_decode_int8_append", "pa_swap_blocks",
            "pa_status_string", "pa_version")
 # Size of the library-owned scratch of pa_paged_decode_no_alloc.
 PA_NO_ALLOC_WORKSPACE_BYTES = 32 << 20
@@ -86,6 +88,12 @@ def _load() -> ctypes.CDLL:
     lib.pa_paged_decode_fp8_append.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, i32, i32,
                                                i32, i64, i32, f32, f32, f32, i32, p, sz, i32, p, p]
     lib.pa_paged_decode_fp8_append.restype = i32
+    lib.pa_reshape_and_cache_int8.argtypes = lib.pa_reshape_and_cache_fp8.argtypes
+    lib.pa_reshape_and_cache_int8.restype = i32
+    lib.pa_paged_decode_int8.argtypes = lib.pa_paged_decode_fp8.argtypes
+    lib.pa_paged_decode_int8.restype = i32
+    lib.pa_paged_decode_int8_append.argtypes = lib.pa_paged_decode_fp8_append.argtypes
+    lib.pa_paged_decode_int8_append.restype = i32
     lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64, i32, p, p]
     lib.pa_swap_blocks.restype = i32
     lib.pa_status_string.argtypes = [i32]
@@ -280,6 +288,49 @@ def pa_paged_decode_fp8_append(out, query, key, value, k_cache, v_cache, block_t
         int(block_tables.shape[1]), num_blocks, int(max_context_len), float(scale),
         float(k_scale), float(v_scale), int(partition_size), _ptr(workspace), ws_bytes,
         _dtype(query), _ptr(d_status), _stream(stream)))
+
+def pa_reshape_and_cache_int8(key, value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
+                              d_status=None, stream=None) -> None:
+    """Quantising cache write: key/value [T][Hkv][D] (fp16/bf16) into int8
+    pools k_cache/v_cache [num_blocks][B][Hkv][D] (int8 tensors)."""
+    num_blocks, block_size, hkv, d = k_cache.shape
+    _check("pa_reshape_and_cache_int8", LIB.pa_reshape_and_cache_int8(
+        _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping),
+        int(slot_mapping.shape[0]), hkv, d, block_size, num_blocks, _dtype(key), float(k_scale),
+        float(v_scale), _ptr(d_status), _stream(stream)))
+
+
+def pa_paged_decode_int8(out, query, k_cache, v_cache, block_tables, context_lens,
+                         max_context_len, scale, k_scale, v_scale, partition_size=0,
+                         workspace=None, d_status=None, stream=None) -> None:
+    """pa_paged_decode over int8 pools (int8 tensors) with per-pool scales."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_paged_decode_int8", LIB.pa_paged_decode_int8(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), num_seqs, hq, hkv, d, block_size, int(block_tables.shape[1]),
+        num_blocks, int(max_context_len), float(scale), float(k_scale), float(v_scale),
+        int(partition_size), _ptr(workspace), ws_bytes, _dtype(query), _ptr(d_status),
+        _stream(stream)))
+
+
+def pa_paged_decode_int8_append(out, query, key, value, k_cache, v_cache, block_tables,
+                                context_lens, max_context_len, scale, k_scale, v_scale,
+                                partition_size=0, workspace=None, d_status=None,
+                                stream=None) -> None:
+    """pa_paged_decode_int8 with each sequence's new token (key/value
+    [S][Hkv][D], fp16/bf16) quantised into its slot inside the launch."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_paged_decode_int8_append", LIB.pa_paged_decode_int8_append(
+        _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), num_seqs, hq, hkv, d, block_size,
+        int(block_tables.shape[1]), num_blocks, int(max_context_len), float(scale),
+        float(k_scale), float(v_scale), int(partition_size), _ptr(workspace), ws_bytes,
+        _dtype(query), _ptr(d_status), _stream(stream)))
+
 
 def _addr(t) -> int:
     """Device-usable address of a CUDA tensor or a pinned host tensor (on a

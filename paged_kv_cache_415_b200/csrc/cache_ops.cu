@@ -15,6 +15,7 @@
 #include <stdint.h>
 
 #include "pa.h"
+#include "pa_codes.cuh"
 #include "pa_common.cuh"
 #include "pa_host.h"
 
@@ -69,11 +70,10 @@ __global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_kernel(
     }
 }
 
-// Quantising variant for e4m3 pools: each vector of 8 input elements
-// becomes 8 codes, e4m3(fp32(x) * inv_scale) rounded to nearest even and
-// saturated at +-448.
-template <typename T>
-__global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_fp8_kernel(
+// Quantising variant for one-byte pools (e4m3 or int8, pa_codes.cuh): each
+// vector of 8 input elements becomes 8 codes of fp32(x) * inv_scale.
+template <typename Codes, typename T>
+__global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_q8_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, uint2* __restrict__ k_cache,
     uint2* __restrict__ v_cache, const int64_t* __restrict__ slot_mapping, int32_t row_vecs,
     int64_t num_slots, float k_inv, float v_inv, int32_t* d_status)
@@ -87,18 +87,6 @@ __global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_fp8_kernel(
         if (threadIdx.x == 0 && blockIdx.y == 0) status_or(d_status, PA_STATUS_BAD_SLOT);
         return;
     }
-    auto quant8 = [](const uint4& w, float inv) -> uint2 {
-        float f[8];
-        unpack8<T>(w, f);
-        uint32_t r[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const __nv_fp8x2_storage_t c = __nv_cvt_float2_to_fp8x2(
-                make_float2(f[2 * j] * inv, f[2 * j + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-            r[j] = static_cast<uint32_t>(c);
-        }
-        return make_uint2(r[0] | (r[1] << 16), r[2] | (r[3] << 16));
-    };
     const int32_t base = blockIdx.y * kCacheThreads * kCacheVecsPerThread + threadIdx.x;
     uint4 a[kCacheVecsPerThread], b[kCacheVecsPerThread];
 #pragma unroll
@@ -113,8 +101,8 @@ __global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_fp8_kernel(
     for (int j = 0; j < kCacheVecsPerThread; ++j) {
         const int32_t i = base + j * kCacheThreads;
         if (i < row_vecs) {
-            k_cache[slot * row_vecs + i] = quant8(a[j], k_inv);
-            v_cache[slot * row_vecs + i] = quant8(b[j], v_inv);
+            k_cache[slot * row_vecs + i] = encode8<Codes, T>(a[j], k_inv);
+            v_cache[slot * row_vecs + i] = encode8<Codes, T>(b[j], v_inv);
         }
     }
 }
@@ -223,11 +211,11 @@ __global__ void __launch_bounds__(kSwapThreads) swap_blocks_kernel(
 }
 
 static pa_status check_pool_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                                  int64_t num_blocks, int32_t dtype, bool allow_fp8 = false)
+                                  int64_t num_blocks, int32_t dtype, bool allow_codes = false)
 {
     if (num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
         return PA_ERR_INVALID_ARG;
-    const bool dtype_ok = supported_dtype(dtype) || (allow_fp8 && dtype == PA_DTYPE_FP8_E4M3);
+    const bool dtype_ok = supported_dtype(dtype) || (allow_codes && code_dtype(dtype));
     if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !dtype_ok)
         return PA_ERR_UNSUPPORTED;
     return PA_OK;
@@ -276,7 +264,7 @@ extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t*
         (d_status && !aligned4(d_status)))
         return PA_ERR_INVALID_ARG;
     if (num_pairs == 0) return PA_OK;
-    const int elem_bytes = dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2;
+    const int elem_bytes = code_dtype(dtype) ? 1 : 2;
     const int64_t block_vecs =
         static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes / 16;
     const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kCopyVecsPerThread;
@@ -288,15 +276,15 @@ extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t*
                              block_mapping, num_pairs, block_vecs, num_blocks, d_status);
 }
 
-extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
-                                              void* v_cache, const int64_t* slot_mapping,
-                                              int32_t num_tokens, int32_t num_kv_heads,
-                                              int32_t head_dim, int32_t block_size,
-                                              int64_t num_blocks, pa_dtype dtype, float k_scale,
-                                              float v_scale, int32_t* d_status,
-                                              pa_stream_t stream)
+namespace pa {
+template <typename Codes>
+static pa_status reshape_and_cache_q8(const void* key, const void* value, void* k_cache,
+                                      void* v_cache, const int64_t* slot_mapping,
+                                      int32_t num_tokens, int32_t num_kv_heads, int32_t head_dim,
+                                      int32_t block_size, int64_t num_blocks, pa_dtype dtype,
+                                      float k_scale, float v_scale, int32_t* d_status,
+                                      pa_stream_t stream)
 {
-    using namespace pa;
     if (num_tokens < 0) return PA_ERR_INVALID_ARG;
     pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
     if (st != PA_OK) return st;
@@ -313,17 +301,42 @@ extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value
     if (chunks > 65535) return PA_ERR_UNSUPPORTED;
     dim3 grid(num_tokens, chunks);
     const float k_inv = 1.0f / k_scale, v_inv = 1.0f / v_scale;
-    if (dtype == PA_DTYPE_F16)
-        return launch_overlapped(reshape_and_cache_fp8_kernel<__half>, grid, dim3(kCacheThreads), 0,
-                                 stream, static_cast<const uint4*>(key),
-                                 static_cast<const uint4*>(value), static_cast<uint2*>(k_cache),
-                                 static_cast<uint2*>(v_cache), slot_mapping, row_vecs,
-                                 num_blocks * block_size, k_inv, v_inv, d_status);
-    return launch_overlapped(reshape_and_cache_fp8_kernel<__nv_bfloat16>, grid,
-                             dim3(kCacheThreads), 0, stream, static_cast<const uint4*>(key),
-                             static_cast<const uint4*>(value), static_cast<uint2*>(k_cache),
-                             static_cast<uint2*>(v_cache), slot_mapping, row_vecs,
-                             num_blocks * block_size, k_inv, v_inv, d_status);
+    auto kernel = dtype == PA_DTYPE_F16 ? reshape_and_cache_q8_kernel<Codes, __half>
+                                        : reshape_and_cache_q8_kernel<Codes, __nv_bfloat16>;
+    return launch_overlapped(kernel, grid, dim3(kCacheThreads), 0, stream,
+                             static_cast<const uint4*>(key), static_cast<const uint4*>(value),
+                             static_cast<uint2*>(k_cache), static_cast<uint2*>(v_cache),
+                             slot_mapping, row_vecs, num_blocks * block_size, k_inv, v_inv,
+                             d_status);
+}
+}  // namespace pa
+
+extern "C" pa_status pa_reshape_and_cache_fp8(const void* key, const void* value, void* k_cache,
+                                              void* v_cache, const int64_t* slot_mapping,
+                                              int32_t num_tokens, int32_t num_kv_heads,
+                                              int32_t head_dim, int32_t block_size,
+                                              int64_t num_blocks, pa_dtype dtype, float k_scale,
+                                              float v_scale, int32_t* d_status,
+                                              pa_stream_t stream)
+{
+    return pa::reshape_and_cache_q8<pa::E4m3Codes>(key, value, k_cache, v_cache, slot_mapping,
+                                                   num_tokens, num_kv_heads, head_dim, block_size,
+                                                   num_blocks, dtype, k_scale, v_scale, d_status,
+                                                   stream);
+}
+
+extern "C" pa_status pa_reshape_and_cache_int8(const void* key, const void* value, void* k_cache,
+                                               void* v_cache, const int64_t* slot_mapping,
+                                               int32_t num_tokens, int32_t num_kv_heads,
+                                               int32_t head_dim, int32_t block_size,
+                                               int64_t num_blocks, pa_dtype dtype, float k_scale,
+                                               float v_scale, int32_t* d_status,
+                                               pa_stream_t stream)
+{
+    return pa::reshape_and_cache_q8<pa::Int8Codes>(key, value, k_cache, v_cache, slot_mapping,
+                                                   num_tokens, num_kv_heads, head_dim, block_size,
+                                                   num_blocks, dtype, k_scale, v_scale, d_status,
+                                                   stream);
 }
 
 namespace pa {
@@ -372,7 +385,7 @@ extern "C" pa_status pa_swap_blocks(const void* src_k, const void* src_v, void* 
         !device_address(dst_k, &dk) || !device_address(dst_v, &dv) ||
         !device_address(block_mapping, &map))
         return PA_ERR_INVALID_ARG;
-    const int elem_bytes = dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2;
+    const int elem_bytes = code_dtype(dtype) ? 1 : 2;
     const int64_t block_vecs =
         static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes / 16;
     const int64_t per_cta = static_cast<int64_t>(kSwapThreads) * kSwapVecsPerThread;

@@ -17,6 +17,8 @@ inline bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7
 inline bool supported_head_dim(int32_t d) { return d == 64 || d == 128; }
 inline bool supported_block_size(int32_t b) { return b == 8 || b == 16 || b == 32; }
 inline bool supported_dtype(int32_t t) { return t == PA_DTYPE_F16 || t == PA_DTYPE_BF16; }
+// One-byte pool element types (block copies and swaps move them as bytes).
+inline bool code_dtype(int32_t t) { return t == PA_DTYPE_FP8_E4M3 || t == PA_DTYPE_INT8; }
 
 // Launch-error check after a kernel launch.
 inline pa_status launch_status()

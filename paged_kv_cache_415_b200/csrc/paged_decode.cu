@@ -33,8 +33,8 @@
 // with more than one partition merges the partitions with the same rule:
 //   M = max_p m_p,  w_p = l_p * 2^(m_p - M),  out = sum_p w_p Ohat_p / sum_p w_p.
 //
-// The grouped-head (paged_decode_mma.cuh), e4m3 (paged_decode_fp8.cuh) and
-// shared-prefix (paged_decode_shared.cuh) kernels are included below; this
+// The grouped-head (paged_decode_mma.cuh), one-byte-code (e4m3 or int8:
+// paged_decode_q8.cuh) and shared-prefix (paged_decode_shared.cuh) kernels are included below; this
 // file also holds the host entry points and their launch logic.
 //
 // The whole computation has a fixed summation order, so results are
@@ -48,6 +48,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "pa.h"
 #include "pa_common.cuh"
@@ -590,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) p
 
 #include "paged_decode_mma.cuh"
 #include "paged_decode_shared.cuh"
-#include "paged_decode_fp8.cuh"
+#include "paged_decode_q8.cuh"
 
 namespace pa {
 
@@ -673,7 +674,7 @@ struct DecodeArgs {
     const void* new_key = nullptr;     // fused append (one token per sequence), or null
     const void* new_value = nullptr;
     int32_t lpt_seqs = 0;              // > 0: longest-first dispatch over this many sequences
-    float k_inv = 1.f, v_inv = 1.f;    // e4m3 pools: reciprocal scales of the fused write
+    float k_inv = 1.f, v_inv = 1.f;    // quantised pools: reciprocal scales of the fused write
 };
 
 constexpr int kMaxDevices = 64;
@@ -773,10 +774,10 @@ static bool encode_pool_map_swizzled(CUtensorMap* map, const void* pool, int32_t
     return res == CUDA_SUCCESS;
 }
 
-// An e4m3 pool [num_blocks][B][Hkv][D] of bytes as a 4-D tensor whose box is
-// one block of one kv head: B rows of D bytes, with the 128-byte swizzle
-// when a row is 128 bytes (else dense).
-static bool encode_pool_map_fp8(CUtensorMap* map, const void* pool, int32_t head_dim,
+// A pool [num_blocks][B][Hkv][D] of one-byte codes as a 4-D tensor whose
+// box is one block of one kv head: B rows of D bytes, with the 128-byte
+// swizzle when a row is 128 bytes (else dense).
+static bool encode_pool_map_q8(CUtensorMap* map, const void* pool, int32_t head_dim,
                                 int32_t num_kv_heads, int32_t block_size, int64_t num_blocks)
 {
     const CUtensorMapSwizzle swz =
@@ -799,16 +800,17 @@ static bool encode_pool_map_fp8(CUtensorMap* map, const void* pool, int32_t head
     return res == CUDA_SUCCESS;
 }
 
-template <typename T, int D, int BS, int G>
-static pa_status launch_decode_fp8(const DecodeArgs& a, float v_scale)
+template <typename Codes, typename T, int D, int BS, int G>
+static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
 {
-    using S = Fp8Shape<D, BS, G>;
+    using S = Q8Shape<D, BS, G>;
     static std::atomic<uint64_t> attr_done{0};
-    auto kernel = paged_decode_fp8_kernel<T, D, BS, G>;
+    auto kernel = std::is_same<Codes, Int8Codes>::value ? paged_decode_int8_kernel<T, D, BS, G>
+                                                        : paged_decode_fp8_kernel<T, D, BS, G>;
     if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
     CUtensorMap tm_k, tm_v;
-    if (!encode_pool_map_fp8(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
-        !encode_pool_map_fp8(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
+    if (!encode_pool_map_q8(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
+        !encode_pool_map_q8(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks))
         return PA_ERR_CUDA;
     dim3 grid(a.num_kv_heads, a.max_parts, a.num_seqs);
     pa_status st = launch_overlapped(
@@ -829,26 +831,26 @@ static pa_status launch_decode_fp8(const DecodeArgs& a, float v_scale)
                              a.partition_size, a.max_parts);
 }
 
-template <typename T, int D, int BS>
-static pa_status dispatch_fp8_group(const DecodeArgs& a, float v_scale)
+template <typename Codes, typename T, int D, int BS>
+static pa_status dispatch_q8_group(const DecodeArgs& a, float v_scale)
 {
     switch (a.num_q_heads / a.num_kv_heads) {
-    case 1: return launch_decode_fp8<T, D, BS, 1>(a, v_scale);
-    case 2: return launch_decode_fp8<T, D, BS, 2>(a, v_scale);
-    case 4: return launch_decode_fp8<T, D, BS, 4>(a, v_scale);
-    case 8: return launch_decode_fp8<T, D, BS, 8>(a, v_scale);
+    case 1: return launch_decode_q8<Codes, T, D, BS, 1>(a, v_scale);
+    case 2: return launch_decode_q8<Codes, T, D, BS, 2>(a, v_scale);
+    case 4: return launch_decode_q8<Codes, T, D, BS, 4>(a, v_scale);
+    case 8: return launch_decode_q8<Codes, T, D, BS, 8>(a, v_scale);
     default: return PA_ERR_UNSUPPORTED;
     }
 }
 
-template <typename T>
-static pa_status dispatch_fp8(const DecodeArgs& a, float v_scale)
+template <typename Codes, typename T>
+static pa_status dispatch_q8(const DecodeArgs& a, float v_scale)
 {
     const int32_t d = a.head_dim, b = a.block_size;
-    if (d == 64 && b == 16) return dispatch_fp8_group<T, 64, 16>(a, v_scale);
-    if (d == 64 && b == 32) return dispatch_fp8_group<T, 64, 32>(a, v_scale);
-    if (d == 128 && b == 16) return dispatch_fp8_group<T, 128, 16>(a, v_scale);
-    if (d == 128 && b == 32) return dispatch_fp8_group<T, 128, 32>(a, v_scale);
+    if (d == 64 && b == 16) return dispatch_q8_group<Codes, T, 64, 16>(a, v_scale);
+    if (d == 64 && b == 32) return dispatch_q8_group<Codes, T, 64, 32>(a, v_scale);
+    if (d == 128 && b == 16) return dispatch_q8_group<Codes, T, 128, 16>(a, v_scale);
+    if (d == 128 && b == 32) return dispatch_q8_group<Codes, T, 128, 32>(a, v_scale);
     return PA_ERR_UNSUPPORTED;
 }
 
@@ -1082,6 +1084,9 @@ extern "C" size_t pa_paged_decode_workspace_size(int32_t num_seqs, int32_t num_q
 
 namespace pa {
 
+// Element format of the K/V pools a decode call reads.
+enum class KvCodes { kPlain, kE4m3, kInt8 };   // 16-bit elements, or one-byte codes
+
 static pa_status decode_impl(void* out, const void* query, const void* k_cache, const void* v_cache,
                              const int32_t* block_tables, const int32_t* context_lens,
                              int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
@@ -1089,8 +1094,9 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
                              int64_t num_blocks, int32_t max_context_len, float scale,
                              int32_t partition_size, void* workspace, size_t workspace_bytes,
                              pa_dtype dtype, int32_t* d_status, pa_stream_t stream,
-                             const void* new_key, const void* new_value, bool fp8 = false,
-                             float k_scale = 1.f, float v_scale = 1.f)
+                             const void* new_key, const void* new_value,
+                             KvCodes codes = KvCodes::kPlain, float k_scale = 1.f,
+                             float v_scale = 1.f)
 {
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       max_context_len, partition_size);
@@ -1105,7 +1111,8 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     if (new_key != nullptr &&
         (new_value == nullptr || !aligned16(new_key) || !aligned16(new_value)))
         return PA_ERR_INVALID_ARG;
-    if (fp8) {
+    const bool quantised = codes != KvCodes::kPlain;
+    if (quantised) {
         if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale))
             return PA_ERR_INVALID_ARG;
         if (block_size % 16 != 0) return PA_ERR_UNSUPPORTED;
@@ -1134,7 +1141,7 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.max_blocks_per_seq = max_blocks_per_seq;
     a.num_blocks = num_blocks;
     a.max_context_len = max_context_len;
-    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * (fp8 ? k_scale : 1.0) *
+    a.scale_log2 = static_cast<float>(static_cast<double>(scale) * (quantised ? k_scale : 1.0) *
                                       1.4426950408889634);
     a.partition_size = partition;
     a.max_parts = max_parts;
@@ -1147,7 +1154,7 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.stream = stream;
     a.new_key = new_key;
     a.new_value = new_value;
-    if (fp8) {
+    if (quantised) {
         a.k_inv = 1.0f / k_scale;      // the quantising write's fp32(1 / scale)
         a.v_inv = 1.0f / v_scale;
     }
@@ -1160,9 +1167,12 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     if (num_seqs <= kThreads && ctas > 2 * static_cast<int64_t>(sm_count()) &&
         (max_parts == 1 || num_seqs <= 32))
         a.lpt_seqs = num_seqs;
-    if (fp8)
-        return dtype == PA_DTYPE_F16 ? dispatch_fp8<__half>(a, v_scale)
-                                     : dispatch_fp8<__nv_bfloat16>(a, v_scale);
+    if (codes == KvCodes::kE4m3)
+        return dtype == PA_DTYPE_F16 ? dispatch_q8<E4m3Codes, __half>(a, v_scale)
+                                     : dispatch_q8<E4m3Codes, __nv_bfloat16>(a, v_scale);
+    if (codes == KvCodes::kInt8)
+        return dtype == PA_DTYPE_F16 ? dispatch_q8<Int8Codes, __half>(a, v_scale)
+                                     : dispatch_q8<Int8Codes, __nv_bfloat16>(a, v_scale);
     return dtype == PA_DTYPE_F16 ? dispatch_dim<__half>(a) : dispatch_dim<__nv_bfloat16>(a);
 }
 
@@ -1198,8 +1208,8 @@ extern "C" pa_status pa_paged_decode_fp8(void* out, const void* query, const voi
     return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
                            num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                            num_blocks, max_context_len, scale, partition_size, workspace,
-                           workspace_bytes, dtype, d_status, stream, nullptr, nullptr, true,
-                           k_scale, v_scale);
+                           workspace_bytes, dtype, d_status, stream, nullptr, nullptr,
+                           pa::KvCodes::kE4m3, k_scale, v_scale);
 }
 
 extern "C" pa_status pa_paged_decode_fp8_append(
@@ -1214,8 +1224,42 @@ extern "C" pa_status pa_paged_decode_fp8_append(
     return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
                            num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
                            num_blocks, max_context_len, scale, partition_size, workspace,
-                           workspace_bytes, dtype, d_status, stream, key, value, true, k_scale,
-                           v_scale);
+                           workspace_bytes, dtype, d_status, stream, key, value,
+                           pa::KvCodes::kE4m3, k_scale, v_scale);
+}
+
+extern "C" pa_status pa_paged_decode_int8(void* out, const void* query, const void* k_cache,
+                                          const void* v_cache, const int32_t* block_tables,
+                                          const int32_t* context_lens, int32_t num_seqs,
+                                          int32_t num_q_heads, int32_t num_kv_heads,
+                                          int32_t head_dim, int32_t block_size,
+                                          int32_t max_blocks_per_seq, int64_t num_blocks,
+                                          int32_t max_context_len, float scale, float k_scale,
+                                          float v_scale, int32_t partition_size, void* workspace,
+                                          size_t workspace_bytes, pa_dtype dtype,
+                                          int32_t* d_status, pa_stream_t stream)
+{
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, nullptr, nullptr,
+                           pa::KvCodes::kInt8, k_scale, v_scale);
+}
+
+extern "C" pa_status pa_paged_decode_int8_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale,
+    float k_scale, float v_scale, int32_t partition_size, void* workspace, size_t workspace_bytes,
+    pa_dtype dtype, int32_t* d_status, pa_stream_t stream)
+{
+    if (key == nullptr || value == nullptr) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, key, value,
+                           pa::KvCodes::kInt8, k_scale, v_scale);
 }
 
 extern "C" pa_status pa_paged_decode_append(void* out, const void* query, const void* key,

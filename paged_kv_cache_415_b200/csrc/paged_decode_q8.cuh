@@ -1,5 +1,5 @@
-// paged_decode_fp8.cuh -- decode over K/V pools stored in FP8 (e4m3) with
-// per-tensor scales.  Included by paged_decode.cu.
+// paged_decode_q8.cuh -- decode over K/V pools of one-byte codes (e4m3 or
+// int8, pa_codes.cuh) with per-pool scales.  Included by paged_decode.cu.
 //
 // "PagedAttention：大模型KV Cache分页管理优化实践" §7 and "vLLM用虚拟内存分页思想
 // 管理KV Cache" (工程实践与局限) name low-precision storage of the cached blocks;
@@ -18,18 +18,21 @@
 //
 // Each lane reads its A fragments straight from the byte tile, pairs codes
 // with byte permutes where two tokens share a register (V^T), and widens
-// them exactly with cvt.rn.f16x2.e4m3x2 (every e4m3 value is an fp16 value).
-// The contraction index may be permuted freely as long as both operands
-// follow it, so every lane reads whole 16-byte runs of one token row.  P
-// moves from the accumulator layout (tokens x heads) to the B layout (heads
-// x tokens) through a 384-byte shared tile with stmatrix.trans / ldmatrix.
-// Scales: k_scale folds into the score scale, v_scale into the output.  The
-// query is rounded once to fp16 (exact for fp16 queries).
+// them exactly to fp16 (Codes::widen4: one cvt per pair for e4m3, a byte
+// permute and one packed subtract per pair for int8).  The contraction index
+// may be permuted freely as long as both operands follow it, so every lane
+// reads whole 16-byte runs of one token row.  P moves from the accumulator
+// layout (tokens x heads) to the B layout (heads x tokens) through a
+// 384-byte shared tile with stmatrix.trans / ldmatrix.  Scales: k_scale
+// folds into the score scale, v_scale into the output.  The query is
+// rounded once to fp16 (exact for fp16 queries).
+
+#include "pa_codes.cuh"
 
 namespace pa {
 
 template <int D, int BS, int G>
-struct Fp8Shape {
+struct Q8Shape {
     static constexpr int SLICES = BS / 16;           // 16-token MMA slices per block
     static constexpr int KW = D / 16;                // k-steps of S^T; 4-code words per K row per lane
     static constexpr int KV16 = KW / 4;              // 16-byte K loads per row per lane
@@ -57,7 +60,7 @@ struct Fp8Shape {
 // row.  D = 128: 128-byte rows with the TMA 128B swizzle (16-byte chunk c
 // of row r sits at chunk c ^ (r & 7)); D = 64: dense 64-byte rows.
 template <int D>
-__device__ __forceinline__ uint32_t fp8_tile_off(int row, int byte)
+__device__ __forceinline__ uint32_t q8_tile_off(int row, int byte)
 {
     if constexpr (D == 128)
         return static_cast<uint32_t>(row * 128 + ((((byte >> 4) ^ (row & 7)) << 4) | (byte & 15)));
@@ -65,21 +68,9 @@ __device__ __forceinline__ uint32_t fp8_tile_off(int row, int byte)
         return static_cast<uint32_t>(row * D + byte);
 }
 
-// Two e4m3 codes per 16-bit half of w -> two packed fp16 pairs, exact:
-// lo = (code0, code1), hi = (code2, code3), low byte in the low half.
-__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t& lo, uint32_t& hi)
-{
-    asm("{\n\t.reg .b16 l, h;\n\t"
-        "mov.b32 {l, h}, %2;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
-        : "=r"(lo), "=r"(hi)
-        : "r"(w));
-}
-
 // 2^x with the special-function unit's approximation (flushes subnormal
 // results to zero); the probabilities it produces are rounded to fp16 next.
-__device__ __forceinline__ float fp8_exp2(float x)
+__device__ __forceinline__ float q8_exp2(float x)
 {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -102,14 +93,14 @@ __device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, uint32_t
                  : "memory");
 }
 
-// Fused cache write for e4m3 pools: the warp that loads the block holding a
-// sequence's new token first quantises that token's K and V row for its kv
-// head exactly as the cache-write kernel does (fp32(x) * fp32(1 / scale),
-// round to nearest even, saturating at +-448) and stores the codes, then
-// makes the writes visible to the tensor-copy engine before the block's
-// tiles are requested.  Warp-uniform.
-template <typename T, int D, int BS>
-__device__ __forceinline__ void append_row_warp_fp8(
+// Fused cache write for quantised pools: the warp that loads the block
+// holding a sequence's new token first encodes that token's K and V row for
+// its kv head exactly as the cache-write kernel does (fp32(x) * fp32(1 /
+// scale), then Codes::encode2) and stores the codes, then makes the writes
+// visible to the tensor-copy engine before the block's tiles are requested.
+// Warp-uniform.
+template <typename Codes, typename T, int D, int BS>
+__device__ __forceinline__ void append_row_warp_q8(
     const T* __restrict__ new_key, const T* __restrict__ new_value, uint8_t* __restrict__ k_cache,
     uint8_t* __restrict__ v_cache, int s, int kvh, int num_kv_heads, int32_t pos, int32_t phys,
     float k_inv, float v_inv, int lane)
@@ -117,21 +108,11 @@ __device__ __forceinline__ void append_row_warp_fp8(
     const int64_t slot = static_cast<int64_t>(phys) * BS + pos % BS;
     const int64_t src = (static_cast<int64_t>(s) * num_kv_heads + kvh) * D;
     const int64_t dst = (slot * num_kv_heads + kvh) * D;
-    auto quant8 = [](const uint4& w, float inv) -> uint2 {
-        float f[8];
-        unpack8<T>(w, f);
-        uint32_t r[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            r[j] = static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(
-                make_float2(f[2 * j] * inv, f[2 * j + 1] * inv), __NV_SATFINITE, __NV_E4M3));
-        return make_uint2(r[0] | (r[1] << 16), r[2] | (r[3] << 16));
-    };
     if (lane < D / 8) {
         const uint4 kv = ld_nc_v4(new_key + src + lane * 8);
         const uint4 vv = ld_nc_v4(new_value + src + lane * 8);
-        *reinterpret_cast<uint2*>(k_cache + dst + lane * 8) = quant8(kv, k_inv);
-        *reinterpret_cast<uint2*>(v_cache + dst + lane * 8) = quant8(vv, v_inv);
+        *reinterpret_cast<uint2*>(k_cache + dst + lane * 8) = encode8<Codes, T>(kv, k_inv);
+        *reinterpret_cast<uint2*>(v_cache + dst + lane * 8) = encode8<Codes, T>(vv, v_inv);
         fence_proxy_async_global();
     }
     __syncwarp();
@@ -142,7 +123,7 @@ template <int D>
 __device__ __forceinline__ void load_words(const unsigned char* tile, int row, int byte,
                                            uint32_t (&w)[4])
 {
-    const uint4 v = *reinterpret_cast<const uint4*>(tile + fp8_tile_off<D>(row, byte));
+    const uint4 v = *reinterpret_cast<const uint4*>(tile + q8_tile_off<D>(row, byte));
     w[0] = v.x;
     w[1] = v.y;
     w[2] = v.z;
@@ -152,9 +133,9 @@ __device__ __forceinline__ void load_words(const unsigned char* tile, int row, i
 // One warp's share of a (sequence, kv head, partition) unit: Q^T fragments,
 // the O^T accumulators and the online-softmax state of heads 2*tig and
 // 2*tig + 1 (rows of N), and the code that consumes one block of K/V bytes.
-template <typename T, int D, int BS, int G>
-struct Fp8Warp {
-    using S = Fp8Shape<D, BS, G>;
+template <typename Codes, typename T, int D, int BS, int G>
+struct Q8Warp {
+    using S = Q8Shape<D, BS, G>;
     int grp, tig;
     uint32_t pt_addr;               // this lane's row of the P^T staging tile
     uint32_t qb[S::KW][2];
@@ -215,8 +196,8 @@ struct Fp8Warp {
                 for (int i = 0; i < 4; ++i) {
                     const int j = 4 * h + i;
                     uint32_t a0, a2, a1, a3;
-                    e4m3x4_to_f16x4(w0[i], a0, a2);
-                    e4m3x4_to_f16x4(w1[i], a1, a3);
+                    Codes::widen4(w0[i], a0, a2);
+                    Codes::widen4(w1[i], a1, a3);
                     if (j & 1)
                         mma_16816<__half>(sb, a0, a1, a2, a3, qb[j][0], qb[j][1]);
                     else
@@ -239,12 +220,12 @@ struct Fp8Warp {
             const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
             const float ms0 = mn0 == -INFINITY ? 0.f : mn0;
             const float ms1 = mn1 == -INFINITY ? 0.f : mn1;
-            const float c0 = fp8_exp2(m_run0 - ms0), c1 = fp8_exp2(m_run1 - ms1);
+            const float c0 = q8_exp2(m_run0 - ms0), c1 = q8_exp2(m_run1 - ms1);
             m_run0 = mn0;
             m_run1 = mn1;
             // P rounds to fp16 for the tensor cores; the sums use the rounded values
-            const uint32_t pk0 = Elem<__half>::from_float2(fp8_exp2(x0 - ms0), fp8_exp2(x1 - ms1));
-            const uint32_t pk1 = Elem<__half>::from_float2(fp8_exp2(x2 - ms0), fp8_exp2(x3 - ms1));
+            const uint32_t pk0 = Elem<__half>::from_float2(q8_exp2(x0 - ms0), q8_exp2(x1 - ms1));
+            const uint32_t pk1 = Elem<__half>::from_float2(q8_exp2(x2 - ms0), q8_exp2(x3 - ms1));
             const float2 r0 = Elem<__half>::to_float2(pk0), r1 = Elem<__half>::to_float2(pk1);
             l_run0 = l_run0 * c0 + (r0.x + r1.x);
             l_run1 = l_run1 * c1 + (r0.y + r1.y);
@@ -287,10 +268,10 @@ struct Fp8Warp {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) vd[q] = w[q];
             } else {
-                const uint2 a = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta, S::DPT * grp));
-                const uint2 b = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta + 1, S::DPT * grp));
-                const uint2 c = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta + 8, S::DPT * grp));
-                const uint2 d = *reinterpret_cast<const uint2*>(vt + fp8_tile_off<D>(ta + 9, S::DPT * grp));
+                const uint2 a = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta, S::DPT * grp));
+                const uint2 b = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 1, S::DPT * grp));
+                const uint2 c = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 8, S::DPT * grp));
+                const uint2 d = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 9, S::DPT * grp));
                 va[0] = a.x; va[1] = a.y;
                 vb[0] = b.x; vb[1] = b.y;
                 vc[0] = c.x; vc[1] = c.y;
@@ -315,12 +296,12 @@ struct Fp8Warp {
                 const uint32_t hi_cd = __byte_perm(vc[q], vd[q], 0x7362);
                 uint32_t a0, a1, a2, a3;
                 // m-tile 2q: rows grp / grp + 8 are dims DPT*grp + 4q + 0 / + 1
-                e4m3x4_to_f16x4(lo_ab, a0, a1);
-                e4m3x4_to_f16x4(lo_cd, a2, a3);
+                Codes::widen4(lo_ab, a0, a1);
+                Codes::widen4(lo_cd, a2, a3);
                 mma_16816<__half>(o[2 * q], a0, a1, a2, a3, pb0, pb1);
                 // m-tile 2q + 1: dims + 2 / + 3
-                e4m3x4_to_f16x4(hi_ab, a0, a1);
-                e4m3x4_to_f16x4(hi_cd, a2, a3);
+                Codes::widen4(hi_ab, a0, a1);
+                Codes::widen4(hi_cd, a2, a3);
                 mma_16816<__half>(o[2 * q + 1], a0, a1, a2, a3, pb0, pb1);
             }
         }
@@ -362,10 +343,12 @@ struct Fp8Warp {
 };
 
 
-template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
-    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-    T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
+// One CTA: (kv head, partition, sequence).  The kernels below instantiate
+// it for each code format.
+template <typename Codes, typename T, int D, int BS, int G>
+__device__ __forceinline__ void paged_decode_q8_cta(
+    const CUtensorMap& tm_k, const CUtensorMap& tm_v, T* __restrict__ out,
+    const T* __restrict__ query, const int32_t* __restrict__ block_tables,
     const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
     int64_t num_blocks, int32_t max_context_len, float scale_log2, float v_scale,
     int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
@@ -374,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
     uint8_t* __restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
-    using S = Fp8Shape<D, BS, G>;
+    using S = Q8Shape<D, BS, G>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -438,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
         const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
         if (warp + kWarps * k == append_blk) {
             if (phys >= 0 && static_cast<int64_t>(phys) < num_blocks)
-                append_row_warp_fp8<T, D, BS>(new_key, new_value, k_cache, v_cache, s, kvh,
+                append_row_warp_q8<Codes, T, D, BS>(new_key, new_value, k_cache, v_cache, s, kvh,
                                               num_kv_heads, ctx - 1, phys, k_inv, v_inv, lane);
             else if (lane == 0)
                 status_or(d_status, PA_STATUS_BAD_SLOT);
@@ -462,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
     for (int k = 0; k < prologue; ++k) issue(k);
     int issued = prologue;
 
-    Fp8Warp<T, D, BS, G> w;
+    Q8Warp<Codes, T, D, BS, G> w;
     w.grp = lane >> 2;
     w.tig = lane & 3;
     w.pt_addr = smem_u32(smem + S::OFF_PT + warp * S::PT_BYTES) + (lane & 7) * S::PT_STRIDE +
@@ -511,5 +494,38 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(
     merge_warps_and_store<T, D, G>(epi_o, epi_m, epi_l, out, ws_o, ws_ml, s, kvh, part, nparts,
                                    num_q_heads, max_parts);
 }
+
+#define PA_Q8_KERNEL_PARAMS                                                                     \
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,        \
+        T *__restrict__ out, const T *__restrict__ query,                                      \
+        const int32_t *__restrict__ block_tables, const int32_t *__restrict__ context_lens,    \
+        int32_t num_q_heads, int32_t max_blocks_per_seq, int64_t num_blocks,                   \
+        int32_t max_context_len, float scale_log2, float v_scale, int32_t partition_size,      \
+        int32_t max_parts, float *__restrict__ ws_o, float2 *__restrict__ ws_ml,               \
+        int32_t *d_status, int32_t lpt_seqs, const T *__restrict__ new_key,                    \
+        const T *__restrict__ new_value, uint8_t *__restrict__ k_cache,                        \
+        uint8_t *__restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv
+#define PA_Q8_KERNEL_ARGS                                                                       \
+    tm_k, tm_v, out, query, block_tables, context_lens, num_q_heads, max_blocks_per_seq,       \
+        num_blocks, max_context_len, scale_log2, v_scale, partition_size, max_parts, ws_o,     \
+        ws_ml, d_status, lpt_seqs, new_key, new_value, k_cache, v_cache, num_kv_heads, k_inv,  \
+        v_inv
+
+// e4m3 pools
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(PA_Q8_KERNEL_PARAMS)
+{
+    paged_decode_q8_cta<E4m3Codes, T, D, BS, G>(PA_Q8_KERNEL_ARGS);
+}
+
+// int8 pools
+template <typename T, int D, int BS, int G>
+__global__ void __launch_bounds__(kThreads, 4) paged_decode_int8_kernel(PA_Q8_KERNEL_PARAMS)
+{
+    paged_decode_q8_cta<Int8Codes, T, D, BS, G>(PA_Q8_KERNEL_ARGS);
+}
+
+#undef PA_Q8_KERNEL_PARAMS
+#undef PA_Q8_KERNEL_ARGS
 
 }  // namespace pa

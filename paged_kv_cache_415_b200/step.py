@@ -9,10 +9,12 @@
 and a device status word), allocated once with torch, and issues the three
 C-ABI calls on one stream.  ``HostPipeline`` feeds a ``DecodeStep`` from
 pinned host buffers step after step with the host-device copies of one step
-overlapping the kernels of the previous one.  Pools of dtype uint8 hold e4m3 codes: the step
-then uses the quantising write and the e4m3 decode with the pools' scales.  ``run_from_host`` is the same step fed from
-pinned host buffers: it copies the step's inputs to the device, runs the
-step and copies the output back, all on the same stream.
+overlapping the kernels of the previous one.  Pools of dtype uint8 (or
+float8_e4m3fn) hold e4m3 codes and pools of dtype int8 hold int8 codes: the
+step then uses that format's quantising write and decode with the pools'
+scales.  ``run_from_host`` is the same step fed from pinned host buffers: it
+copies the step's inputs to the device, runs the step and copies the output
+back, all on the same stream.
 """
 from __future__ import annotations
 
@@ -21,12 +23,23 @@ import torch
 from . import binding as B
 
 
+# Pool dtype -> (cache write, decode, decode with fused write) of that code format.
+_QUANTISED_CALLS = {
+    torch.uint8: ("pa_reshape_and_cache_fp8", "pa_paged_decode_fp8", "pa_paged_decode_fp8_append"),
+    torch.float8_e4m3fn: ("pa_reshape_and_cache_fp8", "pa_paged_decode_fp8",
+                          "pa_paged_decode_fp8_append"),
+    torch.int8: ("pa_reshape_and_cache_int8", "pa_paged_decode_int8",
+                 "pa_paged_decode_int8_append"),
+}
+
+
 class DecodeStep:
     def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor, num_seqs: int,
                  num_q_heads: int, max_context_len: int, partition_size: int = 0,
                  k_scale: float = 1.0, v_scale: float = 1.0):
         self.k_cache, self.v_cache = k_cache, v_cache
-        self.fp8 = k_cache.dtype == torch.uint8
+        names = _QUANTISED_CALLS.get(k_cache.dtype)
+        self.quantised = None if names is None else tuple(getattr(B, n) for n in names)
         self.k_scale, self.v_scale = float(k_scale), float(v_scale)
         num_blocks, self.block_size, self.num_kv_heads, self.head_dim = k_cache.shape
         self.num_blocks = num_blocks
@@ -56,20 +69,19 @@ class DecodeStep:
         if out is None:
             out = torch.empty_like(query)
         mcl = self.max_context_len if max_context_len is None else max_context_len
-        if self.fp8:
+        if self.quantised is not None:
+            write, decode, decode_append = self.quantised
             if fused_append:
-                B.pa_paged_decode_fp8_append(out, query, new_key, new_value, self.k_cache,
-                                             self.v_cache, block_tables, context_lens, mcl, scale,
-                                             self.k_scale, self.v_scale, self.partition_size,
-                                             self.workspace, self.d_status, stream)
+                decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache,
+                              block_tables, context_lens, mcl, scale, self.k_scale, self.v_scale,
+                              self.partition_size, self.workspace, self.d_status, stream)
                 return out
             if slot_mapping is not None and slot_mapping.shape[0] > 0:
-                B.pa_reshape_and_cache_fp8(new_key, new_value, self.k_cache, self.v_cache,
-                                           slot_mapping, self.k_scale, self.v_scale,
-                                           self.d_status, stream)
-            B.pa_paged_decode_fp8(out, query, self.k_cache, self.v_cache, block_tables,
-                                  context_lens, mcl, scale, self.k_scale, self.v_scale,
-                                  self.partition_size, self.workspace, self.d_status, stream)
+                write(new_key, new_value, self.k_cache, self.v_cache, slot_mapping, self.k_scale,
+                      self.v_scale, self.d_status, stream)
+            decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, mcl, scale,
+                   self.k_scale, self.v_scale, self.partition_size, self.workspace, self.d_status,
+                   stream)
             return out
         if fused_append:
             B.pa_paged_decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache,

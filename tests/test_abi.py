@@ -142,7 +142,7 @@ def test_empty_calls_are_no_ops(pa):
     ((FAKE, FAKE, FAKE + 4, 2, 2, 64, 16, 64, 0, None, None), 1),
     ((FAKE, FAKE, FAKE, -1, 2, 64, 16, 64, 0, None, None), 1),
     ((FAKE, FAKE, FAKE, 2, 2, 48, 16, 64, 0, None, None), 2),
-    ((FAKE, FAKE, FAKE, 2, 2, 64, 16, 64, 3, None, None), 2),
+    ((FAKE, FAKE, FAKE, 2, 2, 64, 16, 64, 4, None, None), 2),
 ])
 def test_copy_blocks_rejects_bad_arguments(pa, args, code):
     assert pa.LIB.pa_copy_blocks(*args) == code

@@ -21,10 +21,11 @@ def test_small_workloads_and_config_block(config):
     assert cfg["workload"].startswith(wl.name)
 
 
-def test_fp8_workload_mode():
-    wl = bench.make_workload("llama7b", seqs=3, kv_dtype="fp8")
-    assert wl.extra["kv_dtype"] == "fp8" and wl.k_cache.dtype == np.uint8
-    assert "e4m3" in bench.workload_config(wl, 0, "")["workload"]
+@pytest.mark.parametrize("kv,np_dtype,label", [("fp8", np.uint8, "e4m3"), ("int8", np.int8, "int8")])
+def test_code_workload_modes(kv, np_dtype, label):
+    wl = bench.make_workload("llama7b", seqs=3, kv_dtype=kv)
+    assert wl.extra["kv_dtype"] == kv and wl.k_cache.dtype == np_dtype
+    assert label in bench.workload_config(wl, 0, "")["workload"]
     full = bm.step_bytes(wl)
     base = bm.step_bytes(bench.make_workload("llama7b", seqs=3))
     assert full["kv"] * 2 == base["kv"]
@@ -32,8 +33,9 @@ def test_fp8_workload_mode():
 
 def test_oracle_step_counts_the_step_bytes():
     """The CPU leg times the oracle on the same step the GPU runs and
-    counts the same algorithmic bytes (all sequences, 16-bit and e4m3)."""
-    for kv in ("auto", "fp8"):
+    counts the same algorithmic bytes (all sequences, 16-bit and both code
+    formats)."""
+    for kv in ("auto", "fp8", "int8"):
         wl = bench.make_workload("llama7b", seqs=2, kv_dtype=kv)
         st = bench.OracleStep(wl)
         assert st.bytes == bm.step_bytes(wl)["total"]
@@ -52,7 +54,7 @@ def test_committed_traffic_lines_parse():
                     m = re.match(r"bench-traffic:\s*workload=(\S+)\s+bytes_per_launch=(\d+)\s+"
                                  r"source_sha256=(\w{16})\s*$", line)
                     assert m, line
-                    assert m.group(1).replace("-fp8", "") in names
+                    assert re.sub(r"-(fp8|int8)$", "", m.group(1)) in names
                     assert int(m.group(2)) > 0
                     found += 1
     assert found >= 3

@@ -104,3 +104,21 @@ def test_fp8_pools_mark_every_unheld_slot():
         assert np.all((pool[held] & 0x7F) != 0x7F)
         assert np.all(pool[~held] == 0x7F)
         assert ((pool[held] >> 3) & 0xF).max() <= 14
+
+
+def test_int8_pools_mark_every_unheld_slot_and_count_one_byte():
+    """with_int8_pools: history slots hold codes in [-127, 127], every other
+    slot -128; the byte model counts one byte per cached element."""
+    wl = gen.make_decode("b", seed=5, dtype="f16", context_lens=[1, 33, 20], num_q_heads=2,
+                         num_kv_heads=2, head_dim=16, block_size=16, num_blocks=12, scale=0.25)
+    w8 = gen.with_int8_pools(wl, seed=6)
+    assert w8.extra["kv_dtype"] == "int8" and bm.kv_elem_bytes(w8) == 1
+    assert bm.step_bytes(w8)["kv"] * 2 == bm.step_bytes(wl)["kv"]
+    for pool in (w8.k_cache, w8.v_cache):
+        assert pool.dtype == np.int8
+        held = np.zeros(pool.shape[:2], bool)
+        for s, c in enumerate(w8.context_lens):
+            for pos in range(int(c) - 1):
+                held[w8.block_tables[s, pos // 16], pos % 16] = True
+        assert pool[held].min() >= -127
+        assert np.all(pool[~held] == -128)

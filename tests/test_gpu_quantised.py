@@ -1,9 +1,10 @@
-"""FP8 (e4m3) K/V pools on the GPU against the oracle.
+"""Quantised K/V pools (e4m3 and int8 codes) on the GPU against the oracle.
 
-The quantising cache write is compared bit for bit with the oracle over the
-whole pool (every untouched byte included).  Decode over e4m3 pools is
-compared with the fp64 oracle of the dequantised pools at the tolerance of
-the 16-bit path, |gpu - oracle| <= 2e-3 + 1e-2 |oracle|: the codes widen to
+Every test runs for both code formats.  The quantising cache write is
+compared bit for bit with the oracle over the whole pool (every untouched
+byte included).  Decode over the codes is compared with the fp64 oracle of
+the dequantised pools at the tolerance of the 16-bit path,
+|gpu - oracle| <= 2e-3 + 1e-2 |oracle|: the codes of both formats widen to
 fp16 exactly, so the only extra rounding is the query's to fp16 (exact for
 fp16 queries; for bf16 ones it only touches values below 2^-14) next to the
 probabilities' rounding that the 16-bit tensor-core path has already."""
@@ -20,18 +21,38 @@ from workloads import generators as gen
 
 pytestmark = pytest.mark.gpu
 
+CODES = ["fp8", "int8"]
+_NP = {"fp8": np.uint8, "int8": np.int8}
 
-def _u8(a: np.ndarray) -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint8)).cuda()
+
+def _pool(a: np.ndarray, codes: str) -> torch.Tensor:
+    """Raw code bytes on the device: uint8 for e4m3, int8 for int8 pools."""
+    return torch.from_numpy(np.ascontiguousarray(a).view(_NP[codes])).cuda()
 
 
-class Fp8Device:
-    """A with_fp8_pools workload on the device; step = write, then decode."""
+def _random_pool(rng, shape, codes):
+    return rng.integers(0, 256, size=shape, dtype=np.uint8).view(_NP[codes])
+
+
+def _calls(codes):
+    """(cache write, decode, decode with fused write) of the binding."""
+    from paged_kv_cache_415_b200 import binding as B
+    return (getattr(B, f"pa_reshape_and_cache_{codes}"), getattr(B, f"pa_paged_decode_{codes}"),
+            getattr(B, f"pa_paged_decode_{codes}_append"))
+
+
+def _oracle_calls(codes):
+    return (getattr(oracle, f"reshape_and_cache_{codes}"), getattr(oracle, f"paged_decode_{codes}"))
+
+
+class Q8Device:
+    """A with_code_pools workload on the device; step = write, then decode."""
 
     def __init__(self, wl):
         self.wl = wl
+        self.codes = wl.extra["kv_dtype"]
         self.query = to_dev(wl.query, wl.dtype)
-        self.k_cache, self.v_cache = _u8(wl.k_cache), _u8(wl.v_cache)
+        self.k_cache, self.v_cache = _pool(wl.k_cache, self.codes), _pool(wl.v_cache, self.codes)
         self.block_tables = torch.from_numpy(wl.block_tables).cuda()
         self.context_lens = torch.from_numpy(wl.context_lens).cuda()
         self.new_key = to_dev(wl.new_key, wl.dtype)
@@ -41,9 +62,8 @@ class Fp8Device:
         self.ks, self.vs = wl.extra["k_scale"], wl.extra["v_scale"]
 
     def write(self):
-        from paged_kv_cache_415_b200 import binding as B
-        B.pa_reshape_and_cache_fp8(self.new_key, self.new_value, self.k_cache, self.v_cache,
-                                   self.slot_mapping, self.ks, self.vs, self.d_status)
+        _calls(self.codes)[0](self.new_key, self.new_value, self.k_cache, self.v_cache,
+                              self.slot_mapping, self.ks, self.vs, self.d_status)
 
     def decode(self, partition_size=None, block_tables=None, context_lens=None,
                max_context_len=None):
@@ -57,7 +77,7 @@ class Fp8Device:
                                                     wl.head_dim, wl.block_size, mcl, p)
         ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
         out = torch.full_like(self.query, float("nan"))
-        B.pa_paged_decode_fp8(out, self.query, self.k_cache, self.v_cache, bt, cl, mcl, wl.scale,
+        _calls(self.codes)[1](out, self.query, self.k_cache, self.v_cache, bt, cl, mcl, wl.scale,
                               self.ks, self.vs, p, ws, self.d_status)
         return out
 
@@ -67,14 +87,22 @@ class Fp8Device:
 
 def _oracle_pools(wl):
     kc, vc = wl.k_cache.copy(), wl.v_cache.copy()
-    st = oracle.reshape_and_cache_fp8(wl.new_key, wl.new_value, kc, vc, wl.slot_mapping,
-                                      wl.block_size, wl.dtype, wl.extra["k_scale"],
-                                      wl.extra["v_scale"])
+    st = _oracle_calls(wl.extra["kv_dtype"])[0](wl.new_key, wl.new_value, kc, vc,
+                                                wl.slot_mapping, wl.block_size, wl.dtype,
+                                                wl.extra["k_scale"], wl.extra["v_scale"])
     return kc, vc, st
 
 
+def _oracle_decode(wl, kc, vc, tables=None, ctx=None):
+    tables = wl.block_tables if tables is None else tables
+    ctx = wl.context_lens if ctx is None else ctx
+    return _oracle_calls(wl.extra["kv_dtype"])[1](wl.query, kc, vc, tables, ctx, wl.scale,
+                                                  wl.dtype, wl.extra["k_scale"],
+                                                  wl.extra["v_scale"])
+
+
 def _parity(wl, partition_size=None, what=""):
-    dev = Fp8Device(wl)
+    dev = Q8Device(wl)
     dev.write()
     out = dev.decode(partition_size)
     torch.cuda.synchronize()
@@ -82,8 +110,7 @@ def _parity(wl, partition_size=None, what=""):
     assert st == 0
     assert np.array_equal(dev.k_cache.cpu().numpy(), kc), f"{what}: K pool"
     assert np.array_equal(dev.v_cache.cpu().numpy(), vc), f"{what}: V pool"
-    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, wl.context_lens,
-                                      wl.scale, wl.dtype, wl.extra["k_scale"], wl.extra["v_scale"])
+    ref, st = _oracle_decode(wl, kc, vc)
     assert st == 0
     assert_close(to_f64(out), ref, what or wl.name)
     assert dev.status() == 0
@@ -92,17 +119,17 @@ def _parity(wl, partition_size=None, what=""):
 
 # ---- the quantising cache write -------------------------------------------------
 
+@pytest.mark.parametrize("codes", CODES)
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("scales", [(1 / 64, 1 / 64), (0.0371, 0.2113)], ids=["pow2", "odd"])
-def test_cache_write_bit_exact(dtype, scales):
+def test_cache_write_bit_exact(codes, dtype, scales):
     """Random codes in the pools (a stray write anywhere shows), a mix of
     ordinary, saturating and special values (inf, NaN, -0) in the rows,
     padding slots (-1) and one slot past the pool (status 2)."""
-    from paged_kv_cache_415_b200 import binding as B
     rng = np.random.Generator(np.random.PCG64(31 if dtype == "f16" else 32))
     nb, b, h, d = 24, 16, 4, 128
-    kc = rng.integers(0, 256, size=(nb, b, h, d), dtype=np.uint8)
-    vc = rng.integers(0, 256, size=(nb, b, h, d), dtype=np.uint8)
+    kc = _random_pool(rng, (nb, b, h, d), codes)
+    vc = _random_pool(rng, (nb, b, h, d), codes)
     t = 40
     x = rng.standard_normal((2, t, h, d)).astype(np.float32)
     x[:, ::3] *= 40.0                                       # saturates for small scales
@@ -113,158 +140,166 @@ def test_cache_write_bit_exact(dtype, scales):
     slots[5] = -1
     slots[9] = nb * b + 3
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dk, dv = _u8(kc), _u8(vc)
-    B.pa_reshape_and_cache_fp8(to_dev(key, dtype), to_dev(val, dtype), dk, dv,
-                               torch.from_numpy(slots).cuda(), scales[0], scales[1], status)
+    dk, dv = _pool(kc, codes), _pool(vc, codes)
+    _calls(codes)[0](to_dev(key, dtype), to_dev(val, dtype), dk, dv,
+                     torch.from_numpy(slots).cuda(), scales[0], scales[1], status)
     torch.cuda.synchronize()
     ek, ev = kc.copy(), vc.copy()
-    st = oracle.reshape_and_cache_fp8(key, val, ek, ev, slots, b, dtype, scales[0], scales[1])
+    st = _oracle_calls(codes)[0](key, val, ek, ev, slots, b, dtype, scales[0], scales[1])
     assert np.array_equal(dk.cpu().numpy(), ek)
     assert np.array_equal(dv.cpu().numpy(), ev)
     assert int(status.item()) == st == 2
 
 
-def test_cache_write_rejects_bad_scales():
+@pytest.mark.parametrize("codes", CODES)
+def test_cache_write_rejects_bad_scales(codes):
     from paged_kv_cache_415_b200 import binding as B
-    kc = torch.zeros((4, 16, 2, 64), dtype=torch.uint8, device="cuda")
+    kc = torch.zeros((4, 16, 2, 64), dtype=torch.from_numpy(np.zeros(1, _NP[codes])).dtype,
+                     device="cuda")
     key = torch.zeros((1, 2, 64), dtype=torch.float16, device="cuda")
     slots = torch.zeros(1, dtype=torch.int64, device="cuda")
     for ks in (0.0, -1.0, float("inf"), float("nan")):
         with pytest.raises(B.PAError):
-            B.pa_reshape_and_cache_fp8(key, key, kc, kc.clone(), slots, ks, 1.0)
+            _calls(codes)[0](key, key, kc, kc.clone(), slots, ks, 1.0)
     assert not kc.any()
 
 
-def test_copy_blocks_on_fp8_pools():
+@pytest.mark.parametrize("codes", CODES)
+def test_copy_blocks_on_code_pools(codes):
     """pa_copy_blocks with the one-byte element type moves whole blocks of
     codes (checked against the oracle's copy on the same bytes)."""
     from paged_kv_cache_415_b200 import binding as B
     rng = np.random.Generator(np.random.PCG64(33))
-    kc = rng.integers(0, 256, size=(12, 16, 2, 64), dtype=np.uint8)
-    vc = rng.integers(0, 256, size=(12, 16, 2, 64), dtype=np.uint8)
+    kc = _random_pool(rng, (12, 16, 2, 64), codes)
+    vc = _random_pool(rng, (12, 16, 2, 64), codes)
     m = np.array([[1, 4], [7, 2], [3, 11]], dtype=np.int64)
-    dk, dv = _u8(kc), _u8(vc)
+    dk, dv = _pool(kc, codes), _pool(vc, codes)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     B.pa_copy_blocks(dk, dv, torch.from_numpy(m).cuda(), status)
     torch.cuda.synchronize()
     # the oracle copies 16-bit elements: the same bytes seen as pairs
     ek, ev = kc.copy().view(np.uint16), vc.copy().view(np.uint16)
     assert oracle.copy_blocks(ek, ev, m) == 0
-    assert np.array_equal(dk.cpu().numpy(), ek.view(np.uint8))
-    assert np.array_equal(dv.cpu().numpy(), ev.view(np.uint8))
+    assert np.array_equal(dk.cpu().numpy(), ek.view(_NP[codes]))
+    assert np.array_equal(dv.cpu().numpy(), ev.view(_NP[codes]))
     assert int(status.item()) == 0
 
 
-# ---- decode over e4m3 pools -------------------------------------------------------
+# ---- decode over the codes --------------------------------------------------------
 
-def _instance(head_dim, block_size, group, dtype, partition_blocks=4):
+def _instance(codes, head_dim, block_size, group, dtype, partition_blocks=4):
     rng = np.random.Generator(np.random.PCG64(head_dim * 1000 + block_size * 10 + group + 5))
     ctx = rng.integers(1, 300, size=3, endpoint=True)
     ctx[0] = 1
     nb = int(sum(-(-int(c) // block_size) for c in ctx)) + 8
-    wl = gen.make_decode("fp8-instance", seed=78, dtype=dtype, context_lens=ctx,
+    wl = gen.make_decode("q8-instance", seed=78, dtype=dtype, context_lens=ctx,
                          num_q_heads=2 * group, num_kv_heads=2, head_dim=head_dim,
                          block_size=block_size, num_blocks=nb, scale=1 / math.sqrt(head_dim),
                          partition_size=partition_blocks * block_size)
-    return gen.with_fp8_pools(wl, seed=head_dim + block_size + group)
+    return gen.with_code_pools(wl, codes, seed=head_dim + block_size + group)
 
 
+@pytest.mark.parametrize("codes", CODES)
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
 @pytest.mark.parametrize("group", [1, 2, 4, 8])
 @pytest.mark.parametrize("block_size", [16, 32])
 @pytest.mark.parametrize("head_dim", [64, 128])
-def test_every_fp8_instance(head_dim, block_size, group, dtype):
+def test_every_code_instance(head_dim, block_size, group, dtype, codes):
     """Each (head_dim, block_size, group, query dtype) instance on ragged
     contexts spanning several blocks, warps and partitions of 4 blocks."""
-    _parity(_instance(head_dim, block_size, group, dtype),
-            what=f"fp8 D{head_dim} B{block_size} G{group} {dtype}")
+    _parity(_instance(codes, head_dim, block_size, group, dtype),
+            what=f"{codes} D{head_dim} B{block_size} G{group} {dtype}")
 
 
+@pytest.mark.parametrize("codes", CODES)
 @pytest.mark.parametrize("partition", [16, 512, 0])
-def test_fp8_partition_sweep(partition):
-    wl = gen.with_fp8_pools(oracle_pins.small_gqa(seqs=6), seed=40)
-    _parity(wl, partition_size=partition, what=f"fp8 gqa P{partition}")
+def test_code_partition_sweep(partition, codes):
+    wl = gen.with_code_pools(oracle_pins.small_gqa(seqs=6), codes, seed=40)
+    _parity(wl, partition_size=partition, what=f"{codes} gqa P{partition}")
 
 
-def test_fp8_odd_scales_and_single_token():
+@pytest.mark.parametrize("codes", CODES)
+def test_code_odd_scales_and_single_token(codes):
     """Scales that are not powers of two; a one-token context returns
     v_scale * v0 (to output rounding)."""
     wl = oracle_pins.small_llama(seqs=5)
     ctx = wl.context_lens.copy()
     ctx[0] = 1
-    wl = gen.make_decode("fp8-odd", seed=79, dtype="bf16", context_lens=ctx, num_q_heads=8,
+    wl = gen.make_decode("q8-odd", seed=79, dtype="bf16", context_lens=ctx, num_q_heads=8,
                          num_kv_heads=8, head_dim=128, block_size=16, num_blocks=160,
                          scale=1 / math.sqrt(128))
-    wl = gen.with_fp8_pools(wl, seed=41, k_scale=0.0371, v_scale=0.2113)
-    _parity(wl, partition_size=64, what="fp8 odd scales")
+    pools = {"fp8": gen.with_fp8_pools, "int8": gen.with_int8_pools}[codes]
+    wl = pools(wl, seed=41, k_scale=0.0371, v_scale=0.2113)
+    _parity(wl, partition_size=64, what=f"{codes} odd scales")
 
 
-def test_fp8_unsupported_and_invalid():
+@pytest.mark.parametrize("codes", CODES)
+def test_code_unsupported_and_invalid(codes):
     """Block size 8 has no one-byte tile path (UNSUPPORTED); non-positive or
     non-finite scales are INVALID_ARG; nothing is written."""
     from paged_kv_cache_415_b200 import binding as B
-    wl8 = gen.make_decode("fp8-b8", seed=80, dtype="f16", context_lens=[20, 5], num_q_heads=2,
+    wl8 = gen.make_decode("q8-b8", seed=80, dtype="f16", context_lens=[20, 5], num_q_heads=2,
                           num_kv_heads=2, head_dim=64, block_size=8, num_blocks=8, scale=0.125)
-    wl8 = gen.with_fp8_pools(wl8, seed=42)
-    dev = Fp8Device(wl8)
+    wl8 = gen.with_code_pools(wl8, codes, seed=42)
+    dev = Q8Device(wl8)
     with pytest.raises(B.PAError, match="UNSUPPORTED|unsupported"):
         dev.decode()
-    dev = Fp8Device(_instance(64, 16, 1, "f16"))
+    dev = Q8Device(_instance(codes, 64, 16, 1, "f16"))
     for ks in (0.0, float("nan")):
         dev.ks = ks
         with pytest.raises(B.PAError):
             dev.decode()
 
 
-def test_fp8_empty_context_and_bad_block():
+@pytest.mark.parametrize("codes", CODES)
+def test_code_empty_context_and_bad_block(codes):
     """ctx 0 -> zero row; an out-of-pool block id is skipped and flagged
     (status 1) exactly as the oracle does."""
-    wl = gen.with_fp8_pools(oracle_pins.small_llama(seqs=4), seed=43)
+    wl = gen.with_code_pools(oracle_pins.small_llama(seqs=4), codes, seed=43)
     kc, vc, _ = _oracle_pools(wl)
     wl.k_cache, wl.v_cache = kc, vc
-    dev = Fp8Device(wl)
+    dev = Q8Device(wl)
     ctx = wl.context_lens.copy()
     ctx[0] = 0
     out = dev.decode(context_lens=torch.from_numpy(ctx).cuda(), partition_size=64)
-    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, ctx, wl.scale, wl.dtype,
-                                      dev.ks, dev.vs)
+    ref, st = _oracle_decode(wl, kc, vc, ctx=ctx)
     assert_close(to_f64(out), ref)
     assert dev.status() == st == 0
     tables = wl.block_tables.copy()
     s = int(np.argmax(wl.context_lens))
     tables[s, 0] = wl.num_blocks + 7
     out = dev.decode(block_tables=torch.from_numpy(tables).cuda(), partition_size=64)
-    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, tables, wl.context_lens, wl.scale,
-                                      wl.dtype, dev.ks, dev.vs)
+    ref, st = _oracle_decode(wl, kc, vc, tables=tables)
     assert st == 1 and dev.status() == 1
     assert_close(to_f64(out), ref)
 
 
-def test_fp8_bad_context():
+@pytest.mark.parametrize("codes", CODES)
+def test_code_bad_context(codes):
     """A negative context gives a zero row and PA_STATUS_BAD_CONTEXT, the other
     rows are unaffected, for a small batch and for one of 300 sequences."""
     for seqs in (5, 300):
         ctx = np.random.Generator(np.random.PCG64(seqs)).integers(1, 70, size=seqs, endpoint=True)
         nb = int(sum(-(-int(c) // 16) for c in ctx)) + 8
-        wl = gen.make_decode("fp8-many", seed=81, dtype="bf16", context_lens=ctx, num_q_heads=4,
+        wl = gen.make_decode("q8-many", seed=81, dtype="bf16", context_lens=ctx, num_q_heads=4,
                              num_kv_heads=2, head_dim=64, block_size=16, num_blocks=nb,
                              scale=0.125, partition_size=32)
-        wl = gen.with_fp8_pools(wl, seed=45)
+        wl = gen.with_code_pools(wl, codes, seed=45)
         kc, vc, _ = _oracle_pools(wl)
         wl.k_cache, wl.v_cache = kc, vc
-        dev = Fp8Device(wl)
+        dev = Q8Device(wl)
         bad = wl.context_lens.copy()
         bad[1] = -3
         out = dev.decode(context_lens=torch.from_numpy(bad).cuda())
-        ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, bad, wl.scale,
-                                          wl.dtype, dev.ks, dev.vs)
+        ref, st = _oracle_decode(wl, kc, vc, ctx=bad)
         assert st == 4 and dev.status() == 4, (seqs, st, dev.status())
         assert_close(to_f64(out), ref, f"{seqs} seqs")
 
 
-def test_fp8_deterministic():
-    wl = _instance(128, 16, 4, "bf16")
-    dev = Fp8Device(wl)
+@pytest.mark.parametrize("codes", CODES)
+def test_code_deterministic(codes):
+    wl = _instance(codes, 128, 16, 4, "bf16")
+    dev = Q8Device(wl)
     dev.write()
     a = dev.decode()
     b = dev.decode()
@@ -272,55 +307,59 @@ def test_fp8_deterministic():
 
 
 @pytest.mark.slow
+@pytest.mark.parametrize("codes", CODES)
 @pytest.mark.parametrize("name", ["llama7b", "mistral7b"])
-def test_fp8_full_size(name):
-    """The full-size workload with e4m3 pools, in the launch configuration
-    the benchmark times: write + decode against the whole oracle."""
-    wl = gen.with_fp8_pools(gen.CONFIGS[name](), seed=44)
-    _parity(wl, what=name + "-fp8")
+def test_code_full_size(name, codes):
+    """The full-size workload with quantised pools, in the launch
+    configuration the benchmark times: write + decode against the whole
+    oracle."""
+    wl = gen.with_code_pools(gen.CONFIGS[name](), codes, seed=44)
+    _parity(wl, what=f"{name}-{codes}")
 
 
 # ---- the quantising write fused into the decode launch ----------------------------
 
 def _fused(wl, partition_size=None, tables=None):
     from paged_kv_cache_415_b200 import binding as B
-    dev = Fp8Device(wl)
+    dev = Q8Device(wl)
     p = wl.partition_size if partition_size is None else partition_size
     ws_bytes = B.pa_paged_decode_workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
                                                 wl.head_dim, wl.block_size, wl.max_context_len, p)
     ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device="cuda")
     out = torch.full_like(dev.query, float("nan"))
     bt = dev.block_tables if tables is None else torch.from_numpy(tables).cuda()
-    B.pa_paged_decode_fp8_append(out, dev.query, dev.new_key, dev.new_value, dev.k_cache,
-                                 dev.v_cache, bt, dev.context_lens, wl.max_context_len, wl.scale,
-                                 dev.ks, dev.vs, p, ws, dev.d_status)
+    _calls(dev.codes)[2](out, dev.query, dev.new_key, dev.new_value, dev.k_cache, dev.v_cache,
+                         bt, dev.context_lens, wl.max_context_len, wl.scale, dev.ks, dev.vs, p,
+                         ws, dev.d_status)
     torch.cuda.synchronize()
     return dev, out
 
 
+@pytest.mark.parametrize("codes", CODES)
 @pytest.mark.parametrize("head_dim,block_size,group,dtype,partition",
                          [(128, 16, 1, "f16", 0), (128, 16, 4, "bf16", 64), (64, 32, 2, "f16", 0),
                           (128, 32, 8, "bf16", 96)])
-def test_fp8_fused_append(head_dim, block_size, group, dtype, partition):
-    """pa_paged_decode_fp8_append leaves the pools exactly as the quantising
-    cache write does and returns the decode of the written pools."""
-    wl = _instance(head_dim, block_size, group, dtype)
+def test_code_fused_append(head_dim, block_size, group, dtype, partition, codes):
+    """The fused decode (pa_paged_decode_fp8_append / _int8_append) leaves
+    the pools exactly as the quantising cache write does and returns the
+    decode of the written pools."""
+    wl = _instance(codes, head_dim, block_size, group, dtype)
     assert wl.extra["one_token_per_seq"]
     dev, out = _fused(wl, partition)
     kc, vc, st = _oracle_pools(wl)
     assert st == 0
     assert np.array_equal(dev.k_cache.cpu().numpy(), kc)
     assert np.array_equal(dev.v_cache.cpu().numpy(), vc)
-    ref, st = oracle.paged_decode_fp8(wl.query, kc, vc, wl.block_tables, wl.context_lens,
-                                      wl.scale, wl.dtype, dev.ks, dev.vs)
+    ref, st = _oracle_decode(wl, kc, vc)
     assert st == 0 and dev.status() == 0
-    assert_close(to_f64(out), ref, "fp8 fused append")
+    assert_close(to_f64(out), ref, f"{codes} fused append")
 
 
-def test_fp8_fused_append_bad_slot_is_flagged():
+@pytest.mark.parametrize("codes", CODES)
+def test_code_fused_append_bad_slot_is_flagged(codes):
     """A new token whose block id lies outside the pool is not written
     (PA_STATUS_BAD_SLOT, plus PA_STATUS_BAD_BLOCK for the skipped block)."""
-    wl = _instance(128, 16, 4, "bf16")
+    wl = _instance(codes, 128, 16, 4, "bf16")
     s = int(np.argmax(wl.context_lens))
     c = int(wl.context_lens[s])
     tables = wl.block_tables.copy()
@@ -331,8 +370,7 @@ def test_fp8_fused_append_bad_slot_is_flagged():
     keep = np.ones(wl.num_seqs, bool)
     keep[s] = False
     kc, vc = wl.k_cache.copy(), wl.v_cache.copy()
-    oracle.reshape_and_cache_fp8(wl.new_key[keep], wl.new_value[keep], kc, vc,
-                                 wl.slot_mapping[keep], wl.block_size, wl.dtype,
-                                 wl.extra["k_scale"], wl.extra["v_scale"])
+    _oracle_calls(codes)[0](wl.new_key[keep], wl.new_value[keep], kc, vc, wl.slot_mapping[keep],
+                            wl.block_size, wl.dtype, wl.extra["k_scale"], wl.extra["v_scale"])
     assert np.array_equal(dev.k_cache.cpu().numpy(), kc)
     assert np.array_equal(dev.v_cache.cpu().numpy(), vc)

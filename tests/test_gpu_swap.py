@@ -12,33 +12,38 @@ pytestmark = pytest.mark.gpu
 SHAPE = (16, 8, 128)          # block_size, kv heads, head_dim
 
 
+_CODES = {"fp8": np.uint8, "int8": np.int8}       # one-byte pools: e4m3 or int8 codes
+
+
 def _pool(rng, nb, dtype):
-    if dtype == "fp8":
+    if dtype in _CODES:
         return rng.integers(0, 256, size=(nb,) + SHAPE, dtype=np.uint8)
     return rng.integers(0, 65536, size=(nb,) + SHAPE, dtype=np.uint16)
 
 
-def _dev(a, dtype):
-    if dtype == "fp8":
-        return torch.from_numpy(a).cuda()
-    t = torch.from_numpy(a.view(np.int16)).cuda()
+def _tensor(a, dtype):
+    if dtype in _CODES:
+        return torch.from_numpy(a.view(_CODES[dtype]))
+    t = torch.from_numpy(a.view(np.int16))
     return t.view(torch.float16 if dtype == "f16" else torch.bfloat16)
+
+
+def _dev(a, dtype):
+    return _tensor(a, dtype).cuda()
 
 
 def _host(a, dtype):
-    t = torch.from_numpy(a.view(np.int16) if dtype != "fp8" else a).pin_memory()
-    if dtype == "fp8":
-        return t
-    return t.view(torch.float16 if dtype == "f16" else torch.bfloat16)
+    return _tensor(a, dtype).pin_memory()
 
 
 def _bits(t):
     t = t.cpu() if t.is_cuda else t
-    return t.view(torch.uint8).numpy().copy() if t.dtype == torch.uint8 else \
-        t.view(torch.int16).numpy().view(np.uint16).copy()
+    if t.element_size() == 1:
+        return t.view(torch.uint8).numpy().copy()
+    return t.view(torch.int16).numpy().view(np.uint16).copy()
 
 
-@pytest.mark.parametrize("dtype", ["f16", "bf16", "fp8"])
+@pytest.mark.parametrize("dtype", ["f16", "bf16", "fp8", "int8"])
 def test_swap_out_then_in(dtype):
     """Evict 24 scattered device blocks into a pinned host pool, then bring
     them back into other device blocks; both directions bit-exact."""

@@ -61,9 +61,9 @@ def decode_bytes(ctx: np.ndarray, num_q_heads: int, num_kv_heads: int, head_dim:
 
 
 def kv_elem_bytes(wl) -> int:
-    """Bytes of one cached K/V element: 1 for e4m3 pools, else the element
-    type's."""
-    return 1 if wl.extra.get("kv_dtype") == "fp8" else ELEM_BYTES[wl.dtype]
+    """Bytes of one cached K/V element: 1 for e4m3 and int8 pools, else the
+    element type's."""
+    return 1 if wl.extra.get("kv_dtype") in ("fp8", "int8") else ELEM_BYTES[wl.dtype]
 
 
 def step_bytes(wl) -> dict:

@@ -181,18 +181,23 @@ def e4m3_codes(rng: np.random.Generator, shape, max_exponent_field: int = 14) ->
     return (sign | exp | mant).astype(np.uint8)
 
 
-def with_fp8_pools(wl: DecodeWorkload, seed: int, k_scale: float = 1.0 / 64.0,
-                   v_scale: float = 1.0 / 64.0) -> DecodeWorkload:
-    """A copy of a make_decode workload whose pools are e4m3 codes: every
-    slot that holds a history token gets random codes, every other slot the
-    NaN code (so reading a slot the kernel must not read poisons the
-    output).  Scales are per pool; with 1/64 the largest code (240) stands
-    for 3.75.  extra: kv_dtype = "fp8", k_scale, v_scale."""
+def int8_codes(rng: np.random.Generator, shape) -> np.ndarray:
+    """Random int8 codes, uniform in [-127, 127]."""
+    return rng.integers(-127, 128, size=shape, dtype=np.int8)
+
+
+# The code every slot without a history token holds: NaN for e4m3 (reading it
+# poisons the output), the most negative code for int8 (no NaN exists).
+INT8_POISON = -128
+
+
+def _with_code_pools(wl: DecodeWorkload, seed: int, kv_dtype: str, draw, poison, np_dtype,
+                     k_scale: float, v_scale: float) -> DecodeWorkload:
     rng = np.random.Generator(np.random.PCG64(seed))
     b = wl.block_size
     shape = (wl.num_blocks, b, wl.num_kv_heads, wl.head_dim)
-    k_cache = np.full(shape, E4M3_NAN, dtype=np.uint8)
-    v_cache = np.full(shape, E4M3_NAN, dtype=np.uint8)
+    k_cache = np.full(shape, poison, dtype=np_dtype)
+    v_cache = np.full(shape, poison, dtype=np_dtype)
     new = set(int(x) for x in wl.slot_mapping if x >= 0)
     slots = []
     for s in range(wl.num_seqs):
@@ -203,15 +208,38 @@ def with_fp8_pools(wl: DecodeWorkload, seed: int, k_scale: float = 1.0 / 64.0,
     slots = np.asarray(sorted(set(slots)), dtype=np.int64)
     row = (wl.num_kv_heads, wl.head_dim)
     if slots.size:
-        _scatter(k_cache, slots, e4m3_codes(rng, (slots.size,) + row), b)
-        _scatter(v_cache, slots, e4m3_codes(rng, (slots.size,) + row), b)
+        _scatter(k_cache, slots, draw(rng, (slots.size,) + row), b)
+        _scatter(v_cache, slots, draw(rng, (slots.size,) + row), b)
     out = DecodeWorkload(**{f: getattr(wl, f) for f in wl.__dataclass_fields__})
-    out.name = wl.name + "-fp8"
+    out.name = f"{wl.name}-{kv_dtype}"
     out.k_cache, out.v_cache = k_cache, v_cache
     out.keys = out.values = None
-    out.extra = dict(wl.extra, kv_dtype="fp8", k_scale=float(np.float32(k_scale)),
+    out.extra = dict(wl.extra, kv_dtype=kv_dtype, k_scale=float(np.float32(k_scale)),
                      v_scale=float(np.float32(v_scale)))
     return out
+
+
+def with_fp8_pools(wl: DecodeWorkload, seed: int, k_scale: float = 1.0 / 64.0,
+                   v_scale: float = 1.0 / 64.0) -> DecodeWorkload:
+    """A copy of a make_decode workload whose pools are e4m3 codes: every
+    slot that holds a history token gets random codes, every other slot the
+    NaN code (so reading a slot the kernel must not read poisons the
+    output).  Scales are per pool; with 1/64 the largest code (240) stands
+    for 3.75.  extra: kv_dtype = "fp8", k_scale, v_scale."""
+    return _with_code_pools(wl, seed, "fp8", e4m3_codes, E4M3_NAN, np.uint8, k_scale, v_scale)
+
+
+def with_int8_pools(wl: DecodeWorkload, seed: int, k_scale: float = 1.0 / 64.0,
+                    v_scale: float = 1.0 / 64.0) -> DecodeWorkload:
+    """As with_fp8_pools with int8 codes (uniform in [-127, 127]; slots
+    without a history token hold -128).  With scale 1/64 the codes stand for
+    values up to about 2.  extra: kv_dtype = "int8", k_scale, v_scale."""
+    return _with_code_pools(wl, seed, "int8", int8_codes, INT8_POISON, np.int8, k_scale, v_scale)
+
+
+def with_code_pools(wl: DecodeWorkload, kv_dtype: str, seed: int) -> DecodeWorkload:
+    """with_fp8_pools or with_int8_pools by name ("fp8" / "int8")."""
+    return {"fp8": with_fp8_pools, "int8": with_int8_pools}[kv_dtype](wl, seed=seed)
 
 
 # ---------------------------------------------------------------------------
