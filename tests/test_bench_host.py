@@ -67,3 +67,50 @@ def test_source_hash_ignores_comments_only():
     assert bench.strip_comments(src) == 'int a = 1;\n const char* s = "a//b"; char q = \'/\';'
     assert bench.strip_comments(src) == bench.strip_comments(src.replace("note", "other"))
     assert bench.strip_comments(src) != bench.strip_comments(src.replace("a = 1", "a = 2"))
+
+
+def _json_lines(text):
+    import json
+    return [json.loads(x) for x in text.splitlines() if x.startswith("{")]
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` times the oracle on the host and prints
+    one JSON line with the contract's keys; its value is its own e2e and
+    cpu_baseline value."""
+    import subprocess
+    import sys
+    res = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny",
+                          "--steps", "2", "--warmup", "1"], cwd=bench.ROOT, capture_output=True,
+                         text=True, timeout=300)
+    assert res.returncode == 0, res.stderr
+    lines = _json_lines(res.stdout)
+    assert len(lines) == 1
+    line = lines[0]
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["steps"] == 2 and line["warmup"] == 1
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["value"] == line["value"] and line["cpu_baseline"]["kind"] == "oracle"
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 == line["e2e"]["d2h_bytes_per_step"]
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Launched as the multi-GPU run is (torchrun, two ranks), only rank 0
+    runs the oracle and prints; the other rank exits 0 without output."""
+    import socket
+    import subprocess
+    import sys
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    res = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                          "--nproc-per-node", "2", "--master-addr", "127.0.0.1", "--master-port",
+                          str(port), "bench.py", "--impl", "reference", "--gpus", "2",
+                          "--config", "tiny", "--steps", "1", "--warmup", "1"],
+                         cwd=bench.ROOT, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = _json_lines(res.stdout)
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
