@@ -38,7 +38,15 @@
  *    evicts it from the cache then ([Manager, 第四部分 BlockPool]);
  *  - a request that needs more free blocks than there are fails with
  *    PA_BM_NO_SPACE and leaves every structure unchanged
- *    ([Manager, 第四部分 KVCacheManager 与 allocate_slots()]).
+ *    ([Manager, 第四部分 KVCacheManager 与 allocate_slots()]);
+ *  - swapping (optional, with a host pool attached): a group of sequences
+ *    (the beams of one request, say) moves to host blocks and back, the
+ *    mechanism of evicting a waiting request's KV to CPU memory and
+ *    restoring it when the request is scheduled again
+ *    ([VM-paging, 显存管理与调度策略设计], the eviction paragraph; [Manager,
+ *    第四部分]: the cache manager supplies the mechanism, the scheduler the
+ *    policy).  The byte copies are pa_swap_blocks calls with the pairs the
+ *    manager returns.
  *
  * Slots are physical_block * block_size + offset.  Sequence ids are any
  * int64 chosen by the caller.  The manager is not thread-safe: one caller at
@@ -109,10 +117,51 @@ PA_API int32_t pa_bm_block_table(const pa_block_manager* bm, int64_t seq_id, int
 /* Number of tokens of the sequence (-1 if unknown). */
 PA_API int32_t pa_bm_context_len(const pa_block_manager* bm, int64_t seq_id);
 
+/*
+ * Swapping.  pa_bm_attach_host_pool gives the manager host blocks
+ * [0, num_host_blocks) of a pinned host pool shaped like the device pool
+ * (once per manager).  While a sequence is swapped out it has no device
+ * blocks: pa_bm_append_slots, pa_bm_fork and pa_bm_block_table return
+ * PA_BM_BAD_ARG for it, pa_bm_context_len still answers, and
+ * pa_bm_free_sequence releases its host blocks.
+ *
+ * pa_bm_swap_out -- the group seq_ids[0 .. num_seqs) (distinct, all
+ *   resident) moves to the host pool.  Every distinct device block of the
+ *   group gets one host block, so blocks the group shares stay shared; the
+ *   group's references on the device blocks are dropped, and blocks left
+ *   without users return to the free queue (a full block keeps its hash, so
+ *   a later prefix hit or swap-in can still find it).  pairs_out receives
+ *   *num_pairs (device block, host block) pairs, int64 [capacity][2], for
+ *   pa_swap_blocks from the device pools to the host pools; those copies
+ *   must run before any kernel that writes a block allocated after this
+ *   call (stream order does it when they are enqueued first).
+ * pa_bm_swap_in -- the group (distinct, all swapped out) comes back.  Each
+ *   distinct host block becomes one device block: a full block whose hash is
+ *   still in the prefix cache is revived without a copy, any other block
+ *   gets a fresh device block and a (host block, device block) pair for
+ *   pa_swap_blocks from the host pools to the device pools, to run before the
+ *   group's next decode.  Block tables are in the same order as before.
+ * Both are all or nothing: PA_BM_NO_SPACE when the destination pool lacks
+ * room, PA_BM_CAPACITY when pairs_out has fewer than the needed entries
+ * (one per block of the group suffices), PA_BM_BAD_ARG for an unknown,
+ * repeated or wrongly placed sequence or when no host pool is attached; in
+ * each case nothing changes.
+ */
+PA_API int32_t pa_bm_attach_host_pool(pa_block_manager* bm, int32_t num_host_blocks);
+PA_API int32_t pa_bm_num_free_host_blocks(const pa_block_manager* bm);
+/* 1 if the sequence is swapped out, 0 if resident, -1 if unknown. */
+PA_API int32_t pa_bm_is_swapped(const pa_block_manager* bm, int64_t seq_id);
+PA_API int32_t pa_bm_swap_out(pa_block_manager* bm, const int64_t* seq_ids, int32_t num_seqs,
+                              int64_t* pairs_out, int32_t capacity, int32_t* num_pairs);
+PA_API int32_t pa_bm_swap_in(pa_block_manager* bm, const int64_t* seq_ids, int32_t num_seqs,
+                             int64_t* pairs_out, int32_t capacity, int32_t* num_pairs);
+
 /* Checks every invariant (counts equal table references, free queue holds
  * exactly the blocks with count 0, no cycles, cached hashes map back to
- * their blocks, internal waste <= block_size - 1).  0 = all hold, else a
- * code naming the first violated one. */
+ * their blocks, internal waste <= block_size - 1, and for the host pool:
+ * swapped sequences hold host blocks only, host counts equal references,
+ * the host free list holds exactly the host blocks with count 0).  0 = all
+ * hold, else a code naming the first violated one. */
 PA_API int32_t pa_bm_check(const pa_block_manager* bm);
 
 #ifdef __cplusplus

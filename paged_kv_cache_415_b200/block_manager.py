@@ -1,7 +1,8 @@
 """ctypes binding of the native host block manager (include/pa_block_manager.h).
 
 Argument marshalling only; the block tables, reference counts, free queue,
-copy-on-write decisions and prefix cache live in C++ inside libpa.so.
+copy-on-write decisions, prefix cache and host-pool swap bookkeeping live in
+C++ inside libpa.so.
 """
 from __future__ import annotations
 
@@ -38,6 +39,16 @@ LIB.pa_bm_context_len.argtypes = [_p, _i64]
 LIB.pa_bm_context_len.restype = _i32
 LIB.pa_bm_check.argtypes = [_p]
 LIB.pa_bm_check.restype = _i32
+LIB.pa_bm_attach_host_pool.argtypes = [_p, _i32]
+LIB.pa_bm_attach_host_pool.restype = _i32
+LIB.pa_bm_num_free_host_blocks.argtypes = [_p]
+LIB.pa_bm_num_free_host_blocks.restype = _i32
+LIB.pa_bm_is_swapped.argtypes = [_p, _i64]
+LIB.pa_bm_is_swapped.restype = _i32
+LIB.pa_bm_swap_out.argtypes = [_p, _p, _i32, _p, _i32, _p]
+LIB.pa_bm_swap_out.restype = _i32
+LIB.pa_bm_swap_in.argtypes = [_p, _p, _i32, _p, _i32, _p]
+LIB.pa_bm_swap_in.restype = _i32
 
 
 def _ptr(a):
@@ -119,3 +130,38 @@ class NativeBlockManager:
 
     def check(self) -> int:
         return int(LIB.pa_bm_check(self.h))
+
+    # ---- swapping to a host pool ----------------------------------------------
+
+    def attach_host_pool(self, num_host_blocks: int) -> None:
+        rc = LIB.pa_bm_attach_host_pool(self.h, num_host_blocks)
+        if rc != PA_BM_OK:
+            raise ValueError(f"pa_bm_attach_host_pool: {rc}")
+
+    def num_free_host(self) -> int:
+        return int(LIB.pa_bm_num_free_host_blocks(self.h))
+
+    def is_swapped(self, seq: int) -> int:
+        return int(LIB.pa_bm_is_swapped(self.h, seq))
+
+    def _swap(self, fn, name, seqs):
+        ids = np.ascontiguousarray(list(seqs), dtype=np.int64)
+        cap = max(1, sum(max(0, -(-self.context_len(int(s)) // self.block_size)) for s in ids))
+        pairs = np.empty((cap, 2), dtype=np.int64)
+        n = ctypes.c_int32(0)
+        rc = fn(self.h, _ptr(ids), ids.shape[0], _ptr(pairs), cap, ctypes.byref(n))
+        if rc == PA_BM_NO_SPACE:
+            return None
+        if rc != PA_BM_OK:
+            raise ValueError(f"{name}: {rc}")
+        return [tuple(int(x) for x in pairs[i]) for i in range(n.value)]
+
+    def swap_out(self, seqs):
+        """The group's (device block, host block) copies for pa_swap_blocks,
+        or None when the host pool is too small."""
+        return self._swap(LIB.pa_bm_swap_out, "pa_bm_swap_out", seqs)
+
+    def swap_in(self, seqs):
+        """The group's (host block, device block) copies for pa_swap_blocks,
+        or None when the device pool is too small."""
+        return self._swap(LIB.pa_bm_swap_in, "pa_bm_swap_in", seqs)

@@ -8,6 +8,7 @@
 
 #include <stdint.h>
 
+#include <algorithm>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -43,11 +44,13 @@ struct Block {
 };
 
 struct Seq {
-    std::vector<int32_t> table;
+    std::vector<int32_t> table;       // device blocks (empty while swapped out)
     int32_t len = 0;
     int64_t extra_key = 0;
     std::vector<int32_t> tokens;    // kept only with prefix caching
     uint64_t last_full_hash = kRootHash;
+    bool swapped = false;
+    std::vector<int32_t> host_table;  // host blocks while swapped out
 };
 
 }  // namespace
@@ -59,6 +62,10 @@ struct pa_block_manager {
     int32_t head = -1, tail = -1, nfree = 0;
     std::unordered_map<uint64_t, int32_t> cache;     // hash -> block
     std::unordered_map<int64_t, Seq> seqs;
+    // host pool for swapped-out sequences: reference counts and free ids
+    int32_t num_host = 0;
+    std::vector<int32_t> host_ref;
+    std::vector<int32_t> host_free;                  // a stack; the top is taken first
 
     // ---- free queue: O(1) push at the tail, pop at the head, remove anywhere
     void push_back(int32_t b)
@@ -105,6 +112,32 @@ struct pa_block_manager {
     int64_t slot_of(const Seq& q, int32_t pos) const
     {
         return static_cast<int64_t>(q.table[pos / block_size]) * block_size + pos % block_size;
+    }
+    // Hashes of a sequence's full blocks, from its tokens (prefix caching).
+    std::vector<uint64_t> full_hashes(const Seq& q) const
+    {
+        std::vector<uint64_t> h;
+        uint64_t parent = kRootHash;
+        for (int32_t j = 0; j < q.len / block_size; ++j) {
+            parent = block_hash(parent, q.extra_key,
+                                q.tokens.data() + static_cast<int64_t>(j) * block_size,
+                                block_size);
+            h.push_back(parent);
+        }
+        return h;
+    }
+    // The distinct sequences of a group, each known and in the given swap
+    // state; nullptr entries never returned.
+    bool group(const int64_t* ids, int32_t n, bool swapped, std::vector<Seq*>* out)
+    {
+        if (ids == nullptr || n <= 0 || num_host == 0) return false;
+        for (int32_t i = 0; i < n; ++i) {
+            auto it = seqs.find(ids[i]);
+            if (it == seqs.end() || it->second.swapped != swapped) return false;
+            if (std::find(out->begin(), out->end(), &it->second) != out->end()) return false;
+            out->push_back(&it->second);
+        }
+        return true;
     }
 };
 
@@ -207,7 +240,7 @@ extern "C" int32_t pa_bm_fork(pa_block_manager* bm, int64_t parent, int64_t chil
 {
     if (!bm || parent == child) return PA_BM_BAD_ARG;
     auto it = bm->seqs.find(parent);
-    if (it == bm->seqs.end() || bm->seqs.count(child)) return PA_BM_BAD_ARG;
+    if (it == bm->seqs.end() || it->second.swapped || bm->seqs.count(child)) return PA_BM_BAD_ARG;
     try {
         Seq q = it->second;
         for (int32_t b : q.table) ++bm->blocks[b].ref;
@@ -224,7 +257,7 @@ extern "C" int32_t pa_bm_append_slots(pa_block_manager* bm, int64_t seq_id, cons
 {
     if (!bm || n < 0) return PA_BM_BAD_ARG;
     auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PA_BM_BAD_ARG;
+    if (it == bm->seqs.end() || it->second.swapped) return PA_BM_BAD_ARG;
     if (bm->caching && n > 0 && tokens == nullptr) return PA_BM_BAD_ARG;
     Seq& q = it->second;
     const int32_t B = bm->block_size;
@@ -285,6 +318,8 @@ extern "C" int32_t pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id)
         Block& x = bm->blocks[*r];
         if (--x.ref == 0) bm->push_back(*r);
     }
+    for (auto r = it->second.host_table.rbegin(); r != it->second.host_table.rend(); ++r)
+        if (--bm->host_ref[*r] == 0) bm->host_free.push_back(*r);
     bm->seqs.erase(it);
     return PA_BM_OK;
 }
@@ -294,7 +329,7 @@ extern "C" int32_t pa_bm_block_table(const pa_block_manager* bm, int64_t seq_id,
 {
     if (!bm) return PA_BM_BAD_ARG;
     auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PA_BM_BAD_ARG;
+    if (it == bm->seqs.end() || it->second.swapped) return PA_BM_BAD_ARG;
     const std::vector<int32_t>& t = it->second.table;
     if (num_blocks) *num_blocks = static_cast<int32_t>(t.size());
     if (static_cast<int64_t>(t.size()) > capacity || (!t.empty() && table_out == nullptr))
@@ -310,20 +345,190 @@ extern "C" int32_t pa_bm_context_len(const pa_block_manager* bm, int64_t seq_id)
     return it == bm->seqs.end() ? -1 : it->second.len;
 }
 
+extern "C" int32_t pa_bm_attach_host_pool(pa_block_manager* bm, int32_t num_host_blocks)
+{
+    if (!bm || bm->num_host != 0 || num_host_blocks <= 0) return PA_BM_BAD_ARG;
+    try {
+        bm->host_ref.assign(num_host_blocks, 0);
+        bm->host_free.reserve(num_host_blocks);
+        for (int32_t h = num_host_blocks - 1; h >= 0; --h) bm->host_free.push_back(h);
+    } catch (...) {
+        bm->host_ref.clear();
+        bm->host_free.clear();
+        return PA_BM_BAD_ARG;
+    }
+    bm->num_host = num_host_blocks;
+    return PA_BM_OK;
+}
+
+extern "C" int32_t pa_bm_num_free_host_blocks(const pa_block_manager* bm)
+{
+    return bm ? static_cast<int32_t>(bm->host_free.size()) : 0;
+}
+
+extern "C" int32_t pa_bm_is_swapped(const pa_block_manager* bm, int64_t seq_id)
+{
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : (it->second.swapped ? 1 : 0);
+}
+
+// Evict a group to the host pool ([VM-paging, 显存管理与调度策略设计]: the KV of
+// waiting requests moves to CPU memory under pressure).  Each distinct device
+// block of the group gets one host block, so blocks the group shares stay
+// shared on the host; the group's references on the device blocks are then
+// dropped (last block first, sequence by sequence), and blocks left without
+// users return to the free queue with their hashes.
+extern "C" int32_t pa_bm_swap_out(pa_block_manager* bm, const int64_t* seq_ids, int32_t num_seqs,
+                                  int64_t* pairs_out, int32_t capacity, int32_t* num_pairs)
+{
+    if (!bm) return PA_BM_BAD_ARG;
+    try {
+        std::vector<Seq*> g;
+        if (!bm->group(seq_ids, num_seqs, false, &g)) return PA_BM_BAD_ARG;
+        std::unordered_map<int32_t, int32_t> host_of;  // device block -> host block
+        std::vector<int32_t> order;                    // distinct device blocks, first use first
+        for (Seq* q : g)
+            for (int32_t b : q->table)
+                if (host_of.emplace(b, -1).second) order.push_back(b);
+        const int32_t need = static_cast<int32_t>(order.size());
+        if (need > static_cast<int32_t>(bm->host_free.size())) return PA_BM_NO_SPACE;
+        if (need > capacity || (need > 0 && pairs_out == nullptr)) return PA_BM_CAPACITY;
+        for (Seq* q : g) q->host_table.reserve(q->table.size());
+        for (int32_t i = 0; i < need; ++i) {
+            const int32_t h = bm->host_free.back();
+            bm->host_free.pop_back();
+            host_of[order[i]] = h;
+            pairs_out[2 * i] = order[i];
+            pairs_out[2 * i + 1] = h;
+        }
+        for (Seq* q : g) {
+            for (int32_t b : q->table) {
+                const int32_t h = host_of[b];
+                ++bm->host_ref[h];
+                q->host_table.push_back(h);
+            }
+            for (auto r = q->table.rbegin(); r != q->table.rend(); ++r)
+                if (--bm->blocks[*r].ref == 0) bm->push_back(*r);
+            q->table.clear();
+            q->swapped = true;
+        }
+        if (num_pairs) *num_pairs = need;
+    } catch (...) {
+        return PA_BM_BAD_ARG;
+    }
+    return PA_BM_OK;
+}
+
+// Bring a swapped-out group back.  Each distinct host block becomes one
+// device block: a full block whose hash is still in the prefix cache is
+// revived in place (its bytes never left the device), any other block gets
+// a fresh device block and a (host, device) copy.  All or nothing.
+extern "C" int32_t pa_bm_swap_in(pa_block_manager* bm, const int64_t* seq_ids, int32_t num_seqs,
+                                 int64_t* pairs_out, int32_t capacity, int32_t* num_pairs)
+{
+    if (!bm) return PA_BM_BAD_ARG;
+    try {
+        std::vector<Seq*> g;
+        if (!bm->group(seq_ids, num_seqs, true, &g)) return PA_BM_BAD_ARG;
+        struct Need {
+            int32_t host;
+            bool full;
+            uint64_t hash;
+            int32_t revive;       // cached device block, or -1
+        };
+        std::unordered_map<int32_t, int32_t> index;    // host block -> position in needs
+        std::vector<Need> needs;
+        for (Seq* q : g) {
+            const std::vector<uint64_t> hashes = bm->caching ? bm->full_hashes(*q)
+                                                             : std::vector<uint64_t>();
+            for (size_t j = 0; j < q->host_table.size(); ++j) {
+                const int32_t h = q->host_table[j];
+                if (!index.emplace(h, static_cast<int32_t>(needs.size())).second) continue;
+                Need n{h, j < hashes.size(), j < hashes.size() ? hashes[j] : 0, -1};
+                if (n.full) {
+                    auto c = bm->cache.find(n.hash);
+                    if (c != bm->cache.end()) n.revive = c->second;
+                }
+                needs.push_back(n);
+            }
+        }
+        int32_t fresh = 0, from_free = 0;
+        std::vector<int32_t> revived;
+        for (const Need& n : needs) {
+            if (n.revive < 0) {
+                ++fresh;
+            } else if (std::find(revived.begin(), revived.end(), n.revive) == revived.end()) {
+                revived.push_back(n.revive);
+                from_free += bm->blocks[n.revive].ref == 0;
+            }
+        }
+        if (fresh + from_free > bm->nfree) return PA_BM_NO_SPACE;
+        if (fresh > capacity || (fresh > 0 && pairs_out == nullptr)) return PA_BM_CAPACITY;
+        for (Seq* q : g) q->table.reserve(q->host_table.size());
+
+        std::vector<int32_t> dev(needs.size());
+        for (int32_t b : revived)
+            if (bm->blocks[b].ref == 0) bm->remove(b);  // out of the queue before any take()
+        int32_t pairs = 0;
+        for (size_t i = 0; i < needs.size(); ++i) {
+            const Need& n = needs[i];
+            if (n.revive >= 0) {
+                dev[i] = n.revive;
+                continue;
+            }
+            const int32_t b = bm->take();
+            bm->blocks[b].ref = 0;                     // counted per table entry below
+            if (n.full) bm->register_full_block(b, n.hash);
+            dev[i] = b;
+            pairs_out[2 * pairs] = n.host;
+            pairs_out[2 * pairs + 1] = b;
+            ++pairs;
+        }
+        for (Seq* q : g) {
+            for (int32_t h : q->host_table) {
+                const int32_t b = dev[index[h]];
+                ++bm->blocks[b].ref;
+                q->table.push_back(b);
+            }
+            for (auto r = q->host_table.rbegin(); r != q->host_table.rend(); ++r)
+                if (--bm->host_ref[*r] == 0) bm->host_free.push_back(*r);
+            q->host_table.clear();
+            q->swapped = false;
+        }
+        if (num_pairs) *num_pairs = pairs;
+    } catch (...) {
+        return PA_BM_BAD_ARG;
+    }
+    return PA_BM_OK;
+}
+
 extern "C" int32_t pa_bm_check(const pa_block_manager* bm)
 {
     if (!bm) return 1;
     const int32_t nb = bm->num_blocks, B = bm->block_size;
-    std::vector<int32_t> refs(nb, 0);
+    std::vector<int32_t> refs(nb, 0), host_refs(bm->num_host, 0);
     for (const auto& kv : bm->seqs) {
         const Seq& q = kv.second;
-        const int64_t waste = static_cast<int64_t>(q.table.size()) * B - q.len;
+        const std::vector<int32_t>& t = q.swapped ? q.host_table : q.table;
+        if (q.swapped && !q.table.empty()) return 10;             // swapped: host blocks only
+        if (!q.swapped && !q.host_table.empty()) return 10;
+        const int64_t waste = static_cast<int64_t>(t.size()) * B - q.len;
         if (waste < 0 || waste > B - 1) return 2;                 // internal waste bound
-        for (int32_t b : q.table) {
-            if (b < 0 || b >= nb) return 3;
-            ++refs[b];
+        for (int32_t b : t) {
+            if (b < 0 || b >= (q.swapped ? bm->num_host : nb)) return 3;
+            ++(q.swapped ? host_refs : refs)[b];
         }
     }
+    for (int32_t h = 0; h < bm->num_host; ++h)
+        if (host_refs[h] != bm->host_ref[h]) return 11;          // host counts == references
+    std::vector<char> listed(bm->num_host, 0);
+    for (int32_t h : bm->host_free) {
+        if (h < 0 || h >= bm->num_host || listed[h] || bm->host_ref[h] != 0) return 12;
+        listed[h] = 1;
+    }
+    for (int32_t h = 0; h < bm->num_host; ++h)
+        if ((bm->host_ref[h] == 0) != (listed[h] != 0)) return 12;  // host free <=> count 0
     for (int32_t b = 0; b < nb; ++b)
         if (refs[b] != bm->blocks[b].ref) return 4;               // counts == references
     int32_t count = 0, prev = -1;

@@ -208,3 +208,209 @@ def test_random_streams_with_caching_keep_invariants(native, seed):
     for s in live:
         cc.free_sequence(s)
     assert cc.num_free() == 64 and cc.check() == 0
+
+
+# ---- swapping to a host pool ([VM-paging, 显存管理与调度策略设计], eviction) ------
+
+def _tag(extra, tokens):
+    """The bytes a token's K/V stands for: a function of its whole prefix
+    (and the extra key), so prefix-cache hits and revived blocks must already
+    hold them."""
+    h = (extra * 1000003 + 7) & 0xFFFFFFFF
+    for t in tokens:
+        h = (h * 31 + int(t) + 1) & 0xFFFFFFFF
+    return h
+
+
+class _Pools:
+    """Device and host pools of 32-bit tags (two uint16 per slot), moved
+    only by the oracle's copy_blocks and swap_blocks."""
+
+    def __init__(self, nb, nh, b):
+        self.b = b
+        self.dev = np.zeros((nb, b, 1, 2), np.uint16)
+        self.host = np.zeros((nh, b, 1, 2), np.uint16)
+        self.scratch_dev = np.zeros_like(self.dev)
+        self.scratch_host = np.zeros_like(self.host)
+
+    def write(self, slot, tag):
+        self.dev[slot // self.b, slot % self.b, 0] = (tag & 0xFFFF, tag >> 16)
+
+    def read(self, table, n):
+        out = []
+        for p in range(n):
+            lo, hi = self.dev[table[p // self.b], p % self.b, 0]
+            out.append(int(lo) | (int(hi) << 16))
+        return out
+
+    def cow(self, pairs):
+        import oracle
+        if pairs:
+            assert oracle.copy_blocks(self.dev, self.scratch_dev, np.array(pairs)) == 0
+
+    def swap_out(self, pairs):
+        import oracle
+        if pairs:
+            assert oracle.swap_blocks(self.dev, self.scratch_dev, self.host, self.scratch_host,
+                                      np.array(pairs)) == 0
+
+    def swap_in(self, pairs):
+        import oracle
+        if pairs:
+            assert oracle.swap_blocks(self.host, self.scratch_host, self.dev, self.scratch_dev,
+                                      np.array(pairs)) == 0
+
+
+@pytest.mark.parametrize("caching", [False, True])
+@pytest.mark.parametrize("seed", range(4))
+def test_swap_stream_keeps_every_sequence_intact(native, seed, caching):
+    """Random add / append / fork / free / swap-out / swap-in streams over a
+    small pool: after every operation each resident sequence reads back its
+    own tokens through its block table, with copy-on-write copies and swap
+    copies applied by the oracle, and every invariant of pa_bm_check holds."""
+    rng = np.random.Generator(np.random.PCG64(300 + seed))
+    nb, nh, b = 40, 48, 4
+    cc = native(nb, b, prefix_caching=caching)
+    cc.attach_host_pool(nh)
+    pools = _Pools(nb, nh, b)
+    prompts = [rng.integers(0, 50, size=int(rng.integers(4, 14))).tolist() for _ in range(3)]
+    toks, extra, live, swapped, next_id = {}, {}, [], [], 0
+    swaps = revivals = 0
+
+    def expect(s):
+        return [_tag(extra[s], toks[s][:p + 1]) for p in range(len(toks[s]))]
+
+    for _ in range(400):
+        op = int(rng.integers(0, 6))
+        if op == 0 or not (live or swapped):
+            base = list(prompts[int(rng.integers(0, 3))]) if rng.random() < 0.7 else []
+            t = base + rng.integers(0, 50, size=int(rng.integers(0, 9))).tolist()
+            ek = int(rng.integers(0, 2))
+            r = cc.add_sequence(next_id, len(t), t if caching else None, extra_key=ek)
+            if r is not None:
+                slots, cached = r
+                toks[next_id], extra[next_id] = t, ek
+                for p in range(cached, len(t)):
+                    pools.write(slots[p], _tag(ek, t[:p + 1]))
+                live.append(next_id)
+            next_id += 1
+        elif op == 1 and live:
+            s = live[int(rng.integers(0, len(live)))]
+            new = rng.integers(0, 50, size=int(rng.integers(1, 7))).tolist()
+            r = cc.append_slots(s, len(new), new if caching else None)
+            if r is not None:
+                slots, cow = r
+                pools.cow(cow)
+                for i, tk in enumerate(new):
+                    toks[s].append(tk)
+                    pools.write(slots[i], _tag(extra[s], toks[s]))
+        elif op == 2 and live:
+            s = live[int(rng.integers(0, len(live)))]
+            cc.fork(s, next_id)
+            toks[next_id], extra[next_id] = list(toks[s]), extra[s]
+            live.append(next_id)
+            next_id += 1
+        elif op == 3 and (live or swapped):
+            pool = live if (live and (not swapped or rng.random() < 0.5)) else swapped
+            s = pool.pop(int(rng.integers(0, len(pool))))
+            cc.free_sequence(s)
+        elif op == 4 and live:
+            k = min(len(live), int(rng.integers(1, 4)))
+            group = [live[i] for i in rng.permutation(len(live))[:k]]
+            pairs = cc.swap_out(group)
+            if pairs is not None:
+                pools.swap_out(pairs)
+                for s in group:
+                    live.remove(s)
+                    swapped.append(s)
+                    assert cc.is_swapped(s) == 1
+                swaps += 1
+        elif op == 5 and swapped:
+            k = min(len(swapped), int(rng.integers(1, 4)))
+            group = [swapped[i] for i in rng.permutation(len(swapped))[:k]]
+            blocks = sum(-(-len(toks[s]) // b) for s in group)
+            pairs = cc.swap_in(group)
+            if pairs is not None:
+                pools.swap_in(pairs)
+                revivals += len(pairs) < blocks
+                for s in group:
+                    swapped.remove(s)
+                    live.append(s)
+                    assert cc.is_swapped(s) == 0
+        assert cc.check() == 0
+        for s in live:
+            assert cc.context_len(s) == len(toks[s])
+            assert pools.read(cc.block_table(s), len(toks[s])) == expect(s), s
+    assert swaps > 5
+    assert revivals > 0 or not caching      # swap-ins that copied fewer blocks than they hold
+    for s in live + swapped:
+        cc.free_sequence(s)
+    assert cc.num_free() == nb and cc.num_free_host() == nh and cc.check() == 0
+
+
+def test_swap_keeps_a_group_shared(native):
+    """Three beams sharing a prompt leave as one host copy per distinct
+    block and come back sharing again."""
+    cc = native(32, 4)
+    cc.attach_host_pool(32)
+    cc.add_sequence(0, 10)                   # blocks: 2 full + 1 partial
+    cc.fork(0, 1)
+    cc.fork(0, 2)
+    cc.append_slots(1, 1)                    # copy-on-write of the partial block
+    out = cc.swap_out([0, 1, 2])
+    assert len(out) == 4 and len({h for _, h in out}) == 4     # 3 shared + beam 1's copy
+    assert cc.num_free() == 32 and cc.num_free_host() == 28 and cc.check() == 0
+    assert cc.is_swapped(0) == cc.is_swapped(1) == cc.is_swapped(2) == 1
+    back = cc.swap_in([0, 1, 2])
+    assert len(back) == 4 and cc.num_free_host() == 32 and cc.check() == 0
+    t0, t1, t2 = cc.block_table(0), cc.block_table(1), cc.block_table(2)
+    assert t0 == t2 and t0[:2] == t1[:2] and t0[2] != t1[2]
+    assert [cc.ref(b) for b in t0] == [3, 3, 2] and cc.ref(t1[2]) == 1
+
+
+def test_swap_in_revives_cached_blocks(native):
+    """With prefix caching, full blocks freed by a swap-out keep their
+    hashes; swapping back in revives them without a copy while they have not
+    been reused, and copies only the partial block and reused ones."""
+    cc = native(16, 4, prefix_caching=True)
+    cc.attach_host_pool(8)
+    toks = list(range(14))                                     # 3 full blocks + 2 tokens
+    cc.add_sequence(0, 14, toks)
+    table = cc.block_table(0)
+    assert len(cc.swap_out([0])) == 4 and cc.num_cached() == 3
+    back = cc.swap_in([0])
+    assert len(back) == 1 and back[0][1] not in table[:3]
+    assert cc.block_table(0)[:3] == table[:3] and cc.check() == 0
+    # reuse the freed blocks before swapping in: now every block is copied
+    assert len(cc.swap_out([0])) == 4
+    cc.add_sequence(1, 64, list(range(100, 164)))             # takes the whole pool
+    assert cc.swap_in([0]) is None                             # no room: nothing changes
+    assert cc.is_swapped(0) == 1 and cc.check() == 0
+    cc.free_sequence(1)
+    assert len(cc.swap_in([0])) == 4 and cc.check() == 0
+
+
+def test_swap_refusals_change_nothing(native):
+    cc = native(8, 4)
+    with pytest.raises(ValueError):
+        cc.swap_out([0])                                       # no host pool yet
+    cc.attach_host_pool(2)
+    with pytest.raises(ValueError):
+        cc.attach_host_pool(4)                                 # only once
+    cc.add_sequence(0, 12)                                     # 3 blocks
+    cc.add_sequence(1, 4)
+    state = (cc.num_free(), cc.num_free_host(), cc.block_table(0), cc.block_table(1))
+    assert cc.swap_out([0]) is None                            # 3 blocks > 2 host blocks
+    for bad in ([0, 0], [7], []):
+        with pytest.raises(ValueError):
+            cc.swap_out(bad)
+    with pytest.raises(ValueError):
+        cc.swap_in([1])                                        # resident
+    assert (cc.num_free(), cc.num_free_host(), cc.block_table(0), cc.block_table(1)) == state
+    assert len(cc.swap_out([1])) == 1
+    for call in (lambda: cc.append_slots(1, 1), lambda: cc.fork(1, 5), lambda: cc.block_table(1)):
+        with pytest.raises(ValueError):
+            call()
+    assert cc.context_len(1) == 4 and cc.check() == 0
+    cc.free_sequence(1)                                        # releases its host block
+    assert cc.num_free_host() == 2 and cc.is_swapped(1) == -1 and cc.check() == 0
