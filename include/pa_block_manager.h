@@ -118,6 +118,16 @@ PA_API int32_t pa_bm_block_table(const pa_block_manager* bm, int64_t seq_id, int
 PA_API int32_t pa_bm_context_len(const pa_block_manager* bm, int64_t seq_id);
 
 /*
+ * Watermark ([VM-paging, 显存管理与调度策略设计]: a share of the blocks, 5% say,
+ * is held back so that the requests already running can keep growing when
+ * free blocks run low).  After pa_bm_set_watermark(bm, r), pa_bm_add_sequence
+ * and pa_bm_swap_in return PA_BM_NO_SPACE when they would leave fewer than r
+ * free blocks; pa_bm_append_slots may use the reserve.  0 <= r <=
+ * num_blocks (else PA_BM_BAD_ARG); the default is 0.
+ */
+PA_API int32_t pa_bm_set_watermark(pa_block_manager* bm, int32_t reserved_blocks);
+
+/*
  * Swapping.  pa_bm_attach_host_pool gives the manager host blocks
  * [0, num_host_blocks) of a pinned host pool shaped like the device pool
  * (once per manager).  While a sequence is swapped out it has no device

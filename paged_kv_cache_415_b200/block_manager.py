@@ -39,6 +39,8 @@ LIB.pa_bm_context_len.argtypes = [_p, _i64]
 LIB.pa_bm_context_len.restype = _i32
 LIB.pa_bm_check.argtypes = [_p]
 LIB.pa_bm_check.restype = _i32
+LIB.pa_bm_set_watermark.argtypes = [_p, _i32]
+LIB.pa_bm_set_watermark.restype = _i32
 LIB.pa_bm_attach_host_pool.argtypes = [_p, _i32]
 LIB.pa_bm_attach_host_pool.restype = _i32
 LIB.pa_bm_num_free_host_blocks.argtypes = [_p]
@@ -130,6 +132,12 @@ class NativeBlockManager:
 
     def check(self) -> int:
         return int(LIB.pa_bm_check(self.h))
+
+    def set_watermark(self, reserved_blocks: int) -> None:
+        """Free blocks that admissions (add_sequence, swap_in) must leave."""
+        rc = LIB.pa_bm_set_watermark(self.h, reserved_blocks)
+        if rc != PA_BM_OK:
+            raise ValueError(f"pa_bm_set_watermark: {rc}")
 
     # ---- swapping to a host pool ----------------------------------------------
 

@@ -58,6 +58,7 @@ struct Seq {
 struct pa_block_manager {
     int32_t num_blocks = 0, block_size = 0;
     bool caching = false;
+    int32_t watermark = 0;      // free blocks that admissions must leave untouched
     std::vector<Block> blocks;
     int32_t head = -1, tail = -1, nfree = 0;
     std::unordered_map<uint64_t, int32_t> cache;     // hash -> block
@@ -205,7 +206,7 @@ extern "C" int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, cons
     int32_t revived = 0;
     for (int32_t b : hits) revived += bm->blocks[b].ref == 0;
     const int32_t fresh = nblk - static_cast<int32_t>(hits.size());
-    if (fresh + revived > bm->nfree) return PA_BM_NO_SPACE;
+    if (fresh + revived > bm->nfree - bm->watermark) return PA_BM_NO_SPACE;
 
     Seq q;
     q.extra_key = extra_key;
@@ -345,6 +346,16 @@ extern "C" int32_t pa_bm_context_len(const pa_block_manager* bm, int64_t seq_id)
     return it == bm->seqs.end() ? -1 : it->second.len;
 }
 
+// The watermark of [VM-paging, 显存管理与调度策略设计]: a reserve of free blocks
+// that new (and resumed) requests may not take, so that running requests can
+// still grow when memory is tight.
+extern "C" int32_t pa_bm_set_watermark(pa_block_manager* bm, int32_t reserved_blocks)
+{
+    if (!bm || reserved_blocks < 0 || reserved_blocks > bm->num_blocks) return PA_BM_BAD_ARG;
+    bm->watermark = reserved_blocks;
+    return PA_BM_OK;
+}
+
 extern "C" int32_t pa_bm_attach_host_pool(pa_block_manager* bm, int32_t num_host_blocks)
 {
     if (!bm || bm->num_host != 0 || num_host_blocks <= 0) return PA_BM_BAD_ARG;
@@ -463,7 +474,7 @@ extern "C" int32_t pa_bm_swap_in(pa_block_manager* bm, const int64_t* seq_ids, i
                 from_free += bm->blocks[n.revive].ref == 0;
             }
         }
-        if (fresh + from_free > bm->nfree) return PA_BM_NO_SPACE;
+        if (fresh + from_free > bm->nfree - bm->watermark) return PA_BM_NO_SPACE;
         if (fresh > capacity || (fresh > 0 && pairs_out == nullptr)) return PA_BM_CAPACITY;
         for (Seq* q : g) q->table.reserve(q->host_table.size());
 

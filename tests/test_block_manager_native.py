@@ -414,3 +414,25 @@ def test_swap_refusals_change_nothing(native):
     assert cc.context_len(1) == 4 and cc.check() == 0
     cc.free_sequence(1)                                        # releases its host block
     assert cc.num_free_host() == 2 and cc.is_swapped(1) == -1 and cc.check() == 0
+
+
+def test_watermark_holds_back_admissions_not_appends(native):
+    """With 2 of 10 blocks reserved, a new request (or a swapped group
+    coming back) may not take the last 2 free blocks; a running sequence
+    may."""
+    cc = native(10, 4)
+    cc.attach_host_pool(8)
+    for bad in (-1, 11):
+        with pytest.raises(ValueError):
+            cc.set_watermark(bad)
+    cc.set_watermark(2)
+    assert cc.add_sequence(0, 24) is not None                  # 6 blocks, 4 left
+    assert cc.add_sequence(1, 12) is None                      # would leave 1 < 2
+    assert cc.add_sequence(1, 8) is not None                   # leaves exactly 2
+    assert cc.append_slots(0, 8) is not None and cc.num_free() == 0   # the reserve is usable
+    cc.free_sequence(1)
+    assert len(cc.swap_out([0])) == 8 and cc.num_free() == 10
+    cc.add_sequence(2, 4)                                      # 9 free
+    assert cc.swap_in([0]) is None                             # 8 of 9 would leave 1 < 2
+    cc.set_watermark(1)
+    assert cc.swap_in([0]) is not None and cc.num_free() == 1 and cc.check() == 0
