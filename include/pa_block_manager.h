@@ -166,6 +166,29 @@ PA_API int32_t pa_bm_swap_out(pa_block_manager* bm, const int64_t* seq_ids, int3
 PA_API int32_t pa_bm_swap_in(pa_block_manager* bm, const int64_t* seq_ids, int32_t num_seqs,
                              int64_t* pairs_out, int32_t capacity, int32_t* num_pairs);
 
+/*
+ * Monitoring ([Practice §6.3 实际部署建议]: watch the physical block
+ * utilisation, above 90% as the target, and the hit rate).
+ *   used_blocks     blocks with at least one user;
+ *   stored_tokens   tokens held in them, a shared block counted once (its
+ *                   fill is the most tokens any of its users keeps in it);
+ *                   utilisation = stored_tokens / (used_blocks * block_size),
+ *                   internal waste = 1 - utilisation;
+ *   prefix_queries, prefix_hits   full prompt blocks that
+ *                   pa_bm_add_sequence looked up in the prefix cache, and
+ *                   how many it reused (prefix caching only; successful
+ *                   calls only); hit rate = hits / queries.
+ */
+typedef struct pa_bm_stats_t {
+    int32_t num_blocks, block_size;
+    int32_t used_blocks, free_blocks, cached_blocks;
+    int32_t num_seqs, swapped_seqs, free_host_blocks;
+    int64_t stored_tokens;
+    int64_t prefix_queries, prefix_hits;
+} pa_bm_stats_t;
+
+PA_API int32_t pa_bm_stats(const pa_block_manager* bm, pa_bm_stats_t* out);
+
 /* Checks every invariant (counts equal table references, free queue holds
  * exactly the blocks with count 0, no cycles, cached hashes map back to
  * their blocks, internal waste <= block_size - 1, and for the host pool:

@@ -53,6 +53,27 @@ LIB.pa_bm_swap_in.argtypes = [_p, _p, _i32, _p, _i32, _p]
 LIB.pa_bm_swap_in.restype = _i32
 
 
+class BlockManagerStats(ctypes.Structure):
+    """pa_bm_stats_t (include/pa_block_manager.h)."""
+    _fields_ = [(n, ctypes.c_int32) for n in ("num_blocks", "block_size", "used_blocks",
+                                             "free_blocks", "cached_blocks", "num_seqs",
+                                             "swapped_seqs", "free_host_blocks")] + \
+               [(n, ctypes.c_int64) for n in ("stored_tokens", "prefix_queries", "prefix_hits")]
+
+    @property
+    def utilisation(self) -> float:
+        cap = self.used_blocks * self.block_size
+        return self.stored_tokens / cap if cap else 1.0
+
+    @property
+    def hit_rate(self) -> float:
+        return self.prefix_hits / self.prefix_queries if self.prefix_queries else 0.0
+
+
+LIB.pa_bm_stats.argtypes = [_p, _p]
+LIB.pa_bm_stats.restype = _i32
+
+
 def _ptr(a):
     return None if a is None else ctypes.c_void_p(a.ctypes.data)
 
@@ -132,6 +153,13 @@ class NativeBlockManager:
 
     def check(self) -> int:
         return int(LIB.pa_bm_check(self.h))
+
+    def stats(self) -> BlockManagerStats:
+        st = BlockManagerStats()
+        rc = LIB.pa_bm_stats(self.h, ctypes.byref(st))
+        if rc != PA_BM_OK:
+            raise ValueError(f"pa_bm_stats: {rc}")
+        return st
 
     def set_watermark(self, reserved_blocks: int) -> None:
         """Free blocks that admissions (add_sequence, swap_in) must leave."""

@@ -59,6 +59,7 @@ struct pa_block_manager {
     int32_t num_blocks = 0, block_size = 0;
     bool caching = false;
     int32_t watermark = 0;      // free blocks that admissions must leave untouched
+    int64_t prefix_queries = 0, prefix_hits = 0;   // full prompt blocks looked up / found
     std::vector<Block> blocks;
     int32_t head = -1, tail = -1, nfree = 0;
     std::unordered_map<uint64_t, int32_t> cache;     // hash -> block
@@ -234,6 +235,10 @@ extern "C" int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, cons
         return PA_BM_BAD_ARG;
     }
     if (num_cached) *num_cached = static_cast<int32_t>(hits.size()) * B;
+    if (bm->caching) {
+        bm->prefix_queries += nfull;
+        bm->prefix_hits += static_cast<int64_t>(hits.size());
+    }
     return PA_BM_OK;
 }
 
@@ -508,6 +513,45 @@ extern "C" int32_t pa_bm_swap_in(pa_block_manager* bm, const int64_t* seq_ids, i
             q->swapped = false;
         }
         if (num_pairs) *num_pairs = pairs;
+    } catch (...) {
+        return PA_BM_BAD_ARG;
+    }
+    return PA_BM_OK;
+}
+
+// The monitoring figures of [Practice §6.3 实际部署建议] (block utilisation,
+// hit rate).  A block's fill is the most tokens any of its users holds in it.
+extern "C" int32_t pa_bm_stats(const pa_block_manager* bm, pa_bm_stats_t* out)
+{
+    if (!bm || !out) return PA_BM_BAD_ARG;
+    try {
+        const int32_t B = bm->block_size;
+        std::vector<int32_t> fill(bm->num_blocks, 0);
+        int32_t swapped = 0;
+        for (const auto& kv : bm->seqs) {
+            const Seq& q = kv.second;
+            swapped += q.swapped;
+            for (size_t j = 0; j < q.table.size(); ++j) {
+                const int32_t n = std::min<int32_t>(B, q.len - static_cast<int32_t>(j) * B);
+                fill[q.table[j]] = std::max(fill[q.table[j]], n);
+            }
+        }
+        pa_bm_stats_t st = {};
+        st.num_blocks = bm->num_blocks;
+        st.block_size = B;
+        for (int32_t b = 0; b < bm->num_blocks; ++b) {
+            if (bm->blocks[b].ref == 0) continue;
+            ++st.used_blocks;
+            st.stored_tokens += fill[b];
+        }
+        st.free_blocks = bm->nfree;
+        st.cached_blocks = static_cast<int32_t>(bm->cache.size());
+        st.prefix_queries = bm->prefix_queries;
+        st.prefix_hits = bm->prefix_hits;
+        st.num_seqs = static_cast<int32_t>(bm->seqs.size());
+        st.swapped_seqs = swapped;
+        st.free_host_blocks = static_cast<int32_t>(bm->host_free.size());
+        *out = st;
     } catch (...) {
         return PA_BM_BAD_ARG;
     }

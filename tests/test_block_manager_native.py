@@ -436,3 +436,28 @@ def test_watermark_holds_back_admissions_not_appends(native):
     assert cc.swap_in([0]) is None                             # 8 of 9 would leave 1 < 2
     cc.set_watermark(1)
     assert cc.swap_in([0]) is not None and cc.num_free() == 1 and cc.check() == 0
+
+
+def test_stats_utilisation_and_hit_rate(native):
+    """Utilisation counts each stored token once (shared blocks once) over
+    the capacity of the blocks in use; the hit rate counts full prompt
+    blocks found in the prefix cache."""
+    cc = native(32, 4, prefix_caching=True)
+    st = cc.stats()
+    assert (st.used_blocks, st.stored_tokens, st.prefix_queries) == (0, 0, 0)
+    assert st.utilisation == 1.0 and st.hit_rate == 0.0
+    prompt = list(range(10))                         # 2 full blocks + 2 tokens
+    cc.add_sequence(0, 10, prompt)
+    cc.fork(0, 1)                                    # shares all 3 blocks
+    st = cc.stats()
+    assert (st.used_blocks, st.stored_tokens) == (3, 10) and abs(st.utilisation - 10 / 12) < 1e-12
+    cc.append_slots(1, 1, [99])                      # copy-on-write: 3 + 1 blocks, 10 + 3 tokens
+    st = cc.stats()
+    assert (st.used_blocks, st.stored_tokens, st.num_seqs) == (4, 13, 2)
+    cc.add_sequence(2, 13, prompt + [5, 6, 7])       # 3 full blocks: 2 cached, 1 new
+    st = cc.stats()
+    assert (st.prefix_queries, st.prefix_hits) == (2 + 3, 2) and abs(st.hit_rate - 0.4) < 1e-12
+    # the pages' waste bound: every sequence wastes at most block_size - 1 slots
+    assert st.used_blocks * 4 - st.stored_tokens <= 3 * st.num_seqs
+    assert cc.add_sequence(3, 1000, list(range(1000))) is None      # refused: counters unchanged
+    assert cc.stats().prefix_queries == 5
