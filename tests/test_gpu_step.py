@@ -116,3 +116,29 @@ def test_graph_replay_matches_eager(make):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), ref2.view(torch.int16))
     assert int(stepper.d_status.item()) == 0
+
+
+@pytest.mark.parametrize("codes", ["fp8", "int8"])
+@pytest.mark.parametrize("fused", [True, False], ids=["fused-append", "separate"])
+def test_decode_step_on_code_pools(codes, fused):
+    """DecodeStep over one-byte pools picks that format's write and decode
+    (fused into one launch, or separate): the pools equal the oracle's
+    quantising write bit for bit and the output matches the oracle."""
+    from paged_kv_cache_415_b200.step import DecodeStep
+    from tests.test_gpu_quantised import Q8Device, _instance, _oracle_decode, _oracle_pools
+    wl = _instance(codes, 128, 16, 4, "bf16")
+    assert wl.extra["one_token_per_seq"]
+    dev = Q8Device(wl)
+    stepper = DecodeStep(dev.k_cache, dev.v_cache, wl.num_seqs, wl.num_q_heads,
+                         wl.max_context_len, 0, k_scale=dev.ks, v_scale=dev.vs)
+    out = stepper(dev.query, dev.block_tables, dev.context_lens, wl.scale,
+                  new_key=dev.new_key, new_value=dev.new_value, slot_mapping=dev.slot_mapping,
+                  fused_append=fused)
+    torch.cuda.synchronize()
+    kc, vc, st = _oracle_pools(wl)
+    assert st == 0
+    assert np.array_equal(dev.k_cache.cpu().numpy(), kc)
+    assert np.array_equal(dev.v_cache.cpu().numpy(), vc)
+    ref, st = _oracle_decode(wl, kc, vc)
+    assert st == 0 and int(stepper.d_status.item()) == 0
+    assert_close(to_f64(out), ref, f"{codes} step")
