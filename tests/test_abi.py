@@ -146,3 +146,22 @@ def test_empty_calls_are_no_ops(pa):
 ])
 def test_copy_blocks_rejects_bad_arguments(pa, args, code):
     assert pa.LIB.pa_copy_blocks(*args) == code
+
+
+def test_headers_and_library_from_plain_c(pa, tmp_path):
+    """A C99 program that includes include/*.h alone (no CUDA or C++
+    header) compiles without warnings, links against libpa.so and runs its
+    host-only checks (tests/c/abi_from_c.c)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc is not installed")
+    exe = tmp_path / "abi_from_c"
+    lib_dir = os.path.dirname(pa.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                    "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "abi_from_c.c"),
+                    "-o", str(exe), "-L", lib_dir, "-l:libpa.so", f"-Wl,-rpath,{lib_dir}"],
+                   check=True, capture_output=True, text=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0, res.stderr
+    assert "abi from C ok" in res.stdout
