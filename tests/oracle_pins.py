@@ -253,7 +253,9 @@ def pin_blocked_equals_direct(lib):
 
 def pin_large_magnitude(lib):
     """Scores of several thousand (q scaled by 1000) stay finite thanks to the
-    max subtraction, and each output is a convex combination of V rows."""
+    max subtraction, and each output is a convex combination of V rows.  The
+    blocked form agrees there too: only at such scores does a global max
+    that misses a block (or part of one) change the result, by overflow."""
     wl = small_llama(seqs=3)
     q = (wl.query.view(np.float16).astype(np.float32) * 1000).astype(np.float16).view(np.uint16)
     kc, vc = pool_after_step(wl)
@@ -262,6 +264,31 @@ def pin_large_magnitude(lib):
     for s in range(wl.num_seqs):
         v = brute._f64(wl.values[s], wl.dtype)
         assert np.all(out[s] >= v.min(0) - 1e-9) and np.all(out[s] <= v.max(0) + 1e-9)
+    blocked, _ = run_decode(lib, wl, kc, vc, query=q, blocked=True)
+    assert np.all(np.isfinite(blocked))
+    close(blocked, out)
+
+
+def pin_blocked_max_in_last_block(lib):
+    """The blocked form's global max must cover every block and every token
+    of a block: each head's query points along its sequence's newest key
+    (x 100, so its score is in the thousands and every other far below),
+    which sits in the last block and not at a block's first position.  A
+    max that missed it would overflow; blocked and direct agree instead."""
+    wl = gen.make_decode("blocked-max", seed=gen.SEED_BASE + 9, dtype="f16",
+                         context_lens=[37, 70, 100], num_q_heads=4, num_kv_heads=4,
+                         head_dim=128, block_size=16, num_blocks=24, scale=1 / math.sqrt(128),
+                         keep_logical=False)
+    assert wl.extra["one_token_per_seq"] and all((c - 1) % 16 for c in wl.context_lens)
+    kc, vc = pool_after_step(wl)
+    q = (wl.new_key.view(np.float16).astype(np.float32) * 100).astype(np.float16).view(np.uint16)
+    direct, _ = run_decode(lib, wl, kc, vc, query=q)
+    blocked, _ = run_decode(lib, wl, kc, vc, query=q, blocked=True)
+    assert np.all(np.isfinite(direct)) and np.all(np.isfinite(blocked))
+    close(blocked, direct)
+    # the newest token dominates: the output is (about) its value row
+    newest = wl.new_value.view(np.float16).astype(np.float64)
+    assert np.max(np.abs(direct - newest)) < 1e-6
 
 
 def pin_edge_contexts(lib):

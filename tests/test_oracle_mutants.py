@@ -45,6 +45,10 @@ MUTANTS = {
     "swap_bad_id_not_flagged": ("            status |= 1;\n            continue;", "            continue;"),
     "fp8_v_scaled_by_k_scale": ("(dec(v_cache[r + d]) * v_scale)",
                                 "(dec(v_cache[r + d]) * k_scale)"),
+    "blocked_skips_last_block": ("for (int32_t j = 0; j < nb; ++j) {",
+                                 "for (int32_t j = 0; j + 1 < nb; ++j) {"),
+    "blocked_block_max_first_token_only": ("t < ctx && t < (j + 1) * block_size",
+                                           "t < ctx && t < j * block_size + 1"),
     "int8_unsigned_codes": ("return (double)(int8_t)b;", "return (double)b;"),
     "int8_ties_away": ("else r = fmod(lo, 2.0) == 0.0 ? lo : lo + 1.0;", "else r = lo + 1.0;"),
     "int8_wraps_past_127": ("if (x >= 127.0f) return 127;", "if (x >= 128.0f) return 127;"),
