@@ -45,6 +45,10 @@ MUTANTS = {
     "swap_bad_id_not_flagged": ("            status |= 1;\n            continue;", "            continue;"),
     "fp8_v_scaled_by_k_scale": ("(dec(v_cache[r + d]) * v_scale)",
                                 "(dec(v_cache[r + d]) * k_scale)"),
+    "copy_repeated_dst_not_flagged": ("if (block_mapping[2 * j + 1] == dst && j < i) status |= 8;", ""),
+    "copy_dst_read_by_other_not_flagged": (
+        "if (block_mapping[2 * j] == dst && block_mapping[2 * j] != block_mapping[2 * j + 1])\n"
+        "                status |= 8;", ""),
     "blocked_skips_last_block": ("for (int32_t j = 0; j < nb; ++j) {",
                                  "for (int32_t j = 0; j + 1 < nb; ++j) {"),
     "blocked_block_max_first_token_only": ("t < ctx && t < (j + 1) * block_size",
