@@ -45,6 +45,9 @@ MUTANTS = {
     "swap_bad_id_not_flagged": ("            status |= 1;\n            continue;", "            continue;"),
     "fp8_v_scaled_by_k_scale": ("(dec(v_cache[r + d]) * v_scale)",
                                 "(dec(v_cache[r + d]) * k_scale)"),
+    "e4m3_subnormal_scale": ("v = ldexp((double)frac, -9);", "v = ldexp((double)frac, -10);"),
+    "e4m3_nan_whole_top_binade": ("if (expo == 15 && frac == 7)", "if (expo == 15)"),
+    "f16_subnormal_scale": ("v = ldexp((double)frac, -24);", "v = ldexp((double)frac, -25);"),
     "copy_repeated_dst_not_flagged": ("if (block_mapping[2 * j + 1] == dst && j < i) status |= 8;", ""),
     "copy_dst_read_by_other_not_flagged": (
         "if (block_mapping[2 * j] == dst && block_mapping[2 * j] != block_mapping[2 * j + 1])\n"
