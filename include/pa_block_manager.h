@@ -127,6 +127,16 @@ PA_API int32_t pa_bm_context_len(const pa_block_manager* bm, int64_t seq_id);
  */
 PA_API int32_t pa_bm_set_watermark(pa_block_manager* bm, int32_t reserved_blocks);
 
+/* pa_bm_add_sequence for a request that may draw on the watermark reserve
+ * when high_priority != 0: the two-level allocation of [Practice §7
+ * 演进方向与优化空间], where the reserve is a fast pool kept for high-priority
+ * requests once utilisation is high.  With high_priority == 0 it is
+ * pa_bm_add_sequence. */
+PA_API int32_t pa_bm_add_sequence_priority(pa_block_manager* bm, int64_t seq_id,
+                                           const int32_t* tokens, int32_t num_tokens,
+                                           int64_t extra_key, int32_t high_priority,
+                                           int64_t* slots_out, int32_t* num_cached);
+
 /*
  * Swapping.  pa_bm_attach_host_pool gives the manager host blocks
  * [0, num_host_blocks) of a pinned host pool shaped like the device pool

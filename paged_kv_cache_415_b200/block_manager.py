@@ -27,6 +27,8 @@ LIB.pa_bm_num_cached_blocks.argtypes = [_p]
 LIB.pa_bm_num_cached_blocks.restype = _i32
 LIB.pa_bm_add_sequence.argtypes = [_p, _i64, _p, _i32, _i64, _p, _p]
 LIB.pa_bm_add_sequence.restype = _i32
+LIB.pa_bm_add_sequence_priority.argtypes = [_p, _i64, _p, _i32, _i64, _i32, _p, _p]
+LIB.pa_bm_add_sequence_priority.restype = _i32
 LIB.pa_bm_fork.argtypes = [_p, _i64, _i64]
 LIB.pa_bm_fork.restype = _i32
 LIB.pa_bm_append_slots.argtypes = [_p, _i64, _p, _i32, _p, _p, _i32, _p]
@@ -102,13 +104,16 @@ class NativeBlockManager:
     def num_cached(self) -> int:
         return int(LIB.pa_bm_num_cached_blocks(self.h))
 
-    def add_sequence(self, seq: int, num_tokens: int, tokens=None, extra_key: int = 0):
-        """Returns (slots, cached_tokens), or None when the pool is too small."""
+    def add_sequence(self, seq: int, num_tokens: int, tokens=None, extra_key: int = 0,
+                     high_priority: bool = False):
+        """Returns (slots, cached_tokens), or None when the pool is too small.
+        high_priority: the request may use the watermark reserve."""
         toks = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int32)
         slots = np.empty(num_tokens, dtype=np.int64)
         cached = ctypes.c_int32(0)
-        rc = LIB.pa_bm_add_sequence(self.h, seq, _ptr(toks), num_tokens, extra_key, _ptr(slots),
-                                    ctypes.byref(cached))
+        rc = LIB.pa_bm_add_sequence_priority(self.h, seq, _ptr(toks), num_tokens, extra_key,
+                                             1 if high_priority else 0, _ptr(slots),
+                                             ctypes.byref(cached))
         if rc == PA_BM_NO_SPACE:
             return None
         if rc != PA_BM_OK:

@@ -177,9 +177,9 @@ extern "C" int32_t pa_bm_num_cached_blocks(const pa_block_manager* bm)
     return bm ? static_cast<int32_t>(bm->cache.size()) : 0;
 }
 
-extern "C" int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, const int32_t* tokens,
-                                      int32_t num_tokens, int64_t extra_key, int64_t* slots_out,
-                                      int32_t* num_cached)
+static int32_t add_sequence(pa_block_manager* bm, int64_t seq_id, const int32_t* tokens,
+                            int32_t num_tokens, int64_t extra_key, bool may_use_reserve,
+                            int64_t* slots_out, int32_t* num_cached)
 {
     if (!bm || num_tokens < 0 || bm->seqs.count(seq_id)) return PA_BM_BAD_ARG;
     if (bm->caching && num_tokens > 0 && tokens == nullptr) return PA_BM_BAD_ARG;
@@ -207,7 +207,8 @@ extern "C" int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, cons
     int32_t revived = 0;
     for (int32_t b : hits) revived += bm->blocks[b].ref == 0;
     const int32_t fresh = nblk - static_cast<int32_t>(hits.size());
-    if (fresh + revived > bm->nfree - bm->watermark) return PA_BM_NO_SPACE;
+    const int32_t reserve = may_use_reserve ? 0 : bm->watermark;
+    if (fresh + revived > bm->nfree - reserve) return PA_BM_NO_SPACE;
 
     Seq q;
     q.extra_key = extra_key;
@@ -240,6 +241,24 @@ extern "C" int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, cons
         bm->prefix_hits += static_cast<int64_t>(hits.size());
     }
     return PA_BM_OK;
+}
+
+extern "C" int32_t pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, const int32_t* tokens,
+                                      int32_t num_tokens, int64_t extra_key, int64_t* slots_out,
+                                      int32_t* num_cached)
+{
+    return add_sequence(bm, seq_id, tokens, num_tokens, extra_key, false, slots_out, num_cached);
+}
+
+// The two-level allocation of [Practice §7 演进方向与优化空间]: the watermark
+// reserve is the fast pool that only high-priority requests may draw on.
+extern "C" int32_t pa_bm_add_sequence_priority(pa_block_manager* bm, int64_t seq_id,
+                                               const int32_t* tokens, int32_t num_tokens,
+                                               int64_t extra_key, int32_t high_priority,
+                                               int64_t* slots_out, int32_t* num_cached)
+{
+    return add_sequence(bm, seq_id, tokens, num_tokens, extra_key, high_priority != 0, slots_out,
+                        num_cached);
 }
 
 extern "C" int32_t pa_bm_fork(pa_block_manager* bm, int64_t parent, int64_t child)

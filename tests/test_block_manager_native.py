@@ -488,3 +488,17 @@ def test_paged_waste_matches_the_pages_figure(native):
     assert abs(contiguous_waste * 100 - g["contiguous_waste_pct"]) < 1.0
     assert (1 - st.utilisation) * 100 < g["paged_waste_pct_below"]
     assert st.utilisation * 100 > g["utilisation_target_pct"]
+
+
+def test_high_priority_requests_use_the_reserve(native):
+    """Two-level allocation: with 2 of 8 blocks held back, an ordinary request
+    is refused where a high-priority one is admitted from the reserve; the
+    priority call without priority behaves as pa_bm_add_sequence."""
+    cc = native(8, 4)
+    cc.set_watermark(2)
+    assert cc.add_sequence(0, 24) is not None                  # 6 blocks, 2 left
+    assert cc.add_sequence(1, 4) is None                       # ordinary: reserve untouchable
+    assert cc.add_sequence(1, 4, high_priority=False) is None
+    assert cc.add_sequence(1, 8, high_priority=True) is not None and cc.num_free() == 0
+    assert cc.add_sequence(2, 1, high_priority=True) is None   # nothing left at all
+    assert cc.check() == 0
