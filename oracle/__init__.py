@@ -131,8 +131,17 @@ def reshape_and_cache(key, value, k_cache, v_cache, slot_mapping, block_size, li
 
 
 def copy_blocks(k_cache, v_cache, block_mapping, lib=None) -> int:
-    """In place: for each (src, dst) row of block_mapping, copy block src to dst."""
+    """In place: for each (src, dst) row of block_mapping, copy block src to dst.
+
+    Pools of 16-bit elements, or of one-byte codes (uint8 / int8, head_dim
+    even), which move as the same bytes seen in pairs."""
     block_mapping = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
+    assert k_cache.dtype == v_cache.dtype and k_cache.shape == v_cache.shape
+    assert k_cache.flags["C_CONTIGUOUS"] and v_cache.flags["C_CONTIGUOUS"]
+    if k_cache.dtype.itemsize == 1:
+        assert k_cache.shape[-1] % 2 == 0, "one-byte pools copy as byte pairs"
+        k_cache, v_cache = k_cache.view(np.uint16), v_cache.view(np.uint16)
+    assert k_cache.dtype.itemsize == 2, f"16-bit or one-byte pools, got {k_cache.dtype}"
     num_blocks, bs, hkv, d = k_cache.shape
     return int((lib or load()).oracle_copy_blocks(
         _ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), block_mapping.shape[0],

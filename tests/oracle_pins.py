@@ -143,6 +143,20 @@ def pin_copy_blocks(lib):
     assert oracle.copy_blocks(kc.copy(), vc.copy(), np.array([[1, 4], [4, 2]]), lib=lib) & 8
 
 
+def pin_copy_blocks_of_code_pools(lib):
+    """One-byte pools (e4m3 or int8 codes) copy whole blocks byte for byte,
+    and nothing past the pool: the last block is a destination."""
+    rng = np.random.Generator(np.random.PCG64(6))
+    for dt in (np.uint8, np.int8):
+        kc = rng.integers(0, 256, size=(5, 4, 2, 8), dtype=np.uint8).view(dt)
+        vc = rng.integers(0, 256, size=(5, 4, 2, 8), dtype=np.uint8).view(dt)
+        ek, ev = kc.copy(), vc.copy()
+        ek[4], ev[4] = kc[0], vc[0]
+        ek[1], ev[1] = kc[3], vc[3]
+        st = oracle.copy_blocks(kc, vc, np.array([[0, 4], [3, 1]]), lib=lib)
+        assert st == 0 and np.array_equal(kc, ek) and np.array_equal(vc, ev)
+
+
 def pin_brute_force_tiny(lib):
     """The tiny workload against element-by-element Python loops."""
     wl = gen.tiny()

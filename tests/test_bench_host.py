@@ -35,11 +35,12 @@ def test_oracle_step_counts_the_step_bytes():
     """The CPU leg times the oracle on the same step the GPU runs and
     counts the same algorithmic bytes (all sequences, 16-bit and both code
     formats)."""
-    for kv in ("auto", "fp8", "int8"):
-        wl = bench.make_workload("llama7b", seqs=2, kv_dtype=kv)
-        st = bench.OracleStep(wl)
-        assert st.bytes == bm.step_bytes(wl)["total"]
-        assert st.run() > 0.0
+    for config, seqs in (("llama7b", 2), ("tiny", 0)):          # tiny: block copies too
+        for kv in ("auto", "fp8", "int8"):
+            wl = bench.make_workload(config, seqs=seqs, kv_dtype=kv)
+            st = bench.OracleStep(wl)
+            assert st.bytes == bm.step_bytes(wl)["total"]
+            assert st.run() > 0.0
 
 
 def test_committed_traffic_lines_parse():
