@@ -165,3 +165,18 @@ def test_headers_and_library_from_plain_c(pa, tmp_path):
     res = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0, res.stderr
     assert "abi from C ok" in res.stdout
+
+
+def test_decode_refuses_grids_past_the_launch_limits(pa):
+    """More than 65535 sequences, or more than 65535 context partitions,
+    would exceed the grid's y/z limits: refused as PA_ERR_UNSUPPORTED before
+    any launch (the workspace, when one is needed, is large enough)."""
+    assert _decode(pa, num_seqs=70000, max_context_len=100) == 2
+    assert _decode(pa, num_seqs=65535, max_context_len=100, out=None) == 1   # checks still run
+    mcl, part = 16 * 70000, 16
+    need = pa.pa_paged_decode_workspace_size(1, 8, 2, 128, 16, mcl, part)
+    assert need == 8 * 70000 * (128 + 2) * 4
+    assert _decode(pa, num_seqs=1, max_context_len=mcl, partition_size=part, workspace=FAKE,
+                   workspace_bytes=need) == 2
+    assert _decode(pa, num_seqs=1, max_context_len=mcl, partition_size=part, workspace=FAKE,
+                   workspace_bytes=need - 16) == 1                                # too small first
