@@ -8,6 +8,14 @@
  *   pa_paged_decode       single-query attention over each sequence's
  *                         context, reached through its block table
  *
+ * Declared below as well: pa_paged_decode_append (the cache write fused into
+ * the decode launch), pa_paged_decode_no_alloc (library-owned scratch),
+ * pa_paged_decode_shared_prefix (groups that share a stored prefix read it
+ * once), the _fp8 and _int8 variants over one-byte K/V pools, pa_swap_blocks
+ * (block copies between device and pinned host pools), and the size
+ * queries.  The host block manager that hands out the block ids is declared
+ * in pa_block_manager.h.
+ *
  * Pages cited (title, then section):
  *   [VM-paging] "vLLM用虚拟内存分页思想管理KV Cache"
  *   [Practice]  "PagedAttention：大模型KV Cache分页管理优化实践"
@@ -22,7 +30,8 @@
  *   return as soon as the work is enqueued.
  *
  * Element types.  query, key, value, k_cache, v_cache and out share one
- *   element type: IEEE binary16 (PA_DTYPE_F16) or bfloat16 (PA_DTYPE_BF16).
+ *   element type: IEEE binary16 (PA_DTYPE_F16) or bfloat16 (PA_DTYPE_BF16);
+ *   the _fp8 / _int8 calls take one-byte K/V pools instead (see there).
  *   Attention accumulates in fp32 and rounds the output to nearest even.
  *
  * KV-cache layout (one layer; K and V in two pools of the same shape):
