@@ -180,3 +180,21 @@ def test_decode_refuses_grids_past_the_launch_limits(pa):
                    workspace_bytes=need) == 2
     assert _decode(pa, num_seqs=1, max_context_len=mcl, partition_size=part, workspace=FAKE,
                    workspace_bytes=need - 16) == 1                                # too small first
+
+
+def test_no_fallback_without_the_library(tmp_path):
+    """The package has no CPU path: a copy of it without libpa.so fails at
+    import of the binding, naming the missing library, and an op reached
+    through the package's lazy exports fails the same way."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "paged_kv_cache_415_b200")
+    dst = tmp_path / "paged_kv_cache_415_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "*.o", "__pycache__", "_build"))
+    for code in ("import paged_kv_cache_415_b200.binding",
+                 "import paged_kv_cache_415_b200 as p; p.pa_paged_decode"):
+        res = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True,
+                             text=True, timeout=300)
+        assert res.returncode != 0
+        assert "libpa.so" in res.stderr and "ImportError" in res.stderr, res.stderr[-500:]
