@@ -1,0 +1,54 @@
+"""The oracle and the product path share no code: no module of the product
+package imports the oracle (or the test-side workload generators), and no
+module of the oracle imports the product package.  Checked on the import
+statements of every Python source, and on the C sources' #include lines."""
+import ast
+import os
+import re
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _imports(path):
+    tree = ast.parse(open(path).read(), filename=path)
+    names = set()
+    for node in ast.walk(tree):
+        if isinstance(node, ast.Import):
+            names.update(a.name.split(".")[0] for a in node.names)
+        elif isinstance(node, ast.ImportFrom) and node.module and node.level == 0:
+            names.add(node.module.split(".")[0])
+    return names
+
+
+def _py_files(folder):
+    for dirpath, _, files in os.walk(os.path.join(ROOT, folder)):
+        for f in files:
+            if f.endswith(".py"):
+                yield os.path.join(dirpath, f)
+
+
+def test_product_never_imports_the_oracle():
+    files = list(_py_files("paged_kv_cache_415_b200"))
+    assert files
+    for path in files:
+        bad = _imports(path) & {"oracle", "workloads", "tests"}
+        assert not bad, f"{path} imports {bad}"
+
+
+def test_oracle_never_imports_the_product():
+    files = list(_py_files("oracle"))
+    assert files
+    for path in files:
+        assert "paged_kv_cache_415_b200" not in _imports(path), path
+
+
+def test_c_sources_share_no_headers():
+    """The oracle's C source includes only the C standard library (and
+    OpenMP); the CUDA sources include nothing from oracle/."""
+    oracle_c = open(os.path.join(ROOT, "oracle", "pa_oracle.c")).read()
+    for inc in re.findall(r'#include\s*[<"]([^>"]+)[>"]', oracle_c):
+        assert inc in {"math.h", "stdint.h", "stdlib.h", "string.h", "omp.h"}, inc
+    csrc = os.path.join(ROOT, "paged_kv_cache_415_b200", "csrc")
+    for f in os.listdir(csrc):
+        text = open(os.path.join(csrc, f)).read()
+        assert "oracle" not in " ".join(re.findall(r'#include\s*[<"]([^>"]+)[>"]', text)), f
