@@ -52,3 +52,29 @@ def test_c_sources_share_no_headers():
     for f in os.listdir(csrc):
         text = open(os.path.join(csrc, f)).read()
         assert "oracle" not in " ".join(re.findall(r'#include\s*[<"]([^>"]+)[>"]', text)), f
+
+
+def _tracked_code():
+    import subprocess
+    out = subprocess.run(["git", "ls-files", "*.py", "*.cu", "*.cuh", "*.h", "*.c", "*.cpp"],
+                         cwd=ROOT, capture_output=True, text=True)
+    files = out.stdout.split() if out.returncode == 0 else []
+    if not files:                                    # not a git checkout: walk the sources
+        for folder in ("paged_kv_cache_415_b200", "oracle", "workloads", "tests", "include"):
+            for dirpath, _, names in os.walk(os.path.join(ROOT, folder)):
+                files += [os.path.relpath(os.path.join(dirpath, n), ROOT) for n in names
+                          if n.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp"))]
+        files += ["bench.py", "__graft_entry__.py"]
+    return files
+
+
+def test_code_reads_no_reference_pages_and_no_working_files():
+    """No committed source reaches the reference pages' location or the
+    untracked working folder at run time."""
+    me = os.path.relpath(os.path.abspath(__file__), ROOT)
+    for rel in _tracked_code():
+        if rel == me:
+            continue
+        text = open(os.path.join(ROOT, rel), encoding="utf-8").read()
+        assert "/root/reference" not in text, rel
+        assert not re.search(r"[\"'/]_work[/\"']", text), rel
