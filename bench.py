@@ -4,14 +4,22 @@
 
 A step is the whole hot path over one batch of synthetic input:
 copy_blocks (when the workload has copy-on-write pairs), reshape_and_cache
-of the step's new tokens, paged_decode (plus its split-context reduction).
-The default workload is the LLaMA-7B-shaped decode: 64 sequences, 32/32
-heads, head_dim 128, block_size 16, fp16, contexts uniform in [128, 2048],
-16384-block pool, one new token per sequence.
+of the step's new tokens (fused into the decode launch when every sequence
+appends one token), paged_decode (plus its split-context reduction).
+The default workload is the long-context decode: 16 sequences of 32768
+tokens, 32 query / 8 kv heads, head_dim 128, block_size 16, bf16, a fully
+shuffled 40000-block pool, 512-token partitions merged by the reduction
+kernel, one new token per sequence -- the largest single-GPU workload
+(2.15 GB of K/V per step).  In a one-rank run the other workloads
+(LLaMA-7B MHA, Mistral-7B GQA, the beam search with shared prompts, and the
+one-byte-code pools) are measured after it the same way and reported under
+"per_config".
 
 Metric: algorithmic HBM bytes of the step / device time (GB/s), with the
-time per step.  The K/V a step reads (about 1.1 GB) is far larger than the
-126 MB L2, so no flush is needed between steps.
+time per step.  The K/V a step reads (1.1 to 2.2 GB) is far larger than the
+126 MB L2, so no flush is needed between steps.  For workloads whose
+sequences share stored blocks the roofline fraction counts those blocks
+once (unique bytes).
 
 --impl reference times the fp64 CPU oracle on the host cores instead (the
 only other code path here that runs it), on a bounded sample of the same
@@ -43,11 +51,16 @@ UNIT = "GB/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_GLOB_DIR = os.path.join(ROOT, "profiles")
-KERNEL_SOURCES = ["paged_kv_cache_415_b200/csrc/paged_decode.cu",
-                  "paged_kv_cache_415_b200/csrc/paged_decode_mma.cuh",
-                  "paged_kv_cache_415_b200/csrc/paged_decode_q8.cuh",
-                  "paged_kv_cache_415_b200/csrc/pa_codes.cuh",
-                  "paged_kv_cache_415_b200/csrc/pa_common.cuh"]
+# The device sources of each decode kernel family: a traffic line taken on a
+# family's hash stays valid while those files' code is unchanged.
+_CSRC = "paged_kv_cache_415_b200/csrc/"
+KERNEL_FAMILIES = {
+    "fp32": ["pa_common.cuh", "decode_common.cuh", "paged_decode_fp32.cuh"],
+    "mma": ["pa_common.cuh", "decode_common.cuh", "paged_decode_mma.cuh"],
+    "q8": ["pa_common.cuh", "decode_common.cuh", "pa_codes.cuh", "paged_decode_q8.cuh"],
+    "shared": ["pa_common.cuh", "decode_common.cuh", "paged_decode_mma.cuh",
+               "paged_decode_shared.cuh"],
+}
 NVML_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
@@ -59,10 +72,12 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="llama7b",
+    ap.add_argument("--config", default="long_context",
                     choices=["tiny", "llama7b", "mistral7b", "beam_search", "long_context"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other workloads measured after the headline in a one-rank run")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--partition", type=int, default=-1,
                     help="context partition in tokens (-1 = the workload's, 0 = library's choice)")
@@ -121,20 +136,21 @@ def strip_comments(src: str) -> str:
     return "\n".join(line.rstrip() for line in lines if line.strip())
 
 
-def kernel_source_hash() -> str:
-    """sha256[:16] of the decode kernels' sources, comments and blank lines
-    removed: a profile taken on a hash still describes the current code."""
+def kernel_source_hash(family: str) -> str:
+    """sha256[:16] of a decode kernel family's device sources, comments and
+    blank lines removed: a profile taken on a hash still describes the
+    current code of that family."""
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+    for name in KERNEL_FAMILIES[family]:
+        with open(os.path.join(ROOT, _CSRC + name), encoding="utf-8") as f:
             h.update(strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(config: str):
-    """DRAM bytes per launch of the decode kernel from a committed ncu
-    summary, if it was taken on the current kernel source."""
-    want = kernel_source_hash()
+def profiled_traffic(workload: str, family: str):
+    """DRAM bytes per launch of the decode kernels from a committed ncu
+    summary, if it was taken on the current sources of their family."""
+    want = kernel_source_hash(family)
     if not os.path.isdir(PROFILE_GLOB_DIR):
         return None
     for name in sorted(os.listdir(PROFILE_GLOB_DIR)):
@@ -144,7 +160,7 @@ def profiled_traffic(config: str):
             for line in f:
                 m = re.search(r"bench-traffic:\s*workload=(\S+)\s+bytes_per_launch=(\d+)\s+"
                               r"source_sha256=(\w+)", line)
-                if m and m.group(1) == config and m.group(3) == want:
+                if m and m.group(1) == workload and m.group(3) == want:
                     return int(m.group(2))
     return None
 
@@ -358,6 +374,255 @@ def run_reference(args):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+# Workloads measured in the same run as the headline, each on its own
+# (name, K/V code format, shared-prefix decode), when the run has one rank.
+PER_CONFIG = [("llama7b", "auto", False), ("mistral7b", "auto", False),
+              ("beam_search", "auto", True), ("mistral7b", "fp8", False),
+              ("mistral7b", "int8", False), ("long_context", "fp8", False),
+              ("long_context", "int8", False)]
+
+
+class GpuStep:
+    """One workload resident on the device and its step: the copy-on-write
+    copies, the cache write (fused into the decode launch when every
+    sequence appends one token), the decode and its split-context
+    reduction, all through the C-ABI binding; captured into two CUDA graphs
+    (cache operations, decode) unless eager."""
+
+    def __init__(self, wl, dev, partition=-1, separate=False, shared_prefix=False):
+        import torch
+        from paged_kv_cache_415_b200 import binding as B
+        self.B, self.torch, self.wl, self.dev = B, torch, wl, dev
+        self.tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
+        self.codes = wl.extra.get("kv_dtype")                  # None, "fp8" or "int8"
+        self.quant = self.codes is not None
+        self.k_scale = wl.extra.get("k_scale", 1.0)
+        self.v_scale = wl.extra.get("v_scale", 1.0)
+        if self.quant:
+            self.k_cache = torch.from_numpy(wl.k_cache).to(dev)
+            self.v_cache = torch.from_numpy(wl.v_cache).to(dev)
+        else:
+            self.k_cache, self.v_cache = self.up(wl.k_cache), self.up(wl.v_cache)
+        self.query = self.up(wl.query)
+        self.new_key, self.new_value = self.up(wl.new_key), self.up(wl.new_value)
+        self.slot_mapping = torch.from_numpy(wl.slot_mapping).to(dev)
+        self.block_tables = torch.from_numpy(wl.block_tables).to(dev)
+        self.context_lens = torch.from_numpy(wl.context_lens).to(dev)
+        self.block_mapping = torch.from_numpy(np.ascontiguousarray(wl.block_mapping)).to(dev)
+        self.out = torch.empty_like(self.query)
+        self.d_status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.mcl = wl.max_context_len
+        want = wl.partition_size if partition < 0 else partition
+        self.part = B.pa_paged_decode_partition_size(wl.num_seqs, wl.num_q_heads,
+                                                     wl.num_kv_heads, wl.head_dim,
+                                                     wl.block_size, self.mcl, want)
+        ws_bytes = B.pa_paged_decode_workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
+                                                    wl.head_dim, wl.block_size, self.mcl,
+                                                    self.part)
+        self.max_parts = -(-self.mcl // self.part) if self.mcl > 0 else 1
+        self.n_pairs = int(wl.block_mapping.shape[0])
+        self.fused = (not separate and not shared_prefix
+                      and wl.extra.get("one_token_per_seq", False)
+                      and wl.num_new_tokens == wl.num_seqs)
+        self.shared = shared_prefix and "prefix_lens" in wl.extra and not self.quant
+        self.shared_reduce = False
+        if self.shared:
+            self.group_size = int(wl.extra["group_size"])
+            self.prefix_lens = torch.from_numpy(wl.extra["prefix_lens"]).to(dev)
+            self.mpl = int(wl.extra["prefix_lens"].max())
+            ws_bytes = B.pa_paged_decode_shared_prefix_workspace_size(
+                wl.num_seqs, self.group_size, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                wl.block_size, self.mcl, self.mpl, 0)
+            self.shared_reduce = ws_bytes > 0
+        self.workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        self.stream = torch.cuda.current_stream(dev)
+        self.has_cache = bool(self.n_pairs or (wl.num_new_tokens and not self.fused))
+        self.run_cache, self.run_decode = self.cache_ops, self.decode
+
+    def up(self, bits):
+        return self.torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(self.dev).view(
+            self.tdt)
+
+    def cache_ops(self):
+        B, wl = self.B, self.wl
+        if self.n_pairs:
+            B.pa_copy_blocks(self.k_cache, self.v_cache, self.block_mapping, self.d_status,
+                             self.stream)
+        if wl.num_new_tokens and not self.fused:
+            if self.quant:
+                getattr(B, f"pa_reshape_and_cache_{self.codes}")(
+                    self.new_key, self.new_value, self.k_cache, self.v_cache, self.slot_mapping,
+                    self.k_scale, self.v_scale, self.d_status, self.stream)
+            else:
+                B.pa_reshape_and_cache(self.new_key, self.new_value, self.k_cache, self.v_cache,
+                                       self.slot_mapping, self.d_status, self.stream)
+
+    def decode(self):
+        B, wl = self.B, self.wl
+        if self.quant and self.fused:
+            getattr(B, f"pa_paged_decode_{self.codes}_append")(
+                self.out, self.query, self.new_key, self.new_value, self.k_cache, self.v_cache,
+                self.block_tables, self.context_lens, self.mcl, wl.scale, self.k_scale,
+                self.v_scale, self.part, self.workspace, self.d_status, self.stream)
+        elif self.quant:
+            getattr(B, f"pa_paged_decode_{self.codes}")(
+                self.out, self.query, self.k_cache, self.v_cache, self.block_tables,
+                self.context_lens, self.mcl, wl.scale, self.k_scale, self.v_scale, self.part,
+                self.workspace, self.d_status, self.stream)
+        elif self.fused:
+            B.pa_paged_decode_append(self.out, self.query, self.new_key, self.new_value,
+                                     self.k_cache, self.v_cache, self.block_tables,
+                                     self.context_lens, self.mcl, wl.scale, self.part,
+                                     self.workspace, self.d_status, self.stream)
+        elif self.shared:
+            B.pa_paged_decode_shared_prefix(self.out, self.query, self.k_cache, self.v_cache,
+                                            self.block_tables, self.context_lens,
+                                            self.prefix_lens, self.group_size, self.mcl,
+                                            self.mpl, wl.scale, self.workspace, 0, self.d_status,
+                                            self.stream)
+        else:
+            B.pa_paged_decode(self.out, self.query, self.k_cache, self.v_cache,
+                              self.block_tables, self.context_lens, self.mcl, wl.scale,
+                              self.part, self.workspace, self.d_status, self.stream)
+
+    @property
+    def launches_per_step(self) -> int:
+        wl = self.wl
+        reduce = self.shared_reduce if self.shared else self.max_parts > 1
+        return ((1 if self.n_pairs else 0) + (1 if (wl.num_new_tokens and not self.fused) else 0)
+                + 1 + (1 if reduce else 0))
+
+    def prepare(self, warmup: int, eager: bool, barrier):
+        """Warm-up steps, then (unless eager) the step captured once into two
+        graphs whose replay issues the launches with no host work; checks
+        the status word and that the output is finite."""
+        torch = self.torch
+        for _ in range(warmup):
+            self.cache_ops()
+            self.decode()
+        barrier()
+        if not eager:
+            g_cache, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            saved = self.stream
+            with torch.cuda.graph(g_dec):
+                self.stream = torch.cuda.current_stream(self.dev)
+                self.decode()
+            if self.has_cache:
+                with torch.cuda.graph(g_cache):
+                    self.stream = torch.cuda.current_stream(self.dev)
+                    self.cache_ops()
+            self.stream = saved
+            self.graphs = (g_cache, g_dec)
+            self.run_cache = g_cache.replay if self.has_cache else (lambda: None)
+            self.run_decode = g_dec.replay
+            self.run_cache()
+            self.run_decode()
+            barrier()
+        st = int(self.d_status.item())
+        if st != 0 or not bool(torch.isfinite(self.out.float()).all()):
+            raise SystemExit(f"{self.wl.name}: bad step (status {st})")
+
+    def timed(self, steps: int):
+        """K steps between two events on the launching stream; events also
+        bracket the decode launches of every step.  Returns (elapsed ms,
+        per-step decode ms)."""
+        torch = self.torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(self.stream)
+        for i in range(steps):
+            self.run_cache()
+            ev[i][0].record(self.stream)
+            self.run_decode()
+            ev[i][1].record(self.stream)
+        stop.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return start.elapsed_time(stop), [a.elapsed_time(b) for a, b in ev]
+
+    def kernel_name(self) -> str:
+        wl = self.wl
+        group = wl.num_q_heads // wl.num_kv_heads
+        if self.shared:
+            return "paged_decode_shared_kernel" + (
+                " + paged_decode_shared_reduce_kernel" if self.shared_reduce else "")
+        name = (f"paged_decode_{self.codes}_kernel" if self.quant else
+                "paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
+                else "paged_decode_kernel")
+        return name + (" + paged_decode_reduce_kernel" if self.max_parts > 1 else "")
+
+    def entry(self) -> str:
+        c = self.codes
+        return (f"pa_paged_decode_{c}_append (quantising cache write fused)" if self.quant and self.fused
+                else f"pa_reshape_and_cache_{c} + pa_paged_decode_{c}" if self.quant
+                else "pa_paged_decode_shared_prefix" if self.shared
+                else "pa_paged_decode_append (cache write fused)" if self.fused
+                else "pa_reshape_and_cache + pa_paged_decode")
+
+    def roofline_bytes(self):
+        """(algorithmic bytes of one decode launch, referenced bytes or None).
+        A sharing workload (beams over one stored prompt) counts its K/V on
+        unique bytes -- the blocks the step must read at least once -- and
+        reports the bytes its block tables reference beside them."""
+        from workloads import byte_model as bm
+        step = bm.step_bytes(self.wl)
+        referenced = step["attention"] + (step["append"] if self.fused else 0)
+        if "prefix_lens" not in self.wl.extra:
+            return referenced, None
+        unique = referenced - step["kv"] + bm.unique_kv_bytes(self.wl)
+        return unique, referenced
+
+    def free(self):
+        for name in ("k_cache", "v_cache", "query", "new_key", "new_value", "out", "workspace",
+                     "graphs", "block_tables", "context_lens", "slot_mapping", "block_mapping"):
+            if hasattr(self, name):
+                delattr(self, name)
+        self.run_cache = self.run_decode = None
+        self.torch.cuda.empty_cache()
+
+
+def measure_per_config(name, kv_dtype, shared, args, dev, barrier, peak):
+    """One more workload in the same run: its step timed as the headline's
+    (graph replay, events on the launching stream), reported per layer-step
+    with the decode launches' roofline fraction."""
+    wl = make_workload(name, 0, kv_dtype)
+    g = GpuStep(wl, dev, shared_prefix=shared)
+    g.prepare(args.warmup, args.eager, barrier)
+    sampler = ClockSampler(dev.index or 0)
+    barrier()
+    with sampler:
+        elapsed_ms, decode_ms = g.timed(args.steps)
+    decode_avg = statistics.mean(decode_ms)
+    dbytes, referenced = g.roofline_bytes()
+    achieved = dbytes / (decode_avg * 1e-3) / 1e9
+    label = name + (f"-{kv_dtype}" if kv_dtype != "auto" else "")
+    entry = {"workload": workload_config(wl, g.part, "")["workload"],
+             "us_per_layer_step": round(elapsed_ms / args.steps * 1e3, 2),
+             "kernel": g.kernel_name(), "decode_entry": g.entry(),
+             "avg_launch_us": round(decode_avg * 1e3, 2),
+             "algorithmic_bytes_per_launch": dbytes, "achieved": round(achieved, 1),
+             "frac": round(achieved / peak, 4),
+             "traffic": profiled_traffic(label + ("-shared" if g.shared else ""),
+                                         kernel_family(g)),
+             "sm_mhz": sampler.summary()["sm_mhz"]}
+    if referenced is not None:
+        entry["frac_on"] = "unique K/V bytes (shared blocks counted once)"
+        entry["referenced_bytes_per_launch"] = referenced
+    g.free()
+    del wl
+    return label + ("-shared" if g.shared else ""), entry
+
+
+def kernel_family(g) -> str:
+    """The decode kernel family whose sources a traffic line depends on."""
+    if g.shared:
+        return "shared"
+    if g.quant:
+        return "q8"
+    group = g.wl.num_q_heads // g.wl.num_kv_heads
+    return "mma" if group >= 4 and g.wl.block_size % 16 == 0 else "fp32"
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -373,155 +638,37 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
 
-    from paged_kv_cache_415_b200 import binding as B
     from workloads import byte_model as bm
 
-    wl = make_workload(args.config, args.seqs, args.kv_dtype)
     dev = torch.device("cuda", local)
-    tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
-    codes = wl.extra.get("kv_dtype")                  # None, "fp8" or "int8"
-    quant = codes is not None
-    if quant:
-        q_write, q_decode, q_decode_append = (
-            getattr(B, f"pa_reshape_and_cache_{codes}"), getattr(B, f"pa_paged_decode_{codes}"),
-            getattr(B, f"pa_paged_decode_{codes}_append"))
-    k_scale, v_scale = wl.extra.get("k_scale", 1.0), wl.extra.get("v_scale", 1.0)
-
-    def up(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(tdt)
-
-    if quant:
-        k_cache = torch.from_numpy(wl.k_cache).to(dev)
-        v_cache = torch.from_numpy(wl.v_cache).to(dev)
-    else:
-        k_cache, v_cache = up(wl.k_cache), up(wl.v_cache)
-    query = up(wl.query)
-    new_key, new_value = up(wl.new_key), up(wl.new_value)
-    slot_mapping = torch.from_numpy(wl.slot_mapping).to(dev)
-    block_tables = torch.from_numpy(wl.block_tables).to(dev)
-    context_lens = torch.from_numpy(wl.context_lens).to(dev)
-    block_mapping = torch.from_numpy(np.ascontiguousarray(wl.block_mapping)).to(dev)
-    out = torch.empty_like(query)
-    d_status = torch.zeros(1, dtype=torch.int32, device=dev)
-    mcl = wl.max_context_len
-    want = wl.partition_size if args.partition < 0 else args.partition
-    part = B.pa_paged_decode_partition_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
-                                            wl.head_dim, wl.block_size, mcl, want)
-    ws_bytes = B.pa_paged_decode_workspace_size(wl.num_seqs, wl.num_q_heads, wl.num_kv_heads,
-                                                wl.head_dim, wl.block_size, mcl, part)
-    workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    max_parts = -(-mcl // part) if mcl > 0 else 1
-    n_pairs = int(wl.block_mapping.shape[0])
-    stream = torch.cuda.current_stream(dev)
-
-    fused = (not args.separate and not args.shared_prefix
-             and wl.extra.get("one_token_per_seq", False) and wl.num_new_tokens == wl.num_seqs)
-
-    def cache_ops():
-        if n_pairs:
-            B.pa_copy_blocks(k_cache, v_cache, block_mapping, d_status, stream)
-        if wl.num_new_tokens and quant and not fused:
-            q_write(new_key, new_value, k_cache, v_cache, slot_mapping, k_scale, v_scale,
-                    d_status, stream)
-        elif wl.num_new_tokens and not fused:
-            B.pa_reshape_and_cache(new_key, new_value, k_cache, v_cache, slot_mapping, d_status,
-                                   stream)
-
-    shared = args.shared_prefix and "prefix_lens" in wl.extra and not quant
-    if shared:
-        group_size = int(wl.extra["group_size"])
-        prefix_lens = torch.from_numpy(wl.extra["prefix_lens"]).to(dev)
-        mpl = int(wl.extra["prefix_lens"].max())
-        sws = B.pa_paged_decode_shared_prefix_workspace_size(
-            wl.num_seqs, group_size, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size,
-            mcl, mpl, 0)
-        workspace = torch.empty(max(sws, 16), dtype=torch.uint8, device=dev)
-
-    def decode():
-        if quant and fused:
-            q_decode_append(out, query, new_key, new_value, k_cache, v_cache, block_tables,
-                            context_lens, mcl, wl.scale, k_scale, v_scale, part, workspace,
-                            d_status, stream)
-        elif quant:
-            q_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl, wl.scale,
-                     k_scale, v_scale, part, workspace, d_status, stream)
-        elif fused:
-            B.pa_paged_decode_append(out, query, new_key, new_value, k_cache, v_cache,
-                                     block_tables, context_lens, mcl, wl.scale, part, workspace,
-                                     d_status, stream)
-        elif shared:
-            B.pa_paged_decode_shared_prefix(out, query, k_cache, v_cache, block_tables,
-                                            context_lens, prefix_lens, group_size, mcl, mpl,
-                                            wl.scale, workspace, 0, d_status, stream)
-        else:
-            B.pa_paged_decode(out, query, k_cache, v_cache, block_tables, context_lens, mcl,
-                              wl.scale, part, workspace, d_status, stream)
-
-    shared_parts_gt1 = shared and sws > 0            # a reduction runs after the shared kernel
-    launches_per_step = (1 if n_pairs else 0) + (1 if (wl.num_new_tokens and not fused) else 0) + \
-        1 + (1 if (max_parts > 1 and not shared) or shared_parts_gt1 else 0)
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # warm-up
-    for _ in range(args.warmup):
-        cache_ops()
-        decode()
-    barrier()
-    run_cache, run_decode = cache_ops, decode
-    if not args.eager:
-        # the step's launches captured once; replay issues them with no host work
-        g_cache, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        has_cache = bool(n_pairs or (wl.num_new_tokens and not fused))
-        saved = stream
-        with torch.cuda.graph(g_dec):
-            stream = torch.cuda.current_stream(dev)
-            decode()
-        if has_cache:
-            with torch.cuda.graph(g_cache):
-                stream = torch.cuda.current_stream(dev)
-                cache_ops()
-        stream = saved
-        run_cache = g_cache.replay if has_cache else (lambda: None)
-        run_decode = g_dec.replay
-        run_cache()
-        run_decode()
-        barrier()
-    if int(d_status.item()) != 0 or not torch.isfinite(out.float()).all():
-        raise SystemExit(f"rank {rank}: bad step (status {int(d_status.item())})")
+    wl = make_workload(args.config, args.seqs, args.kv_dtype)
+    g = GpuStep(wl, dev, args.partition, args.separate, args.shared_prefix)
+    g.prepare(args.warmup, args.eager, barrier)
 
-    # timed region: K steps; events bracket the decode kernels of every step
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # timed region: K steps
     sampler = ClockSampler(local)
     barrier()
     with sampler:
-        start.record(stream)
-        for i in range(args.steps):
-            run_cache()
-            ev[i][0].record(stream)
-            run_decode()
-            ev[i][1].record(stream)
-        stop.record(stream)
-        torch.cuda.synchronize(dev)
+        elapsed_ms, decode_ms = g.timed(args.steps)
     barrier()
-    elapsed_ms = start.elapsed_time(stop)
-    decode_ms = [a.elapsed_time(b) for a, b in ev]
 
     # end to end through the public API: pinned host inputs -> device -> step -> host output
     from paged_kv_cache_415_b200.step import DecodeStep, HostPipeline
-    stepper = DecodeStep(k_cache, v_cache, wl.num_seqs, wl.num_q_heads, mcl, part, k_scale,
-                         v_scale)
+    tdt, fused = g.tdt, g.fused
+    stepper = DecodeStep(g.k_cache, g.v_cache, wl.num_seqs, wl.num_q_heads, g.mcl, g.part,
+                         g.k_scale, g.v_scale)
     host = {"query": torch.from_numpy(wl.query.view(np.int16)).view(tdt).pin_memory(),
             "block_tables": torch.from_numpy(wl.block_tables).pin_memory(),
             "context_lens": torch.from_numpy(wl.context_lens).pin_memory(),
-            "out": torch.empty(out.shape, dtype=tdt).pin_memory()}
-    devb = {"query": torch.empty_like(query), "block_tables": torch.empty_like(block_tables),
-            "context_lens": torch.empty_like(context_lens), "out": torch.empty_like(out)}
+            "out": torch.empty(g.out.shape, dtype=tdt).pin_memory()}
+    devb = {"query": torch.empty_like(g.query), "block_tables": torch.empty_like(g.block_tables),
+            "context_lens": torch.empty_like(g.context_lens), "out": torch.empty_like(g.out)}
     if wl.num_new_tokens:
         host["new_key"] = torch.from_numpy(wl.new_key.view(np.int16)).view(tdt).pin_memory()
         host["new_value"] = torch.from_numpy(wl.new_value.view(np.int16)).view(tdt).pin_memory()
@@ -531,7 +678,7 @@ def run_ours(args):
             names += ("slot_mapping",)
         for k in names:
             devb[k] = torch.empty_like(host[k], device=dev)
-    if n_pairs:
+    if g.n_pairs:
         host["block_mapping"] = torch.from_numpy(np.ascontiguousarray(wl.block_mapping)).pin_memory()
         devb["block_mapping"] = torch.empty_like(host["block_mapping"], device=dev)
     h2d = sum(t.numel() * t.element_size() for k, t in host.items() if k != "out")
@@ -545,13 +692,15 @@ def run_ours(args):
         pipe.submit(packed, wl.scale, host_out, fused_append=fused)
     pipe.synchronize()
     barrier()
+    e_sampler = ClockSampler(local)
     e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record(pipe.up)
-    for _ in range(args.steps):
-        pipe.submit(packed, wl.scale, host_out, fused_append=fused)
-    e_stop.record(pipe.down)
-    pipe.synchronize()
-    torch.cuda.synchronize(dev)
+    with e_sampler:
+        e_start.record(pipe.up)
+        for _ in range(args.steps):
+            pipe.submit(packed, wl.scale, host_out, fused_append=fused)
+        e_stop.record(pipe.down)
+        pipe.synchronize()
+        torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = e_start.elapsed_time(e_stop)
 
@@ -563,49 +712,57 @@ def run_ours(args):
     value = whole_job_gbs(step["total"], args.steps, world, elapsed_ms)
     e2e_value = whole_job_gbs(step["total"], args.steps, world, e2e_ms)
     peak, peak_kind = hbm_peak()
-    # the decode launch also carries the step's cache write when it is fused
-    decode_bytes = step["attention"] + (step["append"] if fused else 0)
+    decode_bytes, referenced = g.roofline_bytes()
     achieved = decode_bytes / (decode_avg * 1e-3) / 1e9
-    traffic = profiled_traffic(args.config + (f"-{codes}" if quant else ""))
+    label = args.config + (f"-{g.codes}" if g.quant else "") + ("-shared" if g.shared else "")
+    traffic = profiled_traffic(label, kernel_family(g)) if args.seqs <= 0 else None
     clocks = sampler.summary()
+    clocks = merge_clocks(clocks, e_sampler.summary())
+    kernel_name, entry, launches_per_step = g.kernel_name(), g.entry(), g.launches_per_step
+    config_block = workload_config(wl, g.part, "")
+    del stepper, pipe, devb, host, host_out, packed, views
+    g.free()
+
+    per_config = {}
+    if world == 1 and not args.no_per_config and args.seqs <= 0:
+        for name, kv, shared in PER_CONFIG:
+            if name == args.config and kv == args.kv_dtype and shared == args.shared_prefix:
+                continue
+            key, entry_i = measure_per_config(name, kv, shared, args, dev, barrier, peak)
+            per_config[key] = entry_i
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        g, _, desc, threads = oracle_sample_time(wl, args.cpu_seconds)
-        cpu = {"value": round(g, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+        gb, _, desc, threads = oracle_sample_time(wl, args.cpu_seconds)
+        cpu = {"value": round(gb, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": desc}
 
     if world > 1:
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    group = wl.num_q_heads // wl.num_kv_heads
-    if shared:
-        kernel_name = "paged_decode_shared_kernel" + (
-            " + paged_decode_shared_reduce_kernel" if shared_parts_gt1 else "")
-    else:
-        kernel_name = (f"paged_decode_{codes}_kernel" if quant else
-                       "paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
-                       else "paged_decode_kernel")
-        if max_parts > 1:
-            kernel_name += " + paged_decode_reduce_kernel"
     l2 = (f"no flush: {step['kv'] / 1e9:.2f} GB of K/V per step > 126 MB L2"
           if step["kv"] > 4 * 126e6 else "working set smaller than L2 (values include L2 hits)")
+    config_block["l2"] = l2
+    roof = {"bound": "hbm", "kernel": kernel_name,
+            "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+            "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": traffic, "algorithmic_bytes_per_launch": decode_bytes,
+            "avg_launch_us": round(decode_avg * 1e3, 2)}
+    if referenced is not None:
+        roof["frac_on"] = "unique K/V bytes (shared blocks counted once)"
+        roof["referenced_bytes_per_launch"] = referenced
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": ({"fp8": "f16 (e4m3 K/V)", "int8": "f16 (int8 K/V)"}[codes] if quant
+        "dtype": ({"fp8": "f16 (e4m3 K/V)", "int8": "f16 (int8 K/V)"}[g.codes] if g.quant
                   else wl.dtype),
-        "data": "synthetic", "config": workload_config(wl, part, l2),
+        "data": "synthetic", "config": config_block,
         "us_per_layer_step": round(per_step_ms * 1e3, 2),
         "kv_tokens_per_s": round(world * int(wl.context_lens.sum()) * args.steps / (elapsed_ms * 1e-3)),
         "pct_of_hbm_peak": round(100 * value / world / peak, 2),
-        "roofline": {"bound": "hbm", "kernel": kernel_name,
-                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": traffic, "algorithmic_bytes_per_launch": decode_bytes,
-                     "avg_launch_us": round(decode_avg * 1e3, 2)},
+        "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms / args.steps, 5),
                 "api": "step.HostPipeline: per step, the packed pinned inputs uploaded in one "
@@ -617,19 +774,27 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "bytes_per_step": step,
         "launch": "eager" if args.eager else "CUDA-graph replay (cache ops graph, decode graph)",
-        "decode_entry": (f"pa_paged_decode_{codes}_append (quantising cache write fused)"
-                         if quant and fused else
-                         f"pa_reshape_and_cache_{codes} + pa_paged_decode_{codes}" if quant else
-                         "pa_paged_decode_shared_prefix" if shared else
-                         "pa_paged_decode_append (cache write fused)" if fused else
-                         "pa_reshape_and_cache + pa_paged_decode"),
+        "decode_entry": entry,
     }
-    if "prefix_lens" in wl.extra:
-        uniq = bm.unique_kv_bytes(wl)
-        line["unique_kv_bytes"] = uniq
-        line["unique_kv_gbs_decode"] = round(uniq / (decode_avg * 1e-3) / 1e9, 1)
+    if per_config:
+        line["per_config"] = per_config
     print(json.dumps(line))
     return 0
+
+
+def merge_clocks(a: dict, b: dict) -> dict:
+    """Clock records of the timed region and of the end-to-end loop as one:
+    the median of both regions' samples is not kept per sample, so the
+    record keeps the lower median, the union of reasons and the sample
+    counts of both."""
+    if not b.get("samples"):
+        return a
+    if not a.get("samples"):
+        return dict(b, regions="e2e loop")
+    return {"sm_mhz": min(a["sm_mhz"], b["sm_mhz"]), "sm_max_mhz": a["sm_max_mhz"] or b["sm_max_mhz"],
+            "reasons": sorted(set(a["reasons"]) | set(b["reasons"])),
+            "samples": a["samples"] + b["samples"], "source": a["source"],
+            "regions": "timed region and e2e loop"}
 
 
 # ---------------------------------------------------------------------------

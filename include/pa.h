@@ -489,9 +489,11 @@ PA_API pa_status pa_paged_decode_shared_prefix(
  *    PA_NO_ALLOC_WORKSPACE_BYTES is rejected with PA_ERR_INVALID_ARG before
  *    anything is enqueued; use pa_paged_decode with your own workspace (or a
  *    longer partition_size) for it.
- *  - The first call on a device that needs the scratch looks up the array's
- *    device address (cudaGetSymbolAddress, with that device current) and
- *    keeps it; make that first call before any stream capture.
+ *  - Every call that needs the scratch looks up the array's device address
+ *    in the current device's context (cudaGetSymbolAddress), so a device
+ *    reset or another context never leaves a stale address behind.  The
+ *    first such call on a device also loads the library's device code
+ *    there: make that first call before any stream capture.
  *  - Every call shares the one array, which keeps the previous call's
  *    contents.  Nothing in it needs clearing (every value the reduction reads
  *    is written earlier in the same call), but calls that overlap on the GPU

@@ -40,7 +40,11 @@ EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_
            "pa_paged_decode_fp8_append", "pa_reshape_and_cache_int8", "pa_paged_decode_int8",
            "pa_paged_decode_int8_append", "pa_swap_blocks",
            "pa_status_string", "pa_version")
-# Size of the library-owned scratch of pa_paged_decode_no_alloc.
+# The test entry points declared in include/pa_selftest.h.
+SELFTEST_EXPORTS = ("pa_selftest_bounded_wait", "pa_selftest_decode_abort",
+                    "pa_selftest_shared_prefix_abort")
+# Size of the library-owned scratch of pa_paged_decode_no_alloc (the
+# PA_NO_ALLOC_WORKSPACE_BYTES of include/pa.h; a CPU test compares the two).
 PA_NO_ALLOC_WORKSPACE_BYTES = 32 << 20
 
 
@@ -96,6 +100,16 @@ def _load() -> ctypes.CDLL:
     lib.pa_paged_decode_int8_append.restype = i32
     lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64, i32, p, p]
     lib.pa_swap_blocks.restype = i32
+    lib.pa_selftest_bounded_wait.argtypes = [p, p, ctypes.c_uint32, i32, p]
+    lib.pa_selftest_bounded_wait.restype = i32
+    lib.pa_selftest_decode_abort.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64,
+                                             i32, f32, i32, p, sz, i32, i32, ctypes.c_uint32, p,
+                                             p]
+    lib.pa_selftest_decode_abort.restype = i32
+    lib.pa_selftest_shared_prefix_abort.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32,
+                                                    i32, i32, i64, i32, i32, f32, i32, p, sz, i32,
+                                                    ctypes.c_uint32, p, p]
+    lib.pa_selftest_shared_prefix_abort.restype = i32
     lib.pa_status_string.argtypes = [i32]
     lib.pa_status_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
@@ -352,3 +366,50 @@ def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, d_status=None, str
         _addr(src_k), _addr(src_v), _addr(dst_k), _addr(dst_v), _addr(block_mapping),
         int(block_mapping.shape[0]), hkv, d, block_size, src_nb, dst_nb, _dtype(src_k),
         _ptr(d_status), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Test entry points of the bounded waits (include/pa_selftest.h)
+# ---------------------------------------------------------------------------
+
+def pa_selftest_bounded_wait(d_status, wait_limit_us, num_ctas=1, d_wait_ns=None,
+                             stream=None) -> None:
+    """num_ctas CTAs wait on an mbarrier nothing arrives on, bounded by
+    wait_limit_us; each warp that gives up sets PA_STATUS_TIMEOUT in
+    d_status.  d_wait_ns (int64 [num_ctas], optional) gets each CTA's wait."""
+    _check("pa_selftest_bounded_wait", LIB.pa_selftest_bounded_wait(
+        _ptr(d_status), _ptr(d_wait_ns), int(wait_limit_us), int(num_ctas), _stream(stream)))
+
+
+def pa_selftest_decode_abort(out, query, k_cache, v_cache, block_tables, context_lens,
+                             max_context_len, scale, wait_limit_us, partition_size=0,
+                             workspace=None, d_status=None, stream=None) -> None:
+    """pa_paged_decode (16-bit pools) or the e4m3 / int8 decode (uint8 / int8
+    pools, scales 1) with every warp's first wait sent to an mbarrier that
+    nothing completes: the abort path of a timed-out copy runs in every CTA."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_selftest_decode_abort", LIB.pa_selftest_decode_abort(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), num_seqs, hq, hkv, d, block_size, int(block_tables.shape[1]),
+        num_blocks, int(max_context_len), float(scale), int(partition_size), _ptr(workspace),
+        ws_bytes, _dtype(query), _dtype(k_cache), int(wait_limit_us), _ptr(d_status),
+        _stream(stream)))
+
+
+def pa_selftest_shared_prefix_abort(out, query, k_cache, v_cache, block_tables, context_lens,
+                                    prefix_lens, group_size, max_context_len, max_prefix_len,
+                                    scale, workspace, wait_limit_us, partition_size=0,
+                                    d_status=None, stream=None) -> None:
+    """pa_paged_decode_shared_prefix with every warp's first wait sent to an
+    mbarrier that nothing completes."""
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("pa_selftest_shared_prefix_abort", LIB.pa_selftest_shared_prefix_abort(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+        _ptr(context_lens), _ptr(prefix_lens), num_seqs, int(group_size), hq, hkv, d, block_size,
+        int(block_tables.shape[1]), num_blocks, int(max_context_len), int(max_prefix_len),
+        float(scale), int(partition_size), _ptr(workspace), ws_bytes, _dtype(query),
+        int(wait_limit_us), _ptr(d_status), _stream(stream)))

@@ -98,16 +98,55 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
 }
 
 // Waits for the barrier phase with the given parity.  Returns false if it
-// has not completed after kWaitTimeoutNs (or kWaitMaxPolls polls).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity)
+// has not completed after limit_ns (or kWaitMaxPolls polls).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitTimeoutNs)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 0; i < kWaitMaxPolls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 63u && global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+        if ((i & 63u) == 63u && global_timer_ns() - t0 > limit_ns) return false;
     }
     return false;
+}
+
+// The same wait for a whole warp, with one answer for every lane: true only
+// if every lane saw the phase complete.  A lane that gives up at the limit
+// while another saw the phase complete makes the warp give up, so the warp
+// never diverges on it.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               uint64_t limit_ns = kWaitTimeoutNs)
+{
+    return __all_sync(kFullMask, mbar_wait_bounded(bar, parity, limit_ns)) != 0;
+}
+
+// A warp's ring of copy stages gave up waiting at stage `first_pending`
+// (copies first_pending .. issued - 1 may still be in flight into its shared
+// memory).  Records PA_STATUS_TIMEOUT and waits again, bounded, for each of
+// those copies.  Returns whether all of them landed.  Whatever it returns,
+// the caller must not read or reuse that shared memory: the CTA writes its
+// "no result" through global memory only and returns (store_aborted_rows).
+template <int NSTAGE>
+__device__ __forceinline__ bool drain_after_timeout(uint64_t* wbar, int first_pending, int issued,
+                                                    int32_t* d_status)
+{
+    if ((threadIdx.x & 31) == 0 && d_status != nullptr) atomicOr(d_status, PA_STATUS_TIMEOUT);
+    bool landed = true;
+    for (int k = first_pending; k < issued; ++k)
+        landed &= mbar_wait_warp(&wbar[k % NSTAGE], (k / NSTAGE) & 1);
+    return landed;
+}
+
+// Test hook of the bounded waits (pa_selftest_decode_abort): with a nonzero
+// probe, a warp waits first on `never` -- an mbarrier that nothing arrives
+// on -- with a limit of probe_us microseconds, and gives up there before its
+// first block, so the timeout, the drain of the copies already issued and
+// the abort store all run for real.  With probe_us == 0 (every library
+// call) it returns false at once.  Warp-uniform.
+__device__ __forceinline__ bool probe_gives_up(uint64_t* never, uint32_t probe_us)
+{
+    return probe_us != 0u && !mbar_wait_warp(never, 0u, 1000ull * probe_us);
 }
 
 // Asynchronous bulk copy global -> shared of `bytes` (multiple of 16, both

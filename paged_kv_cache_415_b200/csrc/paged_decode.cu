@@ -1,41 +1,16 @@
-// paged_decode.cu -- single-query attention over a paged KV cache (sm_100a).
+// paged_decode.cu -- host entry points of single-query attention over a
+// paged KV cache (sm_100a): argument checks, the partition choice, the
+// tensor maps of the pools, the dispatch over (element type, head_dim,
+// block_size, query group) to the kernel families, and their launches with
+// programmatic dependent launch.
 //
-// Kernel 1, paged_decode_kernel (query groups G < 4): one CTA per (kv head,
-// context partition, sequence).  The CTA carries the G = Hq / Hkv query heads
-// of its kv head, so every K/V byte is read from HBM once for all of them.
-// Each of its four warps runs its own pipeline over every fourth physical
-// block of the partition:
-//   * the warp's block-table entries sit one per lane (32 blocks per load,
-//     the first chunk read together with the context length) and are
-//     broadcast with a shuffle ("PagedAttention：大模型KV Cache分页管理优化实践"
-//     §3.2: flattened table, warp-level prefetch);
-//   * one lane requests each block's K and V tile of this kv head (block_size
-//     rows of head_dim elements) with two TMA tensor copies into the warp's
-//     shared-memory ring of NSTAGE stages, completion counted on one mbarrier
-//     per stage, so the next blocks are in flight while one is computed
-//     (§4.2 prefetch, §5.2 overlap of copy and compute);
-//   * scores q.k in fp32 (fma.rn.f32 on the 16-bit operands): 8 (or 16)
-//     lanes share a token row and the partial dot products are reduced with
-//     a transposing butterfly of warp shuffles; scale * log2(e) multiplies
-//     the reduced score, so the exponentials are exp2;
-//   * the softmax is the blocked form of §5.1 (分块Softmax算法) run online:
-//     per tile the local max, the running (global) max, the exp-sum rescaled
-//     to it, then the weighted V rows accumulate into fp32 outputs rescaled
-//     the same way.
-// At the end the four warps' (max, sum, output) are merged through shared
-// memory in a fixed order.  A sequence whose context fits one partition gets
-// its output row written directly; otherwise the partition's max, sum and
-// normalised output go to the workspace.  With a fused append, the warp that
-// loads the block holding a sequence's new token writes that token's K/V row
-// first.  Small batches are dispatched longest context first (lpt_sequence).
-//
-// Kernel 2, paged_decode_reduce_kernel: one warp per (sequence, query head)
-// with more than one partition merges the partitions with the same rule:
-//   M = max_p m_p,  w_p = l_p * 2^(m_p - M),  out = sum_p w_p Ohat_p / sum_p w_p.
-//
-// The grouped-head (paged_decode_mma.cuh), one-byte-code (e4m3 or int8:
-// paged_decode_q8.cuh) and shared-prefix (paged_decode_shared.cuh) kernels are included below; this
-// file also holds the host entry points and their launch logic.
+// The kernels live in headers of their own, one per family:
+//   paged_decode_fp32.cuh    query groups G < 4, fp32 CUDA-core arithmetic;
+//   paged_decode_mma.cuh     G >= 4, warp-level tensor-core contractions;
+//   paged_decode_q8.cuh      pools of one-byte codes (e4m3 or int8);
+//   paged_decode_shared.cuh  groups of sequences sharing a stored prefix;
+//   decode_common.cuh        what they share, and the split-context
+//                            reduction kernel.
 //
 // The whole computation has a fixed summation order, so results are
 // deterministic and do not depend on where the blocks sit in the pool.
@@ -53,603 +28,14 @@
 #include "pa.h"
 #include "pa_common.cuh"
 #include "pa_host.h"
-
-namespace pa {
-
-constexpr int kWarps = 4;
-constexpr int kThreads = kWarps * 32;
-constexpr int kReduceRowsPerCta = 4;
-
-template <int D, int BS, int G>
-struct DecodeShape {
-    static constexpr int LPT = (G >= 4 && D == 128) ? 16 : 8;   // lanes per token row
-    static constexpr int RPW = 32 / LPT;                        // token rows per warp pass
-    static constexpr int EPT = D / LPT;                         // elements per lane
-    static constexpr int NCHUNK = EPT / 8;                      // 16-byte chunks per lane
-    // Tokens scored per softmax step: the whole block, or a slice of it so
-    // that a lane never holds more than 16 partial scores.
-    static constexpr int CT_MAX = 16 * RPW / G > RPW ? 16 * RPW / G : RPW;
-    static constexpr int CT = BS < CT_MAX ? BS : CT_MAX;
-    static constexpr int TILES = BS / CT;
-    static constexpr int ITERS = CT / RPW;                      // passes per tile
-    static constexpr int ROW_BYTES = D * 2;
-    static constexpr int TILE_BYTES = BS * ROW_BYTES;           // K (or V) of one block, one head
-    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr int NSTAGE = STAGE_BYTES <= 4096 ? 3 : 2;
-    static constexpr int NVAL = ITERS * G;                      // partial scores per lane
-    static constexpr int NHELD = NVAL >= LPT ? NVAL / LPT : 1;  // scores per lane after reduce
-    static constexpr int SM_TPL = (CT * G + 31) / 32;           // softmax items per lane
-    static constexpr int WARP_STAGE_BYTES = NSTAGE * STAGE_BYTES;
-    static constexpr int OFF_SCORES = kWarps * WARP_STAGE_BYTES;
-    static constexpr int SCORE_FLOATS = CT * G;
-    static constexpr int OFF_CORR = OFF_SCORES + kWarps * SCORE_FLOATS * 4;
-    static constexpr int CORR_FLOATS = (G + 3) / 4 * 4;
-    static constexpr int OFF_BARS = OFF_CORR + kWarps * CORR_FLOATS * 4;
-    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8;
-    static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
-    // CTAs per SM the register budget is sized for: larger groups keep more
-    // live state per lane (q and the output accumulators of every head).
-    static constexpr int MIN_CTAS = G >= 8 ? 2 : 3;
-    static_assert(EPI_BYTES <= OFF_SCORES, "epilogue must fit in the stage buffers");
-    static_assert(EPT % 8 == 0, "lanes hold whole 16-byte chunks");
-    static_assert(CT % RPW == 0 && BS % CT == 0, "tiles split evenly over the warp");
-    static_assert(32 % G == 0, "group size divides the warp");
-    static_assert(NVAL <= 16, "partial scores per lane");
-};
-
-// Sums NVAL per-lane partial values over groups of LPT lanes.  Each halving
-// step sends the half of the values this lane does not keep and adds the
-// partner's copy of the half it keeps, so the shuffle count falls from
-// NVAL*log2(LPT) to about NVAL.  Returns the index of the first value the
-// lane now holds in full; it holds NHELD consecutive values.
-template <int NVAL, int LPT>
-__device__ __forceinline__ int transpose_reduce(float (&v)[NVAL], int c)
-{
-    int base = 0;
-    int n = NVAL;
-#pragma unroll
-    for (int m = LPT / 2; m >= 1; m >>= 1) {
-        if (n > 1) {
-            const bool upper = (c & m) != 0;
-            const int half = n / 2;
-#pragma unroll
-            for (int j = 0; j < NVAL / 2; ++j) {
-                if (j < half) {
-                    const float lo = v[j], hi = v[j + half];
-                    const float send = upper ? lo : hi;
-                    const float keep = upper ? hi : lo;
-                    v[j] = keep + __shfl_xor_sync(kFullMask, send, m);
-                }
-            }
-            if (upper) base += half;
-            n = half;
-        } else {
-            v[0] += __shfl_xor_sync(kFullMask, v[0], m);
-        }
-    }
-    return base;
-}
-
-template <typename T, int D, int G>
-__device__ __forceinline__ void write_zero_rows(T* out, int s, int kvh, int num_q_heads)
-{
-    T* row = out + (static_cast<int64_t>(s) * num_q_heads + kvh * G) * D;
-    for (int i = threadIdx.x; i < G * D / 8; i += blockDim.x)
-        reinterpret_cast<uint4*>(row)[i] = make_uint4(0, 0, 0, 0);
-}
-
-// Longest-first dispatch.  The CTAs of a grid start in blockIdx order, so
-// when CTA z serves the z-th sequence in order of decreasing context length
-// (ties by index), the long contexts start first and the last wave holds
-// the short ones: the tail where few CTAs are left shrinks.  A batch in
-// which adjacent sequences share their stored prefix (the same first
-// physical block, as the beams of one prompt) keeps the grid order instead:
-// there the CTAs of one group running together, reusing the shared blocks
-// in L2, is worth more than the order.  Every thread of the CTA calls this
-// before anything else uses `scratch` (num_seqs + 1 ints of shared memory,
-// reused afterwards); needs num_seqs <= blockDim.x.  The mapping is a
-// permutation, so each sequence is served exactly once; the work of a
-// (sequence, head, partition) does not depend on which CTA runs it, so
-// results are unchanged.
-__device__ __forceinline__ int lpt_sequence(const int32_t* __restrict__ context_lens,
-                                            const int32_t* __restrict__ block_tables,
-                                            int32_t max_blocks_per_seq, int32_t num_seqs,
-                                            int rank, int32_t* scratch)
-{
-    const int t = threadIdx.x;
-    int32_t c = 0;
-    bool shares = false;
-    if (t < num_seqs) {
-        c = context_lens[t];
-        scratch[t] = c;
-        if (t > 0)
-            shares = block_tables[static_cast<int64_t>(t) * max_blocks_per_seq] ==
-                     block_tables[static_cast<int64_t>(t - 1) * max_blocks_per_seq];
-    }
-    if (__syncthreads_or(shares)) return rank;   // grid order; scratch is not read again
-    if (t < num_seqs) {
-        int r = 0;
-        for (int j = 0; j < num_seqs; ++j) {
-            const int32_t cj = scratch[j];
-            r += (cj > c || (cj == c && j < t)) ? 1 : 0;
-        }
-        if (r == rank) scratch[num_seqs] = t;
-    }
-    __syncthreads();
-    const int pick = scratch[num_seqs];
-    __syncthreads();   // scratch is free again
-    return pick;
-}
-
-// A warp's first chunk of table entries (blocks warp + kWarps * lane of the
-// partition), read before the context length is known: the index is checked
-// against the table row only, so the load is in bounds whatever the context,
-// and it overlaps the context-length load instead of following it.  Lanes
-// past the warp's block count discard their entry.
-__device__ __forceinline__ int prefetch_table_chunk(const int32_t* __restrict__ block_tables,
-                                                    int s, int max_blocks_per_seq, int blk_begin,
-                                                    int warp, int lane)
-{
-    const int idx = blk_begin + warp + kWarps * lane;
-    return idx < max_blocks_per_seq
-               ? block_tables[static_cast<int64_t>(s) * max_blocks_per_seq + idx]
-               : -1;
-}
-
-// Fused append: the warp that loads the block holding a sequence's new token
-// (position ctx - 1) first writes that token's K and V row for its kv head
-// into the pools at the given physical block, then makes the writes visible
-// to the tensor-copy engine before the block's tiles are requested.  No
-// other warp or CTA reads that (token, kv head) row.  Warp-uniform; the
-// caller issues the block's copies right after.
-template <typename T, int D, int BS>
-__device__ __forceinline__ void append_row_warp(
-    const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
-    T* __restrict__ v_cache, int s, int kvh, int num_kv_heads, int32_t pos, int32_t phys,
-    int lane)
-{
-    const int64_t slot = static_cast<int64_t>(phys) * BS + pos % BS;
-    const int64_t src = (static_cast<int64_t>(s) * num_kv_heads + kvh) * D;
-    const int64_t dst = (slot * num_kv_heads + kvh) * D;
-    if (lane < D / 8) {
-        const uint4 kv = ld_nc_v4(new_key + src + lane * 8);
-        const uint4 vv = ld_nc_v4(new_value + src + lane * 8);
-        *reinterpret_cast<uint4*>(k_cache + dst + lane * 8) = kv;
-        *reinterpret_cast<uint4*>(v_cache + dst + lane * 8) = vv;
-        fence_proxy_async_global();
-    }
-    __syncwarp();
-    fence_proxy_async_global();
-}
-
-// The CTA's last step: merge the four warps' (max, exp-sum, output) for the
-// G heads of its kv head in a fixed order, then either write the output row
-// (context in one partition) or the partition's max, sum and normalised
-// output to the workspace.  epi_o is [warp][g][D], epi_m / epi_l [warp][g],
-// in shared memory, complete (the caller synchronised the CTA).
-template <typename T, int D, int G>
-__device__ __forceinline__ void merge_warps_and_store(
-    const float* epi_o, const float* epi_m, const float* epi_l, T* __restrict__ out,
-    float* __restrict__ ws_o, float2* __restrict__ ws_ml, int s, int kvh, int part, int nparts,
-    int num_q_heads, int max_parts)
-{
-    for (int idx = threadIdx.x; idx < G * D / 8; idx += kThreads) {
-        const int g = idx / (D / 8);
-        const int d0 = (idx % (D / 8)) * 8;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, epi_m[w * G + g]);
-        const float msub = M == -INFINITY ? 0.f : M;
-        float L = 0.f;
-        float O[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) O[e] = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            const float f = exp2f(epi_m[w * G + g] - msub);
-            L = fmaf(f, epi_l[w * G + g], L);
-            const float4* src = reinterpret_cast<const float4*>(epi_o + (w * G + g) * D + d0);
-            const float4 a = src[0], b = src[1];
-            O[0] = fmaf(f, a.x, O[0]); O[1] = fmaf(f, a.y, O[1]);
-            O[2] = fmaf(f, a.z, O[2]); O[3] = fmaf(f, a.w, O[3]);
-            O[4] = fmaf(f, b.x, O[4]); O[5] = fmaf(f, b.y, O[5]);
-            O[6] = fmaf(f, b.z, O[6]); O[7] = fmaf(f, b.w, O[7]);
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) O[e] *= inv;
-        const int h = kvh * G + g;
-        const int64_t row = static_cast<int64_t>(s) * num_q_heads + h;
-        if (nparts == 1) {
-            *reinterpret_cast<uint4*>(out + row * D + d0) = pack8<T>(O);
-        } else {
-            const int64_t prow = row * max_parts + part;
-            float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + d0);
-            dst[0] = make_float4(O[0], O[1], O[2], O[3]);
-            dst[1] = make_float4(O[4], O[5], O[6], O[7]);
-            if (d0 == 0) ws_ml[prow] = make_float2(M, L);
-        }
-    }
-}
-
-template <typename T, int D, int BS, int G>
-__global__ void __launch_bounds__(kThreads, (DecodeShape<D, BS, G>::MIN_CTAS)) paged_decode_kernel(
-    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-    T* __restrict__ out, const T* __restrict__ query, const int32_t* __restrict__ block_tables,
-    const int32_t* __restrict__ context_lens, int32_t num_q_heads, int32_t max_blocks_per_seq,
-    int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
-    int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status,
-    const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
-    T* __restrict__ v_cache, int32_t num_kv_heads, int32_t lpt_seqs)
-{
-    grid_dependency_wait();   // before any global access (see pa_common.cuh)
-    using S = DecodeShape<D, BS, G>;
-    constexpr int EP = S::EPT / 2;      // element pairs per lane
-    extern __shared__ __align__(128) unsigned char smem[];
-
-    const int kvh = blockIdx.x;
-    const int part = blockIdx.y;
-    const int s = lpt_seqs > 0
-                      ? lpt_sequence(context_lens, block_tables, max_blocks_per_seq, lpt_seqs,
-                                     blockIdx.z, reinterpret_cast<int32_t*>(smem))
-                      : static_cast<int>(blockIdx.z);
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int c = lane % S::LPT;        // position within the token row
-    const int r = lane / S::LPT;        // token row within a pass
-
-    const int pre_tbl = prefetch_table_chunk(block_tables, s, max_blocks_per_seq,
-                                             blockIdx.y * partition_size / BS, warp, lane);
-    const int32_t ctx = context_lens[s];
-    if (ctx < 0 || ctx > max_context_len ||
-        static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * BS) {
-        if (part == 0) {
-            write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
-            if (threadIdx.x == 0) status_or(d_status, PA_STATUS_BAD_CONTEXT);
-        }
-        return;
-    }
-    if (ctx == 0) {
-        if (part == 0) write_zero_rows<T, D, G>(out, s, kvh, num_q_heads);
-        return;
-    }
-    const int tok_begin = part * partition_size;
-    if (tok_begin >= ctx) return;
-    const int tok_end = min(ctx, tok_begin + partition_size);
-    const int nparts = (ctx + partition_size - 1) / partition_size;
-    const int blk_begin = tok_begin / BS;
-    const int nblk = (tok_end - tok_begin + BS - 1) / BS;
-    const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;   // this warp's blocks
-    // the block (of this partition) holding the new token, when appending
-    const int append_blk = (new_key != nullptr && part == nparts - 1) ? (ctx - 1) / BS - blk_begin : -1;
-
-    unsigned char* wstage = smem + warp * S::WARP_STAGE_BYTES;
-    float* wscore = reinterpret_cast<float*>(smem + S::OFF_SCORES) + warp * S::SCORE_FLOATS;
-    float* wcorr = reinterpret_cast<float*>(smem + S::OFF_CORR) + warp * S::CORR_FLOATS;
-    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
-
-    if (lane == 0) {
-#pragma unroll
-        for (int st = 0; st < S::NSTAGE; ++st) mbar_init(&wbar[st], 1);
-        fence_barrier_init();
-    }
-    __syncwarp();
-
-    const int32_t* table = block_tables + static_cast<int64_t>(s) * max_blocks_per_seq + blk_begin;
-    // The warp's k-th block is block warp + kWarps * k of the partition; one
-    // table entry per lane, 32 blocks per load.
-    auto load_table = [&](int chunk) -> int {
-        const int kk = chunk * 32 + lane;
-        return kk < nk ? table[warp + kWarps * kk] : -1;
-    };
-    int prod_chunk = 0, cons_chunk = 0;
-    int prod_tbl = lane < nk ? pre_tbl : -1;   // load_table(0), already in flight
-    int cons_tbl = prod_tbl;
-
-    auto block_tokens = [&](int k) -> int {   // valid tokens of the warp's k-th block
-        const int t0 = tok_begin + (warp + kWarps * k) * BS;
-        return min(BS, tok_end - t0);
-    };
-
-    // Producer: one lane starts the two tensor copies (the K and V tiles of
-    // this kv head: BS rows of D elements) of block k into its stage.
-    auto issue = [&](int k) {
-        const int chunk = k >> 5;
-        if (chunk != prod_chunk) {
-            prod_tbl = load_table(chunk);
-            prod_chunk = chunk;
-        }
-        const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
-        if (warp + kWarps * k == append_blk) {
-            if (phys >= 0 && static_cast<int64_t>(phys) < num_blocks)
-                append_row_warp<T, D, BS>(new_key, new_value, k_cache, v_cache, s, kvh,
-                                          num_kv_heads, ctx - 1, phys, lane);
-            else if (lane == 0)
-                status_or(d_status, PA_STATUS_BAD_SLOT);
-        }
-        if (lane == 0) {
-            const int st = k % S::NSTAGE;
-            const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
-            fence_proxy_async_smem();
-            if (ok) {
-                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE_BYTES);
-                unsigned char* dst = wstage + st * S::STAGE_BYTES;
-                tma_load_4d(dst, &tm_k, 0, kvh, 0, phys, &wbar[st]);
-                tma_load_4d(dst + S::TILE_BYTES, &tm_v, 0, kvh, 0, phys, &wbar[st]);
-            } else {
-                status_or(d_status, PA_STATUS_BAD_BLOCK);
-                mbar_arrive_expect_tx(&wbar[st], 0u);
-            }
-        }
-    };
-
-    const int prologue = min(nk, S::NSTAGE);
-    for (int k = 0; k < prologue; ++k) issue(k);
-    int issued = prologue;
-
-    // q of every head in the group, this lane's elements, kept as the raw
-    // 16-bit input pairs (the products with K are exact in fp32; the scale
-    // is applied to the reduced scores).
-    uint32_t qw[G][EP];
-    {
-        const T* qrow = query + (static_cast<int64_t>(s) * num_q_heads + kvh * G) * D;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
-                const uint4 w = *reinterpret_cast<const uint4*>(qrow + g * D + k2 * 8 * S::LPT + 8 * c);
-                qw[g][k2 * 4 + 0] = w.x;
-                qw[g][k2 * 4 + 1] = w.y;
-                qw[g][k2 * 4 + 2] = w.z;
-                qw[g][k2 * 4 + 3] = w.w;
-            }
-        }
-    }
-
-    float m_run = -INFINITY;     // running max of head (lane % G), log2 units
-    float l_run = 0.f;           // this lane's share of the running exp-sum
-    float2 o2[G][EP];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < EP; ++e) o2[g][e] = make_float2(0.f, 0.f);
-
-    bool aborted = false;
-    int first_pending = 0;
-
-    for (int k = 0; k < nk; ++k) {
-        const int st = k % S::NSTAGE;
-        if (!mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1)) {
-            aborted = true;
-            first_pending = k;
-            break;
-        }
-        const int chunk = k >> 5;
-        if (chunk != cons_chunk) {
-            cons_tbl = load_table(chunk);
-            cons_chunk = chunk;
-        }
-        const int phys = __shfl_sync(kFullMask, cons_tbl, k & 31);
-        const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
-        const int nv = ok ? block_tokens(k) : 0;
-        const unsigned char* stage = wstage + st * S::STAGE_BYTES;
-#pragma unroll 1
-        for (int tile = 0; tile < S::TILES; ++tile) {
-            const unsigned char* ktile = stage + tile * S::CT * S::ROW_BYTES;
-            const unsigned char* vtile = ktile + S::TILE_BYTES;
-            const int tv = nv - tile * S::CT;     // valid tokens in this tile (may be <= 0)
-
-            // ---- scores: this lane's partial dot products (fp32 accumulation) ----
-            float acc[S::NVAL];
-#pragma unroll
-            for (int i = 0; i < S::NVAL; ++i) acc[i] = 0.f;
-#pragma unroll
-            for (int i = 0; i < S::ITERS; ++i) {
-                const int t = i * S::RPW + r;
-#pragma unroll
-                for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(
-                        ktile + t * S::ROW_BYTES + (k2 * 8 * S::LPT + 8 * c) * 2);
-                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-#pragma unroll
-                        for (int g = 0; g < G; ++g)
-                            acc[i * G + g] = fma_pair<T>(qw[g][k2 * 4 + j], words[j], acc[i * G + g]);
-                }
-            }
-            const int base = transpose_reduce<S::NVAL, S::LPT>(acc, c);
-#pragma unroll
-            for (int j = 0; j < S::NHELD; ++j) {
-                const int n = base + j;
-                const int t = (n / G) * S::RPW + r;
-                wscore[t * G + (n % G)] = t < tv ? acc[j] * scale_log2 : -INFINITY;
-            }
-            __syncwarp();
-
-            // ---- blocked softmax, online: tile max, running max, rescale ----
-            {
-                const int g = lane % G;
-                float sv[S::SM_TPL];
-                float mloc = -INFINITY;
-#pragma unroll
-                for (int kk = 0; kk < S::SM_TPL; ++kk) {
-                    const int t = lane / G + (32 / G) * kk;
-                    sv[kk] = t < S::CT ? wscore[t * G + g] : -INFINITY;
-                    mloc = fmaxf(mloc, sv[kk]);
-                }
-#pragma unroll
-                for (int m = G; m < 32; m <<= 1) mloc = fmaxf(mloc, __shfl_xor_sync(kFullMask, mloc, m));
-                const float m_new = fmaxf(m_run, mloc);
-                const float m_sub = m_new == -INFINITY ? 0.f : m_new;
-                const float corr = exp2f(m_run - m_sub);
-                l_run *= corr;
-#pragma unroll
-                for (int kk = 0; kk < S::SM_TPL; ++kk) {
-                    const int t = lane / G + (32 / G) * kk;
-                    if (t < S::CT) {
-                        const float p = exp2f(sv[kk] - m_sub);
-                        l_run += p;
-                        wscore[t * G + g] = p;
-                    }
-                }
-                m_run = m_new;
-                if (lane < G) wcorr[lane] = corr;
-            }
-            __syncwarp();
-
-            // ---- values: rescale, then accumulate p * V (packed fp32 FMA) ----
-            {
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float cg = wcorr[g];
-                    const float2 c2 = make_float2(cg, cg);
-#pragma unroll
-                    for (int e = 0; e < EP; ++e) o2[g][e] = __fmul2_rn(o2[g][e], c2);
-                }
-#pragma unroll
-                for (int i = 0; i < S::ITERS; ++i) {
-                    const int t = i * S::RPW + r;
-                    if (t < tv) {
-                        float2 p2[G];
-#pragma unroll
-                        for (int g = 0; g < G; ++g) {
-                            const float pg = wscore[t * G + g];
-                            p2[g] = make_float2(pg, pg);
-                        }
-#pragma unroll
-                        for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
-                            const uint4 w = *reinterpret_cast<const uint4*>(
-                                vtile + t * S::ROW_BYTES + (k2 * 8 * S::LPT + 8 * c) * 2);
-                            const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float2 vf = Elem<T>::to_float2(words[j]);
-#pragma unroll
-                                for (int g = 0; g < G; ++g)
-                                    o2[g][k2 * 4 + j] = __ffma2_rn(p2[g], vf, o2[g][k2 * 4 + j]);
-                            }
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-        }
-        if (issued < nk) issue(issued++);
-    }
-
-    if (aborted) {
-        if (lane == 0) status_or(d_status, PA_STATUS_TIMEOUT);
-        // Let the copies already started land (each wait bounded) before the
-        // shared memory is reused.
-        for (int k = first_pending; k < issued; ++k) {
-            const int st = k % S::NSTAGE;
-            mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1);
-        }
-    }
-
-    // ---- merge inside the warp ----
-#pragma unroll
-    for (int m = G; m < 32; m <<= 1) l_run += __shfl_xor_sync(kFullMask, l_run, m);
-#pragma unroll
-    for (int m = S::LPT; m < 32; m <<= 1)
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < EP; ++e) {
-                o2[g][e].x += __shfl_xor_sync(kFullMask, o2[g][e].x, m);
-                o2[g][e].y += __shfl_xor_sync(kFullMask, o2[g][e].y, m);
-            }
-
-    __syncthreads();   // every warp is done with its stage buffers
-    float* epi_o = reinterpret_cast<float*>(smem);                 // [warp][g][D]
-    float* epi_m = epi_o + kWarps * G * D;                         // [warp][g]
-    float* epi_l = epi_m + kWarps * G;
-    if (r == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int k2 = 0; k2 < S::NCHUNK; ++k2) {
-                float4* dst = reinterpret_cast<float4*>(epi_o + (warp * G + g) * D + k2 * 8 * S::LPT + 8 * c);
-                dst[0] = make_float4(o2[g][k2 * 4 + 0].x, o2[g][k2 * 4 + 0].y,
-                                     o2[g][k2 * 4 + 1].x, o2[g][k2 * 4 + 1].y);
-                dst[1] = make_float4(o2[g][k2 * 4 + 2].x, o2[g][k2 * 4 + 2].y,
-                                     o2[g][k2 * 4 + 3].x, o2[g][k2 * 4 + 3].y);
-            }
-    }
-    if (lane < G) {
-        epi_m[warp * G + lane] = m_run;
-        epi_l[warp * G + lane] = l_run;
-    }
-    __syncthreads();
-
-    merge_warps_and_store<T, D, G>(epi_o, epi_m, epi_l, out, ws_o, ws_ml, s, kvh, part, nparts,
-                                   num_q_heads, max_parts);
-}
-
-}  // namespace pa
-
+#include "pa_selftest.h"
+#include "decode_common.cuh"
+#include "paged_decode_fp32.cuh"
 #include "paged_decode_mma.cuh"
 #include "paged_decode_shared.cuh"
 #include "paged_decode_q8.cuh"
 
 namespace pa {
-
-// One warp per (sequence, query head) whose context spans several
-// partitions: merge the partitions' (max, exp-sum, normalised output).
-template <typename T, int D>
-__global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_reduce_kernel(
-    T* __restrict__ out, const float* __restrict__ ws_o, const float2* __restrict__ ws_ml,
-    const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t num_q_heads,
-    int32_t max_context_len, int32_t max_blocks_per_seq, int32_t block_size,
-    int32_t partition_size, int32_t max_parts)
-{
-    grid_dependency_wait();
-    constexpr int EPL = D / 32;     // elements per lane
-    const int lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kReduceRowsPerCta + (threadIdx.x >> 5);
-    if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;
-    const int s = static_cast<int>(row / num_q_heads);
-    const int32_t ctx = context_lens[s];
-    if (ctx <= 0 || ctx > max_context_len ||
-        static_cast<int64_t>(ctx) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
-        return;                                     // written by the first kernel
-    const int np = (ctx + partition_size - 1) / partition_size;
-    if (np <= 1) return;
-    const float2* ml = ws_ml + row * max_parts;
-    float M = -INFINITY;
-    for (int p = lane; p < np; p += 32) M = fmaxf(M, ml[p].x);
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFullMask, M, m));
-    const float msub = M == -INFINITY ? 0.f : M;
-    float acc[EPL];
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
-    float W = 0.f;
-    const float* orow = ws_o + row * max_parts * D + lane * EPL;
-    for (int p = 0; p < np; ++p) {
-        const float2 v = ml[p];
-        const float w = v.y * exp2f(v.x - msub);
-        W += w;
-        if (EPL == 4) {
-            const float4 x = *reinterpret_cast<const float4*>(orow + static_cast<int64_t>(p) * D);
-            acc[0] = fmaf(w, x.x, acc[0]);
-            acc[1] = fmaf(w, x.y, acc[1]);
-            acc[2] = fmaf(w, x.z, acc[2]);
-            acc[3] = fmaf(w, x.w, acc[3]);
-        } else {
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, orow[static_cast<int64_t>(p) * D + e], acc[e]);
-        }
-    }
-    const float inv = W > 0.f ? 1.f / W : 0.f;
-    T* dst = out + row * D + lane * EPL;
-#pragma unroll
-    for (int e = 0; e < EPL; e += 2) {
-        const uint32_t packed = Elem<T>::from_float2(acc[e] * inv, acc[e + 1] * inv);
-        *reinterpret_cast<uint32_t*>(dst + e) = packed;
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Host side
@@ -675,6 +61,7 @@ struct DecodeArgs {
     const void* new_value = nullptr;
     int32_t lpt_seqs = 0;              // > 0: longest-first dispatch over this many sequences
     float k_inv = 1.f, v_inv = 1.f;    // quantised pools: reciprocal scales of the fused write
+    uint32_t probe_us = 0;             // test hook of the bounded waits (pa_selftest_*); 0 = off
 };
 
 constexpr int kMaxDevices = 64;
@@ -820,7 +207,8 @@ static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
         a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status, a.lpt_seqs,
         static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
         static_cast<uint8_t*>(const_cast<void*>(a.k_cache)),
-        static_cast<uint8_t*>(const_cast<void*>(a.v_cache)), a.num_kv_heads, a.k_inv, a.v_inv);
+        static_cast<uint8_t*>(const_cast<void*>(a.v_cache)), a.num_kv_heads, a.k_inv, a.v_inv,
+        a.probe_us);
     if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
@@ -876,7 +264,7 @@ static pa_status launch_decode(const DecodeArgs& a)
             a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status,
             static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
             static_cast<T*>(const_cast<void*>(a.k_cache)), static_cast<T*>(const_cast<void*>(a.v_cache)),
-            a.num_kv_heads, a.lpt_seqs);
+            a.num_kv_heads, a.lpt_seqs, a.probe_us);
         if (ls != PA_OK) return ls;
     } else {
         using S = DecodeShape<D, BS, G>;
@@ -893,7 +281,7 @@ static pa_status launch_decode(const DecodeArgs& a)
             a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status,
             static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
             static_cast<T*>(const_cast<void*>(a.k_cache)), static_cast<T*>(const_cast<void*>(a.v_cache)),
-            a.num_kv_heads, a.lpt_seqs);
+            a.num_kv_heads, a.lpt_seqs, a.probe_us);
         if (ls != PA_OK) return ls;
     }
     if (a.max_parts <= 1) return PA_OK;
@@ -964,7 +352,7 @@ static pa_status launch_shared(const SharedArgs& sa)
         static_cast<const T*>(a.query), a.block_tables, a.context_lens, sa.prefix_lens,
         sa.group_size, a.num_q_heads / a.num_kv_heads, a.num_q_heads, a.max_blocks_per_seq,
         a.num_blocks, a.max_context_len, sa.max_prefix_len, a.scale_log2, sa.part_blocks,
-        a.max_parts, a.ws_o, a.ws_ml, a.d_status);
+        a.max_parts, a.ws_o, a.ws_ml, a.d_status, a.probe_us);
     if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
@@ -1096,7 +484,7 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
                              pa_dtype dtype, int32_t* d_status, pa_stream_t stream,
                              const void* new_key, const void* new_value,
                              KvCodes codes = KvCodes::kPlain, float k_scale = 1.f,
-                             float v_scale = 1.f)
+                             float v_scale = 1.f, uint32_t probe_us = 0)
 {
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       max_context_len, partition_size);
@@ -1154,6 +542,7 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.stream = stream;
     a.new_key = new_key;
     a.new_value = new_value;
+    a.probe_us = probe_us;
     if (quantised) {
         a.k_inv = 1.0f / k_scale;      // the quantising write's fp32(1 / scale)
         a.v_inv = 1.0f / v_scale;
@@ -1340,15 +729,17 @@ extern "C" size_t pa_paged_decode_shared_prefix_workspace_size(
     return rows * head_dim * sizeof(float) + rows * sizeof(float2);
 }
 
-extern "C" pa_status pa_paged_decode_shared_prefix(
+namespace pa {
+
+static pa_status shared_prefix_impl(
     void* out, const void* query, const void* k_cache, const void* v_cache,
     const int32_t* block_tables, const int32_t* context_lens, const int32_t* prefix_lens,
     int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t num_kv_heads,
     int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
     int32_t max_context_len, int32_t max_prefix_len, float scale, int32_t partition_size,
-    void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream)
+    void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream,
+    uint32_t probe_us)
 {
-    using namespace pa;
     pa_status st = check_shared_shape(num_seqs, group_size, num_q_heads, num_kv_heads, head_dim,
                                       block_size, max_context_len, max_prefix_len, partition_size);
     if (st != PA_OK) return st;
@@ -1401,7 +792,71 @@ extern "C" pa_status pa_paged_decode_shared_prefix(
     sa.group_size = group_size;
     sa.max_prefix_len = max_prefix_len;
     sa.part_blocks = part_blocks;
+    a.probe_us = probe_us;
     return dtype == PA_DTYPE_F16 ? dispatch_shared<__half>(sa) : dispatch_shared<__nv_bfloat16>(sa);
+}
+
+}  // namespace pa
+
+extern "C" pa_status pa_paged_decode_shared_prefix(
+    void* out, const void* query, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* prefix_lens,
+    int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, int32_t max_prefix_len, float scale, int32_t partition_size,
+    void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream)
+{
+    return pa::shared_prefix_impl(out, query, k_cache, v_cache, block_tables, context_lens,
+                                  prefix_lens, num_seqs, group_size, num_q_heads, num_kv_heads,
+                                  head_dim, block_size, max_blocks_per_seq, num_blocks,
+                                  max_context_len, max_prefix_len, scale, partition_size, workspace,
+                                  workspace_bytes, dtype, d_status, stream, 0u);
+}
+
+// ---------------------------------------------------------------------------
+// Test entry points of the bounded waits (declared in pa_selftest.h): the
+// decode kernels with every warp's first wait sent to an mbarrier that
+// nothing completes, so the timeout and the abort path run for real.
+// ---------------------------------------------------------------------------
+static constexpr uint32_t kMaxProbeUs = 1000000u;   // longest probe wait: 1 s
+
+extern "C" pa_status pa_selftest_decode_abort(
+    void* out, const void* query, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+    int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale,
+    int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+    pa_dtype kv_dtype, uint32_t wait_limit_us, int32_t* d_status, pa_stream_t stream)
+{
+    using namespace pa;
+    if (wait_limit_us == 0u || wait_limit_us > kMaxProbeUs) return PA_ERR_INVALID_ARG;
+    KvCodes codes;
+    if (kv_dtype == dtype) codes = KvCodes::kPlain;
+    else if (kv_dtype == PA_DTYPE_FP8_E4M3) codes = KvCodes::kE4m3;
+    else if (kv_dtype == PA_DTYPE_INT8) codes = KvCodes::kInt8;
+    else return PA_ERR_UNSUPPORTED;
+    return decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                       num_blocks, max_context_len, scale, partition_size, workspace,
+                       workspace_bytes, dtype, d_status, stream, nullptr, nullptr, codes, 1.f, 1.f,
+                       wait_limit_us);
+}
+
+extern "C" pa_status pa_selftest_shared_prefix_abort(
+    void* out, const void* query, const void* k_cache, const void* v_cache,
+    const int32_t* block_tables, const int32_t* context_lens, const int32_t* prefix_lens,
+    int32_t num_seqs, int32_t group_size, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, int32_t max_prefix_len, float scale, int32_t partition_size,
+    void* workspace, size_t workspace_bytes, pa_dtype dtype, uint32_t wait_limit_us,
+    int32_t* d_status, pa_stream_t stream)
+{
+    if (wait_limit_us == 0u || wait_limit_us > kMaxProbeUs) return PA_ERR_INVALID_ARG;
+    return pa::shared_prefix_impl(out, query, k_cache, v_cache, block_tables, context_lens,
+                                  prefix_lens, num_seqs, group_size, num_q_heads, num_kv_heads,
+                                  head_dim, block_size, max_blocks_per_seq, num_blocks,
+                                  max_context_len, max_prefix_len, scale, partition_size, workspace,
+                                  workspace_bytes, dtype, d_status, stream, wait_limit_us);
 }
 
 // ---------------------------------------------------------------------------
@@ -1412,24 +867,17 @@ namespace pa {
 
 static __device__ __align__(256) unsigned char g_no_alloc_workspace[PA_NO_ALLOC_WORKSPACE_BYTES];
 
-static std::mutex g_no_alloc_mutex;
-static void* g_no_alloc_ptr[kMaxDevices];   // device address of the array, per device
-
-// Device address of the array on the current device; looked up once per
-// device (host code may not use the symbol itself as a device pointer).
+// Device address of the array in the current context.  Looked up on every
+// call (host code may not use the symbol itself as a device pointer), so
+// that a cudaDeviceReset or another context on the device never leaves a
+// stale address behind; after the first call on a device the lookup only
+// reads the loaded module's table.
 static pa_status no_alloc_workspace(void** ptr)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_no_alloc_mutex);
-    if (g_no_alloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_no_alloc_workspace) != cudaSuccess || p == nullptr)
-            return PA_ERR_CUDA;
-        g_no_alloc_ptr[dev] = p;
-    }
-    *ptr = g_no_alloc_ptr[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_no_alloc_workspace) != cudaSuccess || p == nullptr)
+        return PA_ERR_CUDA;
+    *ptr = p;
     return PA_OK;
 }
 
@@ -1453,6 +901,11 @@ extern "C" pa_status pa_paged_decode_no_alloc(void* out, const void* query, cons
                                                        head_dim, block_size, max_context_len,
                                                        partition_size);
     if (need > PA_NO_ALLOC_WORKSPACE_BYTES) return PA_ERR_INVALID_ARG;
+    // pointer checks before the array's address is looked up
+    if (!out || !query || !k_cache || !v_cache || !block_tables || !context_lens ||
+        !aligned16(out) || !aligned16(query) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned4(block_tables) || !aligned4(context_lens) || (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
     void* ws = nullptr;
     if (need > 0) {
         st = no_alloc_workspace(&ws);

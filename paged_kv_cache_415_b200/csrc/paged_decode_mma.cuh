@@ -22,6 +22,9 @@
 // 128-byte swizzle: row r (one token's 64 dims, 128 bytes) keeps its 16-byte
 // chunk c at chunk c ^ (r % 8), so the 8 rows an ldmatrix reads fall in
 // different banks.
+#pragma once
+
+#include "decode_common.cuh"
 
 namespace pa {
 
@@ -36,7 +39,8 @@ struct MmaShape {
     static constexpr int NSTAGE = 2;
     static constexpr int WARP_STAGE_BYTES = NSTAGE * STAGE_BYTES;
     static constexpr int OFF_BARS = kWarps * WARP_STAGE_BYTES;
-    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8 + 1024;   // + alignment slack
+    // + a probe barrier per warp, + alignment slack
+    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * (NSTAGE + 1) * 8 + 1024;
     static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
     static_assert(BS % 16 == 0, "whole 16-token slices");
     static_assert(D % 64 == 0, "whole 128-byte rows");
@@ -69,7 +73,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
     int64_t num_blocks, int32_t max_context_len, float scale_log2, int32_t partition_size,
     int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml, int32_t* d_status,
     const T* __restrict__ new_key, const T* __restrict__ new_value, T* __restrict__ k_cache,
-    T* __restrict__ v_cache, int32_t num_kv_heads, int32_t lpt_seqs)
+    T* __restrict__ v_cache, int32_t num_kv_heads, int32_t lpt_seqs, uint32_t probe_us)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = MmaShape<D, BS, G>;
@@ -113,11 +117,11 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
     const int append_blk = (new_key != nullptr && part == nparts - 1) ? (ctx - 1) / BS - blk_begin : -1;
 
     unsigned char* wstage = smem + warp * S::WARP_STAGE_BYTES;
-    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
+    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * (S::NSTAGE + 1);
 
     if (lane == 0) {
 #pragma unroll
-        for (int st = 0; st < S::NSTAGE; ++st) mbar_init(&wbar[st], 1);
+        for (int st = 0; st <= S::NSTAGE; ++st) mbar_init(&wbar[st], 1);   // + the probe barrier
         fence_barrier_init();
     }
     __syncwarp();
@@ -195,12 +199,12 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
 
-    bool aborted = false;
+    bool aborted = nk > 0 && probe_gives_up(&wbar[S::NSTAGE], probe_us);
     int first_pending = 0;
 
-    for (int k = 0; k < nk; ++k) {
+    for (int k = 0; k < (aborted ? 0 : nk); ++k) {
         const int st = k % S::NSTAGE;
-        if (!mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1)) {
+        if (!mbar_wait_warp(&wbar[st], (k / S::NSTAGE) & 1)) {
             aborted = true;
             first_pending = k;
             break;
@@ -301,19 +305,17 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_mma_kernel(
         if (issued < nk) issue(issued++);
     }
 
-    if (aborted) {
-        if (lane == 0) status_or(d_status, PA_STATUS_TIMEOUT);
-        for (int k = first_pending; k < issued; ++k) {
-            const int st = k % S::NSTAGE;
-            mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1);
-        }
-    }
+    if (aborted) drain_after_timeout<S::NSTAGE>(wbar, first_pending, issued, d_status);
 
     // ---- merge inside the warp: exp-sum across the 4 lanes of a head ----
     l_run += __shfl_xor_sync(kFullMask, l_run, 1);
     l_run += __shfl_xor_sync(kFullMask, l_run, 2);
 
-    __syncthreads();   // every warp is done with its stage buffers
+    // every warp is done with its stage buffers, unless one gave up waiting
+    if (__syncthreads_or(aborted)) {
+        store_aborted_rows<T, D, G>(out, ws_o, ws_ml, s, kvh, part, nparts, num_q_heads, max_parts);
+        return;
+    }
     float* epi_o = reinterpret_cast<float*>(smem);                 // [warp][g][D]
     float* epi_m = epi_o + kWarps * G * D;                         // [warp][g]
     float* epi_l = epi_m + kWarps * G;

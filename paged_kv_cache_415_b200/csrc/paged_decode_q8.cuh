@@ -26,7 +26,9 @@
 // 384-byte shared tile with stmatrix.trans / ldmatrix.  Scales: k_scale
 // folds into the score scale, v_scale into the output.  The query is
 // rounded once to fp16 (exact for fp16 queries).
+#pragma once
 
+#include "decode_common.cuh"
 #include "pa_codes.cuh"
 
 namespace pa {
@@ -48,7 +50,8 @@ struct Q8Shape {
     static constexpr int WARP_BYTES = NSTAGE * STAGE;
     static constexpr int OFF_PT = kWarps * WARP_BYTES;
     static constexpr int OFF_BARS = OFF_PT + kWarps * PT_BYTES;
-    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8 + 1024;   // + alignment slack
+    // + a probe barrier per warp, + alignment slack
+    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * (NSTAGE + 1) * 8 + 1024;
     static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
     static_assert(BS % 16 == 0 && (D == 64 || D == 128), "whole 16-token slices");
     static_assert(G >= 1 && G <= 8, "heads are the 8 columns of N");
@@ -354,7 +357,7 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
     float2* __restrict__ ws_ml, int32_t* d_status, int32_t lpt_seqs,
     const T* __restrict__ new_key, const T* __restrict__ new_value, uint8_t* __restrict__ k_cache,
-    uint8_t* __restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv)
+    uint8_t* __restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv, uint32_t probe_us)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = Q8Shape<D, BS, G>;
@@ -396,10 +399,10 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     const int append_blk = (new_key != nullptr && part == nparts - 1) ? (ctx - 1) / BS - blk_begin : -1;
 
     unsigned char* wbase = smem + warp * S::WARP_BYTES;
-    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
+    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * (S::NSTAGE + 1);
     if (lane == 0) {
 #pragma unroll
-        for (int st = 0; st < S::NSTAGE; ++st) mbar_init(&wbar[st], 1);
+        for (int st = 0; st <= S::NSTAGE; ++st) mbar_init(&wbar[st], 1);   // + the probe barrier
         fence_barrier_init();
     }
     __syncwarp();
@@ -453,11 +456,11 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     w.reset();
     w.load_q(query, s, kvh, num_q_heads);
 
-    bool aborted = false;
+    bool aborted = nk > 0 && probe_gives_up(&wbar[S::NSTAGE], probe_us);
     int first_pending = 0;
-    for (int k = 0; k < nk; ++k) {
+    for (int k = 0; k < (aborted ? 0 : nk); ++k) {
         const int st = k % S::NSTAGE;
-        if (!mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1)) {
+        if (!mbar_wait_warp(&wbar[st], (k / S::NSTAGE) & 1)) {
             aborted = true;
             first_pending = k;
             break;
@@ -477,15 +480,13 @@ __device__ __forceinline__ void paged_decode_q8_cta(
         if (issued < nk) issue(issued++);
     }
 
-    if (aborted) {
-        if (lane == 0) status_or(d_status, PA_STATUS_TIMEOUT);
-        for (int k = first_pending; k < issued; ++k) {
-            const int st = k % S::NSTAGE;
-            mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1);
-        }
-    }
+    if (aborted) drain_after_timeout<S::NSTAGE>(wbar, first_pending, issued, d_status);
 
-    __syncthreads();   // every warp is done with its stage buffers
+    // every warp is done with its stage buffers, unless one gave up waiting
+    if (__syncthreads_or(aborted)) {
+        store_aborted_rows<T, D, G>(out, ws_o, ws_ml, s, kvh, part, nparts, num_q_heads, max_parts);
+        return;
+    }
     float* epi_o = reinterpret_cast<float*>(smem);   // [warp][g][D]
     float* epi_m = epi_o + kWarps * G * D;
     float* epi_l = epi_m + kWarps * G;
@@ -504,12 +505,13 @@ __device__ __forceinline__ void paged_decode_q8_cta(
         int32_t max_parts, float *__restrict__ ws_o, float2 *__restrict__ ws_ml,               \
         int32_t *d_status, int32_t lpt_seqs, const T *__restrict__ new_key,                    \
         const T *__restrict__ new_value, uint8_t *__restrict__ k_cache,                        \
-        uint8_t *__restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv
+        uint8_t *__restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv,          \
+        uint32_t probe_us
 #define PA_Q8_KERNEL_ARGS                                                                       \
     tm_k, tm_v, out, query, block_tables, context_lens, num_q_heads, max_blocks_per_seq,       \
         num_blocks, max_context_len, scale_log2, v_scale, partition_size, max_parts, ws_o,     \
         ws_ml, d_status, lpt_seqs, new_key, new_value, k_cache, v_cache, num_kv_heads, k_inv,  \
-        v_inv
+        v_inv, probe_us
 
 // e4m3 pools
 template <typename T, int D, int BS, int G>

@@ -20,6 +20,10 @@
 // its output rows directly; otherwise each part leaves (max, exp-sum,
 // normalised output) partials that a reduction merges with the rule of
 // §5.1.  So a private suffix costs no CTA of its own and no merge.
+#pragma once
+
+#include "decode_common.cuh"
+#include "paged_decode_mma.cuh"   // swz_offset, pack_pair
 
 namespace pa {
 
@@ -36,7 +40,8 @@ struct SharedShape {
     static constexpr int NSTAGE = 2;
     static constexpr int WARP_STAGE_BYTES = NSTAGE * STAGE_BYTES;
     static constexpr int OFF_BARS = kWarps * WARP_STAGE_BYTES;
-    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * NSTAGE * 8 + 1024;
+    // + a probe barrier per warp, + alignment slack
+    static constexpr int SMEM_BYTES = OFF_BARS + kWarps * (NSTAGE + 1) * 8 + 1024;
     static constexpr int EPI_BYTES = kWarps * kSharedRows * (D + 2) * 4;
     static_assert(BS % 16 == 0 && D % 64 == 0, "whole 16-token slices, 128-byte rows");
     static_assert(EPI_BYTES <= OFF_BARS, "epilogue fits in the stage buffers");
@@ -76,7 +81,7 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
     int32_t group_size, int32_t G, int32_t num_q_heads, int32_t max_blocks_per_seq,
     int64_t num_blocks, int32_t max_context_len, int32_t max_prefix_len, float scale_log2,
     int32_t part_blocks, int32_t max_parts, float* __restrict__ ws_o, float2* __restrict__ ws_ml,
-    int32_t* d_status)
+    int32_t* d_status, uint32_t probe_us)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
     using S = SharedShape<D, BS>;
@@ -124,10 +129,10 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
     const int nk = warp < nblk ? (nblk - warp + kWarps - 1) / kWarps : 0;
 
     unsigned char* wstage = smem + warp * S::WARP_STAGE_BYTES;
-    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * S::NSTAGE;
+    uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * (S::NSTAGE + 1);
     if (lane == 0) {
 #pragma unroll
-        for (int st = 0; st < S::NSTAGE; ++st) mbar_init(&wbar[st], 1);
+        for (int st = 0; st <= S::NSTAGE; ++st) mbar_init(&wbar[st], 1);   // + the probe barrier
         fence_barrier_init();
     }
     __syncwarp();
@@ -225,12 +230,12 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
 #pragma unroll
         for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
 
-    bool aborted = false;
+    bool aborted = nk > 0 && probe_gives_up(&wbar[S::NSTAGE], probe_us);
     int first_pending = 0;
 
-    for (int k = 0; k < nk; ++k) {
+    for (int k = 0; k < (aborted ? 0 : nk); ++k) {
         const int st = k % S::NSTAGE;
-        if (!mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1)) {
+        if (!mbar_wait_warp(&wbar[st], (k / S::NSTAGE) & 1)) {
             aborted = true;
             first_pending = k;
             break;
@@ -322,18 +327,31 @@ __global__ void __launch_bounds__(kThreads, 3) paged_decode_shared_kernel(
         if (issued < nk) issue(issued++);
     }
 
-    if (aborted) {
-        if (lane == 0) status_or(d_status, PA_STATUS_TIMEOUT);
-        for (int k = first_pending; k < issued; ++k) {
-            const int st = k % S::NSTAGE;
-            mbar_wait_bounded(&wbar[st], (k / S::NSTAGE) & 1);
-        }
-    }
+    if (aborted) drain_after_timeout<S::NSTAGE>(wbar, first_pending, issued, d_status);
 
     l_run += __shfl_xor_sync(kFullMask, l_run, 1);
     l_run += __shfl_xor_sync(kFullMask, l_run, 2);
 
-    __syncthreads();
+    // every warp is done with its stage buffers, unless one gave up waiting:
+    // then the group's rows get "nothing" through global memory only (zero
+    // rows, or an empty partial the reduction weighs with 0)
+    if (__syncthreads_or(aborted)) {
+        for (int idx = threadIdx.x; idx < rows * (D / 8); idx += kThreads) {
+            const int r = idx / (D / 8);
+            const int d0 = (idx % (D / 8)) * 8;
+            const int64_t row = static_cast<int64_t>(seq0 + r / G) * num_q_heads + kvh * G + r % G;
+            if (nparts == 1) {
+                *reinterpret_cast<uint4*>(out + row * D + d0) = make_uint4(0, 0, 0, 0);
+            } else {
+                const int64_t prow = row * max_parts + part;
+                float4* dst = reinterpret_cast<float4*>(ws_o + prow * D + d0);
+                dst[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                dst[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (d0 == 0) ws_ml[prow] = make_float2(-INFINITY, 0.f);
+            }
+        }
+        return;
+    }
     float* epi_o = reinterpret_cast<float*>(smem);                    // [warp][row][D]
     float* epi_m = epi_o + kWarps * kSharedRows * D;                  // [warp][row]
     float* epi_l = epi_m + kWarps * kSharedRows;

@@ -15,12 +15,20 @@ step then uses that format's quantising write and decode with the pools'
 scales.  ``run_from_host`` is the same step fed from pinned host buffers: it
 copies the step's inputs to the device, runs the step and copies the output
 back, all on the same stream.
+
+Tracing: every step and each of its calls is an NVTX range on the host
+thread that issues it ("pa.step", "pa.copy_blocks", "pa.cache_write",
+"pa.decode"; in ``HostPipeline`` also "pa.upload" and "pa.download"), so a
+timeline profiler shows which launches belong to which step.  Without a
+profiler attached the ranges cost a few hundred nanoseconds of host time.
 """
 from __future__ import annotations
 
 import torch
 
 from . import binding as B
+
+_range = torch.cuda.nvtx.range        # NVTX range on the issuing host thread
 
 
 # Pool dtype -> (cache write, decode, decode with fused write) of that code format.
@@ -64,35 +72,52 @@ class DecodeStep:
         new_value hold one row per sequence, at position context_lens - 1);
         the cache write then runs inside the decode launch
         (pa_paged_decode_append) and slot_mapping is not used."""
+        with _range("pa.step"):
+            return self._step(query, block_tables, context_lens, scale, out, new_key, new_value,
+                              slot_mapping, block_mapping, stream, max_context_len, fused_append)
+
+    def _step(self, query, block_tables, context_lens, scale, out, new_key, new_value,
+              slot_mapping, block_mapping, stream, max_context_len, fused_append):
         if block_mapping is not None and block_mapping.shape[0] > 0:
-            B.pa_copy_blocks(self.k_cache, self.v_cache, block_mapping, self.d_status, stream)
+            with _range("pa.copy_blocks"):
+                B.pa_copy_blocks(self.k_cache, self.v_cache, block_mapping, self.d_status, stream)
         if out is None:
             out = torch.empty_like(query)
         mcl = self.max_context_len if max_context_len is None else max_context_len
+        write_needed = slot_mapping is not None and slot_mapping.shape[0] > 0
         if self.quantised is not None:
             write, decode, decode_append = self.quantised
             if fused_append:
-                decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache,
-                              block_tables, context_lens, mcl, scale, self.k_scale, self.v_scale,
-                              self.partition_size, self.workspace, self.d_status, stream)
+                with _range("pa.decode"):
+                    decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache,
+                                  block_tables, context_lens, mcl, scale, self.k_scale,
+                                  self.v_scale, self.partition_size, self.workspace,
+                                  self.d_status, stream)
                 return out
-            if slot_mapping is not None and slot_mapping.shape[0] > 0:
-                write(new_key, new_value, self.k_cache, self.v_cache, slot_mapping, self.k_scale,
-                      self.v_scale, self.d_status, stream)
-            decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, mcl, scale,
-                   self.k_scale, self.v_scale, self.partition_size, self.workspace, self.d_status,
-                   stream)
+            if write_needed:
+                with _range("pa.cache_write"):
+                    write(new_key, new_value, self.k_cache, self.v_cache, slot_mapping,
+                          self.k_scale, self.v_scale, self.d_status, stream)
+            with _range("pa.decode"):
+                decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, mcl,
+                       scale, self.k_scale, self.v_scale, self.partition_size, self.workspace,
+                       self.d_status, stream)
             return out
         if fused_append:
-            B.pa_paged_decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache,
-                                     block_tables, context_lens, mcl, scale, self.partition_size,
-                                     self.workspace, self.d_status, stream)
+            with _range("pa.decode"):
+                B.pa_paged_decode_append(out, query, new_key, new_value, self.k_cache,
+                                         self.v_cache, block_tables, context_lens, mcl, scale,
+                                         self.partition_size, self.workspace, self.d_status,
+                                         stream)
             return out
-        if slot_mapping is not None and slot_mapping.shape[0] > 0:
-            B.pa_reshape_and_cache(new_key, new_value, self.k_cache, self.v_cache, slot_mapping,
-                                   self.d_status, stream)
-        B.pa_paged_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens, mcl,
-                          scale, self.partition_size, self.workspace, self.d_status, stream)
+        if write_needed:
+            with _range("pa.cache_write"):
+                B.pa_reshape_and_cache(new_key, new_value, self.k_cache, self.v_cache,
+                                       slot_mapping, self.d_status, stream)
+        with _range("pa.decode"):
+            B.pa_paged_decode(out, query, self.k_cache, self.v_cache, block_tables, context_lens,
+                              mcl, scale, self.partition_size, self.workspace, self.d_status,
+                              stream)
         return out
 
     def graph(self, query, block_tables, context_lens, scale, out, new_key=None, new_value=None,
@@ -208,7 +233,7 @@ class HostPipeline:
         if self.used[b]:
             self.up.wait_event(self.computed[b])        # the step that last read set b
             self.compute.wait_event(self.downloaded[b])  # its output has left set b's 'out'
-        with torch.cuda.stream(self.up):
+        with torch.cuda.stream(self.up), _range("pa.upload"):
             dev_buf.copy_(host_packed, non_blocking=True)
             self.uploaded[b].record(self.up)
         self.compute.wait_event(self.uploaded[b])
@@ -218,7 +243,7 @@ class HostPipeline:
                          slot_mapping=dev.get("slot_mapping"),
                          block_mapping=dev.get("block_mapping"), fused_append=fused_append)
         if graph is not None:
-            with torch.cuda.stream(self.compute):
+            with torch.cuda.stream(self.compute), _range("pa.step"):
                 graph.replay()
         else:
             self.stepper(dev["query"], dev["block_tables"], dev["context_lens"], scale,
@@ -233,7 +258,7 @@ class HostPipeline:
                                                       **step_args)
         self.computed[b].record(self.compute)
         self.down.wait_event(self.computed[b])
-        with torch.cuda.stream(self.down):
+        with torch.cuda.stream(self.down), _range("pa.download"):
             host_out.copy_(dev["out"], non_blocking=True)
             self.downloaded[b].record(self.down)
         self.used[b] = True

@@ -10,6 +10,7 @@
 
 #include "pa.h"
 #include "pa_block_manager.h"
+#include "pa_selftest.h"
 
 #define CHECK(n, cond)                                  \
     do {                                                \
@@ -37,6 +38,12 @@ int main(void)
                                        PA_DTYPE_F16, 0.5f, 0.5f, NULL, NULL) == PA_ERR_INVALID_ARG);
     CHECK(8, pa_swap_blocks(NULL, NULL, NULL, NULL, NULL, 1, 2, 64, 16, 8, 8, PA_DTYPE_INT8,
                             NULL, NULL) == PA_ERR_INVALID_ARG);
+
+    /* the test entry points refuse a missing status word or a limit of 0 */
+    CHECK(19, pa_selftest_bounded_wait(NULL, NULL, 1000, 1, NULL) == PA_ERR_INVALID_ARG);
+    CHECK(20, pa_selftest_decode_abort(NULL, NULL, NULL, NULL, NULL, NULL, 4, 2, 2, 64, 16, 4, 64,
+                                       40, 0.125f, 0, NULL, 0, PA_DTYPE_F16, PA_DTYPE_F16, 0, NULL,
+                                       NULL) == PA_ERR_INVALID_ARG);
 
     /* the block manager: allocation, copy-on-write, swap bookkeeping */
     pa_block_manager* bm = pa_bm_create(8, 4, 0);

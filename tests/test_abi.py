@@ -43,6 +43,60 @@ def test_library_exports_every_declared_symbol(pa):
     for name in names:
         assert hasattr(lib, name), f"libpa.so does not export {name}"
     assert set(_declared()) == set(pa.EXPORTS)
+    assert set(_declared(os.path.join(ROOT, "include", "pa_selftest.h"))) == set(pa.SELFTEST_EXPORTS)
+
+
+def test_no_alloc_scratch_size_matches_the_header(pa):
+    """The binding's PA_NO_ALLOC_WORKSPACE_BYTES is the header's #define."""
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+PA_NO_ALLOC_WORKSPACE_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
+    assert m, "PA_NO_ALLOC_WORKSPACE_BYTES not found in pa.h"
+    assert pa.PA_NO_ALLOC_WORKSPACE_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def _no_alloc(pa, **kw):
+    args = dict(out=FAKE, query=FAKE, k_cache=FAKE, v_cache=FAKE, block_tables=FAKE,
+                context_lens=FAKE, num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                block_size=16, max_blocks_per_seq=8, num_blocks=64, max_context_len=100,
+                scale=0.1, partition_size=0, dtype=0, d_status=None, stream=None)
+    args.update(kw)
+    return pa.LIB.pa_paged_decode_no_alloc(*args.values())
+
+
+def test_no_alloc_refuses_oversized_scratch_on_the_host(pa):
+    """A shape whose split-context scratch is larger than the library's
+    fixed array is refused (PA_ERR_INVALID_ARG) before anything is enqueued
+    or any device address is looked up; one just inside the limit gets past
+    that check (and fails on the null pointer instead)."""
+    s, hq, d = 64, 32, 128
+    need = pa.pa_paged_decode_workspace_size(s, hq, hq, d, 16, 8192, 16)
+    assert need > pa.PA_NO_ALLOC_WORKSPACE_BYTES
+    assert _no_alloc(pa, num_seqs=s, num_q_heads=hq, num_kv_heads=hq, max_context_len=8192,
+                     max_blocks_per_seq=512, partition_size=16) == pa.PA_ERR_INVALID_ARG
+    # the largest fitting context for one sequence of 8 query heads, 16-token partitions
+    per_part = 8 * (d + 2) * 4
+    fit = pa.PA_NO_ALLOC_WORKSPACE_BYTES // per_part * 16
+    assert pa.pa_paged_decode_workspace_size(1, 8, 2, d, 16, fit, 16) <= pa.PA_NO_ALLOC_WORKSPACE_BYTES
+    assert pa.pa_paged_decode_workspace_size(1, 8, 2, d, 16, fit + 16, 16) > pa.PA_NO_ALLOC_WORKSPACE_BYTES
+    assert _no_alloc(pa, num_seqs=1, max_context_len=fit + 16, partition_size=16) == pa.PA_ERR_INVALID_ARG
+    assert _no_alloc(pa, num_seqs=1, max_context_len=fit, partition_size=16, out=None) == pa.PA_ERR_INVALID_ARG
+
+
+def test_selftest_entry_points_check_their_arguments(pa):
+    """Refused on the host: a missing status word, a wait limit of 0 or
+    above 1 s, a grid outside 1..1024 CTAs, a key-value type that is neither
+    the query's nor a code type."""
+    B = pa
+    assert B.LIB.pa_selftest_bounded_wait(None, None, 1000, 1, None) == 1
+    assert B.LIB.pa_selftest_bounded_wait(FAKE, None, 0, 1, None) == 1
+    assert B.LIB.pa_selftest_bounded_wait(FAKE, None, 1000001, 1, None) == 1
+    assert B.LIB.pa_selftest_bounded_wait(FAKE, None, 1000, 0, None) == 1
+    assert B.LIB.pa_selftest_bounded_wait(FAKE, None, 1000, 1025, None) == 1
+    assert B.LIB.pa_selftest_bounded_wait(FAKE, FAKE + 4, 1000, 1, None) == 1
+    base = [FAKE] * 6 + [4, 8, 2, 128, 16, 8, 64, 100, 0.1, 0, None, 0, 0]
+    assert B.LIB.pa_selftest_decode_abort(*base, 0, 0, None, None) == 1          # limit 0
+    assert B.LIB.pa_selftest_decode_abort(*base, 0, 2000000, None, None) == 1    # limit > 1 s
+    assert B.LIB.pa_selftest_decode_abort(*base, 1, 1000, None, None) == 2       # bf16 pools, f16 query
 
 
 def test_status_strings(pa):

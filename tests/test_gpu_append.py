@@ -1,13 +1,11 @@
 """pa_paged_decode_append: the step's cache write fused into the decode
 launch.  The pools must equal the oracle's cache write bit for bit, and the
 output the oracle's attention (new tokens included)."""
-import math
 
 import numpy as np
 import pytest
 import torch
 
-import oracle
 from tests import oracle_pins
 from tests.gpu_utils import DeviceWorkload, assert_close, oracle_step, to_bits, to_f64
 from workloads import generators as gen
@@ -76,22 +74,17 @@ def test_append_bad_slot_is_flagged():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["llama7b", "mistral7b"])
-def test_append_full_size_sampled(name):
+@pytest.mark.parametrize("name", ["llama7b", "mistral7b", "long_context"])
+def test_append_full_size(name):
+    """The entry point the benchmark times, on the full workload in its
+    launch configuration: both whole pools bit for bit against the oracle's
+    cache write, and every output row against the full fp64 oracle."""
     wl = gen.CONFIGS[name]()
     dw = DeviceWorkload(wl)
-    out = _append(dw)
+    out = _append(dw, wl.partition_size)
     assert dw.status() == 0
-    kc, vc = oracle_pins.pool_after_step(wl)
-    b = wl.block_size
-    sl = wl.slot_mapping
-    got_k = to_bits(dw.k_cache)
-    assert np.array_equal(got_k[sl // b, sl % b], kc[sl // b, sl % b])
-    rng = np.random.Generator(np.random.PCG64(4))
-    rows = np.stack([rng.integers(0, wl.num_seqs, 48), rng.integers(0, wl.num_q_heads, 48)],
-                    axis=1).astype(np.int32)
-    ref, _ = oracle.paged_decode_rows(rows, wl.query, kc, vc, wl.block_tables, wl.context_lens,
-                                      wl.scale, wl.dtype)
-    got = to_f64(out)
-    assert np.all(np.isfinite(got))
-    assert_close(got[rows[:, 0], rows[:, 1]], ref, name)
+    kc, vc, ref, st = oracle_step(wl)
+    assert st == 0
+    assert np.array_equal(to_bits(dw.k_cache), kc), f"{name}: K pool differs"
+    assert np.array_equal(to_bits(dw.v_cache), vc), f"{name}: V pool differs"
+    assert_close(to_f64(out), ref, f"{name} fused append, every row")
