@@ -6,7 +6,7 @@ CPU-baseline leg of ``bench.py`` may import this package.  The product library
 
 ``pa_oracle.c`` holds the definitions (reshape_and_cache, copy_blocks,
 swap_blocks, paged decode in fp64; the e4m3 and int8 pools' encode, write and
-decode); this module compiles it with gcc (``-O2``, OpenMP, no
+decode, with one scale per pool or one per (token, kv head) row); this module compiles it with gcc (``-O2``, OpenMP, no
 fast-math) into ``liboracle.so`` beside it and wraps it with ctypes.
 ``brute.py`` holds pure-Python/numpy restatements used to pin it.
 
@@ -84,6 +84,13 @@ def load(path: str | None = None):
     lib.oracle_paged_decode_int8.argtypes = [p, p, p, p, p, p, i32, i32, i32, i32, i32, i32,
                                              i64, f64, i32, f64, f64, i32]
     lib.oracle_paged_decode_int8.restype = i32
+    for fmt in ("fp8", "int8"):
+        w = getattr(lib, f"oracle_reshape_and_cache_{fmt}_rowscale")
+        w.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i64, i32]
+        w.restype = i32
+        dcd = getattr(lib, f"oracle_paged_decode_{fmt}_rowscale")
+        dcd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64, f64, i32, i32]
+        dcd.restype = i32
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
     if path is None:
@@ -141,6 +148,11 @@ def copy_blocks(k_cache, v_cache, block_mapping, lib=None) -> int:
     if k_cache.dtype.itemsize == 1:
         assert k_cache.shape[-1] % 2 == 0, "one-byte pools copy as byte pairs"
         k_cache, v_cache = k_cache.view(np.uint16), v_cache.view(np.uint16)
+    elif k_cache.dtype == np.float32:
+        # row-scale pools [num_blocks][Hkv][B]: a block is Hkv * B scales, copied as 16-bit pairs
+        nb = k_cache.shape[0]
+        k_cache = k_cache.view(np.uint16).reshape(nb, 1, 1, -1)
+        v_cache = v_cache.view(np.uint16).reshape(nb, 1, 1, -1)
     assert k_cache.dtype.itemsize == 2, f"16-bit or one-byte pools, got {k_cache.dtype}"
     num_blocks, bs, hkv, d = k_cache.shape
     return int((lib or load()).oracle_copy_blocks(
@@ -154,6 +166,9 @@ def swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, lib=None) -> int:
     pools of any one element type, [num_blocks][B][Hkv][D])."""
     block_mapping = np.ascontiguousarray(block_mapping, dtype=np.int64).reshape(-1, 2)
     assert src_k.dtype == dst_k.dtype and src_k.shape[1:] == dst_k.shape[1:]
+    if src_k.ndim == 3:                  # row-scale pools [num_blocks][Hkv][B]: bytes of a block
+        src_k, src_v, dst_k, dst_v = (a.reshape(a.shape[0], 1, 1, -1)
+                                      for a in (src_k, src_v, dst_k, dst_v))
     for a in (src_k, src_v, dst_k, dst_v):
         assert a.flags["C_CONTIGUOUS"]
     src_nb, bs, hkv, d = src_k.shape
@@ -300,3 +315,74 @@ def paged_decode_int8(query, k_cache, v_cache, block_tables, context_lens, scale
     return _paged_decode_q8((lib or load()).oracle_paged_decode_int8, query, k_cache, v_cache,
                             block_tables, context_lens, scale, dtype, k_scale, v_scale,
                             num_threads)
+
+
+# ---- Row-scaled one-byte caches: one fp32 scale per (token, kv head) row ------
+
+def _scale_pool(a: np.ndarray, num_blocks: int, num_kv_heads: int, block_size: int) -> np.ndarray:
+    assert a.dtype == np.float32 and a.flags["C_CONTIGUOUS"], "scale pools are float32, contiguous"
+    assert a.shape == (num_blocks, num_kv_heads, block_size), a.shape
+    return a
+
+
+def _reshape_and_cache_rowscale(fmt, key, value, k_cache, v_cache, k_scales, v_scales,
+                                slot_mapping, block_size, dtype, lib):
+    key, value = _u16(key), _u16(value)
+    assert k_cache.dtype in (np.uint8, np.int8) and v_cache.dtype == k_cache.dtype
+    assert k_cache.flags["C_CONTIGUOUS"] and v_cache.flags["C_CONTIGUOUS"]
+    slot_mapping = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    num_blocks, bs, hkv, d = k_cache.shape
+    assert bs == block_size
+    _scale_pool(k_scales, num_blocks, hkv, bs)
+    _scale_pool(v_scales, num_blocks, hkv, bs)
+    fn = getattr(lib or load(), f"oracle_reshape_and_cache_{fmt}_rowscale")
+    return int(fn(_ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales),
+                  _ptr(v_scales), _ptr(slot_mapping), key.shape[0], hkv, d, block_size,
+                  num_blocks, _DTYPES[dtype]))
+
+
+def _paged_decode_rowscale(fmt, query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                           context_lens, scale, dtype, num_threads, lib):
+    query = _u16(query)
+    block_tables = np.ascontiguousarray(block_tables, dtype=np.int32)
+    context_lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    s, hq, d = query.shape
+    num_blocks, bs, hkv, _ = k_cache.shape
+    _scale_pool(k_scales, num_blocks, hkv, bs)
+    _scale_pool(v_scales, num_blocks, hkv, bs)
+    out = np.empty((s, hq, d), dtype=np.float64)
+    fn = getattr(lib or load(), f"oracle_paged_decode_{fmt}_rowscale")
+    st = fn(_ptr(out), _ptr(query), _ptr(_code_bytes(k_cache)), _ptr(_code_bytes(v_cache)),
+            _ptr(k_scales), _ptr(v_scales), _ptr(block_tables), _ptr(context_lens), s, hq, hkv,
+            d, bs, block_tables.shape[1], num_blocks, float(scale), _DTYPES[dtype], num_threads)
+    return out, int(st)
+
+
+def reshape_and_cache_fp8_rowscale(key, value, k_cache, v_cache, k_scales, v_scales,
+                                   slot_mapping, block_size, dtype, lib=None) -> int:
+    """Quantising cache write into uint8 e4m3 pools [num_blocks][B][Hkv][D]
+    with one fp32 scale per row in k_scales / v_scales [num_blocks][Hkv][B]:
+    s = fp32(max |x| / 448), code = e4m3(fp32(x * fp32(1 / s)))."""
+    return _reshape_and_cache_rowscale("fp8", key, value, k_cache, v_cache, k_scales, v_scales,
+                                       slot_mapping, block_size, dtype, lib)
+
+
+def reshape_and_cache_int8_rowscale(key, value, k_cache, v_cache, k_scales, v_scales,
+                                    slot_mapping, block_size, dtype, lib=None) -> int:
+    """As reshape_and_cache_fp8_rowscale for int8 pools: s = fp32(max |x| / 127)."""
+    return _reshape_and_cache_rowscale("int8", key, value, k_cache, v_cache, k_scales, v_scales,
+                                       slot_mapping, block_size, dtype, lib)
+
+
+def paged_decode_fp8_rowscale(query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                              context_lens, scale, dtype, num_threads=0, lib=None):
+    """fp64 paged decode over e4m3 pools, each row dequantised with its own scale."""
+    return _paged_decode_rowscale("fp8", query, k_cache, v_cache, k_scales, v_scales,
+                                  block_tables, context_lens, scale, dtype, num_threads, lib)
+
+
+def paged_decode_int8_rowscale(query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                               context_lens, scale, dtype, num_threads=0, lib=None):
+    """fp64 paged decode over int8 pools, each row dequantised with its own scale."""
+    return _paged_decode_rowscale("int8", query, k_cache, v_cache, k_scales, v_scales,
+                                  block_tables, context_lens, scale, dtype, num_threads, lib)

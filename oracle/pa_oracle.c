@@ -35,6 +35,7 @@
  *       (the output row is written as zeros)
  *   8 = copy_blocks: a destination written twice, or also used as a source
  */
+#include <float.h>
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -234,6 +235,100 @@ int32_t oracle_reshape_and_cache_int8(const uint16_t* key, const uint16_t* value
     return reshape_and_cache_q8(key, value, k_cache, v_cache, slot_mapping, num_tokens,
                                 num_kv_heads, head_dim, block_size, num_blocks, dtype, k_scale,
                                 v_scale, f32_to_int8);
+}
+
+/* ------------------------------------------------------------------------
+ * Row-scaled one-byte pools: every (token, kv head) row of K, and of V, has
+ * a scale of its own instead of one per pool.  The scales sit in pools of
+ * fp32 values beside the codes,
+ *   k_scales, v_scales : [num_blocks][num_kv_heads][block_size],
+ * so the cached value of element d of the row of slot `slot`, kv head g, is
+ *   dec(code) * scales[slot / block_size][g][slot % block_size].
+ * The pages name FP8/INT8 storage of the cached blocks ("PagedAttention：
+ * 大模型KV Cache分页管理优化实践" §7, item 2; "vLLM用虚拟内存分页思想管理KV
+ * Cache", 工程实践与局限) and fix no scale granularity; this is the reading
+ * in which a row is quantised once, when it is written, and never again.
+ *
+ * The write takes each row's scale from the row itself:
+ *   amax   = max_d |x_d|              (x_d: the exact fp32 value of the input)
+ *   s      = fp32(amax / code_max)    (code_max 448 for e4m3, 127 for int8)
+ *   code_d = encode(fp32(x_d * fp32(1 / s)))   -- the per-pool write with
+ *            scale s, so the row's largest element takes the top code;
+ * a row with s below the smallest normal fp32 (all zeros, or values below
+ * about 1e-35) stores s = 0 and every code 0.
+ * ---------------------------------------------------------------------- */
+static void quantise_row(const uint16_t* x16, int32_t head_dim, int32_t dtype, float code_max,
+                         uint8_t (*encode)(float), uint8_t* codes, float* scale)
+{
+    float amax = 0.0f;
+    for (int32_t d = 0; d < head_dim; ++d) {
+        const float a = fabsf((float)decode(x16[d], dtype));
+        if (a > amax) amax = a;
+    }
+    const float s = amax / code_max;
+    if (!(s >= FLT_MIN)) {
+        for (int32_t d = 0; d < head_dim; ++d) codes[d] = 0;
+        *scale = 0.0f;
+        return;
+    }
+    const float inv = 1.0f / s;
+    for (int32_t d = 0; d < head_dim; ++d) {
+        const float x = (float)decode(x16[d], dtype);
+        const float xq = x * inv;
+        codes[d] = encode(xq);
+    }
+    *scale = s;
+}
+
+static int32_t reshape_and_cache_q8_rowscale(const uint16_t* key, const uint16_t* value,
+                                             uint8_t* k_cache, uint8_t* v_cache, float* k_scales,
+                                             float* v_scales, const int64_t* slot_mapping,
+                                             int32_t num_tokens, int32_t num_kv_heads,
+                                             int32_t head_dim, int32_t block_size,
+                                             int64_t num_blocks, int32_t dtype, float code_max,
+                                             uint8_t (*encode)(float))
+{
+    int32_t status = 0;
+    for (int32_t t = 0; t < num_tokens; ++t) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0) continue;
+        if (slot >= num_blocks * (int64_t)block_size) { status |= 2; continue; }
+        const int64_t blk = slot / block_size, off = slot % block_size;
+        for (int32_t g = 0; g < num_kv_heads; ++g) {
+            const int64_t src = ((int64_t)t * num_kv_heads + g) * head_dim;
+            const int64_t dst = (slot * num_kv_heads + g) * head_dim;
+            const int64_t si = (blk * num_kv_heads + g) * block_size + off;
+            quantise_row(key + src, head_dim, dtype, code_max, encode, k_cache + dst, &k_scales[si]);
+            quantise_row(value + src, head_dim, dtype, code_max, encode, v_cache + dst,
+                         &v_scales[si]);
+        }
+    }
+    return status;
+}
+
+int32_t oracle_reshape_and_cache_fp8_rowscale(const uint16_t* key, const uint16_t* value,
+                                              uint8_t* k_cache, uint8_t* v_cache, float* k_scales,
+                                              float* v_scales, const int64_t* slot_mapping,
+                                              int32_t num_tokens, int32_t num_kv_heads,
+                                              int32_t head_dim, int32_t block_size,
+                                              int64_t num_blocks, int32_t dtype)
+{
+    return reshape_and_cache_q8_rowscale(key, value, k_cache, v_cache, k_scales, v_scales,
+                                         slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                         block_size, num_blocks, dtype, 448.0f, f32_to_e4m3);
+}
+
+int32_t oracle_reshape_and_cache_int8_rowscale(const uint16_t* key, const uint16_t* value,
+                                               uint8_t* k_cache, uint8_t* v_cache,
+                                               float* k_scales, float* v_scales,
+                                               const int64_t* slot_mapping, int32_t num_tokens,
+                                               int32_t num_kv_heads, int32_t head_dim,
+                                               int32_t block_size, int64_t num_blocks,
+                                               int32_t dtype)
+{
+    return reshape_and_cache_q8_rowscale(key, value, k_cache, v_cache, k_scales, v_scales,
+                                         slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                         block_size, num_blocks, dtype, 127.0f, f32_to_int8);
 }
 
 /* ------------------------------------------------------------------------
@@ -439,16 +534,30 @@ static int32_t decode_row(double* out, const uint16_t* query, const uint16_t* k_
     return status;
 }
 
+/* The scale of the row at element offset r of a row-scaled pool: row
+ * r / head_dim is slot * num_kv_heads + g, and its scale sits at
+ * [slot / block_size][g][slot % block_size] of the scale pool. */
+static double row_scale(const float* scales, int64_t r, int32_t num_kv_heads, int32_t head_dim,
+                        int32_t block_size)
+{
+    const int64_t row = r / head_dim;
+    const int64_t slot = row / num_kv_heads, g = row % num_kv_heads;
+    return (double)scales[((slot / block_size) * num_kv_heads + g) * block_size + slot % block_size];
+}
+
 /* Paged decode over 8-bit pools (e4m3 or int8 codes): every cached element
  * is dequantised, K = dec(code) * k_scale, V = dec(code) * v_scale, in
  * double, and the attention is the direct form of decode_row.  Query and
- * output as in oracle_paged_decode (query bits of `dtype`). */
+ * output as in oracle_paged_decode (query bits of `dtype`).  With row-scale
+ * pools (k_scales / v_scales not NULL) each row's own scale replaces the
+ * pool's. */
 static int32_t decode_row_q8(double* out, const uint16_t* query, const uint8_t* k_cache,
                              const uint8_t* v_cache, const int32_t* block_tables,
                              const int32_t* context_lens, int32_t s, int32_t h,
                              int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                              int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
                              double scale, int32_t dtype, double k_scale, double v_scale,
+                             const float* k_scales, const float* v_scales,
                              double (*dec)(uint8_t))
 {
     int32_t status = 0;
@@ -469,8 +578,10 @@ static int32_t decode_row_q8(double* out, const uint16_t* query, const uint8_t* 
         int64_t r = token_row(table, t, g, num_kv_heads, head_dim, block_size, num_blocks);
         valid[t] = r >= 0;
         if (r < 0) { status |= 1; x[t] = 0.0; continue; }
+        const double ks = k_scales ? row_scale(k_scales, r, num_kv_heads, head_dim, block_size)
+                                   : k_scale;
         double acc = 0.0;
-        for (int32_t d = 0; d < head_dim; ++d) acc += q[d] * (dec(k_cache[r + d]) * k_scale);
+        for (int32_t d = 0; d < head_dim; ++d) acc += q[d] * (dec(k_cache[r + d]) * ks);
         x[t] = scale * acc;
         any = 1;
     }
@@ -482,8 +593,10 @@ static int32_t decode_row_q8(double* out, const uint16_t* query, const uint8_t* 
             if (!valid[t]) continue;
             double w = exp(x[t] - m) / l;
             int64_t r = token_row(table, t, g, num_kv_heads, head_dim, block_size, num_blocks);
+            const double vs = v_scales ? row_scale(v_scales, r, num_kv_heads, head_dim, block_size)
+                                       : v_scale;
             for (int32_t d = 0; d < head_dim; ++d)
-                out[d] += w * (dec(v_cache[r + d]) * v_scale);
+                out[d] += w * (dec(v_cache[r + d]) * vs);
         }
     }
     free(q); free(x); free(valid);
@@ -559,7 +672,8 @@ static int32_t paged_decode_q8(double* out, const uint16_t* query, const uint8_t
                                int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                                int32_t block_size, int32_t max_blocks_per_seq,
                                int64_t num_blocks, double scale, int32_t dtype, double k_scale,
-                               double v_scale, int32_t num_threads, double (*dec)(uint8_t))
+                               double v_scale, const float* k_scales, const float* v_scales,
+                               int32_t num_threads, double (*dec)(uint8_t))
 {
     int32_t status = 0;
     const int64_t rows = (int64_t)num_seqs * num_q_heads;
@@ -570,7 +684,7 @@ static int32_t paged_decode_q8(double* out, const uint16_t* query, const uint8_t
         status |= decode_row_q8(out + r * head_dim, query, k_cache, v_cache, block_tables,
                                 context_lens, s, h, num_q_heads, num_kv_heads, head_dim,
                                 block_size, max_blocks_per_seq, num_blocks, scale, dtype,
-                                k_scale, v_scale, dec);
+                                k_scale, v_scale, k_scales, v_scales, dec);
     }
     return status;
 }
@@ -585,7 +699,8 @@ int32_t oracle_paged_decode_fp8(double* out, const uint16_t* query, const uint8_
 {
     return paged_decode_q8(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
                            num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
-                           num_blocks, scale, dtype, k_scale, v_scale, num_threads, e4m3_to_f64);
+                           num_blocks, scale, dtype, k_scale, v_scale, NULL, NULL, num_threads,
+                           e4m3_to_f64);
 }
 
 int32_t oracle_paged_decode_int8(double* out, const uint16_t* query, const uint8_t* k_cache,
@@ -598,5 +713,40 @@ int32_t oracle_paged_decode_int8(double* out, const uint16_t* query, const uint8
 {
     return paged_decode_q8(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
                            num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
-                           num_blocks, scale, dtype, k_scale, v_scale, num_threads, int8_to_f64);
+                           num_blocks, scale, dtype, k_scale, v_scale, NULL, NULL, num_threads,
+                           int8_to_f64);
+}
+
+/* Paged decode over row-scaled one-byte pools (scale pools as for the
+ * _rowscale write above): each cached row dequantised with its own scale. */
+int32_t oracle_paged_decode_fp8_rowscale(double* out, const uint16_t* query,
+                                         const uint8_t* k_cache, const uint8_t* v_cache,
+                                         const float* k_scales, const float* v_scales,
+                                         const int32_t* block_tables, const int32_t* context_lens,
+                                         int32_t num_seqs, int32_t num_q_heads,
+                                         int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t block_size, int32_t max_blocks_per_seq,
+                                         int64_t num_blocks, double scale, int32_t dtype,
+                                         int32_t num_threads)
+{
+    return paged_decode_q8(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, scale, dtype, 1.0, 1.0, k_scales, v_scales, num_threads,
+                           e4m3_to_f64);
+}
+
+int32_t oracle_paged_decode_int8_rowscale(double* out, const uint16_t* query,
+                                          const uint8_t* k_cache, const uint8_t* v_cache,
+                                          const float* k_scales, const float* v_scales,
+                                          const int32_t* block_tables, const int32_t* context_lens,
+                                          int32_t num_seqs, int32_t num_q_heads,
+                                          int32_t num_kv_heads, int32_t head_dim,
+                                          int32_t block_size, int32_t max_blocks_per_seq,
+                                          int64_t num_blocks, double scale, int32_t dtype,
+                                          int32_t num_threads)
+{
+    return paged_decode_q8(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, scale, dtype, 1.0, 1.0, k_scales, v_scales, num_threads,
+                           int8_to_f64);
 }

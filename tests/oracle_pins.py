@@ -614,4 +614,181 @@ def pin_swap_bytes_of_fp8_pools(lib):
     assert np.array_equal(dst_k, before)
 
 
+# ---- Row-scaled one-byte caches: one fp32 scale per (token, kv head) row ---------
+
+_CODE_MAX = {"fp8": 448.0, "int8": 127.0}
+
+
+def _dec_codes(codes, fmt):
+    """Codes -> float64 with torch's e4m3 decoding or numpy's int8 view."""
+    if fmt == "int8":
+        return np.ascontiguousarray(codes).view(np.int8).astype(np.float64)
+    torch = _torch_e4m3()
+    return (torch.from_numpy(np.ascontiguousarray(codes).view(np.uint8))
+            .view(torch.float8_e4m3fn).to(torch.float64).numpy())
+
+
+def _rows_of_mixed_magnitude(rng, t, h, d, dtype="f16"):
+    """[t][h][d] 16-bit values whose kv heads differ in magnitude by up to
+    10^4 (x1, x0.01, x100, ...), with one all-zero row."""
+    mags = np.array([1.0, 0.01, 100.0, 3.0])[:h].astype(np.float32)
+    x = rng.standard_normal((t, h, d)).astype(np.float32) * mags[None, :, None]
+    x[-1, 1 % h] = 0.0
+    return gen.f32_to_bits(x, dtype)
+
+
+def pin_rowscale_cache_write(lib):
+    """The row-scaled write, both code formats: each written row's scale is
+    fp32(max |x| / code_max); its codes are those of the (pinned) per-pool
+    write with that scale; its largest element takes the top code; the
+    dequantised row is within half a code step of the input; an all-zero
+    row stores scale 0 and zero codes; a slot past the pool sets bit 2;
+    every other code and scale byte is unchanged."""
+    rng = np.random.Generator(np.random.PCG64(31))
+    nb, b, h, d = 6, 4, 3, 16
+    for fmt in ("fp8", "int8"):
+        np_t = np.uint8 if fmt == "fp8" else np.int8
+        write = getattr(oracle, f"reshape_and_cache_{fmt}_rowscale")
+        pool_write = getattr(oracle, f"reshape_and_cache_{fmt}")
+        poison = np.array(0x7f, np.uint8).view(np_t)
+        kc = np.full((nb, b, h, d), poison, np_t)
+        vc = kc.copy()
+        ks = np.full((nb, h, b), -7.0, np.float32)
+        vs = ks.copy()
+        key = _rows_of_mixed_magnitude(rng, 4, h, d)
+        val = _rows_of_mixed_magnitude(rng, 4, h, d)
+        slots = np.array([5, -1, 17, 22])
+        st = write(key, val, kc, vc, ks, vs, slots, b, "f16", lib=lib)
+        assert st == 0
+        assert write(key[:1], val[:1], kc.copy(), vc.copy(), ks.copy(), vs.copy(),
+                     np.array([nb * b]), b, "f16", lib=lib) == 2
+        top = _CODE_MAX[fmt]
+        for t, sl in ((0, 5), (2, 17), (3, 22)):
+            blk, off = sl // b, sl % b
+            for src, pool, scales in ((key, kc, ks), (val, vc, vs)):
+                for g in range(h):
+                    x = src[t, g].view(np.float16).astype(np.float32)
+                    s = scales[blk, g, off]
+                    amax = np.float32(np.max(np.abs(x)))
+                    if amax == 0:
+                        assert s == 0 and not pool[blk, off, g].view(np.uint8).any()
+                        continue
+                    assert s == amax / np.float32(top), (fmt, t, g)
+                    one = np.full((1, 1, 1, d), poison, np_t)
+                    pool_write(src[t:t + 1, g:g + 1], src[t:t + 1, g:g + 1], one, one.copy(),
+                               np.array([0]), 1, "f16", float(s), float(s), lib=lib)
+                    assert np.array_equal(pool[blk, off, g], one[0, 0, 0]), (fmt, t, g)
+                    deq = _dec_codes(pool[blk, off, g], fmt) * float(s)
+                    assert abs(deq[np.argmax(np.abs(x))]) == top * float(s)
+                    step = float(s) * (1.0 if fmt == "int8" else 2.0 ** -9)
+                    rel = 0.0 if fmt == "int8" else 2.0 ** -4
+                    bound = step / 2 + rel * np.abs(x) + 1e-6 * np.abs(x)
+                    assert np.all(np.abs(deq - x) <= bound), (fmt, t, g)
+        touched = np.zeros((nb, b), bool)
+        for sl in (5, 17, 22):
+            touched[sl // b, sl % b] = True
+        assert np.all(kc[~touched].view(np.uint8) == 0x7f)
+        assert np.all(vc[~touched].view(np.uint8) == 0x7f)
+        untouched = np.ones((nb, h, b), bool)
+        for sl in (5, 17, 22):
+            untouched[sl // b, :, sl % b] = False
+        assert np.all(ks[untouched] == -7.0) and np.all(vs[untouched] == -7.0)
+
+
+def _random_rowscale_pools(rng, wl, fmt):
+    """Random codes (no NaN) and positive row scales spanning four orders of
+    magnitude across kv heads."""
+    shape = wl.k_cache.shape
+    pools = []
+    for _ in range(2):
+        c = rng.integers(0, 256, size=shape).astype(np.uint8)
+        if fmt == "fp8":
+            c[(c & 0x7f) == 0x7f] = 0x35
+        pools.append(c.view(np.uint8 if fmt == "fp8" else np.int8))
+    nb, b, h, _ = shape
+    mags = np.geomspace(1e-2, 1e2, h).astype(np.float32)
+    scales = [(rng.uniform(0.5, 2.0, (nb, h, b)).astype(np.float32) * mags[None, :, None]
+               / np.float32(_CODE_MAX[fmt])).astype(np.float32) for _ in range(2)]
+    return pools, scales
+
+
+def pin_rowscale_decode_matches_numpy_attention(lib):
+    """Row-scaled decode, both formats: numpy softmax attention over K/V
+    gathered through the tables, each row dequantised with its own scale
+    from [block][kv head][offset] (<= 1e-12)."""
+    from scipy.special import softmax
+    rng = np.random.Generator(np.random.PCG64(32))
+    for fmt in ("fp8", "int8"):
+        wl = small_gqa(dtype="bf16", seqs=4, head_dim=64)
+        (kc, vc), (ks, vs) = _random_rowscale_pools(rng, wl, fmt)
+        decode = getattr(oracle, f"paged_decode_{fmt}_rowscale")
+        got, st = decode(wl.query, kc, vc, ks, vs, wl.block_tables, wl.context_lens, wl.scale,
+                         wl.dtype, lib=lib)
+        assert st == 0
+        q = oracle.decode_bits(wl.query, "bf16", lib=lib)
+        b, group = wl.block_size, wl.num_q_heads // wl.num_kv_heads
+        for s in range(wl.num_seqs):
+            c = int(wl.context_lens[s])
+            pos = np.arange(c)
+            phys = wl.block_tables[s][pos // b]
+            k = _dec_codes(kc[phys, pos % b], fmt) * ks[phys, :, pos % b][:, :, None]
+            v = _dec_codes(vc[phys, pos % b], fmt) * vs[phys, :, pos % b][:, :, None]
+            k, v = np.repeat(k, group, axis=1), np.repeat(v, group, axis=1)
+            w = softmax(wl.scale * np.einsum("hd,thd->ht", q[s], k), axis=1)
+            close(got[s], np.einsum("ht,thd->hd", w, v), 1e-12)
+
+
+def pin_rowscale_constant_scales_equal_pool_scales(lib):
+    """Scale pools holding one value everywhere give exactly the (pinned)
+    per-pool decode with that scale, and the row-scaled write of rows whose
+    scales all come out equal gives the per-pool write's codes."""
+    rng = np.random.Generator(np.random.PCG64(33))
+    for fmt in ("fp8", "int8"):
+        wl = small_gqa(dtype="f16")
+        (kc, vc), _ = _random_rowscale_pools(rng, wl, fmt)
+        nb, b, h, _ = kc.shape
+        ks = np.full((nb, h, b), 0.0371, np.float32)
+        vs = np.full((nb, h, b), 0.2113, np.float32)
+        a, sa = getattr(oracle, f"paged_decode_{fmt}_rowscale")(
+            wl.query, kc, vc, ks, vs, wl.block_tables, wl.context_lens, wl.scale, "f16", lib=lib)
+        p, sp = getattr(oracle, f"paged_decode_{fmt}")(
+            wl.query, kc, vc, wl.block_tables, wl.context_lens, wl.scale, "f16",
+            float(ks[0, 0, 0]), float(vs[0, 0, 0]), lib=lib)
+        assert sa == sp == 0 and np.array_equal(a, p)
+
+
+def pin_rowscale_permutation_invariance(lib):
+    """Relabelling physical blocks -- codes and scales moved together, tables
+    remapped -- leaves the row-scaled decode bit-identical."""
+    rng = np.random.Generator(np.random.PCG64(34))
+    for fmt in ("fp8", "int8"):
+        wl = small_gqa(dtype="bf16")
+        (kc, vc), (ks, vs) = _random_rowscale_pools(rng, wl, fmt)
+        decode = getattr(oracle, f"paged_decode_{fmt}_rowscale")
+        a, _ = decode(wl.query, kc, vc, ks, vs, wl.block_tables, wl.context_lens, wl.scale,
+                      wl.dtype, lib=lib)
+        perm = rng.permutation(kc.shape[0])            # new id of old block i is perm[i]
+        inv = np.argsort(perm)
+        tables = np.where(wl.block_tables >= 0, perm[np.maximum(wl.block_tables, 0)], -1)
+        moved = [np.ascontiguousarray(x[inv]) for x in (kc, vc, ks, vs)]
+        b2, _ = decode(wl.query, *moved, tables.astype(np.int32), wl.context_lens, wl.scale,
+                       wl.dtype, lib=lib)
+        assert np.array_equal(a, b2)
+
+
+def pin_rowscale_pools_copy_and_swap_as_blocks(lib):
+    """Scale pools move with their blocks: copy_blocks and swap_blocks on a
+    [num_blocks][Hkv][B] fp32 pool copy whole blocks of scales."""
+    rng = np.random.Generator(np.random.PCG64(35))
+    ks = rng.uniform(0, 1, (6, 3, 4)).astype(np.float32)
+    vs = rng.uniform(0, 1, (6, 3, 4)).astype(np.float32)
+    k0, v0 = ks.copy(), vs.copy()
+    assert oracle.copy_blocks(ks, vs, np.array([[1, 4], [2, 5]]), lib=lib) == 0
+    assert np.array_equal(ks[4], k0[1]) and np.array_equal(vs[5], v0[2])
+    assert np.array_equal(ks[:4], k0[:4])
+    hk, hv = np.zeros((2, 3, 4), np.float32), np.zeros((2, 3, 4), np.float32)
+    assert oracle.swap_blocks(ks, vs, hk, hv, np.array([[3, 1]]), lib=lib) == 0
+    assert np.array_equal(hk[1], ks[3]) and np.array_equal(hv[1], vs[3]) and not hk[0].any()
+
+
 PINS = {name: fn for name, fn in globals().items() if name.startswith("pin_")}

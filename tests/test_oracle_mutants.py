@@ -37,14 +37,14 @@ MUTANTS = {
     "e4m3_ties_away": ("else pick = (lo & 1) ? hi : lo;", "else pick = hi;"),
     "e4m3_no_saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7e);",
                            "if (a >= 448.0) return (uint8_t)(sign | 0x7f);"),
-    "fp8_scale_dropped": ("(dec(k_cache[r + d]) * k_scale)", "(dec(k_cache[r + d]))"),
+    "fp8_scale_dropped": ("(dec(k_cache[r + d]) * ks)", "(dec(k_cache[r + d]))"),
     "fp8_write_divides_twice": ("const float kq = kx * k_inv;", "const float kq = kx * k_inv * k_inv;"),
     "swap_only_k": ("dst_v[dst * block_bytes + b] = src_v[src * block_bytes + b];", ""),
     "swap_dst_index_of_src": ("dst_k[dst * block_bytes + b] = src_k[src * block_bytes + b];",
                               "dst_k[src % dst_num_blocks * block_bytes + b] = src_k[src * block_bytes + b];"),
     "swap_bad_id_not_flagged": ("            status |= 1;\n            continue;", "            continue;"),
-    "fp8_v_scaled_by_k_scale": ("(dec(v_cache[r + d]) * v_scale)",
-                                "(dec(v_cache[r + d]) * k_scale)"),
+    "fp8_v_scaled_by_k_scale": ("                                       : v_scale;",
+                                "                                       : k_scale;"),
     "e4m3_subnormal_scale": ("v = ldexp((double)frac, -9);", "v = ldexp((double)frac, -10);"),
     "e4m3_nan_whole_top_binade": ("if (expo == 15 && frac == 7)", "if (expo == 15)"),
     "f16_subnormal_scale": ("v = ldexp((double)frac, -24);", "v = ldexp((double)frac, -25);"),
@@ -60,9 +60,24 @@ MUTANTS = {
     "int8_ties_away": ("else r = fmod(lo, 2.0) == 0.0 ? lo : lo + 1.0;", "else r = lo + 1.0;"),
     "int8_wraps_past_127": ("if (x >= 127.0f) return 127;", "if (x >= 128.0f) return 127;"),
     "int8_nan_saturates": ("if (x != x) return 0;", "if (x != x) return 127;"),
-    "int8_decodes_as_e4m3": ("num_blocks, scale, dtype, k_scale, v_scale, num_threads, int8_to_f64);",
-                             "num_blocks, scale, dtype, k_scale, v_scale, num_threads, e4m3_to_f64);"),
+    "int8_decodes_as_e4m3": ("k_scale, v_scale, NULL, NULL, num_threads,\n                           int8_to_f64);",
+                             "k_scale, v_scale, NULL, NULL, num_threads,\n                           e4m3_to_f64);"),
     "int8_write_uses_e4m3": ("v_scale, f32_to_int8);", "v_scale, f32_to_e4m3);"),
+    # row-scaled one-byte pools
+    "rowscale_neighbour_row": ("* block_size + slot % block_size];",
+                               "* block_size + (slot + 1) % block_size];"),
+    "rowscale_one_scale_for_all_rows": ("row_scale(k_scales, r, num_kv_heads", "row_scale(k_scales, 0, num_kv_heads"),
+    "rowscale_token_major_scales": ("((slot / block_size) * num_kv_heads + g) * block_size + slot % block_size]",
+                                    "(slot / block_size * block_size + slot % block_size) * num_kv_heads + g]"),
+    "rowscale_v_uses_k_scales": ("v_scales ? row_scale(v_scales,", "v_scales ? row_scale(k_scales,"),
+    "rowscale_e4m3_top_code_127": ("block_size, num_blocks, dtype, 448.0f, f32_to_e4m3);",
+                                   "block_size, num_blocks, dtype, 127.0f, f32_to_e4m3);"),
+    "rowscale_stores_amax": ("    *scale = s;\n}", "    *scale = amax;\n}"),
+    "rowscale_zero_row_divides_by_zero": ("if (!(s >= FLT_MIN)) {", "if (!(s >= 0.0f)) {"),
+    "rowscale_write_scale_index_swapped": ("const int64_t si = (blk * num_kv_heads + g) * block_size + off;",
+                                           "const int64_t si = (blk * block_size + off) * num_kv_heads + g;"),
+    "rowscale_amax_ignores_sign": ("const float a = fabsf((float)decode(x16[d], dtype));",
+                                   "const float a = (float)decode(x16[d], dtype);"),
     "swap_no_conflict_check": ("if (block_mapping[2 * j + 1] == block_mapping[2 * i + 1]) status |= 8;", ""),
 }
 
