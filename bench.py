@@ -87,9 +87,11 @@ def parse_args():
     ap.add_argument("--shared-prefix", action="store_true",
                     help="beam_search: decode with pa_paged_decode_shared_prefix (shared "
                          "prompt blocks read once per group)")
-    ap.add_argument("--kv-dtype", default="auto", choices=["auto", "fp8", "int8"],
+    ap.add_argument("--kv-dtype", default="auto",
+                    choices=["auto", "fp8", "int8", "fp8-rows", "int8-rows"],
                     help="fp8 / int8: the same workload with e4m3 / int8 K/V pools (per-pool "
-                         "scales), quantising cache write + decode over the codes")
+                         "scales), quantising cache write + decode over the codes; -rows: one "
+                         "fp32 scale per (token, kv head) row instead")
     ap.add_argument("--swap", choices=["out", "in"], default=None,
                     help="measure pa_swap_blocks instead of the decode step: 512 LLaMA-7B-shaped "
                          "blocks (K and V, 256 KB a pair) device -> pinned host (out) or back (in)")
@@ -239,14 +241,24 @@ def whole_job_gbs(bytes_per_step: int, steps: int, world: int, max_elapsed_ms: f
     return world * bytes_per_step * steps / (max_elapsed_ms * 1e-3) / 1e9
 
 
+_BASE = {}            # the last 16-bit workload made, reused by its code-pool variants
+
+
 def make_workload(config: str, seqs: int = 0, kv_dtype: str = "auto"):
     """The named workload; with seqs > 0 a smaller batch of the same shape
     and a pool sized to it (profiling captures stay a few GB); kv_dtype fp8
-    or int8 redraws its pools as e4m3 or int8 codes."""
+    or int8 redraws its pools as e4m3 or int8 codes (one scale per pool),
+    fp8-rows / int8-rows as codes with one scale per (token, kv head) row."""
     from workloads import generators as gen
-    wl = _make_workload(config, seqs)
+    key = (config, seqs)
+    if key not in _BASE:
+        _BASE.clear()
+        _BASE[key] = _make_workload(config, seqs)
+    wl = _BASE[key]
     if kv_dtype in ("fp8", "int8"):
         wl = gen.with_code_pools(wl, kv_dtype, seed=gen.SEED_BASE + 50)
+    elif kv_dtype in ("fp8-rows", "int8-rows"):
+        wl = gen.with_rowscale_pools(wl, kv_dtype[:-5], seed=gen.SEED_BASE + 50)
     return wl
 
 
@@ -267,6 +279,8 @@ def _make_workload(config: str, seqs: int = 0):
 
 def workload_config(wl, partition_size, l2_note):
     kv = {"fp8": ", e4m3 K/V pools", "int8": ", int8 K/V pools"}.get(wl.extra.get("kv_dtype"), "")
+    if kv and wl.extra.get("rowscale"):
+        kv += " with one scale per (token, kv head) row"
     return {"workload": f"{wl.name}: {wl.num_seqs} seqs, {wl.num_q_heads}/{wl.num_kv_heads} heads, "
                         f"head_dim {wl.head_dim}, block {wl.block_size}, {wl.dtype}{kv}, "
                         f"contexts {int(wl.context_lens.min())}..{int(wl.context_lens.max())} "
@@ -297,8 +311,11 @@ class OracleStep:
         self.q = np.ascontiguousarray(wl.query[:n])
         self.kc, self.vc = wl.k_cache.copy(), wl.v_cache.copy()
         att = bm.decode_bytes(self.ctx, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
-                              wl.block_size, 2, bm.kv_elem_bytes(wl))
+                              wl.block_size, 2, bm.kv_elem_bytes(wl), bm.row_scale_bytes(wl))
         self.codes = wl.extra.get("kv_dtype")          # None, "fp8" or "int8"
+        self.rows = bool(wl.extra.get("rowscale"))
+        if self.rows:
+            self.ks, self.vs = wl.extra["k_scales"].copy(), wl.extra["v_scales"].copy()
         full = bm.step_bytes(wl)
         self.bytes = att["total"] + full["append"] + full["copy"]
         self.threads = oracle.max_threads()
@@ -308,6 +325,17 @@ class OracleStep:
         t0 = time.perf_counter()
         if wl.block_mapping.shape[0]:
             o.copy_blocks(self.kc, self.vc, wl.block_mapping)
+            if self.rows:
+                o.copy_blocks(self.ks, self.vs, wl.block_mapping)
+        if self.rows:
+            write = getattr(o, f"reshape_and_cache_{self.codes}_rowscale")
+            decode = getattr(o, f"paged_decode_{self.codes}_rowscale")
+            if wl.num_new_tokens:
+                write(wl.new_key, wl.new_value, self.kc, self.vc, self.ks, self.vs,
+                      wl.slot_mapping, wl.block_size, wl.dtype)
+            decode(self.q, self.kc, self.vc, self.ks, self.vs, self.tables, self.ctx, wl.scale,
+                   wl.dtype)
+            return time.perf_counter() - t0
         if self.codes is not None:
             ks, vs = wl.extra["k_scale"], wl.extra["v_scale"]
             write = getattr(o, f"reshape_and_cache_{self.codes}")
@@ -376,10 +404,12 @@ def run_reference(args):
 
 # Workloads measured in the same run as the headline, each on its own
 # (name, K/V code format, shared-prefix decode), when the run has one rank.
-PER_CONFIG = [("llama7b", "auto", False), ("mistral7b", "auto", False),
-              ("beam_search", "auto", True), ("mistral7b", "fp8", False),
-              ("mistral7b", "int8", False), ("long_context", "fp8", False),
-              ("long_context", "int8", False)]
+# Variants of one base workload follow each other, so it is drawn once.
+PER_CONFIG = [("long_context", "fp8", False), ("long_context", "int8", False),
+              ("long_context", "fp8-rows", False), ("long_context", "int8-rows", False),
+              ("llama7b", "auto", False), ("mistral7b", "auto", False),
+              ("mistral7b", "fp8", False), ("mistral7b", "int8", False),
+              ("beam_search", "auto", True)]
 
 
 class GpuStep:
@@ -396,6 +426,7 @@ class GpuStep:
         self.tdt = {"f16": torch.float16, "bf16": torch.bfloat16}[wl.dtype]
         self.codes = wl.extra.get("kv_dtype")                  # None, "fp8" or "int8"
         self.quant = self.codes is not None
+        self.rows = bool(wl.extra.get("rowscale"))             # one scale per row
         self.k_scale = wl.extra.get("k_scale", 1.0)
         self.v_scale = wl.extra.get("v_scale", 1.0)
         if self.quant:
@@ -403,6 +434,9 @@ class GpuStep:
             self.v_cache = torch.from_numpy(wl.v_cache).to(dev)
         else:
             self.k_cache, self.v_cache = self.up(wl.k_cache), self.up(wl.v_cache)
+        if self.rows:
+            self.k_scales = torch.from_numpy(wl.extra["k_scales"]).to(dev)
+            self.v_scales = torch.from_numpy(wl.extra["v_scales"]).to(dev)
         self.query = self.up(wl.query)
         self.new_key, self.new_value = self.up(wl.new_key), self.up(wl.new_value)
         self.slot_mapping = torch.from_numpy(wl.slot_mapping).to(dev)
@@ -448,8 +482,15 @@ class GpuStep:
         if self.n_pairs:
             B.pa_copy_blocks(self.k_cache, self.v_cache, self.block_mapping, self.d_status,
                              self.stream)
+            if self.rows:
+                B.pa_copy_block_scales(self.k_scales, self.v_scales, self.block_mapping,
+                                       self.d_status, self.stream)
         if wl.num_new_tokens and not self.fused:
-            if self.quant:
+            if self.rows:
+                getattr(B, f"pa_reshape_and_cache_{self.codes}_rowscale")(
+                    self.new_key, self.new_value, self.k_cache, self.v_cache, self.k_scales,
+                    self.v_scales, self.slot_mapping, self.d_status, self.stream)
+            elif self.quant:
                 getattr(B, f"pa_reshape_and_cache_{self.codes}")(
                     self.new_key, self.new_value, self.k_cache, self.v_cache, self.slot_mapping,
                     self.k_scale, self.v_scale, self.d_status, self.stream)
@@ -459,7 +500,17 @@ class GpuStep:
 
     def decode(self):
         B, wl = self.B, self.wl
-        if self.quant and self.fused:
+        if self.rows and self.fused:
+            getattr(B, f"pa_paged_decode_{self.codes}_rowscale_append")(
+                self.out, self.query, self.new_key, self.new_value, self.k_cache, self.v_cache,
+                self.k_scales, self.v_scales, self.block_tables, self.context_lens, self.mcl,
+                wl.scale, self.part, self.workspace, self.d_status, self.stream)
+        elif self.rows:
+            getattr(B, f"pa_paged_decode_{self.codes}_rowscale")(
+                self.out, self.query, self.k_cache, self.v_cache, self.k_scales, self.v_scales,
+                self.block_tables, self.context_lens, self.mcl, wl.scale, self.part,
+                self.workspace, self.d_status, self.stream)
+        elif self.quant and self.fused:
             getattr(B, f"pa_paged_decode_{self.codes}_append")(
                 self.out, self.query, self.new_key, self.new_value, self.k_cache, self.v_cache,
                 self.block_tables, self.context_lens, self.mcl, wl.scale, self.k_scale,
@@ -489,7 +540,8 @@ class GpuStep:
     def launches_per_step(self) -> int:
         wl = self.wl
         reduce = self.shared_reduce if self.shared else self.max_parts > 1
-        return ((1 if self.n_pairs else 0) + (1 if (wl.num_new_tokens and not self.fused) else 0)
+        copies = (2 if self.rows else 1) if self.n_pairs else 0
+        return (copies + (1 if (wl.num_new_tokens and not self.fused) else 0)
                 + 1 + (1 if reduce else 0))
 
     def prepare(self, warmup: int, eager: bool, barrier):
@@ -553,6 +605,10 @@ class GpuStep:
 
     def entry(self) -> str:
         c = self.codes
+        if self.rows:
+            return (f"pa_paged_decode_{c}_rowscale_append (row-scaled quantising write fused)"
+                    if self.fused else
+                    f"pa_reshape_and_cache_{c}_rowscale + pa_paged_decode_{c}_rowscale")
         return (f"pa_paged_decode_{c}_append (quantising cache write fused)" if self.quant and self.fused
                 else f"pa_reshape_and_cache_{c} + pa_paged_decode_{c}" if self.quant
                 else "pa_paged_decode_shared_prefix" if self.shared
@@ -573,7 +629,8 @@ class GpuStep:
         return unique, referenced
 
     def free(self):
-        for name in ("k_cache", "v_cache", "query", "new_key", "new_value", "out", "workspace",
+        for name in ("k_cache", "v_cache", "k_scales", "v_scales", "query", "new_key",
+                     "new_value", "out", "workspace",
                      "graphs", "block_tables", "context_lens", "slot_mapping", "block_mapping"):
             if hasattr(self, name):
                 delattr(self, name)
@@ -595,7 +652,7 @@ def measure_per_config(name, kv_dtype, shared, args, dev, barrier, peak):
     decode_avg = statistics.mean(decode_ms)
     dbytes, referenced = g.roofline_bytes()
     achieved = dbytes / (decode_avg * 1e-3) / 1e9
-    label = name + (f"-{kv_dtype}" if kv_dtype != "auto" else "")
+    label = name + (f"-{kv_dtype}" if kv_dtype != "auto" else "")   # e.g. mistral7b-int8-rows
     entry = {"workload": workload_config(wl, g.part, "")["workload"],
              "us_per_layer_step": round(elapsed_ms / args.steps * 1e3, 2),
              "kernel": g.kernel_name(), "decode_entry": g.entry(),
@@ -662,7 +719,8 @@ def run_ours(args):
     from paged_kv_cache_415_b200.step import DecodeStep, HostPipeline
     tdt, fused = g.tdt, g.fused
     stepper = DecodeStep(g.k_cache, g.v_cache, wl.num_seqs, wl.num_q_heads, g.mcl, g.part,
-                         g.k_scale, g.v_scale)
+                         g.k_scale, g.v_scale, getattr(g, "k_scales", None),
+                         getattr(g, "v_scales", None))
     host = {"query": torch.from_numpy(wl.query.view(np.int16)).view(tdt).pin_memory(),
             "block_tables": torch.from_numpy(wl.block_tables).pin_memory(),
             "context_lens": torch.from_numpy(wl.context_lens).pin_memory(),
@@ -714,7 +772,8 @@ def run_ours(args):
     peak, peak_kind = hbm_peak()
     decode_bytes, referenced = g.roofline_bytes()
     achieved = decode_bytes / (decode_avg * 1e-3) / 1e9
-    label = args.config + (f"-{g.codes}" if g.quant else "") + ("-shared" if g.shared else "")
+    label = (args.config + (f"-{g.codes}" if g.quant else "") + ("-rows" if g.rows else "")
+             + ("-shared" if g.shared else ""))
     traffic = profiled_traffic(label, kernel_family(g)) if args.seqs <= 0 else None
     clocks = sampler.summary()
     clocks = merge_clocks(clocks, e_sampler.summary())
@@ -756,8 +815,8 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(per_step_ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": ({"fp8": "f16 (e4m3 K/V)", "int8": "f16 (int8 K/V)"}[g.codes] if g.quant
-                  else wl.dtype),
+        "dtype": ({"fp8": "f16 (e4m3 K/V)", "int8": "f16 (int8 K/V)"}[g.codes]
+                  + (", row scales" if g.rows else "") if g.quant else wl.dtype),
         "data": "synthetic", "config": config_block,
         "us_per_layer_step": round(per_step_ms * 1e3, 2),
         "kv_tokens_per_s": round(world * int(wl.context_lens.sum()) * args.steps / (elapsed_ms * 1e-3)),

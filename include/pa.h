@@ -11,7 +11,8 @@
  * Declared below as well: pa_paged_decode_append (the cache write fused into
  * the decode launch), pa_paged_decode_no_alloc (library-owned scratch),
  * pa_paged_decode_shared_prefix (groups that share a stored prefix read it
- * once), the _fp8 and _int8 variants over one-byte K/V pools, pa_swap_blocks
+ * once), the _fp8 and _int8 variants over one-byte K/V pools (one scale per
+ * pool, or one per row with the _rowscale calls), pa_swap_blocks
  * (block copies between device and pinned host pools), and the size
  * queries.  The host block manager that hands out the block ids is declared
  * in pa_block_manager.h.
@@ -106,7 +107,9 @@ typedef enum pa_dtype {
     PA_DTYPE_F16 = 0,
     PA_DTYPE_BF16 = 1,
     PA_DTYPE_FP8_E4M3 = 2,  /* cache pools only: block copies/swaps and the *_fp8 calls */
-    PA_DTYPE_INT8 = 3       /* cache pools only: block copies/swaps and the *_int8 calls */
+    PA_DTYPE_INT8 = 3,      /* cache pools only: block copies/swaps and the *_int8 calls */
+    PA_DTYPE_F32 = 4        /* row-scale pools of the *_rowscale calls: block copies/swaps
+                               only, with head_dim 1 */
 } pa_dtype;
 
 #define PA_STATUS_BAD_BLOCK 1
@@ -418,6 +421,88 @@ PA_API pa_status pa_paged_decode_int8_append(
     int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len, float scale,
     float k_scale, float v_scale, int32_t partition_size, void* workspace, size_t workspace_bytes,
     pa_dtype dtype, int32_t* d_status, pa_stream_t stream);
+
+/*
+ * Row-scaled one-byte KV cache -- e4m3 or int8 code pools as above, but with
+ * one fp32 scale per (token, kv head) row instead of one per pool, so heads
+ * (and tokens) of very different magnitude each keep the full resolution of
+ * the code.  Defined by the same passages as the FP8 pools ([Practice §7
+ * 演进方向与优化空间], [VM-paging, PagedAttention的工程实践与局限]); the
+ * per-row granularity is this library's reading: a row is quantised once,
+ * when it is written, from its own values, and never rewritten.
+ *
+ * Scale pools (caller-owned, fp32, 16-byte aligned, one for K and one for V):
+ *   k_scales, v_scales : [num_blocks][num_kv_heads][block_size]
+ * The cached value of element d of the row of slot `slot`, kv head g, is
+ *   decode(code) * scales[slot / block_size][g][slot % block_size].
+ * A block's scales for one kv head are one contiguous run of block_size
+ * floats.  Block copies and swaps move a scale pool with pa_copy_blocks /
+ * pa_swap_blocks, dtype PA_DTYPE_F32, head_dim 1 (same block ids as the
+ * code pools).  Extra HBM per token: 8 bytes per kv head (3% at D = 128).
+ *
+ * pa_reshape_and_cache_fp8_rowscale / _int8_rowscale -- the quantising
+ * write: for each written (token, kv head) row x,
+ *   s = fp32(max_d |x_d| / code_max)       (code_max 448 e4m3, 127 int8)
+ *   code_d = encode(fp32(x_d * fp32(1 / s))), rounded and saturated as the
+ *            per-pool write does (so the row's largest element takes the
+ *            top code);
+ * a row with s below the smallest normal fp32 (all zeros) stores s = 0 and
+ * zero codes.  The codes go to the slot, s to the scale pools.  Arguments
+ * and errors as pa_reshape_and_cache_fp8 without the two scales; block_size
+ * 8, 16 or 32.
+ *
+ * pa_paged_decode_fp8_rowscale / _int8_rowscale -- pa_paged_decode_fp8 /
+ * _int8 over row-scaled pools: the score of token t is multiplied by its K
+ * row scale, and its V row by its V row scale.  block_size 16 or 32.  The
+ * _append forms write each sequence's new token (key / value of `dtype`,
+ * [num_seqs][num_kv_heads][head_dim]) at position context_lens[s] - 1 with
+ * the row-scaled quantisation above, codes and scales, inside the decode
+ * launch.  Other arguments, results and errors as pa_paged_decode_fp8 and
+ * pa_paged_decode_fp8_append.
+ */
+PA_API pa_status pa_reshape_and_cache_fp8_rowscale(
+    const void* key, const void* value, void* k_cache, void* v_cache, float* k_scales,
+    float* v_scales, const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int64_t num_blocks, pa_dtype dtype, int32_t* d_status,
+    pa_stream_t stream);
+
+PA_API pa_status pa_reshape_and_cache_int8_rowscale(
+    const void* key, const void* value, void* k_cache, void* v_cache, float* k_scales,
+    float* v_scales, const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int64_t num_blocks, pa_dtype dtype, int32_t* d_status,
+    pa_stream_t stream);
+
+PA_API pa_status pa_paged_decode_fp8_rowscale(
+    void* out, const void* query, const void* k_cache, const void* v_cache, const float* k_scales,
+    const float* v_scales, const int32_t* block_tables, const int32_t* context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float scale, int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+    int32_t* d_status, pa_stream_t stream);
+
+PA_API pa_status pa_paged_decode_int8_rowscale(
+    void* out, const void* query, const void* k_cache, const void* v_cache, const float* k_scales,
+    const float* v_scales, const int32_t* block_tables, const int32_t* context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float scale, int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+    int32_t* d_status, pa_stream_t stream);
+
+PA_API pa_status pa_paged_decode_fp8_rowscale_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, float* k_scales, float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, float scale, int32_t partition_size, void* workspace,
+    size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream);
+
+PA_API pa_status pa_paged_decode_int8_rowscale_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, float* k_scales, float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, float scale, int32_t partition_size, void* workspace,
+    size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream);
 
 /*
  * pa_paged_decode_shared_prefix -- pa_paged_decode for batches whose

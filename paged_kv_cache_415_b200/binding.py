@@ -21,7 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpa.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_CUDA = 0, 1, 2, 3
-PA_DTYPE_F16, PA_DTYPE_BF16, PA_DTYPE_FP8_E4M3, PA_DTYPE_INT8 = 0, 1, 2, 3
+PA_DTYPE_F16, PA_DTYPE_BF16, PA_DTYPE_FP8_E4M3, PA_DTYPE_INT8, PA_DTYPE_F32 = 0, 1, 2, 3, 4
 PA_STATUS_BAD_BLOCK = 1
 PA_STATUS_BAD_SLOT = 2
 PA_STATUS_BAD_CONTEXT = 4
@@ -30,7 +30,7 @@ PA_STATUS_TIMEOUT = 16
 
 _DTYPES = {torch.float16: PA_DTYPE_F16, torch.bfloat16: PA_DTYPE_BF16,
            torch.uint8: PA_DTYPE_FP8_E4M3, torch.float8_e4m3fn: PA_DTYPE_FP8_E4M3,
-           torch.int8: PA_DTYPE_INT8}
+           torch.int8: PA_DTYPE_INT8, torch.float32: PA_DTYPE_F32}
 
 # Every entry point declared in include/pa.h.
 EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_size",
@@ -38,7 +38,10 @@ EXPORTS = ("pa_reshape_and_cache", "pa_copy_blocks", "pa_paged_decode_partition_
            "pa_paged_decode_shared_prefix_workspace_size", "pa_paged_decode_shared_prefix",
            "pa_paged_decode_append", "pa_reshape_and_cache_fp8", "pa_paged_decode_fp8",
            "pa_paged_decode_fp8_append", "pa_reshape_and_cache_int8", "pa_paged_decode_int8",
-           "pa_paged_decode_int8_append", "pa_swap_blocks",
+           "pa_paged_decode_int8_append", "pa_reshape_and_cache_fp8_rowscale",
+           "pa_reshape_and_cache_int8_rowscale", "pa_paged_decode_fp8_rowscale",
+           "pa_paged_decode_int8_rowscale", "pa_paged_decode_fp8_rowscale_append",
+           "pa_paged_decode_int8_rowscale_append", "pa_swap_blocks",
            "pa_status_string", "pa_version")
 # The test entry points declared in include/pa_selftest.h.
 SELFTEST_EXPORTS = ("pa_selftest_bounded_wait", "pa_selftest_decode_abort",
@@ -98,6 +101,18 @@ def _load() -> ctypes.CDLL:
     lib.pa_paged_decode_int8.restype = i32
     lib.pa_paged_decode_int8_append.argtypes = lib.pa_paged_decode_fp8_append.argtypes
     lib.pa_paged_decode_int8_append.restype = i32
+    for fmt in ("fp8", "int8"):
+        w = getattr(lib, f"pa_reshape_and_cache_{fmt}_rowscale")
+        w.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i64, i32, p, p]
+        w.restype = i32
+        dcd = getattr(lib, f"pa_paged_decode_{fmt}_rowscale")
+        dcd.argtypes = [p, p, p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64, i32, f32, i32,
+                        p, sz, i32, p, p]
+        dcd.restype = i32
+        app = getattr(lib, f"pa_paged_decode_{fmt}_rowscale_append")
+        app.argtypes = [p, p, p, p, p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i64, i32, f32,
+                        i32, p, sz, i32, p, p]
+        app.restype = i32
     lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i64, i64, i32, p, p]
     lib.pa_swap_blocks.restype = i32
     lib.pa_selftest_bounded_wait.argtypes = [p, p, ctypes.c_uint32, i32, p]
@@ -344,6 +359,114 @@ def pa_paged_decode_int8_append(out, query, key, value, k_cache, v_cache, block_
         int(block_tables.shape[1]), num_blocks, int(max_context_len), float(scale),
         float(k_scale), float(v_scale), int(partition_size), _ptr(workspace), ws_bytes,
         _dtype(query), _ptr(d_status), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Row-scaled one-byte pools: codes [num_blocks][B][Hkv][D] (uint8 e4m3 or
+# int8) and fp32 scales [num_blocks][Hkv][B], one per (token, kv head) row
+# ---------------------------------------------------------------------------
+
+def _rowscale_write(fmt, key, value, k_cache, v_cache, k_scales, v_scales, slot_mapping,
+                    d_status=None, stream=None) -> None:
+    num_blocks, block_size, hkv, d = k_cache.shape
+    fn = f"pa_reshape_and_cache_{fmt}_rowscale"
+    _check(fn, getattr(LIB, fn)(
+        _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales),
+        _ptr(slot_mapping), int(slot_mapping.shape[0]), hkv, d, block_size, num_blocks,
+        _dtype(key), _ptr(d_status), _stream(stream)))
+
+
+def pa_reshape_and_cache_fp8_rowscale(key, value, k_cache, v_cache, k_scales, v_scales,
+                                      slot_mapping, d_status=None, stream=None) -> None:
+    """Quantising write into e4m3 pools with one scale per row:
+    s = max |x| / 448 stored in k_scales / v_scales [num_blocks][Hkv][B]."""
+    _rowscale_write("fp8", key, value, k_cache, v_cache, k_scales, v_scales, slot_mapping,
+                    d_status, stream)
+
+
+def pa_reshape_and_cache_int8_rowscale(key, value, k_cache, v_cache, k_scales, v_scales,
+                                       slot_mapping, d_status=None, stream=None) -> None:
+    """As pa_reshape_and_cache_fp8_rowscale into int8 pools (s = max |x| / 127)."""
+    _rowscale_write("int8", key, value, k_cache, v_cache, k_scales, v_scales, slot_mapping,
+                    d_status, stream)
+
+
+def _rowscale_decode(fmt, out, query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                     context_lens, max_context_len, scale, partition_size, workspace, d_status,
+                     stream) -> None:
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    fn = f"pa_paged_decode_{fmt}_rowscale"
+    _check(fn, getattr(LIB, fn)(
+        _ptr(out), _ptr(query), _ptr(k_cache), _ptr(v_cache), _ptr(k_scales), _ptr(v_scales),
+        _ptr(block_tables), _ptr(context_lens), num_seqs, hq, hkv, d, block_size,
+        int(block_tables.shape[1]), num_blocks, int(max_context_len), float(scale),
+        int(partition_size), _ptr(workspace), ws_bytes, _dtype(query), _ptr(d_status),
+        _stream(stream)))
+
+
+def pa_paged_decode_fp8_rowscale(out, query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                                 context_lens, max_context_len, scale, partition_size=0,
+                                 workspace=None, d_status=None, stream=None) -> None:
+    """pa_paged_decode over e4m3 pools with one scale per row."""
+    _rowscale_decode("fp8", out, query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                     context_lens, max_context_len, scale, partition_size, workspace, d_status,
+                     stream)
+
+
+def pa_paged_decode_int8_rowscale(out, query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                                  context_lens, max_context_len, scale, partition_size=0,
+                                  workspace=None, d_status=None, stream=None) -> None:
+    """pa_paged_decode over int8 pools with one scale per row."""
+    _rowscale_decode("int8", out, query, k_cache, v_cache, k_scales, v_scales, block_tables,
+                     context_lens, max_context_len, scale, partition_size, workspace, d_status,
+                     stream)
+
+
+def _rowscale_append(fmt, out, query, key, value, k_cache, v_cache, k_scales, v_scales,
+                     block_tables, context_lens, max_context_len, scale, partition_size,
+                     workspace, d_status, stream) -> None:
+    num_seqs, hq, d = query.shape
+    num_blocks, block_size, hkv, _ = k_cache.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    fn = f"pa_paged_decode_{fmt}_rowscale_append"
+    _check(fn, getattr(LIB, fn)(
+        _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(k_cache), _ptr(v_cache),
+        _ptr(k_scales), _ptr(v_scales), _ptr(block_tables), _ptr(context_lens), num_seqs, hq,
+        hkv, d, block_size, int(block_tables.shape[1]), num_blocks, int(max_context_len),
+        float(scale), int(partition_size), _ptr(workspace), ws_bytes, _dtype(query),
+        _ptr(d_status), _stream(stream)))
+
+
+def pa_paged_decode_fp8_rowscale_append(out, query, key, value, k_cache, v_cache, k_scales,
+                                        v_scales, block_tables, context_lens, max_context_len,
+                                        scale, partition_size=0, workspace=None, d_status=None,
+                                        stream=None) -> None:
+    """pa_paged_decode_fp8_rowscale with each sequence's new token quantised
+    (codes and row scales) into its slot inside the launch."""
+    _rowscale_append("fp8", out, query, key, value, k_cache, v_cache, k_scales, v_scales,
+                     block_tables, context_lens, max_context_len, scale, partition_size,
+                     workspace, d_status, stream)
+
+
+def pa_paged_decode_int8_rowscale_append(out, query, key, value, k_cache, v_cache, k_scales,
+                                         v_scales, block_tables, context_lens, max_context_len,
+                                         scale, partition_size=0, workspace=None, d_status=None,
+                                         stream=None) -> None:
+    """pa_paged_decode_int8_rowscale with the fused row-scaled cache write."""
+    _rowscale_append("int8", out, query, key, value, k_cache, v_cache, k_scales, v_scales,
+                     block_tables, context_lens, max_context_len, scale, partition_size,
+                     workspace, d_status, stream)
+
+
+def pa_copy_block_scales(k_scales, v_scales, block_mapping, d_status=None, stream=None) -> None:
+    """pa_copy_blocks over the row-scale pools [num_blocks][Hkv][B] (fp32):
+    the scales of each (src, dst) block move with its codes."""
+    num_blocks, hkv, block_size = k_scales.shape
+    _check("pa_copy_blocks", LIB.pa_copy_blocks(
+        _ptr(k_scales), _ptr(v_scales), _ptr(block_mapping), int(block_mapping.shape[0]), hkv,
+        1, block_size, num_blocks, PA_DTYPE_F32, _ptr(d_status), _stream(stream)))
 
 
 def _addr(t) -> int:

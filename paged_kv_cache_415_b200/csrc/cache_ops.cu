@@ -107,6 +107,53 @@ __global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_q8_kernel(
     }
 }
 
+// Row-scaled variant: one warp per (token, kv head) quantises that row of K
+// and of V with a scale of its own (quantise_row_warp: s = max|x| / kMax,
+// codes of x * (1 / s)) and stores the codes at the slot and the scales at
+// [slot / B][kv head][slot % B] of the scale pools.  Grid (token, group of
+// four kv heads).
+constexpr int kRowWarps = kCacheThreads / 32;
+
+template <typename Codes, typename T, int D>
+__global__ void __launch_bounds__(kCacheThreads) reshape_and_cache_rowscale_kernel(
+    const T* __restrict__ key, const T* __restrict__ value, uint8_t* __restrict__ k_cache,
+    uint8_t* __restrict__ v_cache, float* __restrict__ k_scales, float* __restrict__ v_scales,
+    const int64_t* __restrict__ slot_mapping, int32_t num_kv_heads, int32_t block_size,
+    int64_t num_slots, int32_t* d_status)
+{
+    grid_dependency_wait();
+    allow_dependents();
+    const int64_t t = blockIdx.x;
+    const int g = blockIdx.y * kRowWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t slot = slot_mapping[t];
+    if (slot < 0) return;                       // padding token
+    if (slot >= num_slots) {
+        if (threadIdx.x == 0 && blockIdx.y == 0) status_or(d_status, PA_STATUS_BAD_SLOT);
+        return;
+    }
+    if (g >= num_kv_heads) return;              // warp-uniform
+    const int64_t src = (t * num_kv_heads + g) * D;
+    const int64_t dst = (slot * num_kv_heads + g) * D;
+    const int64_t si = ((slot / block_size) * num_kv_heads + g) * block_size + slot % block_size;
+    uint4 kx = make_uint4(0, 0, 0, 0), vx = make_uint4(0, 0, 0, 0);
+    if (lane < D / 8) {
+        kx = ld_nc_v4(key + src + lane * 8);
+        vx = ld_nc_v4(value + src + lane * 8);
+    }
+    float ks, vs;
+    const uint2 kc = quantise_row_warp<Codes, T, D>(kx, ks);
+    const uint2 vc = quantise_row_warp<Codes, T, D>(vx, vs);
+    if (lane < D / 8) {
+        *reinterpret_cast<uint2*>(k_cache + dst + lane * 8) = kc;
+        *reinterpret_cast<uint2*>(v_cache + dst + lane * 8) = vc;
+    }
+    if (lane == 0) {
+        k_scales[si] = ks;
+        v_scales[si] = vs;
+    }
+}
+
 // Grid (pair, K-or-V, chunk of the block).  Whole-block bit copy src -> dst
 // ([VM-paging, 写时复制与块共享机制]; [Practice §4.1 共享内存管理] step 2).
 // The first CTA of each pair also checks the pair against all the others:
@@ -210,15 +257,26 @@ __global__ void __launch_bounds__(kSwapThreads) swap_blocks_kernel(
     }
 }
 
+// Pools the calls accept: 16-bit pools (head_dim 64 or 128); with
+// allow_codes also one-byte code pools, and row-scale pools (PA_DTYPE_F32,
+// head_dim 1: a block holds block_size x num_kv_heads fp32 scales).
 static pa_status check_pool_shape(int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                   int64_t num_blocks, int32_t dtype, bool allow_codes = false)
 {
     if (num_kv_heads <= 0 || num_blocks <= 0 || head_dim <= 0 || block_size <= 0)
         return PA_ERR_INVALID_ARG;
+    if (allow_codes && dtype == PA_DTYPE_F32)
+        return head_dim == 1 && supported_block_size(block_size) ? PA_OK : PA_ERR_UNSUPPORTED;
     const bool dtype_ok = supported_dtype(dtype) || (allow_codes && code_dtype(dtype));
     if (!supported_head_dim(head_dim) || !supported_block_size(block_size) || !dtype_ok)
         return PA_ERR_UNSUPPORTED;
     return PA_OK;
+}
+
+// Bytes of one element of a pool of this type.
+static int pool_elem_bytes(int32_t dtype)
+{
+    return dtype == PA_DTYPE_F32 ? 4 : code_dtype(dtype) ? 1 : 2;
 }
 
 }  // namespace pa
@@ -264,7 +322,7 @@ extern "C" pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int64_t*
         (d_status && !aligned4(d_status)))
         return PA_ERR_INVALID_ARG;
     if (num_pairs == 0) return PA_OK;
-    const int elem_bytes = code_dtype(dtype) ? 1 : 2;
+    const int elem_bytes = pool_elem_bytes(dtype);
     const int64_t block_vecs =
         static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes / 16;
     const int64_t per_cta = static_cast<int64_t>(kCopyThreads) * kCopyVecsPerThread;
@@ -340,6 +398,78 @@ extern "C" pa_status pa_reshape_and_cache_int8(const void* key, const void* valu
 }
 
 namespace pa {
+template <typename Codes, typename T>
+static pa_status launch_rowscale_write(const void* key, const void* value, void* k_cache,
+                                       void* v_cache, float* k_scales, float* v_scales,
+                                       const int64_t* slot_mapping, dim3 grid, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t block_size, int64_t num_slots,
+                                       int32_t* d_status, pa_stream_t stream)
+{
+    auto kernel = head_dim == 128 ? reshape_and_cache_rowscale_kernel<Codes, T, 128>
+                                  : reshape_and_cache_rowscale_kernel<Codes, T, 64>;
+    return launch_overlapped(kernel, grid, dim3(kCacheThreads), 0, stream,
+                             static_cast<const T*>(key), static_cast<const T*>(value),
+                             static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
+                             k_scales, v_scales, slot_mapping, num_kv_heads, block_size, num_slots,
+                             d_status);
+}
+
+template <typename Codes>
+static pa_status reshape_and_cache_rowscale(const void* key, const void* value, void* k_cache,
+                                            void* v_cache, float* k_scales, float* v_scales,
+                                            const int64_t* slot_mapping, int32_t num_tokens,
+                                            int32_t num_kv_heads, int32_t head_dim,
+                                            int32_t block_size, int64_t num_blocks, pa_dtype dtype,
+                                            int32_t* d_status, pa_stream_t stream)
+{
+    if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+    pa_status st = check_pool_shape(num_kv_heads, head_dim, block_size, num_blocks, dtype);
+    if (st != PA_OK) return st;
+    if (!key || !value || !k_cache || !v_cache || !k_scales || !v_scales || !slot_mapping)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(k_scales) || !aligned16(v_scales) || !aligned8(slot_mapping) ||
+        (d_status && !aligned4(d_status)))
+        return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    const int32_t groups = (num_kv_heads + kRowWarps - 1) / kRowWarps;
+    if (groups > 65535) return PA_ERR_UNSUPPORTED;
+    dim3 grid(num_tokens, groups);
+    const int64_t num_slots = num_blocks * block_size;
+    return dtype == PA_DTYPE_F16
+               ? launch_rowscale_write<Codes, __half>(key, value, k_cache, v_cache, k_scales,
+                                                      v_scales, slot_mapping, grid, num_kv_heads,
+                                                      head_dim, block_size, num_slots, d_status,
+                                                      stream)
+               : launch_rowscale_write<Codes, __nv_bfloat16>(
+                     key, value, k_cache, v_cache, k_scales, v_scales, slot_mapping, grid,
+                     num_kv_heads, head_dim, block_size, num_slots, d_status, stream);
+}
+}  // namespace pa
+
+extern "C" pa_status pa_reshape_and_cache_fp8_rowscale(
+    const void* key, const void* value, void* k_cache, void* v_cache, float* k_scales,
+    float* v_scales, const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int64_t num_blocks, pa_dtype dtype, int32_t* d_status,
+    pa_stream_t stream)
+{
+    return pa::reshape_and_cache_rowscale<pa::E4m3Codes>(
+        key, value, k_cache, v_cache, k_scales, v_scales, slot_mapping, num_tokens, num_kv_heads,
+        head_dim, block_size, num_blocks, dtype, d_status, stream);
+}
+
+extern "C" pa_status pa_reshape_and_cache_int8_rowscale(
+    const void* key, const void* value, void* k_cache, void* v_cache, float* k_scales,
+    float* v_scales, const int64_t* slot_mapping, int32_t num_tokens, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int64_t num_blocks, pa_dtype dtype, int32_t* d_status,
+    pa_stream_t stream)
+{
+    return pa::reshape_and_cache_rowscale<pa::Int8Codes>(
+        key, value, k_cache, v_cache, k_scales, v_scales, slot_mapping, num_tokens, num_kv_heads,
+        head_dim, block_size, num_blocks, dtype, d_status, stream);
+}
+
+namespace pa {
 // The address the device uses for p: device and managed memory as is,
 // pinned host memory through its mapping; anything else (pageable host
 // memory, an unknown pointer) is refused, so no kernel ever dereferences it.
@@ -385,7 +515,7 @@ extern "C" pa_status pa_swap_blocks(const void* src_k, const void* src_v, void* 
         !device_address(dst_k, &dk) || !device_address(dst_v, &dv) ||
         !device_address(block_mapping, &map))
         return PA_ERR_INVALID_ARG;
-    const int elem_bytes = code_dtype(dtype) ? 1 : 2;
+    const int elem_bytes = pool_elem_bytes(dtype);
     const int64_t block_vecs =
         static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes / 16;
     const int64_t per_cta = static_cast<int64_t>(kSwapThreads) * kSwapVecsPerThread;

@@ -18,9 +18,12 @@
 //                      lower-addressed code in the low half.
 //   encode2(a, b)      two fp32 values (already times 1 / scale) as two
 //                      codes in the low 16 bits, a in the low byte.
+//   kMax               the largest code magnitude (448 or 127): the code a
+//                      row's largest element takes under a row scale.
 #pragma once
 
 #include <cuda_fp8.h>
+#include <float.h>
 #include <stdint.h>
 
 #include "pa_common.cuh"
@@ -28,6 +31,8 @@
 namespace pa {
 
 struct E4m3Codes {
+    static constexpr float kMax = 448.0f;
+
     static __device__ __forceinline__ void widen4(uint32_t w, uint32_t& lo, uint32_t& hi)
     {
         asm("{\n\t.reg .b16 l, h;\n\t"
@@ -46,6 +51,8 @@ struct E4m3Codes {
 };
 
 struct Int8Codes {
+    static constexpr float kMax = 127.0f;
+
     // Exponent-field construction: with 0x64 as the high byte, an fp16 is
     // 1024 + (low byte), since its unit in [1024, 2048) is 1.  Flipping the
     // sign bit of a code c gives the byte c + 128, so the fp16 0x64:(c + 128)
@@ -84,6 +91,42 @@ __device__ __forceinline__ uint2 encode8(const uint4& w, float inv)
 #pragma unroll
     for (int j = 0; j < 4; ++j) r[j] = Codes::encode2(f[2 * j] * inv, f[2 * j + 1] * inv);
     return make_uint2(r[0] | (r[1] << 16), r[2] | (r[3] << 16));
+}
+
+// Largest magnitude among the 8 elements of a 16-byte vector, exact.
+template <typename T>
+__device__ __forceinline__ float amax8(const uint4& w)
+{
+    float f[8];
+    unpack8<T>(w, f);
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+    return m;
+}
+
+// One row of D elements quantised with a scale of its own, by a whole warp
+// (lanes below D / 8 hold 8 elements each; every lane must call it):
+//   amax = max |x|,  s = fp32(amax / kMax),  codes = encode8(x, fp32(1 / s)),
+// the per-pool encoding with scale s, so the row's largest element takes the
+// top code.  A row whose s is below the smallest normal fp32 (all zeros, or
+// tiny values) gets s = 0 and zero codes.  `x` is the lane's 16-byte input
+// vector (anything on lanes >= D / 8); returns the lane's 8 codes and sets
+// `scale` on every lane.
+template <typename Codes, typename T, int D>
+__device__ __forceinline__ uint2 quantise_row_warp(const uint4& x, float& scale)
+{
+    const int lane = threadIdx.x & 31;
+    float m = lane < D / 8 ? amax8<T>(x) : 0.f;
+#pragma unroll
+    for (int k = 16; k >= 1; k >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, k));
+    const float s = m / Codes::kMax;
+    if (!(s >= FLT_MIN)) {
+        scale = 0.f;
+        return make_uint2(0u, 0u);
+    }
+    scale = s;
+    return encode8<Codes, T>(x, 1.0f / s);
 }
 
 }  // namespace pa

@@ -62,6 +62,8 @@ struct DecodeArgs {
     int32_t lpt_seqs = 0;              // > 0: longest-first dispatch over this many sequences
     float k_inv = 1.f, v_inv = 1.f;    // quantised pools: reciprocal scales of the fused write
     uint32_t probe_us = 0;             // test hook of the bounded waits (pa_selftest_*); 0 = off
+    float* k_scales = nullptr;         // row-scale pools of quantised K/V, or null (pool scales)
+    float* v_scales = nullptr;
 };
 
 constexpr int kMaxDevices = 64;
@@ -187,13 +189,14 @@ static bool encode_pool_map_q8(CUtensorMap* map, const void* pool, int32_t head_
     return res == CUDA_SUCCESS;
 }
 
-template <typename Codes, typename T, int D, int BS, int G>
+template <typename Codes, typename T, int D, int BS, int G, bool ROWS>
 static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
 {
-    using S = Q8Shape<D, BS, G>;
+    using S = Q8Shape<D, BS, G, ROWS>;
     static std::atomic<uint64_t> attr_done{0};
-    auto kernel = std::is_same<Codes, Int8Codes>::value ? paged_decode_int8_kernel<T, D, BS, G>
-                                                        : paged_decode_fp8_kernel<T, D, BS, G>;
+    auto kernel = std::is_same<Codes, Int8Codes>::value
+                      ? paged_decode_int8_kernel<T, D, BS, G, ROWS>
+                      : paged_decode_fp8_kernel<T, D, BS, G, ROWS>;
     if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
     CUtensorMap tm_k, tm_v;
     if (!encode_pool_map_q8(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks) ||
@@ -208,7 +211,7 @@ static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
         static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
         static_cast<uint8_t*>(const_cast<void*>(a.k_cache)),
         static_cast<uint8_t*>(const_cast<void*>(a.v_cache)), a.num_kv_heads, a.k_inv, a.v_inv,
-        a.probe_us);
+        a.probe_us, a.k_scales, a.v_scales);
     if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
     const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
@@ -219,16 +222,23 @@ static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
                              a.partition_size, a.max_parts);
 }
 
+template <typename Codes, typename T, int D, int BS, bool ROWS>
+static pa_status dispatch_q8_group_rows(const DecodeArgs& a, float v_scale)
+{
+    switch (a.num_q_heads / a.num_kv_heads) {
+    case 1: return launch_decode_q8<Codes, T, D, BS, 1, ROWS>(a, v_scale);
+    case 2: return launch_decode_q8<Codes, T, D, BS, 2, ROWS>(a, v_scale);
+    case 4: return launch_decode_q8<Codes, T, D, BS, 4, ROWS>(a, v_scale);
+    case 8: return launch_decode_q8<Codes, T, D, BS, 8, ROWS>(a, v_scale);
+    default: return PA_ERR_UNSUPPORTED;
+    }
+}
+
 template <typename Codes, typename T, int D, int BS>
 static pa_status dispatch_q8_group(const DecodeArgs& a, float v_scale)
 {
-    switch (a.num_q_heads / a.num_kv_heads) {
-    case 1: return launch_decode_q8<Codes, T, D, BS, 1>(a, v_scale);
-    case 2: return launch_decode_q8<Codes, T, D, BS, 2>(a, v_scale);
-    case 4: return launch_decode_q8<Codes, T, D, BS, 4>(a, v_scale);
-    case 8: return launch_decode_q8<Codes, T, D, BS, 8>(a, v_scale);
-    default: return PA_ERR_UNSUPPORTED;
-    }
+    return a.k_scales != nullptr ? dispatch_q8_group_rows<Codes, T, D, BS, true>(a, v_scale)
+                                 : dispatch_q8_group_rows<Codes, T, D, BS, false>(a, v_scale);
 }
 
 template <typename Codes, typename T>
@@ -484,7 +494,8 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
                              pa_dtype dtype, int32_t* d_status, pa_stream_t stream,
                              const void* new_key, const void* new_value,
                              KvCodes codes = KvCodes::kPlain, float k_scale = 1.f,
-                             float v_scale = 1.f, uint32_t probe_us = 0)
+                             float v_scale = 1.f, uint32_t probe_us = 0,
+                             float* k_scales = nullptr, float* v_scales = nullptr)
 {
     pa_status st = check_decode_shape(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
                                       max_context_len, partition_size);
@@ -500,6 +511,10 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
         (new_value == nullptr || !aligned16(new_key) || !aligned16(new_value)))
         return PA_ERR_INVALID_ARG;
     const bool quantised = codes != KvCodes::kPlain;
+    const bool row_scaled = k_scales != nullptr || v_scales != nullptr;
+    if (row_scaled && (!quantised || !k_scales || !v_scales || !aligned16(k_scales) ||
+                 !aligned16(v_scales)))
+        return PA_ERR_INVALID_ARG;
     if (quantised) {
         if (!(k_scale > 0.f) || !(v_scale > 0.f) || !isfinite(k_scale) || !isfinite(v_scale))
             return PA_ERR_INVALID_ARG;
@@ -543,6 +558,8 @@ static pa_status decode_impl(void* out, const void* query, const void* k_cache, 
     a.new_key = new_key;
     a.new_value = new_value;
     a.probe_us = probe_us;
+    a.k_scales = k_scales;
+    a.v_scales = v_scales;
     if (quantised) {
         a.k_inv = 1.0f / k_scale;      // the quantising write's fp32(1 / scale)
         a.v_inv = 1.0f / v_scale;
@@ -649,6 +666,74 @@ extern "C" pa_status pa_paged_decode_int8_append(
                            num_blocks, max_context_len, scale, partition_size, workspace,
                            workspace_bytes, dtype, d_status, stream, key, value,
                            pa::KvCodes::kInt8, k_scale, v_scale);
+}
+
+extern "C" pa_status pa_paged_decode_fp8_rowscale(
+    void* out, const void* query, const void* k_cache, const void* v_cache, const float* k_scales,
+    const float* v_scales, const int32_t* block_tables, const int32_t* context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float scale, int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+    int32_t* d_status, pa_stream_t stream)
+{
+    if (k_scales == nullptr || v_scales == nullptr) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, nullptr, nullptr,
+                           pa::KvCodes::kE4m3, 1.f, 1.f, 0u, const_cast<float*>(k_scales),
+                           const_cast<float*>(v_scales));
+}
+
+extern "C" pa_status pa_paged_decode_fp8_rowscale_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, float* k_scales, float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, float scale, int32_t partition_size, void* workspace,
+    size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream)
+{
+    if (key == nullptr || value == nullptr || k_scales == nullptr || v_scales == nullptr)
+        return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, key, value,
+                           pa::KvCodes::kE4m3, 1.f, 1.f, 0u, k_scales, v_scales);
+}
+
+extern "C" pa_status pa_paged_decode_int8_rowscale(
+    void* out, const void* query, const void* k_cache, const void* v_cache, const float* k_scales,
+    const float* v_scales, const int32_t* block_tables, const int32_t* context_lens,
+    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks, int32_t max_context_len,
+    float scale, int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+    int32_t* d_status, pa_stream_t stream)
+{
+    if (k_scales == nullptr || v_scales == nullptr) return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, nullptr, nullptr,
+                           pa::KvCodes::kInt8, 1.f, 1.f, 0u, const_cast<float*>(k_scales),
+                           const_cast<float*>(v_scales));
+}
+
+extern "C" pa_status pa_paged_decode_int8_rowscale_append(
+    void* out, const void* query, const void* key, const void* value, void* k_cache,
+    void* v_cache, float* k_scales, float* v_scales, const int32_t* block_tables,
+    const int32_t* context_lens, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+    int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int64_t num_blocks,
+    int32_t max_context_len, float scale, int32_t partition_size, void* workspace,
+    size_t workspace_bytes, pa_dtype dtype, int32_t* d_status, pa_stream_t stream)
+{
+    if (key == nullptr || value == nullptr || k_scales == nullptr || v_scales == nullptr)
+        return PA_ERR_INVALID_ARG;
+    return pa::decode_impl(out, query, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                           num_q_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                           num_blocks, max_context_len, scale, partition_size, workspace,
+                           workspace_bytes, dtype, d_status, stream, key, value,
+                           pa::KvCodes::kInt8, 1.f, 1.f, 0u, k_scales, v_scales);
 }
 
 extern "C" pa_status pa_paged_decode_append(void* out, const void* query, const void* key,

@@ -26,6 +26,18 @@
 // 384-byte shared tile with stmatrix.trans / ldmatrix.  Scales: k_scale
 // folds into the score scale, v_scale into the output.  The query is
 // rounded once to fp16 (exact for fp16 queries).
+//
+// Row-scaled pools (ROWS = true): every (token, kv head) row has its own
+// fp32 scale, in pools [num_blocks][num_kv_heads][block_size] beside the
+// codes.  A block's B scales of K and of V for this kv head are one
+// contiguous run each; two more bulk copies bring them into the stage with
+// the tiles, counted on the same mbarrier.  The score of token t is
+// multiplied by its K row scale after the MMA.  The V row scale folds into
+// P: the B operand of O^T += V^T . P^T is p_t * (vs_t / R) in fp16, where R
+// is the largest V row scale seen so far by the warp -- a running reference
+// rescaled like the running max of the softmax -- so P stays in fp16's
+// normal range whatever the scales' magnitude; the epilogue multiplies the
+// output by R.
 #pragma once
 
 #include "decode_common.cuh"
@@ -33,7 +45,7 @@
 
 namespace pa {
 
-template <int D, int BS, int G>
+template <int D, int BS, int G, bool ROWS = false>
 struct Q8Shape {
     static constexpr int SLICES = BS / 16;           // 16-token MMA slices per block
     static constexpr int KW = D / 16;                // k-steps of S^T; 4-code words per K row per lane
@@ -49,7 +61,10 @@ struct Q8Shape {
     static constexpr int PT_BYTES = 8 * PT_STRIDE;
     static constexpr int WARP_BYTES = NSTAGE * STAGE;
     static constexpr int OFF_PT = kWarps * WARP_BYTES;
-    static constexpr int OFF_BARS = OFF_PT + kWarps * PT_BYTES;
+    // row scales of a stage: B floats of K, then B of V
+    static constexpr int SC_STAGE = ROWS ? 2 * BS * 4 : 0;
+    static constexpr int OFF_SC = OFF_PT + kWarps * PT_BYTES;
+    static constexpr int OFF_BARS = OFF_SC + kWarps * NSTAGE * SC_STAGE;
     // + a probe barrier per warp, + alignment slack
     static constexpr int SMEM_BYTES = OFF_BARS + kWarps * (NSTAGE + 1) * 8 + 1024;
     static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
@@ -122,6 +137,40 @@ __device__ __forceinline__ void append_row_warp_q8(
     fence_proxy_async_global();
 }
 
+// The same for row-scaled pools: the warp quantises the row with a scale of
+// its own (quantise_row_warp, as the row-scaled cache-write kernel does) and
+// stores the codes and the scale, then fences both for the copy engine.
+template <typename Codes, typename T, int D, int BS>
+__device__ __forceinline__ void append_row_warp_rowscale(
+    const T* __restrict__ new_key, const T* __restrict__ new_value, uint8_t* __restrict__ k_cache,
+    uint8_t* __restrict__ v_cache, float* __restrict__ k_scales, float* __restrict__ v_scales,
+    int s, int kvh, int num_kv_heads, int32_t pos, int32_t phys, int lane)
+{
+    const int64_t slot = static_cast<int64_t>(phys) * BS + pos % BS;
+    const int64_t src = (static_cast<int64_t>(s) * num_kv_heads + kvh) * D;
+    const int64_t dst = (slot * num_kv_heads + kvh) * D;
+    uint4 kx = make_uint4(0, 0, 0, 0), vx = make_uint4(0, 0, 0, 0);
+    if (lane < D / 8) {
+        kx = ld_nc_v4(new_key + src + lane * 8);
+        vx = ld_nc_v4(new_value + src + lane * 8);
+    }
+    float ks, vs;
+    const uint2 kc = quantise_row_warp<Codes, T, D>(kx, ks);
+    const uint2 vc = quantise_row_warp<Codes, T, D>(vx, vs);
+    if (lane < D / 8) {
+        *reinterpret_cast<uint2*>(k_cache + dst + lane * 8) = kc;
+        *reinterpret_cast<uint2*>(v_cache + dst + lane * 8) = vc;
+    }
+    if (lane == 0) {
+        const int64_t si = (static_cast<int64_t>(phys) * num_kv_heads + kvh) * BS + pos % BS;
+        k_scales[si] = ks;
+        v_scales[si] = vs;
+    }
+    fence_proxy_async_global();
+    __syncwarp();
+    fence_proxy_async_global();
+}
+
 template <int D>
 __device__ __forceinline__ void load_words(const unsigned char* tile, int row, int byte,
                                            uint32_t (&w)[4])
@@ -136,15 +185,16 @@ __device__ __forceinline__ void load_words(const unsigned char* tile, int row, i
 // One warp's share of a (sequence, kv head, partition) unit: Q^T fragments,
 // the O^T accumulators and the online-softmax state of heads 2*tig and
 // 2*tig + 1 (rows of N), and the code that consumes one block of K/V bytes.
-template <typename Codes, typename T, int D, int BS, int G>
+template <typename Codes, typename T, int D, int BS, int G, bool ROWS = false>
 struct Q8Warp {
-    using S = Q8Shape<D, BS, G>;
+    using S = Q8Shape<D, BS, G, ROWS>;
     int grp, tig;
     uint32_t pt_addr;               // this lane's row of the P^T staging tile
     uint32_t qb[S::KW][2];
     float o[S::MT][4];
     float m_run0, m_run1;           // running maxima (log2 units)
     float l_run0, l_run1;           // this lane's share of the exp-sums
+    float vref, vinv;               // ROWS: running reference of the V row scales, 1 / it
 
     __device__ __forceinline__ void reset()
     {
@@ -154,6 +204,7 @@ struct Q8Warp {
             for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
         m_run0 = m_run1 = -INFINITY;
         l_run0 = l_run1 = 0.f;
+        vref = vinv = 0.f;
     }
 
     // Q^T as B fragments, fp16: k-step j holds head grp's dims
@@ -178,9 +229,11 @@ struct Q8Warp {
         }
     }
 
-    // One block: kt / vt are its K and V byte tiles, nv its valid tokens.
+    // One block: kt / vt are its K and V byte tiles, nv its valid tokens;
+    // with ROWS, ksc / vsc its B row scales of K and of V.
     __device__ __forceinline__ void block(const unsigned char* kt, const unsigned char* vt, int nv,
-                                          float scale_log2)
+                                          float scale_log2, const float* ksc = nullptr,
+                                          const float* vsc = nullptr)
     {
 #pragma unroll 1
         for (int sl = 0; sl < S::SLICES; ++sl) {
@@ -208,10 +261,15 @@ struct Q8Warp {
                 }
             }
             // this lane: tokens grp (x0, x1) and grp + 8 (x2, x3); heads 2tig, 2tig + 1
-            const float x0 = grp < tv ? (sa[0] + sb[0]) * scale_log2 : -INFINITY;
-            const float x1 = grp < tv ? (sa[1] + sb[1]) * scale_log2 : -INFINITY;
-            const float x2 = grp + 8 < tv ? (sa[2] + sb[2]) * scale_log2 : -INFINITY;
-            const float x3 = grp + 8 < tv ? (sa[3] + sb[3]) * scale_log2 : -INFINITY;
+            float sla = scale_log2, slb = scale_log2;
+            if constexpr (ROWS) {               // each token's K row scale
+                sla *= ksc[t0 + grp];
+                slb *= ksc[t0 + grp + 8];
+            }
+            const float x0 = grp < tv ? (sa[0] + sb[0]) * sla : -INFINITY;
+            const float x1 = grp < tv ? (sa[1] + sb[1]) * sla : -INFINITY;
+            const float x2 = grp + 8 < tv ? (sa[2] + sb[2]) * slb : -INFINITY;
+            const float x3 = grp + 8 < tv ? (sa[3] + sb[3]) * slb : -INFINITY;
 
             // ---- online softmax per head over the slice's 16 tokens ----
             float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
@@ -226,15 +284,42 @@ struct Q8Warp {
             const float c0 = q8_exp2(m_run0 - ms0), c1 = q8_exp2(m_run1 - ms1);
             m_run0 = mn0;
             m_run1 = mn1;
-            // P rounds to fp16 for the tensor cores; the sums use the rounded values
-            const uint32_t pk0 = Elem<__half>::from_float2(q8_exp2(x0 - ms0), q8_exp2(x1 - ms1));
-            const uint32_t pk1 = Elem<__half>::from_float2(q8_exp2(x2 - ms0), q8_exp2(x3 - ms1));
-            const float2 r0 = Elem<__half>::to_float2(pk0), r1 = Elem<__half>::to_float2(pk1);
-            l_run0 = l_run0 * c0 + (r0.x + r1.x);
-            l_run1 = l_run1 * c1 + (r0.y + r1.y);
-            const float2 cc = make_float2(c0, c1);
+            uint32_t pk0, pk1;
+            float2 cc = make_float2(c0, c1);
+            if constexpr (ROWS) {
+                // V row scales of the slice's tokens relative to the running
+                // reference (rows past the context weigh 0); the reference
+                // grows to the slice's largest scale and rescales O like a
+                // change of the running max does
+                const float va = grp < tv ? vsc[t0 + grp] : 0.f;
+                const float vb = grp + 8 < tv ? vsc[t0 + grp + 8] : 0.f;
+                float vmax = fmaxf(va, vb);
+#pragma unroll
+                for (int m = 4; m < 32; m <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFullMask, vmax, m));
+                if (vmax > vref) {              // warp-uniform
+                    const float fr = vref / vmax;
+                    cc.x *= fr;
+                    cc.y *= fr;
+                    vref = vmax;
+                    vinv = 1.f / vmax;
+                }
+                const float p0 = q8_exp2(x0 - ms0), p1 = q8_exp2(x1 - ms1);
+                const float p2 = q8_exp2(x2 - ms0), p3 = q8_exp2(x3 - ms1);
+                l_run0 = l_run0 * c0 + (p0 + p2);
+                l_run1 = l_run1 * c1 + (p1 + p3);
+                const float ra = va * vinv, rb = vb * vinv;
+                pk0 = Elem<__half>::from_float2(p0 * ra, p1 * ra);
+                pk1 = Elem<__half>::from_float2(p2 * rb, p3 * rb);
+            } else {
+                // P rounds to fp16 for the tensor cores; the sums use the rounded values
+                pk0 = Elem<__half>::from_float2(q8_exp2(x0 - ms0), q8_exp2(x1 - ms1));
+                pk1 = Elem<__half>::from_float2(q8_exp2(x2 - ms0), q8_exp2(x3 - ms1));
+                const float2 r0 = Elem<__half>::to_float2(pk0), r1 = Elem<__half>::to_float2(pk1);
+                l_run0 = l_run0 * c0 + (r0.x + r1.x);
+                l_run1 = l_run1 * c1 + (r0.y + r1.y);
+            }
             // once the running maxima settle, most slices leave them unchanged
-            if (__any_sync(kFullMask, c0 != 1.f || c1 != 1.f)) {
+            if (__any_sync(kFullMask, cc.x != 1.f || cc.y != 1.f)) {
 #pragma unroll
                 for (int mt = 0; mt < S::MT; ++mt) {
                     float2 u = __fmul2_rn(make_float2(o[mt][0], o[mt][1]), cc);
@@ -348,7 +433,7 @@ struct Q8Warp {
 
 // One CTA: (kv head, partition, sequence).  The kernels below instantiate
 // it for each code format.
-template <typename Codes, typename T, int D, int BS, int G>
+template <typename Codes, typename T, int D, int BS, int G, bool ROWS>
 __device__ __forceinline__ void paged_decode_q8_cta(
     const CUtensorMap& tm_k, const CUtensorMap& tm_v, T* __restrict__ out,
     const T* __restrict__ query, const int32_t* __restrict__ block_tables,
@@ -357,10 +442,11 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     int32_t partition_size, int32_t max_parts, float* __restrict__ ws_o,
     float2* __restrict__ ws_ml, int32_t* d_status, int32_t lpt_seqs,
     const T* __restrict__ new_key, const T* __restrict__ new_value, uint8_t* __restrict__ k_cache,
-    uint8_t* __restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv, uint32_t probe_us)
+    uint8_t* __restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv, uint32_t probe_us,
+    float* __restrict__ k_scales, float* __restrict__ v_scales)
 {
     grid_dependency_wait();   // before any global access (see pa_common.cuh)
-    using S = Q8Shape<D, BS, G>;
+    using S = Q8Shape<D, BS, G, ROWS>;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -399,6 +485,7 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     const int append_blk = (new_key != nullptr && part == nparts - 1) ? (ctx - 1) / BS - blk_begin : -1;
 
     unsigned char* wbase = smem + warp * S::WARP_BYTES;
+    float* wsc = reinterpret_cast<float*>(smem + S::OFF_SC) + warp * S::NSTAGE * (S::SC_STAGE / 4);
     uint64_t* wbar = reinterpret_cast<uint64_t*>(smem + S::OFF_BARS) + warp * (S::NSTAGE + 1);
     if (lane == 0) {
 #pragma unroll
@@ -423,21 +510,35 @@ __device__ __forceinline__ void paged_decode_q8_cta(
         }
         const int phys = __shfl_sync(kFullMask, prod_tbl, k & 31);
         if (warp + kWarps * k == append_blk) {
-            if (phys >= 0 && static_cast<int64_t>(phys) < num_blocks)
-                append_row_warp_q8<Codes, T, D, BS>(new_key, new_value, k_cache, v_cache, s, kvh,
-                                              num_kv_heads, ctx - 1, phys, k_inv, v_inv, lane);
-            else if (lane == 0)
+            if (phys >= 0 && static_cast<int64_t>(phys) < num_blocks) {
+                if constexpr (ROWS)
+                    append_row_warp_rowscale<Codes, T, D, BS>(new_key, new_value, k_cache, v_cache,
+                                                              k_scales, v_scales, s, kvh,
+                                                              num_kv_heads, ctx - 1, phys, lane);
+                else
+                    append_row_warp_q8<Codes, T, D, BS>(new_key, new_value, k_cache, v_cache, s,
+                                                        kvh, num_kv_heads, ctx - 1, phys, k_inv,
+                                                        v_inv, lane);
+            } else if (lane == 0) {
                 status_or(d_status, PA_STATUS_BAD_SLOT);
+            }
         }
         if (lane == 0) {
             const int st = k % S::NSTAGE;
             const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
             fence_proxy_async_smem();
             if (ok) {
-                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE);
+                mbar_arrive_expect_tx(&wbar[st], 2u * S::TILE + static_cast<uint32_t>(S::SC_STAGE));
                 unsigned char* dst = wbase + st * S::STAGE;
                 tma_load_4d(dst, &tm_k, 0, kvh, 0, phys, &wbar[st]);
                 tma_load_4d(dst + S::TILE, &tm_v, 0, kvh, 0, phys, &wbar[st]);
+                if constexpr (ROWS) {
+                    // the block's B row scales of this kv head: one contiguous run each
+                    const int64_t so = (static_cast<int64_t>(phys) * num_kv_heads + kvh) * BS;
+                    float* sc = wsc + st * (S::SC_STAGE / 4);
+                    bulk_copy_g2s(sc, k_scales + so, BS * 4, &wbar[st]);
+                    bulk_copy_g2s(sc + BS, v_scales + so, BS * 4, &wbar[st]);
+                }
             } else {
                 status_or(d_status, PA_STATUS_BAD_BLOCK);
                 mbar_arrive_expect_tx(&wbar[st], 0u);
@@ -448,7 +549,7 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     for (int k = 0; k < prologue; ++k) issue(k);
     int issued = prologue;
 
-    Q8Warp<Codes, T, D, BS, G> w;
+    Q8Warp<Codes, T, D, BS, G, ROWS> w;
     w.grp = lane >> 2;
     w.tig = lane & 3;
     w.pt_addr = smem_u32(smem + S::OFF_PT + warp * S::PT_BYTES) + (lane & 7) * S::PT_STRIDE +
@@ -475,7 +576,8 @@ __device__ __forceinline__ void paged_decode_q8_cta(
         const int t0 = tok_begin + (warp + kWarps * k) * BS;
         const int nv = ok ? min(BS, tok_end - t0) : 0;
         const unsigned char* kt = wbase + st * S::STAGE;
-        w.block(kt, kt + S::TILE, nv, scale_log2);
+        const float* sc = wsc + st * (S::SC_STAGE / 4);
+        w.block(kt, kt + S::TILE, nv, scale_log2, sc, sc + BS);
         __syncwarp();   // every lane is done with this stage
         if (issued < nk) issue(issued++);
     }
@@ -490,7 +592,7 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     float* epi_o = reinterpret_cast<float*>(smem);   // [warp][g][D]
     float* epi_m = epi_o + kWarps * G * D;
     float* epi_l = epi_m + kWarps * G;
-    w.store(epi_o, epi_m, epi_l, warp, v_scale);
+    w.store(epi_o, epi_m, epi_l, warp, ROWS ? w.vref : v_scale);
     __syncthreads();
     merge_warps_and_store<T, D, G>(epi_o, epi_m, epi_l, out, ws_o, ws_ml, s, kvh, part, nparts,
                                    num_q_heads, max_parts);
@@ -506,25 +608,25 @@ __device__ __forceinline__ void paged_decode_q8_cta(
         int32_t *d_status, int32_t lpt_seqs, const T *__restrict__ new_key,                    \
         const T *__restrict__ new_value, uint8_t *__restrict__ k_cache,                        \
         uint8_t *__restrict__ v_cache, int32_t num_kv_heads, float k_inv, float v_inv,          \
-        uint32_t probe_us
+        uint32_t probe_us, float *__restrict__ k_scales, float *__restrict__ v_scales
 #define PA_Q8_KERNEL_ARGS                                                                       \
     tm_k, tm_v, out, query, block_tables, context_lens, num_q_heads, max_blocks_per_seq,       \
         num_blocks, max_context_len, scale_log2, v_scale, partition_size, max_parts, ws_o,     \
         ws_ml, d_status, lpt_seqs, new_key, new_value, k_cache, v_cache, num_kv_heads, k_inv,  \
-        v_inv, probe_us
+        v_inv, probe_us, k_scales, v_scales
 
-// e4m3 pools
-template <typename T, int D, int BS, int G>
+// e4m3 pools (ROWS: with row-scale pools; else one scale per pool)
+template <typename T, int D, int BS, int G, bool ROWS>
 __global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(PA_Q8_KERNEL_PARAMS)
 {
-    paged_decode_q8_cta<E4m3Codes, T, D, BS, G>(PA_Q8_KERNEL_ARGS);
+    paged_decode_q8_cta<E4m3Codes, T, D, BS, G, ROWS>(PA_Q8_KERNEL_ARGS);
 }
 
 // int8 pools
-template <typename T, int D, int BS, int G>
+template <typename T, int D, int BS, int G, bool ROWS>
 __global__ void __launch_bounds__(kThreads, 4) paged_decode_int8_kernel(PA_Q8_KERNEL_PARAMS)
 {
-    paged_decode_q8_cta<Int8Codes, T, D, BS, G>(PA_Q8_KERNEL_ARGS);
+    paged_decode_q8_cta<Int8Codes, T, D, BS, G, ROWS>(PA_Q8_KERNEL_ARGS);
 }
 
 #undef PA_Q8_KERNEL_PARAMS

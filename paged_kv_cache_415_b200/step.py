@@ -44,9 +44,17 @@ _QUANTISED_CALLS = {
 class DecodeStep:
     def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor, num_seqs: int,
                  num_q_heads: int, max_context_len: int, partition_size: int = 0,
-                 k_scale: float = 1.0, v_scale: float = 1.0):
+                 k_scale: float = 1.0, v_scale: float = 1.0, k_scales: torch.Tensor = None,
+                 v_scales: torch.Tensor = None):
+        """k_scales / v_scales: fp32 row-scale pools [num_blocks][Hkv][B] of
+        one-byte code pools (one scale per (token, kv head) row; the
+        _rowscale calls), or None for one scale per pool (k_scale, v_scale)."""
         self.k_cache, self.v_cache = k_cache, v_cache
+        self.k_scales, self.v_scales = k_scales, v_scales
         names = _QUANTISED_CALLS.get(k_cache.dtype)
+        if names is not None and k_scales is not None:
+            names = tuple(n.replace("_append", "_rowscale_append") if n.endswith("_append")
+                          else n + "_rowscale" for n in names)
         self.quantised = None if names is None else tuple(getattr(B, n) for n in names)
         self.k_scale, self.v_scale = float(k_scale), float(v_scale)
         num_blocks, self.block_size, self.num_kv_heads, self.head_dim = k_cache.shape
@@ -85,6 +93,26 @@ class DecodeStep:
             out = torch.empty_like(query)
         mcl = self.max_context_len if max_context_len is None else max_context_len
         write_needed = slot_mapping is not None and slot_mapping.shape[0] > 0
+        if self.quantised is not None and self.k_scales is not None:
+            write, decode, decode_append = self.quantised
+            ks, vs = self.k_scales, self.v_scales
+            if block_mapping is not None and block_mapping.shape[0] > 0:
+                with _range("pa.copy_blocks"):
+                    B.pa_copy_block_scales(ks, vs, block_mapping, self.d_status, stream)
+            if fused_append:
+                with _range("pa.decode"):
+                    decode_append(out, query, new_key, new_value, self.k_cache, self.v_cache, ks,
+                                  vs, block_tables, context_lens, mcl, scale, self.partition_size,
+                                  self.workspace, self.d_status, stream)
+                return out
+            if write_needed:
+                with _range("pa.cache_write"):
+                    write(new_key, new_value, self.k_cache, self.v_cache, ks, vs, slot_mapping,
+                          self.d_status, stream)
+            with _range("pa.decode"):
+                decode(out, query, self.k_cache, self.v_cache, ks, vs, block_tables, context_lens,
+                       mcl, scale, self.partition_size, self.workspace, self.d_status, stream)
+            return out
         if self.quantised is not None:
             write, decode, decode_append = self.quantised
             if fused_append:

@@ -252,3 +252,44 @@ def test_no_fallback_without_the_library(tmp_path):
                              text=True, timeout=300)
         assert res.returncode != 0
         assert "libpa.so" in res.stderr and "ImportError" in res.stderr, res.stderr[-500:]
+
+
+def test_rowscale_calls_check_their_arguments(pa):
+    """The row-scaled calls refuse, before any device work: missing or
+    misaligned scale pools, block size 8 in the decode (whole 16-token
+    slices only), a bad query type.  pa_copy_blocks takes scale pools as
+    PA_DTYPE_F32 with head_dim 1 only."""
+    L = pa.LIB
+    w = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 128, 16, 64, 0, None, None]
+    for fn in (L.pa_reshape_and_cache_fp8_rowscale, L.pa_reshape_and_cache_int8_rowscale):
+        bad = list(w); bad[4] = None
+        assert fn(*bad) == 1                                   # no K scale pool
+        bad = list(w); bad[5] = FAKE + 4
+        assert fn(*bad) == 1                                   # V scales not 16-byte aligned
+        bad = list(w); bad[9] = 96
+        assert fn(*bad) == 2                                   # head_dim 96
+        bad = list(w); bad[7] = -1
+        assert fn(*bad) == 1
+        bad = list(w); bad[7] = 0
+        assert fn(*bad) == 0                                   # nothing to write
+    d = [FAKE] * 8 + [4, 8, 2, 128, 16, 8, 64, 100, 0.1, 0, None, 0, 0, None, None]
+    for fn in (L.pa_paged_decode_fp8_rowscale, L.pa_paged_decode_int8_rowscale):
+        bad = list(d); bad[4] = None
+        assert fn(*bad) == 1
+        bad = list(d); bad[5] = FAKE + 8
+        assert fn(*bad) == 1
+        bad = list(d); bad[12] = 8
+        assert fn(*bad) == 2                                   # block size 8
+        bad = list(d); bad[20] = 7
+        assert fn(*bad) == 2                                   # unknown query type
+    a = [FAKE] * 10 + [4, 8, 2, 128, 16, 8, 64, 100, 0.1, 0, None, 0, 0, None, None]
+    for fn in (L.pa_paged_decode_fp8_rowscale_append, L.pa_paged_decode_int8_rowscale_append):
+        bad = list(a); bad[2] = None
+        assert fn(*bad) == 1                                   # no new keys
+        bad = list(a); bad[7] = None
+        assert fn(*bad) == 1                                   # no V scale pool
+    cp = L.pa_copy_blocks
+    assert cp(FAKE, FAKE, FAKE, 0, 8, 1, 16, 64, pa.PA_DTYPE_F32, None, None) == 0
+    assert cp(FAKE, FAKE, FAKE, 2, 8, 2, 16, 64, pa.PA_DTYPE_F32, None, None) == 2   # head_dim 2
+    assert cp(FAKE, FAKE, FAKE, 2, 8, 1, 12, 64, pa.PA_DTYPE_F32, None, None) == 2   # block 12
+    assert cp(FAKE, FAKE, FAKE, 2, 8, 1, 16, 64, pa.PA_DTYPE_F16, None, None) == 2   # 16-bit, D 1

@@ -31,6 +31,24 @@ def test_code_workload_modes(kv, np_dtype, label):
     assert full["kv"] * 2 == base["kv"]
 
 
+@pytest.mark.parametrize("kv", ["fp8-rows", "int8-rows"])
+def test_rowscale_workload_mode(kv):
+    """--kv-dtype fp8-rows / int8-rows: code pools plus fp32 row-scale pools
+    [num_blocks][Hkv][B] (NaN where no history token sits); the byte model
+    adds 4 bytes per (token, kv head) row and per written row."""
+    wl = bench.make_workload("mistral7b", seqs=3, kv_dtype=kv)
+    assert wl.extra["rowscale"] and wl.extra["kv_dtype"] == kv[:-5]
+    nb, b, h = wl.num_blocks, wl.block_size, wl.num_kv_heads
+    assert wl.extra["k_scales"].shape == (nb, h, b) and wl.extra["k_scales"].dtype == np.float32
+    assert "one scale per (token, kv head) row" in bench.workload_config(wl, 0, "")["workload"]
+    plain = bm.step_bytes(bench.make_workload("mistral7b", seqs=3, kv_dtype=kv[:-5]))
+    rows = bm.step_bytes(wl)
+    assert rows["kv"] - plain["kv"] == int(wl.context_lens.sum()) * h * 4 * 2
+    assert rows["append"] - plain["append"] == wl.num_new_tokens * h * 4 * 2
+    st = bench.OracleStep(wl)
+    assert st.bytes == rows["total"] and st.run() > 0.0
+
+
 def test_oracle_step_counts_the_step_bytes():
     """The CPU leg times the oracle on the same step the GPU runs and
     counts the same algorithmic bytes (all sequences, 16-bit and both code

@@ -43,13 +43,16 @@ def paged_waste_slots(context_len: int, block_size: int) -> int:
 
 
 def decode_bytes(ctx: np.ndarray, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                 block_size: int, elem_bytes: int, kv_elem_bytes: int | None = None) -> dict:
+                 block_size: int, elem_bytes: int, kv_elem_bytes: int | None = None,
+                 row_scale_bytes: int = 0) -> dict:
     """Algorithmic bytes of the attention part of one decode step
     (kv_elem_bytes: bytes of a cached K/V element when it differs from the
-    query's, e.g. 1 for e4m3 pools)."""
+    query's, e.g. 1 for e4m3 pools; row_scale_bytes: bytes of the scale each
+    (token, kv head) row carries in row-scaled pools, 4)."""
     ctx = np.asarray(ctx, dtype=np.int64)
     s = ctx.shape[0]
-    row = num_kv_heads * head_dim * (elem_bytes if kv_elem_bytes is None else kv_elem_bytes)
+    row = num_kv_heads * (head_dim * (elem_bytes if kv_elem_bytes is None else kv_elem_bytes)
+                          + row_scale_bytes)
     kv = int(ctx.sum()) * row * 2
     q = s * num_q_heads * head_dim * elem_bytes
     out = q
@@ -66,15 +69,22 @@ def kv_elem_bytes(wl) -> int:
     return 1 if wl.extra.get("kv_dtype") in ("fp8", "int8") else ELEM_BYTES[wl.dtype]
 
 
+def row_scale_bytes(wl) -> int:
+    """Bytes of the scale every (token, kv head) row carries: 4 for
+    row-scaled one-byte pools, else 0."""
+    return 4 if wl.extra.get("rowscale") else 0
+
+
 def step_bytes(wl) -> dict:
     """Algorithmic bytes of a whole decode step of a workload (attention,
     appended tokens, copy-on-write copies)."""
     e = ELEM_BYTES[wl.dtype]
     ekv = kv_elem_bytes(wl)
+    rs = row_scale_bytes(wl)
     att = decode_bytes(wl.context_lens, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
-                       wl.block_size, e, ekv)
+                       wl.block_size, e, ekv, rs)
     row_in = wl.num_kv_heads * wl.head_dim * e
-    row = wl.num_kv_heads * wl.head_dim * ekv
+    row = wl.num_kv_heads * (wl.head_dim * ekv + rs)
     t = wl.num_new_tokens
     append = 2 * t * row_in + 2 * t * row + 8 * t   # K,V read + written, slot ids
     blk = wl.block_size * row
@@ -87,7 +97,7 @@ def step_bytes(wl) -> dict:
 def unique_kv_bytes(wl) -> int:
     """K/V bytes of the distinct physical blocks the step reads (shared
     blocks counted once), for workloads with block sharing."""
-    row = wl.num_kv_heads * wl.head_dim * kv_elem_bytes(wl)
+    row = wl.num_kv_heads * (wl.head_dim * kv_elem_bytes(wl) + row_scale_bytes(wl))
     seen = {}
     for s in range(wl.num_seqs):
         c = int(wl.context_lens[s])

@@ -237,6 +237,38 @@ def with_int8_pools(wl: DecodeWorkload, seed: int, k_scale: float = 1.0 / 64.0,
     return _with_code_pools(wl, seed, "int8", int8_codes, INT8_POISON, np.int8, k_scale, v_scale)
 
 
+def with_rowscale_pools(wl: DecodeWorkload, kv_dtype: str, seed: int) -> DecodeWorkload:
+    """A copy of a make_decode workload with one-byte code pools (as
+    with_code_pools) and fp32 row-scale pools [num_blocks][Hkv][B]: each
+    history row's scale is drawn uniform in [0.5, 2] times a per-kv-head
+    magnitude spread geometrically over [1e-2, 1e2], divided by the format's
+    top code (448 or 127), so the kv heads differ in magnitude by 10^4.  Every
+    scale of a slot without a history token is NaN (reading one poisons the
+    output).  The step's new tokens stay N(0,1) in the 16-bit type.
+    extra: kv_dtype, rowscale = True, k_scales, v_scales."""
+    out = with_code_pools(wl, kv_dtype, seed)
+    rng = np.random.Generator(np.random.PCG64(seed + 1))
+    nb, b, h = wl.num_blocks, wl.block_size, wl.num_kv_heads
+    top = {"fp8": 448.0, "int8": 127.0}[kv_dtype]
+    mags = np.geomspace(1e-2, 1e2, h) if h > 1 else np.ones(1)
+    history = np.zeros((nb, b), bool)
+    new = set(int(x) for x in wl.slot_mapping if x >= 0)
+    for s in range(wl.num_seqs):
+        c = int(wl.context_lens[s])
+        pos = np.arange(c, dtype=np.int64)
+        slots = wl.block_tables[s].astype(np.int64)[pos // b] * b + pos % b
+        slots = np.asarray([x for x in slots.tolist() if x not in new], dtype=np.int64)
+        history[slots // b, slots % b] = True
+    scales = []
+    for _ in range(2):
+        sc = (rng.uniform(0.5, 2.0, (nb, h, b)) * mags[None, :, None] / top).astype(np.float32)
+        sc[np.broadcast_to(~history[:, None, :], sc.shape)] = np.nan
+        scales.append(np.ascontiguousarray(sc))
+    out.name = f"{wl.name}-{kv_dtype}-rows"
+    out.extra = dict(out.extra, rowscale=True, k_scales=scales[0], v_scales=scales[1])
+    return out
+
+
 def with_code_pools(wl: DecodeWorkload, kv_dtype: str, seed: int) -> DecodeWorkload:
     """with_fp8_pools or with_int8_pools by name ("fp8" / "int8")."""
     return {"fp8": with_fp8_pools, "int8": with_int8_pools}[kv_dtype](wl, seed=seed)
