@@ -15,7 +15,12 @@
 //
 //   widen4(w, lo, hi)  the four codes of w as two packed fp16 pairs:
 //                      lo = (code 0, code 1), hi = (code 2, code 3), the
-//                      lower-addressed code in the low half.
+//                      lower-addressed code in the low half, each value
+//                      plus kBias: decode(code) + kBias, exact in fp16.
+//   kBias              0 for e4m3; 1152 for int8, whose widening is a byte
+//                      permute that yields 1152 + c (the decode kernels
+//                      remove the bias once per head instead of once per
+//                      pair of codes).
 //   encode2(a, b)      two fp32 values (already times 1 / scale) as two
 //                      codes in the low 16 bits, a in the low byte.
 //   kMax               the largest code magnitude (448 or 127): the code a
@@ -32,6 +37,7 @@ namespace pa {
 
 struct E4m3Codes {
     static constexpr float kMax = 448.0f;
+    static constexpr float kBias = 0.0f;
 
     static __device__ __forceinline__ void widen4(uint32_t w, uint32_t& lo, uint32_t& hi)
     {
@@ -52,19 +58,17 @@ struct E4m3Codes {
 
 struct Int8Codes {
     static constexpr float kMax = 127.0f;
+    static constexpr float kBias = 1152.0f;
 
     // Exponent-field construction: with 0x64 as the high byte, an fp16 is
     // 1024 + (low byte), since its unit in [1024, 2048) is 1.  Flipping the
     // sign bit of a code c gives the byte c + 128, so the fp16 0x64:(c + 128)
-    // is 1152 + c, and subtracting 1152 leaves c.  Both steps are exact.
+    // is exactly 1152 + c.  The bias is left in (kBias).
     static __device__ __forceinline__ void widen4(uint32_t w, uint32_t& lo, uint32_t& hi)
     {
-        const uint32_t u = w ^ 0x80808080u;                        // c + 128 in every byte
-        const uint32_t lo_b = __byte_perm(u, 0x64646464u, 0x5140);  // [0x64 u1 0x64 u0]
-        const uint32_t hi_b = __byte_perm(u, 0x64646464u, 0x5342);  // [0x64 u3 0x64 u2]
-        constexpr uint32_t kBias = 0x64806480u;                    // fp16 pair (1152, 1152)
-        asm("sub.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(lo_b), "r"(kBias));
-        asm("sub.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(hi_b), "r"(kBias));
+        const uint32_t u = w ^ 0x80808080u;                   // c + 128 in every byte
+        lo = __byte_perm(u, 0x64646464u, 0x5140);              // [0x64 u1 0x64 u0]
+        hi = __byte_perm(u, 0x64646464u, 0x5342);              // [0x64 u3 0x64 u2]
     }
 
     static __device__ __forceinline__ uint32_t encode1(float x)

@@ -18,8 +18,12 @@
 //
 // Each lane reads its A fragments straight from the byte tile, pairs codes
 // with byte permutes where two tokens share a register (V^T), and widens
-// them exactly to fp16 (Codes::widen4: one cvt per pair for e4m3, a byte
-// permute and one packed subtract per pair for int8).  The contraction index
+// them exactly to fp16 (Codes::widen4: one cvt per pair for e4m3; for int8
+// a byte permute per pair that yields 1152 + c).  The int8 bias is removed
+// once per head, not per code: every score of head h carries 1152 * sum_d
+// q[h][d] (subtracted from the scores; the sum is taken once per CTA from
+// the fp16 query the MMA reads), and the output carries 1152 * sum_t p_t
+// (subtracted in the epilogue, from the sum of the P values the MMA read).  The contraction index
 // may be permuted freely as long as both operands follow it, so every lane
 // reads whole 16-byte runs of one token row.  P moves from the accumulator
 // layout (tokens x heads) to the B layout (heads x tokens) through a
@@ -195,6 +199,8 @@ struct Q8Warp {
     float m_run0, m_run1;           // running maxima (log2 units)
     float l_run0, l_run1;           // this lane's share of the exp-sums
     float vref, vinv;               // ROWS: running reference of the V row scales, 1 / it
+    float e0, e1;                   // kBias * sum_d q[h][d] of heads 2tig, 2tig + 1
+    float ps_run0, ps_run1;         // ROWS with a bias: sum of the P values fed to the MMA
 
     __device__ __forceinline__ void reset()
     {
@@ -205,6 +211,8 @@ struct Q8Warp {
         m_run0 = m_run1 = -INFINITY;
         l_run0 = l_run1 = 0.f;
         vref = vinv = 0.f;
+        e0 = e1 = 0.f;
+        ps_run0 = ps_run1 = 0.f;
     }
 
     // Q^T as B fragments, fp16: k-step j holds head grp's dims
@@ -226,6 +234,21 @@ struct Q8Warp {
             }
             qb[j][0] = b0;
             qb[j][1] = b1;
+        }
+        if constexpr (Codes::kBias != 0.f) {
+            // sum of head grp's fp16 query (the values the MMA reads), then
+            // the bias every score of heads 2tig and 2tig + 1 carries
+            float qs = 0.f;
+#pragma unroll
+            for (int j = 0; j < S::KW; ++j) {
+                const float2 a = Elem<__half>::to_float2(qb[j][0]);
+                const float2 b = Elem<__half>::to_float2(qb[j][1]);
+                qs += (a.x + a.y) + (b.x + b.y);
+            }
+            qs += __shfl_xor_sync(kFullMask, qs, 1);
+            qs += __shfl_xor_sync(kFullMask, qs, 2);
+            e0 = Codes::kBias * __shfl_sync(kFullMask, qs, 8 * tig);
+            e1 = Codes::kBias * __shfl_sync(kFullMask, qs, 8 * tig + 4);
         }
     }
 
@@ -266,10 +289,10 @@ struct Q8Warp {
                 sla *= ksc[t0 + grp];
                 slb *= ksc[t0 + grp + 8];
             }
-            const float x0 = grp < tv ? (sa[0] + sb[0]) * sla : -INFINITY;
-            const float x1 = grp < tv ? (sa[1] + sb[1]) * sla : -INFINITY;
-            const float x2 = grp + 8 < tv ? (sa[2] + sb[2]) * slb : -INFINITY;
-            const float x3 = grp + 8 < tv ? (sa[3] + sb[3]) * slb : -INFINITY;
+            const float x0 = grp < tv ? ((sa[0] + sb[0]) - e0) * sla : -INFINITY;
+            const float x1 = grp < tv ? ((sa[1] + sb[1]) - e1) * sla : -INFINITY;
+            const float x2 = grp + 8 < tv ? ((sa[2] + sb[2]) - e0) * slb : -INFINITY;
+            const float x3 = grp + 8 < tv ? ((sa[3] + sb[3]) - e1) * slb : -INFINITY;
 
             // ---- online softmax per head over the slice's 16 tokens ----
             float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
@@ -310,6 +333,11 @@ struct Q8Warp {
                 const float ra = va * vinv, rb = vb * vinv;
                 pk0 = Elem<__half>::from_float2(p0 * ra, p1 * ra);
                 pk1 = Elem<__half>::from_float2(p2 * rb, p3 * rb);
+                if constexpr (Codes::kBias != 0.f) {   // the P values the MMA reads
+                    const float2 f0 = Elem<__half>::to_float2(pk0), f1 = Elem<__half>::to_float2(pk1);
+                    ps_run0 = ps_run0 * cc.x + (f0.x + f1.x);
+                    ps_run1 = ps_run1 * cc.y + (f0.y + f1.y);
+                }
             } else {
                 // P rounds to fp16 for the tensor cores; the sums use the rounded values
                 pk0 = Elem<__half>::from_float2(q8_exp2(x0 - ms0), q8_exp2(x1 - ms1));
@@ -403,6 +431,30 @@ struct Q8Warp {
         for (int m = 4; m < 32; m <<= 1) {
             l_run0 += __shfl_xor_sync(kFullMask, l_run0, m);
             l_run1 += __shfl_xor_sync(kFullMask, l_run1, m);
+        }
+        if constexpr (Codes::kBias != 0.f) {
+            // every V value the MMA read carried the bias: remove kBias times
+            // the sum of the P values it was weighted with (the exp-sum itself
+            // for one scale per pool, whose sum adds exactly those values)
+            float b0 = l_run0, b1 = l_run1;
+            if constexpr (ROWS) {
+#pragma unroll
+                for (int m = 4; m < 32; m <<= 1) {
+                    ps_run0 += __shfl_xor_sync(kFullMask, ps_run0, m);
+                    ps_run1 += __shfl_xor_sync(kFullMask, ps_run1, m);
+                }
+                b0 = ps_run0;
+                b1 = ps_run1;
+            }
+            b0 *= Codes::kBias;
+            b1 *= Codes::kBias;
+#pragma unroll
+            for (int mt = 0; mt < S::MT; ++mt) {
+                o[mt][0] -= b0;
+                o[mt][1] -= b1;
+                o[mt][2] -= b0;
+                o[mt][3] -= b1;
+            }
         }
         const int h0 = 2 * tig, h1 = 2 * tig + 1;
 #pragma unroll

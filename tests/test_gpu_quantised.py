@@ -374,3 +374,26 @@ def test_code_fused_append_bad_slot_is_flagged(codes):
                             wl.block_size, wl.dtype, wl.extra["k_scale"], wl.extra["v_scale"])
     assert np.array_equal(dev.k_cache.cpu().numpy(), kc)
     assert np.array_equal(dev.v_cache.cpu().numpy(), vc)
+
+
+# ---- int8 pools: the widening leaves a bias of 1152 that the kernel removes ------
+
+@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("partition", [0, 8192])
+def test_int8_bias_removal_under_stress(group, partition):
+    """int8 codes widen to 1152 + c; the kernel subtracts 1152 * sum(q) from
+    every score and 1152 * sum(p) from the output.  Stress both: scales of 1
+    (codes are the values, up to +-127), a query that is positive in every
+    dim (sum(q) as large as it gets), contexts up to 8192 tokens and, with an
+    8192-token partition, one warp accumulating 128 blocks."""
+    hkv = 2
+    wl = gen.make_decode("int8-bias", seed=4150 + 90 + group, dtype="f16",
+                         context_lens=np.array([8192, 3000, 1], np.int32),
+                         num_q_heads=hkv * group, num_kv_heads=hkv, head_dim=128, block_size=16,
+                         num_blocks=800, scale=1.0 / 128.0)
+    q = np.abs(wl.query.view(np.float16).astype(np.float32)) * 2.0 + 0.5
+    wl.query = gen.f32_to_bits(q, "f16")
+    wl = gen.with_code_pools(wl, "int8", seed=4150 + 91)
+    wl.extra["k_scale"] = 1.0
+    wl.extra["v_scale"] = 1.0
+    _parity(wl, partition, f"int8 bias stress G={group} P={partition}")
