@@ -133,3 +133,29 @@ def test_reference_arm_under_torchrun_prints_once():
     assert res.returncode == 0, res.stderr[-2000:]
     lines = _json_lines(res.stdout)
     assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_sharing_workload_roofline_counts_unique_bytes():
+    """A workload whose sequences share stored blocks (the beams of a prompt)
+    gets its roofline fraction on unique K/V bytes -- the blocks the step
+    must read at least once -- and reports the referenced bytes beside
+    them; other workloads have no referenced figure."""
+    wl = bench.make_workload("beam_search", seqs=8)
+    g = bench.GpuStep.__new__(bench.GpuStep)
+    g.wl, g.fused = wl, False
+    unique, referenced = g.roofline_bytes()
+    step = bm.step_bytes(wl)
+    assert referenced == step["attention"]
+    assert unique == step["attention"] - step["kv"] + bm.unique_kv_bytes(wl)
+    assert unique < referenced
+    g.wl = bench.make_workload("llama7b", seqs=3)
+    assert g.roofline_bytes() == (bm.step_bytes(g.wl)["attention"], None)
+
+
+def test_clock_records_of_both_regions_merge():
+    a = {"sm_mhz": 1965, "sm_max_mhz": 1965, "reasons": [], "samples": 3, "source": "nvml"}
+    b = {"sm_mhz": 1950, "sm_max_mhz": 1965, "reasons": ["sw_power_cap"], "samples": 40,
+         "source": "nvml"}
+    m = bench.merge_clocks(a, b)
+    assert m["sm_mhz"] == 1950 and m["samples"] == 43 and m["reasons"] == ["sw_power_cap"]
+    assert bench.merge_clocks(a, {"samples": 0}) == a
