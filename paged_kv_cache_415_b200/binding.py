@@ -482,8 +482,14 @@ def _addr(t) -> int:
 
 def pa_swap_blocks(src_k, src_v, dst_k, dst_v, block_mapping, d_status=None, stream=None) -> None:
     """Whole-block copies src -> dst between two pools (one of them usually
-    a pinned host tensor): block_mapping int64 [P][2] of (src, dst) ids."""
-    src_nb, block_size, hkv, d = src_k.shape
+    a pinned host tensor): block_mapping int64 [P][2] of (src, dst) ids.
+    Pools are [num_blocks][B][Hkv][D], or fp32 row-scale pools
+    [num_blocks][Hkv][B] (moved as PA_DTYPE_F32 with head_dim 1)."""
+    if src_k.dim() == 3:
+        src_nb, hkv, block_size = src_k.shape
+        d = 1
+    else:
+        src_nb, block_size, hkv, d = src_k.shape
     dst_nb = dst_k.shape[0]
     _check("pa_swap_blocks", LIB.pa_swap_blocks(
         _addr(src_k), _addr(src_v), _addr(dst_k), _addr(dst_v), _addr(block_mapping),

@@ -241,3 +241,29 @@ def test_rowscale_full_size(fmt, name):
     _same_pools(dev, kc, vc, ks, vs, f"{name} {fmt} rows")
     ref, _ = _oracle_decode(wl, kc, vc, ks, vs)
     assert_close(to_f64(out), ref, f"{name} {fmt} rows, every row")
+
+
+def test_scale_pools_swap_to_host_and_back():
+    """Eviction of row-scaled blocks moves their scales too: pa_swap_blocks
+    with PA_DTYPE_F32 pools, device -> pinned host -> device, bit for bit
+    against the oracle's swap."""
+    from paged_kv_cache_415_b200 import binding as B
+    rng = np.random.Generator(np.random.PCG64(45))
+    ks = rng.standard_normal((10, 8, 16)).astype(np.float32)
+    vs = rng.standard_normal((10, 8, 16)).astype(np.float32)
+    dks, dvs = torch.from_numpy(ks).cuda(), torch.from_numpy(vs).cuda()
+    hk = torch.zeros((4, 8, 16), dtype=torch.float32).pin_memory()
+    hv = torch.zeros((4, 8, 16), dtype=torch.float32).pin_memory()
+    out_pairs = np.array([[2, 0], [7, 3]], np.int64)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    B.pa_swap_blocks(dks, dvs, hk, hv, torch.from_numpy(out_pairs).cuda(), status)
+    torch.cuda.synchronize()
+    ok_k, ok_v = np.zeros((4, 8, 16), np.float32), np.zeros((4, 8, 16), np.float32)
+    assert oracle.swap_blocks(ks, vs, ok_k, ok_v, out_pairs) == 0
+    assert np.array_equal(hk.numpy(), ok_k) and np.array_equal(hv.numpy(), ok_v)
+    back = np.array([[0, 5], [3, 9]], np.int64)
+    B.pa_swap_blocks(hk, hv, dks, dvs, torch.from_numpy(back).cuda(), status)
+    torch.cuda.synchronize()
+    assert oracle.swap_blocks(ok_k, ok_v, ks, vs, back) == 0
+    assert int(status.item()) == 0
+    assert np.array_equal(dks.cpu().numpy(), ks) and np.array_equal(dvs.cpu().numpy(), vs)
