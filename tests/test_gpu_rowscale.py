@@ -4,10 +4,11 @@ on the GPU against the oracle, for e4m3 and int8 codes.
   * the quantising write: codes and scales bit for bit over the whole pools
     (untouched bytes included), on rows whose kv heads differ in magnitude by
     10^4, with an all-zero row, padding tokens and a slot past the pool;
-  * the decode: within the tolerance of the 16-bit path,
-    |gpu - oracle| <= 2e-3 + 1e-2 |oracle|, on pools whose row scales span
-    four orders of magnitude across kv heads, with NaN scales and codes in
-    every slot the kernel must not read;
+  * the decode: within the tolerance of the 16-bit path with its absolute
+    part scaled by each output row's magnitude (assert_close_rows:
+    |gpu - oracle| <= 2e-3 max_d |oracle row| + 1e-2 |oracle|), on pools
+    whose row scales span four orders of magnitude across kv heads, with
+    NaN scales and codes in every slot the kernel must not read;
   * the decode with the fused write: pools bit for bit and every output row;
   * full-size Mistral-7B and long-context workloads in the benchmark's launch
     configuration: pools bit for bit and every output row;
@@ -19,7 +20,7 @@ import torch
 
 import oracle
 from tests import oracle_pins
-from tests.gpu_utils import assert_close, to_dev, to_f64
+from tests.gpu_utils import assert_close_rows, to_dev, to_f64
 from workloads import generators as gen
 
 pytestmark = pytest.mark.gpu
@@ -168,7 +169,7 @@ def test_rowscale_decode(fmt, group, head_dim, block_size, dtype, partition):
     ref, st2 = _oracle_decode(wl, kc, vc, ks, vs)
     assert dev.status() == 0 and st == 0 and st2 == 0
     _same_pools(dev, kc, vc, ks, vs, "pools after the write")
-    assert_close(to_f64(out), ref, f"{fmt} rows G={group} D={head_dim} B={block_size} P={partition}")
+    assert_close_rows(to_f64(out), ref, f"{fmt} rows G={group} D={head_dim} B={block_size} P={partition}")
 
 
 @pytest.mark.parametrize("fmt", CODES)
@@ -181,7 +182,7 @@ def test_rowscale_fused_append(fmt, partition):
     ref, _ = _oracle_decode(wl, kc, vc, ks, vs)
     assert dev.status() == 0 and st == 0
     _same_pools(dev, kc, vc, ks, vs, "pools after the fused write")
-    assert_close(to_f64(out), ref, f"{fmt} rows fused append P={partition}")
+    assert_close_rows(to_f64(out), ref, f"{fmt} rows fused append P={partition}")
 
 
 @pytest.mark.parametrize("fmt", CODES)
@@ -201,7 +202,7 @@ def test_rowscale_heads_of_very_different_magnitude(fmt):
     out = dev.decode(0)
     kc, vc, ks, vs, _ = _oracle_after_write(wl)
     ref, _ = _oracle_decode(wl, kc, vc, ks, vs)
-    assert_close(to_f64(out), ref, f"{fmt} rows, heads 10^4 apart")
+    assert_close_rows(to_f64(out), ref, f"{fmt} rows, heads 10^4 apart")
     # the written rows of the smallest head use the whole code range
     b = wl.block_size
     for sl in wl.slot_mapping[:3]:
@@ -240,7 +241,7 @@ def test_rowscale_full_size(fmt, name):
     assert st == 0
     _same_pools(dev, kc, vc, ks, vs, f"{name} {fmt} rows")
     ref, _ = _oracle_decode(wl, kc, vc, ks, vs)
-    assert_close(to_f64(out), ref, f"{name} {fmt} rows, every row")
+    assert_close_rows(to_f64(out), ref, f"{name} {fmt} rows, every row")
 
 
 def test_scale_pools_swap_to_host_and_back():
