@@ -5,7 +5,7 @@
 // output), the "no result" store of a CTA whose copies timed out, and the
 // split-context reduction kernel.  Included by paged_decode.cu.
 //
-// paged_decode_reduce_kernel: one warp per (sequence, query head) with more
+// paged_decode_reduce_kernel: one CTA per (sequence, query head) with more
 // than one partition merges the partitions with the blocked-softmax rule of
 // "PagedAttention：大模型KV Cache分页管理优化实践" §5.1 applied to partitions:
 //   M = max_p m_p,  w_p = l_p * 2^(m_p - M),  out = sum_p w_p Ohat_p / sum_p w_p.
@@ -15,6 +15,8 @@
 #include <cuda_fp16.h>
 #include <math.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "pa.h"
 #include "pa_common.cuh"
@@ -194,10 +196,20 @@ __device__ __forceinline__ void store_aborted_rows(T* __restrict__ out, float* _
 }
 
 
-// One warp per (sequence, query head) whose context spans several
+// Warps per (sequence, query head) row of the split-context reduction.
+// Each takes every kReduceWarps-th partition with several loads in flight,
+// so the partials of a long context are read by many warps at once; a
+// single warp walking 64 partitions one after the other left the memory
+// system mostly idle (about 3.5 warps per SM on the long-context workload).
+constexpr int kReduceWarps = 8;
+
+// One CTA per (sequence, query head) whose context spans several
 // partitions: merge the partitions' (max, exp-sum, normalised output).
+// Every warp reads the partition maxima (a few hundred bytes) for the global
+// max M, weighs its own partitions by w_p = l_p * 2^(m_p - M), and the warps'
+// sums are added in a fixed order, so the result is deterministic.
 template <typename T, int D>
-__global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_reduce_kernel(
+__global__ void __launch_bounds__(kReduceWarps * 32) paged_decode_reduce_kernel(
     T* __restrict__ out, const float* __restrict__ ws_o, const float2* __restrict__ ws_ml,
     const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t num_q_heads,
     int32_t max_context_len, int32_t max_blocks_per_seq, int32_t block_size,
@@ -205,8 +217,11 @@ __global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_reduce_ke
 {
     grid_dependency_wait();
     constexpr int EPL = D / 32;     // elements per lane
+    __shared__ float s_acc[kReduceWarps][D];
+    __shared__ float s_w[kReduceWarps];
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kReduceRowsPerCta + (threadIdx.x >> 5);
+    const int64_t row = blockIdx.x;
     if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;
     const int s = static_cast<int>(row / num_q_heads);
     const int32_t ctx = context_lens[s];
@@ -226,28 +241,51 @@ __global__ void __launch_bounds__(kReduceRowsPerCta * 32) paged_decode_reduce_ke
     for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
     float W = 0.f;
     const float* orow = ws_o + row * max_parts * D + lane * EPL;
-    for (int p = 0; p < np; ++p) {
-        const float2 v = ml[p];
+    using Vec = typename std::conditional<EPL == 4, float4, float2>::type;
+    auto weigh = [&](const float2 v, const Vec x) {
         const float w = v.y * exp2f(v.x - msub);
         W += w;
-        if (EPL == 4) {
-            const float4 x = *reinterpret_cast<const float4*>(orow + static_cast<int64_t>(p) * D);
-            acc[0] = fmaf(w, x.x, acc[0]);
-            acc[1] = fmaf(w, x.y, acc[1]);
-            acc[2] = fmaf(w, x.z, acc[2]);
-            acc[3] = fmaf(w, x.w, acc[3]);
-        } else {
+        const float* xf = reinterpret_cast<const float*>(&x);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, orow[static_cast<int64_t>(p) * D + e], acc[e]);
+        for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, xf[e], acc[e]);
+    };
+    // four of this warp's partitions per round, all their loads issued first
+    constexpr int kBatch = 4;
+    int p = warp;
+    for (; p + (kBatch - 1) * kReduceWarps < np; p += kBatch * kReduceWarps) {
+        float2 v[kBatch];
+        Vec x[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            const int q = p + j * kReduceWarps;
+            v[j] = ml[q];
+            x[j] = *reinterpret_cast<const Vec*>(orow + static_cast<int64_t>(q) * D);
         }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) weigh(v[j], x[j]);
     }
-    const float inv = W > 0.f ? 1.f / W : 0.f;
+    for (; p < np; p += kReduceWarps)
+        weigh(ml[p], *reinterpret_cast<const Vec*>(orow + static_cast<int64_t>(p) * D));
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) s_acc[warp][lane * EPL + e] = acc[e];
+    if (lane == 0) s_w[warp] = W;
+    __syncthreads();
+    if (warp != 0) return;
+    float a[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) a[e] = 0.f;
+    float Wt = 0.f;
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w) {
+        Wt += s_w[w];
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) a[e] += s_acc[w][lane * EPL + e];
+    }
+    const float inv = Wt > 0.f ? 1.f / Wt : 0.f;
     T* dst = out + row * D + lane * EPL;
 #pragma unroll
-    for (int e = 0; e < EPL; e += 2) {
-        const uint32_t packed = Elem<T>::from_float2(acc[e] * inv, acc[e + 1] * inv);
-        *reinterpret_cast<uint32_t*>(dst + e) = packed;
-    }
+    for (int e = 0; e < EPL; e += 2)
+        *reinterpret_cast<uint32_t*>(dst + e) = Elem<T>::from_float2(a[e] * inv, a[e + 1] * inv);
 }
 
 }  // namespace pa

@@ -214,9 +214,8 @@ static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
         a.probe_us, a.k_scales, a.v_scales);
     if (st != PA_OK || a.max_parts <= 1) return st;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
-    const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
-    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(ctas),
-                             dim3(kReduceRowsPerCta * 32), 0, a.stream, static_cast<T*>(a.out),
+    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(static_cast<unsigned>(rows)),
+                             dim3(kReduceWarps * 32), 0, a.stream, static_cast<T*>(a.out),
                              a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
                              a.max_context_len, a.max_blocks_per_seq, a.block_size,
                              a.partition_size, a.max_parts);
@@ -296,9 +295,8 @@ static pa_status launch_decode(const DecodeArgs& a)
     }
     if (a.max_parts <= 1) return PA_OK;
     const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
-    const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
-    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(ctas),
-                             dim3(kReduceRowsPerCta * 32), 0, a.stream, static_cast<T*>(a.out),
+    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(static_cast<unsigned>(rows)),
+                             dim3(kReduceWarps * 32), 0, a.stream, static_cast<T*>(a.out),
                              a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
                              a.max_context_len, a.max_blocks_per_seq, a.block_size,
                              a.partition_size, a.max_parts);
