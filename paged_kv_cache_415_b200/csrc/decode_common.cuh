@@ -196,32 +196,45 @@ __device__ __forceinline__ void store_aborted_rows(T* __restrict__ out, float* _
 }
 
 
-// Warps per (sequence, query head) row of the split-context reduction.
-// Each takes every kReduceWarps-th partition with several loads in flight,
-// so the partials of a long context are read by many warps at once; a
-// single warp walking 64 partitions one after the other left the memory
-// system mostly idle (about 3.5 warps per SM on the long-context workload).
+// The split-context reduction takes one of two shapes, chosen per launch
+// from the number of partitions:
+//   * many partitions (kWideRowParts or more): one CTA of kReduceWarps warps
+//     per (sequence, query head); every warp weighs every kReduceWarps-th
+//     partition, so a long context's partials are read by many warps at
+//     once (one warp walking 64 partitions in sequence left the memory
+//     system mostly idle: about 3.5 warps per SM on the long-context
+//     workload);
+//   * few partitions: one warp per (sequence, query head), four rows per
+//     CTA, so short rows do not leave seven warps of a CTA idle.
+// Either way every warp keeps the loads of four partitions in flight.
 constexpr int kReduceWarps = 8;
+constexpr int kWideRowParts = 16;
 
-// One CTA per (sequence, query head) whose context spans several
-// partitions: merge the partitions' (max, exp-sum, normalised output).
-// Every warp reads the partition maxima (a few hundred bytes) for the global
-// max M, weighs its own partitions by w_p = l_p * 2^(m_p - M), and the warps'
-// sums are added in a fixed order, so the result is deterministic.
-template <typename T, int D>
-__global__ void __launch_bounds__(kReduceWarps * 32) paged_decode_reduce_kernel(
-    T* __restrict__ out, const float* __restrict__ ws_o, const float2* __restrict__ ws_ml,
-    const int32_t* __restrict__ context_lens, int32_t num_seqs, int32_t num_q_heads,
-    int32_t max_context_len, int32_t max_blocks_per_seq, int32_t block_size,
-    int32_t partition_size, int32_t max_parts)
+// Merge the partitions' (max, exp-sum, normalised output) of the rows whose
+// context spans several partitions (rows of one partition were written by
+// the decode kernel).  M = max_p m_p, w_p = l_p * 2^(m_p - M),
+// out = sum_p w_p Ohat_p / sum_p w_p.  WPR = warps per row (1 or
+// kReduceWarps); with several, the warps' sums are added in a fixed order,
+// so the result is deterministic either way.
+template <typename T, int D, int WPR>
+__global__ void __launch_bounds__(WPR == 1 ? kReduceRowsPerCta * 32 : WPR * 32)
+    paged_decode_reduce_kernel(T* __restrict__ out, const float* __restrict__ ws_o,
+                               const float2* __restrict__ ws_ml,
+                               const int32_t* __restrict__ context_lens, int32_t num_seqs,
+                               int32_t num_q_heads, int32_t max_context_len,
+                               int32_t max_blocks_per_seq, int32_t block_size,
+                               int32_t partition_size, int32_t max_parts)
 {
     grid_dependency_wait();
     constexpr int EPL = D / 32;     // elements per lane
-    __shared__ float s_acc[kReduceWarps][D];
-    __shared__ float s_w[kReduceWarps];
+    constexpr int kSmemWarps = WPR == 1 ? 1 : WPR;
+    __shared__ float s_acc[kSmemWarps][D];
+    __shared__ float s_w[kSmemWarps];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int64_t row = blockIdx.x;
+    const int64_t row = WPR == 1 ? static_cast<int64_t>(blockIdx.x) * kReduceRowsPerCta + warp
+                                 : static_cast<int64_t>(blockIdx.x);
+    const int wr = WPR == 1 ? 0 : warp;             // this warp's place in its row
     if (row >= static_cast<int64_t>(num_seqs) * num_q_heads) return;
     const int s = static_cast<int>(row / num_q_heads);
     const int32_t ctx = context_lens[s];
@@ -251,41 +264,42 @@ __global__ void __launch_bounds__(kReduceWarps * 32) paged_decode_reduce_kernel(
     };
     // four of this warp's partitions per round, all their loads issued first
     constexpr int kBatch = 4;
-    int p = warp;
-    for (; p + (kBatch - 1) * kReduceWarps < np; p += kBatch * kReduceWarps) {
+    int p = wr;
+    for (; p + (kBatch - 1) * WPR < np; p += kBatch * WPR) {
         float2 v[kBatch];
         Vec x[kBatch];
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
-            const int q = p + j * kReduceWarps;
+            const int q = p + j * WPR;
             v[j] = ml[q];
             x[j] = *reinterpret_cast<const Vec*>(orow + static_cast<int64_t>(q) * D);
         }
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) weigh(v[j], x[j]);
     }
-    for (; p < np; p += kReduceWarps)
+    for (; p < np; p += WPR)
         weigh(ml[p], *reinterpret_cast<const Vec*>(orow + static_cast<int64_t>(p) * D));
+    if constexpr (WPR > 1) {
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) s_acc[warp][lane * EPL + e] = acc[e];
-    if (lane == 0) s_w[warp] = W;
-    __syncthreads();
-    if (warp != 0) return;
-    float a[EPL];
+        for (int e = 0; e < EPL; ++e) s_acc[warp][lane * EPL + e] = acc[e];
+        if (lane == 0) s_w[warp] = W;
+        __syncthreads();
+        if (warp != 0) return;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) a[e] = 0.f;
-    float Wt = 0.f;
+        for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+        W = 0.f;
 #pragma unroll
-    for (int w = 0; w < kReduceWarps; ++w) {
-        Wt += s_w[w];
+        for (int w = 0; w < WPR; ++w) {
+            W += s_w[w];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) a[e] += s_acc[w][lane * EPL + e];
+            for (int e = 0; e < EPL; ++e) acc[e] += s_acc[w][lane * EPL + e];
+        }
     }
-    const float inv = Wt > 0.f ? 1.f / Wt : 0.f;
+    const float inv = W > 0.f ? 1.f / W : 0.f;
     T* dst = out + row * D + lane * EPL;
 #pragma unroll
     for (int e = 0; e < EPL; e += 2)
-        *reinterpret_cast<uint32_t*>(dst + e) = Elem<T>::from_float2(a[e] * inv, a[e + 1] * inv);
+        *reinterpret_cast<uint32_t*>(dst + e) = Elem<T>::from_float2(acc[e] * inv, acc[e + 1] * inv);
 }
 
 }  // namespace pa

@@ -189,6 +189,28 @@ static bool encode_pool_map_q8(CUtensorMap* map, const void* pool, int32_t head_
     return res == CUDA_SUCCESS;
 }
 
+// The split-context reduction after a decode launch whose contexts span
+// several partitions: a CTA of kReduceWarps warps per (sequence, query head)
+// when there are many partitions, else one warp per row.
+template <typename T, int D>
+static pa_status launch_reduce(const DecodeArgs& a)
+{
+    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
+    if (a.max_parts >= kWideRowParts)
+        return launch_overlapped(paged_decode_reduce_kernel<T, D, kReduceWarps>,
+                                 dim3(static_cast<unsigned>(rows)), dim3(kReduceWarps * 32), 0,
+                                 a.stream, static_cast<T*>(a.out), a.ws_o, a.ws_ml,
+                                 a.context_lens, a.num_seqs, a.num_q_heads, a.max_context_len,
+                                 a.max_blocks_per_seq, a.block_size, a.partition_size,
+                                 a.max_parts);
+    const unsigned ctas = static_cast<unsigned>((rows + kReduceRowsPerCta - 1) / kReduceRowsPerCta);
+    return launch_overlapped(paged_decode_reduce_kernel<T, D, 1>, dim3(ctas),
+                             dim3(kReduceRowsPerCta * 32), 0, a.stream, static_cast<T*>(a.out),
+                             a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
+                             a.max_context_len, a.max_blocks_per_seq, a.block_size,
+                             a.partition_size, a.max_parts);
+}
+
 template <typename Codes, typename T, int D, int BS, int G, bool ROWS>
 static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
 {
@@ -213,12 +235,7 @@ static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
         static_cast<uint8_t*>(const_cast<void*>(a.v_cache)), a.num_kv_heads, a.k_inv, a.v_inv,
         a.probe_us, a.k_scales, a.v_scales);
     if (st != PA_OK || a.max_parts <= 1) return st;
-    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
-    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(static_cast<unsigned>(rows)),
-                             dim3(kReduceWarps * 32), 0, a.stream, static_cast<T*>(a.out),
-                             a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
-                             a.max_context_len, a.max_blocks_per_seq, a.block_size,
-                             a.partition_size, a.max_parts);
+    return launch_reduce<T, D>(a);
 }
 
 template <typename Codes, typename T, int D, int BS, bool ROWS>
@@ -294,12 +311,7 @@ static pa_status launch_decode(const DecodeArgs& a)
         if (ls != PA_OK) return ls;
     }
     if (a.max_parts <= 1) return PA_OK;
-    const int64_t rows = static_cast<int64_t>(a.num_seqs) * a.num_q_heads;
-    return launch_overlapped(paged_decode_reduce_kernel<T, D>, dim3(static_cast<unsigned>(rows)),
-                             dim3(kReduceWarps * 32), 0, a.stream, static_cast<T*>(a.out),
-                             a.ws_o, a.ws_ml, a.context_lens, a.num_seqs, a.num_q_heads,
-                             a.max_context_len, a.max_blocks_per_seq, a.block_size,
-                             a.partition_size, a.max_parts);
+    return launch_reduce<T, D>(a);
 }
 
 template <typename T, int D, int BS>

@@ -16,7 +16,7 @@ import torch
 
 import oracle
 from tests import oracle_pins
-from tests.gpu_utils import assert_close, to_dev, to_f64
+from tests.gpu_utils import assert_close, assert_close_rows, to_dev, to_f64
 from workloads import generators as gen
 
 pytestmark = pytest.mark.gpu
@@ -101,7 +101,7 @@ def _oracle_decode(wl, kc, vc, tables=None, ctx=None):
                                                   wl.extra["v_scale"])
 
 
-def _parity(wl, partition_size=None, what=""):
+def _parity(wl, partition_size=None, what="", row_scaled_tolerance=False):
     dev = Q8Device(wl)
     dev.write()
     out = dev.decode(partition_size)
@@ -112,7 +112,7 @@ def _parity(wl, partition_size=None, what=""):
     assert np.array_equal(dev.v_cache.cpu().numpy(), vc), f"{what}: V pool"
     ref, st = _oracle_decode(wl, kc, vc)
     assert st == 0
-    assert_close(to_f64(out), ref, what or wl.name)
+    (assert_close_rows if row_scaled_tolerance else assert_close)(to_f64(out), ref, what or wl.name)
     assert dev.status() == 0
     return dev, out
 
@@ -385,7 +385,10 @@ def test_int8_bias_removal_under_stress(group, partition):
     every score and 1152 * sum(p) from the output.  Stress both: scales of 1
     (codes are the values, up to +-127), a query that is positive in every
     dim (sum(q) as large as it gets), contexts up to 8192 tokens and, with an
-    8192-token partition, one warp accumulating 128 blocks."""
+    8192-token partition, one warp accumulating 128 blocks.  With scales of
+    1 the outputs are up to ~127 (the fp16 rounding of P alone moves them by
+    ~0.03), so the absolute part of the tolerance scales with each output
+    row's magnitude (assert_close_rows)."""
     hkv = 2
     wl = gen.make_decode("int8-bias", seed=4150 + 90 + group, dtype="f16",
                          context_lens=np.array([8192, 3000, 1], np.int32),
@@ -396,4 +399,4 @@ def test_int8_bias_removal_under_stress(group, partition):
     wl = gen.with_code_pools(wl, "int8", seed=4150 + 91)
     wl.extra["k_scale"] = 1.0
     wl.extra["v_scale"] = 1.0
-    _parity(wl, partition, f"int8 bias stress G={group} P={partition}")
+    _parity(wl, partition, f"int8 bias stress G={group} P={partition}", row_scaled_tolerance=True)
