@@ -60,14 +60,8 @@ struct Q8Shape {
     static constexpr bool SWIZZLE = (D == 128);      // 128-byte rows, 128B TMA swizzle
     static constexpr int TILE = BS * D;              // bytes of one K (or V) tile of one head
     static constexpr int STAGE = 2 * TILE;
-    // 16-token blocks are consumed two at a time (one softmax step for two
-    // blocks), from a ring of four; a 32-token block is one such step itself
-    static constexpr bool PAIR = (BS == 16);
-    static constexpr int NSTAGE = PAIR ? 4 : (STAGE <= 4096 ? 3 : 2);
-    // P^T staging tile: per head row the P of two 16-token slices (64 bytes)
-    // and 16 bytes of padding, so the 8 rows an ldmatrix reads hit 8
-    // different groups of 4 banks
-    static constexpr int PT_STRIDE = 80;
+    static constexpr int NSTAGE = STAGE <= 4096 ? 3 : 2;
+    static constexpr int PT_STRIDE = 48;             // bytes per head row of the P^T tile
     static constexpr int PT_BYTES = 8 * PT_STRIDE;
     static constexpr int WARP_BYTES = NSTAGE * STAGE;
     static constexpr int OFF_PT = kWarps * WARP_BYTES;
@@ -78,8 +72,7 @@ struct Q8Shape {
     // + a probe barrier per warp, + alignment slack
     static constexpr int SMEM_BYTES = OFF_BARS + kWarps * (NSTAGE + 1) * 8 + 1024;
     static constexpr int EPI_BYTES = kWarps * G * (D + 2) * 4;
-    static_assert(BS == 16 || BS == 32, "one or two 16-token slices per block");
-    static_assert(D == 64 || D == 128, "whole 16-byte code runs per lane");
+    static_assert(BS % 16 == 0 && (D == 64 || D == 128), "whole 16-token slices");
     static_assert(G >= 1 && G <= 8, "heads are the 8 columns of N");
     static_assert(STAGE % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
     static_assert(EPI_BYTES <= OFF_BARS, "epilogue fits in the warp buffers");
@@ -111,15 +104,6 @@ __device__ __forceinline__ void stmatrix_x2_trans(uint32_t smem_addr, uint32_t r
     asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1, %2};"
                  :
                  : "r"(smem_addr), "r"(r0), "r"(r1)
-                 : "memory");
-}
-
-__device__ __forceinline__ void stmatrix_x4_trans(uint32_t smem_addr, uint32_t r0, uint32_t r1,
-                                                  uint32_t r2, uint32_t r3)
-{
-    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};"
-                 :
-                 : "r"(smem_addr), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
                  : "memory");
 }
 
@@ -268,224 +252,175 @@ struct Q8Warp {
         }
     }
 
-    // S^T of one 16-token slice (tokens t0 .. t0 + 15 of the K tile kt):
-    // s[0], s[1] = token t0 + grp, heads 2tig and 2tig + 1; s[2], s[3] =
-    // token t0 + grp + 8.  Two accumulator chains, added at the end.
-    __device__ __forceinline__ void qk(const unsigned char* kt, int t0, float (&s)[4]) const
+    // One block: kt / vt are its K and V byte tiles, nv its valid tokens;
+    // with ROWS, ksc / vsc its B row scales of K and of V.
+    __device__ __forceinline__ void block(const unsigned char* kt, const unsigned char* vt, int nv,
+                                          float scale_log2, const float* ksc = nullptr,
+                                          const float* vsc = nullptr)
     {
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h = 0; h < S::KV16; ++h) {
-            uint32_t w0[4], w1[4];
-            load_words<D>(kt, t0 + grp, (D / 4) * tig + 16 * h, w0);
-            load_words<D>(kt, t0 + grp + 8, (D / 4) * tig + 16 * h, w1);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = 4 * h + i;
-                uint32_t a0, a2, a1, a3;
-                Codes::widen4(w0[i], a0, a2);
-                Codes::widen4(w1[i], a1, a3);
-                if (j & 1)
-                    mma_16816<__half>(sb, a0, a1, a2, a3, qb[j][0], qb[j][1]);
-                else
-                    mma_16816<__half>(sa, a0, a1, a2, a3, qb[j][0], qb[j][1]);
-            }
-        }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) s[e] = sa[e] + sb[e];
-    }
+#pragma unroll 1
+        for (int sl = 0; sl < S::SLICES; ++sl) {
+            const int t0 = sl * 16;
+            const int tv = nv - t0;             // valid tokens of this slice
+            if (tv <= 0) break;
 
-    // O^T += V^T . P^T for one 16-token slice (tokens t0 .. t0 + 15 of the V
-    // tile vt, tv of them valid): this lane reads tokens 2tig, 2tig + 1,
-    // 2tig + 8, 2tig + 9 of the slice; pb0 / pb1 are the P^T fragments.
-    __device__ __forceinline__ void pv(const unsigned char* vt, int t0, int tv, uint32_t pb0,
-                                       uint32_t pb1)
-    {
-        const int ta = t0 + 2 * tig;
-        uint32_t va[S::VQ], vb[S::VQ], vc[S::VQ], vd[S::VQ];
-        if constexpr (S::VQ == 4) {
-            uint32_t w[4];
-            load_words<D>(vt, ta, S::DPT * grp, w);
+            // ---- S^T = K . Q^T: rows grp and grp + 8 of the slice ----
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) va[q] = w[q];
-            load_words<D>(vt, ta + 1, S::DPT * grp, w);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) vb[q] = w[q];
-            load_words<D>(vt, ta + 8, S::DPT * grp, w);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) vc[q] = w[q];
-            load_words<D>(vt, ta + 9, S::DPT * grp, w);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) vd[q] = w[q];
-        } else {
-            const uint2 a = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta, S::DPT * grp));
-            const uint2 b = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 1, S::DPT * grp));
-            const uint2 c = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 8, S::DPT * grp));
-            const uint2 d = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 9, S::DPT * grp));
-            va[0] = a.x; va[1] = a.y;
-            vb[0] = b.x; vb[1] = b.y;
-            vc[0] = c.x; vc[1] = c.y;
-            vd[0] = d.x; vd[1] = d.y;
-        }
-        if (tv < 16) {   // rows past the context may hold any code (NaN included)
-            const int ra = 2 * tig;
-#pragma unroll
-            for (int q = 0; q < S::VQ; ++q) {
-                va[q] = ra < tv ? va[q] : 0u;
-                vb[q] = ra + 1 < tv ? vb[q] : 0u;
-                vc[q] = ra + 8 < tv ? vc[q] : 0u;
-                vd[q] = ra + 9 < tv ? vd[q] : 0u;
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < S::VQ; ++q) {
-            // token pairs per dim: [b1 a1 b0 a0] and [b3 a3 b2 a2]
-            const uint32_t lo_ab = __byte_perm(va[q], vb[q], 0x5140);
-            const uint32_t hi_ab = __byte_perm(va[q], vb[q], 0x7362);
-            const uint32_t lo_cd = __byte_perm(vc[q], vd[q], 0x5140);
-            const uint32_t hi_cd = __byte_perm(vc[q], vd[q], 0x7362);
-            uint32_t a0, a1, a2, a3;
-            // m-tile 2q: rows grp / grp + 8 are dims DPT*grp + 4q + 0 / + 1
-            Codes::widen4(lo_ab, a0, a1);
-            Codes::widen4(lo_cd, a2, a3);
-            mma_16816<__half>(o[2 * q], a0, a1, a2, a3, pb0, pb1);
-            // m-tile 2q + 1: dims + 2 / + 3
-            Codes::widen4(hi_ab, a0, a1);
-            Codes::widen4(hi_cd, a2, a3);
-            mma_16816<__half>(o[2 * q + 1], a0, a1, a2, a3, pb0, pb1);
-        }
-    }
-
-    // Two 16-token slices a and b in one step of the online softmax: their
-    // scores, one max / rescale / exp-sum update for both, P of both moved
-    // into the B layout with one stmatrix.x4 / ldmatrix.x4, then O^T for
-    // both.  kt* / vt* are the slices' K and V tiles, t0* their first token
-    // in the tile, tv* their valid tokens (<= 0: the slice takes no part),
-    // ksc* / vsc* (ROWS) the tiles' row scales.
-    __device__ __forceinline__ void unit(const unsigned char* kta, const unsigned char* vta, int t0a,
-                                         int tva, const float* ksca, const float* vsca,
-                                         const unsigned char* ktb, const unsigned char* vtb, int t0b,
-                                         int tvb, const float* kscb, const float* vscb,
-                                         float scale_log2)
-    {
-        float sA[4], sB[4];
-        qk(kta, t0a, sA);
-        qk(ktb, t0b, sB);
-        // this lane: slice a tokens grp (x0, x1) and grp + 8 (x2, x3), slice b
-        // likewise (x4 .. x7); even entries head 2tig, odd entries 2tig + 1
-        float s0 = scale_log2, s1 = scale_log2, s2 = scale_log2, s3 = scale_log2;
-        if constexpr (ROWS) {                   // each token's K row scale
-            s0 *= ksca[t0a + grp];
-            s1 *= ksca[t0a + grp + 8];
-            s2 *= kscb[t0b + grp];
-            s3 *= kscb[t0b + grp + 8];
-        }
-        float x[8];
-        x[0] = grp < tva ? (sA[0] - e0) * s0 : -INFINITY;
-        x[1] = grp < tva ? (sA[1] - e1) * s0 : -INFINITY;
-        x[2] = grp + 8 < tva ? (sA[2] - e0) * s1 : -INFINITY;
-        x[3] = grp + 8 < tva ? (sA[3] - e1) * s1 : -INFINITY;
-        x[4] = grp < tvb ? (sB[0] - e0) * s2 : -INFINITY;
-        x[5] = grp < tvb ? (sB[1] - e1) * s2 : -INFINITY;
-        x[6] = grp + 8 < tvb ? (sB[2] - e0) * s3 : -INFINITY;
-        x[7] = grp + 8 < tvb ? (sB[3] - e1) * s3 : -INFINITY;
-
-        // ---- online softmax per head over the unit's 32 tokens ----
-        float mx0 = fmaxf(fmaxf(x[0], x[2]), fmaxf(x[4], x[6]));
-        float mx1 = fmaxf(fmaxf(x[1], x[3]), fmaxf(x[5], x[7]));
-#pragma unroll
-        for (int m = 4; m < 32; m <<= 1) {
-            mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, m));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, m));
-        }
-        const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
-        const float ms0 = mn0 == -INFINITY ? 0.f : mn0;
-        const float ms1 = mn1 == -INFINITY ? 0.f : mn1;
-        const float c0 = q8_exp2(m_run0 - ms0), c1 = q8_exp2(m_run1 - ms1);
-        m_run0 = mn0;
-        m_run1 = mn1;
-        float p[8];
-#pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-            p[i] = q8_exp2(x[i] - ms0);
-            p[i + 1] = q8_exp2(x[i + 1] - ms1);
-        }
-        uint32_t pk[4];
-        float2 cc = make_float2(c0, c1);
-        if constexpr (ROWS) {
-            // V row scales of the unit's tokens relative to the running
-            // reference (rows past the context weigh 0); the reference grows
-            // to the unit's largest scale and rescales O like a change of
-            // the running max does
-            float vr[4];
-            vr[0] = grp < tva ? vsca[t0a + grp] : 0.f;
-            vr[1] = grp + 8 < tva ? vsca[t0a + grp + 8] : 0.f;
-            vr[2] = grp < tvb ? vscb[t0b + grp] : 0.f;
-            vr[3] = grp + 8 < tvb ? vscb[t0b + grp + 8] : 0.f;
-            float vmax = fmaxf(fmaxf(vr[0], vr[1]), fmaxf(vr[2], vr[3]));
-#pragma unroll
-            for (int m = 4; m < 32; m <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFullMask, vmax, m));
-            if (vmax > vref) {                  // warp-uniform
-                const float fr = vref / vmax;
-                cc.x *= fr;
-                cc.y *= fr;
-                vref = vmax;
-                vinv = 1.f / vmax;
-            }
-            l_run0 = l_run0 * c0 + ((p[0] + p[2]) + (p[4] + p[6]));
-            l_run1 = l_run1 * c1 + ((p[1] + p[3]) + (p[5] + p[7]));
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float r = vr[i] * vinv;
-                pk[i] = Elem<__half>::from_float2(p[2 * i] * r, p[2 * i + 1] * r);
-            }
-            if constexpr (Codes::kBias != 0.f) {   // the P values the MMA reads
-                float f0 = 0.f, f1 = 0.f;
+            for (int h = 0; h < S::KV16; ++h) {
+                uint32_t w0[4], w1[4];
+                load_words<D>(kt, t0 + grp, (D / 4) * tig + 16 * h, w0);
+                load_words<D>(kt, t0 + grp + 8, (D / 4) * tig + 16 * h, w1);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float2 f = Elem<__half>::to_float2(pk[i]);
-                    f0 += f.x;
-                    f1 += f.y;
+                    const int j = 4 * h + i;
+                    uint32_t a0, a2, a1, a3;
+                    Codes::widen4(w0[i], a0, a2);
+                    Codes::widen4(w1[i], a1, a3);
+                    if (j & 1)
+                        mma_16816<__half>(sb, a0, a1, a2, a3, qb[j][0], qb[j][1]);
+                    else
+                        mma_16816<__half>(sa, a0, a1, a2, a3, qb[j][0], qb[j][1]);
                 }
-                ps_run0 = ps_run0 * cc.x + f0;
-                ps_run1 = ps_run1 * cc.y + f1;
             }
-        } else {
-            // P rounds to fp16 for the tensor cores; the sums use the rounded values
-            float f0 = 0.f, f1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                pk[i] = Elem<__half>::from_float2(p[2 * i], p[2 * i + 1]);
-                const float2 f = Elem<__half>::to_float2(pk[i]);
-                f0 += f.x;
-                f1 += f.y;
+            // this lane: tokens grp (x0, x1) and grp + 8 (x2, x3); heads 2tig, 2tig + 1
+            float sla = scale_log2, slb = scale_log2;
+            if constexpr (ROWS) {               // each token's K row scale
+                sla *= ksc[t0 + grp];
+                slb *= ksc[t0 + grp + 8];
             }
-            l_run0 = l_run0 * c0 + f0;
-            l_run1 = l_run1 * c1 + f1;
-        }
-        // once the running maxima settle, most units leave them unchanged
-        if (__any_sync(kFullMask, cc.x != 1.f || cc.y != 1.f)) {
-#pragma unroll
-            for (int mt = 0; mt < S::MT; ++mt) {
-                float2 u = __fmul2_rn(make_float2(o[mt][0], o[mt][1]), cc);
-                float2 v = __fmul2_rn(make_float2(o[mt][2], o[mt][3]), cc);
-                o[mt][0] = u.x;
-                o[mt][1] = u.y;
-                o[mt][2] = v.x;
-                o[mt][3] = v.y;
-            }
-        }
+            const float x0 = grp < tv ? ((sa[0] + sb[0]) - e0) * sla : -INFINITY;
+            const float x1 = grp < tv ? ((sa[1] + sb[1]) - e1) * sla : -INFINITY;
+            const float x2 = grp + 8 < tv ? ((sa[2] + sb[2]) - e0) * slb : -INFINITY;
+            const float x3 = grp + 8 < tv ? ((sa[3] + sb[3]) - e1) * slb : -INFINITY;
 
-        // ---- P (tokens x heads) -> P^T B fragments (heads x tokens), both slices ----
-        uint32_t pb[4];
-        __syncwarp();
-        stmatrix_x4_trans(pt_addr, pk[0], pk[1], pk[2], pk[3]);
-        __syncwarp();
-        ldmatrix_x4(pb, pt_addr);
+            // ---- online softmax per head over the slice's 16 tokens ----
+            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int m = 4; m < 32; m <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFullMask, mx0, m));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFullMask, mx1, m));
+            }
+            const float mn0 = fmaxf(m_run0, mx0), mn1 = fmaxf(m_run1, mx1);
+            const float ms0 = mn0 == -INFINITY ? 0.f : mn0;
+            const float ms1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float c0 = q8_exp2(m_run0 - ms0), c1 = q8_exp2(m_run1 - ms1);
+            m_run0 = mn0;
+            m_run1 = mn1;
+            uint32_t pk0, pk1;
+            float2 cc = make_float2(c0, c1);
+            if constexpr (ROWS) {
+                // V row scales of the slice's tokens relative to the running
+                // reference (rows past the context weigh 0); the reference
+                // grows to the slice's largest scale and rescales O like a
+                // change of the running max does
+                const float va = grp < tv ? vsc[t0 + grp] : 0.f;
+                const float vb = grp + 8 < tv ? vsc[t0 + grp + 8] : 0.f;
+                float vmax = fmaxf(va, vb);
+#pragma unroll
+                for (int m = 4; m < 32; m <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(kFullMask, vmax, m));
+                if (vmax > vref) {              // warp-uniform
+                    const float fr = vref / vmax;
+                    cc.x *= fr;
+                    cc.y *= fr;
+                    vref = vmax;
+                    vinv = 1.f / vmax;
+                }
+                const float p0 = q8_exp2(x0 - ms0), p1 = q8_exp2(x1 - ms1);
+                const float p2 = q8_exp2(x2 - ms0), p3 = q8_exp2(x3 - ms1);
+                l_run0 = l_run0 * c0 + (p0 + p2);
+                l_run1 = l_run1 * c1 + (p1 + p3);
+                const float ra = va * vinv, rb = vb * vinv;
+                pk0 = Elem<__half>::from_float2(p0 * ra, p1 * ra);
+                pk1 = Elem<__half>::from_float2(p2 * rb, p3 * rb);
+                if constexpr (Codes::kBias != 0.f) {   // the P values the MMA reads
+                    const float2 f0 = Elem<__half>::to_float2(pk0), f1 = Elem<__half>::to_float2(pk1);
+                    ps_run0 = ps_run0 * cc.x + (f0.x + f1.x);
+                    ps_run1 = ps_run1 * cc.y + (f0.y + f1.y);
+                }
+            } else {
+                // P rounds to fp16 for the tensor cores; the sums use the rounded values
+                pk0 = Elem<__half>::from_float2(q8_exp2(x0 - ms0), q8_exp2(x1 - ms1));
+                pk1 = Elem<__half>::from_float2(q8_exp2(x2 - ms0), q8_exp2(x3 - ms1));
+                const float2 r0 = Elem<__half>::to_float2(pk0), r1 = Elem<__half>::to_float2(pk1);
+                l_run0 = l_run0 * c0 + (r0.x + r1.x);
+                l_run1 = l_run1 * c1 + (r0.y + r1.y);
+            }
+            // once the running maxima settle, most slices leave them unchanged
+            if (__any_sync(kFullMask, cc.x != 1.f || cc.y != 1.f)) {
+#pragma unroll
+                for (int mt = 0; mt < S::MT; ++mt) {
+                    float2 u = __fmul2_rn(make_float2(o[mt][0], o[mt][1]), cc);
+                    float2 v = __fmul2_rn(make_float2(o[mt][2], o[mt][3]), cc);
+                    o[mt][0] = u.x;
+                    o[mt][1] = u.y;
+                    o[mt][2] = v.x;
+                    o[mt][3] = v.y;
+                }
+            }
 
-        // ---- O^T += V^T . P^T for both slices ----
-        pv(vta, t0a, tva, pb[0], pb[1]);
-        pv(vtb, t0b, tvb, pb[2], pb[3]);
+            // ---- P (tokens x heads) -> P^T B fragments (heads x tokens) ----
+            uint32_t pb0, pb1;
+            __syncwarp();
+            stmatrix_x2_trans(pt_addr, pk0, pk1);
+            __syncwarp();
+            ldmatrix_x2(pb0, pb1, pt_addr);
+
+            // ---- O^T += V^T . P^T: tokens 2tig, 2tig+1, 2tig+8, 2tig+9 ----
+            const int ta = t0 + 2 * tig;
+            uint32_t va[S::VQ], vb[S::VQ], vc[S::VQ], vd[S::VQ];
+            if constexpr (S::VQ == 4) {
+                uint32_t w[4];
+                load_words<D>(vt, ta, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) va[q] = w[q];
+                load_words<D>(vt, ta + 1, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vb[q] = w[q];
+                load_words<D>(vt, ta + 8, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vc[q] = w[q];
+                load_words<D>(vt, ta + 9, S::DPT * grp, w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vd[q] = w[q];
+            } else {
+                const uint2 a = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta, S::DPT * grp));
+                const uint2 b = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 1, S::DPT * grp));
+                const uint2 c = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 8, S::DPT * grp));
+                const uint2 d = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 9, S::DPT * grp));
+                va[0] = a.x; va[1] = a.y;
+                vb[0] = b.x; vb[1] = b.y;
+                vc[0] = c.x; vc[1] = c.y;
+                vd[0] = d.x; vd[1] = d.y;
+            }
+            if (tv < 16) {   // rows past the context may hold any code (NaN included)
+                const int ra = 2 * tig;
+#pragma unroll
+                for (int q = 0; q < S::VQ; ++q) {
+                    va[q] = ra < tv ? va[q] : 0u;
+                    vb[q] = ra + 1 < tv ? vb[q] : 0u;
+                    vc[q] = ra + 8 < tv ? vc[q] : 0u;
+                    vd[q] = ra + 9 < tv ? vd[q] : 0u;
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < S::VQ; ++q) {
+                // token pairs per dim: [b1 a1 b0 a0] and [b3 a3 b2 a2]
+                const uint32_t lo_ab = __byte_perm(va[q], vb[q], 0x5140);
+                const uint32_t hi_ab = __byte_perm(va[q], vb[q], 0x7362);
+                const uint32_t lo_cd = __byte_perm(vc[q], vd[q], 0x5140);
+                const uint32_t hi_cd = __byte_perm(vc[q], vd[q], 0x7362);
+                uint32_t a0, a1, a2, a3;
+                // m-tile 2q: rows grp / grp + 8 are dims DPT*grp + 4q + 0 / + 1
+                Codes::widen4(lo_ab, a0, a1);
+                Codes::widen4(lo_cd, a2, a3);
+                mma_16816<__half>(o[2 * q], a0, a1, a2, a3, pb0, pb1);
+                // m-tile 2q + 1: dims + 2 / + 3
+                Codes::widen4(hi_ab, a0, a1);
+                Codes::widen4(hi_cd, a2, a3);
+                mma_16816<__half>(o[2 * q + 1], a0, a1, a2, a3, pb0, pb1);
+            }
+        }
     }
 
     // The warp's (max, exp-sum, output) of its heads into the epilogue area.
@@ -669,76 +604,34 @@ __device__ __forceinline__ void paged_decode_q8_cta(
     Q8Warp<Codes, T, D, BS, G, ROWS> w;
     w.grp = lane >> 2;
     w.tig = lane & 3;
-    // row (lane & 7) of matrix (lane >> 3) of the P^T tile: matrices 0 and 1
-    // are the first slice's tokens 0-7 and 8-15, matrices 2 and 3 the second's
     w.pt_addr = smem_u32(smem + S::OFF_PT + warp * S::PT_BYTES) + (lane & 7) * S::PT_STRIDE +
-                (lane >> 3) * 16;
+                ((lane >> 3) & 1) * 16;
     w.reset();
     w.load_q(query, s, kvh, num_q_heads);
 
     bool aborted = nk > 0 && probe_gives_up(&wbar[S::NSTAGE], probe_us);
     int first_pending = 0;
-    auto tokens_of = [&](int k, int phys) {     // valid tokens of the warp's k-th block
+    for (int k = 0; k < (aborted ? 0 : nk); ++k) {
+        const int st = k % S::NSTAGE;
+        if (!mbar_wait_warp(&wbar[st], (k / S::NSTAGE) & 1)) {
+            aborted = true;
+            first_pending = k;
+            break;
+        }
+        const int chunk = k >> 5;
+        if (chunk != cons_chunk) {
+            cons_tbl = load_table(chunk);
+            cons_chunk = chunk;
+        }
+        const int phys = __shfl_sync(kFullMask, cons_tbl, k & 31);
         const bool ok = phys >= 0 && static_cast<int64_t>(phys) < num_blocks;
-        return ok ? min(BS, tok_end - (tok_begin + (warp + kWarps * k) * BS)) : 0;
-    };
-    if constexpr (S::PAIR) {
-        // blocks k and k + 1 (stages k % 4 and k % 4 + 1) in one softmax step
-        for (int k = 0; k < (aborted ? 0 : nk); k += 2) {
-            const bool two = k + 1 < nk;
-            const int st = k % S::NSTAGE;
-            const uint32_t ph = (k / S::NSTAGE) & 1;
-            if (!mbar_wait_warp(&wbar[st], ph)) {
-                aborted = true;
-                first_pending = k;
-                break;
-            }
-            if (two && !mbar_wait_warp(&wbar[st + 1], ph)) {
-                aborted = true;
-                first_pending = k + 1;
-                break;
-            }
-            const int chunk = k >> 5;              // k even: k and k + 1 share a chunk
-            if (chunk != cons_chunk) {
-                cons_tbl = load_table(chunk);
-                cons_chunk = chunk;
-            }
-            const int pa = __shfl_sync(kFullMask, cons_tbl, k & 31);
-            const int pb = __shfl_sync(kFullMask, cons_tbl, (k + 1) & 31);
-            const int nva = tokens_of(k, pa);
-            const int nvb = two ? tokens_of(k + 1, pb) : 0;
-            const unsigned char* kta = wbase + st * S::STAGE;
-            const unsigned char* ktb = kta + S::STAGE;
-            const float* sca = wsc + st * (S::SC_STAGE / 4);
-            const float* scb = sca + S::SC_STAGE / 4;
-            w.unit(kta, kta + S::TILE, 0, nva, sca, sca + BS, ktb, ktb + S::TILE, 0, nvb, scb,
-                   scb + BS, scale_log2);
-            __syncwarp();   // every lane is done with both stages
-            if (issued < nk) issue(issued++);
-            if (issued < nk) issue(issued++);
-        }
-    } else {
-        // a 32-token block: its two 16-token slices in one softmax step
-        for (int k = 0; k < (aborted ? 0 : nk); ++k) {
-            const int st = k % S::NSTAGE;
-            if (!mbar_wait_warp(&wbar[st], (k / S::NSTAGE) & 1)) {
-                aborted = true;
-                first_pending = k;
-                break;
-            }
-            const int chunk = k >> 5;
-            if (chunk != cons_chunk) {
-                cons_tbl = load_table(chunk);
-                cons_chunk = chunk;
-            }
-            const int nv = tokens_of(k, __shfl_sync(kFullMask, cons_tbl, k & 31));
-            const unsigned char* kt = wbase + st * S::STAGE;
-            const float* sc = wsc + st * (S::SC_STAGE / 4);
-            w.unit(kt, kt + S::TILE, 0, nv, sc, sc + BS, kt, kt + S::TILE, 16, nv - 16, sc,
-                   sc + BS, scale_log2);
-            __syncwarp();   // every lane is done with this stage
-            if (issued < nk) issue(issued++);
-        }
+        const int t0 = tok_begin + (warp + kWarps * k) * BS;
+        const int nv = ok ? min(BS, tok_end - t0) : 0;
+        const unsigned char* kt = wbase + st * S::STAGE;
+        const float* sc = wsc + st * (S::SC_STAGE / 4);
+        w.block(kt, kt + S::TILE, nv, scale_log2, sc, sc + BS);
+        __syncwarp();   // every lane is done with this stage
+        if (issued < nk) issue(issued++);
     }
 
     if (aborted) drain_after_timeout<S::NSTAGE>(wbar, first_pending, issued, d_status);
@@ -776,14 +669,14 @@ __device__ __forceinline__ void paged_decode_q8_cta(
 
 // e4m3 pools (ROWS: with row-scale pools; else one scale per pool)
 template <typename T, int D, int BS, int G, bool ROWS>
-__global__ void __launch_bounds__(kThreads, 3) paged_decode_fp8_kernel(PA_Q8_KERNEL_PARAMS)
+__global__ void __launch_bounds__(kThreads, 4) paged_decode_fp8_kernel(PA_Q8_KERNEL_PARAMS)
 {
     paged_decode_q8_cta<E4m3Codes, T, D, BS, G, ROWS>(PA_Q8_KERNEL_ARGS);
 }
 
 // int8 pools
 template <typename T, int D, int BS, int G, bool ROWS>
-__global__ void __launch_bounds__(kThreads, 3) paged_decode_int8_kernel(PA_Q8_KERNEL_PARAMS)
+__global__ void __launch_bounds__(kThreads, 4) paged_decode_int8_kernel(PA_Q8_KERNEL_PARAMS)
 {
     paged_decode_q8_cta<Int8Codes, T, D, BS, G, ROWS>(PA_Q8_KERNEL_ARGS);
 }
