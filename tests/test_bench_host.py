@@ -73,7 +73,8 @@ def test_committed_traffic_lines_parse():
                     m = re.match(r"bench-traffic:\s*workload=(\S+)\s+bytes_per_launch=(\d+)\s+"
                                  r"source_sha256=(\w{16})\s*$", line)
                     assert m, line
-                    assert re.sub(r"-(fp8|int8|shared)$", "", m.group(1)) in names
+                    base = re.sub(r"-((fp8|int8)(-rows)?|shared)$", "", m.group(1))
+                    assert base in names, m.group(1)
                     assert int(m.group(2)) > 0
                     found += 1
     assert found >= 3
