@@ -57,7 +57,8 @@ _CSRC = "paged_kv_cache_415_b200/csrc/"
 KERNEL_FAMILIES = {
     "fp32": ["pa_common.cuh", "decode_common.cuh", "paged_decode_fp32.cuh"],
     "mma": ["pa_common.cuh", "decode_common.cuh", "paged_decode_mma.cuh"],
-    "q8": ["pa_common.cuh", "decode_common.cuh", "pa_codes.cuh", "paged_decode_q8.cuh"],
+    "q8": ["pa_common.cuh", "decode_common.cuh", "pa_codes.cuh", "paged_decode_q8.cuh",
+           "paged_decode_q8_pair.cuh"],
     "shared": ["pa_common.cuh", "decode_common.cuh", "paged_decode_mma.cuh",
                "paged_decode_shared.cuh"],
 }
@@ -598,7 +599,10 @@ class GpuStep:
         if self.shared:
             return "paged_decode_shared_kernel" + (
                 " + paged_decode_shared_reduce_kernel" if self.shared_reduce else "")
-        name = (f"paged_decode_{self.codes}_kernel" if self.quant else
+        # one-byte pools: a CTA per pair of kv heads when the kv-head count is
+        # even and a CTA per kv head would give each warp fewer than 16 blocks
+        pair = (wl.num_kv_heads % 2 == 0 and self.part < 16 * 4 * wl.block_size)
+        name = (f"paged_decode_{self.codes}{'_pair' if pair else ''}_kernel" if self.quant else
                 "paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
                 else "paged_decode_kernel")
         return name + (" + paged_decode_reduce_kernel" if self.max_parts > 1 else "")

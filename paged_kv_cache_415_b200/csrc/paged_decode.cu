@@ -34,6 +34,7 @@
 #include "paged_decode_mma.cuh"
 #include "paged_decode_shared.cuh"
 #include "paged_decode_q8.cuh"
+#include "paged_decode_q8_pair.cuh"
 
 namespace pa {
 
@@ -164,10 +165,11 @@ static bool encode_pool_map_swizzled(CUtensorMap* map, const void* pool, int32_t
 }
 
 // A pool [num_blocks][B][Hkv][D] of one-byte codes as a 4-D tensor whose
-// box is one block of one kv head: B rows of D bytes, with the 128-byte
-// swizzle when a row is 128 bytes (else dense).
+// box is one block of `heads` adjacent kv heads (1 or 2): B x heads rows of
+// D bytes, with the 128-byte swizzle when a row is 128 bytes (else dense).
 static bool encode_pool_map_q8(CUtensorMap* map, const void* pool, int32_t head_dim,
-                                int32_t num_kv_heads, int32_t block_size, int64_t num_blocks)
+                                int32_t num_kv_heads, int32_t block_size, int64_t num_blocks,
+                                uint32_t heads = 1u)
 {
     const CUtensorMapSwizzle swz =
         head_dim == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
@@ -179,7 +181,7 @@ static bool encode_pool_map_q8(CUtensorMap* map, const void* pool, int32_t head_
                                 static_cast<cuuint64_t>(num_blocks)};
     const cuuint64_t row = static_cast<cuuint64_t>(head_dim);
     const cuuint64_t strides[3] = {row, row * num_kv_heads, row * num_kv_heads * block_size};
-    const cuuint32_t box[4] = {static_cast<cuuint32_t>(head_dim), 1u,
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(head_dim), heads,
                                static_cast<cuuint32_t>(block_size), 1u};
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     const CUresult res = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(pool), dims,
@@ -211,9 +213,47 @@ static pa_status launch_reduce(const DecodeArgs& a)
                              a.partition_size, a.max_parts);
 }
 
+// A CTA per pair of adjacent kv heads (one copy brings both heads' rows of a
+// block, and each warp takes twice the blocks): with an even number of kv
+// heads, when a CTA per kv head would give each warp fewer than
+// kPairBelowBlocks blocks of its partition.  There the per-CTA prologue and
+// epilogue weigh enough that twice the blocks per warp pays (long contexts
+// in 512-token partitions: 8 blocks per warp); above it, the shorter CTAs of
+// the per-head kernel balance ragged batches better.
+constexpr int kPairBelowBlocks = 16;
+
+template <typename Codes, typename T, int D, int BS, int G, bool ROWS>
+static pa_status launch_decode_q8_pair(const DecodeArgs& a, float v_scale)
+{
+    using S = Q8PairShape<D, BS, G, ROWS>;
+    static std::atomic<uint64_t> attr_done{0};
+    auto kernel = std::is_same<Codes, Int8Codes>::value
+                      ? paged_decode_int8_pair_kernel<T, D, BS, G, ROWS>
+                      : paged_decode_fp8_pair_kernel<T, D, BS, G, ROWS>;
+    if (!ensure_smem_attr(kernel, S::SMEM_BYTES, attr_done)) return PA_ERR_CUDA;
+    CUtensorMap tm_k, tm_v;
+    if (!encode_pool_map_q8(&tm_k, a.k_cache, D, a.num_kv_heads, BS, a.num_blocks, 2u) ||
+        !encode_pool_map_q8(&tm_v, a.v_cache, D, a.num_kv_heads, BS, a.num_blocks, 2u))
+        return PA_ERR_CUDA;
+    dim3 grid(a.num_kv_heads / 2, a.max_parts, a.num_seqs);
+    pa_status st = launch_overlapped(
+        kernel, grid, dim3(kThreads), S::SMEM_BYTES, a.stream, tm_k, tm_v, static_cast<T*>(a.out),
+        static_cast<const T*>(a.query), a.block_tables, a.context_lens, a.num_q_heads,
+        a.max_blocks_per_seq, a.num_blocks, a.max_context_len, a.scale_log2, v_scale,
+        a.partition_size, a.max_parts, a.ws_o, a.ws_ml, a.d_status, a.lpt_seqs,
+        static_cast<const T*>(a.new_key), static_cast<const T*>(a.new_value),
+        static_cast<uint8_t*>(const_cast<void*>(a.k_cache)),
+        static_cast<uint8_t*>(const_cast<void*>(a.v_cache)), a.num_kv_heads, a.k_inv, a.v_inv,
+        a.probe_us, a.k_scales, a.v_scales);
+    if (st != PA_OK || a.max_parts <= 1) return st;
+    return launch_reduce<T, D>(a);
+}
+
 template <typename Codes, typename T, int D, int BS, int G, bool ROWS>
 static pa_status launch_decode_q8(const DecodeArgs& a, float v_scale)
 {
+    if (a.num_kv_heads % 2 == 0 && a.partition_size < kPairBelowBlocks * kWarps * BS)
+        return launch_decode_q8_pair<Codes, T, D, BS, G, ROWS>(a, v_scale);
     using S = Q8Shape<D, BS, G, ROWS>;
     static std::atomic<uint64_t> attr_done{0};
     auto kernel = std::is_same<Codes, Int8Codes>::value

@@ -189,10 +189,15 @@ __device__ __forceinline__ void load_words(const unsigned char* tile, int row, i
 // One warp's share of a (sequence, kv head, partition) unit: Q^T fragments,
 // the O^T accumulators and the online-softmax state of heads 2*tig and
 // 2*tig + 1 (rows of N), and the code that consumes one block of K/V bytes.
-template <typename Codes, typename T, int D, int BS, int G, bool ROWS = false>
+//
+// HP is the number of kv heads a tile holds: 1, or 2 when one copy brings
+// two adjacent kv heads (their rows interleave: line 2r + h of the tile is
+// token r of head h), hsel the head this warp reads.
+template <typename Codes, typename T, int D, int BS, int G, bool ROWS = false, int HP = 1>
 struct Q8Warp {
     using S = Q8Shape<D, BS, G, ROWS>;
     int grp, tig;
+    int hsel = 0;                   // HP = 2: which of the tile's two heads
     uint32_t pt_addr;               // this lane's row of the P^T staging tile
     uint32_t qb[S::KW][2];
     float o[S::MT][4];
@@ -201,6 +206,9 @@ struct Q8Warp {
     float vref, vinv;               // ROWS: running reference of the V row scales, 1 / it
     float e0, e1;                   // kBias * sum_d q[h][d] of heads 2tig, 2tig + 1
     float ps_run0, ps_run1;         // ROWS with a bias: sum of the P values fed to the MMA
+
+    // tile line of token row r
+    __device__ __forceinline__ int line(int r) const { return HP == 1 ? r : r * HP + hsel; }
 
     __device__ __forceinline__ void reset()
     {
@@ -269,8 +277,8 @@ struct Q8Warp {
 #pragma unroll
             for (int h = 0; h < S::KV16; ++h) {
                 uint32_t w0[4], w1[4];
-                load_words<D>(kt, t0 + grp, (D / 4) * tig + 16 * h, w0);
-                load_words<D>(kt, t0 + grp + 8, (D / 4) * tig + 16 * h, w1);
+                load_words<D>(kt, line(t0 + grp), (D / 4) * tig + 16 * h, w0);
+                load_words<D>(kt, line(t0 + grp + 8), (D / 4) * tig + 16 * h, w1);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int j = 4 * h + i;
@@ -371,23 +379,23 @@ struct Q8Warp {
             uint32_t va[S::VQ], vb[S::VQ], vc[S::VQ], vd[S::VQ];
             if constexpr (S::VQ == 4) {
                 uint32_t w[4];
-                load_words<D>(vt, ta, S::DPT * grp, w);
+                load_words<D>(vt, line(ta), S::DPT * grp, w);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) va[q] = w[q];
-                load_words<D>(vt, ta + 1, S::DPT * grp, w);
+                load_words<D>(vt, line(ta + 1), S::DPT * grp, w);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) vb[q] = w[q];
-                load_words<D>(vt, ta + 8, S::DPT * grp, w);
+                load_words<D>(vt, line(ta + 8), S::DPT * grp, w);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) vc[q] = w[q];
-                load_words<D>(vt, ta + 9, S::DPT * grp, w);
+                load_words<D>(vt, line(ta + 9), S::DPT * grp, w);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) vd[q] = w[q];
             } else {
-                const uint2 a = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta, S::DPT * grp));
-                const uint2 b = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 1, S::DPT * grp));
-                const uint2 c = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 8, S::DPT * grp));
-                const uint2 d = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(ta + 9, S::DPT * grp));
+                const uint2 a = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(line(ta), S::DPT * grp));
+                const uint2 b = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(line(ta + 1), S::DPT * grp));
+                const uint2 c = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(line(ta + 8), S::DPT * grp));
+                const uint2 d = *reinterpret_cast<const uint2*>(vt + q8_tile_off<D>(line(ta + 9), S::DPT * grp));
                 va[0] = a.x; va[1] = a.y;
                 vb[0] = b.x; vb[1] = b.y;
                 vc[0] = c.x; vc[1] = c.y;
@@ -680,8 +688,5 @@ __global__ void __launch_bounds__(kThreads, 4) paged_decode_int8_kernel(PA_Q8_KE
 {
     paged_decode_q8_cta<Int8Codes, T, D, BS, G, ROWS>(PA_Q8_KERNEL_ARGS);
 }
-
-#undef PA_Q8_KERNEL_PARAMS
-#undef PA_Q8_KERNEL_ARGS
 
 }  // namespace pa

@@ -46,11 +46,11 @@ def small_llama(seed_shift=0, seqs=4, max_ctx=300, keep_logical=True):
                            num_blocks=160, scale=1 / math.sqrt(128), keep_logical=keep_logical)
 
 
-def small_gqa(block_size=16, dtype="bf16", seqs=5, head_dim=128, keep_logical=True):
+def small_gqa(block_size=16, dtype="bf16", seqs=5, head_dim=128, keep_logical=True, kv_heads=2):
     ctx = np.random.Generator(np.random.PCG64(11)).integers(1, 260, size=seqs, endpoint=True)
     nb = int(sum(-(-int(c) // block_size) for c in ctx)) + 16
     return gen.make_decode("gqa-small", seed=gen.SEED_BASE + 3, dtype=dtype, context_lens=ctx,
-                           num_q_heads=8, num_kv_heads=2, head_dim=head_dim,
+                           num_q_heads=4 * kv_heads, num_kv_heads=kv_heads, head_dim=head_dim,
                            block_size=block_size, num_blocks=nb, scale=1 / math.sqrt(head_dim),
                            keep_logical=keep_logical)
 

@@ -187,13 +187,13 @@ def test_copy_blocks_on_code_pools(codes):
 
 # ---- decode over the codes --------------------------------------------------------
 
-def _instance(codes, head_dim, block_size, group, dtype, partition_blocks=4):
+def _instance(codes, head_dim, block_size, group, dtype, partition_blocks=4, hkv=2):
     rng = np.random.Generator(np.random.PCG64(head_dim * 1000 + block_size * 10 + group + 5))
     ctx = rng.integers(1, 300, size=3, endpoint=True)
     ctx[0] = 1
     nb = int(sum(-(-int(c) // block_size) for c in ctx)) + 8
     wl = gen.make_decode("q8-instance", seed=78, dtype=dtype, context_lens=ctx,
-                         num_q_heads=2 * group, num_kv_heads=2, head_dim=head_dim,
+                         num_q_heads=hkv * group, num_kv_heads=hkv, head_dim=head_dim,
                          block_size=block_size, num_blocks=nb, scale=1 / math.sqrt(head_dim),
                          partition_size=partition_blocks * block_size)
     return gen.with_code_pools(wl, codes, seed=head_dim + block_size + group)
@@ -212,8 +212,10 @@ def test_every_code_instance(head_dim, block_size, group, dtype, codes):
 
 
 @pytest.mark.parametrize("codes", CODES)
-@pytest.mark.parametrize("partition", [16, 512, 0])
+@pytest.mark.parametrize("partition", [16, 512, 0, 1024])
 def test_code_partition_sweep(partition, codes):
+    """Partitions below 16 blocks per warp take the kernel with a CTA per
+    pair of kv heads, 1024 tokens (64 blocks) the one with a CTA per kv head."""
     wl = gen.with_code_pools(oracle_pins.small_gqa(seqs=6), codes, seed=40)
     _parity(wl, partition_size=partition, what=f"{codes} gqa P{partition}")
 
@@ -353,6 +355,25 @@ def test_code_fused_append(head_dim, block_size, group, dtype, partition, codes)
     ref, st = _oracle_decode(wl, kc, vc)
     assert st == 0 and dev.status() == 0
     assert_close(to_f64(out), ref, f"{codes} fused append")
+
+
+@pytest.mark.parametrize("codes", CODES)
+@pytest.mark.parametrize("hkv,group,head_dim,block_size,dtype", [
+    (1, 4, 128, 16, "bf16"), (3, 2, 128, 16, "f16"), (5, 1, 64, 32, "bf16"), (3, 8, 128, 32, "f16")])
+def test_code_odd_kv_heads(hkv, group, head_dim, block_size, dtype, codes):
+    """An odd number of kv heads takes the kernel with a CTA per kv head (an
+    even number takes a CTA per pair of adjacent kv heads): decode over
+    partitions of 4 blocks, then the fused append, against the oracle."""
+    wl = _instance(codes, head_dim, block_size, group, dtype, hkv=hkv)
+    _parity(wl, what=f"{codes} Hkv{hkv} G{group} D{head_dim} B{block_size} {dtype}")
+    dev, out = _fused(wl)
+    kc, vc, st = _oracle_pools(wl)
+    assert st == 0
+    assert np.array_equal(dev.k_cache.cpu().numpy(), kc)
+    assert np.array_equal(dev.v_cache.cpu().numpy(), vc)
+    ref, st = _oracle_decode(wl, kc, vc)
+    assert st == 0 and dev.status() == 0
+    assert_close(to_f64(out), ref, f"{codes} Hkv{hkv} fused append")
 
 
 @pytest.mark.parametrize("codes", CODES)

@@ -147,8 +147,7 @@ def test_rowscale_write_bit_exact(fmt, dtype, head_dim, block_size):
     assert np.array_equal(dvs.cpu().numpy().view(np.uint32), vs.view(np.uint32))
 
 
-def _gqa(group, head_dim, block_size, dtype="bf16", seqs=5):
-    hkv = 4
+def _gqa(group, head_dim, block_size, dtype="bf16", seqs=5, hkv=4):
     return gen.make_decode("rows", seed=4150 + 70 + group, dtype=dtype,
                            context_lens=np.array([1, 17, 200, 33, 511][:seqs], np.int32),
                            num_q_heads=hkv * group, num_kv_heads=hkv, head_dim=head_dim,
@@ -159,7 +158,7 @@ def _gqa(group, head_dim, block_size, dtype="bf16", seqs=5):
 @pytest.mark.parametrize("group,head_dim,block_size,dtype", [
     (1, 128, 16, "f16"), (2, 64, 16, "bf16"), (4, 128, 16, "bf16"), (8, 128, 32, "f16"),
     (4, 64, 32, "f16")])
-@pytest.mark.parametrize("partition", [0, 32])
+@pytest.mark.parametrize("partition", [0, 32, 2048])
 def test_rowscale_decode(fmt, group, head_dim, block_size, dtype, partition):
     wl = gen.with_rowscale_pools(_gqa(group, head_dim, block_size, dtype), fmt, seed=7)
     dev = RowDevice(wl)
@@ -170,6 +169,22 @@ def test_rowscale_decode(fmt, group, head_dim, block_size, dtype, partition):
     assert dev.status() == 0 and st == 0 and st2 == 0
     _same_pools(dev, kc, vc, ks, vs, "pools after the write")
     assert_close_rows(to_f64(out), ref, f"{fmt} rows G={group} D={head_dim} B={block_size} P={partition}")
+
+
+@pytest.mark.parametrize("fmt", CODES)
+@pytest.mark.parametrize("group,hkv", [(4, 3), (1, 5)])
+@pytest.mark.parametrize("partition", [0, 32])
+def test_rowscale_odd_kv_heads(fmt, group, hkv, partition):
+    """An odd number of kv heads takes the kernel with a CTA per kv head
+    (an even number a CTA per pair of kv heads)."""
+    wl = gen.with_rowscale_pools(_gqa(group, 128, 16, "bf16", hkv=hkv), fmt, seed=10)
+    dev = RowDevice(wl)
+    dev.write()
+    out = dev.decode(partition)
+    kc, vc, ks, vs, st = _oracle_after_write(wl)
+    ref, st2 = _oracle_decode(wl, kc, vc, ks, vs)
+    assert dev.status() == 0 and st == 0 and st2 == 0
+    assert_close_rows(to_f64(out), ref, f"{fmt} rows Hkv={hkv} G={group} P={partition}")
 
 
 @pytest.mark.parametrize("fmt", CODES)

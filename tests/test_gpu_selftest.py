@@ -101,9 +101,13 @@ def test_decode_abort_path(case, partition):
 
 @pytest.mark.parametrize("codes", ["fp8", "int8"])
 @pytest.mark.parametrize("partition", [0, 32])
-def test_decode_abort_path_code_pools(codes, partition):
+@pytest.mark.parametrize("kv_heads", [2, 3])
+def test_decode_abort_path_code_pools(codes, partition, kv_heads):
+    """Both one-byte kernels: a CTA per pair of kv heads (2) and a CTA per
+    kv head (3)."""
     from paged_kv_cache_415_b200 import binding as B
-    wl = gen.with_code_pools(oracle_pins.small_gqa(keep_logical=False), codes, seed=77)
+    wl = gen.with_code_pools(oracle_pins.small_gqa(keep_logical=False, kv_heads=kv_heads), codes,
+                             seed=77)
     np_t = {"fp8": np.uint8, "int8": np.int8}[codes]
     dw = DeviceWorkload.__new__(DeviceWorkload)
     dw.wl = wl
