@@ -310,11 +310,11 @@ def test_code_deterministic(codes):
 
 @pytest.mark.slow
 @pytest.mark.parametrize("codes", CODES)
-@pytest.mark.parametrize("name", ["llama7b", "mistral7b"])
+@pytest.mark.parametrize("name", ["llama7b", "mistral7b", "long_context"])
 def test_code_full_size(name, codes):
-    """The full-size workload with quantised pools, in the launch
-    configuration the benchmark times: write + decode against the whole
-    oracle."""
+    """The full-size workload with quantised pools (long_context: the
+    kernel with a CTA per pair of kv heads): write + decode against the
+    whole oracle."""
     wl = gen.with_code_pools(gen.CONFIGS[name](), codes, seed=44)
     _parity(wl, what=f"{name}-{codes}")
 
@@ -335,6 +335,25 @@ def _fused(wl, partition_size=None, tables=None):
                          ws, dev.d_status)
     torch.cuda.synchronize()
     return dev, out
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("codes", CODES)
+@pytest.mark.parametrize("name", ["mistral7b", "long_context"])
+def test_code_fused_append_full_size(name, codes):
+    """The entry point the benchmark times on one-byte pools (quantising
+    write fused into the decode, the workload's partitions), at full size:
+    both pools bit for bit and every output row against the oracle."""
+    wl = gen.with_code_pools(gen.CONFIGS[name](), codes, seed=45)
+    assert wl.extra["one_token_per_seq"]
+    dev, out = _fused(wl)
+    kc, vc, st = _oracle_pools(wl)
+    assert st == 0
+    assert np.array_equal(dev.k_cache.cpu().numpy(), kc), f"{name}-{codes}: K pool"
+    assert np.array_equal(dev.v_cache.cpu().numpy(), vc), f"{name}-{codes}: V pool"
+    ref, st = _oracle_decode(wl, kc, vc)
+    assert st == 0 and dev.status() == 0
+    assert_close(to_f64(out), ref, f"{name}-{codes} fused, every row")
 
 
 @pytest.mark.parametrize("codes", CODES)
