@@ -296,8 +296,8 @@ PA_API pa_status pa_paged_decode(void* out, const void* query, const void* k_cac
  * whose slot is given by its own block table:
  *   slot = block_tables[s][(ctx - 1) / block_size] * block_size + (ctx - 1) % block_size.
  * The CTA that owns a sequence's last context partition writes that token's
- * K/V row for its kv head before loading any tile, so no separate cache-write
- * kernel (and no launch dependency) is needed.
+ * K/V row of each kv head it serves before loading the block that holds it,
+ * so no separate cache-write kernel (and no launch dependency) is needed.
  *
  * key, value     [num_seqs][num_kv_heads][head_dim], 16-byte aligned: the new
  *                token of every sequence.  k_cache / v_cache are written.
