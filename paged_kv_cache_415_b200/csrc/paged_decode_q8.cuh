@@ -23,7 +23,9 @@
 // once per head, not per code: every score of head h carries 1152 * sum_d
 // q[h][d] (subtracted from the scores; the sum is taken once per CTA from
 // the fp16 query the MMA reads), and the output carries 1152 * sum_t p_t
-// (subtracted in the epilogue, from the sum of the P values the MMA read).  The contraction index
+// (subtracted every kBiasFlushBlocks blocks and in the epilogue, from the
+// sum of the P values the MMA read, so the accumulator never holds more
+// than a few blocks' worth of it).  The contraction index
 // may be permuted freely as long as both operands follow it, so every lane
 // reads whole 16-byte runs of one token row.  P moves from the accumulator
 // layout (tokens x heads) to the B layout (heads x tokens) through a
@@ -89,6 +91,10 @@ __device__ __forceinline__ uint32_t q8_tile_off(int row, int byte)
     else
         return static_cast<uint32_t>(row * D + byte);
 }
+
+// Blocks between two removals of the int8 bias from the output accumulator
+// (Q8Warp::flush_bias).
+constexpr int kBiasFlushBlocks = 8;
 
 // 2^x with the special-function unit's approximation (flushes subnormal
 // results to zero); the probabilities it produces are rounded to fp16 next.
@@ -205,7 +211,7 @@ struct Q8Warp {
     float l_run0, l_run1;           // this lane's share of the exp-sums
     float vref, vinv;               // ROWS: running reference of the V row scales, 1 / it
     float e0, e1;                   // kBias * sum_d q[h][d] of heads 2tig, 2tig + 1
-    float ps_run0, ps_run1;         // ROWS with a bias: sum of the P values fed to the MMA
+    float ps_run0, ps_run1;         // int8: sum of the P values fed to the MMA since the last flush
 
     // tile line of token row r
     __device__ __forceinline__ int line(int r) const { return HP == 1 ? r : r * HP + hsel; }
@@ -353,6 +359,10 @@ struct Q8Warp {
                 const float2 r0 = Elem<__half>::to_float2(pk0), r1 = Elem<__half>::to_float2(pk1);
                 l_run0 = l_run0 * c0 + (r0.x + r1.x);
                 l_run1 = l_run1 * c1 + (r0.y + r1.y);
+                if constexpr (Codes::kBias != 0.f) {   // the P values the MMA reads
+                    ps_run0 = ps_run0 * c0 + (r0.x + r1.x);
+                    ps_run1 = ps_run1 * c1 + (r0.y + r1.y);
+                }
             }
             // once the running maxima settle, most slices leave them unchanged
             if (__any_sync(kFullMask, cc.x != 1.f || cc.y != 1.f)) {
@@ -431,28 +441,20 @@ struct Q8Warp {
         }
     }
 
-    // The warp's (max, exp-sum, output) of its heads into the epilogue area.
-    __device__ __forceinline__ void store(float* epi_o, float* epi_m, float* epi_l, int warp,
-                                          float v_scale)
+    // int8 codes: every V value the MMA read carried the bias, so O holds
+    // kBias times the sum of the P values it was weighted with.  Remove what
+    // has gathered since the last call (the sum over the warp's lanes) and
+    // start that sum again.  Called every kBiasFlushBlocks blocks and before
+    // the epilogue, it keeps the bias in O to a few blocks' worth, so the
+    // fp32 cancellation does not grow with the partition.  Warp-uniform.
+    __device__ __forceinline__ void flush_bias()
     {
-#pragma unroll
-        for (int m = 4; m < 32; m <<= 1) {
-            l_run0 += __shfl_xor_sync(kFullMask, l_run0, m);
-            l_run1 += __shfl_xor_sync(kFullMask, l_run1, m);
-        }
         if constexpr (Codes::kBias != 0.f) {
-            // every V value the MMA read carried the bias: remove kBias times
-            // the sum of the P values it was weighted with (the exp-sum itself
-            // for one scale per pool, whose sum adds exactly those values)
-            float b0 = l_run0, b1 = l_run1;
-            if constexpr (ROWS) {
+            float b0 = ps_run0, b1 = ps_run1;
 #pragma unroll
-                for (int m = 4; m < 32; m <<= 1) {
-                    ps_run0 += __shfl_xor_sync(kFullMask, ps_run0, m);
-                    ps_run1 += __shfl_xor_sync(kFullMask, ps_run1, m);
-                }
-                b0 = ps_run0;
-                b1 = ps_run1;
+            for (int m = 4; m < 32; m <<= 1) {
+                b0 += __shfl_xor_sync(kFullMask, b0, m);
+                b1 += __shfl_xor_sync(kFullMask, b1, m);
             }
             b0 *= Codes::kBias;
             b1 *= Codes::kBias;
@@ -463,7 +465,20 @@ struct Q8Warp {
                 o[mt][2] -= b0;
                 o[mt][3] -= b1;
             }
+            ps_run0 = ps_run1 = 0.f;
         }
+    }
+
+    // The warp's (max, exp-sum, output) of its heads into the epilogue area.
+    __device__ __forceinline__ void store(float* epi_o, float* epi_m, float* epi_l, int warp,
+                                          float v_scale)
+    {
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+            l_run0 += __shfl_xor_sync(kFullMask, l_run0, m);
+            l_run1 += __shfl_xor_sync(kFullMask, l_run1, m);
+        }
+        flush_bias();
         const int h0 = 2 * tig, h1 = 2 * tig + 1;
 #pragma unroll
         for (int q = 0; q < S::VQ; ++q) {
@@ -638,6 +653,7 @@ __device__ __forceinline__ void paged_decode_q8_cta(
         const unsigned char* kt = wbase + st * S::STAGE;
         const float* sc = wsc + st * (S::SC_STAGE / 4);
         w.block(kt, kt + S::TILE, nv, scale_log2, sc, sc + BS);
+        if (k % kBiasFlushBlocks == kBiasFlushBlocks - 1) w.flush_bias();
         __syncwarp();   // every lane is done with this stage
         if (issued < nk) issue(issued++);
     }

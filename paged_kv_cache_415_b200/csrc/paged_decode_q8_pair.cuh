@@ -273,6 +273,7 @@ __device__ __forceinline__ void paged_decode_q8_pair_cta(
         const unsigned char* kt = ring + st * S::STAGE;
         const float* sc = rsc + st * (S::SC_STAGE / 4);
         w.block(kt, kt + S::TILE, nv, scale_log2, sc + hsel * BS, sc + 2 * BS + hsel * BS);
+        if (k % kBiasFlushBlocks == kBiasFlushBlocks - 1) w.flush_bias();
         __syncwarp();   // every lane is done with this stage
         if (lane == 0) mbar_arrive(&empty[st]);
         if (producer && issued < nk) {

@@ -172,6 +172,29 @@ def test_rowscale_decode(fmt, group, head_dim, block_size, dtype, partition):
 
 
 @pytest.mark.parametrize("fmt", CODES)
+@pytest.mark.parametrize("group,hkv,partition", [(4, 2, 2048), (1, 4, 2048), (4, 3, 4096), (4, 2, 8192)])
+def test_rowscale_long_partitions(fmt, group, hkv, partition):
+    """One warp accumulating many blocks: partitions of 2048-8192 tokens (up
+    to 128 blocks per warp), contexts of up to 8000.  int8 codes widen to 1152 + c, so
+    the output accumulator carries the bias of every token it has summed;
+    the kernel must keep that from costing precision over a long partition.
+    Every output row against the fp64 oracle at the row-scaled tolerance."""
+    ctx = np.array([2000, 1999, 8000, 33], np.int32)
+    nb = int(sum(-(-int(c) // 16) for c in ctx)) + 8
+    wl = gen.make_decode("rows-long", seed=4150 + 80 + group, dtype="bf16", context_lens=ctx,
+                         num_q_heads=hkv * group, num_kv_heads=hkv, head_dim=128, block_size=16,
+                         num_blocks=nb, scale=128 ** -0.5)
+    wl = gen.with_rowscale_pools(wl, fmt, seed=11)
+    dev = RowDevice(wl)
+    dev.write()
+    out = dev.decode(partition)
+    kc, vc, ks, vs, st = _oracle_after_write(wl)
+    ref, st2 = _oracle_decode(wl, kc, vc, ks, vs)
+    assert dev.status() == 0 and st == 0 and st2 == 0
+    assert_close_rows(to_f64(out), ref, f"{fmt} rows long partition G={group} Hkv={hkv} P={partition}")
+
+
+@pytest.mark.parametrize("fmt", CODES)
 @pytest.mark.parametrize("group,hkv", [(4, 3), (1, 5)])
 @pytest.mark.parametrize("partition", [0, 32])
 def test_rowscale_odd_kv_heads(fmt, group, hkv, partition):
