@@ -54,6 +54,10 @@ PROFILE_GLOB_DIR = os.path.join(ROOT, "profiles")
 # The device sources of each decode kernel family: a traffic line taken on a
 # family's hash stays valid while those files' code is unchanged.
 _CSRC = "paged_kv_cache_415_b200/csrc/"
+# Blocks per warp below which the library decodes one-byte pools with a CTA
+# per pair of kv heads (kPairBelowBlocks in csrc/paged_decode.cu).
+PAIR_BELOW_BLOCKS = 16
+
 KERNEL_FAMILIES = {
     "fp32": ["pa_common.cuh", "decode_common.cuh", "paged_decode_fp32.cuh"],
     "mma": ["pa_common.cuh", "decode_common.cuh", "paged_decode_mma.cuh"],
@@ -600,8 +604,9 @@ class GpuStep:
             return "paged_decode_shared_kernel" + (
                 " + paged_decode_shared_reduce_kernel" if self.shared_reduce else "")
         # one-byte pools: a CTA per pair of kv heads when the kv-head count is
-        # even and a CTA per kv head would give each warp fewer than 16 blocks
-        pair = (wl.num_kv_heads % 2 == 0 and self.part < 16 * 4 * wl.block_size)
+        # even and a CTA per kv head (4 warps) would give each warp fewer than
+        # PAIR_BELOW_BLOCKS blocks of its partition (the library's rule)
+        pair = (wl.num_kv_heads % 2 == 0 and self.part < PAIR_BELOW_BLOCKS * 4 * wl.block_size)
         name = (f"paged_decode_{self.codes}{'_pair' if pair else ''}_kernel" if self.quant else
                 "paged_decode_mma_kernel" if group >= 4 and wl.block_size % 16 == 0
                 else "paged_decode_kernel")

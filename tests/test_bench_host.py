@@ -160,3 +160,14 @@ def test_clock_records_of_both_regions_merge():
     m = bench.merge_clocks(a, b)
     assert m["sm_mhz"] == 1950 and m["samples"] == 43 and m["reasons"] == ["sw_power_cap"]
     assert bench.merge_clocks(a, {"samples": 0}) == a
+
+
+def test_pair_rule_matches_the_library():
+    """The bench names the one-byte kernel the library picks: its
+    blocks-per-warp threshold is the library's kPairBelowBlocks."""
+    src = os.path.join(os.path.dirname(bench.__file__), "paged_kv_cache_415_b200", "csrc",
+                       "paged_decode.cu")
+    with open(src, encoding="utf-8") as f:
+        m = re.search(r"constexpr int kPairBelowBlocks = (\d+);", f.read())
+    assert m, "kPairBelowBlocks not found"
+    assert int(m.group(1)) == bench.PAIR_BELOW_BLOCKS
